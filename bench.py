@@ -1,0 +1,479 @@
+#!/usr/bin/env python
+"""Benchmark of the SFA operator: prefill + decode tokens/s on B200.
+
+One step = state reset, prefill of the workload's prompt, then its decode
+steps, for every layer and sequence (the whole hot path on one batch of
+synthetic input).  A token is one sequence position through all layers.
+
+Default workload: the Qwen2.5-0.5B attention shape (24 layers, 14 query / 2
+KV heads, head_dim 64, batch 1, prefill 512 + 128 decode steps, k = 16,
+bf16 inputs).  L2 is flushed (256 MB write) before every timed step, outside
+the step's events.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs under torch.distributed.run as independent replicas (the
+operator has no cross-stream exchange), timed per rank and reduced with MAX.
+``--impl reference`` times the fp64 oracle on the host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "SFA prefill & decode tokens/s on 1 B200; achieved HBM GB/s vs ~8 TB/s peak"
+UNIT = "tokens/s"
+L2_FLUSH_BYTES = 256 << 20
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="qwen05b")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def workload_bytes(w):
+    """Algorithmic bytes (what the method must move; no re-reads).
+
+    decode launch: per (layer, sequence) q (e*H), out (4H), ring slot read +
+    write (8H), ring sum r/w (8H), field r/w (8H), new K/V read and window
+    write (4e*nkv*d), window read (2k*e*nkv*d), S r/w (8*nkv*d); per layer the
+    64 x H fp32 slots (256H).
+    prefill call of n tokens: per token-layer q, k, v read and out write
+    (e*H + 2e*nkv*d + 4H); per stream the final state write; per layer slots.
+    """
+    e = 4 if w.in_dtype == "f32" else 2
+    H, S, k = w.hidden, w.n_kv_heads * w.head_dim, w.window_k
+    per_seq_layer = (28 + e) * H + (4 * e + 8 + 2 * k * e) * S
+    decode = w.n_layers * (w.batch * per_seq_layer + 256 * H)
+    n = w.prefill_n[0]
+    state_write = 2 * k * S * e + 4 * S + 72 * H
+    prefill = (w.n_layers * w.batch * (n * (e * H + 2 * e * S + 4 * H) + state_write)
+               + w.n_layers * 256 * H)
+    return decode, prefill
+
+
+class ClockSampler:
+    """nvidia-smi samples of the SM clock and throttle reasons while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: str):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            threading.Thread(target=self._read, daemon=True).start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[4:8]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def gpu_index_for(device) -> str:
+    import torch
+    try:
+        uuid = str(torch.cuda.get_device_properties(device).uuid)
+        out = subprocess.run(["nvidia-smi", "--query-gpu=index,uuid", "--format=csv,noheader"],
+                             capture_output=True, text=True, timeout=20).stdout
+        for line in out.splitlines():
+            idx, u = [s.strip() for s in line.split(",")]
+            if uuid in u or u.endswith(uuid):
+                return idx
+    except Exception:
+        pass
+    return os.environ.get("CUDA_VISIBLE_DEVICES", "0").split(",")[0] or "0"
+
+
+def kernel_traffic(kernel_src: str, name: str):
+    """DRAM bytes per launch from a committed ncu summary, only if it was
+    taken on the current kernel source (matching sha256)."""
+    path = os.path.join(ROOT, "profiles", f"{name}_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        sha = hashlib.sha256(open(kernel_src, "rb").read()).hexdigest()
+        if d.get("kernel_sha256") == sha:
+            return float(d["dram_bytes_per_launch"]), d.get("workload")
+    except Exception:
+        pass
+    return None, None
+
+
+# ------------------------------------------------------------------ oracle
+
+
+def oracle_tokens_per_s(w, layers, n_tokens, src, slots_np):
+    """Times the fp64 oracle on `layers` x batch streams over n_tokens."""
+    import numpy as np
+    import oracle
+    f = lambda x: float(np.float32(x))
+    v = w.values
+    p = oracle.OracleParams(w.n_q_heads, w.n_kv_heads, w.head_dim, w.window_k,
+                            gamma_far=f(v.gamma_far), alpha_far=f(v.alpha_far))
+    q, k, vv = src.get(0, n_tokens)
+    sel = lambda x: x[layers].float().cpu().numpy()
+    qn, kn, vn = sel(q), sel(k), sel(vv)
+    st = oracle.OracleState(p, len(layers) * w.batch)
+    slots = slots_np[layers]
+    t0 = time.perf_counter()
+    _, used = oracle.run_layers(p, f(v.alpha_base), f(v.cross_decay), slots, qn, kn, vn, st,
+                                n_layers=w.n_layers)
+    dt = time.perf_counter() - t0
+    tokens = w.batch * n_tokens * len(layers) / w.n_layers  # positions through all layers
+    return tokens / dt, used, dt
+
+
+def run_reference(args, w):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    import numpy as np
+    import torch
+    from workloads import TokenSource, make_slots
+    src = TokenSource(w, "cpu")
+    slots_np = make_slots(w, "cpu").numpy()
+    n_tok = 64  # bounded sample per step: one layer, 64 positions
+    for _ in range(args.warmup):
+        oracle_tokens_per_s(w, [0], n_tok, src, slots_np)
+    times, used = [], 1
+    for s in range(args.steps):
+        _, used, dt = oracle_tokens_per_s(w, [s % w.n_layers], n_tok, src, slots_np)
+        times.append(dt)
+    total = sum(times)
+    tokens = args.steps * w.batch * n_tok / w.n_layers
+    value = tokens / total
+    sample = (f"per step: 1 layer x {w.batch} seq x {n_tok} positions of the {w.name} "
+              f"workload, scaled to positions through all {w.n_layers} layers")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": used, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w):
+    return {
+        "workload": (f"{w.name}: {w.n_layers} layers, {w.n_q_heads}q/{w.n_kv_heads}kv heads, "
+                     f"head_dim {w.head_dim}, batch {w.batch}, prefill {w.prefill_n[0]} + "
+                     f"{w.decode_steps} decode steps, k={w.window_k}"),
+        "global_batch": w.batch, "seq_len": w.prefill_n[0] + w.decode_steps,
+        "in_dtype": w.in_dtype, "window_k": w.window_k,
+        "l2": "flushed before every timed step (256 MB write)",
+        "parallelism": "replicas",
+    }
+
+
+# ------------------------------------------------------------------ ours
+
+
+def main():
+    args = parse()
+    from workloads import get_workload
+    w = get_workload(args.workload)
+    if args.impl == "reference":
+        run_reference(args, w)
+        return
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    import kv_cache_compression_sfa_b200 as sfa
+    from kv_cache_compression_sfa_b200 import build as sfa_build
+    from workloads import TokenSource, make_slots
+
+    rank, world, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    sfa_build.build()
+
+    v = w.values
+    cfg = sfa.SfaConfig(n_layers=w.n_layers, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads,
+                        head_dim=w.head_dim, window_k=w.window_k, gamma_far=v.gamma_far,
+                        alpha_far=v.alpha_far, ema_gamma=v.ema_gamma, temperature=v.temperature,
+                        clip_eps=v.clip_eps, alpha_base=v.alpha_base, cross_decay=v.cross_decay,
+                        in_dtype=sfa.SFA_F32 if w.in_dtype == "f32" else sfa.SFA_BF16)
+    n_pre, n_dec = w.prefill_n[0], w.decode_steps
+    L, B, H = w.n_layers, w.batch, w.hidden
+    src = TokenSource(w, dev, salt=rank)
+    slots = make_slots(w, dev)
+    qp, kp, vp = src.get(0, n_pre)
+    qa, ka, va = src.get(n_pre, n_pre + n_dec)
+    qd = [qa[:, :, t].contiguous() for t in range(n_dec)]
+    kd = [ka[:, :, t].contiguous() for t in range(n_dec)]
+    vd = [va[:, :, t].contiguous() for t in range(n_dec)]
+    op = sfa.SfaOperator(cfg, slots, B, max_prefill=n_pre, device=dev)
+    out_p = torch.empty((L, B, n_pre, H), dtype=torch.float32, device=dev)
+    out_d = torch.empty((n_dec, L, B, H), dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def prefill_part():
+        op.reset()
+        op.prefill(qp, kp, vp, out=out_p)
+
+    def decode_part():
+        for t in range(n_dec):
+            op.decode(qd[t], kd[t], vd[t], out=out_d[t])
+
+    # eager warm-up, then capture both halves as CUDA graphs
+    prefill_part()
+    decode_part()
+    torch.cuda.synchronize()
+    rc = op.check()
+    if rc != 0:
+        raise SystemExit(f"device error during warm-up: {sfa.sfa_status_string(rc)}")
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    g_pre, g_dec = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(g_pre, stream=side):
+            prefill_part()
+        with torch.cuda.graph(g_dec, stream=side):
+            decode_part()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        g_pre.replay()
+        g_dec.replay()
+    torch.cuda.synchronize()
+    if op.check() != 0:
+        raise SystemExit("device error during warm-up")
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    sampler = ClockSampler(gpu_index_for(dev)) if rank == 0 else None
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+        time.sleep(0.1)
+    for s in range(args.steps):
+        flush.zero_()
+        ev[s][0].record()
+        g_pre.replay()
+        ev[s][1].record()
+        g_dec.replay()
+        ev[s][2].record()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop() if sampler else None
+    pre_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    dec_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    total_ms = sum(pre_ms) + sum(dec_ms)
+    rc = op.check()
+    if rc != 0:
+        raise SystemExit(f"device error in the timed region: {sfa.sfa_status_string(rc)}")
+    t = torch.tensor([total_ms, sum(pre_ms), sum(dec_ms)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms, pre_tot, dec_tot = (float(x) for x in t.tolist())
+    tokens_per_step = B * (n_pre + n_dec)
+    value = world * tokens_per_step * args.steps / (total_ms / 1e3)
+    ms_per_step = total_ms / args.steps
+
+    # ---- roofline of the dominant kernel (decode: 128 of 130 launches/step)
+    peak, peak_kind = measured_peaks()
+    dec_bytes, pre_bytes = workload_bytes(w)
+    dec_launch_ms = dec_tot / (args.steps * n_dec)
+    dec_gbs = dec_bytes / (dec_launch_ms / 1e3) / 1e9
+    pre_ms_avg = pre_tot / args.steps
+    pre_gbs = pre_bytes / (pre_ms_avg / 1e3) / 1e9
+    traffic, _ = kernel_traffic(os.path.join(ROOT, "kv_cache_compression_sfa_b200", "csrc",
+                                             "sfa_decode.cu"), "decode")
+
+    # ---- e2e through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        e2e = measure_e2e(args, w, op, qp, kp, vp, qa, ka, va, n_pre, n_dec, world, dev)
+
+    # ---- oracle on the host cores (rank 0, N = 1 only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w)
+
+    if world > 1:
+        dist.barrier()
+        del g_pre, g_dec
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": workload_config(w),
+        "prefill": {"tokens_per_s": world * B * n_pre * args.steps / (pre_tot / 1e3),
+                    "ms": pre_ms_avg, "algorithmic_bytes": pre_bytes,
+                    "achieved_gbs": pre_gbs, "frac": pre_gbs / peak},
+        "decode": {"tokens_per_s": world * B * n_dec * args.steps / (dec_tot / 1e3),
+                   "us_per_step": 1e3 * dec_launch_ms, "algorithmic_bytes": dec_bytes,
+                   "achieved_gbs": dec_gbs, "frac": dec_gbs / peak},
+        "roofline": {"bound": "hbm", "kernel": "sfa decode step", "achieved": dec_gbs,
+                     "peak": peak, "unit": "GB/s", "frac": dec_gbs / peak,
+                     "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
+                     if peak_kind == "measured" else "fallback 6.65 TB/s",
+                     "traffic": traffic},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": args.steps * (2 + n_dec),
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def measure_e2e(args, w, op, qp, kp, vp, qa, ka, va, n_pre, n_dec, world, dev):
+    """Same metric through SfaOperator with pinned host inputs and outputs:
+    every step copies its q/k/v host->device, runs reset + prefill + decode
+    steps, and reads all outputs back."""
+    import torch
+    import torch.distributed as dist
+    L, B, H = w.n_layers, w.batch, w.hidden
+    # decode inputs step-major ([step, L, B, heads, d]) so each step's slice
+    # is contiguous on the device
+    step_major = [x.permute(2, 0, 1, 3, 4).contiguous() for x in (qa, ka, va)]
+    host_in = [x.cpu().pin_memory() for x in (qp, kp, vp, *step_major)]
+    dev_in = [torch.empty_like(x, device=dev) for x in host_in]
+    h_out_p = torch.empty((L, B, n_pre, H), dtype=torch.float32).pin_memory()
+    h_out_d = torch.empty((n_dec, L, B, H), dtype=torch.float32).pin_memory()
+    d_out_p = torch.empty((L, B, n_pre, H), dtype=torch.float32, device=dev)
+    d_out_d = torch.empty((n_dec, L, B, H), dtype=torch.float32, device=dev)
+    h2d = sum(x.numel() * x.element_size() for x in host_in)
+    d2h = (h_out_p.numel() + h_out_d.numel()) * 4
+    steps = max(3, min(args.steps, 200))
+
+    def one():
+        for h, d in zip(host_in, dev_in):
+            d.copy_(h, non_blocking=True)
+        op.reset()
+        op.prefill(dev_in[0], dev_in[1], dev_in[2], out=d_out_p)
+        h_out_p.copy_(d_out_p, non_blocking=True)
+        for t in range(n_dec):
+            op.decode(dev_in[3][t], dev_in[4][t], dev_in[5][t], out=d_out_d[t])
+        h_out_d.copy_(d_out_d, non_blocking=True)
+
+    for _ in range(3):
+        one()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        one()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = float(t.item())
+    value = world * B * (n_pre + n_dec) * steps / (ms / 1e3)
+    return {"value": value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "steps": steps, "l2": "not flushed (host copies between steps)"}
+
+
+def cpu_baseline(w):
+    import numpy as np
+    from workloads import TokenSource, make_slots
+    src = TokenSource(w, "cpu")
+    slots_np = make_slots(w, "cpu").numpy()
+    n_tok = w.prefill_n[0] + w.decode_steps
+    # bounded sample: as many layers (all sequences, all positions of the
+    # step) as fit in ~15 s, estimated from a one-layer run
+    rate1, used1, dt1 = oracle_tokens_per_s(w, [0], n_tok, src, slots_np)
+    n_layers = max(1, min(w.n_layers, int(15.0 / max(dt1, 1e-3))))
+    layers = list(range(n_layers))
+    rate, used, dt = oracle_tokens_per_s(w, layers, n_tok, src, slots_np)
+    return {"value": rate, "unit": UNIT, "cores": used, "kind": "oracle",
+            "sample": (f"{n_layers} of {w.n_layers} layers x {w.batch} seq x {n_tok} positions "
+                       f"(the full step's positions), {dt:.1f} s; tokens scaled to positions "
+                       f"through all layers")}
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,187 @@
+/*
+ * sfa.h — C ABI of the Signal Field Attention (SFA) operator for one NVIDIA
+ * B200 (sm_100a).
+ *
+ * The operator (definitions by source page):
+ *   [P1] "Signal Field Attention (SFA)：8KB代码实现4.16倍推理加速与248倍内存压缩"
+ *        §2.1: near-field softmax attention over the last k tokens (eq.
+ *        O_near), far-field EWMA of keys (eq. S_t), fusion O = O_near + α·S
+ *        (eq. O).  §2.2: O(k·d) state.
+ *   [P3] "Dalin Soma SFA基于信号场注意力机制的神经网络推理加速框架"
+ *        §2.1: ring-buffer mean (16 slots), EMA field (γ = 0.98), semantic
+ *        pool (64 slots, T = 0.07).  §2.2: enhancement = ring_mean +
+ *        0.5·field + 0.5·semantic, clipped to ±ε, scaled by
+ *        α_layer = α_base·(0.3 + 0.7·layer/(L−1))·decay^layer, added to the
+ *        attention output.
+ *   [P2] "Signal Field Attention (SFA)" (README page): SFA_Config defaults
+ *        and the engine calls init(n_layers, hidden) /
+ *        compute_enhancement(layer, attn_output), which this ABI follows
+ *        with caller-owned buffers.
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers on the current CUDA device and
+ *     must be 16-byte aligned.  The caller owns all of them.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Work is enqueued asynchronously; nothing synchronises except
+ *     sfa_check_device_status.
+ *   - Return value: SFA_OK (0) or a negative sfa_status.  No call throws, no
+ *     kernel traps.  Errors detected on the device (a state whose header does
+ *     not match the handle, a bounded wait that ran out) are latched in the
+ *     handle and reported by sfa_check_device_status.
+ *   - Layer-major, token-major layouts (d = head_dim, H = n_q_heads·d):
+ *       prefill q   [L][batch][n][n_q_heads][d]    in_dtype
+ *               k,v [L][batch][n][n_kv_heads][d]   in_dtype
+ *               out [L][batch][n][H]               fp32
+ *       decode  q   [L][batch][n_q_heads][d], k,v [L][batch][n_kv_heads][d],
+ *               out [L][batch][H].
+ *   - One state buffer serves `batch` sequences for all layers.  A state is
+ *     used by one stream at a time; stream order serialises calls.  The
+ *     compute calls never modify the handle, so it may be shared across
+ *     streams and host threads (only sfa_debug_set_lookback and
+ *     sfa_destroy modify it).
+ */
+#ifndef SFA_H
+#define SFA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SFA_API __attribute__((visibility("default")))
+#else
+#define SFA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SFA_ABI_VERSION 1
+
+typedef enum sfa_status {
+  SFA_OK = 0,
+  SFA_ERR_INVALID_ARG = -1,     /* null pointer, negative size, bad value  */
+  SFA_ERR_UNSUPPORTED = -2,     /* valid but not built: see sfa_init       */
+  SFA_ERR_ALIGNMENT = -3,       /* a pointer is not 16-byte aligned         */
+  SFA_ERR_STATE_MISMATCH = -4,  /* state header is not this handle's/batch */
+  SFA_ERR_CUDA = -5,            /* a CUDA runtime call or launch failed     */
+  SFA_ERR_DEVICE_TIMEOUT = -6,  /* a bounded device-side wait ran out       */
+  SFA_ERR_WORKSPACE = -7        /* workspace smaller than required          */
+} sfa_status;
+
+typedef enum sfa_dtype { SFA_F32 = 0, SFA_BF16 = 1 } sfa_dtype;
+
+/* Operator configuration.  Field names follow the pages' SFA_Config. */
+typedef struct sfa_config {
+  int n_layers;        /* L >= 1                                            */
+  int n_q_heads;       /* query heads; hidden = n_q_heads*head_dim <= 8192  */
+  int n_kv_heads;      /* KV heads, divides n_q_heads (GQA)                  */
+  int head_dim;        /* 64 or 128                                          */
+  int window_k;        /* near window k, 1..256            [P1 §2.1, §2.2]   */
+  float gamma_far;     /* far-field EWMA decay, [0, 1)     [P1 eq. S_t]      */
+  float alpha_far;     /* far-field mixing coefficient     [P1 eq. O]        */
+  int ring_size;       /* must be 16                       [P3 §2.1 ch. 1]   */
+  float ema_gamma;     /* EMA field decay (0.98)           [P3 §2.1 ch. 2]   */
+  int n_slots;         /* must be 64                       [P3 §2.1 ch. 3]   */
+  float temperature;   /* pool temperature (0.07), > 0     [P3 §2.1 ch. 3]   */
+  float clip_eps;      /* enhancement clip ε (0.5), >= 0   [P3 §2.2]         */
+  float alpha_base;    /* base strength (0.1)              [P3 §2.2]         */
+  float cross_decay;   /* per-layer decay (0.8)            [P3 §2.2]         */
+  int in_dtype;        /* sfa_dtype of q, k, v; state and out are fp32       */
+  const float* slots;  /* DEVICE [L][n_slots][hidden] fp32 semantic slots;
+                          copied by sfa_init, may be freed afterwards        */
+} sfa_config;
+
+typedef struct sfa_handle sfa_handle;
+
+/* Byte layout of a state buffer (host-side arithmetic only).
+ * The buffer is a 256-byte header followed by L*batch stream blocks of
+ * stream_stride bytes, stream (layer l, sequence b) at index l*batch + b.
+ * Offsets below are relative to the start of a stream block. */
+typedef struct sfa_state_layout {
+  size_t header_bytes;   /* 256                                            */
+  size_t stream_stride;  /* bytes per (layer, sequence) stream, 256-aligned */
+  size_t total_bytes;    /* header + L*batch*stream_stride                 */
+  size_t off_pos;        /* int64 position (tokens folded in)              */
+  size_t off_win_k;      /* [window_k][n_kv][d] in_dtype, slot = pos mod k */
+  size_t off_win_v;      /* same                                           */
+  size_t off_far;        /* S [n_kv][d] fp32                               */
+  size_t off_field;      /* EMA field [hidden] fp32                        */
+  size_t off_ring_sum;   /* sum of the ring slots [hidden] fp32            */
+  size_t off_ring;       /* ring [16][hidden] fp32, slot = pos mod 16      */
+} sfa_state_layout;
+
+/* Fills `cfg` with the pages' defaults ([P2 SFA_Config] usage example:
+ * alpha_base 0.1, cross_decay 0.8, ema_gamma 0.98, ring_size 16, 64 slots,
+ * clip 0.5; [P3 §2.1] temperature 0.07; [P1 §2.2] k = 16) plus
+ * gamma_far 0.9, alpha_far 0.1, bf16 inputs.  Shape fields are zeroed and
+ * slots is NULL.  No CUDA call. */
+SFA_API void sfa_config_default(sfa_config* cfg);
+
+/* Validates a configuration without touching the GPU: SFA_OK,
+ * SFA_ERR_INVALID_ARG (null, non-positive sizes, non-finite or out-of-range
+ * scalars, n_q % n_kv != 0) or SFA_ERR_UNSUPPORTED (head_dim not 64/128,
+ * window_k > 256, ring_size != 16, n_slots != 64, hidden > 8192).  The slots
+ * pointer is checked for NULL and alignment only. */
+SFA_API int sfa_config_validate(const sfa_config* cfg);
+
+/* State layout for `batch` sequences of `cfg` (host arithmetic, no CUDA). */
+SFA_API int sfa_state_layout_for(const sfa_config* cfg, int batch, sfa_state_layout* out);
+
+/* Creates a handle on the current device: validates cfg, copies the slots,
+ * precomputes slot norms and the alpha_layer table, allocates the device
+ * error word.  *out receives the handle, or NULL on error. */
+SFA_API int sfa_init(const sfa_config* cfg, sfa_handle** out);
+
+/* Frees the handle's device memory (synchronises the device first). */
+SFA_API int sfa_destroy(sfa_handle* h);
+
+/* Bytes of a state buffer for `batch` sequences; 0 on invalid input. */
+SFA_API size_t sfa_state_bytes(const sfa_handle* h, int batch);
+
+/* Bytes of prefill workspace for a call of n tokens x `batch`; 0 when the
+ * call needs none or on invalid input.  The workspace holds the cross-tile
+ * carries of the parallel scans; its content need not be initialised. */
+SFA_API size_t sfa_prefill_workspace_bytes(const sfa_handle* h, int batch, long long n);
+
+/* Zeroes `state` (state_bytes(h, batch) bytes) and writes its header for
+ * this handle and batch: every stream back to position 0. */
+SFA_API int sfa_state_reset(const sfa_handle* h, void* state, int batch, void* stream);
+
+/* Folds n >= 0 tokens per sequence into the state and writes their outputs.
+ * Equivalent to n calls of sfa_decode_step (same results within rounding).
+ * Continues from each stream's current position.  n == 0 enqueues nothing.
+ * workspace: sfa_prefill_workspace_bytes(h, batch, n) bytes (may be NULL if
+ * that is 0); workspace_bytes is its size, checked. */
+SFA_API int sfa_prefill(const sfa_handle* h, const void* q, const void* k, const void* v,
+                long long n, int batch, void* state, float* out, void* workspace,
+                size_t workspace_bytes, void* stream);
+
+/* Folds one token per sequence into the state and writes its output.
+ * One kernel launch covers all layers and sequences; no workspace. */
+SFA_API int sfa_decode_step(const sfa_handle* h, const void* q, const void* k, const void* v,
+                    int batch, void* state, float* out, void* stream);
+
+/* Synchronises `stream`, then returns and clears the first error latched on
+ * the device since the last check (SFA_OK if none), or SFA_ERR_CUDA if the
+ * stream reports a CUDA error. */
+SFA_API int sfa_check_device_status(const sfa_handle* h, void* stream);
+
+/* Static description of a status code. */
+SFA_API const char* sfa_status_string(int status);
+
+/* ABI version of the loaded library (SFA_ABI_VERSION it was built with). */
+SFA_API int sfa_abi_version(void);
+
+/* Test hook for the device-side bounded waits of sfa_prefill (not needed in
+ * normal use).  spin_limit: maximum polls of a look-back flag before the
+ * wait gives up and latches SFA_ERR_DEVICE_TIMEOUT (0 restores the default).
+ * withhold_tile: a tile index whose cross-tile publications are skipped, so
+ * that its successors' waits run out (-1 disables).  Affects later calls on
+ * this handle only. */
+SFA_API int sfa_debug_set_lookback(sfa_handle* h, unsigned int spin_limit, long long withhold_tile);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SFA_H */

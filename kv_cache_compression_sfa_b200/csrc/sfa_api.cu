@@ -1,0 +1,415 @@
+// sfa_api.cu — the C ABI declared in include/sfa.h: configuration checks,
+// state and workspace layout, handle set-up, launch configuration and the
+// device error latch.
+//
+// Sources (web pages):
+//   [P1] "Signal Field Attention (SFA)：8KB代码实现4.16倍推理加速与248倍内存压缩"
+//   [P2] "Signal Field Attention (SFA)" (project README page): SFA_Config
+//        defaults, engine init(n_layers, hidden) / per-layer enhancement call.
+//   [P3] "Dalin Soma SFA基于信号场注意力机制的神经网络推理加速框架" §2.2:
+//        alpha_layer = alpha_base·(0.3 + 0.7·layer_ratio)·decay^layer.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "sfa_internal.h"
+
+using namespace sfa;
+
+struct sfa_handle {
+  uint32_t magic;
+  sfa_config cfg;        // cfg.slots points at the handle's own copy
+  int device;
+  float* slots;          // [L][64][H]
+  float* slot_norm;      // [L][64]
+  float* alpha_layer;    // [L]
+  int* err;              // device error word
+  uint64_t cfg_hash;
+  int prefill_cs;
+  unsigned spin_limit;
+  long long withhold_tile;
+};
+
+namespace {
+
+constexpr uint32_t kHandleMagic = 0x48414653u;  // "SFAH"
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int hidden_of(const sfa_config* c) { return c->n_q_heads * c->head_dim; }
+
+size_t in_bytes(int dtype) { return dtype == SFA_F32 ? 4 : 2; }
+
+uint64_t fnv1a(uint64_t h, const void* data, size_t n) {
+  const unsigned char* p = static_cast<const unsigned char*>(data);
+  for (size_t i = 0; i < n; ++i) {
+    h ^= p[i];
+    h *= 1099511628211ull;
+  }
+  return h;
+}
+
+uint64_t config_hash(const sfa_config* c) {
+  uint64_t h = 1469598103934665603ull;
+  const int ints[] = {c->n_layers, c->n_q_heads, c->n_kv_heads, c->head_dim, c->window_k,
+                      c->ring_size, c->n_slots, c->in_dtype, SFA_ABI_VERSION};
+  const float flts[] = {c->gamma_far, c->alpha_far, c->ema_gamma, c->temperature,
+                        c->clip_eps, c->alpha_base, c->cross_decay};
+  h = fnv1a(h, ints, sizeof(ints));
+  h = fnv1a(h, flts, sizeof(flts));
+  return h;
+}
+
+StreamOffsets stream_offsets(const sfa_config* c) {
+  const long long H = hidden_of(c);
+  const long long win = static_cast<long long>(c->window_k) * c->n_kv_heads * c->head_dim *
+                        static_cast<long long>(in_bytes(c->in_dtype));
+  StreamOffsets o;
+  o.pos = 0;
+  o.win_k = 256;
+  o.win_v = o.win_k + align256(win);
+  o.far = o.win_v + align256(win);
+  o.field = o.far + align256(4LL * c->n_kv_heads * c->head_dim);
+  o.ring_sum = o.field + align256(4 * H);
+  o.ring = o.ring_sum + align256(4 * H);
+  o.stride = o.ring + align256(4LL * kRing * H);
+  return o;
+}
+
+// Smallest cluster whose per-CTA hidden slice is at most `max_slice`.
+int smallest_cluster(int nq, int d, int max_slice) {
+  for (int cs = 1; cs <= kMaxCluster; ++cs)
+    if (nq % cs == 0 && (nq / cs) * d <= max_slice) return cs;
+  return 0;
+}
+
+// Decode: enough CTAs to cover the SMs when there are few streams.
+int decode_cluster(int nq, int d, long long streams) {
+  int best = 0;
+  for (int cs = 1; cs <= kMaxCluster; ++cs) {
+    if (nq % cs != 0 || (nq / cs) * d > kMaxSlice) continue;
+    best = cs;
+    if (streams * cs >= 2 * 148) break;
+  }
+  return best;
+}
+
+int prefill_cluster(int nq, int d) {
+  const int cs = smallest_cluster(nq, d, 256);
+  return cs ? cs : smallest_cluster(nq, d, kMaxSlice);
+}
+
+PrefillWorkspace prefill_workspace(const sfa_config* c, int cs, int batch, long long n) {
+  PrefillWorkspace w;
+  const long long streams = static_cast<long long>(c->n_layers) * batch;
+  const long long tiles = streams * ((n + kTile - 1) / kTile);
+  const long long H = hidden_of(c);
+  const long long sdim = static_cast<long long>(c->n_kv_heads) * c->head_dim;
+  w.flags_s = 256;
+  w.flags_f = w.flags_s + align256(4 * tiles * c->n_kv_heads);
+  w.flags_end = w.flags_f + align256(4 * tiles * cs);
+  w.agg_s = w.flags_end;
+  w.incl_s = w.agg_s + align256(4 * tiles * sdim);
+  w.agg_f = w.incl_s + align256(4 * tiles * sdim);
+  w.incl_f = w.agg_f + align256(4 * tiles * H);
+  w.halo = w.incl_f + align256(4 * tiles * H);
+  w.total = w.halo + align256(4 * tiles * kHalo * H);
+  return w;
+}
+
+bool handle_ok(const sfa_handle* h) { return h != nullptr && h->magic == kHandleMagic; }
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? SFA_OK : SFA_ERR_CUDA; }
+
+template <typename P>
+void fill_common(P& p, const sfa_handle* h, int batch, void* state) {
+  const sfa_config* c = &h->cfg;
+  p.state = static_cast<unsigned char*>(state);
+  p.slots = h->slots;
+  p.slot_norm = h->slot_norm;
+  p.alpha_layer = h->alpha_layer;
+  p.err = h->err;
+  p.cfg_hash = h->cfg_hash;
+  p.so = stream_offsets(c);
+  p.L = c->n_layers;
+  p.B = batch;
+  p.nq = c->n_q_heads;
+  p.nkv = c->n_kv_heads;
+  p.K = c->window_k;
+  p.H = hidden_of(c);
+  p.G = c->n_q_heads / c->n_kv_heads;
+  p.gamma_far = c->gamma_far;
+  p.alpha_far = c->alpha_far;
+  p.ema_gamma = c->ema_gamma;
+  p.inv_temp = 1.0f / c->temperature;
+  p.clip_eps = c->clip_eps;
+  p.score_scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(c->head_dim)));
+}
+
+}  // namespace
+
+extern "C" {
+
+void sfa_config_default(sfa_config* c) {
+  if (!c) return;
+  std::memset(c, 0, sizeof(*c));
+  c->window_k = 16;
+  c->gamma_far = 0.9f;
+  c->alpha_far = 0.1f;
+  c->ring_size = kRing;
+  c->ema_gamma = 0.98f;
+  c->n_slots = kSlots;
+  c->temperature = 0.07f;
+  c->clip_eps = 0.5f;
+  c->alpha_base = 0.1f;
+  c->cross_decay = 0.8f;
+  c->in_dtype = SFA_BF16;
+  c->slots = nullptr;
+}
+
+int sfa_config_validate(const sfa_config* c) {
+  if (!c) return SFA_ERR_INVALID_ARG;
+  if (c->n_layers <= 0 || c->n_q_heads <= 0 || c->n_kv_heads <= 0 || c->head_dim <= 0 ||
+      c->window_k <= 0 || c->ring_size <= 0 || c->n_slots <= 0)
+    return SFA_ERR_INVALID_ARG;
+  if (c->n_q_heads % c->n_kv_heads != 0) return SFA_ERR_INVALID_ARG;
+  const float scalars[] = {c->gamma_far, c->alpha_far, c->ema_gamma, c->temperature,
+                           c->clip_eps, c->alpha_base, c->cross_decay};
+  for (float s : scalars)
+    if (!std::isfinite(s)) return SFA_ERR_INVALID_ARG;
+  if (c->gamma_far < 0.f || c->gamma_far > 1.f || c->ema_gamma < 0.f || c->ema_gamma > 1.f)
+    return SFA_ERR_INVALID_ARG;
+  if (!(c->temperature > 0.f) || c->clip_eps < 0.f) return SFA_ERR_INVALID_ARG;
+  if (c->in_dtype != SFA_F32 && c->in_dtype != SFA_BF16) return SFA_ERR_INVALID_ARG;
+  if (c->slots == nullptr) return SFA_ERR_INVALID_ARG;
+  if (!aligned16(c->slots)) return SFA_ERR_ALIGNMENT;
+  if (c->head_dim != 64 && c->head_dim != 128) return SFA_ERR_UNSUPPORTED;
+  if (c->window_k > kMaxWindow || c->ring_size != kRing || c->n_slots != kSlots)
+    return SFA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(c->n_q_heads) * c->head_dim > kMaxHidden) return SFA_ERR_UNSUPPORTED;
+  if (smallest_cluster(c->n_q_heads, c->head_dim, kMaxSlice) == 0) return SFA_ERR_UNSUPPORTED;
+  return SFA_OK;
+}
+
+int sfa_state_layout_for(const sfa_config* c, int batch, sfa_state_layout* out) {
+  if (!c || !out || batch <= 0) return SFA_ERR_INVALID_ARG;
+  const int v = sfa_config_validate(c);
+  if (v != SFA_OK) return v;
+  const StreamOffsets o = stream_offsets(c);
+  out->header_bytes = kHeaderBytes;
+  out->stream_stride = static_cast<size_t>(o.stride);
+  out->total_bytes = kHeaderBytes + static_cast<size_t>(o.stride) * c->n_layers * batch;
+  out->off_pos = static_cast<size_t>(o.pos);
+  out->off_win_k = static_cast<size_t>(o.win_k);
+  out->off_win_v = static_cast<size_t>(o.win_v);
+  out->off_far = static_cast<size_t>(o.far);
+  out->off_field = static_cast<size_t>(o.field);
+  out->off_ring_sum = static_cast<size_t>(o.ring_sum);
+  out->off_ring = static_cast<size_t>(o.ring);
+  return SFA_OK;
+}
+
+int sfa_init(const sfa_config* cfg, sfa_handle** out) {
+  if (!out) return SFA_ERR_INVALID_ARG;
+  *out = nullptr;
+  const int v = sfa_config_validate(cfg);
+  if (v != SFA_OK) return v;
+  sfa_handle* h = new (std::nothrow) sfa_handle();
+  if (!h) return SFA_ERR_CUDA;
+  h->magic = kHandleMagic;
+  h->cfg = *cfg;
+  h->cfg_hash = config_hash(cfg);
+  h->prefill_cs = prefill_cluster(cfg->n_q_heads, cfg->head_dim);
+  h->spin_limit = kDefaultSpinLimit;
+  h->withhold_tile = -1;
+  const int L = cfg->n_layers, H = hidden_of(cfg);
+  const size_t slot_bytes = sizeof(float) * static_cast<size_t>(L) * kSlots * H;
+  cudaError_t e = cudaGetDevice(&h->device);
+  if (e == cudaSuccess) e = cudaMalloc(&h->slots, slot_bytes);
+  if (e == cudaSuccess) e = cudaMalloc(&h->slot_norm, sizeof(float) * L * kSlots);
+  if (e == cudaSuccess) e = cudaMalloc(&h->alpha_layer, sizeof(float) * L);
+  if (e == cudaSuccess) e = cudaMalloc(&h->err, sizeof(int));
+  if (e == cudaSuccess) e = cudaMemcpy(h->slots, cfg->slots, slot_bytes, cudaMemcpyDefault);
+  if (e == cudaSuccess) e = cudaMemset(h->err, 0, sizeof(int));
+  if (e == cudaSuccess) e = prefill_prepare(h->device);
+  if (e == cudaSuccess &&
+      prefill_smem_bytes(cfg->n_q_heads / h->prefill_cs, cfg->head_dim) > prefill_smem_limit(h->device))
+    e = cudaErrorInvalidConfiguration;
+  if (e == cudaSuccess) e = launch_slot_norms(h->slots, h->slot_norm, L, H, nullptr);
+  if (e == cudaSuccess) {
+    // [P3 §2.2] alpha_layer = alpha_base*(0.3 + 0.7*layer/(L-1))*decay^layer;
+    // the ratio is 0 for a single-layer model.
+    std::vector<float> a(L);
+    for (int l = 0; l < L; ++l) {
+      const double ratio = L > 1 ? static_cast<double>(l) / (L - 1) : 0.0;
+      a[l] = static_cast<float>(static_cast<double>(cfg->alpha_base) * (0.3 + 0.7 * ratio) *
+                                std::pow(static_cast<double>(cfg->cross_decay), l));
+    }
+    e = cudaMemcpy(h->alpha_layer, a.data(), sizeof(float) * L, cudaMemcpyHostToDevice);
+  }
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    cudaFree(h->slots);
+    cudaFree(h->slot_norm);
+    cudaFree(h->alpha_layer);
+    cudaFree(h->err);
+    h->magic = 0;
+    delete h;
+    return SFA_ERR_CUDA;
+  }
+  h->cfg.slots = h->slots;
+  *out = h;
+  return SFA_OK;
+}
+
+int sfa_destroy(sfa_handle* h) {
+  if (!handle_ok(h)) return SFA_ERR_INVALID_ARG;
+  cudaError_t e = cudaDeviceSynchronize();
+  cudaFree(h->slots);
+  cudaFree(h->slot_norm);
+  cudaFree(h->alpha_layer);
+  cudaFree(h->err);
+  h->magic = 0;
+  delete h;
+  return cuda_status(e);
+}
+
+size_t sfa_state_bytes(const sfa_handle* h, int batch) {
+  if (!handle_ok(h) || batch <= 0) return 0;
+  sfa_state_layout lay;
+  if (sfa_state_layout_for(&h->cfg, batch, &lay) != SFA_OK) return 0;
+  return lay.total_bytes;
+}
+
+size_t sfa_prefill_workspace_bytes(const sfa_handle* h, int batch, long long n) {
+  if (!handle_ok(h) || batch <= 0 || n <= 0) return 0;
+  return static_cast<size_t>(prefill_workspace(&h->cfg, h->prefill_cs, batch, n).total);
+}
+
+int sfa_state_reset(const sfa_handle* h, void* state, int batch, void* stream) {
+  if (!handle_ok(h) || !state || batch <= 0) return SFA_ERR_INVALID_ARG;
+  if (!aligned16(state)) return SFA_ERR_ALIGNMENT;
+  const size_t bytes = sfa_state_bytes(h, batch);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(state, 0, bytes, s);
+  if (e != cudaSuccess) return SFA_ERR_CUDA;
+  StateHeader hd;
+  std::memset(&hd, 0, sizeof(hd));
+  hd.magic = kMagic;
+  hd.abi = SFA_ABI_VERSION;
+  hd.cfg_hash = h->cfg_hash;
+  hd.batch = batch;
+  hd.n_layers = h->cfg.n_layers;
+  hd.stream_stride = static_cast<uint64_t>(stream_offsets(&h->cfg).stride);
+  return cuda_status(launch_write_header(static_cast<unsigned char*>(state), hd, s));
+}
+
+int sfa_prefill(const sfa_handle* h, const void* q, const void* k, const void* v, long long n,
+                int batch, void* state, float* out, void* workspace, size_t workspace_bytes,
+                void* stream) {
+  if (!handle_ok(h) || n < 0 || batch <= 0) return SFA_ERR_INVALID_ARG;
+  if (n == 0) return SFA_OK;
+  if (!q || !k || !v || !state || !out) return SFA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(state) || !aligned16(out) ||
+      !aligned16(workspace))
+    return SFA_ERR_ALIGNMENT;
+  const sfa_config* c = &h->cfg;
+  const PrefillWorkspace w = prefill_workspace(c, h->prefill_cs, batch, n);
+  if (!workspace || workspace_bytes < static_cast<size_t>(w.total)) return SFA_ERR_WORKSPACE;
+  const long long streams = static_cast<long long>(c->n_layers) * batch;
+  const long long tiles_per_stream = (n + kTile - 1) / kTile;
+  if (streams * tiles_per_stream * h->prefill_cs > 0x7fffffffLL) return SFA_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // Ticket counter and look-back flags start empty on every call.
+  cudaError_t e = cudaMemsetAsync(workspace, 0, static_cast<size_t>(w.flags_end), s);
+  if (e != cudaSuccess) return SFA_ERR_CUDA;
+  PrefillParams p;
+  std::memset(&p, 0, sizeof(p));
+  fill_common(p, h, batch, state);
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.out = out;
+  p.ws = static_cast<unsigned char*>(workspace);
+  p.n = n;
+  p.CS = h->prefill_cs;
+  p.HPC = c->n_q_heads / p.CS;
+  p.tiles_per_stream = static_cast<int>(tiles_per_stream);
+  p.n_streams = static_cast<int>(streams);
+  p.n_tiles = streams * tiles_per_stream;
+  p.ws_flags_s = w.flags_s;
+  p.ws_flags_f = w.flags_f;
+  p.ws_agg_s = w.agg_s;
+  p.ws_incl_s = w.incl_s;
+  p.ws_agg_f = w.agg_f;
+  p.ws_incl_f = w.incl_f;
+  p.ws_halo = w.halo;
+  p.spin_limit = h->spin_limit;
+  p.withhold_tile = h->withhold_tile;
+  e = launch_prefill(p, c->in_dtype, c->head_dim, prefill_smem_bytes(p.HPC, c->head_dim), s);
+  return cuda_status(e);
+}
+
+int sfa_decode_step(const sfa_handle* h, const void* q, const void* k, const void* v, int batch,
+                    void* state, float* out, void* stream) {
+  if (!handle_ok(h) || batch <= 0 || !q || !k || !v || !state || !out) return SFA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(state) || !aligned16(out))
+    return SFA_ERR_ALIGNMENT;
+  const sfa_config* c = &h->cfg;
+  if (batch > 65535 || c->n_layers > 65535) return SFA_ERR_UNSUPPORTED;
+  DecodeParams p;
+  std::memset(&p, 0, sizeof(p));
+  fill_common(p, h, batch, state);
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.out = out;
+  p.CS = decode_cluster(c->n_q_heads, c->head_dim, static_cast<long long>(c->n_layers) * batch);
+  p.HPC = c->n_q_heads / p.CS;
+  return cuda_status(launch_decode(p, c->in_dtype, c->head_dim, static_cast<cudaStream_t>(stream)));
+}
+
+int sfa_check_device_status(const sfa_handle* h, void* stream) {
+  if (!handle_ok(h)) return SFA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return SFA_ERR_CUDA;
+  int code = 0;
+  e = cudaMemcpy(&code, h->err, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return SFA_ERR_CUDA;
+  if (code != 0) {
+    e = cudaMemset(h->err, 0, sizeof(int));
+    if (e != cudaSuccess) return SFA_ERR_CUDA;
+  }
+  return code;
+}
+
+const char* sfa_status_string(int status) {
+  switch (status) {
+    case SFA_OK: return "ok";
+    case SFA_ERR_INVALID_ARG: return "invalid argument";
+    case SFA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case SFA_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    case SFA_ERR_STATE_MISMATCH: return "state header does not match the handle or batch";
+    case SFA_ERR_CUDA: return "CUDA error";
+    case SFA_ERR_DEVICE_TIMEOUT: return "bounded device wait ran out";
+    case SFA_ERR_WORKSPACE: return "workspace too small";
+    default: return "unknown status";
+  }
+}
+
+int sfa_abi_version(void) { return SFA_ABI_VERSION; }
+
+int sfa_debug_set_lookback(sfa_handle* h, unsigned int spin_limit, long long withhold_tile) {
+  if (!handle_ok(h)) return SFA_ERR_INVALID_ARG;
+  h->spin_limit = spin_limit ? spin_limit : kDefaultSpinLimit;
+  h->withhold_tile = withhold_tile < 0 ? -1 : withhold_tile;
+  return SFA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,115 @@
+// sfa_internal.h — layouts and kernel parameter blocks shared by the host
+// launch layer (sfa_api.cu) and the kernels (sfa_decode.cu, sfa_prefill.cu).
+//
+// Sources (web pages):
+//   [P1] "Signal Field Attention (SFA)：8KB代码实现4.16倍推理加速与248倍内存压缩"
+//   [P2] "Signal Field Attention (SFA)" (project README page)
+//   [P3] "Dalin Soma SFA基于信号场注意力机制的神经网络推理加速框架"
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cstddef>
+#include <cstdint>
+
+#include "sfa.h"
+
+namespace sfa {
+
+constexpr uint32_t kMagic = 0x31414653u;  // "SFA1"
+constexpr size_t kHeaderBytes = 256;
+constexpr int kRing = 16;                 // ring-buffer slots [P3 §2.1 channel 1]
+constexpr int kSlots = 64;                // semantic slots [P3 §2.1 channel 3]
+constexpr int kMaxHidden = 8192;
+constexpr int kMaxWindow = 256;
+constexpr int kMaxSlice = 512;            // hidden elements owned by one CTA
+constexpr int kMaxCluster = 8;            // portable cluster size
+constexpr float kNormFloor = 1e-12f;      // cosine norm clamp
+
+// Prefill tiling.
+constexpr int kTile = 64;                 // tokens per prefill tile
+constexpr int kHalo = kRing - 1;          // x rows a tile needs from before it
+constexpr int kPrefillThreads = 256;
+constexpr int kDecodeThreads = 128;
+
+// Look-back flag values.
+constexpr unsigned kFlagEmpty = 0u;
+constexpr unsigned kFlagAgg = 1u;
+constexpr unsigned kFlagIncl = 2u;
+constexpr unsigned kDefaultSpinLimit = 1u << 21;
+
+// First bytes of every state buffer.
+struct StateHeader {
+  uint32_t magic;
+  uint32_t abi;
+  uint64_t cfg_hash;
+  int32_t batch;
+  int32_t n_layers;
+  uint64_t stream_stride;
+};
+static_assert(sizeof(StateHeader) <= kHeaderBytes, "header too large");
+
+// Byte offsets inside one (layer, sequence) stream block.
+struct StreamOffsets {
+  long long pos, win_k, win_v, far, field, ring_sum, ring;
+  long long stride;
+};
+
+struct DecodeParams {
+  const void* q;
+  const void* k;
+  const void* v;
+  float* out;
+  unsigned char* state;
+  const float* slots;       // [L][64][H]
+  const float* slot_norm;   // [L][64], clamped at kNormFloor
+  const float* alpha_layer; // [L]
+  int* err;
+  uint64_t cfg_hash;
+  StreamOffsets so;
+  int L, B, nq, nkv, K, H, G, CS, HPC;
+  float gamma_far, alpha_far, ema_gamma, inv_temp, clip_eps, score_scale;
+};
+
+struct PrefillParams {
+  const void* q;
+  const void* k;
+  const void* v;
+  float* out;
+  unsigned char* state;
+  unsigned char* ws;
+  const float* slots;
+  const float* slot_norm;
+  const float* alpha_layer;
+  int* err;
+  uint64_t cfg_hash;
+  StreamOffsets so;
+  long long n;              // tokens per stream in this call
+  int L, B, nq, nkv, K, H, G, CS, HPC;
+  int tiles_per_stream, n_streams;
+  long long n_tiles;
+  // workspace byte offsets
+  long long ws_flags_s, ws_flags_f, ws_agg_s, ws_incl_s, ws_agg_f, ws_incl_f, ws_halo;
+  float gamma_far, alpha_far, ema_gamma, inv_temp, clip_eps, score_scale;
+  unsigned spin_limit;
+  long long withhold_tile;
+};
+
+// Workspace layout for a prefill call (bytes).
+struct PrefillWorkspace {
+  long long flags_s, flags_f, flags_end;  // [0, flags_end) is cleared per call
+  long long agg_s, incl_s, agg_f, incl_f, halo, total;
+};
+
+inline long long align256(long long x) { return (x + 255) & ~255LL; }
+
+// Launchers (return the CUDA error of the launch).
+cudaError_t launch_decode(const DecodeParams& p, int in_dtype, int head_dim, cudaStream_t s);
+cudaError_t launch_prefill(const PrefillParams& p, int in_dtype, int head_dim,
+                           size_t smem_bytes, cudaStream_t s);
+size_t prefill_smem_bytes(int HPC, int head_dim);
+cudaError_t prefill_prepare(int device);
+size_t prefill_smem_limit(int device);
+cudaError_t launch_write_header(unsigned char* state, StateHeader h, cudaStream_t s);
+cudaError_t launch_slot_norms(const float* slots, float* norms, int L, int H, cudaStream_t s);
+
+}  // namespace sfa
