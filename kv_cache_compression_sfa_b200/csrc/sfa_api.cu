@@ -12,6 +12,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <algorithm>
 #include <cstring>
 #include <new>
 #include <vector>
@@ -30,6 +31,7 @@ struct sfa_handle {
   int* err;              // device error word
   uint64_t cfg_hash;
   int prefill_cs;
+  PrefillPlan plan;
   unsigned spin_limit;
   long long withhold_tile;
 };
@@ -87,20 +89,16 @@ int smallest_cluster(int nq, int d, int max_slice) {
   return 0;
 }
 
-// Decode: enough CTAs to cover the SMs when there are few streams.
-int decode_cluster(int nq, int d, long long streams) {
-  int best = 0;
-  for (int cs = 1; cs <= kMaxCluster; ++cs) {
-    if (nq % cs != 0 || (nq / cs) * d > kMaxSlice) continue;
-    best = cs;
-    if (streams * cs >= 2 * 148) break;
-  }
-  return best;
-}
-
-int prefill_cluster(int nq, int d) {
-  const int cs = smallest_cluster(nq, d, 256);
-  return cs ? cs : smallest_cluster(nq, d, kMaxSlice);
+// Cluster sizes to try, best first: slices of at most 256 hidden elements
+// (smallest cluster first), then at most 512.
+std::vector<int> cluster_candidates(int nq, int d) {
+  std::vector<int> out;
+  for (int lim : {256, kMaxSlice})
+    for (int cs = 1; cs <= kMaxCluster; ++cs)
+      if (nq % cs == 0 && (nq / cs) * d <= lim &&
+          std::find(out.begin(), out.end(), cs) == out.end())
+        out.push_back(cs);
+  return out;
 }
 
 PrefillWorkspace prefill_workspace(const sfa_config* c, int cs, int batch, long long n) {
@@ -109,9 +107,11 @@ PrefillWorkspace prefill_workspace(const sfa_config* c, int cs, int batch, long 
   const long long tiles = streams * ((n + kTile - 1) / kTile);
   const long long H = hidden_of(c);
   const long long sdim = static_cast<long long>(c->n_kv_heads) * c->head_dim;
-  w.flags_s = 256;
-  w.flags_f = w.flags_s + align256(4 * tiles * c->n_kv_heads);
-  w.flags_end = w.flags_f + align256(4 * tiles * cs);
+  w.fs_agg = 256;  // [0, 256): ticket counter
+  w.fs_incl = w.fs_agg + align256(4 * tiles * c->n_kv_heads);
+  w.ff_agg = w.fs_incl + align256(4 * tiles * c->n_kv_heads);
+  w.ff_incl = w.ff_agg + align256(4 * tiles * cs);
+  w.flags_end = w.ff_incl + align256(4 * tiles * cs);
   w.agg_s = w.flags_end;
   w.incl_s = w.agg_s + align256(4 * tiles * sdim);
   w.agg_f = w.incl_s + align256(4 * tiles * sdim);
@@ -119,6 +119,17 @@ PrefillWorkspace prefill_workspace(const sfa_config* c, int cs, int batch, long 
   w.halo = w.incl_f + align256(4 * tiles * H);
   w.total = w.halo + align256(4 * tiles * kHalo * H);
   return w;
+}
+
+// Most KV heads any CTA of a cluster of `cs` needs.
+int max_kv_heads_per_cta(int nq, int nkv, int cs) {
+  const int hpc = nq / cs, g = nq / nkv;
+  int best = 0;
+  for (int r = 0; r < cs; ++r) {
+    const int h0 = r * hpc;
+    best = std::max(best, (h0 + hpc - 1) / g - h0 / g + 1);
+  }
+  return best;
 }
 
 bool handle_ok(const sfa_handle* h) { return h != nullptr && h->magic == kHandleMagic; }
@@ -223,7 +234,7 @@ int sfa_init(const sfa_config* cfg, sfa_handle** out) {
   h->magic = kHandleMagic;
   h->cfg = *cfg;
   h->cfg_hash = config_hash(cfg);
-  h->prefill_cs = prefill_cluster(cfg->n_q_heads, cfg->head_dim);
+  h->prefill_cs = 0;
   h->spin_limit = kDefaultSpinLimit;
   h->withhold_tile = -1;
   const int L = cfg->n_layers, H = hidden_of(cfg);
@@ -236,9 +247,28 @@ int sfa_init(const sfa_config* cfg, sfa_handle** out) {
   if (e == cudaSuccess) e = cudaMemcpy(h->slots, cfg->slots, slot_bytes, cudaMemcpyDefault);
   if (e == cudaSuccess) e = cudaMemset(h->err, 0, sizeof(int));
   if (e == cudaSuccess) e = prefill_prepare(h->device);
-  if (e == cudaSuccess &&
-      prefill_smem_bytes(cfg->n_q_heads / h->prefill_cs, cfg->head_dim) > prefill_smem_limit(h->device))
-    e = cudaErrorInvalidConfiguration;
+  if (e == cudaSuccess) e = decode_prepare(h->device);
+  if (e == cudaSuccess) {
+    // First cluster size for which both kernels have a shared-memory plan
+    // and at least one cluster fits on the device.
+    const size_t limit = prefill_smem_limit(h->device);
+    for (int cs : cluster_candidates(cfg->n_q_heads, cfg->head_dim)) {
+      const int hpc = cfg->n_q_heads / cs;
+      PrefillPlan plan;
+      if (!plan_prefill(hpc, cfg->head_dim, static_cast<int>(in_bytes(cfg->in_dtype)),
+                        max_kv_heads_per_cta(cfg->n_q_heads, cfg->n_kv_heads, cs), cfg->window_k,
+                        limit, &plan))
+        continue;
+      const size_t dsm = decode_smem_bytes(hpc, cfg->head_dim);
+      if (dsm > limit) continue;
+      if (prefill_max_active_clusters(cs, plan.total, cfg->in_dtype, cfg->head_dim) < 1) continue;
+      if (decode_max_active_clusters(cs, dsm, cfg->in_dtype, cfg->head_dim) < 1) continue;
+      h->prefill_cs = cs;
+      h->plan = plan;
+      break;
+    }
+    if (h->prefill_cs == 0) e = cudaErrorInvalidConfiguration;
+  }
   if (e == cudaSuccess) e = launch_slot_norms(h->slots, h->slot_norm, L, H, nullptr);
   if (e == cudaSuccess) {
     // [P3 §2.2] alpha_layer = alpha_base*(0.3 + 0.7*layer/(L-1))*decay^layer;
@@ -342,8 +372,13 @@ int sfa_prefill(const sfa_handle* h, const void* q, const void* k, const void* v
   p.tiles_per_stream = static_cast<int>(tiles_per_stream);
   p.n_streams = static_cast<int>(streams);
   p.n_tiles = streams * tiles_per_stream;
-  p.ws_flags_s = w.flags_s;
-  p.ws_flags_f = w.flags_f;
+  p.NGm = max_kv_heads_per_cta(c->n_q_heads, c->n_kv_heads, p.CS);
+  p.plan = h->plan;
+  p.KB = h->plan.KB;
+  p.ws_fs_agg = w.fs_agg;
+  p.ws_fs_incl = w.fs_incl;
+  p.ws_ff_agg = w.ff_agg;
+  p.ws_ff_incl = w.ff_incl;
   p.ws_agg_s = w.agg_s;
   p.ws_incl_s = w.incl_s;
   p.ws_agg_f = w.agg_f;
@@ -351,7 +386,7 @@ int sfa_prefill(const sfa_handle* h, const void* q, const void* k, const void* v
   p.ws_halo = w.halo;
   p.spin_limit = h->spin_limit;
   p.withhold_tile = h->withhold_tile;
-  e = launch_prefill(p, c->in_dtype, c->head_dim, prefill_smem_bytes(p.HPC, c->head_dim), s);
+  e = launch_prefill(p, c->in_dtype, c->head_dim, s);
   return cuda_status(e);
 }
 
@@ -369,7 +404,7 @@ int sfa_decode_step(const sfa_handle* h, const void* q, const void* k, const voi
   p.k = k;
   p.v = v;
   p.out = out;
-  p.CS = decode_cluster(c->n_q_heads, c->head_dim, static_cast<long long>(c->n_layers) * batch);
+  p.CS = h->prefill_cs;
   p.HPC = c->n_q_heads / p.CS;
   return cuda_status(launch_decode(p, c->in_dtype, c->head_dim, static_cast<cudaStream_t>(stream)));
 }

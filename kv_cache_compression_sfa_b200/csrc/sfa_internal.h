@@ -22,7 +22,7 @@ constexpr int kSlots = 64;                // semantic slots [P3 §2.1 channel 3]
 constexpr int kMaxHidden = 8192;
 constexpr int kMaxWindow = 256;
 constexpr int kMaxSlice = 512;            // hidden elements owned by one CTA
-constexpr int kMaxCluster = 8;            // portable cluster size
+constexpr int kMaxCluster = 16;           // largest (non-portable) cluster size
 constexpr float kNormFloor = 1e-12f;      // cosine norm clamp
 
 // Prefill tiling.
@@ -30,6 +30,7 @@ constexpr int kTile = 64;                 // tokens per prefill tile
 constexpr int kHalo = kRing - 1;          // x rows a tile needs from before it
 constexpr int kPrefillThreads = 256;
 constexpr int kDecodeThreads = 128;
+constexpr int kGroup = 16;                // tiles per look-back group
 
 // Look-back flag values.
 constexpr unsigned kFlagEmpty = 0u;
@@ -70,6 +71,16 @@ struct DecodeParams {
   float gamma_far, alpha_far, ema_gamma, inv_temp, clip_eps, score_scale;
 };
 
+// Shared-memory plan of the prefill kernel (byte offsets).
+struct PrefillPlan {
+  int bars, xs, halo, fcar, sst, sagg, ml;  // persistent regions
+  int u0;                                   // start of the union below
+  int qst, kb, vb;                          // near-field staging (phase 1)
+  int sl, part, wts, semc;                  // pool buffers (phase 2)
+  int KB;                                   // rows per staged key/value block
+  int total;
+};
+
 struct PrefillParams {
   const void* q;
   const void* k;
@@ -85,18 +96,22 @@ struct PrefillParams {
   StreamOffsets so;
   long long n;              // tokens per stream in this call
   int L, B, nq, nkv, K, H, G, CS, HPC;
+  int NGm;                  // most KV heads any CTA needs
+  int KB;                   // rows per staged key/value block
   int tiles_per_stream, n_streams;
   long long n_tiles;
   // workspace byte offsets
-  long long ws_flags_s, ws_flags_f, ws_agg_s, ws_incl_s, ws_agg_f, ws_incl_f, ws_halo;
+  long long ws_fs_agg, ws_fs_incl, ws_ff_agg, ws_ff_incl;
+  long long ws_agg_s, ws_incl_s, ws_agg_f, ws_incl_f, ws_halo;
   float gamma_far, alpha_far, ema_gamma, inv_temp, clip_eps, score_scale;
   unsigned spin_limit;
   long long withhold_tile;
+  PrefillPlan plan;
 };
 
 // Workspace layout for a prefill call (bytes).
 struct PrefillWorkspace {
-  long long flags_s, flags_f, flags_end;  // [0, flags_end) is cleared per call
+  long long fs_agg, fs_incl, ff_agg, ff_incl, flags_end;  // [0, flags_end) cleared per call
   long long agg_s, incl_s, agg_f, incl_f, halo, total;
 };
 
@@ -104,10 +119,13 @@ inline long long align256(long long x) { return (x + 255) & ~255LL; }
 
 // Launchers (return the CUDA error of the launch).
 cudaError_t launch_decode(const DecodeParams& p, int in_dtype, int head_dim, cudaStream_t s);
-cudaError_t launch_prefill(const PrefillParams& p, int in_dtype, int head_dim,
-                           size_t smem_bytes, cudaStream_t s);
-size_t prefill_smem_bytes(int HPC, int head_dim);
+cudaError_t launch_prefill(const PrefillParams& p, int in_dtype, int head_dim, cudaStream_t s);
+bool plan_prefill(int HPC, int D, int esz, int NGm, int K, size_t budget, PrefillPlan* out);
 cudaError_t prefill_prepare(int device);
+cudaError_t decode_prepare(int device);
+size_t decode_smem_bytes(int HPC, int head_dim);
+int prefill_max_active_clusters(int cs, size_t smem, int in_dtype, int head_dim);
+int decode_max_active_clusters(int cs, size_t smem, int in_dtype, int head_dim);
 size_t prefill_smem_limit(int device);
 cudaError_t launch_write_header(unsigned char* state, StateHeader h, cudaStream_t s);
 cudaError_t launch_slot_norms(const float* slots, float* norms, int L, int H, cudaStream_t s);
