@@ -13,6 +13,7 @@
 #include <cmath>
 #include <cstdint>
 #include <algorithm>
+#include <type_traits>
 #include <cstring>
 #include <new>
 #include <vector>
@@ -28,10 +29,12 @@ struct sfa_handle {
   float* slots;          // [L][64][H]
   float* slot_norm;      // [L][64]
   float* alpha_layer;    // [L]
+  unsigned char* slot_img;  // [L][H/64][hi, lo] bf16 blocks for the prefill pool MMAs
   int* err;              // device error word
   uint64_t cfg_hash;
   int prefill_cs;
   PrefillPlan plan;
+  int decode_budget;
   unsigned spin_limit;
   long long withhold_tile;
 };
@@ -132,6 +135,10 @@ int max_kv_heads_per_cta(int nq, int nkv, int cs) {
   return best;
 }
 
+int decode_budget(size_t limit) {
+  return static_cast<int>(std::min(static_cast<size_t>(kDecodeSmemBudget), limit));
+}
+
 bool handle_ok(const sfa_handle* h) { return h != nullptr && h->magic == kHandleMagic; }
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? SFA_OK : SFA_ERR_CUDA; }
@@ -142,6 +149,7 @@ void fill_common(P& p, const sfa_handle* h, int batch, void* state) {
   p.state = static_cast<unsigned char*>(state);
   p.slots = h->slots;
   p.slot_norm = h->slot_norm;
+  if constexpr (std::is_same<P, PrefillParams>::value) p.slot_img = h->slot_img;
   p.alpha_layer = h->alpha_layer;
   p.err = h->err;
   p.cfg_hash = h->cfg_hash;
@@ -244,6 +252,7 @@ int sfa_init(const sfa_config* cfg, sfa_handle** out) {
   if (e == cudaSuccess) e = cudaMalloc(&h->slot_norm, sizeof(float) * L * kSlots);
   if (e == cudaSuccess) e = cudaMalloc(&h->alpha_layer, sizeof(float) * L);
   if (e == cudaSuccess) e = cudaMalloc(&h->err, sizeof(int));
+  if (e == cudaSuccess) e = cudaMalloc(&h->slot_img, slot_bytes);  // bf16 hi + lo per slot element
   if (e == cudaSuccess) e = cudaMemcpy(h->slots, cfg->slots, slot_bytes, cudaMemcpyDefault);
   if (e == cudaSuccess) e = cudaMemset(h->err, 0, sizeof(int));
   if (e == cudaSuccess) e = prefill_prepare(h->device);
@@ -259,17 +268,21 @@ int sfa_init(const sfa_config* cfg, sfa_handle** out) {
                         max_kv_heads_per_cta(cfg->n_q_heads, cfg->n_kv_heads, cs), cfg->window_k,
                         limit, &plan))
         continue;
-      const size_t dsm = decode_smem_bytes(hpc, cfg->head_dim);
+      const size_t dsm = decode_smem_bytes(hpc, cfg->head_dim, static_cast<int>(in_bytes(cfg->in_dtype)),
+                                           max_kv_heads_per_cta(cfg->n_q_heads, cfg->n_kv_heads, cs),
+                                           cfg->window_k, decode_budget(limit));
       if (dsm > limit) continue;
       if (prefill_max_active_clusters(cs, plan.total, cfg->in_dtype, cfg->head_dim) < 1) continue;
       if (decode_max_active_clusters(cs, dsm, cfg->in_dtype, cfg->head_dim) < 1) continue;
       h->prefill_cs = cs;
       h->plan = plan;
+      h->decode_budget = decode_budget(limit);
       break;
     }
     if (h->prefill_cs == 0) e = cudaErrorInvalidConfiguration;
   }
   if (e == cudaSuccess) e = launch_slot_norms(h->slots, h->slot_norm, L, H, nullptr);
+  if (e == cudaSuccess) e = launch_slot_image(h->slots, h->slot_img, L, H, nullptr);
   if (e == cudaSuccess) {
     // [P3 §2.2] alpha_layer = alpha_base*(0.3 + 0.7*layer/(L-1))*decay^layer;
     // the ratio is 0 for a single-layer model.
@@ -287,6 +300,7 @@ int sfa_init(const sfa_config* cfg, sfa_handle** out) {
     cudaFree(h->slots);
     cudaFree(h->slot_norm);
     cudaFree(h->alpha_layer);
+    cudaFree(h->slot_img);
     cudaFree(h->err);
     h->magic = 0;
     delete h;
@@ -303,6 +317,7 @@ int sfa_destroy(sfa_handle* h) {
   cudaFree(h->slots);
   cudaFree(h->slot_norm);
   cudaFree(h->alpha_layer);
+  cudaFree(h->slot_img);
   cudaFree(h->err);
   h->magic = 0;
   delete h;
@@ -406,6 +421,8 @@ int sfa_decode_step(const sfa_handle* h, const void* q, const void* k, const voi
   p.out = out;
   p.CS = h->prefill_cs;
   p.HPC = c->n_q_heads / p.CS;
+  p.NGm = max_kv_heads_per_cta(c->n_q_heads, c->n_kv_heads, p.CS);
+  p.smem_budget = h->decode_budget;
   return cuda_status(launch_decode(p, c->in_dtype, c->head_dim, static_cast<cudaStream_t>(stream)));
 }
 

@@ -97,6 +97,20 @@ struct Load16<__nv_bfloat16> {
   }
 };
 
+template <>
+struct VecLoad<float, 8> {
+  __device__ __forceinline__ static void run(const float* p, float* o) {
+    VecLoad<float, 4>::run(p, o);
+    VecLoad<float, 4>::run(p + 4, o + 4);
+  }
+};
+template <>
+struct VecLoad<__nv_bfloat16, 8> {
+  __device__ __forceinline__ static void run(const __nv_bfloat16* p, float* o) {
+    Load16<__nv_bfloat16>::run(p, o);
+  }
+};
+
 template <typename T>
 __device__ __forceinline__ float to_f32(T v);
 template <>
@@ -191,6 +205,15 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, unsigned by
 // later bulk copies (async proxy) into the same bytes.
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Split cluster barrier: arrive (release) once this CTA is done reading its
+// peers' shared memory, wait (acquire) before leaving.
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
 // ---- programmatic dependent launch ----------------------------------------

@@ -68,8 +68,12 @@ struct DecodeParams {
   uint64_t cfg_hash;
   StreamOffsets so;
   int L, B, nq, nkv, K, H, G, CS, HPC;
+  int NGm;          // most KV heads any CTA needs
+  int smem_budget;  // shared-memory bytes the plan may use (window staged if it fits)
   float gamma_far, alpha_far, ema_gamma, inv_temp, clip_eps, score_scale;
 };
+
+constexpr int kDecodeSmemBudget = 112 * 1024;  // keeps two decode CTAs per SM
 
 // Shared-memory plan of the prefill kernel (byte offsets).
 struct PrefillPlan {
@@ -91,6 +95,7 @@ struct PrefillParams {
   const float* slots;
   const float* slot_norm;
   const float* alpha_layer;
+  const unsigned char* slot_img;  // pre-split bf16 slot blocks
   int* err;
   uint64_t cfg_hash;
   StreamOffsets so;
@@ -123,11 +128,14 @@ cudaError_t launch_prefill(const PrefillParams& p, int in_dtype, int head_dim, c
 bool plan_prefill(int HPC, int D, int esz, int NGm, int K, size_t budget, PrefillPlan* out);
 cudaError_t prefill_prepare(int device);
 cudaError_t decode_prepare(int device);
-size_t decode_smem_bytes(int HPC, int head_dim);
+size_t decode_smem_bytes(int HPC, int head_dim, int esz, int NGm, int K, int budget);
 int prefill_max_active_clusters(int cs, size_t smem, int in_dtype, int head_dim);
 int decode_max_active_clusters(int cs, size_t smem, int in_dtype, int head_dim);
 size_t prefill_smem_limit(int device);
 cudaError_t launch_write_header(unsigned char* state, StateHeader h, cudaStream_t s);
 cudaError_t launch_slot_norms(const float* slots, float* norms, int L, int H, cudaStream_t s);
+// Pre-split bf16 slot blocks for the prefill pool MMAs ([L][H/64][hi, lo]
+// 64 x 64 blocks, 8 KB each); H must be a multiple of 64.
+cudaError_t launch_slot_image(const float* slots, unsigned char* img, int L, int H, cudaStream_t s);
 
 }  // namespace sfa

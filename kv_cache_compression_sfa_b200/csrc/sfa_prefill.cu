@@ -17,8 +17,15 @@
 // t0-k .. t0+T-1: the windows plus the keys that leave them) are brought
 // into shared memory by the bulk-copy engine in key blocks of up to KB rows;
 // the near field runs an online softmax per (token, head) across the blocks
-// with the running output kept in the x tile.  The slot slice is staged once
-// per tile and feeds both pool contractions.
+// with the running output kept in the x tile (two (token, head) pairs per
+// warp when k <= 16).
+//
+// Semantic pool on the tensor cores (tcgen05, accumulators in tensor
+// memory): scores[T x 64] = x[T x HS] . slot^T and sem[T x HS] =
+// w[T x 64] . slot, each as three bf16 MMAs (hi*hi + hi*lo + lo*hi of the
+// split operands, about 16 significant bits) accumulated in fp32.  The slot
+// slice arrives by bulk copy as bf16 hi/lo blocks laid out at sfa_init so
+// that one copy feeds both contractions.
 //
 // Recurrences as parallel scans across tiles, with a deterministic
 // look-back: tiles are grouped by kGroup; a tile's carry-in is the inclusive
@@ -32,16 +39,17 @@
 // Every wait is bounded; a wait that runs out latches SFA_ERR_DEVICE_TIMEOUT
 // and the kernel still finishes.
 //
-// The semantic pool needs |x| and x·slot_j over all of hidden: partial sums
-// of the slice are reduce-scattered across the cluster through distributed
-// shared memory (rank r finishes tokens r, r+CS, ...) and the softmax
-// weights are written into every CTA's shared memory.
+// The pool needs |x| and x·slot_j over all of hidden: partial sums of the
+// slice are reduce-scattered across the cluster through distributed shared
+// memory (rank r finishes tokens r, r+CS, ...) and the softmax weights are
+// written into every CTA's shared memory.
 #include <cooperative_groups.h>
 #include <cuda_bf16.h>
 
 #include <algorithm>
 
 #include "sfa_common.cuh"
+#include "sfa_umma.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -51,14 +59,106 @@ namespace {
 constexpr int NT = kPrefillThreads;
 constexpr int NW = NT / 32;
 constexpr int kPartStride = kSlots + 1;  // 64 partial dots + |x|^2 per token
-constexpr int kCW = 64;                  // columns per combine chunk
+constexpr int kCW = kBlk;                // columns per combine chunk
+constexpr int kSemStride = kCW + 4;      // padded row of the sem chunk
 constexpr int kSeg = 4;                  // token segments per column in the epilogue
 constexpr int kEvChunk = 16;             // evicted-key loads in flight per thread
+constexpr int kTmemCols = 256;           // scores (64) + two 64-column sem buffers
+static_assert(kTile == kBlk, "tile tokens are the M of the pool MMAs");
+
+// Near field over one staged key block for all (token, head) pairs of the
+// tile [P1 §2.1 eq. O_near].  LP lanes serve one pair: lane a scores key
+// lo+base+a in full, online softmax across chunks and blocks, then P·V with
+// the LP lanes over head dims, accumulated into the pair's row of the x
+// tile.  Running max and denominator per pair live in mrun/lrun.
+template <typename Tin, int D, int LP>
+__device__ __forceinline__ void near_block(const Tin* qst, const unsigned char* kb,
+                                           const unsigned char* vb, float* xs, float* mrun,
+                                           float* lrun, int rowB, int HS, int XS, int HPC, int G,
+                                           int g_lo, int K, long long t0, int Tt, long long bs,
+                                           long long be, float score_scale, int h0, int warp,
+                                           int lane) {
+  constexpr int PPW = 32 / LP;  // pairs per warp
+  constexpr int EPL = D / LP;   // head dims per lane in P·V
+  constexpr int VE = Load16<Tin>::N;
+  const int sub = lane / LP, sl = lane % LP;
+  const int gbase = sub * LP;   // first lane of this sub-group
+  for (int pb = warp * PPW; pb < Tt * HPC; pb += NW * PPW) {
+    const int pair = pb + sub;
+    const bool live = pair < Tt * HPC;
+    const int r = live ? pair / HPC : 0;
+    const int hh = live ? pair % HPC : 0;
+    const int gg = (h0 + hh) / G - g_lo;  // KV head of this pair, local to the CTA
+    const long long pt = t0 + r;
+    const long long wlo = pt - K + 1 > 0 ? pt - K + 1 : 0;
+    const long long lo = wlo > bs ? wlo : bs;
+    const long long hi = pt < be - 1 ? pt : be - 1;
+    const int cnt_pair = (live && lo <= hi) ? static_cast<int>(hi - lo + 1) : 0;
+    int cnt_max = cnt_pair;  // the sub-pairs of a warp run the same number of chunks
+    if (LP < 32) cnt_max = max(cnt_max, __shfl_xor_sync(0xffffffffu, cnt_max, 16));
+    if (cnt_max == 0) continue;
+    float* orow = xs + r * XS + hh * D + sl * EPL;
+    float m = live ? mrun[pair] : 0.f;
+    float den = live ? lrun[pair] : 0.f;
+    float o[EPL];
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) o[e] = live ? orow[e] : 0.f;
+    const Tin* qrow = qst + r * HS + hh * D;
+    for (int base = 0; base < cnt_max; base += LP) {
+      const int cnt = max(0, min(LP, cnt_pair - base));
+      float s = -INFINITY;
+      if (sl < cnt) {
+        const Tin* kr = reinterpret_cast<const Tin*>(kb + (lo + base + sl - bs) * rowB) + gg * D;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};  // independent chains
+#pragma unroll
+        for (int i = 0; i < D; i += VE) {
+          float kv[VE], qv[VE];
+          Load16<Tin>::run(kr + i, kv);
+          Load16<Tin>::run(qrow + i, qv);
+#pragma unroll
+          for (int e = 0; e < VE; ++e) acc[e & 3] = fmaf(qv[e], kv[e], acc[e & 3]);
+        }
+        s = ((acc[0] + acc[1]) + (acc[2] + acc[3])) * score_scale;
+      }
+      float cm = s;
+#pragma unroll
+      for (int off = LP / 2; off > 0; off >>= 1) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, off));
+      const float mn = (cnt > 0) ? fmaxf(m, cm) : m;
+      const float corr = (cnt > 0) ? expf(m - mn) : 1.f;
+      const float pj = (sl < cnt) ? expf(s - mn) : 0.f;
+      float ps = pj;
+#pragma unroll
+      for (int off = LP / 2; off > 0; off >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
+      den = fmaf(den, corr, ps);
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) o[e] *= corr;
+      const int cmax = min(LP, cnt_max - base);
+      for (int c = 0; c < cmax; ++c) {
+        const float pc = __shfl_sync(0xffffffffu, pj, gbase + c);
+        if (c < cnt) {
+          const Tin* vr = reinterpret_cast<const Tin*>(vb + (lo + base + c - bs) * rowB) + gg * D + sl * EPL;
+          float vv[EPL];
+          VecLoad<Tin, EPL>::run(vr, vv);
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) o[e] = fmaf(pc, vv[e], o[e]);
+        }
+      }
+      m = mn;
+    }
+    if (live) {
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) orow[e] = o[e];
+      if (sl == 0) {
+        mrun[pair] = m;
+        lrun[pair] = den;
+      }
+    }
+  }
+}
 
 template <typename Tin, int D>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
 prefill_kernel(const PrefillParams p) {
-  constexpr int EPL = D / 32;
   constexpr int ESZ = static_cast<int>(sizeof(Tin));
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = static_cast<int>(cluster.block_rank());
@@ -68,6 +168,14 @@ prefill_kernel(const PrefillParams p) {
   const PrefillPlan& pl = p.plan;
   const int HPC = p.HPC;
   const int HS = HPC * D, XS = HS + 4;
+  const int nch = HS / kBlk;                               // 64-column chunks of the slice
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smb + pl.bars);
+  uint64_t* bar_kv = bars + 0;                             // key/value blocks (+ queries)
+  uint64_t* bar_sl = bars + 1;                             // slot image
+  uint64_t* bar_ms = bars + 2;                             // [2] score MMAs done, per x buffer
+  uint64_t* bar_sd = bars + 4;                             // all score MMAs done
+  uint64_t* bar_mc = bars + 5;                             // [2] sem MMAs done, per accumulator
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8);
   float* xs = reinterpret_cast<float*>(smb + pl.xs);      // [T][XS]  x (O accumulator first)
   float* halo = reinterpret_cast<float*>(smb + pl.halo);  // [15][HS] x of the 15 tokens before
   float* fcar = reinterpret_cast<float*>(smb + pl.fcar);  // [HS]     field carried in
@@ -76,15 +184,14 @@ prefill_kernel(const PrefillParams p) {
   float* mrun = reinterpret_cast<float*>(smb + pl.ml);    // [T*HPC]  running max
   float* lrun = mrun + kTile * HPC;                       // [T*HPC]  running denominator
   float* segc = lrun + kTile * HPC;                       // [kSeg][kCW] epilogue carries
-  uint64_t* bar_kv = reinterpret_cast<uint64_t*>(smb + pl.bars);
-  uint64_t* bar_sl = bar_kv + 1;
   Tin* qst = reinterpret_cast<Tin*>(smb + pl.qst);        // [T][HS]   queries
   unsigned char* kb = smb + pl.kb;                        // [KB][rowB] key block
   unsigned char* vb = smb + pl.vb;                        // [KB][rowB] value block
-  float* sl = reinterpret_cast<float*>(smb + pl.sl);      // [64][XS]  slot slice
+  unsigned char* simg = smb + pl.sl;                      // [nch][hi,lo] slot blocks
   float* part = reinterpret_cast<float*>(smb + pl.part);  // [T][65]   pool partials
   float* wts = reinterpret_cast<float*>(smb + pl.wts);    // [T][64]   pool weights
-  float* semc = reinterpret_cast<float*>(smb + pl.semc);  // [T][kCW]  semantic chunk
+  unsigned char* xw = smb + pl.semc;                      // x blocks [2][hi,lo] | w blocks + sem chunk
+  float* semc = reinterpret_cast<float*>(xw + 2 * kBlkBytes);  // [T][kSemStride]
 
   __shared__ unsigned long long s_ticket;
   __shared__ long long s_pos;
@@ -92,8 +199,7 @@ prefill_kernel(const PrefillParams p) {
   __shared__ int s_bad;  // a staging wait ran out: skip global writes
 
   if (tid == 0) {
-    mbar_init(bar_kv, 1);
-    mbar_init(bar_sl, 1);
+    for (int i = 0; i < 7; ++i) mbar_init(bars + i, 1);
     mbar_fence_init();
     s_bad = 0;
   }
@@ -103,9 +209,13 @@ prefill_kernel(const PrefillParams p) {
   // ---- ticket: the tile this cluster serves ----------------------------
   if (rank == 0 && tid == 0) s_ticket = atomicAdd(reinterpret_cast<unsigned long long*>(p.ws), 1ull);
   if (tid == 0) {
-    const StateHeader* hdr = reinterpret_cast<const StateHeader*>(p.state);
-    s_ok = (hdr->magic == kMagic && hdr->cfg_hash == p.cfg_hash && hdr->batch == p.B &&
-            hdr->n_layers == p.L);
+    const uint4 h0v = __ldcg(reinterpret_cast<const uint4*>(p.state));
+    const uint4 h1v = __ldcg(reinterpret_cast<const uint4*>(p.state + 16));
+    StateHeader hd;
+    reinterpret_cast<uint4*>(&hd)[0] = h0v;
+    reinterpret_cast<uint4*>(&hd)[1] = h1v;
+    s_ok = (hd.magic == kMagic) & (hd.cfg_hash == p.cfg_hash) & (hd.batch == p.B) &
+           (hd.n_layers == p.L);
   }
   cluster.sync();
   const long long ticket = static_cast<long long>(*cluster.map_shared_rank(&s_ticket, 0));
@@ -114,6 +224,10 @@ prefill_kernel(const PrefillParams p) {
     cluster.sync();  // rank 0's s_ticket must outlive the peers' reads
     return;
   }
+  // Tensor memory for the pool accumulators (at most two CTAs per SM, so the
+  // allocation never waits).
+  if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
+
   const long long tile = ticket / p.n_streams;
   const int stream = static_cast<int>(ticket % p.n_streams);
   const int l = stream / p.B;
@@ -123,8 +237,11 @@ prefill_kernel(const PrefillParams p) {
   const bool group_end = (tile % kGroup == kGroup - 1) && !last;
 
   unsigned char* blk = p.state + kHeaderBytes + static_cast<long long>(stream) * p.so.stride;
-  if (tid == 0) s_pos = *reinterpret_cast<const volatile long long*>(blk + p.so.pos);
+  if (tid == 0) s_pos = __ldcg(reinterpret_cast<const long long*>(blk + p.so.pos));
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
   const long long pos0 = s_pos;
   Tin* win_k = reinterpret_cast<Tin*>(blk + p.so.win_k);
   Tin* win_v = reinterpret_cast<Tin*>(blk + p.so.win_v);
@@ -158,11 +275,13 @@ prefill_kernel(const PrefillParams p) {
   float* incl_f = reinterpret_cast<float*>(p.ws + p.ws_incl_f);
   float* halo_ws = reinterpret_cast<float*>(p.ws + p.ws_halo);
 
+  // Slot of absolute position j >= 0 in the k-slot window.
+  auto wslot = [&](long long j) -> long long { return j % K; };
   // Key row of absolute position j >= 0 for KV head g: from the input if it
   // belongs to this call, else from window slot j mod k (the state holds
   // positions pos0-k .. pos0-1).
   auto key_row = [&](long long j, int g) -> const Tin* {
-    return (j >= pos0) ? kin + ((j - pos0) * nkv + g) * D : win_k + ((j % K) * nkv + g) * D;
+    return (j >= pos0) ? kin + ((j - pos0) * nkv + g) * D : win_k + (wslot(j) * nkv + g) * D;
   };
   auto evictions = [&](long long a, int len) -> int {  // positions p in [a, a+len) with p >= k
     const long long lo = a > K ? a : static_cast<long long>(K);
@@ -183,159 +302,145 @@ prefill_kernel(const PrefillParams p) {
     const int valid = rows > first_valid ? rows - static_cast<int>(first_valid) : 0;
     const unsigned row_bytes = static_cast<unsigned>(NG * D * ESZ);
     unsigned bytes = 2u * row_bytes * valid;
-    if (bi == 0) bytes += static_cast<unsigned>(Tt * HS * ESZ);
+    if (bi == 0) {
+      bytes += static_cast<unsigned>(Tt * HS * ESZ);
+      if (gstart == 0) bytes += static_cast<unsigned>(HS * 4);
+      if (tile == 0)
+        for (int r = 0; r < kHalo; ++r)
+          if (t0 - kHalo + r >= 0) bytes += static_cast<unsigned>(HS * 4);
+    }
     fence_proxy_async_smem();
     if (lane == 0) mbar_arrive_expect_tx(bar_kv, bytes);
     __syncwarp();
     for (int r = static_cast<int>(first_valid) + lane; r < rows; r += 32) {
       const long long j = bs + r;
-      const Tin* ks = (j >= pos0) ? kin + ((j - pos0) * nkv + g_lo) * D : win_k + ((j % K) * nkv + g_lo) * D;
-      const Tin* vs = (j >= pos0) ? vin + ((j - pos0) * nkv + g_lo) * D : win_v + ((j % K) * nkv + g_lo) * D;
+      const Tin* ks = (j >= pos0) ? kin + ((j - pos0) * nkv + g_lo) * D : win_k + (wslot(j) * nkv + g_lo) * D;
+      const Tin* vs = (j >= pos0) ? vin + ((j - pos0) * nkv + g_lo) * D : win_v + (wslot(j) * nkv + g_lo) * D;
       bulk_g2s(kb + r * rowB, ks, row_bytes, bar_kv);
       bulk_g2s(vb + r * rowB, vs, row_bytes, bar_kv);
     }
-    if (bi == 0)
+    if (bi == 0) {
       for (int r = lane; r < Tt; r += 32)
         bulk_g2s(qst + r * HS, qin + ((t0 - pos0 + r) * p.nq + h0) * D,
                  static_cast<unsigned>(HS * ESZ), bar_kv);
+      // carries from the state, read before this tile publishes anything
+      // (the stream's last tile overwrites them once all tiles have)
+      if (gstart == 0 && lane == 0) bulk_g2s(fcar, field + rank * HS, static_cast<unsigned>(HS * 4), bar_kv);
+      if (tile == 0 && lane < kHalo && t0 - kHalo + lane >= 0)
+        bulk_g2s(halo + lane * HS, ring + static_cast<size_t>((t0 - kHalo + lane) % kRing) * p.H + rank * HS,
+                 static_cast<unsigned>(HS * 4), bar_kv);
+    }
   };
   issue_block(0);
-
-  // ---- (A) far field: this tile's aggregate of the keys leaving the window
-  // (read straight from global memory, independent loads in flight).
-  for (int idx = tid; idx < NG * D; idx += NT) {
-    const int gg = idx / D, i = idx % D, g = g_lo + gg;
-    float a = 0.f;
-    for (int r0 = 0; r0 < Tt; r0 += kEvChunk) {
-      float ev[kEvChunk];
-#pragma unroll
-      for (int u = 0; u < kEvChunk; ++u) {
-        const long long pt = t0 + r0 + u;
-        ev[u] = (r0 + u < Tt && pt >= K) ? to_f32<Tin>(key_row(pt - K, g)[i]) : 0.f;
-      }
-#pragma unroll
-      for (int u = 0; u < kEvChunk; ++u)
-        if (r0 + u < Tt && t0 + r0 + u >= K) a = ewma(gf, a, ev[u]);
-    }
-    sagg[idx] = a;
-    if (g >= own_lo && publish) agg_s[(ticket * nkv + g) * D + i] = a;
-  }
-  // running state of the near field
+  if (tile == 0)  // ring rows before position 0 are zero
+    for (int idx = tid; idx < kHalo * HS; idx += NT)
+      if (t0 - kHalo + idx / HS < 0) halo[idx] = 0.f;
+  // running state of the near field (overlaps the copies in flight)
   for (int i = tid; i < kTile * HPC; i += NT) {
     mrun[i] = -INFINITY;
     lrun[i] = 0.f;
   }
   for (int i = tid; i < kTile * XS; i += NT) xs[i] = 0.f;
+  if (!mbar_wait_bounded(bar_kv, 0, kMbarPollLimit, p.err)) s_bad = 1;
+  // Keys that leave the window at the tile's tokens are rows 0 .. Tt-1 of the
+  // staged span when the first block covers them; otherwise read them from
+  // global memory.
+  bool ev_staged = p.KB >= Tt;
+  // Folds the keys that leave the window at tokens r_from .. Tt-1 into s
+  // (EWMA), calling visit(r, s) after every token; staged rows or global.
+  auto scan_evicted = [&](int gg, int i, int r_from, float s, auto&& visit) -> float {
+    if (ev_staged) {
+      const Tin* col = reinterpret_cast<const Tin*>(kb) + gg * D + i;
+      const int pitch = rowB / ESZ;
+      for (int r = 0; r < Tt; ++r) {
+        if (r >= r_from) s = ewma(gf, s, to_f32<Tin>(col[r * pitch]));
+        visit(r, s);
+      }
+    } else {
+      for (int r0 = 0; r0 < Tt; r0 += kEvChunk) {
+        float ev[kEvChunk];
+#pragma unroll
+        for (int u = 0; u < kEvChunk; ++u)
+          ev[u] = (r0 + u < Tt && r0 + u >= r_from) ? to_f32<Tin>(key_row(t0 + r0 + u - K, g_lo + gg)[i]) : 0.f;
+#pragma unroll
+        for (int u = 0; u < kEvChunk; ++u) {
+          const int r = r0 + u;
+          if (r < Tt) {
+            if (r >= r_from) s = ewma(gf, s, ev[u]);
+            visit(r, s);
+          }
+        }
+      }
+    }
+    return s;
+  };
+
+  // ---- (A) far field: this tile's aggregate of the keys leaving the window
+  // (read straight from global memory, independent loads in flight).
+  const int r_ev = static_cast<int>(max(0LL, min(static_cast<long long>(Tt), K - t0)));  // first token that evicts
+  for (int idx = tid; idx < NG * D; idx += NT) {
+    const int gg = idx / D, i = idx % D, g = g_lo + gg;
+    const float a = scan_evicted(gg, i, r_ev, 0.f, [](int, float) {});
+    sagg[idx] = a;
+    if (g >= own_lo && publish) agg_s[(ticket * nkv + g) * D + i] = a;
+  }
   __syncthreads();
   if (tid == 0 && publish) {
     __threadfence();
     for (int g = own_lo; g <= g_hi; ++g) st_release_u32(&fs_agg[ticket * nkv + g], 1u);
   }
 
-  // ---- (B) near field [P1 §2.1 eq. O_near]: per key block, each warp takes
-  // (token, head) pairs; lane a scores key cb+a in full, online softmax,
-  // then P·V with lanes over head dims into the x tile.
+  // ---- (B) near field [P1 §2.1 eq. O_near], block by block ---------------
   for (int bi = 0; bi < n_blocks; ++bi) {
-    if (!mbar_wait_bounded(bar_kv, bi & 1, kMbarPollLimit, p.err)) s_bad = 1;
+    if (bi > 0 && !mbar_wait_bounded(bar_kv, bi & 1, kMbarPollLimit, p.err)) s_bad = 1;
     const long long bs = kv_start + static_cast<long long>(bi) * p.KB;
     const long long be = bs + min(p.KB, kv_rows - bi * p.KB);  // exclusive
-    for (int pair = warp; pair < Tt * HPC; pair += NW) {
-      const int r = pair / HPC, hh = pair % HPC;
-      const int gg = (h0 + hh) / G - g_lo;
-      const long long pt = t0 + r;
-      const long long wlo = pt - K + 1 > 0 ? pt - K + 1 : 0;
-      const long long lo = wlo > bs ? wlo : bs;
-      const long long hi = pt < be - 1 ? pt : be - 1;
-      if (lo > hi) continue;
-      const Tin* qrow = qst + r * HS + hh * D;
-      float* orow = xs + r * XS + hh * D + lane * EPL;
-      float m = mrun[pair], den = lrun[pair];
-      float o[EPL];
-#pragma unroll
-      for (int e = 0; e < EPL; ++e) o[e] = orow[e];
-      for (long long cb = lo; cb <= hi; cb += 32) {
-        const int cnt = static_cast<int>(min(32LL, hi - cb + 1));
-        float s = -INFINITY;
-        if (lane < cnt) {
-          const Tin* kr = reinterpret_cast<const Tin*>(kb + (cb + lane - bs) * rowB) + gg * D;
-          constexpr int VE = Load16<Tin>::N;
-          float acc = 0.f;
-#pragma unroll
-          for (int i = 0; i < D; i += VE) {
-            float kv[VE], qv[VE];
-            Load16<Tin>::run(kr + i, kv);
-            Load16<Tin>::run(qrow + i, qv);
-#pragma unroll
-            for (int e = 0; e < VE; ++e) acc = fmaf(qv[e], kv[e], acc);
-          }
-          s = acc * p.score_scale;
-        }
-        const float mn = fmaxf(m, warp_max(s));
-        const float corr = expf(m - mn);
-        const float pj = (lane < cnt) ? expf(s - mn) : 0.f;
-        den = fmaf(den, corr, warp_sum(pj));
-#pragma unroll
-        for (int e = 0; e < EPL; ++e) o[e] *= corr;
-        for (int c = 0; c < cnt; ++c) {
-          const float pc = __shfl_sync(0xffffffffu, pj, c);
-          const Tin* vr = reinterpret_cast<const Tin*>(vb + (cb + c - bs) * rowB) + gg * D + lane * EPL;
-          float vv[EPL];
-          VecLoad<Tin, EPL>::run(vr, vv);
-#pragma unroll
-          for (int e = 0; e < EPL; ++e) o[e] = fmaf(pc, vv[e], o[e]);
-        }
-        m = mn;
-      }
-#pragma unroll
-      for (int e = 0; e < EPL; ++e) orow[e] = o[e];
-      if (lane == 0) {
-        mrun[pair] = m;
-        lrun[pair] = den;
-      }
-    }
+    if (K <= 16)
+      near_block<Tin, D, 16>(qst, kb, vb, xs, mrun, lrun, rowB, HS, XS, HPC, G, g_lo, K, t0, Tt,
+                             bs, be, p.score_scale, h0, warp, lane);
+    else
+      near_block<Tin, D, 32>(qst, kb, vb, xs, mrun, lrun, rowB, HS, XS, HPC, G, g_lo, K, t0, Tt,
+                             bs, be, p.score_scale, h0, warp, lane);
     __syncthreads();  // the block buffers are free again
     if (bi + 1 < n_blocks) issue_block(bi + 1);
   }
+  if (n_blocks > 1) ev_staged = false;  // the staged rows were replaced by later blocks
   // normalise: O = acc / den
-  for (int idx = tid; idx < Tt * HS; idx += NT) {
-    const int r = idx / HS, c = idx % HS;
-    xs[r * XS + c] /= lrun[r * HPC + c / D];
-  }
+  for (int i = tid; i < Tt * HPC; i += NT) lrun[i] = 1.f / lrun[i];
+  __syncthreads();
+  for (int r = warp; r < Tt; r += NW)
+    for (int c = lane; c < HS; c += 32) xs[r * XS + c] *= lrun[r * HPC + c / D];
 
-  // Slot slice for both pool contractions; the staging buffers are free.
-  const float* slot_base = p.slots + static_cast<size_t>(l) * kSlots * p.H + static_cast<size_t>(rank) * HS;
-  if (warp == 0) {
-    fence_proxy_async_smem();
-    if (lane == 0) mbar_arrive_expect_tx(bar_sl, kSlots * HS * 4u);
-    __syncwarp();
-    for (int j = lane; j < kSlots; j += 32)
-      bulk_g2s(sl + j * XS, slot_base + static_cast<size_t>(j) * p.H, HS * 4u, bar_sl);
-  }
 
   // ---- (C) far field carry-in (deterministic look-back), then the scan --
   // carry = INCL(end of previous group) or the state, folded with the
-  // aggregates of the group's earlier tiles in order.
+  // aggregates of the group's earlier tiles in order.  Warp 0 polls all the
+  // flags at once (lane per flag); then every carry element loads all its
+  // terms at once and folds them in order.
+  const int n_prev = static_cast<int>(tile - gstart);  // earlier tiles of the group (< kGroup)
   {
-    const bool from_state = (gstart == 0);
-    if (!from_state) {
-      if (tid == 0)
-        for (int g = g_lo; g <= g_hi; ++g) wait_flag(&fs_incl[ticket_of(gstart - 1) * nkv + g], p.spin_limit, p.err);
-      __syncthreads();
+    if (warp == 0) {
+      const int n_flags = (n_prev + (gstart > 0 ? 1 : 0)) * NG;
+      for (int f = lane; f < n_flags; f += 32) {
+        const int gg = f % NG, jj = f / NG;
+        const unsigned* fl = (jj < n_prev) ? &fs_agg[ticket_of(gstart + jj) * nkv + g_lo + gg]
+                                           : &fs_incl[ticket_of(gstart - 1) * nkv + g_lo + gg];
+        wait_flag(fl, p.spin_limit, p.err);
+      }
     }
+    __syncthreads();
     for (int idx = tid; idx < NG * D; idx += NT) {
       const int g = g_lo + idx / D, i = idx % D;
-      sst[idx] = from_state ? far[g * D + i] : __ldcg(incl_s + (ticket_of(gstart - 1) * nkv + g) * D + i);
-    }
-    for (long long j = gstart; j < tile; ++j) {
-      __syncthreads();
-      if (tid == 0)
-        for (int g = g_lo; g <= g_hi; ++g) wait_flag(&fs_agg[ticket_of(j) * nkv + g], p.spin_limit, p.err);
-      __syncthreads();
-      const float mul = powf(gf, static_cast<float>(evictions(pos0 + j * kTile, kTile)));
-      for (int idx = tid; idx < NG * D; idx += NT) {
-        const int g = g_lo + idx / D, i = idx % D;
-        sst[idx] = fmaf(mul, sst[idx], __ldcg(agg_s + (ticket_of(j) * nkv + g) * D + i));
-      }
+      float terms[kGroup];
+#pragma unroll
+      for (int jj = 0; jj < kGroup - 1; ++jj)
+        terms[jj] = (jj < n_prev) ? __ldcg(agg_s + (ticket_of(gstart + jj) * nkv + g) * D + i) : 0.f;
+      float acc = (gstart == 0) ? far[g * D + i] : __ldcg(incl_s + (ticket_of(gstart - 1) * nkv + g) * D + i);
+#pragma unroll
+      for (int jj = 0; jj < kGroup - 1; ++jj)
+        if (jj < n_prev)
+          acc = fmaf(powf(gf, static_cast<float>(evictions(pos0 + (gstart + jj) * kTile, kTile))), acc, terms[jj]);
+      sst[idx] = acc;
     }
     __syncthreads();
     if (group_end && publish) {
@@ -355,42 +460,31 @@ prefill_kernel(const PrefillParams p) {
   for (int idx = tid; idx < NG * D; idx += NT) {
     const int gg = idx / D, i = idx % D, g = g_lo + gg;
     const int hh_lo = max(0, g * G - h0), hh_hi = min(HPC, (g + 1) * G - h0);
-    float s = sst[idx];
-    for (int r0 = 0; r0 < Tt; r0 += kEvChunk) {
-      float ev[kEvChunk];
-#pragma unroll
-      for (int u = 0; u < kEvChunk; ++u) {
-        const long long pt = t0 + r0 + u;
-        ev[u] = (r0 + u < Tt && pt >= K) ? to_f32<Tin>(key_row(pt - K, g)[i]) : 0.f;
+    (void)g;
+    const float s = scan_evicted(gg, i, r_ev, sst[idx], [&](int r, float sv) {
+      for (int hh = hh_lo; hh < hh_hi; ++hh) {
+        float* xp = xs + r * XS + hh * D + i;
+        *xp = fmaf(p.alpha_far, sv, *xp);
       }
-#pragma unroll
-      for (int u = 0; u < kEvChunk; ++u) {
-        const int r = r0 + u;
-        if (r < Tt) {
-          if (t0 + r >= K) s = ewma(gf, s, ev[u]);
-          for (int hh = hh_lo; hh < hh_hi; ++hh) {
-            float* xp = xs + r * XS + hh * D + i;
-            *xp = fmaf(p.alpha_far, s, *xp);
-          }
-        }
-      }
-    }
+    });
     sst[idx] = s;  // S at the end of the tile
   }
   __syncthreads();
+  // Slot blocks (bf16 hi/lo, laid out for both pool MMAs); the staging
+  // buffers are free now.
+  const unsigned char* img = p.slot_img +
+      (static_cast<size_t>(l) * (p.H / kBlk) + static_cast<size_t>(rank) * nch) * 2 * kBlkBytes;
+  if (tid == 0) {
+    fence_proxy_async_smem();
+    mbar_arrive_expect_tx(bar_sl, static_cast<unsigned>(nch * 2 * kBlkBytes));
+    for (int c = 0; c < nch; ++c)
+      bulk_g2s(simg + c * 2 * kBlkBytes, img + static_cast<size_t>(c) * 2 * kBlkBytes,
+               2u * kBlkBytes, bar_sl);
+  }
 
   // ---- (D) EMA field aggregate; tail rows for the successor -------------
-  // Tiles of the first group read the state field (and tile 0 the state
-  // ring rows) now, before any flag is published: the stream's last tile
-  // overwrites them once every earlier tile has published.
-  if (gstart == 0)
-    for (int e = tid; e < HS; e += NT) fcar[e] = field[rank * HS + e];
-  if (tile == 0)
-    for (int idx = tid; idx < kHalo * HS; idx += NT) {
-      const int r = idx / HS, e = idx % HS;
-      const long long q = t0 - kHalo + r;
-      halo[idx] = (q >= 0) ? ring[static_cast<size_t>(q % kRing) * p.H + rank * HS + e] : 0.f;
-    }
+  // (Tiles of the first group staged the state field, and tile 0 the state
+  // ring rows, with the first key block.)
   for (int e = tid; e < HS; e += NT) {
     float a = 0.f;
     for (int r = 0; r < Tt; ++r) a = ewma(ge, a, xs[r * XS + e]);
@@ -407,65 +501,88 @@ prefill_kernel(const PrefillParams p) {
     st_release_u32(&ff_agg[ticket * p.CS + rank], 1u);
   }
 
-  // ---- (E) pool partial sums over this slice [P3 §2.1 channel 3] ---------
-  // scores[T x 64] = x[T x HS] · slot^T, register-blocked 4 tokens x 4 slots.
-  if (!mbar_wait_bounded(bar_sl, 0, kMbarPollLimit, p.err)) s_bad = 1;
-  {
-    const int ty = tid / 16, tx = tid % 16;
-    float acc[4][4];
+  // ---- (E) pool scores on the tensor cores [P3 §2.1 channel 3] -----------
+  // scores[T x 64] (tensor memory, columns 0..63) = sum over 64-column chunks
+  // of x_chunk . slot_chunk^T, each as hi*hi + hi*lo + lo*hi.
+  const uint32_t idesc_s = umma_idesc_bf16(kBlk, kSlots, false);
+  const uint32_t idesc_c = umma_idesc_bf16(kBlk, kCW, true);
+  for (int c = 0; c < nch; ++c) {
+    const int buf = c & 1;
+    unsigned char* xhi = xw + buf * 2 * kBlkBytes;
+    unsigned char* xlo = xhi + kBlkBytes;
+    if (c >= 2)  // the MMAs of chunk c-2 have finished reading this x buffer
+      if (!mbar_wait_bounded(bar_ms + buf, ((c - 2) >> 1) & 1, kMbarPollLimit, p.err)) s_bad = 1;
+    stage_split_block(xs + c * kBlk, XS, xhi, xlo, tid, NT);
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+      if (c == 0 && !mbar_wait_bounded(bar_sl, 0, kMbarPollLimit, p.err)) s_bad = 1;
+      tc_fence_after();
+      const unsigned char* shi = simg + c * 2 * kBlkBytes;
+      const unsigned char* slo = shi + kBlkBytes;
 #pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) acc[a][c] = 0.f;
-    for (int e = 0; e < HS; e += 4) {
-      float4 xa[4], sb[4];
-#pragma unroll
-      for (int a = 0; a < 4; ++a) xa[a] = *reinterpret_cast<const float4*>(xs + (ty * 4 + a) * XS + e);
-#pragma unroll
-      for (int c = 0; c < 4; ++c) sb[c] = *reinterpret_cast<const float4*>(sl + (tx + 16 * c) * XS + e);
-#pragma unroll
-      for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          acc[a][c] = fmaf(xa[a].x, sb[c].x, fmaf(xa[a].y, sb[c].y,
-                      fmaf(xa[a].z, sb[c].z, fmaf(xa[a].w, sb[c].w, acc[a][c]))));
-    }
-#pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) part[(ty * 4 + a) * kPartStride + tx + 16 * c] = acc[a][c];
-    for (int r = warp; r < kTile; r += NW) {
-      float ss = 0.f;
-      for (int e = lane; e < HS; e += 32) ss = fmaf(xs[r * XS + e], xs[r * XS + e], ss);
-      ss = warp_sum(ss);
-      if (lane == 0) part[r * kPartStride + kSlots] = ss;
+      for (int s = 0; s < kBlk / 16; ++s) {
+        const uint64_t ah = umma_desc(xhi + s * 2048, 1024, 128), al = umma_desc(xlo + s * 2048, 1024, 128);
+        const uint64_t bh = umma_desc(shi + s * 2048, 1024, 128), bl = umma_desc(slo + s * 2048, 1024, 128);
+        umma_bf16(tmem, ah, bh, idesc_s, c > 0 || s > 0);
+        umma_bf16(tmem, ah, bl, idesc_s, true);
+        umma_bf16(tmem, al, bh, idesc_s, true);
+      }
+      umma_commit(bar_ms + buf);
     }
   }
+  if (tid == 0) umma_commit(bar_sd);
+  // |x|^2 per token (CUDA cores) while the tensor cores finish
+  for (int r = warp; r < kTile; r += NW) {
+    float ss = 0.f;
+    for (int e = lane; e < HS; e += 32) ss = fmaf(xs[r * XS + e], xs[r * XS + e], ss);
+    ss = warp_sum(ss);
+    if (lane == 0) part[r * kPartStride + kSlots] = ss;
+  }
+  if (!mbar_wait_bounded(bar_sd, 0, kMbarPollLimit, p.err)) s_bad = 1;
+  tc_fence_after();
+  {  // accumulator row r (token) sits in lane (r%16) + 32*(r/16) for M = 64
+    const int sp = warp & 3, colh = (warp >> 2) * 32;
+    float v[32];
+    tmem_ld32(tmem + (static_cast<uint32_t>(32 * sp) << 16) + colh, v);
+    if (lane < 16) {
+      const int r = 16 * sp + lane;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) part[r * kPartStride + colh + j] = v[j];
+    }
+  }
+  tc_fence_before();
 
   // ---- (F) EMA field carry-in (deterministic look-back); tail rows ------
   {
-    if (gstart > 0) {
-      if (tid == 0) wait_flag(&ff_incl[ticket_of(gstart - 1) * p.CS + rank], p.spin_limit, p.err);
-      __syncthreads();
-      for (int e = tid; e < HS; e += NT)
-        fcar[e] = __ldcg(incl_f + ticket_of(gstart - 1) * p.H + rank * HS + e);
+    if (warp == 0) {
+      const int n_flags = n_prev + (gstart > 0 ? 1 : 0);
+      for (int f = lane; f < n_flags; f += 32) {
+        const unsigned* fl = (f < n_prev) ? &ff_agg[ticket_of(gstart + f) * p.CS + rank]
+                                          : &ff_incl[ticket_of(gstart - 1) * p.CS + rank];
+        wait_flag(fl, p.spin_limit, p.err);
+      }
+      // the predecessor's tail rows come with its aggregate (or, across a
+      // group boundary, with the inclusive value published after it)
     }
+    __syncthreads();
     const float mul_full = powf(ge, static_cast<float>(kTile));
-    for (long long j = gstart; j < tile; ++j) {
-      __syncthreads();
-      if (tid == 0) wait_flag(&ff_agg[ticket_of(j) * p.CS + rank], p.spin_limit, p.err);
-      __syncthreads();
-      for (int e = tid; e < HS; e += NT)
-        fcar[e] = fmaf(mul_full, fcar[e], __ldcg(agg_f + ticket_of(j) * p.H + rank * HS + e));
+    for (int e = tid; e < HS; e += NT) {
+      float terms[kGroup];
+#pragma unroll
+      for (int jj = 0; jj < kGroup - 1; ++jj)
+        terms[jj] = (jj < n_prev) ? __ldcg(agg_f + ticket_of(gstart + jj) * p.H + rank * HS + e) : 0.f;
+      float acc = (gstart == 0) ? fcar[e] : __ldcg(incl_f + ticket_of(gstart - 1) * p.H + rank * HS + e);
+#pragma unroll
+      for (int jj = 0; jj < kGroup - 1; ++jj)
+        if (jj < n_prev) acc = fmaf(mul_full, acc, terms[jj]);
+      fcar[e] = acc;
     }
-    if (tile > 0) {  // x rows of the 15 tokens before the tile, from the predecessor
-      if (tid == 0) wait_flag(&ff_agg[ticket_of(tile - 1) * p.CS + rank], p.spin_limit, p.err);
-      __syncthreads();
+    if (tile > 0)  // x rows of the 15 tokens before the tile, from the predecessor
       for (int idx = tid; idx < kHalo * HS; idx += NT) {
         const int r = idx / HS, e = idx % HS;
         halo[idx] = __ldcg(halo_ws + (ticket_of(tile - 1) * kHalo + r) * p.H + rank * HS + e);
       }
-    }
     __syncthreads();
     if (group_end && publish) {
       const float mul = powf(ge, static_cast<float>(Tt));
@@ -509,50 +626,70 @@ prefill_kernel(const PrefillParams p) {
   }
   cluster.sync();
 
-  // ---- (H) per column chunk: semantic mix (GEMM), then ring, field,
-  // fusion, clip, output [P3 §2.1 channels 1–3, §2.2].
+  // ---- (H) semantic mix on the tensor cores, then per column chunk: ring,
+  // field, fusion, clip, output [P3 §2.1 channels 1–3, §2.2].
+  // sem chunk c [T x 64] = w[T x 64] . slot_chunk_c, accumulators alternate
+  // between tensor-memory columns 64..127 and 128..191.
+  unsigned char* whi = xw;  // the x blocks are dead: all score MMAs finished
+  unsigned char* wlo = xw + kBlkBytes;
+  stage_split_block(wts, kSlots, whi, wlo, tid, NT);
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  auto issue_sem = [&](int c) {  // tid 0 only
+    tc_fence_after();
+    const uint32_t dst = tmem + kSlots + (c & 1) * kCW;
+    const unsigned char* shi = simg + c * 2 * kBlkBytes;
+    const unsigned char* slo = shi + kBlkBytes;
+#pragma unroll
+    for (int s = 0; s < kSlots / 16; ++s) {
+      const uint64_t ah = umma_desc(whi + s * 2048, 1024, 128), al = umma_desc(wlo + s * 2048, 1024, 128);
+      const uint64_t bh = umma_desc(shi + s * 256, 128, 1024), bl = umma_desc(slo + s * 256, 128, 1024);
+      umma_bf16(dst, ah, bh, idesc_c, s > 0);
+      umma_bf16(dst, ah, bl, idesc_c, true);
+      umma_bf16(dst, al, bh, idesc_c, true);
+    }
+    umma_commit(bar_mc + (c & 1));
+  };
+  if (tid == 0) {
+    issue_sem(0);
+    if (nch > 1) issue_sem(1);
+  }
   const float a_l = p.alpha_layer[l];
   const bool write_ok = !s_bad;
   float* out = p.out + (in_row0 + (t0 - pos0)) * p.H + rank * HS;
-  for (int c0 = 0; c0 < HS; c0 += kCW) {
-    {  // semc[T x 64] = wts[T x 64] · slot[64 x cols c0..c0+63]
-      const int ty = tid / 16, tx = tid % 16;
-      float acc[4][4];
+  for (int c = 0; c < nch; ++c) {
+    const int buf = c & 1;
+    if (!mbar_wait_bounded(bar_mc + buf, (c >> 1) & 1, kMbarPollLimit, p.err)) s_bad = 1;
+    tc_fence_after();
+    {
+      const int sp = warp & 3, colh = (warp >> 2) * 32;
+      float v[32];
+      tmem_ld32(tmem + (static_cast<uint32_t>(32 * sp) << 16) + kSlots + buf * kCW + colh, v);
+      if (lane < 16) {
+        float* dst = semc + (16 * sp + lane) * kSemStride + colh;
 #pragma unroll
-      for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) acc[a][c] = 0.f;
-#pragma unroll 4
-      for (int j = 0; j < kSlots; ++j) {
-        const float4 s4 = *reinterpret_cast<const float4*>(sl + j * XS + c0 + tx * 4);
-#pragma unroll
-        for (int a = 0; a < 4; ++a) {
-          const float w = wts[(ty * 4 + a) * kSlots + j];
-          acc[a][0] = fmaf(w, s4.x, acc[a][0]);
-          acc[a][1] = fmaf(w, s4.y, acc[a][1]);
-          acc[a][2] = fmaf(w, s4.z, acc[a][2]);
-          acc[a][3] = fmaf(w, s4.w, acc[a][3]);
-        }
+        for (int j = 0; j < 32; j += 4)
+          *reinterpret_cast<float4*>(dst + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
       }
-#pragma unroll
-      for (int a = 0; a < 4; ++a)
-        *reinterpret_cast<float4*>(semc + (ty * 4 + a) * kCW + tx * 4) =
-            make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
     }
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0 && c + 2 < nch) issue_sem(c + 2);  // overlaps the epilogue below
     // field: per-segment aggregates, then carries folded in segment order
-    const int c = tid % kCW, sg = tid / kCW;  // column, token segment
-    const int e = c0 + c;
+    const int cc = tid % kCW, sg = tid / kCW;  // column, token segment
+    const int e = c * kCW + cc;
     const int r_lo = sg * (kTile / kSeg), r_hi = min(Tt, r_lo + kTile / kSeg);
     {
       float a = 0.f;
       for (int r = r_lo; r < r_hi; ++r) a = ewma(ge, a, xs[r * XS + e]);
-      segc[sg * kCW + c] = a;
+      segc[sg * kCW + cc] = a;
     }
     __syncthreads();
     float f = fcar[e];
     for (int s2 = 0; s2 < sg; ++s2) {
       const int len = max(0, min(Tt, (s2 + 1) * (kTile / kSeg)) - s2 * (kTile / kSeg));
-      f = fmaf(powf(ge, static_cast<float>(len)), f, segc[s2 * kCW + c]);
+      f = fmaf(powf(ge, static_cast<float>(len)), f, segc[s2 * kCW + cc]);
     }
     // ring: sum of the 16 positions ending at r, from the x tile and the halo
     auto xat = [&](int r) -> float { return r >= 0 ? xs[r * XS + e] : halo[(r + kHalo) * HS + e]; };
@@ -563,7 +700,7 @@ prefill_kernel(const PrefillParams p) {
       if (r > r_lo) rs += xat(r) - xat(r - kRing);
       const float x = xs[r * XS + e];
       f = ewma(ge, f, x);
-      float u = rs * (1.0f / kRing) + 0.5f * f + 0.5f * semc[r * kCW + c];
+      float u = rs * (1.0f / kRing) + 0.5f * f + 0.5f * semc[r * kSemStride + cc];
       u = fminf(fmaxf(u, -p.clip_eps), p.clip_eps);
       if (write_ok) out[static_cast<long long>(r) * p.H + e] = fmaf(a_l, u, x);
     }
@@ -603,12 +740,20 @@ prefill_kernel(const PrefillParams p) {
         const int g = own_lo + static_cast<int>((idx / D) % n_own);
         const int i = static_cast<int>(idx % D);
         const long long src = ((j - pos0) * nkv + g) * D + i;
-        const long long dst = ((j % K) * nkv + g) * D + i;
+        const long long dst = (wslot(j) * nkv + g) * D + i;
         win_k[dst] = kin[src];
         win_v[dst] = vin[src];
       }
     }
     if (rank == 0 && tid == 0) *reinterpret_cast<long long*>(blk + p.so.pos) = pos0 + p.n;
+  }
+
+  // every tensor-core operation has completed (last sem commit waited)
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
   }
 }
 
@@ -643,48 +788,6 @@ cudaError_t launch_t(const PrefillParams& p, cudaStream_t s) {
   return cudaLaunchKernelEx(&cfg, prefill_kernel<Tin, D>, p);
 }
 
-}  // namespace
-
-// Shared-memory plan: persistent regions, then a union of the staging
-// buffers (near-field phase) and the pool buffers (pool phase).  The key
-// block is as tall as fits, up to the whole span t0-k .. t0+T-1.
-bool plan_prefill(int HPC, int D, int esz, int NGm, int K, size_t budget, PrefillPlan* out) {
-  const int HS = HPC * D, XS = HS + 4;
-  auto a16 = [](long long x) { return static_cast<int>((x + 15) & ~15LL); };
-  PrefillPlan p;
-  int off = 0;
-  p.bars = off;                 off += 16;
-  p.xs = off;                   off += a16(4LL * kTile * XS);
-  p.halo = off;                 off += a16(4LL * kHalo * HS);
-  p.fcar = off;                 off += a16(4LL * HS);
-  p.sst = off;                  off += a16(4LL * NGm * D);
-  p.sagg = off;                 off += a16(4LL * NGm * D);
-  p.ml = off;                   off += a16(4LL * (2 * kTile * HPC + kSeg * kCW));
-  p.u0 = off;
-  // pool phase
-  int q = off;
-  p.sl = q;                     q += a16(4LL * kSlots * XS);
-  p.part = q;                   q += a16(4LL * kTile * kPartStride);
-  p.wts = q;                    q += a16(4LL * kTile * kSlots);
-  p.semc = q;                   q += a16(4LL * kTile * kCW);
-  const int pool_end = q;
-  // staging phase
-  q = off;
-  p.qst = q;                    q += a16(static_cast<long long>(kTile) * HS * esz);
-  const int row_b = NGm * D * esz + 16;
-  const long long room = static_cast<long long>(budget) - q;
-  int kb_rows = static_cast<int>(room / (2LL * row_b));
-  kb_rows = std::min(kb_rows, kTile + K);
-  if (kb_rows < 32) return false;
-  p.KB = kb_rows;
-  p.kb = q;                     q += a16(static_cast<long long>(row_b) * kb_rows);
-  p.vb = q;                     q += a16(static_cast<long long>(row_b) * kb_rows);
-  p.total = std::max(q, pool_end);
-  if (static_cast<size_t>(p.total) > budget) return false;
-  *out = p;
-  return true;
-}
-
 template <typename Tin, int D>
 int max_clusters_t(int cs, size_t smem) {
   cudaLaunchConfig_t cfg = {};
@@ -704,6 +807,53 @@ int max_clusters_t(int cs, size_t smem) {
     return 0;
   }
   return n;
+}
+
+}  // namespace
+
+// Shared-memory plan: persistent regions, then a union of the staging
+// buffers (near-field phase) and the pool buffers (pool phase).  The key
+// block is as tall as fits, up to the whole span t0-k .. t0+T-1.  The plan
+// never drops below a third of the SM's shared memory, so at most two CTAs
+// share an SM and their tensor-memory allocations (256 columns each) always
+// fit at once.
+bool plan_prefill(int HPC, int D, int esz, int NGm, int K, size_t budget, PrefillPlan* out) {
+  const int HS = HPC * D, XS = HS + 4;
+  if (HS % kBlk != 0) return false;
+  auto a16 = [](long long x) { return static_cast<int>((x + 15) & ~15LL); };
+  PrefillPlan p;
+  int off = 0;
+  p.bars = off;                 off += 128;  // mbarriers and the tensor-memory address
+  p.xs = off;                   off += a16(4LL * kTile * XS);
+  p.halo = off;                 off += a16(4LL * kHalo * HS);
+  p.fcar = off;                 off += a16(4LL * HS);
+  p.sst = off;                  off += a16(4LL * NGm * D);
+  p.sagg = off;                 off += a16(4LL * NGm * D);
+  p.ml = off;                   off += a16(4LL * (2 * kTile * HPC + kSeg * kCW));
+  p.u0 = off;
+  // pool phase: slot blocks, partials, weights, x blocks | w blocks + sem chunk
+  int q = off;
+  p.sl = q;                     q += a16(static_cast<long long>(HS / kBlk) * 2 * kBlkBytes);
+  p.part = q;                   q += a16(4LL * kTile * kPartStride);
+  p.wts = q;                    q += a16(4LL * kTile * kSlots);
+  p.semc = q;                   q += a16(std::max(4LL * kBlkBytes, 2LL * kBlkBytes + 4LL * kTile * kSemStride));
+  const int pool_end = q;
+  // staging phase
+  q = off;
+  p.qst = q;                    q += a16(static_cast<long long>(kTile) * HS * esz);
+  const int row_b = NGm * D * esz + 16;
+  const long long room = static_cast<long long>(budget) - q;
+  int kb_rows = static_cast<int>(room / (2LL * row_b));
+  kb_rows = std::min(kb_rows, kTile + K);
+  if (kb_rows < 32) return false;
+  p.KB = kb_rows;
+  p.kb = q;                     q += a16(static_cast<long long>(row_b) * kb_rows);
+  p.vb = q;                     q += a16(static_cast<long long>(row_b) * kb_rows);
+  p.total = std::max(q, pool_end);
+  p.total = std::max<int>(p.total, static_cast<int>((budget + 1024) / 3) + 1);
+  if (static_cast<size_t>(p.total) > budget) return false;
+  *out = p;
+  return true;
 }
 
 int prefill_max_active_clusters(int cs, size_t smem, int in_dtype, int head_dim) {

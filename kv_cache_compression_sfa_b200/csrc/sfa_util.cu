@@ -2,6 +2,7 @@
 #include <cuda_runtime.h>
 
 #include "sfa_common.cuh"
+#include "sfa_umma.cuh"
 
 namespace sfa {
 namespace {
@@ -23,6 +24,26 @@ __global__ void slot_norm_kernel(const float* slots, float* norms, int H) {
   if (threadIdx.x == 0) norms[row] = fmaxf(static_cast<float>(sqrt(red[0])), kNormFloor);
 }
 
+// Pre-split slot blocks for the prefill pool MMAs: for layer l and 64-column
+// chunk c of hidden, a [64 slots x 64 columns] bf16 hi block followed by the
+// lo block (slot = hi + lo to about 16 significant bits), both in the
+// core-matrix layout of sfa_umma.cuh.  One thread per element.
+__global__ void slot_image_kernel(const float* slots, unsigned char* img, int L, int H) {
+  const long long n = static_cast<long long>(L) * kSlots * H;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int l = static_cast<int>(i / (static_cast<long long>(kSlots) * H));
+    const int rem = static_cast<int>(i % (static_cast<long long>(kSlots) * H));
+    const int j = rem / H, h = rem % H;
+    const int c = h / kBlk, col = h % kBlk;
+    unsigned char* blk = img + (static_cast<size_t>(l) * (H / kBlk) + c) * 2 * kBlkBytes;
+    __nv_bfloat16 hi, lo;
+    split_bf16(slots[i], hi, lo);
+    *reinterpret_cast<__nv_bfloat16*>(blk + blk_off(j, col)) = hi;
+    *reinterpret_cast<__nv_bfloat16*>(blk + kBlkBytes + blk_off(j, col)) = lo;
+  }
+}
+
 __global__ void write_header_kernel(unsigned char* state, StateHeader h) {
   if (threadIdx.x == 0 && blockIdx.x == 0) *reinterpret_cast<StateHeader*>(state) = h;
 }
@@ -31,6 +52,11 @@ __global__ void write_header_kernel(unsigned char* state, StateHeader h) {
 
 cudaError_t launch_slot_norms(const float* slots, float* norms, int L, int H, cudaStream_t s) {
   slot_norm_kernel<<<L * kSlots, 256, 0, s>>>(slots, norms, H);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_slot_image(const float* slots, unsigned char* img, int L, int H, cudaStream_t s) {
+  slot_image_kernel<<<592, 256, 0, s>>>(slots, img, L, H);
   return cudaGetLastError();
 }
 
