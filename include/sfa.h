@@ -173,6 +173,28 @@ SFA_API const char* sfa_status_string(int status);
 /* ABI version of the loaded library (SFA_ABI_VERSION it was built with). */
 SFA_API int sfa_abi_version(void);
 
+/* Bytes of the fixed device scratch behind sfa_prefill_static_ws. */
+#define SFA_STATIC_WORKSPACE_BYTES (16u << 20)
+
+/* sfa_prefill without a caller-provided workspace, for callers that cannot
+ * allocate: an operator hook inside another engine that receives only its
+ * input/output tensors and no allocator, or a serving loop that forbids
+ * cudaMalloc in steady state because it can synchronise the device.  (The
+ * pages have no counterpart: this is a deployment variant of sfa_prefill.)
+ * The cross-tile scratch is one file-scope device array of
+ * SFA_STATIC_WORKSPACE_BYTES that every GPU loading the library holds until
+ * the process exits; nothing is allocated or freed.  The first call on a
+ * device looks up the array's device address (with that device current)
+ * and caches it, so make that first call before any stream capture.  Every
+ * call on a device shares the array: the parts that must start at zero are
+ * cleared on `stream` by each call, and calls that overlap on the GPU (other
+ * streams, other host threads) race on it.  Returns SFA_ERR_WORKSPACE when
+ * sfa_prefill_workspace_bytes(h, batch, n) exceeds the array (split the
+ * prefill into smaller chunks), otherwise exactly what sfa_prefill returns;
+ * results equal sfa_prefill's. */
+SFA_API int sfa_prefill_static_ws(const sfa_handle* h, const void* q, const void* k, const void* v,
+                                  long long n, int batch, void* state, float* out, void* stream);
+
 /* Test hook for the device-side bounded waits of sfa_prefill (not needed in
  * normal use).  spin_limit: maximum polls of a look-back flag before the
  * wait gives up and latches SFA_ERR_DEVICE_TIMEOUT (0 restores the default).

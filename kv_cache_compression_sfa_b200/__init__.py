@@ -43,7 +43,7 @@ EXPORTED = (
     "sfa_config_default", "sfa_config_validate", "sfa_state_layout_for", "sfa_init",
     "sfa_destroy", "sfa_state_bytes", "sfa_prefill_workspace_bytes", "sfa_state_reset",
     "sfa_prefill", "sfa_decode_step", "sfa_check_device_status", "sfa_status_string",
-    "sfa_abi_version", "sfa_debug_set_lookback",
+    "sfa_abi_version", "sfa_debug_set_lookback", "sfa_prefill_static_ws",
 )
 
 
@@ -104,6 +104,7 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
             "sfa_status_string": (ctypes.c_char_p, [i]),
             "sfa_abi_version": (i, []),
             "sfa_debug_set_lookback": (i, [vp, ctypes.c_uint, ll]),
+            "sfa_prefill_static_ws": (i, [vp, vp, vp, vp, ll, i, vp, vp, vp]),
         }
         for name, (res, args) in sigs.items():
             fn = getattr(lib, name)
@@ -273,6 +274,24 @@ def sfa_prefill(h: Handle, q, k, v, n: int, batch: int, state: torch.Tensor, out
                                     workspace.numel(), _stream_ptr(stream))
     if rc != SFA_OK:
         raise SfaError(rc, "sfa_prefill")
+
+
+SFA_STATIC_WORKSPACE_BYTES = 16 << 20
+
+
+def sfa_prefill_static_ws(h: Handle, q, k, v, n: int, batch: int, state: torch.Tensor,
+                          out: torch.Tensor, stream=None) -> None:
+    """sfa_prefill on the library's fixed device scratch (no workspace
+    argument, nothing allocated); see include/sfa.h for the limits."""
+    if n == 0:
+        return
+    qp, kp, vp = _qkv_checks(h, q, k, v, n, batch)
+    sp = _dev(state, "state", torch.uint8, sfa_state_bytes(h, batch))
+    op = _dev(out, "out", torch.float32, h.cfg.n_layers * batch * n * h.cfg.hidden)
+    rc = load_library().sfa_prefill_static_ws(h.ptr, qp, kp, vp, n, batch, sp, op,
+                                              _stream_ptr(stream))
+    if rc != SFA_OK:
+        raise SfaError(rc, "sfa_prefill_static_ws")
 
 
 def sfa_decode_step(h: Handle, q, k, v, batch: int, state: torch.Tensor, out: torch.Tensor,

@@ -1,0 +1,70 @@
+// sfa_static_ws.cu — sfa_prefill_static_ws: a prefill entry point that
+// allocates nothing.
+//
+// Some callers cannot hand the operator a workspace.  A custom-op hook inside
+// another inference engine may receive only the operator's input and output
+// tensors and no allocator, and a serving loop may forbid cudaMalloc in its
+// steady state because an allocation can synchronise the device.  For them,
+// the prefill's cross-tile scratch (look-back flags, carries and tail rows)
+// lives in one file-scope device array of fixed size, reserved when the
+// library is loaded and held by every GPU that loads it until the process
+// exits.  The caller still passes inputs, outputs and the state.
+//
+// The work itself is exactly sfa_prefill's: this entry point only supplies
+// the array's device address as the workspace.
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "sfa_internal.h"
+
+namespace {
+
+// Scratch shared by every call on a device (16 MiB: one 512-token prefill of
+// a 24-layer, hidden-896 model needs about 12 MB).
+constexpr size_t kStaticWorkspaceBytes = SFA_STATIC_WORKSPACE_BYTES;
+static __device__ __align__(256) unsigned char g_static_ws[kStaticWorkspaceBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_ws_mutex;
+void* g_ws_ptr[kMaxDevices] = {};
+
+// Device address of the array on the current device.  The array's name is
+// only a host-side stand-in, so the address is looked up once per device,
+// with that device current, and cached.
+int static_ws_address(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SFA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_ws_mutex);
+  if (g_ws_ptr[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_static_ws) != cudaSuccess || ptr == nullptr) {
+      cudaGetLastError();
+      return SFA_ERR_CUDA;
+    }
+    g_ws_ptr[dev] = ptr;
+  }
+  *out = g_ws_ptr[dev];
+  return SFA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int sfa_prefill_static_ws(const sfa_handle* h, const void* q, const void* k, const void* v,
+                          long long n, int batch, void* state, float* out, void* stream) {
+  if (n < 0 || batch <= 0) return SFA_ERR_INVALID_ARG;
+  if (n == 0) return SFA_OK;
+  const size_t need = sfa_prefill_workspace_bytes(h, batch, n);
+  if (need == 0) return SFA_ERR_INVALID_ARG;
+  if (need > kStaticWorkspaceBytes) return SFA_ERR_WORKSPACE;  // call exceeds the fixed scratch
+  void* ws = nullptr;
+  const int rc = static_ws_address(&ws);
+  if (rc != SFA_OK) return rc;
+  // sfa_prefill clears the part of the workspace that must start at zero
+  // (ticket counter and look-back flags) on the stream before its kernel.
+  return sfa_prefill(h, q, k, v, n, batch, state, out, ws, kStaticWorkspaceBytes, stream);
+}
+
+}  // extern "C"
