@@ -216,6 +216,12 @@ __device__ __forceinline__ void cluster_wait() {
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
+// The same for shared memory of other CTAs of the cluster written through
+// distributed shared memory.
+__device__ __forceinline__ void fence_proxy_async_cluster() {
+  asm volatile("fence.proxy.async.shared::cluster;" ::: "memory");
+}
+
 // ---- programmatic dependent launch ----------------------------------------
 // Everything a kernel reads that an earlier kernel of the stream may write
 // must come after pdl_wait(); pdl_trigger() lets the next kernel's CTAs be

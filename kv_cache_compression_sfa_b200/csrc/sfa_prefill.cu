@@ -157,7 +157,7 @@ __device__ __forceinline__ void near_block(const Tin* qst, const unsigned char* 
 }
 
 template <typename Tin, int D>
-__global__ void __launch_bounds__(kPrefillThreads, 1)
+__global__ void __launch_bounds__(kPrefillThreads, 2)
 prefill_kernel(const PrefillParams p) {
   constexpr int ESZ = static_cast<int>(sizeof(Tin));
   cg::cluster_group cluster = cg::this_cluster();
@@ -188,10 +188,9 @@ prefill_kernel(const PrefillParams p) {
   unsigned char* kb = smb + pl.kb;                        // [KB][rowB] key block
   unsigned char* vb = smb + pl.vb;                        // [KB][rowB] value block
   unsigned char* simg = smb + pl.sl;                      // [nch][hi,lo] slot blocks
-  float* part = reinterpret_cast<float*>(smb + pl.part);  // [T][65]   pool partials
-  float* wts = reinterpret_cast<float*>(smb + pl.wts);    // [T][64]   pool weights
-  unsigned char* xw = smb + pl.semc;                      // x blocks [2][hi,lo] | w blocks + sem chunk
-  float* semc = reinterpret_cast<float*>(xw + 2 * kBlkBytes);  // [T][kSemStride]
+  float* part = reinterpret_cast<float*>(smb + pl.part);  // [T][65]   pool partials, then
+  float* semc = part;                                     // [T][68]   the sem chunk
+  unsigned char* xw = smb + pl.semc;                      // x block (hi, lo), then w block (hi, lo)
 
   __shared__ unsigned long long s_ticket;
   __shared__ long long s_pos;
@@ -506,12 +505,11 @@ prefill_kernel(const PrefillParams p) {
   // of x_chunk . slot_chunk^T, each as hi*hi + hi*lo + lo*hi.
   const uint32_t idesc_s = umma_idesc_bf16(kBlk, kSlots, false);
   const uint32_t idesc_c = umma_idesc_bf16(kBlk, kCW, true);
+  unsigned char* xhi = xw;
+  unsigned char* xlo = xw + kBlkBytes;
   for (int c = 0; c < nch; ++c) {
-    const int buf = c & 1;
-    unsigned char* xhi = xw + buf * 2 * kBlkBytes;
-    unsigned char* xlo = xhi + kBlkBytes;
-    if (c >= 2)  // the MMAs of chunk c-2 have finished reading this x buffer
-      if (!mbar_wait_bounded(bar_ms + buf, ((c - 2) >> 1) & 1, kMbarPollLimit, p.err)) s_bad = 1;
+    if (c >= 1)  // the MMAs of chunk c-1 have finished reading the x block
+      if (!mbar_wait_bounded(bar_ms, (c - 1) & 1, kMbarPollLimit, p.err)) s_bad = 1;
     stage_split_block(xs + c * kBlk, XS, xhi, xlo, tid, NT);
     fence_proxy_async_smem();
     __syncthreads();
@@ -528,7 +526,7 @@ prefill_kernel(const PrefillParams p) {
         umma_bf16(tmem, ah, bl, idesc_s, true);
         umma_bf16(tmem, al, bh, idesc_s, true);
       }
-      umma_commit(bar_ms + buf);
+      umma_commit(bar_ms);
     }
   }
   if (tid == 0) umma_commit(bar_sd);
@@ -617,12 +615,20 @@ prefill_kernel(const PrefillParams p) {
       const float mx = warp_max(fmaxf(c0, c1));
       const float e0 = expf(c0 - mx), e1 = expf(c1 - mx);
       const float inv = 1.f / warp_sum(e0 + e1);
+      __nv_bfloat16 h0, l0, h1, l1;
+      split_bf16(e0 * inv, h0, l0);
+      split_bf16(e1 * inv, h1, l1);
+      const int o0 = blk_off(r, lane), o1 = blk_off(r, lane + 32);
       for (int q = 0; q < p.CS; ++q) {
-        float* rw = cluster.map_shared_rank(wts, q) + r * kSlots;
-        rw[lane] = e0 * inv;
-        rw[lane + 32] = e1 * inv;
+        unsigned char* wq = cluster.map_shared_rank(xw, q);  // the x blocks are dead everywhere
+        *reinterpret_cast<__nv_bfloat16*>(wq + o0) = h0;
+        *reinterpret_cast<__nv_bfloat16*>(wq + kBlkBytes + o0) = l0;
+        *reinterpret_cast<__nv_bfloat16*>(wq + o1) = h1;
+        *reinterpret_cast<__nv_bfloat16*>(wq + kBlkBytes + o1) = l1;
       }
     }
+    // rows of tokens past the tile end feed MMA rows that are never read
+    fence_proxy_async_cluster();
   }
   cluster.sync();
 
@@ -630,9 +636,8 @@ prefill_kernel(const PrefillParams p) {
   // field, fusion, clip, output [P3 §2.1 channels 1–3, §2.2].
   // sem chunk c [T x 64] = w[T x 64] . slot_chunk_c, accumulators alternate
   // between tensor-memory columns 64..127 and 128..191.
-  unsigned char* whi = xw;  // the x blocks are dead: all score MMAs finished
+  unsigned char* whi = xw;  // written by the cluster in (G)
   unsigned char* wlo = xw + kBlkBytes;
-  stage_split_block(wts, kSlots, whi, wlo, tid, NT);
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
@@ -831,12 +836,12 @@ bool plan_prefill(int HPC, int D, int esz, int NGm, int K, size_t budget, Prefil
   p.sagg = off;                 off += a16(4LL * NGm * D);
   p.ml = off;                   off += a16(4LL * (2 * kTile * HPC + kSeg * kCW));
   p.u0 = off;
-  // pool phase: slot blocks, partials, weights, x blocks | w blocks + sem chunk
+  // pool phase: slot blocks, partials | sem chunk, x block | w block
   int q = off;
   p.sl = q;                     q += a16(static_cast<long long>(HS / kBlk) * 2 * kBlkBytes);
-  p.part = q;                   q += a16(4LL * kTile * kPartStride);
-  p.wts = q;                    q += a16(4LL * kTile * kSlots);
-  p.semc = q;                   q += a16(std::max(4LL * kBlkBytes, 2LL * kBlkBytes + 4LL * kTile * kSemStride));
+  p.part = q;                   q += a16(4LL * kTile * std::max(kPartStride, kSemStride));
+  p.wts = q;
+  p.semc = q;                   q += a16(2LL * kBlkBytes);
   const int pool_end = q;
   // staging phase
   q = off;

@@ -97,11 +97,19 @@ class Pair:
         self.ostate = oracle.OracleState(self.p, len(self.layers) * len(self.seqs))
         self.t = 0  # tokens folded in so far
 
+    def _streams(self, x: torch.Tensor) -> torch.Tensor:
+        """The oracle's (layer, sequence) streams of x, selected where x lives
+        (a full-size batch is gigabytes; only the chosen streams go to the host)."""
+        L, S = self.layers, self.seqs
+        if len(L) != x.shape[0]:
+            x = x.index_select(0, torch.tensor(L, device=x.device))
+        if len(S) != x.shape[1]:
+            x = x.index_select(1, torch.tensor(S, device=x.device))
+        return x.cpu()
+
     def _oracle(self, q, k, v) -> np.ndarray:
         L, S = self.layers, self.seqs
-        qs = q[L][:, S] if len(S) != q.shape[1] else q[L]
-        ks = k[L][:, S] if len(S) != k.shape[1] else k[L]
-        vs = v[L][:, S] if len(S) != v.shape[1] else v[L]
+        qs, ks, vs = self._streams(q), self._streams(k), self._streams(v)
         pairs = [(l, b) for l in L for b in S]
         alpha = [oracle_alpha(self.w, l) for (l, _) in pairs]
         sl = np.stack([self.slots_np[l] for (l, _) in pairs]).astype(np.float32)
@@ -125,7 +133,7 @@ class Pair:
         self.t += n
         if not check:
             return None
-        ref = self._oracle(q.cpu(), k.cpu(), v.cpu())
+        ref = self._oracle(q, k, v)
         return self._select(out), ref
 
     def decode(self, check: bool = True):
@@ -135,7 +143,7 @@ class Pair:
         self.t += 1
         if not check:
             return None
-        ref = self._oracle(q.cpu()[:, :, None], k.cpu()[:, :, None], v.cpu()[:, :, None])
+        ref = self._oracle(q[:, :, None], k[:, :, None], v[:, :, None])
         return self._select(out)[:, :, None], ref
 
     def decode_many(self, steps: int) -> Tuple[np.ndarray, np.ndarray]:
@@ -146,7 +154,7 @@ class Pair:
             qs, ks, vs = (x[:, :, s].to(self.device).contiguous() for x in (q, k, v))
             outs.append(self._select(self.op.decode(qs, ks, vs)))
         self.t += steps
-        ref = self._oracle(q.cpu(), k.cpu(), v.cpu())
+        ref = self._oracle(q, k, v)
         return np.stack(outs, axis=2), ref
 
     def compare_state(self, tol: float):
