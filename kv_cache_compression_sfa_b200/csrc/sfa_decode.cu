@@ -12,9 +12,11 @@
 // `rank` owns query heads [rank*HPC, (rank+1)*HPC), i.e. the hidden slice
 // [rank*HS, (rank+1)*HS) with HS = HPC*head_dim.  The semantic pool needs
 // |x| and x·slot_j over the whole hidden vector, so each CTA forms partial
-// sums over its slice and the cluster adds them through distributed shared
-// memory; every CTA then holds the same 64 softmax weights and mixes the
-// slots for its own slice.
+// sums over its slice and pushes them into every peer's shared memory with
+// asynchronous stores that complete bytes on the peer's mbarrier; no
+// cluster-wide barrier sits on the critical path.  Every CTA then adds the
+// same partials in rank order, holds the same 64 softmax weights and mixes
+// the slots for its own slice.
 //
 // Latency.  A decode step of a small batch is bound by memory latency, not
 // bandwidth.  Every operand a CTA needs is brought into shared memory by the
@@ -28,11 +30,15 @@
 //
 // Ordering.  The window slot t mod k and the far state S are read by every
 // CTA that needs that KV head and written by one owner CTA (the one holding
-// the group's first query head) after the first cluster barrier, when all
-// reads are done.  Ring, ring-sum and field elements belong to exactly one
-// CTA.  The stream position is advanced by rank 0 after the same barrier.
+// the group's first query head) once the partials of all ranks have reached
+// it: a rank sends only after its own reads are done.  Ring, ring-sum and
+// field elements belong to exactly one CTA.  The stream position is
+// advanced by rank 0 at the same point.  A CTA leaves only after all peers
+// have stored into it, and it never reads a peer's shared memory.
 #include <cooperative_groups.h>
 #include <cuda_bf16.h>
+
+#include <type_traits>
 
 #include "sfa_common.cuh"
 
@@ -42,13 +48,16 @@ namespace sfa {
 namespace {
 
 constexpr int NW = kDecodeThreads / 32;
-constexpr int kRedStride = kSlots + 4;  // per-warp partials: 64 dots + |x|^2
+constexpr int kRedStride = kSlots + 4;            // pool partials: 64 dots, |x|^2, 3 pad
+constexpr int kRedChunks = kRedStride / 4;        // float4 chunks sent to each peer
+constexpr unsigned kRedBytes = kRedStride * 4u;   // bytes each CTA sends each peer
+constexpr int kMaxCols = kMaxSlice / kDecodeThreads;  // slice columns per thread
 
 // Shared-memory plan (byte offsets).  Slot rows and window slots are padded
 // by 16 bytes so that lanes reading different rows at the same column hit
 // distinct banks.
 struct DecodePlan {
-  int bars, sl, qf, xs, red, part, wts, qraw, kc, vc, sg, fld, rsm, wk, wv, total;
+  int bars, sl, xs, red, inbox, wts, qraw, kc, vc, sg, fld, rsm, wk, wv, total;
   int rec;         // bytes per staged window slot (NGm heads + pad)
   bool stage_win;  // window staged in shared memory
 };
@@ -60,13 +69,12 @@ __host__ __device__ inline DecodePlan decode_plan(int HPC, int D, int esz, int N
   const int HS = HPC * D;
   DecodePlan p;
   int o = 0;
-  p.bars = o;  o += 16;
+  p.bars = o;  o += 32;
   p.sl = o;    o += a16(4LL * kSlots * (HS + 4));
-  p.qf = o;    o += a16(4LL * HS);
   p.xs = o;    o += a16(4LL * HS);
   p.red = o;   o += a16(4LL * NW * kRedStride);
-  p.part = o;  o += a16(4LL * kRedStride);
-  p.wts = o;   o += a16(4LL * kSlots);
+  p.inbox = o; o += a16(4LL * kMaxCluster * kRedStride);
+  p.wts = o;   o += a16(4LL * NW * kSlots);
   p.qraw = o;  o += a16(static_cast<long long>(HS) * esz);
   p.kc = o;    o += a16(static_cast<long long>(NGm) * D * esz);
   p.vc = o;    o += a16(static_cast<long long>(NGm) * D * esz);
@@ -83,11 +91,28 @@ __host__ __device__ inline DecodePlan decode_plan(int HPC, int D, int esz, int N
   return p;
 }
 
+// Address of the same shared-memory location in CTA `rank` of the cluster.
+__device__ __forceinline__ unsigned map_rank(unsigned smem_addr, unsigned rank) {
+  unsigned r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr), "r"(rank));
+  return r;
+}
+
+// 16-byte store into a peer CTA's shared memory whose arrival is counted in
+// bytes on the peer's mbarrier.
+__device__ __forceinline__ void st_async_v4(unsigned addr, float4 v, unsigned bar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::
+          "r"(addr), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(bar)
+      : "memory");
+}
+
 template <typename Tin, int D>
-__global__ void __launch_bounds__(kDecodeThreads)
+__global__ void __launch_bounds__(kDecodeThreads, 3)
 decode_kernel(const DecodeParams p) {
-  constexpr int EPL = D / 32;  // elements of a head row per lane
+  constexpr int EPL = D / 32;  // elements of a head row per lane in P·V
   constexpr int ESZ = static_cast<int>(sizeof(Tin));
+  constexpr int VE = Load16<Tin>::N;
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = static_cast<int>(cluster.block_rank());
   const int b = blockIdx.y, l = blockIdx.z;
@@ -102,29 +127,35 @@ decode_kernel(const DecodeParams p) {
   const DecodePlan pl = decode_plan(HPC, D, ESZ, p.NGm, K, p.smem_budget);
   uint64_t* bar_sl = reinterpret_cast<uint64_t*>(smb + pl.bars);
   uint64_t* bar_in = bar_sl + 1;
-  float* sl = reinterpret_cast<float*>(smb + pl.sl);      // [64][HS+4] slot slice
-  float* qf = reinterpret_cast<float*>(smb + pl.qf);      // [HS] queries, fp32
-  float* xs = reinterpret_cast<float*>(smb + pl.xs);      // [HS] x_t
-  float* red = reinterpret_cast<float*>(smb + pl.red);    // [NW][68] per-warp pool partials
-  float* part = reinterpret_cast<float*>(smb + pl.part);  // [68] CTA pool partials
-  float* wts = reinterpret_cast<float*>(smb + pl.wts);    // [64] pool weights
-  Tin* qraw = reinterpret_cast<Tin*>(smb + pl.qraw);      // [HS] queries as stored
-  Tin* kc = reinterpret_cast<Tin*>(smb + pl.kc);          // [NG][D] K_t
-  Tin* vc = reinterpret_cast<Tin*>(smb + pl.vc);          // [NG][D] V_t
-  float* sg = reinterpret_cast<float*>(smb + pl.sg);      // [NG][D] S before this step
-  float* fld = reinterpret_cast<float*>(smb + pl.fld);    // [HS] field before this step
-  float* rsm = reinterpret_cast<float*>(smb + pl.rsm);    // [HS] ring sum before this step
-  unsigned char* wk = smb + pl.wk;                        // [K][rec] window keys
-  unsigned char* wv = smb + pl.wv;                        // [K][rec] window values
+  uint64_t* bar_red = bar_sl + 2;
+  float* sl = reinterpret_cast<float*>(smb + pl.sl);        // [64][HS+4] slot slice
+  float* xs = reinterpret_cast<float*>(smb + pl.xs);        // [HS] x_t
+  float* red = reinterpret_cast<float*>(smb + pl.red);      // [NW][68] per-warp pool partials
+  float* inbox = reinterpret_cast<float*>(smb + pl.inbox);  // [CS][68] partials of every rank
+  float* wts = reinterpret_cast<float*>(smb + pl.wts) + warp * kSlots;  // this warp's weights
+  Tin* qraw = reinterpret_cast<Tin*>(smb + pl.qraw);        // [HS] queries as stored
+  Tin* kc = reinterpret_cast<Tin*>(smb + pl.kc);            // [NG][D] K_t
+  Tin* vc = reinterpret_cast<Tin*>(smb + pl.vc);            // [NG][D] V_t
+  float* sg = reinterpret_cast<float*>(smb + pl.sg);        // [NG][D] S before this step
+  float* fld = reinterpret_cast<float*>(smb + pl.fld);      // [HS] field before this step
+  float* rsm = reinterpret_cast<float*>(smb + pl.rsm);      // [HS] ring sum before this step
+  unsigned char* wk = smb + pl.wk;                          // [K][rec] window keys
+  unsigned char* wv = smb + pl.wv;                          // [K][rec] window values
   __shared__ long long s_pos;
   __shared__ int s_ok;
 
   if (tid == 0) {
     mbar_init(bar_sl, 1);
     mbar_init(bar_in, 1);
+    mbar_init(bar_red, 1);
     mbar_fence_init();
+    // the partials of all CS ranks (this one included) complete the phase
+    mbar_arrive_expect_tx(bar_red, static_cast<unsigned>(p.CS) * kRedBytes);
   }
   __syncthreads();
+  // Barrier initialisation visible to the peers before any of them stores
+  // into this CTA (they wait on this arrival just before sending).
+  cluster_arrive();
   pdl_trigger();
 
   // Slot slice: constant since sfa_init, so it may be fetched before the
@@ -136,15 +167,11 @@ decode_kernel(const DecodeParams p) {
     for (int j = lane; j < kSlots; j += 32)
       bulk_g2s(sl + j * (HS + 4), slot_base + static_cast<size_t>(j) * p.H, HS * 4u, bar_sl);
   }
-
-  // Other per-layer constants: slot norms and alpha_layer.
-  float nrm0 = 0.f, nrm1 = 0.f, a_l = 0.f;
-  if (warp == 0) {
-    const float* nrm = p.slot_norm + static_cast<size_t>(l) * kSlots;
-    nrm0 = nrm[lane];
-    nrm1 = nrm[lane + 32];
-  }
-  if (tid < HS / 4) a_l = p.alpha_layer[l];
+  // Other per-layer constants: slot norms (lane j: slots j, j+32; every
+  // warp forms the softmax itself) and alpha_layer.
+  const float* nrm = p.slot_norm + static_cast<size_t>(l) * kSlots;
+  const float inrm0 = 1.f / nrm[lane], inrm1 = 1.f / nrm[lane + 32];
+  const float a_l = p.alpha_layer[l];
 
   pdl_wait();  // state and inputs may be written by the previous kernel
 
@@ -195,6 +222,7 @@ decode_kernel(const DecodeParams p) {
   if (!s_ok) {  // the same header for every CTA: the whole grid leaves here
     mbar_wait_bounded(bar_sl, 0, kMbarPollLimit, p.err);  // no copy may land after exit
     mbar_wait_bounded(bar_in, 0, kMbarPollLimit, p.err);
+    cluster_wait();
     if (tid == 0 && rank == 0 && b == 0 && l == 0) latch_error(p.err, SFA_ERR_STATE_MISMATCH);
     return;
   }
@@ -207,99 +235,122 @@ decode_kernel(const DecodeParams p) {
   const int rslot = static_cast<int>(t % kRing);
 
   // The ring slot being replaced depends on t: one round trip later,
-  // overlapped with the near field.
-  const int c4 = tid;  // float4 index within the slice
-  const bool ep = c4 < HS / 4;
-  const int gi = rank * HS + c4 * 4;
-  float4 ring_old = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (ep) ring_old = *reinterpret_cast<const float4*>(ring + static_cast<size_t>(rslot) * p.H + gi);
+  // overlapped with the near field.  Thread tid owns slice columns
+  // tid, tid + 128, ... in the epilogue.
+  const int ncol = (HS - tid + kDecodeThreads - 1) / kDecodeThreads;  // columns of this thread
+  float ring_old[kMaxCols];
+  float* ring_row = ring + static_cast<size_t>(rslot) * p.H + rank * HS;
+#pragma unroll
+  for (int m = 0; m < kMaxCols; ++m)
+    ring_old[m] = (m < ncol) ? ring_row[tid + m * kDecodeThreads] : 0.f;
 
   bool ok = mbar_wait_bounded(bar_in, 0, kMbarPollLimit, p.err);
-  for (int i = tid * 4; i < HS; i += kDecodeThreads * 4) {
-    float v[4];
-    VecLoad<Tin, 4>::run(qraw + i, v);
-    *reinterpret_cast<float4*>(qf + i) = make_float4(v[0], v[1], v[2], v[3]);
-  }
-  __syncthreads();
 
-  // Row of the a-th window position (a = 0 .. nwin-1, position j0+a) for
-  // local KV head gg: K_t/V_t from the input copy, older positions from the
-  // window (shared or global memory); a == -1 names the evicted key t-k.
+  // Window slot of the a-th window position (a = 0 .. nwin-1 is position
+  // j0+a; a == -1 names the evicted key t-k).
   auto wslot = [&](int a) -> int {
     if (a < 0) return eslot;
     const int s2 = slot0 + a;
     return s2 >= K ? s2 - K : s2;
   };
-  auto krow = [&](int a, int gg) -> const Tin* {
-    if (a == nwin - 1) return kc + gg * D;
-    const int sl2 = wslot(a);
-    return pl.stage_win ? reinterpret_cast<const Tin*>(wk + sl2 * pl.rec) + gg * D
-                        : win_k + (static_cast<size_t>(sl2) * nkv + g_lo + gg) * D;
-  };
-  auto vrow = [&](int a, int gg) -> const Tin* {
-    if (a == nwin - 1) return vc + gg * D;
-    const int sl2 = wslot(a);
-    return pl.stage_win ? reinterpret_cast<const Tin*>(wv + sl2 * pl.rec) + gg * D
-                        : win_v + (static_cast<size_t>(sl2) * nkv + g_lo + gg) * D;
-  };
 
-  // (1)-(4) near field per query head [P1 §2.1 eq. O_near]: lane a scores
-  // window position j0+a in full (chunks of 32 keys), online softmax across
-  // chunks, P·V with lanes over head dims; far field with the evicted key
-  // [P1 §2.1 eq. S_t]; x = O_near + alpha_far * S [P1 §2.1 eq. O].
-  for (int hh = warp; hh < HPC; hh += NW) {
-    const int gg = (h0 + hh) / G - g_lo;
-    const float* qh = qf + hh * D;
-    float m = -INFINITY, den = 0.f, o[EPL];
+  // (1)-(4) near field per query head [P1 §2.1 eq. O_near]: a chunk of KPC
+  // window positions at a time, LPK = 32/KPC lanes per position splitting
+  // the q·K dot product; online softmax across chunks; P·V with lanes over
+  // head dims.  Then the far field with the evicted key [P1 §2.1 eq. S_t]
+  // and x = O_near + alpha_far * S [P1 §2.1 eq. O].  STAGED: window rows in
+  // shared memory (else read from global memory).
+  auto near_field = [&](auto staged_c, auto kpc_c) {
+    constexpr bool STAGED = decltype(staged_c)::value;
+    constexpr int KPC = decltype(kpc_c)::value;
+    constexpr int LPK = 32 / KPC;
+    constexpr int DL = D / LPK;  // dims of the score per lane
+    auto krow = [&](int a, int gg) -> const Tin* {
+      if (a == nwin - 1) return kc + gg * D;
+      const int s2 = wslot(a);
+      if constexpr (STAGED) return reinterpret_cast<const Tin*>(wk + s2 * pl.rec) + gg * D;
+      else return win_k + (static_cast<size_t>(s2) * nkv + g_lo + gg) * D;
+    };
+    auto vrow = [&](int a, int gg) -> const Tin* {
+      if (a == nwin - 1) return vc + gg * D;
+      const int s2 = wslot(a);
+      if constexpr (STAGED) return reinterpret_cast<const Tin*>(wv + s2 * pl.rec) + gg * D;
+      else return win_v + (static_cast<size_t>(s2) * nkv + g_lo + gg) * D;
+    };
+    const int key = lane / LPK, part = lane % LPK;
+    for (int hh = warp; hh < HPC; hh += NW) {
+      const int gg = (h0 + hh) / G - g_lo;
+      const Tin* qh = qraw + hh * D + part * DL;
+      float m = -INFINITY, den = 0.f, o[EPL];
 #pragma unroll
-    for (int e = 0; e < EPL; ++e) o[e] = 0.f;
-    for (int base = 0; base < nwin; base += 32) {
-      const int cnt = min(32, nwin - base);
-      float s = -INFINITY;
-      if (lane < cnt) {
-        const Tin* kp = krow(base + lane, gg);
-        constexpr int VE = Load16<Tin>::N;
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};  // independent chains
+      for (int e = 0; e < EPL; ++e) o[e] = 0.f;
+      for (int base = 0; base < nwin; base += KPC) {
+        const int cnt = min(KPC, nwin - base);
+        // Rows past cnt are clamped to the chunk's last one (their weight
+        // is zero), so every load is unconditional and issued at once.
+        float s;
+        {
+          const Tin* kp = krow(base + min(key, cnt - 1), gg) + part * DL;
+          float acc[4] = {0.f, 0.f, 0.f, 0.f};  // independent chains
+#pragma unroll 4
+          for (int i = 0; i < DL; i += VE) {
+            float kv[VE], qv[VE];
+            Load16<Tin>::run(kp + i, kv);
+            Load16<Tin>::run(qh + i, qv);
 #pragma unroll
-        for (int i = 0; i < D; i += VE) {
-          float kv[VE];
-          Load16<Tin>::run(kp + i, kv);
-#pragma unroll
-          for (int e = 0; e < VE; ++e) acc[e & 3] = fmaf(qh[i + e], kv[e], acc[e & 3]);
-        }
-        s = ((acc[0] + acc[1]) + (acc[2] + acc[3])) * p.score_scale;
-      }
-      const float mn = fmaxf(m, warp_max(s));
-      const float corr = expf(m - mn);
-      const float pj = (lane < cnt) ? expf(s - mn) : 0.f;
-      den = fmaf(den, corr, warp_sum(pj));
-#pragma unroll
-      for (int e = 0; e < EPL; ++e) o[e] *= corr;
-      for (int c0 = 0; c0 < cnt; c0 += 8) {
-        float vv[8][EPL];
-#pragma unroll
-        for (int u = 0; u < 8; ++u)
-          if (c0 + u < cnt) VecLoad<Tin, EPL>::run(vrow(base + c0 + u, gg) + lane * EPL, vv[u]);
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const float pc = __shfl_sync(0xffffffffu, pj, (c0 + u) & 31);
-          if (c0 + u < cnt) {
-#pragma unroll
-            for (int e = 0; e < EPL; ++e) o[e] = fmaf(pc, vv[u][e], o[e]);
+            for (int e = 0; e < VE; ++e) acc[e & 3] = fmaf(qv[e], kv[e], acc[e & 3]);
           }
+          s = (acc[0] + acc[1]) + (acc[2] + acc[3]);
         }
-      }
-      m = mn;
-    }
-    const float inv = 1.f / den;
-    float ev[EPL];
-    if (evict) VecLoad<Tin, EPL>::run(krow(-1, gg) + lane * EPL, ev);
+        if (LPK == 2) s += __shfl_xor_sync(0xffffffffu, s, 1);
+        s = (key < cnt) ? s * p.score_scale : -INFINITY;
+        const float mn = fmaxf(m, warp_max(s));
+        const float corr = expf(m - mn);
+        const float pj = (key < cnt) ? expf(s - mn) : 0.f;
+        den = fmaf(den, corr, warp_sum(part == 0 ? pj : 0.f));
 #pragma unroll
-    for (int e = 0; e < EPL; ++e) {
-      const float s_old = sg[gg * D + lane * EPL + e];
-      const float s_new = evict ? ewma(p.gamma_far, s_old, ev[e]) : s_old;
-      xs[hh * D + lane * EPL + e] = fmaf(p.alpha_far, s_new, o[e] * inv);
+        for (int e = 0; e < EPL; ++e) o[e] *= corr;
+        for (int c0 = 0; c0 < cnt; c0 += 8) {
+          float vv[8][EPL], o2[EPL];
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            VecLoad<Tin, EPL>::run(vrow(base + min(c0 + u, cnt - 1), gg) + lane * EPL, vv[u]);
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) o2[e] = 0.f;
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            // position c0+u >= cnt has pj == 0 on its lane
+            const float pc = __shfl_sync(0xffffffffu, pj, (c0 + u) * LPK);
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) {
+              if (u & 1) o2[e] = fmaf(pc, vv[u][e], o2[e]);
+              else o[e] = fmaf(pc, vv[u][e], o[e]);
+            }
+          }
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) o[e] += o2[e];
+        }
+        m = mn;
+      }
+      const float inv = 1.f / den;
+      float ev[EPL];
+      if (evict) VecLoad<Tin, EPL>::run(krow(-1, gg) + lane * EPL, ev);
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) {
+        const float s_old = sg[gg * D + lane * EPL + e];
+        const float s_new = evict ? ewma(p.gamma_far, s_old, ev[e]) : s_old;
+        xs[hh * D + lane * EPL + e] = fmaf(p.alpha_far, s_new, o[e] * inv);
+      }
     }
+  };
+  using T_ = std::true_type;
+  using F_ = std::false_type;
+  using K16 = std::integral_constant<int, 16>;
+  using K32 = std::integral_constant<int, 32>;
+  if (pl.stage_win) {
+    if (K <= 16) near_field(T_{}, K16{}); else near_field(T_{}, K32{});
+  } else {
+    if (K <= 16) near_field(F_{}, K16{}); else near_field(F_{}, K32{});
   }
   __syncthreads();
 
@@ -313,6 +364,7 @@ decode_kernel(const DecodeParams p) {
     const float* r1 = sl + (lane + 32) * (HS + 4) + warp * q4;
     float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0;  // one chain per component
     float ss = 0.f;
+#pragma unroll 4
     for (int e = 0; e < q4; e += 4) {
       const float4 xv = *reinterpret_cast<const float4*>(x0 + e);
       const float4 a = *reinterpret_cast<const float4*>(r0 + e);
@@ -326,95 +378,103 @@ decode_kernel(const DecodeParams p) {
     ss = warp_sum(ss);
     red[warp * kRedStride + lane] = (a0.x + a0.y) + (a0.z + a0.w);
     red[warp * kRedStride + lane + 32] = (a1.x + a1.y) + (a1.z + a1.w);
-    if (lane == 0) red[warp * kRedStride + kSlots] = ss;
+    if (lane < kRedStride - kSlots) red[warp * kRedStride + kSlots + lane] = (lane == 0) ? ss : 0.f;
   }
   __syncthreads();
-  if (tid <= kSlots) {
-    float acc = 0.f;
-#pragma unroll
-    for (int w = 0; w < NW; ++w) acc += red[w * kRedStride + tid];
-    part[tid] = acc;
-  }
-  // Partials visible to the cluster; every CTA has finished reading the
-  // window slot, S and pos of this stream (its copies have landed).
-  cluster.sync();
+  // Every peer has initialised its barriers (arrival at the top).
+  cluster_wait();
 
-  // (7b) add the partials of all ranks in rank order (identical in every
-  // CTA), softmax(cos/T), weights to shared memory.  Thread i < 65 fetches
-  // entry i from every rank (all remote loads in flight), warp 0 finishes.
-  if (tid <= kSlots) {
-    float v[kMaxCluster];
+  // (7b) push this CTA's partials (sum over its warps) to every rank's inbox
+  // row `rank`; the stores complete bytes on the receiver's barrier.
+  for (int idx = tid; idx < p.CS * kRedChunks; idx += kDecodeThreads) {
+    const int peer = idx / kRedChunks, c = idx % kRedChunks;
+    float4 v = *reinterpret_cast<const float4*>(red + c * 4);
 #pragma unroll
-    for (int r = 0; r < kMaxCluster; ++r)
-      v[r] = (r < p.CS) ? cluster.map_shared_rank(part, r)[tid] : 0.f;
-    float acc = 0.f;
-#pragma unroll
-    for (int r = 0; r < kMaxCluster; ++r) acc += v[r];
-    red[tid] = acc;  // per-warp partials are no longer needed
+    for (int w = 1; w < NW; ++w) {
+      const float4 u = *reinterpret_cast<const float4*>(red + w * kRedStride + c * 4);
+      v.x += u.x; v.y += u.y; v.z += u.z; v.w += u.w;
+    }
+    st_async_v4(map_rank(smem_u32(inbox + rank * kRedStride + c * 4), peer), v,
+                map_rank(smem_u32(bar_red), peer));
   }
-  cluster_arrive();  // done with the peers' shared memory
-  __syncthreads();
-  if (warp == 0) {
-    const float d0 = red[lane], d1 = red[lane + 32], ss = red[kSlots];
-    const float nx = fmaxf(sqrtf(ss), kNormFloor);
-    const float c0 = d0 / (nx * nrm0) * p.inv_temp;
-    const float c1 = d1 / (nx * nrm1) * p.inv_temp;
+  // All ranks' partials have landed here; every rank has also finished
+  // reading the window slot, S and position of this stream.
+  ok = mbar_wait_bounded(bar_red, 0, kMbarPollLimit, p.err) && ok;
+
+  // Sum in rank order (identical in every CTA and warp), softmax(cos/T);
+  // each warp keeps its own copy of the weights.
+  {
+    float v0[kMaxCluster], v1[kMaxCluster], vs[kMaxCluster];
+#pragma unroll
+    for (int r = 0; r < kMaxCluster; ++r) {
+      const bool in = r < p.CS;
+      v0[r] = in ? inbox[r * kRedStride + lane] : 0.f;
+      v1[r] = in ? inbox[r * kRedStride + lane + 32] : 0.f;
+      vs[r] = in ? inbox[r * kRedStride + kSlots] : 0.f;
+    }
+    float d0 = 0.f, d1 = 0.f, ss = 0.f;
+#pragma unroll
+    for (int r = 0; r < kMaxCluster; ++r) {
+      d0 += v0[r];
+      d1 += v1[r];
+      ss += vs[r];
+    }
+    const float inx = p.inv_temp / fmaxf(sqrtf(ss), kNormFloor);
+    const float c0 = d0 * inrm0 * inx;
+    const float c1 = d1 * inrm1 * inx;
     const float mx = warp_max(fmaxf(c0, c1));
     const float e0 = expf(c0 - mx), e1 = expf(c1 - mx);
     const float inv = 1.f / warp_sum(e0 + e1);
     wts[lane] = e0 * inv;
     wts[lane + 32] = e1 * inv;
+    __syncwarp();
   }
-  __syncthreads();
 
-  // (5)(6)(7c)(8): ring, field, semantic mix, fusion, clip, scale, output.
-  if (ep && ok) {
-    const int i = c4 * 4;
-    float4 se = make_float4(0.f, 0.f, 0.f, 0.f), so = se;  // even / odd slots
-#pragma unroll 16
-    for (int j = 0; j < kSlots; j += 2) {
-      const float4 s4 = *reinterpret_cast<const float4*>(sl + j * (HS + 4) + i);
-      const float4 t4 = *reinterpret_cast<const float4*>(sl + (j + 1) * (HS + 4) + i);
-      const float w0 = wts[j], w1 = wts[j + 1];
-      se.x = fmaf(w0, s4.x, se.x); se.y = fmaf(w0, s4.y, se.y);
-      se.z = fmaf(w0, s4.z, se.z); se.w = fmaf(w0, s4.w, se.w);
-      so.x = fmaf(w1, t4.x, so.x); so.y = fmaf(w1, t4.y, so.y);
-      so.z = fmaf(w1, t4.z, so.z); so.w = fmaf(w1, t4.w, so.w);
-    }
-    const float4 sem = make_float4(se.x + so.x, se.y + so.y, se.z + so.z, se.w + so.w);
-    const float4 x4 = *reinterpret_cast<const float4*>(xs + i);
-    const float4 rs4 = *reinterpret_cast<const float4*>(rsm + i);
-    const float4 f4 = *reinterpret_cast<const float4*>(fld + i);
-    const float xv[4] = {x4.x, x4.y, x4.z, x4.w};
-    const float ov[4] = {ring_old.x, ring_old.y, ring_old.z, ring_old.w};
-    float rv[4] = {rs4.x, rs4.y, rs4.z, rs4.w};
-    float fv[4] = {f4.x, f4.y, f4.z, f4.w};
-    const float sv[4] = {sem.x, sem.y, sem.z, sem.w};
-    float outv[4];
+  // (5)(6)(7c)(8): ring, field, semantic mix, fusion, clip, scale, output;
+  // thread tid takes slice columns tid, tid + 128, ...
+  if (ok) {
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      rv[e] = (rv[e] - ov[e]) + xv[e];          // ring sum after storing x_t
-      fv[e] = ewma(p.ema_gamma, fv[e], xv[e]);  // EMA field
-      float u = rv[e] * (1.0f / kRing) + 0.5f * fv[e] + 0.5f * sv[e];
+    for (int m = 0; m < kMaxCols; ++m) {
+      if (m >= ncol) break;
+      const int c = tid + m * kDecodeThreads;
+      float a[4] = {0.f, 0.f, 0.f, 0.f};  // independent chains
+#pragma unroll 4
+      for (int j = 0; j < kSlots; j += 4) {
+        const float4 w4 = *reinterpret_cast<const float4*>(wts + j);
+        a[0] = fmaf(w4.x, sl[j * (HS + 4) + c], a[0]);
+        a[1] = fmaf(w4.y, sl[(j + 1) * (HS + 4) + c], a[1]);
+        a[2] = fmaf(w4.z, sl[(j + 2) * (HS + 4) + c], a[2]);
+        a[3] = fmaf(w4.w, sl[(j + 3) * (HS + 4) + c], a[3]);
+      }
+      const float sem = (a[0] + a[1]) + (a[2] + a[3]);
+      const float x = xs[c];
+      const float rv = (rsm[c] - ring_old[m]) + x;   // ring sum after storing x_t
+      const float fv = ewma(p.ema_gamma, fld[c], x);  // EMA field
+      float u = rv * (1.0f / kRing) + 0.5f * fv + 0.5f * sem;
       u = fminf(fmaxf(u, -p.clip_eps), p.clip_eps);
-      outv[e] = fmaf(a_l, u, xv[e]);
+      const int gi = rank * HS + c;
+      ring_row[c] = x;
+      ring_sum[gi] = rv;
+      field[gi] = fv;
+      p.out[stream * p.H + gi] = fmaf(a_l, u, x);
     }
-    *reinterpret_cast<float4*>(ring + static_cast<size_t>(rslot) * p.H + gi) = x4;
-    *reinterpret_cast<float4*>(ring_sum + gi) = make_float4(rv[0], rv[1], rv[2], rv[3]);
-    *reinterpret_cast<float4*>(field + gi) = make_float4(fv[0], fv[1], fv[2], fv[3]);
-    *reinterpret_cast<float4*>(p.out + stream * p.H + gi) = make_float4(outv[0], outv[1], outv[2], outv[3]);
   }
 
   // (1)(2) write-back of the KV heads this CTA owns, from the staged copies:
   // S with the evicted key, then K_t, V_t into slot t mod k.  Every CTA of
-  // the cluster has read the old values (first cluster barrier above).
+  // the cluster has read the old values (its partials have arrived).
   if (ok) {
     const int n_own = g_hi - own_lo + 1;
     for (int idx = tid; idx < n_own * D; idx += kDecodeThreads) {
       const int gg = own_lo - g_lo + idx / D;
       const int i = idx % D;
       float s = sg[gg * D + i];
-      if (evict) s = ewma(p.gamma_far, s, to_f32<Tin>(krow(-1, gg)[i]));
+      if (evict) {
+        const int s2 = eslot;
+        const Tin* er = pl.stage_win ? reinterpret_cast<const Tin*>(wk + s2 * pl.rec) + gg * D
+                                     : win_k + (static_cast<size_t>(s2) * nkv + g_lo + gg) * D;
+        s = ewma(p.gamma_far, s, to_f32<Tin>(er[i]));
+      }
       const size_t wo = (static_cast<size_t>(eslot) * nkv + g_lo + gg) * D + i;
       far[(g_lo + gg) * D + i] = s;
       win_k[wo] = kc[gg * D + i];
@@ -422,9 +482,6 @@ decode_kernel(const DecodeParams p) {
     }
     if (rank == 0 && tid == 0) *reinterpret_cast<long long*>(blk + p.so.pos) = t + 1;
   }
-
-  // No CTA may leave while a peer can still read its `part` array.
-  cluster_wait();
 }
 
 template <typename Tin, int D>
