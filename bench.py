@@ -1,16 +1,25 @@
 #!/usr/bin/env python
 """Benchmark of the SFA operator: prefill + decode tokens/s on B200.
 
-One step = state reset, prefill of the workload's prompt, then its decode
-steps, for every layer and sequence (the whole hot path on one batch of
-synthetic input).  A token is one sequence position through all layers.
+One step is one pass of the whole hot path over one batch of synthetic
+input; a token is one sequence position through all layers.  Three kinds of
+step, chosen by the workload:
+
+  * prefill + decode (default; tiny, qwen05b, qwen7b_decode): state reset,
+    prefill of the prompt, then the decode steps, every layer and sequence;
+    L2 is flushed (256 MB write) before every timed step, outside its events.
+  * prefill only (long_prefill): state reset and one prefill of the batch.
+  * decode only (batched_decode and the k x gamma_far x alpha sweep points):
+    the prompt is prefilled once, untimed; a step is the workload's decode
+    steps over all layers and sequences (each decode call moves more than
+    the L2, so nothing is flushed).
 
 Default workload: the Qwen2.5-0.5B attention shape (24 layers, 14 query / 2
 KV heads, head_dim 64, batch 1, prefill 512 + 128 decode steps, k = 16,
-bf16 inputs).  L2 is flushed (256 MB write) before every timed step, outside
-the step's events.
+bf16 inputs).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--workload NAME] [--context N]
 
 N > 1 runs under torch.distributed.run as independent replicas (the
 operator has no cross-stream exchange), timed per rank and reduced with MAX.
@@ -47,6 +56,8 @@ def parse():
     ap.add_argument("--workload", default="qwen05b")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--context", type=int, default=0,
+                    help="prompt length (default: the workload's first prefill length)")
     return ap.parse_args()
 
 
@@ -65,7 +76,7 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def workload_bytes(w):
+def workload_bytes(w, n_pre=None):
     """Algorithmic bytes (what the method must move; no re-reads).
 
     decode launch: per (layer, sequence) q (e*H), out (4H), ring slot read +
@@ -79,7 +90,7 @@ def workload_bytes(w):
     H, S, k = w.hidden, w.n_kv_heads * w.head_dim, w.window_k
     per_seq_layer = (28 + e) * H + (4 * e + 8 + 2 * k * e) * S
     decode = w.n_layers * (w.batch * per_seq_layer + 256 * H)
-    n = w.prefill_n[0]
+    n = w.prefill_n[0] if n_pre is None else n_pre
     state_write = 2 * k * S * e + 4 * S + 72 * H
     prefill = (w.n_layers * w.batch * (n * (e * H + 2 * e * S + 4 * H) + state_write)
                + w.n_layers * 256 * H)
@@ -155,10 +166,10 @@ def gpu_index_for(device) -> str:
     return os.environ.get("CUDA_VISIBLE_DEVICES", "0").split(",")[0] or "0"
 
 
-def kernel_traffic(kernel_src: str, name: str):
+def kernel_traffic(kernel_src: str, name: str, workload: str):
     """DRAM bytes per launch from a committed ncu summary, only if it was
-    taken on the current kernel source (matching sha256)."""
-    path = os.path.join(ROOT, "profiles", f"{name}_traffic.json")
+    taken on the current kernel source (matching sha256) and workload."""
+    path = os.path.join(ROOT, "profiles", f"{name}_traffic_{workload}.json")
     try:
         with open(path) as f:
             d = json.load(f)
@@ -173,54 +184,54 @@ def kernel_traffic(kernel_src: str, name: str):
 # ------------------------------------------------------------------ oracle
 
 
-def oracle_tokens_per_s(w, layers, n_tokens, src, slots_np):
-    """Times the fp64 oracle on `layers` x batch streams over n_tokens."""
+def oracle_tokens_per_s(w, layers, n_tokens, src, slots_np, seqs=None):
+    """Times the fp64 oracle on `layers` x `seqs` streams over n_tokens."""
     import numpy as np
     import oracle
     f = lambda x: float(np.float32(x))
     v = w.values
+    seqs = list(range(w.batch)) if seqs is None else list(seqs)
     p = oracle.OracleParams(w.n_q_heads, w.n_kv_heads, w.head_dim, w.window_k,
                             gamma_far=f(v.gamma_far), alpha_far=f(v.alpha_far))
     q, k, vv = src.get(0, n_tokens)
-    sel = lambda x: x[layers].float().cpu().numpy()
+    sel = lambda x: x[layers][:, seqs].float().cpu().numpy()
     qn, kn, vn = sel(q), sel(k), sel(vv)
-    st = oracle.OracleState(p, len(layers) * w.batch)
+    st = oracle.OracleState(p, len(layers) * len(seqs))
     slots = slots_np[layers]
     t0 = time.perf_counter()
     _, used = oracle.run_layers(p, f(v.alpha_base), f(v.cross_decay), slots, qn, kn, vn, st,
                                 n_layers=w.n_layers)
     dt = time.perf_counter() - t0
-    tokens = w.batch * n_tokens * len(layers) / w.n_layers  # positions through all layers
+    tokens = len(seqs) * n_tokens * len(layers) / w.n_layers  # positions through all layers
     return tokens / dt, used, dt
 
 
-def run_reference(args, w):
+def run_reference(args, w, n_pre):
     rank, world, _ = dist_env()
     if rank != 0:
         return
-    import numpy as np
-    import torch
     from workloads import TokenSource, make_slots
     src = TokenSource(w, "cpu")
     slots_np = make_slots(w, "cpu").numpy()
-    n_tok = 64  # bounded sample per step: one layer, 64 positions
+    n_tok = 64  # bounded sample per step: one layer, a few sequences, 64 positions
+    seqs = list(range(min(w.batch, 4)))
     for _ in range(args.warmup):
-        oracle_tokens_per_s(w, [0], n_tok, src, slots_np)
+        oracle_tokens_per_s(w, [0], n_tok, src, slots_np, seqs)
     times, used = [], 1
     for s in range(args.steps):
-        _, used, dt = oracle_tokens_per_s(w, [s % w.n_layers], n_tok, src, slots_np)
+        _, used, dt = oracle_tokens_per_s(w, [s % w.n_layers], n_tok, src, slots_np, seqs)
         times.append(dt)
     total = sum(times)
-    tokens = args.steps * w.batch * n_tok / w.n_layers
+    tokens = args.steps * len(seqs) * n_tok / w.n_layers
     value = tokens / total
-    sample = (f"per step: 1 layer x {w.batch} seq x {n_tok} positions of the {w.name} "
+    sample = (f"per step: 1 layer x {len(seqs)} seq x {n_tok} positions of the {w.name} "
               f"workload, scaled to positions through all {w.n_layers} layers")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": workload_config(w),
+        "config": workload_config(w, n_pre),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": used, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -228,30 +239,59 @@ def run_reference(args, w):
     print(json.dumps(line), flush=True)
 
 
-def workload_config(w):
+def step_kind(w) -> str:
+    if w.decode_steps == 0:
+        return "prefill"
+    if w.batch >= 64:
+        return "decode"
+    return "step"
+
+
+def workload_config(w, n_pre=None):
+    n_pre = w.prefill_n[0] if n_pre is None else n_pre
+    kind = step_kind(w)
+    if kind == "decode":
+        what = (f"prefill {n_pre} (untimed) then {w.decode_steps} decode steps")
+        l2 = "not flushed: every decode call moves more bytes than the 126 MB L2"
+    elif kind == "prefill":
+        what = f"prefill {n_pre}"
+        l2 = "flushed before every timed step (256 MB write); inputs exceed L2"
+    else:
+        what = f"prefill {n_pre} + {w.decode_steps} decode steps"
+        l2 = "flushed before every timed step (256 MB write)"
     return {
         "workload": (f"{w.name}: {w.n_layers} layers, {w.n_q_heads}q/{w.n_kv_heads}kv heads, "
-                     f"head_dim {w.head_dim}, batch {w.batch}, prefill {w.prefill_n[0]} + "
-                     f"{w.decode_steps} decode steps, k={w.window_k}"),
-        "global_batch": w.batch, "seq_len": w.prefill_n[0] + w.decode_steps,
-        "in_dtype": w.in_dtype, "window_k": w.window_k,
-        "l2": "flushed before every timed step (256 MB write)",
-        "parallelism": "replicas",
+                     f"head_dim {w.head_dim}, batch {w.batch}, {what}, k={w.window_k}"),
+        "global_batch": w.batch, "seq_len": n_pre + w.decode_steps,
+        "in_dtype": w.in_dtype, "window_k": w.window_k, "step": kind,
+        "l2": l2, "parallelism": "replicas",
     }
 
 
+def sfa_config_for(sfa, w):
+    v = w.values
+    return sfa.SfaConfig(n_layers=w.n_layers, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads,
+                         head_dim=w.head_dim, window_k=w.window_k, gamma_far=v.gamma_far,
+                         alpha_far=v.alpha_far, ema_gamma=v.ema_gamma, temperature=v.temperature,
+                         clip_eps=v.clip_eps, alpha_base=v.alpha_base, cross_decay=v.cross_decay,
+                         in_dtype=sfa.SFA_F32 if w.in_dtype == "f32" else sfa.SFA_BF16)
+
+
 # ------------------------------------------------------------------ ours
+
+
+DECODE_RING = 64  # distinct decode inputs cycled by the decode-only step
 
 
 def main():
     args = parse()
     from workloads import get_workload
     w = get_workload(args.workload)
+    n_pre = args.context or w.prefill_n[0]
     if args.impl == "reference":
-        run_reference(args, w)
+        run_reference(args, w, n_pre)
         return
 
-    import numpy as np
     import torch
     import torch.distributed as dist
     import kv_cache_compression_sfa_b200 as sfa
@@ -269,56 +309,95 @@ def main():
                                 device_id=dev)
     sfa_build.build()
 
-    v = w.values
-    cfg = sfa.SfaConfig(n_layers=w.n_layers, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads,
-                        head_dim=w.head_dim, window_k=w.window_k, gamma_far=v.gamma_far,
-                        alpha_far=v.alpha_far, ema_gamma=v.ema_gamma, temperature=v.temperature,
-                        clip_eps=v.clip_eps, alpha_base=v.alpha_base, cross_decay=v.cross_decay,
-                        in_dtype=sfa.SFA_F32 if w.in_dtype == "f32" else sfa.SFA_BF16)
-    n_pre, n_dec = w.prefill_n[0], w.decode_steps
+    kind = step_kind(w)
+    n_dec = w.decode_steps
     L, B, H = w.n_layers, w.batch, w.hidden
     src = TokenSource(w, dev, salt=rank)
     slots = make_slots(w, dev)
-    qp, kp, vp = src.get(0, n_pre)
-    qa, ka, va = src.get(n_pre, n_pre + n_dec)
-    qd = [qa[:, :, t].contiguous() for t in range(n_dec)]
-    kd = [ka[:, :, t].contiguous() for t in range(n_dec)]
-    vd = [va[:, :, t].contiguous() for t in range(n_dec)]
-    op = sfa.SfaOperator(cfg, slots, B, max_prefill=n_pre, device=dev)
-    out_p = torch.empty((L, B, n_pre, H), dtype=torch.float32, device=dev)
-    out_d = torch.empty((n_dec, L, B, H), dtype=torch.float32, device=dev)
+    chunk = 128 if kind == "decode" else n_pre
+    op = sfa.SfaOperator(sfa_config_for(sfa, w), slots, B, max_prefill=chunk, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
-    def prefill_part():
-        op.reset()
-        op.prefill(qp, kp, vp, out=out_p)
+    if kind == "decode":
+        # untimed prompt, in chunks; then a ring of distinct decode inputs
+        n_ring = min(DECODE_RING, n_dec)
+        out_c = torch.empty((L, B, chunk, H), dtype=torch.float32, device=dev)
+        for t0 in range(0, n_pre, chunk):
+            q, k, v = src.get(t0, min(n_pre, t0 + chunk))
+            op.prefill(q, k, v, out=out_c[:, :, :q.shape[2]])
+            del q, k, v
+        del out_c
+        qa, ka, va = src.get(n_pre, n_pre + n_ring)
+        qd = [qa[:, :, t].contiguous() for t in range(n_ring)]
+        kd = [ka[:, :, t].contiguous() for t in range(n_ring)]
+        vd = [va[:, :, t].contiguous() for t in range(n_ring)]
+        del qa, ka, va
+        out_d = torch.empty((n_ring, L, B, H), dtype=torch.float32, device=dev)
+        replays = max(1, n_dec // n_ring)
+        n_dec = replays * n_ring
 
-    def decode_part():
-        for t in range(n_dec):
-            op.decode(qd[t], kd[t], vd[t], out=out_d[t])
+        def part_a():
+            pass
+
+        def part_b():
+            for t in range(n_ring):
+                op.decode(qd[t], kd[t], vd[t], out=out_d[t])
+    else:
+        qp, kp, vp = src.get(0, n_pre)
+        qa, ka, va = src.get(n_pre, n_pre + n_dec)
+        qd = [qa[:, :, t].contiguous() for t in range(n_dec)]
+        kd = [ka[:, :, t].contiguous() for t in range(n_dec)]
+        vd = [va[:, :, t].contiguous() for t in range(n_dec)]
+        out_p = torch.empty((L, B, n_pre, H), dtype=torch.float32, device=dev)
+        out_d = torch.empty((n_dec, L, B, H), dtype=torch.float32, device=dev)
+        replays = 1
+
+        def part_a():
+            op.reset()
+            op.prefill(qp, kp, vp, out=out_p)
+
+        def part_b():
+            for t in range(n_dec):
+                op.decode(qd[t], kd[t], vd[t], out=out_d[t])
 
     # eager warm-up, then capture both halves as CUDA graphs
-    prefill_part()
-    decode_part()
+    part_a()
+    part_b()
     torch.cuda.synchronize()
     rc = op.check()
     if rc != 0:
         raise SystemExit(f"device error during warm-up: {sfa.sfa_status_string(rc)}")
     side = torch.cuda.Stream()
     side.wait_stream(torch.cuda.current_stream())
-    g_pre, g_dec = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    g_a, g_b = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    has_a, has_b = kind != "decode", kind != "prefill"
     with torch.cuda.stream(side):
-        with torch.cuda.graph(g_pre, stream=side):
-            prefill_part()
-        with torch.cuda.graph(g_dec, stream=side):
-            decode_part()
+        if has_a:
+            with torch.cuda.graph(g_a, stream=side):
+                part_a()
+        if has_b:
+            with torch.cuda.graph(g_b, stream=side):
+                part_b()
     torch.cuda.current_stream().wait_stream(side)
     torch.cuda.synchronize()
+    flush_each = kind != "decode"
+
+    def one_step(ev=None):
+        if flush_each:
+            flush.zero_()
+        if ev:
+            ev[0].record()
+        if has_a:
+            g_a.replay()
+        if ev:
+            ev[1].record()
+        for _ in range(replays if has_b else 0):
+            g_b.replay()
+        if ev:
+            ev[2].record()
 
     for _ in range(args.warmup):
-        flush.zero_()
-        g_pre.replay()
-        g_dec.replay()
+        one_step()
     torch.cuda.synchronize()
     if op.check() != 0:
         raise SystemExit("device error during warm-up")
@@ -332,81 +411,88 @@ def main():
         sampler.start()
         time.sleep(0.1)
     for s in range(args.steps):
-        flush.zero_()
-        ev[s][0].record()
-        g_pre.replay()
-        ev[s][1].record()
-        g_dec.replay()
-        ev[s][2].record()
+        one_step(ev[s])
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     clocks = sampler.stop() if sampler else None
     pre_ms = [e[0].elapsed_time(e[1]) for e in ev]
     dec_ms = [e[1].elapsed_time(e[2]) for e in ev]
-    total_ms = sum(pre_ms) + sum(dec_ms)
     rc = op.check()
     if rc != 0:
         raise SystemExit(f"device error in the timed region: {sfa.sfa_status_string(rc)}")
-    t = torch.tensor([total_ms, sum(pre_ms), sum(dec_ms)], dtype=torch.float64, device=dev)
+    t = torch.tensor([sum(pre_ms) + sum(dec_ms), sum(pre_ms), sum(dec_ms)], dtype=torch.float64,
+                     device=dev)
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     total_ms, pre_tot, dec_tot = (float(x) for x in t.tolist())
-    tokens_per_step = B * (n_pre + n_dec)
+    timed_pre = n_pre if has_a else 0
+    tokens_per_step = B * (timed_pre + (n_dec if has_b else 0))
     value = world * tokens_per_step * args.steps / (total_ms / 1e3)
     ms_per_step = total_ms / args.steps
 
-    # ---- roofline of the dominant kernel (decode: 128 of 130 launches/step)
+    # ---- roofline of the dominant kernel
     peak, peak_kind = measured_peaks()
-    dec_bytes, pre_bytes = workload_bytes(w)
-    dec_launch_ms = dec_tot / (args.steps * n_dec)
-    dec_gbs = dec_bytes / (dec_launch_ms / 1e3) / 1e9
-    pre_ms_avg = pre_tot / args.steps
-    pre_gbs = pre_bytes / (pre_ms_avg / 1e3) / 1e9
-    traffic, _ = kernel_traffic(os.path.join(ROOT, "kv_cache_compression_sfa_b200", "csrc",
-                                             "sfa_decode.cu"), "decode")
+    dec_bytes, pre_bytes = workload_bytes(w, n_pre)
+    section = {}
+    if has_a:
+        pre_ms_avg = pre_tot / args.steps
+        pre_gbs = pre_bytes / (pre_ms_avg / 1e3) / 1e9
+        section["prefill"] = {"tokens_per_s": world * B * n_pre * args.steps / (pre_tot / 1e3),
+                              "ms": pre_ms_avg, "algorithmic_bytes": pre_bytes,
+                              "achieved_gbs": pre_gbs, "frac": pre_gbs / peak}
+    if has_b:
+        dec_launch_ms = dec_tot / (args.steps * n_dec)
+        dec_gbs = dec_bytes / (dec_launch_ms / 1e3) / 1e9
+        section["decode"] = {"tokens_per_s": world * B * n_dec * args.steps / (dec_tot / 1e3),
+                             "us_per_step": 1e3 * dec_launch_ms, "algorithmic_bytes": dec_bytes,
+                             "achieved_gbs": dec_gbs, "frac": dec_gbs / peak}
+    dominant = "decode" if has_b and (not has_a or dec_tot >= pre_tot) else "prefill"
+    dom = section[dominant]
+    traffic, _ = kernel_traffic(
+        os.path.join(ROOT, "kv_cache_compression_sfa_b200", "csrc", f"sfa_{dominant}.cu"),
+        dominant, w.name)
+    peak_src = (f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
+                if peak_kind == "measured" else "fallback 6.65 TB/s")
 
     # ---- e2e through the public API with host buffers
     e2e = None
     if not args.no_e2e:
-        e2e = measure_e2e(args, w, op, qp, kp, vp, qa, ka, va, n_pre, n_dec, world, dev)
+        if kind == "decode":
+            e2e = measure_e2e_decode(args, w, op, qd, kd, vd, n_dec, world, dev)
+        else:
+            e2e = measure_e2e(args, w, op, qp, kp, vp, qd, kd, vd, n_pre, n_dec, world, dev)
 
     # ---- oracle on the host cores (rank 0, N = 1 only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(w)
+        cpu = cpu_baseline(w, n_pre)
 
     if world > 1:
         dist.barrier()
-        del g_pre, g_dec
+        del g_a, g_b
         dist.destroy_process_group()
     if rank != 0:
         return
+    launches_per_step = (2 if has_a else 0) + (n_dec if has_b else 0)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": workload_config(w),
-        "prefill": {"tokens_per_s": world * B * n_pre * args.steps / (pre_tot / 1e3),
-                    "ms": pre_ms_avg, "algorithmic_bytes": pre_bytes,
-                    "achieved_gbs": pre_gbs, "frac": pre_gbs / peak},
-        "decode": {"tokens_per_s": world * B * n_dec * args.steps / (dec_tot / 1e3),
-                   "us_per_step": 1e3 * dec_launch_ms, "algorithmic_bytes": dec_bytes,
-                   "achieved_gbs": dec_gbs, "frac": dec_gbs / peak},
-        "roofline": {"bound": "hbm", "kernel": "sfa decode step", "achieved": dec_gbs,
-                     "peak": peak, "unit": "GB/s", "frac": dec_gbs / peak,
-                     "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
-                     if peak_kind == "measured" else "fallback 6.65 TB/s",
-                     "traffic": traffic},
+        "config": workload_config(w, n_pre),
+        **section,
+        "roofline": {"bound": "hbm", "kernel": f"sfa {dominant}", "achieved": dom["achieved_gbs"],
+                     "peak": peak, "unit": "GB/s", "frac": dom["achieved_gbs"] / peak,
+                     "peak_source": peak_src, "traffic": traffic},
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": args.steps * (2 + n_dec),
+        "gpu_launches": args.steps * launches_per_step,
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)
 
 
-def measure_e2e(args, w, op, qp, kp, vp, qa, ka, va, n_pre, n_dec, world, dev):
+def measure_e2e(args, w, op, qp, kp, vp, qd, kd, vd, n_pre, n_dec, world, dev):
     """Same metric through SfaOperator with pinned host inputs and outputs:
     every step copies its q/k/v host->device, runs reset + prefill + decode
     steps, and reads all outputs back."""
@@ -415,8 +501,8 @@ def measure_e2e(args, w, op, qp, kp, vp, qa, ka, va, n_pre, n_dec, world, dev):
     L, B, H = w.n_layers, w.batch, w.hidden
     # decode inputs step-major ([step, L, B, heads, d]) so each step's slice
     # is contiguous on the device
-    step_major = [x.permute(2, 0, 1, 3, 4).contiguous() for x in (qa, ka, va)]
-    host_in = [x.cpu().pin_memory() for x in (qp, kp, vp, *step_major)]
+    dec = [torch.stack(x) if x else None for x in (qd, kd, vd)]
+    host_in = [x.cpu().pin_memory() for x in (qp, kp, vp, *dec) if x is not None]
     dev_in = [torch.empty_like(x, device=dev) for x in host_in]
     h_out_p = torch.empty((L, B, n_pre, H), dtype=torch.float32).pin_memory()
     h_out_d = torch.empty((n_dec, L, B, H), dtype=torch.float32).pin_memory()
@@ -434,8 +520,47 @@ def measure_e2e(args, w, op, qp, kp, vp, qa, ka, va, n_pre, n_dec, world, dev):
         h_out_p.copy_(d_out_p, non_blocking=True)
         for t in range(n_dec):
             op.decode(dev_in[3][t], dev_in[4][t], dev_in[5][t], out=d_out_d[t])
-        h_out_d.copy_(d_out_d, non_blocking=True)
+        if n_dec:
+            h_out_d.copy_(d_out_d, non_blocking=True)
 
+    ms = _time_e2e(one, steps, world, dev)
+    value = world * B * (n_pre + n_dec) * steps / (ms / 1e3)
+    return {"value": value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "steps": steps, "l2": "not flushed (host copies between steps)"}
+
+
+def measure_e2e_decode(args, w, op, qd, kd, vd, n_dec, world, dev):
+    """Decode-only step through SfaOperator: each decode call copies its
+    q/k/v from pinned host memory and its output back."""
+    import torch
+    L, B, H = w.n_layers, w.batch, w.hidden
+    n_ring = len(qd)
+    host = [[x.cpu().pin_memory() for x in xs] for xs in (qd, kd, vd)]
+    dq, dk, dv = (torch.empty_like(x[0], device=dev) for x in (qd, kd, vd))
+    d_out = torch.empty((L, B, H), dtype=torch.float32, device=dev)
+    h_out = torch.empty((n_dec, L, B, H), dtype=torch.float32).pin_memory()
+    per = sum(x[0].numel() * x[0].element_size() for x in host)
+    steps = max(3, min(args.steps, 5))
+
+    def one():
+        for t in range(n_dec):
+            r = t % n_ring
+            dq.copy_(host[0][r], non_blocking=True)
+            dk.copy_(host[1][r], non_blocking=True)
+            dv.copy_(host[2][r], non_blocking=True)
+            op.decode(dq, dk, dv, out=d_out)
+            h_out[t].copy_(d_out, non_blocking=True)
+
+    ms = _time_e2e(one, steps, world, dev)
+    value = world * B * n_dec * steps / (ms / 1e3)
+    return {"value": value, "unit": UNIT, "h2d_bytes_per_step": per * n_dec,
+            "d2h_bytes_per_step": n_dec * L * B * H * 4, "steps": steps,
+            "l2": "not flushed"}
+
+
+def _time_e2e(one, steps, world, dev):
+    import torch
+    import torch.distributed as dist
     for _ in range(3):
         one()
     torch.cuda.synchronize()
@@ -451,28 +576,26 @@ def measure_e2e(args, w, op, qp, kp, vp, qa, ka, va, n_pre, n_dec, world, dev):
     t = torch.tensor([ms], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms = float(t.item())
-    value = world * B * (n_pre + n_dec) * steps / (ms / 1e3)
-    return {"value": value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "steps": steps, "l2": "not flushed (host copies between steps)"}
+    return float(t.item())
 
 
-def cpu_baseline(w):
+def cpu_baseline(w, n_pre):
     import numpy as np
     from workloads import TokenSource, make_slots
     src = TokenSource(w, "cpu")
     slots_np = make_slots(w, "cpu").numpy()
-    n_tok = w.prefill_n[0] + w.decode_steps
-    # bounded sample: as many layers (all sequences, all positions of the
-    # step) as fit in ~15 s, estimated from a one-layer run
-    rate1, used1, dt1 = oracle_tokens_per_s(w, [0], n_tok, src, slots_np)
+    n_tok = n_pre + w.decode_steps
+    # bounded sample: positions 0 .. n_tok-1 of as many (layer, sequence)
+    # streams as fit in ~15 s, estimated from one layer of a few sequences
+    seqs = list(range(min(w.batch, 4)))
+    rate1, used1, dt1 = oracle_tokens_per_s(w, [0], n_tok, src, slots_np, seqs)
     n_layers = max(1, min(w.n_layers, int(15.0 / max(dt1, 1e-3))))
     layers = list(range(n_layers))
-    rate, used, dt = oracle_tokens_per_s(w, layers, n_tok, src, slots_np)
+    rate, used, dt = oracle_tokens_per_s(w, layers, n_tok, src, slots_np, seqs)
     return {"value": rate, "unit": UNIT, "cores": used, "kind": "oracle",
-            "sample": (f"{n_layers} of {w.n_layers} layers x {w.batch} seq x {n_tok} positions "
-                       f"(the full step's positions), {dt:.1f} s; tokens scaled to positions "
-                       f"through all layers")}
+            "sample": (f"{n_layers} of {w.n_layers} layers x {len(seqs)} of {w.batch} seq x "
+                       f"{n_tok} positions, {dt:.1f} s; tokens scaled to positions through all "
+                       f"layers")}
 
 
 if __name__ == "__main__":

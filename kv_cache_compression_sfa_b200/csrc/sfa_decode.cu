@@ -51,13 +51,15 @@ constexpr int NW = kDecodeThreads / 32;
 constexpr int kRedStride = kSlots + 4;            // pool partials: 64 dots, |x|^2, 3 pad
 constexpr int kRedChunks = kRedStride / 4;        // float4 chunks sent to each peer
 constexpr unsigned kRedBytes = kRedStride * 4u;   // bytes each CTA sends each peer
-constexpr int kMaxCols = kMaxSlice / kDecodeThreads;  // slice columns per thread
+constexpr int kColsPerPass = kDecodeThreads / 2;     // epilogue: two threads per column
+constexpr int kMaxCols = kMaxSlice / kColsPerPass;   // columns per thread pair
+constexpr int kMaxHeadsCta = kMaxSlice / 64;         // query heads one CTA can own
 
 // Shared-memory plan (byte offsets).  Slot rows and window slots are padded
 // by 16 bytes so that lanes reading different rows at the same column hit
 // distinct banks.
 struct DecodePlan {
-  int bars, sl, xs, red, inbox, wts, qraw, kc, vc, sg, fld, rsm, wk, wv, total;
+  int bars, sl, xs, red, inbox, wts, pb, mrg, qraw, kc, vc, sg, fld, rsm, wk, wv, total;
   int rec;         // bytes per staged window slot (NGm heads + pad)
   bool stage_win;  // window staged in shared memory
 };
@@ -75,6 +77,8 @@ __host__ __device__ inline DecodePlan decode_plan(int HPC, int D, int esz, int N
   p.red = o;   o += a16(4LL * NW * kRedStride);
   p.inbox = o; o += a16(4LL * kMaxCluster * kRedStride);
   p.wts = o;   o += a16(4LL * NW * kSlots);
+  p.pb = o;    o += a16(4LL * NW * 32);
+  p.mrg = o;   o += a16(4LL * (NW > kMaxHeadsCta ? NW : kMaxHeadsCta) * (D + 4));
   p.qraw = o;  o += a16(static_cast<long long>(HS) * esz);
   p.kc = o;    o += a16(static_cast<long long>(NGm) * D * esz);
   p.vc = o;    o += a16(static_cast<long long>(NGm) * D * esz);
@@ -108,7 +112,7 @@ __device__ __forceinline__ void st_async_v4(unsigned addr, float4 v, unsigned ba
 }
 
 template <typename Tin, int D>
-__global__ void __launch_bounds__(kDecodeThreads, 3)
+__global__ void __launch_bounds__(kDecodeThreads, 2)
 decode_kernel(const DecodeParams p) {
   constexpr int EPL = D / 32;  // elements of a head row per lane in P·V
   constexpr int ESZ = static_cast<int>(sizeof(Tin));
@@ -133,6 +137,8 @@ decode_kernel(const DecodeParams p) {
   float* red = reinterpret_cast<float*>(smb + pl.red);      // [NW][68] per-warp pool partials
   float* inbox = reinterpret_cast<float*>(smb + pl.inbox);  // [CS][68] partials of every rank
   float* wts = reinterpret_cast<float*>(smb + pl.wts) + warp * kSlots;  // this warp's weights
+  float* pb = reinterpret_cast<float*>(smb + pl.pb) + warp * 32;        // this warp's chunk weights
+  float* mrg = reinterpret_cast<float*>(smb + pl.mrg);     // [head][key part][D + 4] partial softmax
   Tin* qraw = reinterpret_cast<Tin*>(smb + pl.qraw);        // [HS] queries as stored
   Tin* kc = reinterpret_cast<Tin*>(smb + pl.kc);            // [NG][D] K_t
   Tin* vc = reinterpret_cast<Tin*>(smb + pl.vc);            // [NG][D] V_t
@@ -234,33 +240,39 @@ decode_kernel(const DecodeParams p) {
   const bool evict = t >= K;
   const int rslot = static_cast<int>(t % kRing);
 
-  // The ring slot being replaced depends on t: one round trip later,
-  // overlapped with the near field.  Thread tid owns slice columns
-  // tid, tid + 128, ... in the epilogue.
-  const int ncol = (HS - tid + kDecodeThreads - 1) / kDecodeThreads;  // columns of this thread
+  // Epilogue mapping: lanes l and l+16 of warp w share slice column
+  // 16w + (l & 15) (+ 128 m), each mixing half of the slots.  The ring slot
+  // being replaced depends on t: one round trip later, overlapped with the
+  // near field.
+  const int ecol = warp * 16 + (lane & 15), ehalf = lane >> 4;
+  const int ncol = (HS - ecol + kColsPerPass - 1) / kColsPerPass;  // uniform over a warp
   float ring_old[kMaxCols];
   float* ring_row = ring + static_cast<size_t>(rslot) * p.H + rank * HS;
 #pragma unroll
   for (int m = 0; m < kMaxCols; ++m)
-    ring_old[m] = (m < ncol) ? ring_row[tid + m * kDecodeThreads] : 0.f;
+    ring_old[m] = (m < ncol && ehalf == 0) ? ring_row[ecol + m * kColsPerPass] : 0.f;
 
   bool ok = mbar_wait_bounded(bar_in, 0, kMbarPollLimit, p.err);
 
   // Window slot of the a-th window position (a = 0 .. nwin-1 is position
-  // j0+a; a == -1 names the evicted key t-k).
+  // j0+a).
   auto wslot = [&](int a) -> int {
-    if (a < 0) return eslot;
     const int s2 = slot0 + a;
     return s2 >= K ? s2 - K : s2;
   };
 
-  // (1)-(4) near field per query head [P1 §2.1 eq. O_near]: a chunk of KPC
-  // window positions at a time, LPK = 32/KPC lanes per position splitting
-  // the q·K dot product; online softmax across chunks; P·V with lanes over
-  // head dims.  Then the far field with the evicted key [P1 §2.1 eq. S_t]
-  // and x = O_near + alpha_far * S [P1 §2.1 eq. O].  STAGED: window rows in
-  // shared memory (else read from global memory).
-  auto near_field = [&](auto staged_c, auto kpc_c) {
+  // (1)-(2) near field per query head [P1 §2.1 eq. O_near].  WPH warps share
+  // a head, each taking a contiguous part of the window; a warp scores KPC
+  // positions at a time with LPK = 32/KPC lanes per position splitting the
+  // q·K dot product, keeps an online softmax (max m, denominator, P·V with
+  // lanes over head dims) and leaves it in `mrg` for the merge below.
+  // STAGED: window rows in shared memory (else read from global memory).
+  int wph = 1;
+  while (wph * 2 * HPC <= NW) wph *= 2;
+  const int gw = warp / wph, sw = warp % wph, n_gw = NW / wph;
+  const int per = (nwin + wph - 1) / wph;
+  const int k_lo = min(nwin, sw * per), k_hi = min(nwin, k_lo + per);
+  auto near_part = [&](auto staged_c, auto kpc_c) {
     constexpr bool STAGED = decltype(staged_c)::value;
     constexpr int KPC = decltype(kpc_c)::value;
     constexpr int LPK = 32 / KPC;
@@ -278,14 +290,14 @@ decode_kernel(const DecodeParams p) {
       else return win_v + (static_cast<size_t>(s2) * nkv + g_lo + gg) * D;
     };
     const int key = lane / LPK, part = lane % LPK;
-    for (int hh = warp; hh < HPC; hh += NW) {
+    for (int hh = gw; hh < HPC; hh += n_gw) {
       const int gg = (h0 + hh) / G - g_lo;
       const Tin* qh = qraw + hh * D + part * DL;
       float m = -INFINITY, den = 0.f, o[EPL];
 #pragma unroll
       for (int e = 0; e < EPL; ++e) o[e] = 0.f;
-      for (int base = 0; base < nwin; base += KPC) {
-        const int cnt = min(KPC, nwin - base);
+      for (int base = k_lo; base < k_hi; base += KPC) {
+        const int cnt = min(KPC, k_hi - base);
         // Rows past cnt are clamped to the chunk's last one (their weight
         // is zero), so every load is unconditional and issued at once.
         float s;
@@ -302,60 +314,92 @@ decode_kernel(const DecodeParams p) {
           }
           s = (acc[0] + acc[1]) + (acc[2] + acc[3]);
         }
-        if (LPK == 2) s += __shfl_xor_sync(0xffffffffu, s, 1);
+#pragma unroll
+        for (int off = 1; off < LPK; off <<= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
         s = (key < cnt) ? s * p.score_scale : -INFINITY;
-        const float mn = fmaxf(m, warp_max(s));
+        // the LPK lanes of a position hold equal values: reduce over positions
+        float mx = s;
+#pragma unroll
+        for (int off = 16; off >= LPK; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        const float mn = fmaxf(m, mx);
         const float corr = expf(m - mn);
         const float pj = (key < cnt) ? expf(s - mn) : 0.f;
-        den = fmaf(den, corr, warp_sum(part == 0 ? pj : 0.f));
+        float ps = pj;
+#pragma unroll
+        for (int off = 16; off >= LPK; off >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
+        den = fmaf(den, corr, ps);
+        if (part == 0) pb[key] = pj;  // weights of the chunk, read back as broadcasts
+        __syncwarp();
 #pragma unroll
         for (int e = 0; e < EPL; ++e) o[e] *= corr;
-        for (int c0 = 0; c0 < cnt; c0 += 8) {
-          float vv[8][EPL], o2[EPL];
+        for (int c0 = 0; c0 < cnt; c0 += 4) {
+          float vv[4][EPL];
 #pragma unroll
-          for (int u = 0; u < 8; ++u)
+          for (int u = 0; u < 4; ++u)
             VecLoad<Tin, EPL>::run(vrow(base + min(c0 + u, cnt - 1), gg) + lane * EPL, vv[u]);
+          const float4 pc = *reinterpret_cast<const float4*>(pb + c0);  // 0 past cnt
 #pragma unroll
-          for (int e = 0; e < EPL; ++e) o2[e] = 0.f;
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            // position c0+u >= cnt has pj == 0 on its lane
-            const float pc = __shfl_sync(0xffffffffu, pj, (c0 + u) * LPK);
-#pragma unroll
-            for (int e = 0; e < EPL; ++e) {
-              if (u & 1) o2[e] = fmaf(pc, vv[u][e], o2[e]);
-              else o[e] = fmaf(pc, vv[u][e], o[e]);
-            }
-          }
-#pragma unroll
-          for (int e = 0; e < EPL; ++e) o[e] += o2[e];
+          for (int e = 0; e < EPL; ++e)
+            o[e] = fmaf(pc.x, vv[0][e], fmaf(pc.y, vv[1][e], fmaf(pc.z, vv[2][e], fmaf(pc.w, vv[3][e], o[e]))));
         }
+        __syncwarp();  // pb is rewritten by the next chunk
         m = mn;
       }
-      const float inv = 1.f / den;
-      float ev[EPL];
-      if (evict) VecLoad<Tin, EPL>::run(krow(-1, gg) + lane * EPL, ev);
+      float* mp = mrg + (hh * wph + sw) * (D + 4);
 #pragma unroll
-      for (int e = 0; e < EPL; ++e) {
-        const float s_old = sg[gg * D + lane * EPL + e];
-        const float s_new = evict ? ewma(p.gamma_far, s_old, ev[e]) : s_old;
-        xs[hh * D + lane * EPL + e] = fmaf(p.alpha_far, s_new, o[e] * inv);
+      for (int e = 0; e < EPL; ++e) mp[lane * EPL + e] = o[e];
+      if (lane == 0) {
+        mp[D] = m;
+        mp[D + 1] = den;
       }
     }
   };
   using T_ = std::true_type;
   using F_ = std::false_type;
+  using K4 = std::integral_constant<int, 4>;
+  using K8 = std::integral_constant<int, 8>;
   using K16 = std::integral_constant<int, 16>;
   using K32 = std::integral_constant<int, 32>;
-  if (pl.stage_win) {
-    if (K <= 16) near_field(T_{}, K16{}); else near_field(T_{}, K32{});
-  } else {
-    if (K <= 16) near_field(F_{}, K16{}); else near_field(F_{}, K32{});
+  {
+    const int pmax = (K + wph - 1) / wph;  // most positions a warp ever takes
+    if (pl.stage_win) {
+      if (pmax <= 4) near_part(T_{}, K4{});
+      else if (pmax <= 8) near_part(T_{}, K8{});
+      else if (pmax <= 16) near_part(T_{}, K16{});
+      else near_part(T_{}, K32{});
+    } else {
+      if (pmax <= 8) near_part(F_{}, K8{});
+      else near_part(F_{}, K32{});
+    }
   }
   __syncthreads();
 
-  // (7a) pool partial sums over this slice [P3 §2.1 channel 3]: warp w takes a
-  // quarter of the slice, lane j slots j and j+32.
+  // (3)-(4) merge the parts of each head (log-sum-exp), far field with the
+  // evicted key [P1 §2.1 eq. S_t], x = O_near + alpha_far * S [P1 §2.1 eq. O].
+  for (int idx = tid; idx < HS; idx += kDecodeThreads) {
+    const int hh = idx / D, i = idx % D;
+    const float* mp = mrg + hh * wph * (D + 4);
+    float mstar = -INFINITY;
+    for (int q = 0; q < wph; ++q) mstar = fmaxf(mstar, mp[q * (D + 4) + D]);
+    float num = 0.f, den = 0.f;
+    for (int q = 0; q < wph; ++q) {
+      const float sc = expf(mp[q * (D + 4) + D] - mstar);
+      num = fmaf(sc, mp[q * (D + 4) + i], num);
+      den = fmaf(sc, mp[q * (D + 4) + D + 1], den);
+    }
+    const int gg = (h0 + hh) / G - g_lo;
+    float s_new = sg[gg * D + i];
+    if (evict) {
+      const Tin* er = pl.stage_win ? reinterpret_cast<const Tin*>(wk + eslot * pl.rec) + gg * D
+                                   : win_k + (static_cast<size_t>(eslot) * nkv + g_lo + gg) * D;
+      s_new = ewma(p.gamma_far, s_new, to_f32<Tin>(er[i]));
+    }
+    xs[idx] = fmaf(p.alpha_far, s_new, num / den);
+  }
+  __syncthreads();
+
+  // (7a) pool partial sums over this slice [P3 §2.1 channel 3]: warp w takes
+  // an eighth of the slice, lane j slots j and j+32.
   ok = mbar_wait_bounded(bar_sl, 0, kMbarPollLimit, p.err) && ok;
   {
     const int q4 = HS / NW;  // elements per warp
@@ -430,33 +474,38 @@ decode_kernel(const DecodeParams p) {
     __syncwarp();
   }
 
-  // (5)(6)(7c)(8): ring, field, semantic mix, fusion, clip, scale, output;
-  // thread tid takes slice columns tid, tid + 128, ...
+  // (5)(6)(7c)(8): ring, field, semantic mix, fusion, clip, scale, output.
+  // Half h of a column's thread pair mixes slots 8i + 4h .. 8i + 4h + 3
+  // (rows four apart: the two halves hit disjoint banks).
   if (ok) {
 #pragma unroll
     for (int m = 0; m < kMaxCols; ++m) {
       if (m >= ncol) break;
-      const int c = tid + m * kDecodeThreads;
+      const int c = ecol + m * kColsPerPass;
       float a[4] = {0.f, 0.f, 0.f, 0.f};  // independent chains
-#pragma unroll 4
-      for (int j = 0; j < kSlots; j += 4) {
+#pragma unroll
+      for (int j8 = 0; j8 < kSlots; j8 += 8) {
+        const int j = j8 + 4 * ehalf;
         const float4 w4 = *reinterpret_cast<const float4*>(wts + j);
         a[0] = fmaf(w4.x, sl[j * (HS + 4) + c], a[0]);
         a[1] = fmaf(w4.y, sl[(j + 1) * (HS + 4) + c], a[1]);
         a[2] = fmaf(w4.z, sl[(j + 2) * (HS + 4) + c], a[2]);
         a[3] = fmaf(w4.w, sl[(j + 3) * (HS + 4) + c], a[3]);
       }
-      const float sem = (a[0] + a[1]) + (a[2] + a[3]);
-      const float x = xs[c];
-      const float rv = (rsm[c] - ring_old[m]) + x;   // ring sum after storing x_t
-      const float fv = ewma(p.ema_gamma, fld[c], x);  // EMA field
-      float u = rv * (1.0f / kRing) + 0.5f * fv + 0.5f * sem;
-      u = fminf(fmaxf(u, -p.clip_eps), p.clip_eps);
-      const int gi = rank * HS + c;
-      ring_row[c] = x;
-      ring_sum[gi] = rv;
-      field[gi] = fv;
-      p.out[stream * p.H + gi] = fmaf(a_l, u, x);
+      float sem = (a[0] + a[1]) + (a[2] + a[3]);
+      sem += __shfl_xor_sync(0xffffffffu, sem, 16);
+      if (ehalf == 0) {
+        const float x = xs[c];
+        const float rv = (rsm[c] - ring_old[m]) + x;   // ring sum after storing x_t
+        const float fv = ewma(p.ema_gamma, fld[c], x);  // EMA field
+        float u = rv * (1.0f / kRing) + 0.5f * fv + 0.5f * sem;
+        u = fminf(fmaxf(u, -p.clip_eps), p.clip_eps);
+        const int gi = rank * HS + c;
+        ring_row[c] = x;
+        ring_sum[gi] = rv;
+        field[gi] = fv;
+        p.out[stream * p.H + gi] = fmaf(a_l, u, x);
+      }
     }
   }
 

@@ -29,7 +29,7 @@ constexpr float kNormFloor = 1e-12f;      // cosine norm clamp
 constexpr int kTile = 64;                 // tokens per prefill tile
 constexpr int kHalo = kRing - 1;          // x rows a tile needs from before it
 constexpr int kPrefillThreads = 256;
-constexpr int kDecodeThreads = 128;
+constexpr int kDecodeThreads = 256;
 constexpr int kGroup = 16;                // tiles per look-back group
 
 // Look-back flag values.
