@@ -58,6 +58,10 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--context", type=int, default=0,
                     help="prompt length (default: the workload's first prefill length)")
+    ap.add_argument("--report", choices=["context", "enhancement"], default=None,
+                    help="instead of the bench line: state footprint and decode time against "
+                         "the context, or the enhancement share and its angle to x")
+    ap.add_argument("--max-context", type=int, default=65536)
     return ap.parse_args()
 
 
@@ -286,6 +290,9 @@ DECODE_RING = 64  # distinct decode inputs cycled by the decode-only step
 def main():
     args = parse()
     from workloads import get_workload
+    if args.report:
+        run_report(args)
+        return
     w = get_workload(args.workload)
     n_pre = args.context or w.prefill_n[0]
     if args.impl == "reference":
@@ -596,6 +603,128 @@ def cpu_baseline(w, n_pre):
             "sample": (f"{n_layers} of {w.n_layers} layers x {len(seqs)} of {w.batch} seq x "
                        f"{n_tok} positions, {dt:.1f} s; tokens scaled to positions through all "
                        f"layers")}
+
+
+# ------------------------------------------------------------------ reports
+
+
+def full_kv_bytes(w, n: int) -> int:
+    """Bytes of a full K/V cache for one sequence at context n, all layers."""
+    e = 4 if w.in_dtype == "f32" else 2
+    return 2 * n * w.n_kv_heads * w.head_dim * e * w.n_layers
+
+
+def enhancement_stats(x, out):
+    """Per (layer, sequence, token): cos(enh, x) and |enh| / |out| with
+    enh = out - x; returns medians and 90th percentiles over all rows."""
+    import numpy as np
+    x = np.asarray(x, np.float64).reshape(-1, np.shape(x)[-1])
+    out = np.asarray(out, np.float64).reshape(-1, np.shape(out)[-1])
+    enh = out - x
+    ne = np.linalg.norm(enh, axis=1)
+    nx = np.linalg.norm(x, axis=1)
+    no = np.linalg.norm(out, axis=1)
+    ok = (ne > 0) & (nx > 0)
+    cos = (enh * x).sum(axis=1)[ok] / (ne[ok] * nx[ok])
+    share = ne[no > 0] / no[no > 0]
+    q = lambda a, p: float(np.percentile(a, p)) if a.size else 0.0
+    return {"cos_median": q(cos, 50), "abs_cos_p90": q(np.abs(cos), 90),
+            "share_median": q(share, 50), "share_p90": q(share, 90), "rows": int(x.shape[0])}
+
+
+def run_report(args):
+    import dataclasses
+    import numpy as np
+    import torch
+    import kv_cache_compression_sfa_b200 as sfa
+    from kv_cache_compression_sfa_b200 import build as sfa_build
+    from workloads import ALPHA_PRESETS, TokenSource, get_workload, make_slots
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py --report needs a CUDA device")
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    sfa_build.build()
+
+    if args.report == "context":
+        # state bytes per sequence vs a full K/V cache, and decode time per
+        # step after prompts of growing length [P1 §2.2, §3.4]
+        w = get_workload(args.workload if args.workload != "qwen05b" else "qwen7b_decode")
+        src = TokenSource(w, dev)
+        op = sfa.SfaOperator(sfa_config_for(sfa, w), make_slots(w, dev), w.batch,
+                             max_prefill=4096, device=dev)
+        lay = op.layout()
+        state_per_seq = lay.stream_stride * w.n_layers
+        n_dec = 64
+        rows = []
+        ctx = 1024
+        while ctx <= args.max_context:
+            op.reset()
+            for t0 in range(0, ctx, 4096):
+                q, k, v = src.get(t0, min(ctx, t0 + 4096))
+                op.prefill(q, k, v)
+                del q, k, v
+            qa, ka, va = src.get(ctx, ctx + n_dec)
+            qd = [qa[:, :, t].contiguous() for t in range(n_dec)]
+            kd = [ka[:, :, t].contiguous() for t in range(n_dec)]
+            vd = [va[:, :, t].contiguous() for t in range(n_dec)]
+            out_d = torch.empty((n_dec, w.n_layers, w.batch, w.hidden), dtype=torch.float32,
+                                device=dev)
+            for t in range(n_dec):  # warm-up (advances the state; cost is flat in t)
+                op.decode(qd[t], kd[t], vd[t], out=out_d[t])
+            g = torch.cuda.CUDAGraph()
+            side = torch.cuda.Stream()
+            side.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(side):
+                with torch.cuda.graph(g, stream=side):
+                    for t in range(n_dec):
+                        op.decode(qd[t], kd[t], vd[t], out=out_d[t])
+            torch.cuda.current_stream().wait_stream(side)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            reps = 4
+            e0.record()
+            for _ in range(reps):
+                g.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            if op.check() != 0:
+                raise SystemExit("device error in the context report")
+            us = 1e3 * e0.elapsed_time(e1) / (reps * n_dec)
+            rows.append({"context": ctx, "decode_us_per_step": us,
+                         "sfa_state_bytes_per_seq": state_per_seq,
+                         "full_kv_bytes_per_seq": full_kv_bytes(w, ctx),
+                         "compression": full_kv_bytes(w, ctx) / state_per_seq})
+            del g, qd, kd, vd, out_d, qa, ka, va
+            ctx *= 2
+        print(json.dumps({"report": "context", "workload": w.name, "n_layers": w.n_layers,
+                          "window_k": w.window_k, "rows": rows}), flush=True)
+        return
+
+    # enhancement share and its angle to x against alpha_base [P2 calibration]
+    w = get_workload(args.workload)
+    n = args.context or w.prefill_n[0]
+    src = TokenSource(w, dev)
+    slots = make_slots(w, dev)
+    q, k, v = src.get(0, n)
+    res = []
+    presets = [(0.0, 0.8)] + [(0.1, 0.8)] + list(ALPHA_PRESETS)
+    outs = {}
+    for ab, dec in presets:
+        wv = w.replace(values=dataclasses.replace(w.values, alpha_base=ab, cross_decay=dec))
+        op = sfa.SfaOperator(sfa_config_for(sfa, wv), slots, w.batch, max_prefill=n, device=dev)
+        outs[(ab, dec)] = op.prefill(q, k, v).cpu().numpy()
+        if op.check() != 0:
+            raise SystemExit("device error in the enhancement report")
+    x = outs[(0.0, 0.8)]  # alpha_base = 0: out == x exactly
+    for ab, dec in presets[1:]:
+        st = enhancement_stats(x, outs[(ab, dec)])
+        per_layer = [enhancement_stats(x[l], outs[(ab, dec)][l])["share_median"]
+                     for l in (0, w.n_layers // 2, w.n_layers - 1)]
+        res.append({"alpha_base": ab, "cross_decay": dec, **st,
+                    "share_median_layers_first_mid_last": per_layer})
+    print(json.dumps({"report": "enhancement", "workload": w.name, "tokens": n,
+                      "data": "synthetic N(0,1) activations; not comparable with trained models",
+                      "rows": res}), flush=True)
 
 
 if __name__ == "__main__":

@@ -75,3 +75,27 @@ def test_reference_arm_prints_one_json_line():
     assert d["cpu_baseline"]["kind"] == "oracle"
     assert d["e2e"]["h2d_bytes_per_step"] == 0
     assert d["config"]["step"] == "step"
+
+
+def test_full_kv_bytes_per_token_7b():
+    # K and V, 4 KV heads x 128 dims, bf16, 28 layers: 57,344 B per token
+    w = WORKLOADS["qwen7b_decode"]
+    assert bench.full_kv_bytes(w, 1) == 57_344
+    assert bench.full_kv_bytes(w, 65536) == 65536 * 57_344
+
+
+def test_enhancement_stats_closed_forms():
+    import numpy as np
+    rng = np.random.default_rng(0)
+    x = rng.standard_normal((50, 64))
+    # enh parallel to x with |enh| = 0.1 |x|: cos 1, share 0.1 / 1.1
+    st = bench.enhancement_stats(x, 1.1 * x)
+    assert abs(st["cos_median"] - 1.0) < 1e-12
+    assert abs(st["share_median"] - 0.1 / 1.1) < 1e-12
+    # enh orthogonal to x: cos 0, share = |e| / sqrt(|x|^2 + |e|^2)
+    e = rng.standard_normal((50, 64))
+    e -= (e * x).sum(1, keepdims=True) / (x * x).sum(1, keepdims=True) * x
+    st = bench.enhancement_stats(x, x + e)
+    assert st["abs_cos_p90"] < 1e-12
+    share = np.linalg.norm(e, axis=1) / np.linalg.norm(x + e, axis=1)
+    assert abs(st["share_median"] - np.median(share)) < 1e-12
