@@ -162,6 +162,40 @@ SFA_API int sfa_prefill(const sfa_handle* h, const void* q, const void* k, const
 SFA_API int sfa_decode_step(const sfa_handle* h, const void* q, const void* k, const void* v,
                     int batch, void* state, float* out, void* stream);
 
+/* Serving variants.  The pages call the enhancement once per layer from
+ * inside the model's attention ([P2] usage example and llama.cpp
+ * integration: one call per layer with that layer's attention output); a
+ * serving loop also drops finished sequences from a decode step.  These calls serve a range of layers and, for decode, a list of
+ * sequences; the arithmetic is exactly that of the full calls.
+ *
+ * Bytes of prefill workspace for a sfa_prefill_layers call of layer_count
+ * layers; 0 on invalid input (layer_count outside 1 .. n_layers). */
+SFA_API size_t sfa_prefill_layers_workspace_bytes(const sfa_handle* h, int layer_count, int batch,
+                                                  long long n);
+
+/* sfa_prefill for layers layer_begin .. layer_begin + layer_count - 1 of the
+ * state only.  q, k, v and out hold those layers alone, [layer_count][batch]
+ * [n][...] in the layouts of sfa_prefill; workspace:
+ * sfa_prefill_layers_workspace_bytes(h, layer_count, batch, n).  Other layers'
+ * streams are untouched.  SFA_ERR_INVALID_ARG for a range outside 0 .. L-1. */
+SFA_API int sfa_prefill_layers(const sfa_handle* h, int layer_begin, int layer_count,
+                               const void* q, const void* k, const void* v, long long n, int batch,
+                               void* state, float* out, void* workspace, size_t workspace_bytes,
+                               void* stream);
+
+/* sfa_decode_step for layers layer_begin .. layer_begin + layer_count - 1 and
+ * n_seq sequences of the batch.  seq_ids: NULL (then n_seq must equal batch
+ * and row i is sequence i) or a DEVICE array of n_seq DISTINCT sequence
+ * indices in [0, batch) (row i is sequence seq_ids[i]; duplicates race on
+ * that sequence's state).  q [layer_count][n_seq][n_q][d], k and v
+ * [layer_count][n_seq][n_kv][d], out [layer_count][n_seq][hidden] fp32.
+ * Sequences not listed keep their state and position.  An index out of range
+ * is skipped on the device and latched as SFA_ERR_INVALID_ARG for
+ * sfa_check_device_status; host-visible errors as for sfa_decode_step. */
+SFA_API int sfa_decode_step_ex(const sfa_handle* h, int layer_begin, int layer_count,
+                               const int* seq_ids, int n_seq, const void* q, const void* k,
+                               const void* v, int batch, void* state, float* out, void* stream);
+
 /* Synchronises `stream`, then returns and clears the first error latched on
  * the device since the last check (SFA_OK if none), or SFA_ERR_CUDA if the
  * stream reports a CUDA error. */

@@ -44,6 +44,7 @@ EXPORTED = (
     "sfa_destroy", "sfa_state_bytes", "sfa_prefill_workspace_bytes", "sfa_state_reset",
     "sfa_prefill", "sfa_decode_step", "sfa_check_device_status", "sfa_status_string",
     "sfa_abi_version", "sfa_debug_set_lookback", "sfa_prefill_static_ws",
+    "sfa_prefill_layers_workspace_bytes", "sfa_prefill_layers", "sfa_decode_step_ex",
 )
 
 
@@ -105,6 +106,9 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
             "sfa_abi_version": (i, []),
             "sfa_debug_set_lookback": (i, [vp, ctypes.c_uint, ll]),
             "sfa_prefill_static_ws": (i, [vp, vp, vp, vp, ll, i, vp, vp, vp]),
+            "sfa_prefill_layers_workspace_bytes": (sz, [vp, i, i, ll]),
+            "sfa_prefill_layers": (i, [vp, i, i, vp, vp, vp, ll, i, vp, vp, vp, sz, vp]),
+            "sfa_decode_step_ex": (i, [vp, i, i, vp, i, vp, vp, vp, i, vp, vp, vp]),
         }
         for name, (res, args) in sigs.items():
             fn = getattr(lib, name)
@@ -251,9 +255,9 @@ def sfa_state_reset(h: Handle, state: torch.Tensor, batch: int, stream=None) -> 
         raise SfaError(rc, "sfa_state_reset")
 
 
-def _qkv_checks(h: Handle, q, k, v, tokens: int, batch: int):
+def _qkv_checks(h: Handle, q, k, v, tokens: int, batch: int, layers: Optional[int] = None):
     c = h.cfg
-    rows = c.n_layers * batch * tokens
+    rows = (c.n_layers if layers is None else layers) * batch * tokens
     return (_dev(q, "q", c.torch_dtype, rows * c.n_q_heads * c.head_dim),
             _dev(k, "k", c.torch_dtype, rows * c.n_kv_heads * c.head_dim),
             _dev(v, "v", c.torch_dtype, rows * c.n_kv_heads * c.head_dim))
@@ -274,6 +278,46 @@ def sfa_prefill(h: Handle, q, k, v, n: int, batch: int, state: torch.Tensor, out
                                     workspace.numel(), _stream_ptr(stream))
     if rc != SFA_OK:
         raise SfaError(rc, "sfa_prefill")
+
+
+def sfa_prefill_layers_workspace_bytes(h: Handle, layer_count: int, batch: int, n: int) -> int:
+    return int(load_library().sfa_prefill_layers_workspace_bytes(h.ptr, layer_count, batch, n))
+
+
+def sfa_prefill_layers(h: Handle, layer_begin: int, layer_count: int, q, k, v, n: int,
+                       batch: int, state: torch.Tensor, out: torch.Tensor,
+                       workspace: Optional[torch.Tensor], stream=None) -> None:
+    """sfa_prefill for layers layer_begin .. layer_begin+layer_count-1 only;
+    q/k/v/out hold those layers alone."""
+    if n == 0:
+        return
+    qp, kp, vp = _qkv_checks(h, q, k, v, n, batch, layer_count)
+    sp = _dev(state, "state", torch.uint8, sfa_state_bytes(h, batch))
+    op = _dev(out, "out", torch.float32, layer_count * batch * n * h.cfg.hidden)
+    need = sfa_prefill_layers_workspace_bytes(h, layer_count, batch, n)
+    if workspace is None or workspace.numel() < need:
+        raise SfaError(SFA_ERR_WORKSPACE, "sfa_prefill_layers")
+    wp = _dev(workspace, "workspace", torch.uint8)
+    rc = load_library().sfa_prefill_layers(h.ptr, layer_begin, layer_count, qp, kp, vp, n, batch,
+                                           sp, op, wp, workspace.numel(), _stream_ptr(stream))
+    if rc != SFA_OK:
+        raise SfaError(rc, "sfa_prefill_layers")
+
+
+def sfa_decode_step_ex(h: Handle, layer_begin: int, layer_count: int,
+                       seq_ids: Optional[torch.Tensor], q, k, v, batch: int,
+                       state: torch.Tensor, out: torch.Tensor, stream=None) -> None:
+    """sfa_decode_step for a layer range and (optionally) a device int32
+    tensor of distinct sequence indices; q/k/v/out rows follow seq_ids."""
+    n_seq = batch if seq_ids is None else int(seq_ids.numel())
+    qp, kp, vp = _qkv_checks(h, q, k, v, 1, n_seq, layer_count)
+    sp = _dev(state, "state", torch.uint8, sfa_state_bytes(h, batch))
+    op = _dev(out, "out", torch.float32, layer_count * n_seq * h.cfg.hidden)
+    ip = None if seq_ids is None else _dev(seq_ids, "seq_ids", torch.int32, n_seq)
+    rc = load_library().sfa_decode_step_ex(h.ptr, layer_begin, layer_count, ip, n_seq, qp, kp, vp,
+                                           batch, sp, op, _stream_ptr(stream))
+    if rc != SFA_OK:
+        raise SfaError(rc, "sfa_decode_step_ex")
 
 
 SFA_STATIC_WORKSPACE_BYTES = 16 << 20
@@ -361,6 +405,32 @@ class SfaOperator:
             out = torch.empty((c.n_layers, self.batch, c.hidden), dtype=torch.float32,
                               device=self.device)
         sfa_decode_step(self.handle, q, k, v, self.batch, self.state, out, stream)
+        return out
+
+    def prefill_layers(self, layer_begin: int, q, k, v, out: Optional[torch.Tensor] = None,
+                       stream=None):
+        """Prefill of layers layer_begin .. layer_begin + q.shape[0] - 1."""
+        lc, n = q.shape[0], q.shape[2]
+        if out is None:
+            out = torch.empty((lc, self.batch, n, self.cfg.hidden), dtype=torch.float32,
+                              device=self.device)
+        if n > 0:
+            need = sfa_prefill_layers_workspace_bytes(self.handle, lc, self.batch, n)
+            if self.workspace is None or self.workspace.numel() < need:
+                self.workspace = torch.empty(need, dtype=torch.uint8, device=self.device)
+            sfa_prefill_layers(self.handle, layer_begin, lc, q, k, v, n, self.batch, self.state,
+                               out, self.workspace, stream)
+        return out
+
+    def decode_ex(self, layer_begin: int, q, k, v, seq_ids: Optional[torch.Tensor] = None,
+                  out: Optional[torch.Tensor] = None, stream=None):
+        """Decode of layers layer_begin .. layer_begin + q.shape[0] - 1 for the
+        sequences in seq_ids (int32, on the device; None = all)."""
+        lc, ns = q.shape[0], q.shape[1]
+        if out is None:
+            out = torch.empty((lc, ns, self.cfg.hidden), dtype=torch.float32, device=self.device)
+        sfa_decode_step_ex(self.handle, layer_begin, lc, seq_ids, q, k, v, self.batch,
+                           self.state, out, stream)
         return out
 
     def check(self, stream=None) -> int:

@@ -104,9 +104,9 @@ std::vector<int> cluster_candidates(int nq, int d) {
   return out;
 }
 
-PrefillWorkspace prefill_workspace(const sfa_config* c, int cs, int batch, long long n) {
+PrefillWorkspace prefill_workspace(const sfa_config* c, int cs, int layers, int batch, long long n) {
   PrefillWorkspace w;
-  const long long streams = static_cast<long long>(c->n_layers) * batch;
+  const long long streams = static_cast<long long>(layers) * batch;
   const long long tiles = streams * ((n + kTile - 1) / kTile);
   const long long H = hidden_of(c);
   const long long sdim = static_cast<long long>(c->n_kv_heads) * c->head_dim;
@@ -332,8 +332,17 @@ size_t sfa_state_bytes(const sfa_handle* h, int batch) {
 }
 
 size_t sfa_prefill_workspace_bytes(const sfa_handle* h, int batch, long long n) {
-  if (!handle_ok(h) || batch <= 0 || n <= 0) return 0;
-  return static_cast<size_t>(prefill_workspace(&h->cfg, h->prefill_cs, batch, n).total);
+  if (!handle_ok(h)) return 0;
+  return sfa_prefill_layers_workspace_bytes(h, h->cfg.n_layers, batch, n);
+}
+
+size_t sfa_prefill_layers_workspace_bytes(const sfa_handle* h, int layer_count, int batch,
+                                          long long n) {
+  if (!handle_ok(h) || batch <= 0 || n <= 0 || layer_count <= 0 ||
+      layer_count > h->cfg.n_layers)
+    return 0;
+  return static_cast<size_t>(
+      prefill_workspace(&h->cfg, h->prefill_cs, layer_count, batch, n).total);
 }
 
 int sfa_state_reset(const sfa_handle* h, void* state, int batch, void* stream) {
@@ -357,16 +366,26 @@ int sfa_state_reset(const sfa_handle* h, void* state, int batch, void* stream) {
 int sfa_prefill(const sfa_handle* h, const void* q, const void* k, const void* v, long long n,
                 int batch, void* state, float* out, void* workspace, size_t workspace_bytes,
                 void* stream) {
+  if (!handle_ok(h)) return SFA_ERR_INVALID_ARG;
+  return sfa_prefill_layers(h, 0, h->cfg.n_layers, q, k, v, n, batch, state, out, workspace,
+                            workspace_bytes, stream);
+}
+
+int sfa_prefill_layers(const sfa_handle* h, int layer_begin, int layer_count, const void* q,
+                       const void* k, const void* v, long long n, int batch, void* state,
+                       float* out, void* workspace, size_t workspace_bytes, void* stream) {
   if (!handle_ok(h) || n < 0 || batch <= 0) return SFA_ERR_INVALID_ARG;
+  if (layer_begin < 0 || layer_count <= 0 || layer_begin + layer_count > h->cfg.n_layers)
+    return SFA_ERR_INVALID_ARG;
   if (n == 0) return SFA_OK;
   if (!q || !k || !v || !state || !out) return SFA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(state) || !aligned16(out) ||
       !aligned16(workspace))
     return SFA_ERR_ALIGNMENT;
   const sfa_config* c = &h->cfg;
-  const PrefillWorkspace w = prefill_workspace(c, h->prefill_cs, batch, n);
+  const PrefillWorkspace w = prefill_workspace(c, h->prefill_cs, layer_count, batch, n);
   if (!workspace || workspace_bytes < static_cast<size_t>(w.total)) return SFA_ERR_WORKSPACE;
-  const long long streams = static_cast<long long>(c->n_layers) * batch;
+  const long long streams = static_cast<long long>(layer_count) * batch;
   const long long tiles_per_stream = (n + kTile - 1) / kTile;
   if (streams * tiles_per_stream * h->prefill_cs > 0x7fffffffLL) return SFA_ERR_UNSUPPORTED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -382,6 +401,7 @@ int sfa_prefill(const sfa_handle* h, const void* q, const void* k, const void* v
   p.out = out;
   p.ws = static_cast<unsigned char*>(workspace);
   p.n = n;
+  p.l0 = layer_begin;
   p.CS = h->prefill_cs;
   p.HPC = c->n_q_heads / p.CS;
   p.tiles_per_stream = static_cast<int>(tiles_per_stream);
@@ -407,14 +427,30 @@ int sfa_prefill(const sfa_handle* h, const void* q, const void* k, const void* v
 
 int sfa_decode_step(const sfa_handle* h, const void* q, const void* k, const void* v, int batch,
                     void* state, float* out, void* stream) {
+  if (!handle_ok(h)) return SFA_ERR_INVALID_ARG;
+  return sfa_decode_step_ex(h, 0, h->cfg.n_layers, nullptr, batch, q, k, v, batch, state, out,
+                            stream);
+}
+
+int sfa_decode_step_ex(const sfa_handle* h, int layer_begin, int layer_count, const int* seq_ids,
+                       int n_seq, const void* q, const void* k, const void* v, int batch,
+                       void* state, float* out, void* stream) {
   if (!handle_ok(h) || batch <= 0 || !q || !k || !v || !state || !out) return SFA_ERR_INVALID_ARG;
+  if (layer_begin < 0 || layer_count <= 0 || layer_begin + layer_count > h->cfg.n_layers)
+    return SFA_ERR_INVALID_ARG;
+  if (n_seq <= 0 || (seq_ids == nullptr && n_seq != batch) || n_seq > batch)
+    return SFA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(state) || !aligned16(out))
     return SFA_ERR_ALIGNMENT;
   const sfa_config* c = &h->cfg;
-  if (batch > 65535 || c->n_layers > 65535) return SFA_ERR_UNSUPPORTED;
+  if (n_seq > 65535 || layer_count > 65535) return SFA_ERR_UNSUPPORTED;
   DecodeParams p;
   std::memset(&p, 0, sizeof(p));
   fill_common(p, h, batch, state);
+  p.l0 = layer_begin;
+  p.Lc = layer_count;
+  p.seq_ids = seq_ids;
+  p.n_seq = n_seq;
   p.q = q;
   p.k = k;
   p.v = v;

@@ -119,7 +119,8 @@ decode_kernel(const DecodeParams p) {
   constexpr int VE = Load16<Tin>::N;
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = static_cast<int>(cluster.block_rank());
-  const int b = blockIdx.y, l = blockIdx.z;
+  const int bi = blockIdx.y, li = blockIdx.z;  // call-relative sequence and layer
+  const int l = p.l0 + li;                      // layer of the state
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int HPC = p.HPC, HS = HPC * D;
   const int K = p.K, G = p.G, nkv = p.nkv;
@@ -181,7 +182,14 @@ decode_kernel(const DecodeParams p) {
 
   pdl_wait();  // state and inputs may be written by the previous kernel
 
-  const long long stream = static_cast<long long>(l) * p.B + b;
+  // Sequence served: from the caller's list, checked against the batch (an
+  // index out of range leaves the cluster without touching the state).
+  int b = bi;
+  if (p.seq_ids) b = __ldcg(p.seq_ids + bi);
+  const bool b_ok = b >= 0 && b < p.B;
+  if (!b_ok) b = 0;
+  const long long stream = static_cast<long long>(l) * p.B + b;  // state stream
+  const long long io = static_cast<long long>(li) * p.n_seq + bi;  // input / output row
   unsigned char* blk = p.state + kHeaderBytes + stream * p.so.stride;
   Tin* win_k = reinterpret_cast<Tin*>(blk + p.so.win_k);
   Tin* win_v = reinterpret_cast<Tin*>(blk + p.so.win_v);
@@ -189,9 +197,9 @@ decode_kernel(const DecodeParams p) {
   float* field = reinterpret_cast<float*>(blk + p.so.field);
   float* ring_sum = reinterpret_cast<float*>(blk + p.so.ring_sum);
   float* ring = reinterpret_cast<float*>(blk + p.so.ring);
-  const Tin* qin = static_cast<const Tin*>(p.q) + (stream * p.nq + h0) * D;
-  const Tin* kin = static_cast<const Tin*>(p.k) + stream * nkv * D;
-  const Tin* vin = static_cast<const Tin*>(p.v) + stream * nkv * D;
+  const Tin* qin = static_cast<const Tin*>(p.q) + (io * p.nq + h0) * D;
+  const Tin* kin = static_cast<const Tin*>(p.k) + io * nkv * D;
+  const Tin* vin = static_cast<const Tin*>(p.v) + io * nkv * D;
 
   if (tid == 0) {  // header and position: independent loads, one round trip
     const uint4 h0v = __ldcg(reinterpret_cast<const uint4*>(p.state));
@@ -225,11 +233,14 @@ decode_kernel(const DecodeParams p) {
       }
   }
   __syncthreads();
-  if (!s_ok) {  // the same header for every CTA: the whole grid leaves here
+  if (!s_ok || !b_ok) {  // uniform over the cluster (same header, same sequence)
     mbar_wait_bounded(bar_sl, 0, kMbarPollLimit, p.err);  // no copy may land after exit
     mbar_wait_bounded(bar_in, 0, kMbarPollLimit, p.err);
     cluster_wait();
-    if (tid == 0 && rank == 0 && b == 0 && l == 0) latch_error(p.err, SFA_ERR_STATE_MISMATCH);
+    if (tid == 0 && rank == 0) {
+      if (!s_ok && bi == 0 && li == 0) latch_error(p.err, SFA_ERR_STATE_MISMATCH);
+      if (s_ok && !b_ok) latch_error(p.err, SFA_ERR_INVALID_ARG);
+    }
     return;
   }
   const long long t = s_pos;
@@ -504,7 +515,7 @@ decode_kernel(const DecodeParams p) {
         ring_row[c] = x;
         ring_sum[gi] = rv;
         field[gi] = fv;
-        p.out[stream * p.H + gi] = fmaf(a_l, u, x);
+        p.out[io * p.H + gi] = fmaf(a_l, u, x);
       }
     }
   }
@@ -537,7 +548,7 @@ template <typename Tin, int D>
 cudaError_t launch_t(const DecodeParams& p, cudaStream_t s) {
   const DecodePlan pl = decode_plan(p.HPC, D, static_cast<int>(sizeof(Tin)), p.NGm, p.K, p.smem_budget);
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p.CS, p.B, p.L);
+  cfg.gridDim = dim3(p.CS, p.n_seq, p.Lc);
   cfg.blockDim = dim3(kDecodeThreads, 1, 1);
   cfg.dynamicSmemBytes = static_cast<size_t>(pl.total);
   cfg.stream = s;

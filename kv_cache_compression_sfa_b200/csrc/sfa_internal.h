@@ -68,6 +68,9 @@ struct DecodeParams {
   uint64_t cfg_hash;
   StreamOffsets so;
   int L, B, nq, nkv, K, H, G, CS, HPC;
+  int l0, Lc;            // layers l0 .. l0+Lc-1 of the state are served
+  const int* seq_ids;    // [n_seq] sequences served (device), or null: 0 .. n_seq-1
+  int n_seq;
   int NGm;          // most KV heads any CTA needs
   int smem_budget;  // shared-memory bytes the plan may use (window staged if it fits)
   float gamma_far, alpha_far, ema_gamma, inv_temp, clip_eps, score_scale;
@@ -101,6 +104,7 @@ struct PrefillParams {
   StreamOffsets so;
   long long n;              // tokens per stream in this call
   int L, B, nq, nkv, K, H, G, CS, HPC;
+  int l0;                   // first layer of the state served (streams are l0*B + ...)
   int NGm;                  // most KV heads any CTA needs
   int KB;                   // rows per staged key/value block
   int tiles_per_stream, n_streams;

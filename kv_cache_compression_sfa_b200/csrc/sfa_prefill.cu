@@ -228,14 +228,15 @@ prefill_kernel(const PrefillParams p) {
   if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
 
   const long long tile = ticket / p.n_streams;
-  const int stream = static_cast<int>(ticket % p.n_streams);
-  const int l = stream / p.B;
+  const int stream = static_cast<int>(ticket % p.n_streams);  // call-relative (layer, seq)
+  const int l = p.l0 + stream / p.B;                          // layer of the state
   const bool last = (tile == p.tiles_per_stream - 1);
   const bool publish = (ticket != p.withhold_tile);
   const long long gstart = (tile / kGroup) * kGroup;         // first tile of this group
   const bool group_end = (tile % kGroup == kGroup - 1) && !last;
 
-  unsigned char* blk = p.state + kHeaderBytes + static_cast<long long>(stream) * p.so.stride;
+  unsigned char* blk = p.state + kHeaderBytes +
+                      (static_cast<long long>(p.l0) * p.B + stream) * p.so.stride;
   if (tid == 0) s_pos = __ldcg(reinterpret_cast<const long long*>(blk + p.so.pos));
   tc_fence_before();
   __syncthreads();
