@@ -14,6 +14,7 @@
 #include <cstdint>
 #include <algorithm>
 #include <type_traits>
+#include <cstdlib>
 #include <cstring>
 #include <new>
 #include <vector>
@@ -37,6 +38,7 @@ struct sfa_handle {
   int decode_budget;
   unsigned spin_limit;
   long long withhold_tile;
+  bool force_simt_near;  // test hook: CUDA-core near field even where the tensor-core one applies
 };
 
 namespace {
@@ -245,6 +247,13 @@ int sfa_init(const sfa_config* cfg, sfa_handle** out) {
   h->prefill_cs = 0;
   h->spin_limit = kDefaultSpinLimit;
   h->withhold_tile = -1;
+  // Test hook (environment, read once per handle): SFA_CUDA_CORE_NEAR_FIELD=1
+  // keeps the prefill near field on the CUDA cores, so both paths can be
+  // checked against the oracle on the same workload.
+  {
+    const char* env = std::getenv("SFA_CUDA_CORE_NEAR_FIELD");
+    h->force_simt_near = env != nullptr && env[0] == '1';
+  }
   const int L = cfg->n_layers, H = hidden_of(cfg);
   const size_t slot_bytes = sizeof(float) * static_cast<size_t>(L) * kSlots * H;
   cudaError_t e = cudaGetDevice(&h->device);
@@ -264,9 +273,13 @@ int sfa_init(const sfa_config* cfg, sfa_handle** out) {
     for (int cs : cluster_candidates(cfg->n_q_heads, cfg->head_dim)) {
       const int hpc = cfg->n_q_heads / cs;
       PrefillPlan plan;
-      if (!plan_prefill(hpc, cfg->head_dim, static_cast<int>(in_bytes(cfg->in_dtype)),
-                        max_kv_heads_per_cta(cfg->n_q_heads, cfg->n_kv_heads, cs), cfg->window_k,
-                        limit, &plan))
+      const int ngm = max_kv_heads_per_cta(cfg->n_q_heads, cfg->n_kv_heads, cs);
+      const int esz = static_cast<int>(in_bytes(cfg->in_dtype));
+      // tensor-core near field for bf16 inputs and windows of at most 16
+      // positions, else the CUDA-core one
+      const bool tc = cfg->in_dtype == SFA_BF16 && cfg->window_k <= 16 && !h->force_simt_near;
+      if (!(tc && plan_prefill(hpc, cfg->head_dim, esz, ngm, cfg->window_k, limit, true, &plan)) &&
+          !plan_prefill(hpc, cfg->head_dim, esz, ngm, cfg->window_k, limit, false, &plan))
         continue;
       const size_t dsm = decode_smem_bytes(hpc, cfg->head_dim, static_cast<int>(in_bytes(cfg->in_dtype)),
                                            max_kv_heads_per_cta(cfg->n_q_heads, cfg->n_kv_heads, cs),

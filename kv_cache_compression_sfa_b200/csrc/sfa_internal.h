@@ -82,7 +82,9 @@ constexpr int kDecodeSmemBudget = 112 * 1024;  // keeps two decode CTAs per SM
 struct PrefillPlan {
   int bars, xs, halo, fcar, sst, sagg, ml;  // persistent regions
   int u0;                                   // start of the union below
-  int qst, kb, vb;                          // near-field staging (phase 1)
+  int tc;                                   // near field on the tensor cores (bf16, k <= 16)
+  int qst, kb, vb;                          // near-field staging (phase 1, CUDA-core near field)
+  int qa, kvp, pa;                          // near-field MMA operands (phase 1, tensor-core near field)
   int sl, part, wts, semc;                  // pool buffers (phase 2)
   int KB;                                   // rows per staged key/value block
   int total;
@@ -129,7 +131,7 @@ inline long long align256(long long x) { return (x + 255) & ~255LL; }
 // Launchers (return the CUDA error of the launch).
 cudaError_t launch_decode(const DecodeParams& p, int in_dtype, int head_dim, cudaStream_t s);
 cudaError_t launch_prefill(const PrefillParams& p, int in_dtype, int head_dim, cudaStream_t s);
-bool plan_prefill(int HPC, int D, int esz, int NGm, int K, size_t budget, PrefillPlan* out);
+bool plan_prefill(int HPC, int D, int esz, int NGm, int K, size_t budget, bool tc, PrefillPlan* out);
 cudaError_t prefill_prepare(int device);
 cudaError_t decode_prepare(int device);
 size_t decode_smem_bytes(int HPC, int head_dim, int esz, int NGm, int K, int budget);

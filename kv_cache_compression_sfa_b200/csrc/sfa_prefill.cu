@@ -44,6 +44,8 @@
 // memory (rank r finishes tokens r, r+CS, ...) and the softmax weights are
 // written into every CTA's shared memory.
 #include <cooperative_groups.h>
+#include <cstring>
+#include <type_traits>
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -64,6 +66,12 @@ constexpr int kSemStride = kCW + 4;      // padded row of the sem chunk
 constexpr int kSeg = 4;                  // token segments per column in the epilogue
 constexpr int kEvChunk = 16;             // evicted-key loads in flight per thread
 constexpr int kTmemCols = 256;           // scores (64) + two 64-column sem buffers
+// Tensor-core near field: key span t0-16 .. t0+63 of a tile (k <= 16) as the
+// N of the score MMA, 8-row groups of that span, and the column of the
+// P·V accumulator in tensor memory.
+constexpr int kSpan = kTile + 16;
+constexpr int kSpanR8 = kSpan / 8;
+constexpr int kTmemO = 128;
 static_assert(kTile == kBlk, "tile tokens are the M of the pool MMAs");
 
 // Near field over one staged key block for all (token, head) pairs of the
@@ -175,18 +183,25 @@ prefill_kernel(const PrefillParams p) {
   uint64_t* bar_ms = bars + 2;                             // [2] score MMAs done, per x buffer
   uint64_t* bar_sd = bars + 4;                             // all score MMAs done
   uint64_t* bar_mc = bars + 5;                             // [2] sem MMAs done, per accumulator
+  uint64_t* bar_nf = bars + 7;                             // near-field MMAs done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8);
   float* xs = reinterpret_cast<float*>(smb + pl.xs);      // [T][XS]  x (O accumulator first)
   float* halo = reinterpret_cast<float*>(smb + pl.halo);  // [15][HS] x of the 15 tokens before
   float* fcar = reinterpret_cast<float*>(smb + pl.fcar);  // [HS]     field carried in
   float* sst = reinterpret_cast<float*>(smb + pl.sst);    // [NGm][D] S carried in / at tile end
   float* sagg = reinterpret_cast<float*>(smb + pl.sagg);  // [NGm][D] this tile's S aggregate
-  float* mrun = reinterpret_cast<float*>(smb + pl.ml);    // [T*HPC]  running max
+  float* segc = reinterpret_cast<float*>(smb + pl.ml);    // [kSeg][kCW] epilogue carries
+  float* mrun = segc + kSeg * kCW;                        // [T*HPC]  running max (CUDA-core near field)
   float* lrun = mrun + kTile * HPC;                       // [T*HPC]  running denominator
-  float* segc = lrun + kTile * HPC;                       // [kSeg][kCW] epilogue carries
   Tin* qst = reinterpret_cast<Tin*>(smb + pl.qst);        // [T][HS]   queries
   unsigned char* kb = smb + pl.kb;                        // [KB][rowB] key block
   unsigned char* vb = smb + pl.vb;                        // [KB][rowB] value block
+  // tensor-core near field: packed query block [64 x D], key and value blocks
+  // [kSpan x D] per KV head, P block [64 x kSpan] (hi, lo)
+  unsigned char* qa = smb + pl.qa;
+  unsigned char* kvp = smb + pl.kvp;
+  unsigned char* pa = smb + pl.pa;
+  const bool tc = pl.tc != 0;
   unsigned char* simg = smb + pl.sl;                      // [nch][hi,lo] slot blocks
   float* part = reinterpret_cast<float*>(smb + pl.part);  // [T][65]   pool partials, then
   float* semc = part;                                     // [T][68]   the sem chunk
@@ -196,9 +211,11 @@ prefill_kernel(const PrefillParams p) {
   __shared__ long long s_pos;
   __shared__ int s_ok;
   __shared__ int s_bad;  // a staging wait ran out: skip global writes
+  __shared__ float s_gpow[kGroup];  // gamma_far^(evictions) of the group's earlier tiles
+  __shared__ float s_gseg[kSeg];    // ema_gamma^(length) of the epilogue's token segments
 
   if (tid == 0) {
-    for (int i = 0; i < 7; ++i) mbar_init(bars + i, 1);
+    for (int i = 0; i < 8; ++i) mbar_init(bars + i, 1);
     mbar_fence_init();
     s_bad = 0;
   }
@@ -283,6 +300,17 @@ prefill_kernel(const PrefillParams p) {
   auto key_row = [&](long long j, int g) -> const Tin* {
     return (j >= pos0) ? kin + ((j - pos0) * nkv + g) * D : win_k + (wslot(j) * nkv + g) * D;
   };
+  auto val_row = [&](long long j, int g) -> const Tin* {
+    return (j >= pos0) ? vin + ((j - pos0) * nkv + g) * D : win_v + (wslot(j) * nkv + g) * D;
+  };
+  // Byte offset of element (c, d) in a packed [kSpan x D] key/value block:
+  // 8 x 16-byte core matrices, the next span-row group 128 bytes on, the next
+  // 8 dims kSpanR8 * 128 bytes on.  The same block is the K-major B of q·K^T
+  // and the MN-major B of P·V.
+  auto kv_off = [](int c, int d) -> int {
+    return ((d >> 3) * kSpanR8 + (c >> 3)) * 128 + (c & 7) * 16 + (d & 7) * 2;
+  };
+  const int kvblk = kSpan * D * 2;
   auto evictions = [&](long long a, int len) -> int {  // positions p in [a, a+len) with p >= k
     const long long lo = a > K ? a : static_cast<long long>(K);
     const long long hi = a + len;
@@ -301,9 +329,9 @@ prefill_kernel(const PrefillParams p) {
     const long long first_valid = bs < 0 ? -bs : 0;      // rows at negative positions stay unused
     const int valid = rows > first_valid ? rows - static_cast<int>(first_valid) : 0;
     const unsigned row_bytes = static_cast<unsigned>(NG * D * ESZ);
-    unsigned bytes = 2u * row_bytes * valid;
+    unsigned bytes = tc ? 0u : 2u * row_bytes * valid;
     if (bi == 0) {
-      bytes += static_cast<unsigned>(Tt * HS * ESZ);
+      if (!tc) bytes += static_cast<unsigned>(Tt * HS * ESZ);
       if (gstart == 0) bytes += static_cast<unsigned>(HS * 4);
       if (tile == 0)
         for (int r = 0; r < kHalo; ++r)
@@ -312,7 +340,7 @@ prefill_kernel(const PrefillParams p) {
     fence_proxy_async_smem();
     if (lane == 0) mbar_arrive_expect_tx(bar_kv, bytes);
     __syncwarp();
-    for (int r = static_cast<int>(first_valid) + lane; r < rows; r += 32) {
+    for (int r = static_cast<int>(first_valid) + lane; r < (tc ? 0 : rows); r += 32) {
       const long long j = bs + r;
       const Tin* ks = (j >= pos0) ? kin + ((j - pos0) * nkv + g_lo) * D : win_k + (wslot(j) * nkv + g_lo) * D;
       const Tin* vs = (j >= pos0) ? vin + ((j - pos0) * nkv + g_lo) * D : win_v + (wslot(j) * nkv + g_lo) * D;
@@ -320,7 +348,7 @@ prefill_kernel(const PrefillParams p) {
       bulk_g2s(vb + r * rowB, vs, row_bytes, bar_kv);
     }
     if (bi == 0) {
-      for (int r = lane; r < Tt; r += 32)
+      for (int r = lane; r < (tc ? 0 : Tt); r += 32)
         bulk_g2s(qst + r * HS, qin + ((t0 - pos0 + r) * p.nq + h0) * D,
                  static_cast<unsigned>(HS * ESZ), bar_kv);
       // carries from the state, read before this tile publishes anything
@@ -335,21 +363,89 @@ prefill_kernel(const PrefillParams p) {
   if (tile == 0)  // ring rows before position 0 are zero
     for (int idx = tid; idx < kHalo * HS; idx += NT)
       if (t0 - kHalo + idx / HS < 0) halo[idx] = 0.f;
-  // running state of the near field (overlaps the copies in flight)
-  for (int i = tid; i < kTile * HPC; i += NT) {
-    mrun[i] = -INFINITY;
-    lrun[i] = 0.f;
+  // Query block of head hh for the tensor-core near field: loads (rows past
+  // the tile are zero) and packed stores [64 x D], split so the loads of the
+  // next head overlap the current head's MMAs.
+  constexpr int kQChunks = (kTile * (D / 8) + NT - 1) / NT;  // 16-byte chunks per thread
+  auto q_load = [&](int hh, uint4 (&val)[kQChunks]) {
+#pragma unroll
+    for (int u = 0; u < kQChunks; ++u) {
+      const int idx = u * NT + tid;
+      const int d8 = idx / kTile, r = idx % kTile;
+      val[u] = make_uint4(0u, 0u, 0u, 0u);
+      if (idx < kTile * (D / 8) && r < Tt)
+        val[u] = *reinterpret_cast<const uint4*>(qin + ((t0 - pos0 + r) * p.nq + h0 + hh) * D + d8 * 8);
+    }
+  };
+  auto q_store = [&](const uint4 (&val)[kQChunks]) {
+#pragma unroll
+    for (int u = 0; u < kQChunks; ++u) {
+      const int idx = u * NT + tid;
+      if (idx < kTile * (D / 8)) *reinterpret_cast<uint4*>(qa + blk_off(idx % kTile, (idx / kTile) * 8)) = val[u];
+    }
+  };
+  if constexpr (ESZ == 2) {
+    if (tc) {
+      {
+        uint4 qv[kQChunks];
+        q_load(0, qv);
+        q_store(qv);
+      }
+      // key and value rows of the span (positions t0-16 .. t0+63) for every
+      // KV head of the CTA, packed for the MMAs; rows before position 0 or
+      // past the tile are zero.  Four 16-byte loads in flight per thread.
+      constexpr int D8 = D / 8;
+      const int per = kSpan * D8;
+      const int total = 2 * NG * per;
+      for (int b0 = 0; b0 < total; b0 += 4 * NT) {
+        uint4 val[4];
+        int dst[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int idx = b0 + u * NT + tid;
+          val[u] = make_uint4(0u, 0u, 0u, 0u);
+          dst[u] = -1;
+          if (idx < total) {
+            const int which = idx / (NG * per), rem = idx % (NG * per);
+            const int gg = rem / per, r2 = rem % per;
+            const int d8 = r2 / kSpan, c = r2 % kSpan;
+            const long long j = kv_start + c;
+            dst[u] = (which * p.NGm + gg) * kvblk + kv_off(c, d8 * 8);
+            if (j >= 0 && c < kv_rows) {
+              const Tin* row = which ? val_row(j, g_lo + gg) : key_row(j, g_lo + gg);
+              val[u] = *reinterpret_cast<const uint4*>(row + d8 * 8);
+            }
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (dst[u] >= 0) *reinterpret_cast<uint4*>(kvp + dst[u]) = val[u];
+      }
+      for (int i = tid; i < 2 * kTile * kSpan * 2 / 16; i += NT)  // P blocks start at zero
+        reinterpret_cast<uint4*>(pa)[i] = make_uint4(0u, 0u, 0u, 0u);
+    }
   }
+  if (!tc)  // running state of the near field (overlaps the copies in flight)
+    for (int i = tid; i < kTile * HPC; i += NT) {
+      mrun[i] = -INFINITY;
+      lrun[i] = 0.f;
+    }
   for (int i = tid; i < kTile * XS; i += NT) xs[i] = 0.f;
   if (!mbar_wait_bounded(bar_kv, 0, kMbarPollLimit, p.err)) s_bad = 1;
   // Keys that leave the window at the tile's tokens are rows 0 .. Tt-1 of the
   // staged span when the first block covers them; otherwise read them from
   // global memory.
-  bool ev_staged = p.KB >= Tt;
+  bool ev_staged = tc || p.KB >= Tt;
   // Folds the keys that leave the window at tokens r_from .. Tt-1 into s
   // (EWMA), calling visit(r, s) after every token; staged rows or global.
   auto scan_evicted = [&](int gg, int i, int r_from, float s, auto&& visit) -> float {
-    if (ev_staged) {
+    if (ev_staged && tc) {  // packed key block: span row r is position t0 - k + r
+      const unsigned char* kg = kvp + gg * kvblk;
+      for (int r = 0; r < Tt; ++r) {
+        if (r >= r_from) s = ewma(gf, s, to_f32<Tin>(*reinterpret_cast<const Tin*>(kg + kv_off(r, i))));
+        visit(r, s);
+      }
+    } else if (ev_staged) {
       const Tin* col = reinterpret_cast<const Tin*>(kb) + gg * D + i;
       const int pitch = rowB / ESZ;
       for (int r = 0; r < Tt; ++r) {
@@ -390,27 +486,154 @@ prefill_kernel(const PrefillParams p) {
     for (int g = own_lo; g <= g_hi; ++g) st_release_u32(&fs_agg[ticket * nkv + g], 1u);
   }
 
-  // ---- (B) near field [P1 §2.1 eq. O_near], block by block ---------------
-  for (int bi = 0; bi < n_blocks; ++bi) {
-    if (bi > 0 && !mbar_wait_bounded(bar_kv, bi & 1, kMbarPollLimit, p.err)) s_bad = 1;
-    const long long bs = kv_start + static_cast<long long>(bi) * p.KB;
-    const long long be = bs + min(p.KB, kv_rows - bi * p.KB);  // exclusive
-    if (K <= 16)
-      near_block<Tin, D, 16>(qst, kb, vb, xs, mrun, lrun, rowB, HS, XS, HPC, G, g_lo, K, t0, Tt,
-                             bs, be, p.score_scale, h0, warp, lane);
-    else
-      near_block<Tin, D, 32>(qst, kb, vb, xs, mrun, lrun, rowB, HS, XS, HPC, G, g_lo, K, t0, Tt,
-                             bs, be, p.score_scale, h0, warp, lane);
-    __syncthreads();  // the block buffers are free again
-    if (bi + 1 < n_blocks) issue_block(bi + 1);
+  // ---- (B) near field [P1 §2.1 eq. O_near] ---------------------------------
+  bool near_done = false;
+  if constexpr (ESZ == 2) {
+    if (tc) {
+      // On the tensor cores, one query head at a time:
+      //   S[64 x kSpan] = Q_h . K_g^T (tensor memory, columns 0..kSpan-1);
+      //   softmax over the band of each row (token r sees span rows r+1 ..
+      //   r+k, positions t0+r-k+1 .. t0+r, none before position 0);
+      //   P split into bf16 hi + lo (about 16 significant bits);
+      //   O[64 x D] = P_hi . V_g + P_lo . V_g (columns kTmemO..), into the x tile.
+      // Accumulator row r sits in lane (r % 16) + 32 (r / 16); warp w (w < 4)
+      // loads span columns 32 (w / 2) .. + 63, which hold the bands of its 16 rows.
+      const uint32_t idesc_qk = umma_idesc_bf16(kTile, kSpan, false);
+      const uint32_t idesc_pv = umma_idesc_bf16(kTile, D, true);
+      const int sp = warp & 3, pbase = 32 * (sp >> 1);
+      const int cmin = kv_start < 0 ? static_cast<int>(-kv_start) : 0;  // first row at position >= 0
+      unsigned char* pa_hi = pa;
+      unsigned char* pa_lo = pa + kTile * kSpan * 2;
+      unsigned nf_par = 0;
+      for (int hh = 0; hh < HPC; ++hh) {
+        const int gg = (h0 + hh) / G - g_lo;
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+          tc_fence_after();
+          const unsigned char* kg = kvp + gg * kvblk;
+#pragma unroll
+          for (int s2 = 0; s2 < D / 16; ++s2)
+            umma_bf16(tmem, umma_desc(qa + s2 * 2048, 1024, 128),
+                      umma_desc(kg + s2 * 2 * kSpanR8 * 128, kSpanR8 * 128, 128), idesc_qk, s2 > 0);
+          umma_commit(bar_nf);
+        }
+        uint4 qn[kQChunks];  // the next head's queries, in flight during the MMAs
+        if (hh + 1 < HPC) q_load(hh + 1, qn);
+        if (!mbar_wait_bounded(bar_nf, nf_par, kMbarPollLimit, p.err)) s_bad = 1;
+        nf_par ^= 1u;
+        tc_fence_after();
+        if (hh + 1 < HPC) q_store(qn);  // the score MMAs have read the query block
+        if (warp < 4) {
+          float v[64];
+          tmem_ld32(tmem + (static_cast<uint32_t>(32 * sp) << 16) + pbase, *reinterpret_cast<float(*)[32]>(v));
+          tmem_ld32(tmem + (static_cast<uint32_t>(32 * sp) << 16) + pbase + 32,
+                    *reinterpret_cast<float(*)[32]>(v + 32));
+          // The bands of rows 16 sp .. 16 sp + 15 lie in span columns
+          // 16 sp .. 16 sp + 31: loaded columns J0 .. J0 + 31 with
+          // J0 = 16 (sp & 1); only those are scored and written (the other
+          // P columns stay zero).
+          auto band = [&](auto j0_c) {
+            constexpr int J0 = decltype(j0_c)::value;
+            const int r = 16 * sp + lane;
+            float mx = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int c = pbase + J0 + j;
+              const bool in = c >= r + 1 && c <= r + K && c >= cmin;
+              v[J0 + j] = in ? v[J0 + j] * p.score_scale : -INFINITY;
+              mx = fmaxf(mx, v[J0 + j]);
+            }
+            float sum = 0.f;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              v[J0 + j] = __expf(v[J0 + j] - mx);  // 0 outside the band
+              sum += v[J0 + j];
+            }
+            const float inv = 1.f / sum;
+#pragma unroll
+            for (int g8 = 0; g8 < 4; ++g8) {
+              uint32_t hw[4], lw[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                __nv_bfloat16 h0b, l0b, h1b, l1b;
+                split_bf16(v[J0 + 8 * g8 + 2 * e] * inv, h0b, l0b);
+                split_bf16(v[J0 + 8 * g8 + 2 * e + 1] * inv, h1b, l1b);
+                hw[e] = static_cast<uint32_t>(__bfloat16_as_ushort(h0b)) |
+                        (static_cast<uint32_t>(__bfloat16_as_ushort(h1b)) << 16);
+                lw[e] = static_cast<uint32_t>(__bfloat16_as_ushort(l0b)) |
+                        (static_cast<uint32_t>(__bfloat16_as_ushort(l1b)) << 16);
+              }
+              const int off = blk_off(r, pbase + J0 + 8 * g8);
+              *reinterpret_cast<uint4*>(pa_hi + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+              *reinterpret_cast<uint4*>(pa_lo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+            }
+          };
+          if (lane < 16) {
+            if (sp & 1) band(std::integral_constant<int, 16>{});
+            else band(std::integral_constant<int, 0>{});
+          }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+          tc_fence_after();
+          const unsigned char* vg = kvp + (p.NGm + gg) * kvblk;
+#pragma unroll
+          for (int s2 = 0; s2 < kSpan / 16; ++s2) {
+            const uint64_t bv = umma_desc(vg + s2 * 256, 128, kSpanR8 * 128);
+            umma_bf16(tmem + kTmemO, umma_desc(pa_hi + s2 * 2048, 1024, 128), bv, idesc_pv, s2 > 0);
+            umma_bf16(tmem + kTmemO, umma_desc(pa_lo + s2 * 2048, 1024, 128), bv, idesc_pv, true);
+          }
+          umma_commit(bar_nf);
+        }
+        if (!mbar_wait_bounded(bar_nf, nf_par, kMbarPollLimit, p.err)) s_bad = 1;
+        nf_par ^= 1u;
+        tc_fence_after();
+        {  // O rows into the x tile: warps w and w + 4 take halves of the head
+          const int colh = (warp >> 2) * (D / 2);
+          const int r = 16 * sp + lane;
+#pragma unroll
+          for (int c0 = 0; c0 < D / 2; c0 += 32) {
+            float v[32];
+            tmem_ld32(tmem + (static_cast<uint32_t>(32 * sp) << 16) + kTmemO + colh + c0, v);
+            if (lane < 16 && r < Tt) {
+              float* dst = xs + r * XS + hh * D + colh + c0;
+#pragma unroll
+              for (int j = 0; j < 32; j += 4)
+                *reinterpret_cast<float4*>(dst + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+            }
+          }
+        }
+        tc_fence_before();
+        __syncthreads();
+      }
+      near_done = true;
+    }
   }
-  if (n_blocks > 1) ev_staged = false;  // the staged rows were replaced by later blocks
-  // normalise: O = acc / den
-  for (int i = tid; i < Tt * HPC; i += NT) lrun[i] = 1.f / lrun[i];
-  __syncthreads();
-  for (int r = warp; r < Tt; r += NW)
-    for (int c = lane; c < HS; c += 32) xs[r * XS + c] *= lrun[r * HPC + c / D];
-
+  if (!near_done) {  // on the CUDA cores, block by block
+    for (int bi = 0; bi < n_blocks; ++bi) {
+      if (bi > 0 && !mbar_wait_bounded(bar_kv, bi & 1, kMbarPollLimit, p.err)) s_bad = 1;
+      const long long bs = kv_start + static_cast<long long>(bi) * p.KB;
+      const long long be = bs + min(p.KB, kv_rows - bi * p.KB);  // exclusive
+      if (K <= 16)
+        near_block<Tin, D, 16>(qst, kb, vb, xs, mrun, lrun, rowB, HS, XS, HPC, G, g_lo, K, t0, Tt,
+                               bs, be, p.score_scale, h0, warp, lane);
+      else
+        near_block<Tin, D, 32>(qst, kb, vb, xs, mrun, lrun, rowB, HS, XS, HPC, G, g_lo, K, t0, Tt,
+                               bs, be, p.score_scale, h0, warp, lane);
+      __syncthreads();  // the block buffers are free again
+      if (bi + 1 < n_blocks) issue_block(bi + 1);
+    }
+    if (n_blocks > 1) ev_staged = false;  // the staged rows were replaced by later blocks
+    // normalise: O = acc / den
+    for (int i = tid; i < Tt * HPC; i += NT) lrun[i] = 1.f / lrun[i];
+    __syncthreads();
+    for (int r = warp; r < Tt; r += NW)
+      for (int c = lane; c < HS; c += 32) xs[r * XS + c] *= lrun[r * HPC + c / D];
+  }
 
   // ---- (C) far field carry-in (deterministic look-back), then the scan --
   // carry = INCL(end of previous group) or the state, folded with the
@@ -428,6 +651,8 @@ prefill_kernel(const PrefillParams p) {
         wait_flag(fl, p.spin_limit, p.err);
       }
     }
+    if (tid < kGroup - 1)
+      s_gpow[tid] = powf(gf, static_cast<float>(evictions(pos0 + (gstart + tid) * kTile, kTile)));
     __syncthreads();
     for (int idx = tid; idx < NG * D; idx += NT) {
       const int g = g_lo + idx / D, i = idx % D;
@@ -439,7 +664,7 @@ prefill_kernel(const PrefillParams p) {
 #pragma unroll
       for (int jj = 0; jj < kGroup - 1; ++jj)
         if (jj < n_prev)
-          acc = fmaf(powf(gf, static_cast<float>(evictions(pos0 + (gstart + jj) * kTile, kTile))), acc, terms[jj]);
+          acc = fmaf(s_gpow[jj], acc, terms[jj]);
       sst[idx] = acc;
     }
     __syncthreads();
@@ -603,12 +828,22 @@ prefill_kernel(const PrefillParams p) {
     const float* nrm = p.slot_norm + static_cast<size_t>(l) * kSlots;
     const float n0 = nrm[lane], n1 = nrm[lane + 32];
     for (int r = rank + p.CS * warp; r < Tt; r += p.CS * NW) {
+      // every rank's partials in flight at once, added in rank order
+      float v0[kMaxCluster], v1[kMaxCluster], vs[kMaxCluster];
+#pragma unroll
+      for (int q = 0; q < kMaxCluster; ++q) {
+        const bool in = q < p.CS;
+        const float* rp = cluster.map_shared_rank(part, in ? q : 0) + r * kPartStride;
+        v0[q] = in ? rp[lane] : 0.f;
+        v1[q] = in ? rp[lane + 32] : 0.f;
+        vs[q] = in ? rp[kSlots] : 0.f;
+      }
       float d0 = 0.f, d1 = 0.f, ss = 0.f;
-      for (int q = 0; q < p.CS; ++q) {
-        const float* rp = cluster.map_shared_rank(part, q) + r * kPartStride;
-        d0 += rp[lane];
-        d1 += rp[lane + 32];
-        ss += rp[kSlots];
+#pragma unroll
+      for (int q = 0; q < kMaxCluster; ++q) {
+        d0 += v0[q];
+        d1 += v1[q];
+        ss += vs[q];
       }
       const float nx = fmaxf(sqrtf(ss), kNormFloor);
       const float c0 = d0 / (nx * n0) * p.inv_temp;
@@ -663,6 +898,10 @@ prefill_kernel(const PrefillParams p) {
   }
   const float a_l = p.alpha_layer[l];
   const bool write_ok = !s_bad;
+  if (tid < kSeg) {
+    const int len = max(0, min(Tt, (tid + 1) * (kTile / kSeg)) - tid * (kTile / kSeg));
+    s_gseg[tid] = powf(ge, static_cast<float>(len));
+  }  // read after the first barrier of the chunk loop below
   float* out = p.out + (in_row0 + (t0 - pos0)) * p.H + rank * HS;
   for (int c = 0; c < nch; ++c) {
     const int buf = c & 1;
@@ -693,10 +932,7 @@ prefill_kernel(const PrefillParams p) {
     }
     __syncthreads();
     float f = fcar[e];
-    for (int s2 = 0; s2 < sg; ++s2) {
-      const int len = max(0, min(Tt, (s2 + 1) * (kTile / kSeg)) - s2 * (kTile / kSeg));
-      f = fmaf(powf(ge, static_cast<float>(len)), f, segc[s2 * kCW + cc]);
-    }
+    for (int s2 = 0; s2 < sg; ++s2) f = fmaf(s_gseg[s2], f, segc[s2 * kCW + cc]);
     // ring: sum of the 16 positions ending at r, from the x tile and the halo
     auto xat = [&](int r) -> float { return r >= 0 ? xs[r * XS + e] : halo[(r + kHalo) * HS + e]; };
     float rs = 0.f;
@@ -823,11 +1059,15 @@ int max_clusters_t(int cs, size_t smem) {
 // never drops below a third of the SM's shared memory, so at most two CTAs
 // share an SM and their tensor-memory allocations (256 columns each) always
 // fit at once.
-bool plan_prefill(int HPC, int D, int esz, int NGm, int K, size_t budget, PrefillPlan* out) {
+bool plan_prefill(int HPC, int D, int esz, int NGm, int K, size_t budget, bool tc,
+                  PrefillPlan* out) {
   const int HS = HPC * D, XS = HS + 4;
   if (HS % kBlk != 0) return false;
+  if (tc && (esz != 2 || K > kSpan - kTile)) return false;
   auto a16 = [](long long x) { return static_cast<int>((x + 15) & ~15LL); };
   PrefillPlan p;
+  std::memset(&p, 0, sizeof(p));
+  p.tc = tc ? 1 : 0;
   int off = 0;
   p.bars = off;                 off += 128;  // mbarriers and the tensor-memory address
   p.xs = off;                   off += a16(4LL * kTile * XS);
@@ -835,7 +1075,8 @@ bool plan_prefill(int HPC, int D, int esz, int NGm, int K, size_t budget, Prefil
   p.fcar = off;                 off += a16(4LL * HS);
   p.sst = off;                  off += a16(4LL * NGm * D);
   p.sagg = off;                 off += a16(4LL * NGm * D);
-  p.ml = off;                   off += a16(4LL * (2 * kTile * HPC + kSeg * kCW));
+  // epilogue carries, then (CUDA-core near field) running max / denominator
+  p.ml = off;                   off += a16(4LL * (kSeg * kCW + (tc ? 0 : 2 * kTile * HPC)));
   p.u0 = off;
   // pool phase: slot blocks, partials | sem chunk, x block | w block
   int q = off;
@@ -844,17 +1085,26 @@ bool plan_prefill(int HPC, int D, int esz, int NGm, int K, size_t budget, Prefil
   p.wts = q;
   p.semc = q;                   q += a16(2LL * kBlkBytes);
   const int pool_end = q;
-  // staging phase
   q = off;
-  p.qst = q;                    q += a16(static_cast<long long>(kTile) * HS * esz);
-  const int row_b = NGm * D * esz + 16;
-  const long long room = static_cast<long long>(budget) - q;
-  int kb_rows = static_cast<int>(room / (2LL * row_b));
-  kb_rows = std::min(kb_rows, kTile + K);
-  if (kb_rows < 32) return false;
-  p.KB = kb_rows;
-  p.kb = q;                     q += a16(static_cast<long long>(row_b) * kb_rows);
-  p.vb = q;                     q += a16(static_cast<long long>(row_b) * kb_rows);
+  if (tc) {
+    // near-field phase on the tensor cores: one query block, key and value
+    // blocks of every KV head of the CTA, the P block (hi, lo)
+    p.qa = q;                   q += a16(2LL * kTile * D);
+    p.kvp = q;                  q += a16(2LL * 2 * NGm * kSpan * D);
+    p.pa = q;                   q += a16(2LL * 2 * kTile * kSpan);
+    p.KB = kSpan;
+  } else {
+    // near-field phase on the CUDA cores: staged queries and key/value rows
+    p.qst = q;                  q += a16(static_cast<long long>(kTile) * HS * esz);
+    const int row_b = NGm * D * esz + 16;
+    const long long room = static_cast<long long>(budget) - q;
+    int kb_rows = static_cast<int>(room / (2LL * row_b));
+    kb_rows = std::min(kb_rows, kTile + K);
+    if (kb_rows < 32) return false;
+    p.KB = kb_rows;
+    p.kb = q;                   q += a16(static_cast<long long>(row_b) * kb_rows);
+    p.vb = q;                   q += a16(static_cast<long long>(row_b) * kb_rows);
+  }
   p.total = std::max(q, pool_end);
   p.total = std::max<int>(p.total, static_cast<int>((budget + 1024) / 3) + 1);
   if (static_cast<size_t>(p.total) > budget) return false;
