@@ -80,7 +80,7 @@ constexpr int kDecodeSmemBudget = 112 * 1024;  // keeps two decode CTAs per SM
 
 // Shared-memory plan of the prefill kernel (byte offsets).
 struct PrefillPlan {
-  int bars, xs, halo, fcar, sst, sagg, ml;  // persistent regions
+  int bars, xs, halo, fcar, sst, sagg, sega, ml;  // persistent regions
   int u0;                                   // start of the union below
   int tc;                                   // near field on the tensor cores (bf16, k <= 16)
   int qst, kb, vb;                          // near-field staging (phase 1, CUDA-core near field)

@@ -190,6 +190,7 @@ prefill_kernel(const PrefillParams p) {
   float* fcar = reinterpret_cast<float*>(smb + pl.fcar);  // [HS]     field carried in
   float* sst = reinterpret_cast<float*>(smb + pl.sst);    // [NGm][D] S carried in / at tile end
   float* sagg = reinterpret_cast<float*>(smb + pl.sagg);  // [NGm][D] this tile's S aggregate
+  float* segA = reinterpret_cast<float*>(smb + pl.sega);  // [nseg][NG*D] scan segment aggregates
   float* segc = reinterpret_cast<float*>(smb + pl.ml);    // [kSeg][kCW] epilogue carries
   float* mrun = segc + kSeg * kCW;                        // [T*HPC]  running max (CUDA-core near field)
   float* lrun = mrun + kTile * HPC;                       // [T*HPC]  running denominator
@@ -211,7 +212,7 @@ prefill_kernel(const PrefillParams p) {
   __shared__ long long s_pos;
   __shared__ int s_ok;
   __shared__ int s_bad;  // a staging wait ran out: skip global writes
-  __shared__ float s_gpow[kGroup];  // gamma_far^(evictions) of the group's earlier tiles
+  __shared__ float s_gpn[kTile + 1];  // gamma_far^n, n = 0 .. kTile
   __shared__ float s_gseg[kSeg];    // ema_gamma^(length) of the epilogue's token segments
 
   if (tid == 0) {
@@ -436,32 +437,34 @@ prefill_kernel(const PrefillParams p) {
   // staged span when the first block covers them; otherwise read them from
   // global memory.
   bool ev_staged = tc || p.KB >= Tt;
-  // Folds the keys that leave the window at tokens r_from .. Tt-1 into s
-  // (EWMA), calling visit(r, s) after every token; staged rows or global.
-  auto scan_evicted = [&](int gg, int i, int r_from, float s, auto&& visit) -> float {
+  // Folds the keys that leave the window at tokens r of [r_lo, r_hi) with
+  // r >= r_from into s (EWMA), calling visit(r, s) after every token; staged
+  // rows or global memory.
+  auto scan_evicted = [&](int gg, int i, int r_lo, int r_hi, int r_from, float s,
+                          auto&& visit) -> float {
     if (ev_staged && tc) {  // packed key block: span row r is position t0 - k + r
       const unsigned char* kg = kvp + gg * kvblk;
-      for (int r = 0; r < Tt; ++r) {
+      for (int r = r_lo; r < r_hi; ++r) {
         if (r >= r_from) s = ewma(gf, s, to_f32<Tin>(*reinterpret_cast<const Tin*>(kg + kv_off(r, i))));
         visit(r, s);
       }
     } else if (ev_staged) {
       const Tin* col = reinterpret_cast<const Tin*>(kb) + gg * D + i;
       const int pitch = rowB / ESZ;
-      for (int r = 0; r < Tt; ++r) {
+      for (int r = r_lo; r < r_hi; ++r) {
         if (r >= r_from) s = ewma(gf, s, to_f32<Tin>(col[r * pitch]));
         visit(r, s);
       }
     } else {
-      for (int r0 = 0; r0 < Tt; r0 += kEvChunk) {
+      for (int r0 = r_lo; r0 < r_hi; r0 += kEvChunk) {
         float ev[kEvChunk];
 #pragma unroll
         for (int u = 0; u < kEvChunk; ++u)
-          ev[u] = (r0 + u < Tt && r0 + u >= r_from) ? to_f32<Tin>(key_row(t0 + r0 + u - K, g_lo + gg)[i]) : 0.f;
+          ev[u] = (r0 + u < r_hi && r0 + u >= r_from) ? to_f32<Tin>(key_row(t0 + r0 + u - K, g_lo + gg)[i]) : 0.f;
 #pragma unroll
         for (int u = 0; u < kEvChunk; ++u) {
           const int r = r0 + u;
-          if (r < Tt) {
+          if (r < r_hi) {
             if (r >= r_from) s = ewma(gf, s, ev[u]);
             visit(r, s);
           }
@@ -471,12 +474,30 @@ prefill_kernel(const PrefillParams p) {
     return s;
   };
 
-  // ---- (A) far field: this tile's aggregate of the keys leaving the window
-  // (read straight from global memory, independent loads in flight).
+  // ---- (A) far field: this tile's aggregate of the keys leaving the window.
+  // The tile's tokens split into nseg (1, 2 or 4) segments per (KV head, dim)
+  // as the threads allow; each segment is folded from zero, then the
+  // segments are combined in order: fold(c, seg) = gamma^(evictions) c + agg.
   const int r_ev = static_cast<int>(max(0LL, min(static_cast<long long>(Tt), K - t0)));  // first token that evicts
-  for (int idx = tid; idx < NG * D; idx += NT) {
-    const int gg = idx / D, i = idx % D, g = g_lo + gg;
-    const float a = scan_evicted(gg, i, r_ev, 0.f, [](int, float) {});
+  const int ne = NG * D;
+  int nseg = 1;
+  while (nseg < 4 && ne * nseg * 2 <= NT) nseg *= 2;
+  const int seg_len = kTile / nseg;
+  auto seg_ev = [&](int sg) -> int {  // evicting tokens of segment sg
+    const int a = max(sg * seg_len, r_ev), b = min(Tt, (sg + 1) * seg_len);
+    return b > a ? b - a : 0;
+  };
+  if (tid <= kTile) s_gpn[tid] = powf(gf, static_cast<float>(tid));
+  if (tid < ne * nseg) {
+    const int elem = tid % ne, sg = tid / ne;
+    segA[sg * ne + elem] = scan_evicted(elem / D, elem % D, sg * seg_len, min(Tt, (sg + 1) * seg_len),
+                                        r_ev, 0.f, [](int, float) {});
+  }
+  __syncthreads();
+  for (int idx = tid; idx < ne; idx += NT) {
+    const int g = g_lo + idx / D, i = idx % D;
+    float a = 0.f;
+    for (int sg = 0; sg < nseg; ++sg) a = fmaf(s_gpn[seg_ev(sg)], a, segA[sg * ne + idx]);
     sagg[idx] = a;
     if (g >= own_lo && publish) agg_s[(ticket * nkv + g) * D + i] = a;
   }
@@ -651,8 +672,6 @@ prefill_kernel(const PrefillParams p) {
         wait_flag(fl, p.spin_limit, p.err);
       }
     }
-    if (tid < kGroup - 1)
-      s_gpow[tid] = powf(gf, static_cast<float>(evictions(pos0 + (gstart + tid) * kTile, kTile)));
     __syncthreads();
     for (int idx = tid; idx < NG * D; idx += NT) {
       const int g = g_lo + idx / D, i = idx % D;
@@ -664,12 +683,12 @@ prefill_kernel(const PrefillParams p) {
 #pragma unroll
       for (int jj = 0; jj < kGroup - 1; ++jj)
         if (jj < n_prev)
-          acc = fmaf(s_gpow[jj], acc, terms[jj]);
+          acc = fmaf(s_gpn[evictions(pos0 + (gstart + jj) * kTile, kTile)], acc, terms[jj]);
       sst[idx] = acc;
     }
     __syncthreads();
     if (group_end && publish) {
-      const float mul = powf(gf, static_cast<float>(evictions(t0, Tt)));
+      const float mul = s_gpn[evictions(t0, Tt)];
       for (int idx = tid; idx < NG * D; idx += NT) {
         const int g = g_lo + idx / D, i = idx % D;
         if (g >= own_lo) incl_s[(ticket * nkv + g) * D + i] = fmaf(mul, sst[idx], sagg[idx]);
@@ -681,18 +700,24 @@ prefill_kernel(const PrefillParams p) {
       }
     }
   }
-  // scan: S_t per token, x = O_near + alpha_far * S_t  [P1 §2.1 eq. O]
-  for (int idx = tid; idx < NG * D; idx += NT) {
-    const int gg = idx / D, i = idx % D, g = g_lo + gg;
+  // scan: S_t per token, x = O_near + alpha_far * S_t  [P1 §2.1 eq. O];
+  // segment sg starts from the carry folded with the earlier segments'
+  // aggregates.  The last segment leaves S at the tile end in its own
+  // segA entry, which no other thread reads.
+  if (tid < ne * nseg) {
+    const int elem = tid % ne, sg = tid / ne;
+    const int gg = elem / D, i = elem % D, g = g_lo + gg;
     const int hh_lo = max(0, g * G - h0), hh_hi = min(HPC, (g + 1) * G - h0);
-    (void)g;
-    const float s = scan_evicted(gg, i, r_ev, sst[idx], [&](int r, float sv) {
-      for (int hh = hh_lo; hh < hh_hi; ++hh) {
-        float* xp = xs + r * XS + hh * D + i;
-        *xp = fmaf(p.alpha_far, sv, *xp);
-      }
-    });
-    sst[idx] = s;  // S at the end of the tile
+    float c = sst[elem];
+    for (int s2 = 0; s2 < sg; ++s2) c = fmaf(s_gpn[seg_ev(s2)], c, segA[s2 * ne + elem]);
+    c = scan_evicted(gg, i, sg * seg_len, min(Tt, (sg + 1) * seg_len), r_ev, c,
+                     [&](int r, float sv) {
+                       for (int hh = hh_lo; hh < hh_hi; ++hh) {
+                         float* xp = xs + r * XS + hh * D + i;
+                         *xp = fmaf(p.alpha_far, sv, *xp);
+                       }
+                     });
+    if (sg == nseg - 1) segA[sg * ne + elem] = c;
   }
   __syncthreads();
   // Slot blocks (bf16 hi/lo, laid out for both pool MMAs); the staging
@@ -970,7 +995,7 @@ prefill_kernel(const PrefillParams p) {
   if (last && write_ok) {
     for (int idx = tid; idx < NG * D; idx += NT) {
       const int g = g_lo + idx / D, i = idx % D;
-      if (g >= own_lo) far[g * D + i] = sst[idx];
+      if (g >= own_lo) far[g * D + i] = segA[(nseg - 1) * ne + idx];  // S at the tile end
     }
     if (own_lo <= g_hi) {
       const long long t_end = pos0 + p.n - 1;
@@ -1075,6 +1100,7 @@ bool plan_prefill(int HPC, int D, int esz, int NGm, int K, size_t budget, bool t
   p.fcar = off;                 off += a16(4LL * HS);
   p.sst = off;                  off += a16(4LL * NGm * D);
   p.sagg = off;                 off += a16(4LL * NGm * D);
+  p.sega = off;                 off += a16(4LL * NT);   // far-field scan segments
   // epilogue carries, then (CUDA-core near field) running max / denominator
   p.ml = off;                   off += a16(4LL * (kSeg * kCW + (tc ? 0 : 2 * kTile * HPC)));
   p.u0 = off;
