@@ -39,6 +39,9 @@ struct sfa_handle {
   unsigned spin_limit;
   long long withhold_tile;
   bool force_simt_near;  // test hook: CUDA-core near field even where the tensor-core one applies
+  bool tile_ok;          // the batch-tiled decode fits this configuration
+  int tile_smem;         // its dynamic shared memory per CTA
+  int tile_mode;         // -1: by batch size; 0: never; 1: always (test hook)
 };
 
 namespace {
@@ -151,7 +154,7 @@ void fill_common(P& p, const sfa_handle* h, int batch, void* state) {
   p.state = static_cast<unsigned char*>(state);
   p.slots = h->slots;
   p.slot_norm = h->slot_norm;
-  if constexpr (std::is_same<P, PrefillParams>::value) p.slot_img = h->slot_img;
+  p.slot_img = h->slot_img;
   p.alpha_layer = h->alpha_layer;
   p.err = h->err;
   p.cfg_hash = h->cfg_hash;
@@ -253,6 +256,10 @@ int sfa_init(const sfa_config* cfg, sfa_handle** out) {
   {
     const char* env = std::getenv("SFA_CUDA_CORE_NEAR_FIELD");
     h->force_simt_near = env != nullptr && env[0] == '1';
+    // SFA_DECODE_TILE=0 / 1 turns the batch-tiled decode off / on for every
+    // batch size (default: from kDecodeTileMinSeqs sequences per call).
+    const char* tenv = std::getenv("SFA_DECODE_TILE");
+    h->tile_mode = (tenv && tenv[0] == '0') ? 0 : (tenv && tenv[0] == '1') ? 1 : -1;
   }
   const int L = cfg->n_layers, H = hidden_of(cfg);
   const size_t slot_bytes = sizeof(float) * static_cast<size_t>(L) * kSlots * H;
@@ -266,6 +273,7 @@ int sfa_init(const sfa_config* cfg, sfa_handle** out) {
   if (e == cudaSuccess) e = cudaMemset(h->err, 0, sizeof(int));
   if (e == cudaSuccess) e = prefill_prepare(h->device);
   if (e == cudaSuccess) e = decode_prepare(h->device);
+  if (e == cudaSuccess) e = decode_tile_prepare(h->device);
   if (e == cudaSuccess) {
     // First cluster size for which both kernels have a shared-memory plan
     // and at least one cluster fits on the device.
@@ -290,6 +298,10 @@ int sfa_init(const sfa_config* cfg, sfa_handle** out) {
       h->prefill_cs = cs;
       h->plan = plan;
       h->decode_budget = decode_budget(limit);
+      const size_t tsm = decode_tile_smem_bytes(hpc, cfg->head_dim, limit);
+      h->tile_smem = static_cast<int>(tsm);
+      h->tile_ok = tsm <= limit &&
+                   decode_tile_max_active_clusters(cs, tsm, cfg->in_dtype, cfg->head_dim) >= 1;
       break;
     }
     if (h->prefill_cs == 0) e = cudaErrorInvalidConfiguration;
@@ -472,7 +484,16 @@ int sfa_decode_step_ex(const sfa_handle* h, int layer_begin, int layer_count, co
   p.HPC = c->n_q_heads / p.CS;
   p.NGm = max_kv_heads_per_cta(c->n_q_heads, c->n_kv_heads, p.CS);
   p.smem_budget = h->decode_budget;
-  return cuda_status(launch_decode(p, c->in_dtype, c->head_dim, static_cast<cudaStream_t>(stream)));
+  p.tile_smem = h->tile_smem;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // Batch-tiled decode from kDecodeTileMinSeqs sequences with windows of at
+  // most kDecodeTileMaxWindow positions (longer windows: each warp walks its
+  // window serially and the per-stream kernel, which splits it, is faster).
+  const bool tile = h->tile_ok &&
+                    (h->tile_mode == 1 || (h->tile_mode < 0 && n_seq >= kDecodeTileMinSeqs &&
+                                           c->window_k <= kDecodeTileMaxWindow));
+  if (tile) return cuda_status(launch_decode_tile(p, c->in_dtype, c->head_dim, s));
+  return cuda_status(launch_decode(p, c->in_dtype, c->head_dim, s));
 }
 
 int sfa_check_device_status(const sfa_handle* h, void* stream) {

@@ -30,6 +30,9 @@ constexpr int kTile = 64;                 // tokens per prefill tile
 constexpr int kHalo = kRing - 1;          // x rows a tile needs from before it
 constexpr int kPrefillThreads = 256;
 constexpr int kDecodeThreads = 256;
+constexpr int kDecodeTileThreads = 256;     // batch-tiled decode (64 sequences per tile)
+constexpr int kDecodeTileMinSeqs = 64;      // batch-tiled decode from this many sequences per call
+constexpr int kDecodeTileMaxWindow = 64;    // ... and windows of at most this many positions
 constexpr int kGroup = 16;                // tiles per look-back group
 
 // Look-back flag values.
@@ -64,6 +67,7 @@ struct DecodeParams {
   const float* slots;       // [L][64][H]
   const float* slot_norm;   // [L][64], clamped at kNormFloor
   const float* alpha_layer; // [L]
+  const unsigned char* slot_img;  // pre-split bf16 slot blocks (batch-tiled decode)
   int* err;
   uint64_t cfg_hash;
   StreamOffsets so;
@@ -73,6 +77,7 @@ struct DecodeParams {
   int n_seq;
   int NGm;          // most KV heads any CTA needs
   int smem_budget;  // shared-memory bytes the plan may use (window staged if it fits)
+  int tile_smem;    // dynamic shared memory of the batch-tiled decode
   float gamma_far, alpha_far, ema_gamma, inv_temp, clip_eps, score_scale;
 };
 
@@ -130,6 +135,10 @@ inline long long align256(long long x) { return (x + 255) & ~255LL; }
 
 // Launchers (return the CUDA error of the launch).
 cudaError_t launch_decode(const DecodeParams& p, int in_dtype, int head_dim, cudaStream_t s);
+cudaError_t launch_decode_tile(const DecodeParams& p, int in_dtype, int head_dim, cudaStream_t s);
+cudaError_t decode_tile_prepare(int device);
+size_t decode_tile_smem_bytes(int HPC, int head_dim, size_t limit);
+int decode_tile_max_active_clusters(int cs, size_t smem, int in_dtype, int head_dim);
 cudaError_t launch_prefill(const PrefillParams& p, int in_dtype, int head_dim, cudaStream_t s);
 bool plan_prefill(int HPC, int D, int esz, int NGm, int K, size_t budget, bool tc, PrefillPlan* out);
 cudaError_t prefill_prepare(int device);

@@ -119,3 +119,30 @@ def test_cuda_core_near_field_on_bf16_inputs(monkeypatch):
     w = _tiny_variant(name="cuda_core_near_bf16", n_layers=2, batch=2, n_q_heads=14,
                       n_kv_heads=2, head_dim=64, window_k=16, in_dtype="bf16")
     _run_schedule(w, [("p", 130), ("d", 5), ("p", 70)])
+
+
+@pytest.mark.parametrize("name,over,schedule",
+                         [e for e in EDGE if e[0] in ("gqa_f32_d64", "mha_k1", "k256_spans_tiles",
+                                                      "d128_f32_multilayer", "gqa7_bf16",
+                                                      "decode_from_empty", "eight_heads_per_cta")],
+                         ids=lambda x: x if isinstance(x, str) else "")
+def test_batch_tiled_decode_on_edge_schedules(monkeypatch, name, over, schedule):
+    """The batch-tiled decode (64 sequences per cluster, pool on the tensor
+    cores) serves every batch when SFA_DECODE_TILE=1; same bar as above."""
+    monkeypatch.setenv("SFA_DECODE_TILE", "1")
+    w = _tiny_variant(name=name + "_tiled", **over)
+    _run_schedule(w, schedule)
+
+
+def test_batch_tiled_decode_partial_tile_and_sequence_list(monkeypatch):
+    """70 sequences (a full and a partial tile), then a permuted subset."""
+    w = _tiny_variant(name="tiled_70", n_layers=2, batch=70, n_q_heads=14, n_kv_heads=2,
+                      head_dim=64, window_k=16, in_dtype="bf16")
+    pair = Pair(w, seqs=[0, 1, 63, 64, 69])
+    tol = TOL[w.in_dtype]
+    got, ref = pair.prefill(20)
+    assert_close(got, ref, tol, "prefill")
+    got, ref = pair.decode_many(6)  # 70 >= 64 sequences: the batch-tiled decode
+    assert_close(got, ref, tol, "tiled decode")
+    assert pair.status() == 0
+    pair.compare_state(tol)
