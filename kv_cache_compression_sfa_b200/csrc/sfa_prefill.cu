@@ -387,31 +387,34 @@ prefill_kernel(const PrefillParams p) {
   };
   if constexpr (ESZ == 2) {
     if (tc) {
-      {
-        uint4 qv[kQChunks];
-        q_load(0, qv);
-        q_store(qv);
-      }
-      // key and value rows of the span (positions t0-16 .. t0+63) for every
-      // KV head of the CTA, packed for the MMAs; rows before position 0 or
-      // past the tile are zero.  Four 16-byte loads in flight per thread.
+      // Head 0's query block and the key and value rows of the span
+      // (positions t0-16 .. t0+63) for every KV head of the CTA, packed for
+      // the MMAs; rows before position 0 or past the tile are zero.  One
+      // pass of 16-byte loads, eight in flight per thread.
       constexpr int D8 = D / 8;
       const int per = kSpan * D8;
-      const int total = 2 * NG * per;
-      for (int b0 = 0; b0 < total; b0 += 4 * NT) {
-        uint4 val[4];
-        int dst[4];
+      const int nq_chunks = kTile * D8;
+      const int total = nq_chunks + 2 * NG * per;
+      for (int b0 = 0; b0 < total; b0 += 8 * NT) {
+        uint4 val[8];
+        int dst[8];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < 8; ++u) {
           const int idx = b0 + u * NT + tid;
           val[u] = make_uint4(0u, 0u, 0u, 0u);
           dst[u] = -1;
-          if (idx < total) {
-            const int which = idx / (NG * per), rem = idx % (NG * per);
+          if (idx < nq_chunks) {
+            const int d8 = idx / kTile, r = idx % kTile;
+            dst[u] = pl.qa + blk_off(r, d8 * 8);  // offsets from the shared-memory base
+            if (r < Tt)
+              val[u] = *reinterpret_cast<const uint4*>(qin + ((t0 - pos0 + r) * p.nq + h0) * D + d8 * 8);
+          } else if (idx < total) {
+            const int kvi = idx - nq_chunks;
+            const int which = kvi / (NG * per), rem = kvi % (NG * per);
             const int gg = rem / per, r2 = rem % per;
             const int d8 = r2 / kSpan, c = r2 % kSpan;
             const long long j = kv_start + c;
-            dst[u] = (which * p.NGm + gg) * kvblk + kv_off(c, d8 * 8);
+            dst[u] = pl.kvp + (which * p.NGm + gg) * kvblk + kv_off(c, d8 * 8);
             if (j >= 0 && c < kv_rows) {
               const Tin* row = which ? val_row(j, g_lo + gg) : key_row(j, g_lo + gg);
               val[u] = *reinterpret_cast<const uint4*>(row + d8 * 8);
@@ -419,8 +422,8 @@ prefill_kernel(const PrefillParams p) {
           }
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-          if (dst[u] >= 0) *reinterpret_cast<uint4*>(kvp + dst[u]) = val[u];
+        for (int u = 0; u < 8; ++u)
+          if (dst[u] >= 0) *reinterpret_cast<uint4*>(smb + dst[u]) = val[u];
       }
       for (int i = tid; i < 2 * kTile * kSpan * 2 / 16; i += NT)  // P blocks start at zero
         reinterpret_cast<uint4*>(pa)[i] = make_uint4(0u, 0u, 0u, 0u);
@@ -433,6 +436,7 @@ prefill_kernel(const PrefillParams p) {
     }
   for (int i = tid; i < kTile * XS; i += NT) xs[i] = 0.f;
   if (!mbar_wait_bounded(bar_kv, 0, kMbarPollLimit, p.err)) s_bad = 1;
+  __syncthreads();  // the packed blocks and zeroed rows written above are read by other threads
   // Keys that leave the window at the tile's tokens are rows 0 .. Tt-1 of the
   // staged span when the first block covers them; otherwise read them from
   // global memory.
