@@ -23,6 +23,14 @@ __device__ __forceinline__ float warp_max(float v) {
   return v;
 }
 
+// Maximum over the full warp in one instruction (sm_100a float redux);
+// every lane must take part.
+__device__ __forceinline__ float warp_max_redux(float v) {
+  float r;
+  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+  return r;
+}
+
 // First error wins; later errors are dropped until the host clears the word.
 __device__ __forceinline__ void latch_error(int* err, int code) { atomicCAS(err, 0, code); }
 

@@ -219,10 +219,7 @@ decode_tile_kernel(const DecodeParams p) {
 #pragma unroll
         for (int off = 1; off < LPK; off <<= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
         s = (key < cnt) ? s * p.score_scale : -INFINITY;
-        float mx = s;
-#pragma unroll
-        for (int off = 16; off >= LPK; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-        const float mn = fmaxf(m, mx);
+        const float mn = fmaxf(m, warp_max_redux(s));
         const float corr = expf(m - mn);
         const float pj = (key < cnt) ? expf(s - mn) : 0.f;
         float ps = pj;
@@ -334,7 +331,7 @@ decode_tile_kernel(const DecodeParams p) {
       const float nx = fmaxf(sqrtf(ss), kNormFloor);
       const float c0 = d0 / (nx * n0) * p.inv_temp;
       const float c1 = d1 / (nx * n1) * p.inv_temp;
-      const float mx = warp_max(fmaxf(c0, c1));
+      const float mx = warp_max_redux(fmaxf(c0, c1));
       const float e0 = expf(c0 - mx), e1 = expf(c1 - mx);
       const float inv = 1.f / warp_sum(e0 + e1);
       __nv_bfloat16 hb0, lb0, hb1, lb1;

@@ -877,7 +877,7 @@ prefill_kernel(const PrefillParams p) {
       const float nx = fmaxf(sqrtf(ss), kNormFloor);
       const float c0 = d0 / (nx * n0) * p.inv_temp;
       const float c1 = d1 / (nx * n1) * p.inv_temp;
-      const float mx = warp_max(fmaxf(c0, c1));
+      const float mx = warp_max_redux(fmaxf(c0, c1));
       const float e0 = expf(c0 - mx), e1 = expf(c1 - mx);
       const float inv = 1.f / warp_sum(e0 + e1);
       __nv_bfloat16 h0, l0, h1, l1;
