@@ -139,9 +139,11 @@ SFA_API int sfa_destroy(sfa_handle* h);
 /* Bytes of a state buffer for `batch` sequences; 0 on invalid input. */
 SFA_API size_t sfa_state_bytes(const sfa_handle* h, int batch);
 
-/* Bytes of prefill workspace for a call of n tokens x `batch`; 0 when the
- * call needs none or on invalid input.  The workspace holds the cross-tile
- * carries of the parallel scans; its content need not be initialised. */
+/* Bytes of prefill workspace for a call of n tokens x `batch`; 0 on invalid
+ * input.  The workspace holds each stream's position at the start of the
+ * call, the far-field state at its end and the pool weights of every
+ * 64-token tile (16 KB per tile and stream); its content need not be
+ * initialised. */
 SFA_API size_t sfa_prefill_workspace_bytes(const sfa_handle* h, int batch, long long n);
 
 /* Zeroes `state` (state_bytes(h, batch) bytes) and writes its header for
@@ -220,9 +222,9 @@ SFA_API int sfa_abi_version(void);
  * the process exits; nothing is allocated or freed.  The first call on a
  * device looks up the array's device address (with that device current)
  * and caches it, so make that first call before any stream capture.  Every
- * call on a device shares the array: the parts that must start at zero are
- * cleared on `stream` by each call, and calls that overlap on the GPU (other
- * streams, other host threads) race on it.  Returns SFA_ERR_WORKSPACE when
+ * call on a device shares the array, which keeps the last call's contents
+ * (nothing in it has to start at zero), and calls that overlap on the GPU
+ * (other streams, other host threads) race on it.  Returns SFA_ERR_WORKSPACE when
  * sfa_prefill_workspace_bytes(h, batch, n) exceeds the array (split the
  * prefill into smaller chunks), otherwise exactly what sfa_prefill returns;
  * results equal sfa_prefill's. */
@@ -230,11 +232,12 @@ SFA_API int sfa_prefill_static_ws(const sfa_handle* h, const void* q, const void
                                   long long n, int batch, void* state, float* out, void* stream);
 
 /* Test hook for the device-side bounded waits of sfa_prefill (not needed in
- * normal use).  spin_limit: maximum polls of a look-back flag before the
- * wait gives up and latches SFA_ERR_DEVICE_TIMEOUT (0 restores the default).
- * withhold_tile: a tile index whose cross-tile publications are skipped, so
- * that its successors' waits run out (-1 disables).  Affects later calls on
- * this handle only. */
+ * normal use).  withhold_tile: tile index (tile * streams + stream, streams =
+ * layers x batch of the call) whose pool-weight CTA waits on a barrier that
+ * nothing completes (-1 disables); spin_limit: polls before that wait gives
+ * up and latches SFA_ERR_DEVICE_TIMEOUT (0 restores the default).  The
+ * kernel still finishes and the context stays usable.  Affects later calls
+ * on this handle only. */
 SFA_API int sfa_debug_set_lookback(sfa_handle* h, unsigned int spin_limit, long long withhold_tile);
 
 #ifdef __cplusplus

@@ -33,12 +33,11 @@ struct sfa_handle {
   unsigned char* slot_img;  // [L][H/64][hi, lo] bf16 blocks for the prefill pool MMAs
   int* err;              // device error word
   uint64_t cfg_hash;
-  int prefill_cs;
-  PrefillPlan plan;
+  int cs;               // CTAs per cluster of the decode kernels
+  NearPlan near;         // shared-memory plan of the prefill near-field kernel
   int decode_budget;
   unsigned spin_limit;
   long long withhold_tile;
-  bool force_simt_near;  // test hook: CUDA-core near field even where the tensor-core one applies
   bool tile_ok;          // the batch-tiled decode fits this configuration
   int tile_smem;         // its dynamic shared memory per CTA
   int tile_mode;         // -1: by batch size; 0: never; 1: always (test hook)
@@ -47,6 +46,7 @@ struct sfa_handle {
 namespace {
 
 constexpr uint32_t kHandleMagic = 0x48414653u;  // "SFAH"
+constexpr long long kBlkBytesHost = 64 * 64 * 2;  // one 64 x 64 bf16 block
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -109,23 +109,17 @@ std::vector<int> cluster_candidates(int nq, int d) {
   return out;
 }
 
-PrefillWorkspace prefill_workspace(const sfa_config* c, int cs, int layers, int batch, long long n) {
+// Workspace of a prefill call: the streams' positions, S at the end of the
+// call and the pool weights of every tile (two 8 KB bf16 blocks).
+PrefillWorkspace prefill_workspace(const sfa_config* c, int layers, int batch, long long n) {
   PrefillWorkspace w;
   const long long streams = static_cast<long long>(layers) * batch;
   const long long tiles = streams * ((n + kTile - 1) / kTile);
-  const long long H = hidden_of(c);
   const long long sdim = static_cast<long long>(c->n_kv_heads) * c->head_dim;
-  w.fs_agg = 256;  // [0, 256): ticket counter
-  w.fs_incl = w.fs_agg + align256(4 * tiles * c->n_kv_heads);
-  w.ff_agg = w.fs_incl + align256(4 * tiles * c->n_kv_heads);
-  w.ff_incl = w.ff_agg + align256(4 * tiles * cs);
-  w.flags_end = w.ff_incl + align256(4 * tiles * cs);
-  w.agg_s = w.flags_end;
-  w.incl_s = w.agg_s + align256(4 * tiles * sdim);
-  w.agg_f = w.incl_s + align256(4 * tiles * sdim);
-  w.incl_f = w.agg_f + align256(4 * tiles * H);
-  w.halo = w.incl_f + align256(4 * tiles * H);
-  w.total = w.halo + align256(4 * tiles * kHalo * H);
+  w.pos = 0;
+  w.sfin = align256(8 * streams);
+  w.w = w.sfin + align256(4 * streams * sdim);
+  w.total = w.w + tiles * 2LL * kBlkBytesHost;
   return w;
 }
 
@@ -247,17 +241,13 @@ int sfa_init(const sfa_config* cfg, sfa_handle** out) {
   h->magic = kHandleMagic;
   h->cfg = *cfg;
   h->cfg_hash = config_hash(cfg);
-  h->prefill_cs = 0;
+  h->cs = 0;
   h->spin_limit = kDefaultSpinLimit;
   h->withhold_tile = -1;
-  // Test hook (environment, read once per handle): SFA_CUDA_CORE_NEAR_FIELD=1
-  // keeps the prefill near field on the CUDA cores, so both paths can be
-  // checked against the oracle on the same workload.
   {
-    const char* env = std::getenv("SFA_CUDA_CORE_NEAR_FIELD");
-    h->force_simt_near = env != nullptr && env[0] == '1';
-    // SFA_DECODE_TILE=0 / 1 turns the batch-tiled decode off / on for every
-    // batch size (default: from kDecodeTileMinSeqs sequences per call).
+    // Test hook (environment, read once per handle): SFA_DECODE_TILE=0 / 1
+    // turns the batch-tiled decode off / on for every batch size (default:
+    // from kDecodeTileMinSeqs sequences per call).
     const char* tenv = std::getenv("SFA_DECODE_TILE");
     h->tile_mode = (tenv && tenv[0] == '0') ? 0 : (tenv && tenv[0] == '1') ? 1 : -1;
   }
@@ -275,28 +265,30 @@ int sfa_init(const sfa_config* cfg, sfa_handle** out) {
   if (e == cudaSuccess) e = decode_prepare(h->device);
   if (e == cudaSuccess) e = decode_tile_prepare(h->device);
   if (e == cudaSuccess) {
-    // First cluster size for which both kernels have a shared-memory plan
-    // and at least one cluster fits on the device.
+    // Prefill near-field plan; the decode kernels' cluster size: the first
+    // candidate whose decode plan fits and of which one cluster fits on the
+    // device.
     const size_t limit = prefill_smem_limit(h->device);
+    const int esz = static_cast<int>(in_bytes(cfg->in_dtype));
+    // Test hook (environment, read once per handle): SFA_CUDA_CORE_NEAR_FIELD=1
+    // keeps the prefill near field on the CUDA cores where the tensor-core
+    // one applies (bf16, k <= 16), so both can be checked on one workload.
+    const char* nenv = std::getenv("SFA_CUDA_CORE_NEAR_FIELD");
+    const bool tc = !(nenv && nenv[0] == '1');
+    if (!(tc && plan_near(cfg->head_dim, esz, cfg->window_k, limit, true, &h->near)) &&
+        !plan_near(cfg->head_dim, esz, cfg->window_k, limit, false, &h->near))
+      e = cudaErrorInvalidConfiguration;
+    if (static_cast<size_t>(std::max(prefill_pool_smem(), prefill_out_smem())) > limit)
+      e = cudaErrorInvalidConfiguration;
     for (int cs : cluster_candidates(cfg->n_q_heads, cfg->head_dim)) {
+      if (e != cudaSuccess) break;
       const int hpc = cfg->n_q_heads / cs;
-      PrefillPlan plan;
-      const int ngm = max_kv_heads_per_cta(cfg->n_q_heads, cfg->n_kv_heads, cs);
-      const int esz = static_cast<int>(in_bytes(cfg->in_dtype));
-      // tensor-core near field for bf16 inputs and windows of at most 16
-      // positions, else the CUDA-core one
-      const bool tc = cfg->in_dtype == SFA_BF16 && cfg->window_k <= 16 && !h->force_simt_near;
-      if (!(tc && plan_prefill(hpc, cfg->head_dim, esz, ngm, cfg->window_k, limit, true, &plan)) &&
-          !plan_prefill(hpc, cfg->head_dim, esz, ngm, cfg->window_k, limit, false, &plan))
-        continue;
-      const size_t dsm = decode_smem_bytes(hpc, cfg->head_dim, static_cast<int>(in_bytes(cfg->in_dtype)),
+      const size_t dsm = decode_smem_bytes(hpc, cfg->head_dim, esz,
                                            max_kv_heads_per_cta(cfg->n_q_heads, cfg->n_kv_heads, cs),
                                            cfg->window_k, decode_budget(limit));
       if (dsm > limit) continue;
-      if (prefill_max_active_clusters(cs, plan.total, cfg->in_dtype, cfg->head_dim) < 1) continue;
       if (decode_max_active_clusters(cs, dsm, cfg->in_dtype, cfg->head_dim) < 1) continue;
-      h->prefill_cs = cs;
-      h->plan = plan;
+      h->cs = cs;
       h->decode_budget = decode_budget(limit);
       const size_t tsm = decode_tile_smem_bytes(hpc, cfg->head_dim, limit);
       h->tile_smem = static_cast<int>(tsm);
@@ -304,7 +296,7 @@ int sfa_init(const sfa_config* cfg, sfa_handle** out) {
                    decode_tile_max_active_clusters(cs, tsm, cfg->in_dtype, cfg->head_dim) >= 1;
       break;
     }
-    if (h->prefill_cs == 0) e = cudaErrorInvalidConfiguration;
+    if (e == cudaSuccess && h->cs == 0) e = cudaErrorInvalidConfiguration;
   }
   if (e == cudaSuccess) e = launch_slot_norms(h->slots, h->slot_norm, L, H, nullptr);
   if (e == cudaSuccess) e = launch_slot_image(h->slots, h->slot_img, L, H, nullptr);
@@ -366,8 +358,7 @@ size_t sfa_prefill_layers_workspace_bytes(const sfa_handle* h, int layer_count, 
   if (!handle_ok(h) || batch <= 0 || n <= 0 || layer_count <= 0 ||
       layer_count > h->cfg.n_layers)
     return 0;
-  return static_cast<size_t>(
-      prefill_workspace(&h->cfg, h->prefill_cs, layer_count, batch, n).total);
+  return static_cast<size_t>(prefill_workspace(&h->cfg, layer_count, batch, n).total);
 }
 
 int sfa_state_reset(const sfa_handle* h, void* state, int batch, void* stream) {
@@ -408,15 +399,12 @@ int sfa_prefill_layers(const sfa_handle* h, int layer_begin, int layer_count, co
       !aligned16(workspace))
     return SFA_ERR_ALIGNMENT;
   const sfa_config* c = &h->cfg;
-  const PrefillWorkspace w = prefill_workspace(c, h->prefill_cs, layer_count, batch, n);
+  const PrefillWorkspace w = prefill_workspace(c, layer_count, batch, n);
   if (!workspace || workspace_bytes < static_cast<size_t>(w.total)) return SFA_ERR_WORKSPACE;
   const long long streams = static_cast<long long>(layer_count) * batch;
   const long long tiles_per_stream = (n + kTile - 1) / kTile;
-  if (streams * tiles_per_stream * h->prefill_cs > 0x7fffffffLL) return SFA_ERR_UNSUPPORTED;
+  if (streams > 65535 || tiles_per_stream > 0x7fffffffLL) return SFA_ERR_UNSUPPORTED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // Ticket counter and look-back flags start empty on every call.
-  cudaError_t e = cudaMemsetAsync(workspace, 0, static_cast<size_t>(w.flags_end), s);
-  if (e != cudaSuccess) return SFA_ERR_CUDA;
   PrefillParams p;
   std::memset(&p, 0, sizeof(p));
   fill_common(p, h, batch, state);
@@ -427,27 +415,17 @@ int sfa_prefill_layers(const sfa_handle* h, int layer_begin, int layer_count, co
   p.ws = static_cast<unsigned char*>(workspace);
   p.n = n;
   p.l0 = layer_begin;
-  p.CS = h->prefill_cs;
-  p.HPC = c->n_q_heads / p.CS;
   p.tiles_per_stream = static_cast<int>(tiles_per_stream);
   p.n_streams = static_cast<int>(streams);
-  p.n_tiles = streams * tiles_per_stream;
-  p.NGm = max_kv_heads_per_cta(c->n_q_heads, c->n_kv_heads, p.CS);
-  p.plan = h->plan;
-  p.KB = h->plan.KB;
-  p.ws_fs_agg = w.fs_agg;
-  p.ws_fs_incl = w.fs_incl;
-  p.ws_ff_agg = w.ff_agg;
-  p.ws_ff_incl = w.ff_incl;
-  p.ws_agg_s = w.agg_s;
-  p.ws_incl_s = w.incl_s;
-  p.ws_agg_f = w.agg_f;
-  p.ws_incl_f = w.incl_f;
-  p.ws_halo = w.halo;
+  p.ws_pos = w.pos;
+  p.ws_sfin = w.sfin;
+  p.ws_w = w.w;
   p.spin_limit = h->spin_limit;
   p.withhold_tile = h->withhold_tile;
-  e = launch_prefill(p, c->in_dtype, c->head_dim, s);
-  return cuda_status(e);
+  p.near = h->near;
+  p.pool_smem = prefill_pool_smem();
+  p.out_smem = prefill_out_smem();
+  return cuda_status(launch_prefill(p, c->in_dtype, c->head_dim, s));
 }
 
 int sfa_decode_step(const sfa_handle* h, const void* q, const void* k, const void* v, int batch,
@@ -480,7 +458,7 @@ int sfa_decode_step_ex(const sfa_handle* h, int layer_begin, int layer_count, co
   p.k = k;
   p.v = v;
   p.out = out;
-  p.CS = h->prefill_cs;
+  p.CS = h->cs;
   p.HPC = c->n_q_heads / p.CS;
   p.NGm = max_kv_heads_per_cta(c->n_q_heads, c->n_kv_heads, p.CS);
   p.smem_budget = h->decode_budget;

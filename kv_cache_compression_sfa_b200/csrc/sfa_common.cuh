@@ -1,6 +1,6 @@
 // sfa_common.cuh — device helpers shared by the SFA kernels: vector loads of
-// the input dtype, warp reductions, the error latch and the acquire/release
-// flag accesses of the prefill look-back.
+// the input dtype, warp reductions, the error latch, mbarriers, bulk and
+// asynchronous copies, and programmatic dependent launch.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -126,33 +126,6 @@ __device__ __forceinline__ float to_f32<float>(float v) { return v; }
 template <>
 __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
 
-// gpu-scope acquire load / release store of a 32-bit look-back flag.
-__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
-  unsigned v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-__device__ __forceinline__ void st_release_u32(unsigned* p, unsigned v) {
-  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-// Polls a flag until it is non-empty, at most `limit` times.  A wait that
-// runs out latches SFA_ERR_DEVICE_TIMEOUT and reports kFlagIncl so that the
-// caller finishes its work (with invalid data) instead of hanging.
-__device__ __forceinline__ unsigned wait_flag(const unsigned* f, unsigned limit, int* err) {
-  unsigned v = ld_acquire_u32(f);
-  unsigned polls = 0;
-  while (v == kFlagEmpty) {
-    if (++polls > limit) {
-      latch_error(err, SFA_ERR_DEVICE_TIMEOUT);
-      return kFlagIncl;
-    }
-    __nanosleep(128);
-    v = ld_acquire_u32(f);
-  }
-  return v;
-}
-
 // ---- shared-memory addresses, mbarriers and 1-D bulk copies (TMA engine) --
 
 __device__ __forceinline__ unsigned smem_u32(const void* p) {
@@ -207,6 +180,18 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, unsigned by
           "r"(smem_u32(dst)),
       "l"(src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
+}
+
+// 16-byte global -> shared copy that bypasses the registers (and L1);
+// completion is tracked per thread by commit groups.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// Waits until at most N of this thread's commit groups are still in flight.
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 // Orders this thread's earlier generic-proxy shared-memory accesses before

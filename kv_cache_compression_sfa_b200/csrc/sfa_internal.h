@@ -27,19 +27,14 @@ constexpr float kNormFloor = 1e-12f;      // cosine norm clamp
 
 // Prefill tiling.
 constexpr int kTile = 64;                 // tokens per prefill tile
-constexpr int kHalo = kRing - 1;          // x rows a tile needs from before it
+constexpr int kHalo = kRing - 1;          // x rows a token needs from before its tile
 constexpr int kPrefillThreads = 256;
 constexpr int kDecodeThreads = 256;
 constexpr int kDecodeTileThreads = 256;     // batch-tiled decode (64 sequences per tile)
 constexpr int kDecodeTileMinSeqs = 64;      // batch-tiled decode from this many sequences per call
 constexpr int kDecodeTileMaxWindow = 64;    // ... and windows of at most this many positions
-constexpr int kGroup = 16;                // tiles per look-back group
 
-// Look-back flag values.
-constexpr unsigned kFlagEmpty = 0u;
-constexpr unsigned kFlagAgg = 1u;
-constexpr unsigned kFlagIncl = 2u;
-constexpr unsigned kDefaultSpinLimit = 1u << 21;
+constexpr unsigned kDefaultSpinLimit = 1u << 21;  // polls of a bounded wait
 
 // First bytes of every state buffer.
 struct StateHeader {
@@ -83,15 +78,17 @@ struct DecodeParams {
 
 constexpr int kDecodeSmemBudget = 112 * 1024;  // keeps two decode CTAs per SM
 
-// Shared-memory plan of the prefill kernel (byte offsets).
-struct PrefillPlan {
-  int bars, xs, halo, fcar, sst, sagg, sega, ml;  // persistent regions
-  int u0;                                   // start of the union below
-  int tc;                                   // near field on the tensor cores (bf16, k <= 16)
-  int qst, kb, vb;                          // near-field staging (phase 1, CUDA-core near field)
-  int qa, kvp, pa;                          // near-field MMA operands (phase 1, tensor-core near field)
-  int sl, part, wts, semc;                  // pool buffers (phase 2)
-  int KB;                                   // rows per staged key/value block
+// Shared-memory plan of the prefill near-field kernel (byte offsets).  Each
+// stage holds one tile's queries of one head and the keys and values of its
+// span (positions t0-k .. t0+T-1), rows padded by 16 bytes.
+struct NearPlan {
+  int tc;                 // near field on the tensor cores (bf16 inputs, k <= 16)
+  int stages;             // 2 or 1 staged buffers; 0: keys and values read from global memory
+  int row;                // CUDA cores: padded bytes of one staged row
+  int q[2], k[2], v[2];   // stage offsets (tensor cores: MMA operand blocks)
+  int pa;                 // tensor cores: P blocks (hi, lo)
+  int ga;                 // tensor cores: far-field weight blocks G (hi, lo)
+  int xs;                 // CUDA cores: x tile [kTile][D + 4] fp32
   int total;
 };
 
@@ -110,25 +107,24 @@ struct PrefillParams {
   uint64_t cfg_hash;
   StreamOffsets so;
   long long n;              // tokens per stream in this call
-  int L, B, nq, nkv, K, H, G, CS, HPC;
+  int L, B, nq, nkv, K, H, G;
   int l0;                   // first layer of the state served (streams are l0*B + ...)
-  int NGm;                  // most KV heads any CTA needs
-  int KB;                   // rows per staged key/value block
   int tiles_per_stream, n_streams;
-  long long n_tiles;
-  // workspace byte offsets
-  long long ws_fs_agg, ws_fs_incl, ws_ff_agg, ws_ff_incl;
-  long long ws_agg_s, ws_incl_s, ws_agg_f, ws_incl_f, ws_halo;
+  // workspace byte offsets: stream positions, S at the end of the call, pool weights
+  long long ws_pos, ws_sfin, ws_w;
   float gamma_far, alpha_far, ema_gamma, inv_temp, clip_eps, score_scale;
-  unsigned spin_limit;
-  long long withhold_tile;
-  PrefillPlan plan;
+  unsigned spin_limit;      // polls of a bounded wait before it gives up
+  long long withhold_tile;  // test hook: this tile's pool CTA waits on a barrier nothing completes
+  NearPlan near;
+  int pool_smem, out_smem;
 };
 
-// Workspace layout for a prefill call (bytes).
+// Workspace layout for a prefill call (bytes); nothing in it needs clearing.
 struct PrefillWorkspace {
-  long long fs_agg, fs_incl, ff_agg, ff_incl, flags_end;  // [0, flags_end) cleared per call
-  long long agg_s, incl_s, agg_f, incl_f, halo, total;
+  long long pos;    // [streams] int64 position at the start of the call
+  long long sfin;   // [streams][n_kv][d] fp32 far state at the end of the call
+  long long w;      // [streams * tiles][hi, lo] 64 x 64 bf16 pool-weight blocks
+  long long total;
 };
 
 inline long long align256(long long x) { return (x + 255) & ~255LL; }
@@ -140,11 +136,15 @@ cudaError_t decode_tile_prepare(int device);
 size_t decode_tile_smem_bytes(int HPC, int head_dim, size_t limit);
 int decode_tile_max_active_clusters(int cs, size_t smem, int in_dtype, int head_dim);
 cudaError_t launch_prefill(const PrefillParams& p, int in_dtype, int head_dim, cudaStream_t s);
-bool plan_prefill(int HPC, int D, int esz, int NGm, int K, size_t budget, bool tc, PrefillPlan* out);
+// Near-field plan for head_dim D, input element size esz and window K within
+// `limit` bytes of shared memory, on the tensor cores if tc (bf16, K <= 16);
+// false if none fits.
+bool plan_near(int D, int esz, int K, size_t limit, bool tc, NearPlan* out);
+int prefill_pool_smem();
+int prefill_out_smem();
 cudaError_t prefill_prepare(int device);
 cudaError_t decode_prepare(int device);
 size_t decode_smem_bytes(int HPC, int head_dim, int esz, int NGm, int K, int budget);
-int prefill_max_active_clusters(int cs, size_t smem, int in_dtype, int head_dim);
 int decode_max_active_clusters(int cs, size_t smem, int in_dtype, int head_dim);
 size_t prefill_smem_limit(int device);
 cudaError_t launch_write_header(unsigned char* state, StateHeader h, cudaStream_t s);

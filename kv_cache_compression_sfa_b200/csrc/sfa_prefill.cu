@@ -1,5 +1,6 @@
-// sfa_prefill.cu — SFA prefill: n tokens per (layer, sequence) stream, in
-// parallel over token tiles.
+// sfa_prefill.cu — SFA prefill: n tokens per (layer, sequence) stream in
+// three kernels, each parallel over independent work units with no waits
+// between CTAs.
 //
 // Sources (web pages):
 //   [P1] "Signal Field Attention (SFA)：8KB代码实现4.16倍推理加速与248倍内存压缩"
@@ -7,116 +8,105 @@
 //   [P3] "Dalin Soma SFA基于信号场注意力机制的神经网络推理加速框架"
 //        §2.1 channels 1–3, §2.2 fusion, clip and alpha_layer, §2.4 ring mean.
 //
-// Work unit: one tile of kTile consecutive tokens of one stream, served by a
-// cluster of CS CTAs; CTA `rank` owns query heads [rank*HPC, (rank+1)*HPC)
-// and hence hidden slice [rank*HS, (rank+1)*HS).  Tiles take an ordered
-// ticket from a global counter (tile-major over streams), so a tile only
-// ever waits on tiles with smaller tickets, which are running or done.
+// 1. near_kernel, one CTA per (stream, query head), walks the stream's
+//    tiles of kTile tokens in order.  Per tile: queries and the key/value
+//    span (positions t0-k .. t0+T-1) staged in shared memory by cp.async,
+//    the next tile's copy in flight during this one's arithmetic; the
+//    far-field EWMA S of the head's KV group carried in registers across
+//    tiles [P1 §2.1 eq. S_t]; the near field as an online softmax per token
+//    on the CUDA cores [P1 §2.1 eq. O_near]; x = O_near + alpha_far * S
+//    [P1 §2.1 eq. O] written into `out`, which holds x until step 3.
+// 2. pool_kernel, one CTA per (stream, tile): the cosine scores of the
+//    tile's tokens against the 64 slots, x[T x H] . slot^T on the tcgen05
+//    tensor cores (three bf16 MMAs per 64-column chunk, hi*hi + hi*lo +
+//    lo*hi of split operands, about 16 significant bits, fp32 accumulators
+//    in tensor memory) with the next chunk's copy in flight; |x|, softmax of
+//    cos/T [P3 §2.1 channel 3]; the weights stored in the workspace as split
+//    bf16 blocks in the MMA operand layout.
+// 3. out_kernel, one CTA per (stream, 64 hidden columns), walks the tiles in
+//    order: sem[T x 64] = w . slot_chunk on the tensor cores; per column the
+//    ring sum over the last 16 x (a sliding sum, the 15 rows before the tile
+//    kept from the previous one) and the EMA field (carried across tiles),
+//    four token segments per column joined by their carries; the fusion,
+//    clip and scale [P3 §2.1, §2.2] overwrite x in `out`.  At the stream's
+//    end: ring slots, ring sum, field; one CTA per stream also writes the
+//    window, S and the position.
 //
-// Staging.  The tile's queries and the keys/values it needs (positions
-// t0-k .. t0+T-1: the windows plus the keys that leave them) are brought
-// into shared memory by the bulk-copy engine in key blocks of up to KB rows;
-// the near field runs an online softmax per (token, head) across the blocks
-// with the running output kept in the x tile (two (token, head) pairs per
-// warp when k <= 16).
-//
-// Semantic pool on the tensor cores (tcgen05, accumulators in tensor
-// memory): scores[T x 64] = x[T x HS] . slot^T and sem[T x HS] =
-// w[T x 64] . slot, each as three bf16 MMAs (hi*hi + hi*lo + lo*hi of the
-// split operands, about 16 significant bits) accumulated in fp32.  The slot
-// slice arrives by bulk copy as bf16 hi/lo blocks laid out at sfa_init so
-// that one copy feeds both contractions.
-//
-// Recurrences as parallel scans across tiles, with a deterministic
-// look-back: tiles are grouped by kGroup; a tile's carry-in is the inclusive
-// value at the end of the previous group (or the stream's state) folded with
-// the aggregates of the earlier tiles of its own group, always in the same
-// order, so results do not depend on timing.
-//   * far-field EWMA S (per KV head; depends on keys only) [P1 §2.1 eq. S_t];
-//   * EMA field (per hidden element; depends on x) [P3 §2.1 channel 2];
-//   * ring mean: a sliding 16-token sum; the 15 rows of x before a tile come
-//     from its predecessor's published tail rows (or the state ring).
-// Every wait is bounded; a wait that runs out latches SFA_ERR_DEVICE_TIMEOUT
-// and the kernel still finishes.
-//
-// The pool needs |x| and x·slot_j over all of hidden: partial sums of the
-// slice are reduce-scattered across the cluster through distributed shared
-// memory (rank r finishes tokens r, r+CS, ...) and the softmax weights are
-// written into every CTA's shared memory.
-#include <cooperative_groups.h>
-#include <cstring>
-#include <type_traits>
+// Kernels are chained by programmatic dependent launch; each waits for its
+// predecessor before touching what that one writes.  Every wait of a kernel
+// is on its own copies or MMAs and is bounded; a wait that runs out latches
+// SFA_ERR_DEVICE_TIMEOUT and the kernel still finishes.
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <cstring>
 
 #include "sfa_common.cuh"
 #include "sfa_umma.cuh"
-
-namespace cg = cooperative_groups;
 
 namespace sfa {
 namespace {
 
 constexpr int NT = kPrefillThreads;
 constexpr int NW = NT / 32;
-constexpr int kPartStride = kSlots + 1;  // 64 partial dots + |x|^2 per token
-constexpr int kCW = kBlk;                // columns per combine chunk
-constexpr int kSemStride = kCW + 4;      // padded row of the sem chunk
-constexpr int kSeg = 4;                  // token segments per column in the epilogue
-constexpr int kEvChunk = 16;             // evicted-key loads in flight per thread
-constexpr int kTmemCols = 256;           // scores (64) + two 64-column sem buffers
-// Tensor-core near field: key span t0-16 .. t0+63 of a tile (k <= 16) as the
-// N of the score MMA, 8-row groups of that span, and the column of the
-// P·V accumulator in tensor memory.
-constexpr int kSpan = kTile + 16;
-constexpr int kSpanR8 = kSpan / 8;
-constexpr int kTmemO = 128;
+constexpr int kTmemCols = 64;          // one 64 x 64 fp32 accumulator
+constexpr int kSeg = 4;                // token segments per column in out_kernel
+constexpr int kSegLen = kTile / kSeg;
+constexpr int kScStride = kSlots + 1;  // padded row of the staged scores
+constexpr int kXsPad = 4;              // x tile row padding (floats) in near_kernel
 static_assert(kTile == kBlk, "tile tokens are the M of the pool MMAs");
+static_assert(kSegLen >= kRing, "a segment's ring window reaches back at most one segment");
 
-// Near field over one staged key block for all (token, head) pairs of the
-// tile [P1 §2.1 eq. O_near].  LP lanes serve one pair: lane a scores key
-// lo+base+a in full, online softmax across chunks and blocks, then P·V with
-// the LP lanes over head dims, accumulated into the pair's row of the x
-// tile.  Running max and denominator per pair live in mrun/lrun.
-template <typename Tin, int D, int LP>
-__device__ __forceinline__ void near_block(const Tin* qst, const unsigned char* kb,
-                                           const unsigned char* vb, float* xs, float* mrun,
-                                           float* lrun, int rowB, int HS, int XS, int HPC, int G,
-                                           int g_lo, int K, long long t0, int Tt, long long bs,
-                                           long long be, float score_scale, int h0, int warp,
-                                           int lane) {
-  constexpr int PPW = 32 / LP;  // pairs per warp
+// Every kernel checks the state header (same answer in every CTA).
+__device__ __forceinline__ bool header_matches(const PrefillParams& p) {
+  const uint4 h0v = __ldcg(reinterpret_cast<const uint4*>(p.state));
+  const uint4 h1v = __ldcg(reinterpret_cast<const uint4*>(p.state + 16));
+  StateHeader hd;
+  reinterpret_cast<uint4*>(&hd)[0] = h0v;
+  reinterpret_cast<uint4*>(&hd)[1] = h1v;
+  return hd.magic == kMagic && hd.cfg_hash == p.cfg_hash && hd.batch == p.B && hd.n_layers == p.L;
+}
+
+__device__ __forceinline__ unsigned char* stream_block(const PrefillParams& p, int s) {
+  return p.state + kHeaderBytes + (static_cast<long long>(p.l0) * p.B + s) * p.so.stride;
+}
+
+// ======================================================================
+// 1. near field, far field and x
+// ======================================================================
+
+// Near field of the tile's tokens for one query head [P1 §2.1 eq. O_near]:
+// LP lanes serve a token; lane a scores key base+a in full, online softmax
+// across chunks of LP keys, then P·V with the LP lanes over head dims; the
+// result is added to the token's row of the x tile (which holds alpha*S).
+// krow(j)/vrow(j): key/value row of absolute position j.
+template <typename Tin, int D, int LP, typename KR, typename VR>
+__device__ __forceinline__ void near_tile(const unsigned char* qs, int RB, float* xs, int Tt,
+                                          long long t0, int K, float scale, int warp, int lane,
+                                          KR krow, VR vrow) {
+  constexpr int PPW = 32 / LP;  // tokens per warp
   constexpr int EPL = D / LP;   // head dims per lane in P·V
   constexpr int VE = Load16<Tin>::N;
+  constexpr int XS = D + kXsPad;
   const int sub = lane / LP, sl = lane % LP;
-  const int gbase = sub * LP;   // first lane of this sub-group
-  for (int pb = warp * PPW; pb < Tt * HPC; pb += NW * PPW) {
-    const int pair = pb + sub;
-    const bool live = pair < Tt * HPC;
-    const int r = live ? pair / HPC : 0;
-    const int hh = live ? pair % HPC : 0;
-    const int gg = (h0 + hh) / G - g_lo;  // KV head of this pair, local to the CTA
+  const int gbase = sub * LP;
+  for (int rb = warp * PPW; rb < Tt; rb += NW * PPW) {
+    const int r = rb + sub;
+    const bool live = r < Tt;
     const long long pt = t0 + r;
-    const long long wlo = pt - K + 1 > 0 ? pt - K + 1 : 0;
-    const long long lo = wlo > bs ? wlo : bs;
-    const long long hi = pt < be - 1 ? pt : be - 1;
-    const int cnt_pair = (live && lo <= hi) ? static_cast<int>(hi - lo + 1) : 0;
-    int cnt_max = cnt_pair;  // the sub-pairs of a warp run the same number of chunks
+    const long long lo = pt - K + 1 > 0 ? pt - K + 1 : 0;
+    const int cnt = live ? static_cast<int>(pt - lo + 1) : 0;
+    int cnt_max = cnt;  // the tokens of a warp run the same number of chunks
     if (LP < 32) cnt_max = max(cnt_max, __shfl_xor_sync(0xffffffffu, cnt_max, 16));
-    if (cnt_max == 0) continue;
-    float* orow = xs + r * XS + hh * D + sl * EPL;
-    float m = live ? mrun[pair] : 0.f;
-    float den = live ? lrun[pair] : 0.f;
-    float o[EPL];
+    const Tin* qrow = reinterpret_cast<const Tin*>(qs + (live ? r : 0) * RB);
+    float m = -INFINITY, den = 0.f, o[EPL];
 #pragma unroll
-    for (int e = 0; e < EPL; ++e) o[e] = live ? orow[e] : 0.f;
-    const Tin* qrow = qst + r * HS + hh * D;
+    for (int e = 0; e < EPL; ++e) o[e] = 0.f;
     for (int base = 0; base < cnt_max; base += LP) {
-      const int cnt = max(0, min(LP, cnt_pair - base));
-      float s = -INFINITY;
-      if (sl < cnt) {
-        const Tin* kr = reinterpret_cast<const Tin*>(kb + (lo + base + sl - bs) * rowB) + gg * D;
+      const int cc = max(0, min(LP, cnt - base));  // this token's keys in the chunk
+      float sc = -INFINITY;
+      if (sl < cc) {
+        const Tin* kr = krow(lo + base + sl);
         float acc[4] = {0.f, 0.f, 0.f, 0.f};  // independent chains
 #pragma unroll
         for (int i = 0; i < D; i += VE) {
@@ -126,14 +116,14 @@ __device__ __forceinline__ void near_block(const Tin* qst, const unsigned char* 
 #pragma unroll
           for (int e = 0; e < VE; ++e) acc[e & 3] = fmaf(qv[e], kv[e], acc[e & 3]);
         }
-        s = ((acc[0] + acc[1]) + (acc[2] + acc[3])) * score_scale;
+        sc = ((acc[0] + acc[1]) + (acc[2] + acc[3])) * scale;
       }
-      float cm = s;
+      float cm = sc;
 #pragma unroll
       for (int off = LP / 2; off > 0; off >>= 1) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, off));
-      const float mn = (cnt > 0) ? fmaxf(m, cm) : m;
-      const float corr = (cnt > 0) ? expf(m - mn) : 1.f;
-      const float pj = (sl < cnt) ? expf(s - mn) : 0.f;
+      const float mn = (cc > 0) ? fmaxf(m, cm) : m;
+      const float corr = (cc > 0) ? expf(m - mn) : 1.f;
+      const float pj = (sl < cc) ? expf(sc - mn) : 0.f;
       float ps = pj;
 #pragma unroll
       for (int off = LP / 2; off > 0; off >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
@@ -143,10 +133,9 @@ __device__ __forceinline__ void near_block(const Tin* qst, const unsigned char* 
       const int cmax = min(LP, cnt_max - base);
       for (int c = 0; c < cmax; ++c) {
         const float pc = __shfl_sync(0xffffffffu, pj, gbase + c);
-        if (c < cnt) {
-          const Tin* vr = reinterpret_cast<const Tin*>(vb + (lo + base + c - bs) * rowB) + gg * D + sl * EPL;
+        if (c < cc) {
           float vv[EPL];
-          VecLoad<Tin, EPL>::run(vr, vv);
+          VecLoad<Tin, EPL>::run(vrow(lo + base + c) + sl * EPL, vv);
 #pragma unroll
           for (int e = 0; e < EPL; ++e) o[e] = fmaf(pc, vv[e], o[e]);
         }
@@ -154,872 +143,869 @@ __device__ __forceinline__ void near_block(const Tin* qst, const unsigned char* 
       m = mn;
     }
     if (live) {
+      const float inv = 1.f / den;
+      float* xr = xs + r * XS + sl * EPL;
 #pragma unroll
-      for (int e = 0; e < EPL; ++e) orow[e] = o[e];
-      if (sl == 0) {
-        mrun[pair] = m;
-        lrun[pair] = den;
-      }
+      for (int e = 0; e < EPL; ++e) xr[e] = fmaf(o[e], inv, xr[e]);
     }
   }
 }
 
 template <typename Tin, int D>
-__global__ void __launch_bounds__(kPrefillThreads, 2)
-prefill_kernel(const PrefillParams p) {
+__global__ void __launch_bounds__(NT, 2) near_kernel(const PrefillParams p) {
   constexpr int ESZ = static_cast<int>(sizeof(Tin));
-  cg::cluster_group cluster = cg::this_cluster();
-  const int rank = static_cast<int>(cluster.block_rank());
+  constexpr int C16 = D * ESZ / 16;  // 16-byte chunks of one head row
+  constexpr int XS = D + kXsPad;
+  const int h = blockIdx.x, s = blockIdx.y;  // query head, call-relative stream
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-
   extern __shared__ __align__(16) unsigned char smb[];
-  const PrefillPlan& pl = p.plan;
-  const int HPC = p.HPC;
-  const int HS = HPC * D, XS = HS + 4;
-  const int nch = HS / kBlk;                               // 64-column chunks of the slice
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smb + pl.bars);
-  uint64_t* bar_kv = bars + 0;                             // key/value blocks (+ queries)
-  uint64_t* bar_sl = bars + 1;                             // slot image
-  uint64_t* bar_ms = bars + 2;                             // [2] score MMAs done, per x buffer
-  uint64_t* bar_sd = bars + 4;                             // all score MMAs done
-  uint64_t* bar_mc = bars + 5;                             // [2] sem MMAs done, per accumulator
-  uint64_t* bar_nf = bars + 7;                             // near-field MMAs done
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8);
-  float* xs = reinterpret_cast<float*>(smb + pl.xs);      // [T][XS]  x (O accumulator first)
-  float* halo = reinterpret_cast<float*>(smb + pl.halo);  // [15][HS] x of the 15 tokens before
-  float* fcar = reinterpret_cast<float*>(smb + pl.fcar);  // [HS]     field carried in
-  float* sst = reinterpret_cast<float*>(smb + pl.sst);    // [NGm][D] S carried in / at tile end
-  float* sagg = reinterpret_cast<float*>(smb + pl.sagg);  // [NGm][D] this tile's S aggregate
-  float* segA = reinterpret_cast<float*>(smb + pl.sega);  // [nseg][NG*D] scan segment aggregates
-  float* segc = reinterpret_cast<float*>(smb + pl.ml);    // [kSeg][kCW] epilogue carries
-  float* mrun = segc + kSeg * kCW;                        // [T*HPC]  running max (CUDA-core near field)
-  float* lrun = mrun + kTile * HPC;                       // [T*HPC]  running denominator
-  Tin* qst = reinterpret_cast<Tin*>(smb + pl.qst);        // [T][HS]   queries
-  unsigned char* kb = smb + pl.kb;                        // [KB][rowB] key block
-  unsigned char* vb = smb + pl.vb;                        // [KB][rowB] value block
-  // tensor-core near field: packed query block [64 x D], key and value blocks
-  // [kSpan x D] per KV head, P block [64 x kSpan] (hi, lo)
-  unsigned char* qa = smb + pl.qa;
-  unsigned char* kvp = smb + pl.kvp;
-  unsigned char* pa = smb + pl.pa;
-  const bool tc = pl.tc != 0;
-  unsigned char* simg = smb + pl.sl;                      // [nch][hi,lo] slot blocks
-  float* part = reinterpret_cast<float*>(smb + pl.part);  // [T][65]   pool partials, then
-  float* semc = part;                                     // [T][68]   the sem chunk
-  unsigned char* xw = smb + pl.semc;                      // x block (hi, lo), then w block (hi, lo)
-
-  __shared__ unsigned long long s_ticket;
-  __shared__ long long s_pos;
+  const NearPlan& np = p.near;
   __shared__ int s_ok;
-  __shared__ int s_bad;  // a staging wait ran out: skip global writes
-  __shared__ float s_gpn[kTile + 1];  // gamma_far^n, n = 0 .. kTile
-  __shared__ float s_gseg[kSeg];    // ema_gamma^(length) of the epilogue's token segments
+  __shared__ long long s_pos;
 
-  if (tid == 0) {
-    for (int i = 0; i < 8; ++i) mbar_init(bars + i, 1);
-    mbar_fence_init();
-    s_bad = 0;
-  }
   pdl_trigger();
-  pdl_wait();
-
-  // ---- ticket: the tile this cluster serves ----------------------------
-  if (rank == 0 && tid == 0) s_ticket = atomicAdd(reinterpret_cast<unsigned long long*>(p.ws), 1ull);
+  pdl_wait();  // the state may be written by the previous kernel of the stream
+  unsigned char* blk = stream_block(p, s);
   if (tid == 0) {
-    const uint4 h0v = __ldcg(reinterpret_cast<const uint4*>(p.state));
-    const uint4 h1v = __ldcg(reinterpret_cast<const uint4*>(p.state + 16));
-    StateHeader hd;
-    reinterpret_cast<uint4*>(&hd)[0] = h0v;
-    reinterpret_cast<uint4*>(&hd)[1] = h1v;
-    s_ok = (hd.magic == kMagic) & (hd.cfg_hash == p.cfg_hash) & (hd.batch == p.B) &
-           (hd.n_layers == p.L);
+    s_ok = header_matches(p);
+    s_pos = __ldcg(reinterpret_cast<const long long*>(blk + p.so.pos));
   }
-  cluster.sync();
-  const long long ticket = static_cast<long long>(*cluster.map_shared_rank(&s_ticket, 0));
-  if (!s_ok) {  // uniform over the whole grid: every CTA reads the same header
-    if (tid == 0 && rank == 0 && ticket == 0) latch_error(p.err, SFA_ERR_STATE_MISMATCH);
-    cluster.sync();  // rank 0's s_ticket must outlive the peers' reads
+  __syncthreads();
+  if (!s_ok) {  // uniform over the grid
+    if (tid == 0 && h == 0 && s == 0) latch_error(p.err, SFA_ERR_STATE_MISMATCH);
     return;
   }
-  // Tensor memory for the pool accumulators (at most two CTAs per SM, so the
-  // allocation never waits).
+  const long long pos0 = s_pos;
+  if (tid == 0 && h == 0) reinterpret_cast<long long*>(p.ws + p.ws_pos)[s] = pos0;
+  const int K = p.K, nkv = p.nkv, g = h / p.G;
+  const Tin* win_k = reinterpret_cast<const Tin*>(blk + p.so.win_k);
+  const Tin* win_v = reinterpret_cast<const Tin*>(blk + p.so.win_v);
+  const float* far = reinterpret_cast<const float*>(blk + p.so.far);
+  const long long in_row0 = static_cast<long long>(s) * p.n;  // first input row of the stream
+  const Tin* qin = static_cast<const Tin*>(p.q) + in_row0 * p.nq * D;
+  const Tin* kin = static_cast<const Tin*>(p.k) + in_row0 * nkv * D;
+  const Tin* vin = static_cast<const Tin*>(p.v) + in_row0 * nkv * D;
+  // Key/value row of absolute position j >= 0 for KV head g: from the input
+  // if it belongs to this call, else from window slot j mod k (the state
+  // holds positions pos0-k .. pos0-1).
+  auto krow_g = [&](long long j) -> const Tin* {
+    return j >= pos0 ? kin + ((j - pos0) * nkv + g) * D : win_k + ((j % K) * nkv + g) * D;
+  };
+  auto vrow_g = [&](long long j) -> const Tin* {
+    return j >= pos0 ? vin + ((j - pos0) * nkv + g) * D : win_v + ((j % K) * nkv + g) * D;
+  };
+  const int RB = np.row;
+  float* xs = reinterpret_cast<float*>(smb + np.xs);
+
+  // Copies of tile i into stage st: its queries and (staged plans) the key
+  // and value rows of positions t0-k .. t0+Tt-1; positions before 0 are
+  // never read and stay unloaded.
+  auto issue = [&](int i, int st) {
+    const long long t0 = pos0 + static_cast<long long>(i) * kTile;
+    const int Tt = static_cast<int>(min(static_cast<long long>(kTile), p.n - static_cast<long long>(i) * kTile));
+    unsigned char* qs = smb + np.q[st];
+    for (int c = tid; c < Tt * C16; c += NT) {
+      const int r = c / C16, u = c % C16;
+      cp_async16(qs + r * RB + u * 16,
+                 reinterpret_cast<const unsigned char*>(qin + ((t0 - pos0 + r) * p.nq + h) * D) + u * 16);
+    }
+    if (np.stages > 0) {
+      unsigned char* ks = smb + np.k[st];
+      unsigned char* vs = smb + np.v[st];
+      const int R = Tt + K;
+      for (int c = tid; c < R * C16; c += NT) {
+        const int r = c / C16, u = c % C16;
+        const long long j = t0 - K + r;
+        if (j < 0) continue;
+        cp_async16(ks + r * RB + u * 16, reinterpret_cast<const unsigned char*>(krow_g(j)) + u * 16);
+        cp_async16(vs + r * RB + u * 16, reinterpret_cast<const unsigned char*>(vrow_g(j)) + u * 16);
+      }
+    }
+    cp_async_commit();
+  };
+
+  float sreg = (tid < D) ? far[g * D + tid] : 0.f;  // S of KV head g, dim tid, carried across tiles
+  const float gf = p.gamma_far, af = p.alpha_far;
+  const int tiles = p.tiles_per_stream;
+  issue(0, 0);
+  for (int i = 0; i < tiles; ++i) {
+    const int st = (np.stages == 2) ? (i & 1) : 0;
+    if (np.stages == 2 && i + 1 < tiles) {
+      issue(i + 1, st ^ 1);  // that stage was released at the end of tile i-1
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+    const long long t0 = pos0 + static_cast<long long>(i) * kTile;
+    const int Tt = static_cast<int>(min(static_cast<long long>(kTile), p.n - static_cast<long long>(i) * kTile));
+    const unsigned char* qs = smb + np.q[st];
+    const unsigned char* ks = smb + np.k[st];
+    const unsigned char* vs = smb + np.v[st];
+    const bool staged = np.stages > 0;
+
+    // Far field [P1 §2.1 eq. S_t]: token t0+r evicts position t0+r-k (span
+    // row r) once t0+r >= k; x starts as alpha_far * S_t.
+    if (tid < D) {
+      const int r_ev = static_cast<int>(max(0LL, min(static_cast<long long>(Tt), K - t0)));
+      for (int r = 0; r < r_ev; ++r) xs[r * XS + tid] = af * sreg;
+      if (staged) {
+        const Tin* col = reinterpret_cast<const Tin*>(ks) + tid;
+        const int pitch = RB / ESZ;
+        for (int r = r_ev; r < Tt; ++r) {
+          sreg = ewma(gf, sreg, to_f32<Tin>(col[r * pitch]));
+          xs[r * XS + tid] = af * sreg;
+        }
+      } else {
+        for (int r = r_ev; r < Tt; ++r) {
+          sreg = ewma(gf, sreg, to_f32<Tin>(krow_g(t0 + r - K)[tid]));
+          xs[r * XS + tid] = af * sreg;
+        }
+      }
+    }
+    __syncthreads();
+
+    // Near field, added onto alpha_far * S.
+    const long long span0 = t0 - K;  // position of span row 0
+    auto krow_s = [&](long long j) -> const Tin* {
+      return reinterpret_cast<const Tin*>(ks + static_cast<int>(j - span0) * RB);
+    };
+    auto vrow_s = [&](long long j) -> const Tin* {
+      return reinterpret_cast<const Tin*>(vs + static_cast<int>(j - span0) * RB);
+    };
+    if (staged) {
+      if (K <= 16) near_tile<Tin, D, 16>(qs, RB, xs, Tt, t0, K, p.score_scale, warp, lane, krow_s, vrow_s);
+      else near_tile<Tin, D, 32>(qs, RB, xs, Tt, t0, K, p.score_scale, warp, lane, krow_s, vrow_s);
+    } else {
+      if (K <= 16) near_tile<Tin, D, 16>(qs, RB, xs, Tt, t0, K, p.score_scale, warp, lane, krow_g, vrow_g);
+      else near_tile<Tin, D, 32>(qs, RB, xs, Tt, t0, K, p.score_scale, warp, lane, krow_g, vrow_g);
+    }
+    __syncthreads();
+
+    // x rows into out (this head's columns).
+    float* orow0 = p.out + (in_row0 + (t0 - pos0)) * p.H + h * D;
+    for (int c = tid; c < Tt * (D / 4); c += NT) {
+      const int r = c / (D / 4), c4 = (c % (D / 4)) * 4;
+      *reinterpret_cast<float4*>(orow0 + static_cast<long long>(r) * p.H + c4) =
+          *reinterpret_cast<const float4*>(xs + r * XS + c4);
+    }
+    __syncthreads();  // the stage and the x tile are free again
+    if (np.stages != 2 && i + 1 < tiles) issue(i + 1, 0);
+  }
+  // S at the end of the call, from the group's first query head.
+  if (tid < D && h % p.G == 0)
+    reinterpret_cast<float*>(p.ws + p.ws_sfin)[(static_cast<long long>(s) * nkv + g) * D + tid] = sreg;
+}
+
+// Near field and far field on the tensor cores (bf16 inputs, k <= 16).
+// Per tile, with the span fixed at positions t0-16 .. t0+63 (kNS rows):
+//   scores[64 x kNS] = Q . K_span^T (tensor memory, columns 0 .. kNS-1;
+//   bf16 products are exact, fp32 accumulation) [P1 §2.1 eq. O_near];
+//   softmax over the band of each row (token r sees span rows r+17-k ..
+//   r+16, none before position 0), P split into bf16 hi + lo;
+//   X[64 x D] = P . V_span + G . K_span (columns kTmemO ..), each product
+//   as hi + lo of the split left operand.
+// The far field [P1 §2.1 eq. S_t] inside a tile is linear in the keys it
+// evicts: with r_ev the first token of the tile that evicts (token r evicts
+// position t0+r-k, span row r+16-k) and S0 the state at the tile start,
+//   S_r = gamma^m(r) S0 + sum_{r_ev <= j <= r} (1-gamma) gamma^(r-j) e_j,
+// m(r) = max(0, r - r_ev + 1).  G[r][c] = alpha_far (1-gamma) gamma^(r-j)
+// for span row c = j+16-k holds the second term, so X = O_near + alpha_far
+// (S_r - gamma^m(r) S0) and the epilogue adds alpha_far gamma^m(r) S0
+// [P1 §2.1 eq. O].  S at the tile end (the next tile's S0) is one dot
+// product per dim over the evicted keys, with no chain from token to token.
+// Operand blocks use the core-matrix layout of sfa_umma.cuh; the key and
+// value blocks put 8-dim groups kDStr bytes apart (16 bytes of padding) so
+// that threads reading one key row hit distinct banks.  The key and value
+// blocks are the MN-major B of G.K and P.V.
+constexpr int kNS = kTile + 16;
+constexpr int kDStr = (kNS / 8) * 128 + 16;
+constexpr int kTmemNear = 256;
+constexpr int kTmemO = 128;
+
+__device__ __forceinline__ int kv_off(int c, int d) {
+  return (d >> 3) * kDStr + (c >> 3) * 128 + (c & 7) * 16 + (d & 7) * 2;
+}
+
+template <int D>
+__global__ void __launch_bounds__(NT, 2) near_tc_kernel(const PrefillParams p) {
+  using Tin = __nv_bfloat16;
+  constexpr int C16 = D / 8;  // 16-byte chunks of one head row
+  constexpr int kBlkKV = (D / 8) * kDStr;
+  const int h = blockIdx.x, s = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  extern __shared__ __align__(16) unsigned char smb[];
+  const NearPlan& np = p.near;
+  __shared__ __align__(8) uint64_t s_bar;
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_ok;
+  __shared__ long long s_pos;
+  __shared__ float s_s0[128];        // S at the tile start (this head's KV group)
+  __shared__ float s_gpow[kTile + 1];  // gamma_far^m
+
+  pdl_trigger();
+  pdl_wait();
+  unsigned char* blk = stream_block(p, s);
+  if (tid <= kTile) s_gpow[tid] = powf(p.gamma_far, static_cast<float>(tid));
+  if (tid == 0) {
+    s_ok = header_matches(p);
+    s_pos = __ldcg(reinterpret_cast<const long long*>(blk + p.so.pos));
+    mbar_init(&s_bar, 1);
+    mbar_fence_init();
+  }
+  __syncthreads();
+  if (!s_ok) {
+    if (tid == 0 && h == 0 && s == 0) latch_error(p.err, SFA_ERR_STATE_MISMATCH);
+    return;
+  }
+  if (warp == 0) tmem_alloc(&s_tmem, kTmemNear);
+  const long long pos0 = s_pos;
+  if (tid == 0 && h == 0) reinterpret_cast<long long*>(p.ws + p.ws_pos)[s] = pos0;
+  const int K = p.K, nkv = p.nkv, g = h / p.G;
+  const Tin* win_k = reinterpret_cast<const Tin*>(blk + p.so.win_k);
+  const Tin* win_v = reinterpret_cast<const Tin*>(blk + p.so.win_v);
+  const float* far = reinterpret_cast<const float*>(blk + p.so.far);
+  const long long in_row0 = static_cast<long long>(s) * p.n;
+  const Tin* qin = static_cast<const Tin*>(p.q) + in_row0 * p.nq * D;
+  const Tin* kin = static_cast<const Tin*>(p.k) + in_row0 * nkv * D;
+  const Tin* vin = static_cast<const Tin*>(p.v) + in_row0 * nkv * D;
+  auto krow_g = [&](long long j) -> const Tin* {
+    return j >= pos0 ? kin + ((j - pos0) * nkv + g) * D : win_k + ((j % K) * nkv + g) * D;
+  };
+  auto vrow_g = [&](long long j) -> const Tin* {
+    return j >= pos0 ? vin + ((j - pos0) * nkv + g) * D : win_v + ((j % K) * nkv + g) * D;
+  };
+  unsigned char* pa_hi = smb + np.pa;
+  unsigned char* pa_lo = pa_hi + kTile * kNS * 2;
+  unsigned char* ga_hi = smb + np.ga;
+  unsigned char* ga_lo = ga_hi + kTile * kNS * 2;
+  for (int i = tid; i < 2 * kTile * kNS * 2 / 16; i += NT)  // P columns outside the bands stay zero
+    reinterpret_cast<uint4*>(pa_hi)[i] = make_uint4(0u, 0u, 0u, 0u);
+  const float gf = p.gamma_far, af = p.alpha_far;
+  // G for the tiles whose first evicting token is r_ev (0 once t0 >= k).
+  auto build_g = [&](int r_ev) {
+    for (int i = tid; i < kTile * kNS; i += NT) {
+      const int r = i / kNS, c = i % kNS;
+      const int j = c - 16 + K;  // token whose evicted key is span row c
+      float gv = 0.f;
+      if (j >= r_ev && j <= r) gv = af * (1.0f - gf) * s_gpow[r - j];
+      __nv_bfloat16 hb, lb;
+      split_bf16(gv, hb, lb);
+      const int off = blk_off(r, c);
+      *reinterpret_cast<__nv_bfloat16*>(ga_hi + off) = hb;
+      *reinterpret_cast<__nv_bfloat16*>(ga_lo + off) = lb;
+    }
+  };
+  if (tid < D) s_s0[tid] = far[g * D + tid];
+  __syncthreads();  // s_gpow, s_s0
+  int g_built = -1;
+
+  // Copies of tile i into stage st: queries (rows past the tile zero) and
+  // the span rows of positions t0-16 .. t0+Tt-1 (others zero).
+  auto issue = [&](int i, int st) {
+    const long long t0 = pos0 + static_cast<long long>(i) * kTile;
+    const int Tt = static_cast<int>(min(static_cast<long long>(kTile), p.n - static_cast<long long>(i) * kTile));
+    unsigned char* qa = smb + np.q[st];
+    unsigned char* kb = smb + np.k[st];
+    unsigned char* vb = smb + np.v[st];
+    for (int c = tid; c < kTile * C16; c += NT) {
+      const int r = c / C16, u = c % C16;
+      unsigned char* dst = qa + blk_off(r, 8 * u);
+      if (r < Tt) cp_async16(dst, qin + ((t0 - pos0 + r) * p.nq + h) * D + 8 * u);
+      else *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+    }
+    for (int c = tid; c < kNS * C16; c += NT) {
+      const int r = c / C16, u = c % C16;
+      const long long j = t0 - 16 + r;
+      const int off = kv_off(r, 8 * u);
+      if (j >= 0 && r < 16 + Tt) {
+        cp_async16(kb + off, krow_g(j) + 8 * u);
+        cp_async16(vb + off, vrow_g(j) + 8 * u);
+      } else {
+        *reinterpret_cast<uint4*>(kb + off) = make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(vb + off) = make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+    cp_async_commit();
+  };
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+  const uint32_t idesc_qk = umma_idesc_bf16(kTile, kNS, false);
+  const uint32_t idesc_pv = umma_idesc_bf16(kTile, D, true);
+  float sreg = 0.f;  // S at the tile end (threads tid < D, dim tid)
+  const int tiles = p.tiles_per_stream;
+  unsigned par = 0;
+  bool ok = true;
+  issue(0, 0);
+  for (int i = 0; i < tiles; ++i) {
+    const int st = (np.stages == 2) ? (i & 1) : 0;
+    if (np.stages == 2 && i + 1 < tiles) {
+      issue(i + 1, st ^ 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    const long long t0 = pos0 + static_cast<long long>(i) * kTile;
+    const int Tt = static_cast<int>(min(static_cast<long long>(kTile), p.n - static_cast<long long>(i) * kTile));
+    const int r_ev = static_cast<int>(max(0LL, min(static_cast<long long>(Tt), K - t0)));
+    if (r_ev != g_built) {  // uniform: the first tile of a stream start, then once more
+      build_g(r_ev);
+      g_built = r_ev;
+    }
+    fence_proxy_async_smem();  // copies, zero fills and G seen by the MMAs
+    __syncthreads();
+    const unsigned char* qa = smb + np.q[st];
+    const unsigned char* kb = smb + np.k[st];
+    const unsigned char* vb = smb + np.v[st];
+    if (tid == 0) {
+      tc_fence_after();
+#pragma unroll
+      for (int k2 = 0; k2 < D / 16; ++k2)
+        umma_bf16(tmem, umma_desc(qa + k2 * 2048, 1024, 128), umma_desc(kb + 2 * k2 * kDStr, kDStr, 128),
+                  idesc_qk, k2 > 0);
+      umma_commit(&s_bar);
+    }
+    // S at the tile end while the scores form: gamma^m S0 plus the evicted
+    // keys' weighted sum (independent terms, four accumulators).
+    if (tid < D) {
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int j = 0; j < kTile; ++j) {
+        const float e = __bfloat162float(*reinterpret_cast<const Tin*>(kb + kv_off(j + 16 - K, tid)));
+        const float w = (j >= r_ev && j < Tt) ? (1.0f - gf) * s_gpow[max(0, Tt - 1 - j)] : 0.f;
+        acc[j & 3] = fmaf(w, e, acc[j & 3]);
+      }
+      sreg = fmaf(s_gpow[max(0, Tt - r_ev)], s_s0[tid], (acc[0] + acc[1]) + (acc[2] + acc[3]));
+    }
+    if (!mbar_wait_bounded(&s_bar, par, kMbarPollLimit, p.err)) ok = false;
+    par ^= 1u;
+    tc_fence_after();
+    // Band softmax: warp sp (< 4) holds rows 16 sp .. 16 sp + 15 in lanes
+    // 0 .. 15, whose bands lie in span columns 16 sp .. 16 sp + 31.
+    if (warp < 4) {
+      const int sp = warp;
+      float v[32];
+      tmem_ld32(tmem + (static_cast<uint32_t>(32 * sp) << 16) + 16 * sp, v);
+      if (lane < 16) {
+        const int r = 16 * sp + lane;
+        const int cmin = t0 < 16 ? static_cast<int>(16 - t0) : 0;  // first row at position >= 0
+        float mx = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int c = 16 * sp + j;
+          const bool in = c >= r + 17 - K && c <= r + 16 && c >= cmin;
+          v[j] = in ? v[j] * p.score_scale : -INFINITY;
+          mx = fmaxf(mx, v[j]);
+        }
+        float sum = 0.f;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          v[j] = __expf(v[j] - mx);  // 0 outside the band
+          sum += v[j];
+        }
+        const float inv = 1.f / sum;
+#pragma unroll
+        for (int g8 = 0; g8 < 4; ++g8) {
+          uint32_t hw[4], lw[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            __nv_bfloat16 h0b, l0b, h1b, l1b;
+            split_bf16(v[8 * g8 + 2 * e] * inv, h0b, l0b);
+            split_bf16(v[8 * g8 + 2 * e + 1] * inv, h1b, l1b);
+            hw[e] = static_cast<uint32_t>(__bfloat16_as_ushort(h0b)) |
+                    (static_cast<uint32_t>(__bfloat16_as_ushort(h1b)) << 16);
+            lw[e] = static_cast<uint32_t>(__bfloat16_as_ushort(l0b)) |
+                    (static_cast<uint32_t>(__bfloat16_as_ushort(l1b)) << 16);
+          }
+          const int off = blk_off(r, 16 * sp + 8 * g8);
+          *reinterpret_cast<uint4*>(pa_hi + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+          *reinterpret_cast<uint4*>(pa_lo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+        }
+      }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+#pragma unroll
+      for (int k2 = 0; k2 < kNS / 16; ++k2) {
+        const uint64_t bv = umma_desc(vb + k2 * 256, 128, kDStr);
+        const uint64_t bk = umma_desc(kb + k2 * 256, 128, kDStr);
+        umma_bf16(tmem + kTmemO, umma_desc(pa_hi + k2 * 2048, 1024, 128), bv, idesc_pv, k2 > 0);
+        umma_bf16(tmem + kTmemO, umma_desc(pa_lo + k2 * 2048, 1024, 128), bv, idesc_pv, true);
+        umma_bf16(tmem + kTmemO, umma_desc(ga_hi + k2 * 2048, 1024, 128), bk, idesc_pv, true);
+        umma_bf16(tmem + kTmemO, umma_desc(ga_lo + k2 * 2048, 1024, 128), bk, idesc_pv, true);
+      }
+      umma_commit(&s_bar);
+    }
+    if (!mbar_wait_bounded(&s_bar, par, kMbarPollLimit, p.err)) ok = false;
+    par ^= 1u;
+    tc_fence_after();
+    {  // x = X + alpha_far gamma^m(r) S0 into out: warp w takes rows 16 (w%4) ..,
+       // half the head dims
+      const int sp = warp & 3, colh = (warp >> 2) * (D / 2);
+      const int r = 16 * sp + lane;
+      const float c0s = af * s_gpow[min(kTile, max(0, r - r_ev + 1))];
+      float* orow = p.out + (in_row0 + (t0 - pos0) + r) * p.H + h * D + colh;
+#pragma unroll
+      for (int c0 = 0; c0 < D / 2; c0 += 32) {
+        float v[32];
+        tmem_ld32(tmem + (static_cast<uint32_t>(32 * sp) << 16) + kTmemO + colh + c0, v);
+        if (lane < 16 && r < Tt && ok) {
+          const float* s0 = s_s0 + colh + c0;
+#pragma unroll
+          for (int j = 0; j < 32; j += 4)
+            *reinterpret_cast<float4*>(orow + c0 + j) =
+                make_float4(fmaf(c0s, s0[j], v[j]), fmaf(c0s, s0[j + 1], v[j + 1]),
+                            fmaf(c0s, s0[j + 2], v[j + 2]), fmaf(c0s, s0[j + 3], v[j + 3]));
+        }
+      }
+    }
+    tc_fence_before();
+    __syncthreads();  // stage, P, S0 and accumulators free again
+    if (tid < D) s_s0[tid] = sreg;  // read after the next tile's barriers
+    if (np.stages != 2 && i + 1 < tiles) issue(i + 1, 0);
+  }
+  if (tid < D && h % p.G == 0)
+    reinterpret_cast<float*>(p.ws + p.ws_sfin)[(static_cast<long long>(s) * nkv + g) * D + tid] = sreg;
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemNear);
+  }
+}
+
+// ======================================================================
+// 2. pool scores and weights
+// ======================================================================
+
+// Shared-memory plan of pool_kernel (byte offsets).
+struct PoolPlan {
+  static constexpr int bars = 0;                        // 6 mbarriers
+  static constexpr int tmem = 64;                       // tensor-memory address
+  static constexpr int xf = 128;                        // [2][64][64] fp32 x chunks
+  static constexpr int img = xf + 2 * kBlk * kBlk * 4;  // [2][hi, lo] slot blocks
+  static constexpr int xsp = img + 2 * 2 * kBlkBytes;   // [2][hi, lo] split x blocks
+  static constexpr int sc = xsp + 2 * 2 * kBlkBytes;    // [64][65] fp32 scores
+  static constexpr int ss = sc + kTile * kScStride * 4; // [64] |x|^2
+  static constexpr int total = ss + kTile * 4;
+};
+
+__global__ void __launch_bounds__(NT, 2) pool_kernel(const PrefillParams p) {
+  const int tile = blockIdx.x, s = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  extern __shared__ __align__(16) unsigned char smb[];
+  uint64_t* bar_img = reinterpret_cast<uint64_t*>(smb + PoolPlan::bars);  // [2] slot blocks landed
+  uint64_t* bar_mma = bar_img + 2;                                       // [2] MMAs of a stage done
+  uint64_t* bar_probe = bar_img + 4;                                     // test hook only
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smb + PoolPlan::tmem);
+  float* sc = reinterpret_cast<float*>(smb + PoolPlan::sc);
+  float* ssq = reinterpret_cast<float*>(smb + PoolPlan::ss);
+  __shared__ int s_ok;
+
+  pdl_trigger();
+  pdl_wait();  // x is written by near_kernel
+  if (tid == 0) {
+    s_ok = header_matches(p);
+    for (int b = 0; b < 5; ++b) mbar_init(bar_img + b, 1);
+    mbar_fence_init();
+  }
+  __syncthreads();
+  if (!s_ok) return;
   if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
+  const int l = p.l0 + s / p.B;
+  const long long n0 = static_cast<long long>(tile) * kTile;
+  const int Tt = static_cast<int>(min(static_cast<long long>(kTile), p.n - n0));
+  const int nch = p.H / kBlk;
+  const float* xrow0 = p.out + (static_cast<long long>(s) * p.n + n0) * p.H;
+  const unsigned char* img_l = p.slot_img + static_cast<size_t>(l) * nch * 2 * kBlkBytes;
+  bool ok = true;
 
-  const long long tile = ticket / p.n_streams;
-  const int stream = static_cast<int>(ticket % p.n_streams);  // call-relative (layer, seq)
-  const int l = p.l0 + stream / p.B;                          // layer of the state
-  const bool last = (tile == p.tiles_per_stream - 1);
-  const bool publish = (ticket != p.withhold_tile);
-  const long long gstart = (tile / kGroup) * kGroup;         // first tile of this group
-  const bool group_end = (tile % kGroup == kGroup - 1) && !last;
-
-  unsigned char* blk = p.state + kHeaderBytes +
-                      (static_cast<long long>(p.l0) * p.B + stream) * p.so.stride;
-  if (tid == 0) s_pos = __ldcg(reinterpret_cast<const long long*>(blk + p.so.pos));
+  // Copies of chunk c into stage st: x columns 64c .. 64c+63 of the tile's
+  // rows (rows past the tile are zero) and the slot blocks of the chunk.
+  auto issue_x = [&](int c, int st) {
+    float* xf = reinterpret_cast<float*>(smb + PoolPlan::xf) + st * kBlk * kBlk;
+    for (int i = tid; i < kBlk * kBlk / 4; i += NT) {
+      const int r = i / (kBlk / 4), c4 = (i % (kBlk / 4)) * 4;
+      if (r < Tt) cp_async16(xf + r * kBlk + c4, xrow0 + static_cast<long long>(r) * p.H + c * kBlk + c4);
+      else *reinterpret_cast<float4*>(xf + r * kBlk + c4) = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    cp_async_commit();
+  };
+  auto issue_img = [&](int c, int st) {  // one thread
+    mbar_arrive_expect_tx(bar_img + st, 2u * kBlkBytes);
+    bulk_g2s(smb + PoolPlan::img + st * 2 * kBlkBytes, img_l + static_cast<size_t>(c) * 2 * kBlkBytes,
+             2u * kBlkBytes, bar_img + st);
+  };
+  if (tid == 0) {
+    issue_img(0, 0);
+    if (nch > 1) issue_img(1, 1);
+  }
+  issue_x(0, 0);
+  if (nch > 1) issue_x(1, 1);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const long long pos0 = s_pos;
-  Tin* win_k = reinterpret_cast<Tin*>(blk + p.so.win_k);
-  Tin* win_v = reinterpret_cast<Tin*>(blk + p.so.win_v);
-  float* far = reinterpret_cast<float*>(blk + p.so.far);
-  float* field = reinterpret_cast<float*>(blk + p.so.field);
-  float* ring_sum = reinterpret_cast<float*>(blk + p.so.ring_sum);
-  float* ring = reinterpret_cast<float*>(blk + p.so.ring);
+  const uint32_t idesc = umma_idesc_bf16(kBlk, kSlots, false);
 
-  const long long t0 = pos0 + tile * kTile;  // first position of the tile
-  const int Tt = static_cast<int>(min(static_cast<long long>(kTile), p.n - tile * kTile));
-  const int K = p.K, G = p.G, nkv = p.nkv;
-  const int h0 = rank * HPC;
-  const int g_lo = h0 / G, g_hi = (h0 + HPC - 1) / G;
-  const int NG = g_hi - g_lo + 1;
-  const int own_lo = (h0 + G - 1) / G;  // KV heads whose carries this CTA publishes
-  const float gf = p.gamma_far, ge = p.ema_gamma;
-  const int rowB = p.NGm * D * ESZ + 16;  // padded key/value row in shared memory
-
-  const long long in_row0 = static_cast<long long>(stream) * p.n;  // first input row of the stream
-  const Tin* kin = static_cast<const Tin*>(p.k) + in_row0 * nkv * D;
-  const Tin* vin = static_cast<const Tin*>(p.v) + in_row0 * nkv * D;
-  const Tin* qin = static_cast<const Tin*>(p.q) + in_row0 * p.nq * D;
-
-  unsigned* fs_agg = reinterpret_cast<unsigned*>(p.ws + p.ws_fs_agg);
-  unsigned* fs_incl = reinterpret_cast<unsigned*>(p.ws + p.ws_fs_incl);
-  unsigned* ff_agg = reinterpret_cast<unsigned*>(p.ws + p.ws_ff_agg);
-  unsigned* ff_incl = reinterpret_cast<unsigned*>(p.ws + p.ws_ff_incl);
-  float* agg_s = reinterpret_cast<float*>(p.ws + p.ws_agg_s);
-  float* incl_s = reinterpret_cast<float*>(p.ws + p.ws_incl_s);
-  float* agg_f = reinterpret_cast<float*>(p.ws + p.ws_agg_f);
-  float* incl_f = reinterpret_cast<float*>(p.ws + p.ws_incl_f);
-  float* halo_ws = reinterpret_cast<float*>(p.ws + p.ws_halo);
-
-  // Slot of absolute position j >= 0 in the k-slot window.
-  auto wslot = [&](long long j) -> long long { return j % K; };
-  // Key row of absolute position j >= 0 for KV head g: from the input if it
-  // belongs to this call, else from window slot j mod k (the state holds
-  // positions pos0-k .. pos0-1).
-  auto key_row = [&](long long j, int g) -> const Tin* {
-    return (j >= pos0) ? kin + ((j - pos0) * nkv + g) * D : win_k + (wslot(j) * nkv + g) * D;
-  };
-  auto val_row = [&](long long j, int g) -> const Tin* {
-    return (j >= pos0) ? vin + ((j - pos0) * nkv + g) * D : win_v + (wslot(j) * nkv + g) * D;
-  };
-  // Byte offset of element (c, d) in a packed [kSpan x D] key/value block:
-  // 8 x 16-byte core matrices, the next span-row group 128 bytes on, the next
-  // 8 dims kSpanR8 * 128 bytes on.  The same block is the K-major B of q·K^T
-  // and the MN-major B of P·V.
-  auto kv_off = [](int c, int d) -> int {
-    return ((d >> 3) * kSpanR8 + (c >> 3)) * 128 + (c & 7) * 16 + (d & 7) * 2;
-  };
-  const int kvblk = kSpan * D * 2;
-  auto evictions = [&](long long a, int len) -> int {  // positions p in [a, a+len) with p >= k
-    const long long lo = a > K ? a : static_cast<long long>(K);
-    const long long hi = a + len;
-    return hi > lo ? static_cast<int>(hi - lo) : 0;
-  };
-  auto ticket_of = [&](long long j) -> long long { return j * p.n_streams + stream; };
-
-  // ---- staging of block `bi` of key/value rows (and the queries with block 0)
-  const long long kv_start = t0 - K;                       // position of block row 0
-  const int kv_rows = Tt + K;                              // positions t0-k .. t0+Tt-1
-  const int n_blocks = (kv_rows + p.KB - 1) / p.KB;
-  auto issue_block = [&](int bi) {
-    if (warp != 0) return;
-    const long long bs = kv_start + static_cast<long long>(bi) * p.KB;
-    const int rows = min(p.KB, kv_rows - bi * p.KB);
-    const long long first_valid = bs < 0 ? -bs : 0;      // rows at negative positions stay unused
-    const int valid = rows > first_valid ? rows - static_cast<int>(first_valid) : 0;
-    const unsigned row_bytes = static_cast<unsigned>(NG * D * ESZ);
-    unsigned bytes = tc ? 0u : 2u * row_bytes * valid;
-    if (bi == 0) {
-      if (!tc) bytes += static_cast<unsigned>(Tt * HS * ESZ);
-      if (gstart == 0) bytes += static_cast<unsigned>(HS * 4);
-      if (tile == 0)
-        for (int r = 0; r < kHalo; ++r)
-          if (t0 - kHalo + r >= 0) bytes += static_cast<unsigned>(HS * 4);
-    }
-    fence_proxy_async_smem();
-    if (lane == 0) mbar_arrive_expect_tx(bar_kv, bytes);
-    __syncwarp();
-    for (int r = static_cast<int>(first_valid) + lane; r < (tc ? 0 : rows); r += 32) {
-      const long long j = bs + r;
-      const Tin* ks = (j >= pos0) ? kin + ((j - pos0) * nkv + g_lo) * D : win_k + (wslot(j) * nkv + g_lo) * D;
-      const Tin* vs = (j >= pos0) ? vin + ((j - pos0) * nkv + g_lo) * D : win_v + (wslot(j) * nkv + g_lo) * D;
-      bulk_g2s(kb + r * rowB, ks, row_bytes, bar_kv);
-      bulk_g2s(vb + r * rowB, vs, row_bytes, bar_kv);
-    }
-    if (bi == 0) {
-      for (int r = lane; r < (tc ? 0 : Tt); r += 32)
-        bulk_g2s(qst + r * HS, qin + ((t0 - pos0 + r) * p.nq + h0) * D,
-                 static_cast<unsigned>(HS * ESZ), bar_kv);
-      // carries from the state, read before this tile publishes anything
-      // (the stream's last tile overwrites them once all tiles have)
-      if (gstart == 0 && lane == 0) bulk_g2s(fcar, field + rank * HS, static_cast<unsigned>(HS * 4), bar_kv);
-      if (tile == 0 && lane < kHalo && t0 - kHalo + lane >= 0)
-        bulk_g2s(halo + lane * HS, ring + static_cast<size_t>((t0 - kHalo + lane) % kRing) * p.H + rank * HS,
-                 static_cast<unsigned>(HS * 4), bar_kv);
-    }
-  };
-  issue_block(0);
-  if (tile == 0)  // ring rows before position 0 are zero
-    for (int idx = tid; idx < kHalo * HS; idx += NT)
-      if (t0 - kHalo + idx / HS < 0) halo[idx] = 0.f;
-  // Query block of head hh for the tensor-core near field: loads (rows past
-  // the tile are zero) and packed stores [64 x D], split so the loads of the
-  // next head overlap the current head's MMAs.
-  constexpr int kQChunks = (kTile * (D / 8) + NT - 1) / NT;  // 16-byte chunks per thread
-  auto q_load = [&](int hh, uint4 (&val)[kQChunks]) {
-#pragma unroll
-    for (int u = 0; u < kQChunks; ++u) {
-      const int idx = u * NT + tid;
-      const int d8 = idx / kTile, r = idx % kTile;
-      val[u] = make_uint4(0u, 0u, 0u, 0u);
-      if (idx < kTile * (D / 8) && r < Tt)
-        val[u] = *reinterpret_cast<const uint4*>(qin + ((t0 - pos0 + r) * p.nq + h0 + hh) * D + d8 * 8);
-    }
-  };
-  auto q_store = [&](const uint4 (&val)[kQChunks]) {
-#pragma unroll
-    for (int u = 0; u < kQChunks; ++u) {
-      const int idx = u * NT + tid;
-      if (idx < kTile * (D / 8)) *reinterpret_cast<uint4*>(qa + blk_off(idx % kTile, (idx / kTile) * 8)) = val[u];
-    }
-  };
-  if constexpr (ESZ == 2) {
-    if (tc) {
-      // Head 0's query block and the key and value rows of the span
-      // (positions t0-16 .. t0+63) for every KV head of the CTA, packed for
-      // the MMAs; rows before position 0 or past the tile are zero.  One
-      // pass of 16-byte loads, eight in flight per thread.
-      constexpr int D8 = D / 8;
-      const int per = kSpan * D8;
-      const int nq_chunks = kTile * D8;
-      const int total = nq_chunks + 2 * NG * per;
-      for (int b0 = 0; b0 < total; b0 += 8 * NT) {
-        uint4 val[8];
-        int dst[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int idx = b0 + u * NT + tid;
-          val[u] = make_uint4(0u, 0u, 0u, 0u);
-          dst[u] = -1;
-          if (idx < nq_chunks) {
-            const int d8 = idx / kTile, r = idx % kTile;
-            dst[u] = pl.qa + blk_off(r, d8 * 8);  // offsets from the shared-memory base
-            if (r < Tt)
-              val[u] = *reinterpret_cast<const uint4*>(qin + ((t0 - pos0 + r) * p.nq + h0) * D + d8 * 8);
-          } else if (idx < total) {
-            const int kvi = idx - nq_chunks;
-            const int which = kvi / (NG * per), rem = kvi % (NG * per);
-            const int gg = rem / per, r2 = rem % per;
-            const int d8 = r2 / kSpan, c = r2 % kSpan;
-            const long long j = kv_start + c;
-            dst[u] = pl.kvp + (which * p.NGm + gg) * kvblk + kv_off(c, d8 * 8);
-            if (j >= 0 && c < kv_rows) {
-              const Tin* row = which ? val_row(j, g_lo + gg) : key_row(j, g_lo + gg);
-              val[u] = *reinterpret_cast<const uint4*>(row + d8 * 8);
-            }
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < 8; ++u)
-          if (dst[u] >= 0) *reinterpret_cast<uint4*>(smb + dst[u]) = val[u];
-      }
-      for (int i = tid; i < 2 * kTile * kSpan * 2 / 16; i += NT)  // P blocks start at zero
-        reinterpret_cast<uint4*>(pa)[i] = make_uint4(0u, 0u, 0u, 0u);
-    }
-  }
-  if (!tc)  // running state of the near field (overlaps the copies in flight)
-    for (int i = tid; i < kTile * HPC; i += NT) {
-      mrun[i] = -INFINITY;
-      lrun[i] = 0.f;
-    }
-  for (int i = tid; i < kTile * XS; i += NT) xs[i] = 0.f;
-  if (!mbar_wait_bounded(bar_kv, 0, kMbarPollLimit, p.err)) s_bad = 1;
-  __syncthreads();  // the packed blocks and zeroed rows written above are read by other threads
-  // Keys that leave the window at the tile's tokens are rows 0 .. Tt-1 of the
-  // staged span when the first block covers them; otherwise read them from
-  // global memory.
-  bool ev_staged = tc || p.KB >= Tt;
-  // Folds the keys that leave the window at tokens r of [r_lo, r_hi) with
-  // r >= r_from into s (EWMA), calling visit(r, s) after every token; staged
-  // rows or global memory.
-  auto scan_evicted = [&](int gg, int i, int r_lo, int r_hi, int r_from, float s,
-                          auto&& visit) -> float {
-    if (ev_staged && tc) {  // packed key block: span row r is position t0 - k + r
-      const unsigned char* kg = kvp + gg * kvblk;
-      for (int r = r_lo; r < r_hi; ++r) {
-        if (r >= r_from) s = ewma(gf, s, to_f32<Tin>(*reinterpret_cast<const Tin*>(kg + kv_off(r, i))));
-        visit(r, s);
-      }
-    } else if (ev_staged) {
-      const Tin* col = reinterpret_cast<const Tin*>(kb) + gg * D + i;
-      const int pitch = rowB / ESZ;
-      for (int r = r_lo; r < r_hi; ++r) {
-        if (r >= r_from) s = ewma(gf, s, to_f32<Tin>(col[r * pitch]));
-        visit(r, s);
-      }
-    } else {
-      for (int r0 = r_lo; r0 < r_hi; r0 += kEvChunk) {
-        float ev[kEvChunk];
-#pragma unroll
-        for (int u = 0; u < kEvChunk; ++u)
-          ev[u] = (r0 + u < r_hi && r0 + u >= r_from) ? to_f32<Tin>(key_row(t0 + r0 + u - K, g_lo + gg)[i]) : 0.f;
-#pragma unroll
-        for (int u = 0; u < kEvChunk; ++u) {
-          const int r = r0 + u;
-          if (r < r_hi) {
-            if (r >= r_from) s = ewma(gf, s, ev[u]);
-            visit(r, s);
-          }
-        }
-      }
-    }
-    return s;
-  };
-
-  // ---- (A) far field: this tile's aggregate of the keys leaving the window.
-  // The tile's tokens split into nseg (1, 2 or 4) segments per (KV head, dim)
-  // as the threads allow; each segment is folded from zero, then the
-  // segments are combined in order: fold(c, seg) = gamma^(evictions) c + agg.
-  const int r_ev = static_cast<int>(max(0LL, min(static_cast<long long>(Tt), K - t0)));  // first token that evicts
-  const int ne = NG * D;
-  int nseg = 1;
-  while (nseg < 4 && ne * nseg * 2 <= NT) nseg *= 2;
-  const int seg_len = kTile / nseg;
-  auto seg_ev = [&](int sg) -> int {  // evicting tokens of segment sg
-    const int a = max(sg * seg_len, r_ev), b = min(Tt, (sg + 1) * seg_len);
-    return b > a ? b - a : 0;
-  };
-  if (tid <= kTile) s_gpn[tid] = powf(gf, static_cast<float>(tid));
-  if (tid < ne * nseg) {
-    const int elem = tid % ne, sg = tid / ne;
-    segA[sg * ne + elem] = scan_evicted(elem / D, elem % D, sg * seg_len, min(Tt, (sg + 1) * seg_len),
-                                        r_ev, 0.f, [](int, float) {});
-  }
-  __syncthreads();
-  for (int idx = tid; idx < ne; idx += NT) {
-    const int g = g_lo + idx / D, i = idx % D;
-    float a = 0.f;
-    for (int sg = 0; sg < nseg; ++sg) a = fmaf(s_gpn[seg_ev(sg)], a, segA[sg * ne + idx]);
-    sagg[idx] = a;
-    if (g >= own_lo && publish) agg_s[(ticket * nkv + g) * D + i] = a;
-  }
-  __syncthreads();
-  if (tid == 0 && publish) {
-    __threadfence();
-    for (int g = own_lo; g <= g_hi; ++g) st_release_u32(&fs_agg[ticket * nkv + g], 1u);
-  }
-
-  // ---- (B) near field [P1 §2.1 eq. O_near] ---------------------------------
-  bool near_done = false;
-  if constexpr (ESZ == 2) {
-    if (tc) {
-      // On the tensor cores, one query head at a time:
-      //   S[64 x kSpan] = Q_h . K_g^T (tensor memory, columns 0..kSpan-1);
-      //   softmax over the band of each row (token r sees span rows r+1 ..
-      //   r+k, positions t0+r-k+1 .. t0+r, none before position 0);
-      //   P split into bf16 hi + lo (about 16 significant bits);
-      //   O[64 x D] = P_hi . V_g + P_lo . V_g (columns kTmemO..), into the x tile.
-      // Accumulator row r sits in lane (r % 16) + 32 (r / 16); warp w (w < 4)
-      // loads span columns 32 (w / 2) .. + 63, which hold the bands of its 16 rows.
-      const uint32_t idesc_qk = umma_idesc_bf16(kTile, kSpan, false);
-      const uint32_t idesc_pv = umma_idesc_bf16(kTile, D, true);
-      const int sp = warp & 3, pbase = 32 * (sp >> 1);
-      const int cmin = kv_start < 0 ? static_cast<int>(-kv_start) : 0;  // first row at position >= 0
-      unsigned char* pa_hi = pa;
-      unsigned char* pa_lo = pa + kTile * kSpan * 2;
-      unsigned nf_par = 0;
-      for (int hh = 0; hh < HPC; ++hh) {
-        const int gg = (h0 + hh) / G - g_lo;
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0) {
-          tc_fence_after();
-          const unsigned char* kg = kvp + gg * kvblk;
-#pragma unroll
-          for (int s2 = 0; s2 < D / 16; ++s2)
-            umma_bf16(tmem, umma_desc(qa + s2 * 2048, 1024, 128),
-                      umma_desc(kg + s2 * 2 * kSpanR8 * 128, kSpanR8 * 128, 128), idesc_qk, s2 > 0);
-          umma_commit(bar_nf);
-        }
-        uint4 qn[kQChunks];  // the next head's queries, in flight during the MMAs
-        if (hh + 1 < HPC) q_load(hh + 1, qn);
-        if (!mbar_wait_bounded(bar_nf, nf_par, kMbarPollLimit, p.err)) s_bad = 1;
-        nf_par ^= 1u;
-        tc_fence_after();
-        if (hh + 1 < HPC) q_store(qn);  // the score MMAs have read the query block
-        if (warp < 4) {
-          float v[64];
-          tmem_ld32(tmem + (static_cast<uint32_t>(32 * sp) << 16) + pbase, *reinterpret_cast<float(*)[32]>(v));
-          tmem_ld32(tmem + (static_cast<uint32_t>(32 * sp) << 16) + pbase + 32,
-                    *reinterpret_cast<float(*)[32]>(v + 32));
-          // The bands of rows 16 sp .. 16 sp + 15 lie in span columns
-          // 16 sp .. 16 sp + 31: loaded columns J0 .. J0 + 31 with
-          // J0 = 16 (sp & 1); only those are scored and written (the other
-          // P columns stay zero).
-          auto band = [&](auto j0_c) {
-            constexpr int J0 = decltype(j0_c)::value;
-            const int r = 16 * sp + lane;
-            float mx = -INFINITY;
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const int c = pbase + J0 + j;
-              const bool in = c >= r + 1 && c <= r + K && c >= cmin;
-              v[J0 + j] = in ? v[J0 + j] * p.score_scale : -INFINITY;
-              mx = fmaxf(mx, v[J0 + j]);
-            }
-            float sum = 0.f;
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              v[J0 + j] = __expf(v[J0 + j] - mx);  // 0 outside the band
-              sum += v[J0 + j];
-            }
-            const float inv = 1.f / sum;
-#pragma unroll
-            for (int g8 = 0; g8 < 4; ++g8) {
-              uint32_t hw[4], lw[4];
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                __nv_bfloat16 h0b, l0b, h1b, l1b;
-                split_bf16(v[J0 + 8 * g8 + 2 * e] * inv, h0b, l0b);
-                split_bf16(v[J0 + 8 * g8 + 2 * e + 1] * inv, h1b, l1b);
-                hw[e] = static_cast<uint32_t>(__bfloat16_as_ushort(h0b)) |
-                        (static_cast<uint32_t>(__bfloat16_as_ushort(h1b)) << 16);
-                lw[e] = static_cast<uint32_t>(__bfloat16_as_ushort(l0b)) |
-                        (static_cast<uint32_t>(__bfloat16_as_ushort(l1b)) << 16);
-              }
-              const int off = blk_off(r, pbase + J0 + 8 * g8);
-              *reinterpret_cast<uint4*>(pa_hi + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-              *reinterpret_cast<uint4*>(pa_lo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-            }
-          };
-          if (lane < 16) {
-            if (sp & 1) band(std::integral_constant<int, 16>{});
-            else band(std::integral_constant<int, 0>{});
-          }
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0) {
-          tc_fence_after();
-          const unsigned char* vg = kvp + (p.NGm + gg) * kvblk;
-#pragma unroll
-          for (int s2 = 0; s2 < kSpan / 16; ++s2) {
-            const uint64_t bv = umma_desc(vg + s2 * 256, 128, kSpanR8 * 128);
-            umma_bf16(tmem + kTmemO, umma_desc(pa_hi + s2 * 2048, 1024, 128), bv, idesc_pv, s2 > 0);
-            umma_bf16(tmem + kTmemO, umma_desc(pa_lo + s2 * 2048, 1024, 128), bv, idesc_pv, true);
-          }
-          umma_commit(bar_nf);
-        }
-        if (!mbar_wait_bounded(bar_nf, nf_par, kMbarPollLimit, p.err)) s_bad = 1;
-        nf_par ^= 1u;
-        tc_fence_after();
-        {  // O rows into the x tile: warps w and w + 4 take halves of the head
-          const int colh = (warp >> 2) * (D / 2);
-          const int r = 16 * sp + lane;
-#pragma unroll
-          for (int c0 = 0; c0 < D / 2; c0 += 32) {
-            float v[32];
-            tmem_ld32(tmem + (static_cast<uint32_t>(32 * sp) << 16) + kTmemO + colh + c0, v);
-            if (lane < 16 && r < Tt) {
-              float* dst = xs + r * XS + hh * D + colh + c0;
-#pragma unroll
-              for (int j = 0; j < 32; j += 4)
-                *reinterpret_cast<float4*>(dst + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
-            }
-          }
-        }
-        tc_fence_before();
-        __syncthreads();
-      }
-      near_done = true;
-    }
-  }
-  if (!near_done) {  // on the CUDA cores, block by block
-    for (int bi = 0; bi < n_blocks; ++bi) {
-      if (bi > 0 && !mbar_wait_bounded(bar_kv, bi & 1, kMbarPollLimit, p.err)) s_bad = 1;
-      const long long bs = kv_start + static_cast<long long>(bi) * p.KB;
-      const long long be = bs + min(p.KB, kv_rows - bi * p.KB);  // exclusive
-      if (K <= 16)
-        near_block<Tin, D, 16>(qst, kb, vb, xs, mrun, lrun, rowB, HS, XS, HPC, G, g_lo, K, t0, Tt,
-                               bs, be, p.score_scale, h0, warp, lane);
-      else
-        near_block<Tin, D, 32>(qst, kb, vb, xs, mrun, lrun, rowB, HS, XS, HPC, G, g_lo, K, t0, Tt,
-                               bs, be, p.score_scale, h0, warp, lane);
-      __syncthreads();  // the block buffers are free again
-      if (bi + 1 < n_blocks) issue_block(bi + 1);
-    }
-    if (n_blocks > 1) ev_staged = false;  // the staged rows were replaced by later blocks
-    // normalise: O = acc / den
-    for (int i = tid; i < Tt * HPC; i += NT) lrun[i] = 1.f / lrun[i];
-    __syncthreads();
-    for (int r = warp; r < Tt; r += NW)
-      for (int c = lane; c < HS; c += 32) xs[r * XS + c] *= lrun[r * HPC + c / D];
-  }
-
-  // ---- (C) far field carry-in (deterministic look-back), then the scan --
-  // carry = INCL(end of previous group) or the state, folded with the
-  // aggregates of the group's earlier tiles in order.  Warp 0 polls all the
-  // flags at once (lane per flag); then every carry element loads all its
-  // terms at once and folds them in order.
-  const int n_prev = static_cast<int>(tile - gstart);  // earlier tiles of the group (< kGroup)
-  {
-    if (warp == 0) {
-      const int n_flags = (n_prev + (gstart > 0 ? 1 : 0)) * NG;
-      for (int f = lane; f < n_flags; f += 32) {
-        const int gg = f % NG, jj = f / NG;
-        const unsigned* fl = (jj < n_prev) ? &fs_agg[ticket_of(gstart + jj) * nkv + g_lo + gg]
-                                           : &fs_incl[ticket_of(gstart - 1) * nkv + g_lo + gg];
-        wait_flag(fl, p.spin_limit, p.err);
-      }
-    }
-    __syncthreads();
-    for (int idx = tid; idx < NG * D; idx += NT) {
-      const int g = g_lo + idx / D, i = idx % D;
-      float terms[kGroup];
-#pragma unroll
-      for (int jj = 0; jj < kGroup - 1; ++jj)
-        terms[jj] = (jj < n_prev) ? __ldcg(agg_s + (ticket_of(gstart + jj) * nkv + g) * D + i) : 0.f;
-      float acc = (gstart == 0) ? far[g * D + i] : __ldcg(incl_s + (ticket_of(gstart - 1) * nkv + g) * D + i);
-#pragma unroll
-      for (int jj = 0; jj < kGroup - 1; ++jj)
-        if (jj < n_prev)
-          acc = fmaf(s_gpn[evictions(pos0 + (gstart + jj) * kTile, kTile)], acc, terms[jj]);
-      sst[idx] = acc;
-    }
-    __syncthreads();
-    if (group_end && publish) {
-      const float mul = s_gpn[evictions(t0, Tt)];
-      for (int idx = tid; idx < NG * D; idx += NT) {
-        const int g = g_lo + idx / D, i = idx % D;
-        if (g >= own_lo) incl_s[(ticket * nkv + g) * D + i] = fmaf(mul, sst[idx], sagg[idx]);
-      }
-      __syncthreads();
-      if (tid == 0) {
-        __threadfence();
-        for (int g = own_lo; g <= g_hi; ++g) st_release_u32(&fs_incl[ticket * nkv + g], 1u);
-      }
-    }
-  }
-  // scan: S_t per token, x = O_near + alpha_far * S_t  [P1 §2.1 eq. O];
-  // segment sg starts from the carry folded with the earlier segments'
-  // aggregates.  The last segment leaves S at the tile end in its own
-  // segA entry, which no other thread reads.
-  if (tid < ne * nseg) {
-    const int elem = tid % ne, sg = tid / ne;
-    const int gg = elem / D, i = elem % D, g = g_lo + gg;
-    const int hh_lo = max(0, g * G - h0), hh_hi = min(HPC, (g + 1) * G - h0);
-    float c = sst[elem];
-    for (int s2 = 0; s2 < sg; ++s2) c = fmaf(s_gpn[seg_ev(s2)], c, segA[s2 * ne + elem]);
-    c = scan_evicted(gg, i, sg * seg_len, min(Tt, (sg + 1) * seg_len), r_ev, c,
-                     [&](int r, float sv) {
-                       for (int hh = hh_lo; hh < hh_hi; ++hh) {
-                         float* xp = xs + r * XS + hh * D + i;
-                         *xp = fmaf(p.alpha_far, sv, *xp);
-                       }
-                     });
-    if (sg == nseg - 1) segA[sg * ne + elem] = c;
-  }
-  __syncthreads();
-  // Slot blocks (bf16 hi/lo, laid out for both pool MMAs); the staging
-  // buffers are free now.
-  const unsigned char* img = p.slot_img +
-      (static_cast<size_t>(l) * (p.H / kBlk) + static_cast<size_t>(rank) * nch) * 2 * kBlkBytes;
-  if (tid == 0) {
-    fence_proxy_async_smem();
-    mbar_arrive_expect_tx(bar_sl, static_cast<unsigned>(nch * 2 * kBlkBytes));
-    for (int c = 0; c < nch; ++c)
-      bulk_g2s(simg + c * 2 * kBlkBytes, img + static_cast<size_t>(c) * 2 * kBlkBytes,
-               2u * kBlkBytes, bar_sl);
-  }
-
-  // ---- (D) EMA field aggregate; tail rows for the successor -------------
-  // (Tiles of the first group staged the state field, and tile 0 the state
-  // ring rows, with the first key block.)
-  for (int e = tid; e < HS; e += NT) {
-    float a = 0.f;
-    for (int r = 0; r < Tt; ++r) a = ewma(ge, a, xs[r * XS + e]);
-    if (publish) {
-      agg_f[ticket * p.H + rank * HS + e] = a;
-      if (!last)
-        for (int r = 0; r < kHalo; ++r)
-          halo_ws[(ticket * kHalo + r) * p.H + rank * HS + e] = xs[(Tt - kHalo + r) * XS + e];
-    }
-  }
-  __syncthreads();
-  if (tid == 0 && publish) {
-    __threadfence();
-    st_release_u32(&ff_agg[ticket * p.CS + rank], 1u);
-  }
-
-  // ---- (E) pool scores on the tensor cores [P3 §2.1 channel 3] -----------
-  // scores[T x 64] (tensor memory, columns 0..63) = sum over 64-column chunks
-  // of x_chunk . slot_chunk^T, each as hi*hi + hi*lo + lo*hi.
-  const uint32_t idesc_s = umma_idesc_bf16(kBlk, kSlots, false);
-  const uint32_t idesc_c = umma_idesc_bf16(kBlk, kCW, true);
-  unsigned char* xhi = xw;
-  unsigned char* xlo = xw + kBlkBytes;
+  // |x|^2: thread tid covers columns 4*(tid%16) .. +3 of rows tid/16 + 16m.
+  float sq[4] = {0.f, 0.f, 0.f, 0.f};
   for (int c = 0; c < nch; ++c) {
-    if (c >= 1)  // the MMAs of chunk c-1 have finished reading the x block
-      if (!mbar_wait_bounded(bar_ms, (c - 1) & 1, kMbarPollLimit, p.err)) s_bad = 1;
-    stage_split_block(xs + c * kBlk, XS, xhi, xlo, tid, NT);
+    const int st = c & 1;
+    const unsigned ph = static_cast<unsigned>((c >> 1) & 1);
+    if (c + 1 < nch) cp_async_wait<1>();
+    else cp_async_wait<0>();
+    __syncthreads();  // x chunk c visible to all threads
+    // The split blocks of stage st were read by the MMAs of chunk c-2.
+    if (c >= 2 && !mbar_wait_bounded(bar_mma + st, ph ^ 1u, kMbarPollLimit, p.err)) ok = false;
+    const float* xf = reinterpret_cast<const float*>(smb + PoolPlan::xf) + st * kBlk * kBlk;
+    unsigned char* xhi = smb + PoolPlan::xsp + st * 2 * kBlkBytes;
+    unsigned char* xlo = xhi + kBlkBytes;
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int i = m * NT + tid;
+      const int r = i / (kBlk / 4), c4 = (i % (kBlk / 4)) * 4;
+      const float4 v = *reinterpret_cast<const float4*>(xf + r * kBlk + c4);
+      sq[m] = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, sq[m]))));
+      __nv_bfloat16 hh[4], ll[4];
+      split_bf16(v.x, hh[0], ll[0]);
+      split_bf16(v.y, hh[1], ll[1]);
+      split_bf16(v.z, hh[2], ll[2]);
+      split_bf16(v.w, hh[3], ll[3]);
+      const int off = blk_off(r, c4);
+      *reinterpret_cast<uint2*>(xhi + off) = *reinterpret_cast<const uint2*>(hh);
+      *reinterpret_cast<uint2*>(xlo + off) = *reinterpret_cast<const uint2*>(ll);
+    }
     fence_proxy_async_smem();
-    __syncthreads();
+    tc_fence_before();
+    __syncthreads();  // split blocks written; x chunk c consumed
+    if (c + 2 < nch) issue_x(c + 2, st);
     if (tid == 0) {
-      if (c == 0 && !mbar_wait_bounded(bar_sl, 0, kMbarPollLimit, p.err)) s_bad = 1;
+      if (!mbar_wait_bounded(bar_img + st, ph, kMbarPollLimit, p.err)) ok = false;
       tc_fence_after();
-      const unsigned char* shi = simg + c * 2 * kBlkBytes;
+      const unsigned char* shi = smb + PoolPlan::img + st * 2 * kBlkBytes;
       const unsigned char* slo = shi + kBlkBytes;
 #pragma unroll
-      for (int s = 0; s < kBlk / 16; ++s) {
-        const uint64_t ah = umma_desc(xhi + s * 2048, 1024, 128), al = umma_desc(xlo + s * 2048, 1024, 128);
-        const uint64_t bh = umma_desc(shi + s * 2048, 1024, 128), bl = umma_desc(slo + s * 2048, 1024, 128);
-        umma_bf16(tmem, ah, bh, idesc_s, c > 0 || s > 0);
-        umma_bf16(tmem, ah, bl, idesc_s, true);
-        umma_bf16(tmem, al, bh, idesc_s, true);
+      for (int k = 0; k < kBlk / 16; ++k) {
+        const uint64_t ah = umma_desc(xhi + k * 2048, 1024, 128), al = umma_desc(xlo + k * 2048, 1024, 128);
+        const uint64_t bh = umma_desc(shi + k * 2048, 1024, 128), bl = umma_desc(slo + k * 2048, 1024, 128);
+        umma_bf16(tmem, ah, bh, idesc, c > 0 || k > 0);
+        umma_bf16(tmem, ah, bl, idesc, true);
+        umma_bf16(tmem, al, bh, idesc, true);
       }
-      umma_commit(bar_ms);
+      umma_commit(bar_mma + st);
+      if (c + 2 < nch) {  // the slot blocks of stage st are free once these MMAs finish
+        if (!mbar_wait_bounded(bar_mma + st, ph, kMbarPollLimit, p.err)) ok = false;
+        issue_img(c + 2, st);
+      }
     }
   }
-  if (tid == 0) umma_commit(bar_sd);
-  // |x|^2 per token (CUDA cores) while the tensor cores finish
-  for (int r = warp; r < kTile; r += NW) {
-    float ss = 0.f;
-    for (int e = lane; e < HS; e += 32) ss = fmaf(xs[r * XS + e], xs[r * XS + e], ss);
-    ss = warp_sum(ss);
-    if (lane == 0) part[r * kPartStride + kSlots] = ss;
+  // |x|^2 per row: 16 threads (half a warp) share a row.
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    float v = sq[m];
+    v += __shfl_xor_sync(0xffffffffu, v, 8);
+    v += __shfl_xor_sync(0xffffffffu, v, 4);
+    v += __shfl_xor_sync(0xffffffffu, v, 2);
+    v += __shfl_xor_sync(0xffffffffu, v, 1);
+    if ((tid & 15) == 0) ssq[m * (NT / 16) + tid / 16] = v;
   }
-  if (!mbar_wait_bounded(bar_sd, 0, kMbarPollLimit, p.err)) s_bad = 1;
+  // Test hook: a bounded wait on a barrier that nothing completes.
+  if (tid == 0 && static_cast<long long>(tile) * p.n_streams + s == p.withhold_tile) {
+    mbar_arrive_expect_tx(bar_probe, 16u);
+    mbar_wait_bounded(bar_probe, 0, p.spin_limit, p.err);
+  }
+  {  // wait for the last MMAs (both stages' final commits)
+    const int last = nch - 1;
+    if (!mbar_wait_bounded(bar_mma + (last & 1), static_cast<unsigned>((last >> 1) & 1), kMbarPollLimit, p.err))
+      ok = false;
+    if (nch > 1 && !mbar_wait_bounded(bar_mma + ((last - 1) & 1),
+                                      static_cast<unsigned>(((last - 1) >> 1) & 1), kMbarPollLimit, p.err))
+      ok = false;
+  }
   tc_fence_after();
   {  // accumulator row r (token) sits in lane (r%16) + 32*(r/16) for M = 64
     const int sp = warp & 3, colh = (warp >> 2) * 32;
     float v[32];
     tmem_ld32(tmem + (static_cast<uint32_t>(32 * sp) << 16) + colh, v);
     if (lane < 16) {
-      const int r = 16 * sp + lane;
+      float* dst = sc + (16 * sp + lane) * kScStride + colh;
 #pragma unroll
-      for (int j = 0; j < 32; ++j) part[r * kPartStride + colh + j] = v[j];
+      for (int j = 0; j < 32; ++j) dst[j] = v[j];
     }
   }
   tc_fence_before();
-
-  // ---- (F) EMA field carry-in (deterministic look-back); tail rows ------
-  {
-    if (warp == 0) {
-      const int n_flags = n_prev + (gstart > 0 ? 1 : 0);
-      for (int f = lane; f < n_flags; f += 32) {
-        const unsigned* fl = (f < n_prev) ? &ff_agg[ticket_of(gstart + f) * p.CS + rank]
-                                          : &ff_incl[ticket_of(gstart - 1) * p.CS + rank];
-        wait_flag(fl, p.spin_limit, p.err);
-      }
-      // the predecessor's tail rows come with its aggregate (or, across a
-      // group boundary, with the inclusive value published after it)
-    }
-    __syncthreads();
-    const float mul_full = powf(ge, static_cast<float>(kTile));
-    for (int e = tid; e < HS; e += NT) {
-      float terms[kGroup];
-#pragma unroll
-      for (int jj = 0; jj < kGroup - 1; ++jj)
-        terms[jj] = (jj < n_prev) ? __ldcg(agg_f + ticket_of(gstart + jj) * p.H + rank * HS + e) : 0.f;
-      float acc = (gstart == 0) ? fcar[e] : __ldcg(incl_f + ticket_of(gstart - 1) * p.H + rank * HS + e);
-#pragma unroll
-      for (int jj = 0; jj < kGroup - 1; ++jj)
-        if (jj < n_prev) acc = fmaf(mul_full, acc, terms[jj]);
-      fcar[e] = acc;
-    }
-    if (tile > 0)  // x rows of the 15 tokens before the tile, from the predecessor
-      for (int idx = tid; idx < kHalo * HS; idx += NT) {
-        const int r = idx / HS, e = idx % HS;
-        halo[idx] = __ldcg(halo_ws + (ticket_of(tile - 1) * kHalo + r) * p.H + rank * HS + e);
-      }
-    __syncthreads();
-    if (group_end && publish) {
-      const float mul = powf(ge, static_cast<float>(Tt));
-      for (int e = tid; e < HS; e += NT) {
-        const long long o = ticket * p.H + rank * HS + e;
-        incl_f[o] = fmaf(mul, fcar[e], agg_f[o]);
-      }
-      __syncthreads();
-      if (tid == 0) {
-        __threadfence();
-        st_release_u32(&ff_incl[ticket * p.CS + rank], 1u);
-      }
-    }
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
   }
 
-  // ---- (G) cluster reduce-scatter of the pool sums, softmax(cos/T) -------
-  cluster.sync();
-  {
-    const float* nrm = p.slot_norm + static_cast<size_t>(l) * kSlots;
-    const float n0 = nrm[lane], n1 = nrm[lane + 32];
-    for (int r = rank + p.CS * warp; r < Tt; r += p.CS * NW) {
-      // every rank's partials in flight at once, added in rank order
-      float v0[kMaxCluster], v1[kMaxCluster], vs[kMaxCluster];
-#pragma unroll
-      for (int q = 0; q < kMaxCluster; ++q) {
-        const bool in = q < p.CS;
-        const float* rp = cluster.map_shared_rank(part, in ? q : 0) + r * kPartStride;
-        v0[q] = in ? rp[lane] : 0.f;
-        v1[q] = in ? rp[lane + 32] : 0.f;
-        vs[q] = in ? rp[kSlots] : 0.f;
-      }
-      float d0 = 0.f, d1 = 0.f, ss = 0.f;
-#pragma unroll
-      for (int q = 0; q < kMaxCluster; ++q) {
-        d0 += v0[q];
-        d1 += v1[q];
-        ss += vs[q];
-      }
-      const float nx = fmaxf(sqrtf(ss), kNormFloor);
-      const float c0 = d0 / (nx * n0) * p.inv_temp;
-      const float c1 = d1 / (nx * n1) * p.inv_temp;
+  // softmax(cos/T) per token [P3 §2.1 channel 3]; weights split into bf16
+  // hi/lo blocks in the MMA operand layout (in shared memory, where the x
+  // split blocks were), then copied to the workspace.  Rows past the tile
+  // get zero weights.
+  const float* nrm = p.slot_norm + static_cast<size_t>(l) * kSlots;
+  const float n0v = nrm[lane], n1v = nrm[lane + 32];
+  unsigned char* wsm = smb + PoolPlan::xsp;
+  for (int r = warp; r < kTile; r += NW) {
+    float w0 = 0.f, w1 = 0.f;
+    if (r < Tt) {
+      const float nx = fmaxf(sqrtf(ssq[r]), kNormFloor);
+      const float c0 = sc[r * kScStride + lane] / (nx * n0v) * p.inv_temp;
+      const float c1 = sc[r * kScStride + lane + 32] / (nx * n1v) * p.inv_temp;
       const float mx = warp_max_redux(fmaxf(c0, c1));
       const float e0 = expf(c0 - mx), e1 = expf(c1 - mx);
       const float inv = 1.f / warp_sum(e0 + e1);
-      __nv_bfloat16 h0, l0, h1, l1;
-      split_bf16(e0 * inv, h0, l0);
-      split_bf16(e1 * inv, h1, l1);
-      const int o0 = blk_off(r, lane), o1 = blk_off(r, lane + 32);
-      for (int q = 0; q < p.CS; ++q) {
-        unsigned char* wq = cluster.map_shared_rank(xw, q);  // the x blocks are dead everywhere
-        *reinterpret_cast<__nv_bfloat16*>(wq + o0) = h0;
-        *reinterpret_cast<__nv_bfloat16*>(wq + kBlkBytes + o0) = l0;
-        *reinterpret_cast<__nv_bfloat16*>(wq + o1) = h1;
-        *reinterpret_cast<__nv_bfloat16*>(wq + kBlkBytes + o1) = l1;
-      }
+      w0 = e0 * inv;
+      w1 = e1 * inv;
     }
-    // rows of tokens past the tile end feed MMA rows that are never read
-    fence_proxy_async_cluster();
+    __nv_bfloat16 h0, l0, h1, l1;
+    split_bf16(w0, h0, l0);
+    split_bf16(w1, h1, l1);
+    const int o0 = blk_off(r, lane), o1 = blk_off(r, lane + 32);
+    *reinterpret_cast<__nv_bfloat16*>(wsm + o0) = h0;
+    *reinterpret_cast<__nv_bfloat16*>(wsm + kBlkBytes + o0) = l0;
+    *reinterpret_cast<__nv_bfloat16*>(wsm + o1) = h1;
+    *reinterpret_cast<__nv_bfloat16*>(wsm + kBlkBytes + o1) = l1;
   }
-  cluster.sync();
-
-  // ---- (H) semantic mix on the tensor cores, then per column chunk: ring,
-  // field, fusion, clip, output [P3 §2.1 channels 1–3, §2.2].
-  // sem chunk c [T x 64] = w[T x 64] . slot_chunk_c, accumulators alternate
-  // between tensor-memory columns 64..127 and 128..191.
-  unsigned char* whi = xw;  // written by the cluster in (G)
-  unsigned char* wlo = xw + kBlkBytes;
-  fence_proxy_async_smem();
-  tc_fence_before();
   __syncthreads();
-  auto issue_sem = [&](int c) {  // tid 0 only
-    tc_fence_after();
-    const uint32_t dst = tmem + kSlots + (c & 1) * kCW;
-    const unsigned char* shi = simg + c * 2 * kBlkBytes;
-    const unsigned char* slo = shi + kBlkBytes;
-#pragma unroll
-    for (int s = 0; s < kSlots / 16; ++s) {
-      const uint64_t ah = umma_desc(whi + s * 2048, 1024, 128), al = umma_desc(wlo + s * 2048, 1024, 128);
-      const uint64_t bh = umma_desc(shi + s * 256, 128, 1024), bl = umma_desc(slo + s * 256, 128, 1024);
-      umma_bf16(dst, ah, bh, idesc_c, s > 0);
-      umma_bf16(dst, ah, bl, idesc_c, true);
-      umma_bf16(dst, al, bh, idesc_c, true);
+  uint4* wblk = reinterpret_cast<uint4*>(
+      p.ws + p.ws_w + (static_cast<long long>(s) * p.tiles_per_stream + tile) * 2 * kBlkBytes);
+  if (ok)
+    for (int i = tid; i < 2 * kBlkBytes / 16; i += NT) wblk[i] = reinterpret_cast<const uint4*>(wsm)[i];
+}
+
+// ======================================================================
+// 3. semantic mix, ring, field, fusion, output and state
+// ======================================================================
+
+struct OutPlan {
+  static constexpr int bars = 0;                          // 5 mbarriers
+  static constexpr int tmem = 64;
+  static constexpr int img = 128;                         // [hi, lo] slot block of the columns
+  static constexpr int wb = img + 2 * kBlkBytes;          // [2][hi, lo] weight blocks
+  static constexpr int xt = wb + 2 * 2 * kBlkBytes;       // [2][64][64] fp32 x tiles
+  static constexpr int halo = xt + 2 * kTile * kBlk * 4;  // [15][64] x before the tile
+  static constexpr int sem = halo + kHalo * kBlk * 4;     // [64][65] sem
+  static constexpr int segc = sem + kTile * kScStride * 4;  // [kSeg][64] field segment aggregates
+  static constexpr int fcar = segc + kSeg * kBlk * 4;     // [64] field at the tile start
+  static constexpr int total = fcar + kBlk * 4;
+};
+
+template <typename Tin>
+__global__ void __launch_bounds__(NT, 2) out_kernel(const PrefillParams p) {
+  const int cb = blockIdx.x, s = blockIdx.y;  // 64-column block, call-relative stream
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  extern __shared__ __align__(16) unsigned char smb[];
+  uint64_t* bar_img = reinterpret_cast<uint64_t*>(smb + OutPlan::bars);
+  uint64_t* bar_w = bar_img + 1;    // [2] weight blocks landed
+  uint64_t* bar_mma = bar_img + 3;  // sem MMAs done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smb + OutPlan::tmem);
+  float* halo = reinterpret_cast<float*>(smb + OutPlan::halo);
+  float* semc = reinterpret_cast<float*>(smb + OutPlan::sem);
+  float* segc = reinterpret_cast<float*>(smb + OutPlan::segc);
+  float* fcar = reinterpret_cast<float*>(smb + OutPlan::fcar);
+  __shared__ int s_ok;
+  __shared__ long long s_pos;
+  __shared__ float s_gseg[kSeg];
+
+  pdl_trigger();
+  pdl_wait();  // weights from pool_kernel (and, before it, x from near_kernel)
+  unsigned char* blk = stream_block(p, s);
+  if (tid == 0) {
+    s_ok = header_matches(p);
+    // the state's position is rewritten by this kernel: read the copy
+    s_pos = reinterpret_cast<const long long*>(p.ws + p.ws_pos)[s];
+    for (int b = 0; b < 4; ++b) mbar_init(bar_img + b, 1);
+    mbar_fence_init();
+  }
+  __syncthreads();
+  if (!s_ok) return;
+  if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
+  const long long pos0 = s_pos;
+  const int l = p.l0 + s / p.B;
+  const int col0 = cb * kBlk;
+  const long long in_row0 = static_cast<long long>(s) * p.n;
+  float* field = reinterpret_cast<float*>(blk + p.so.field);
+  float* ring_sum = reinterpret_cast<float*>(blk + p.so.ring_sum);
+  float* ring = reinterpret_cast<float*>(blk + p.so.ring);
+  const int tiles = p.tiles_per_stream;
+  const unsigned char* wall = p.ws + p.ws_w + static_cast<long long>(s) * tiles * 2 * kBlkBytes;
+  const float ge = p.ema_gamma;
+  const float a_l = p.alpha_layer[l];
+
+  auto tile_rows = [&](int i) -> int {
+    return static_cast<int>(min(static_cast<long long>(kTile), p.n - static_cast<long long>(i) * kTile));
+  };
+  auto issue_x = [&](int i, int st) {
+    float* xt = reinterpret_cast<float*>(smb + OutPlan::xt) + st * kTile * kBlk;
+    const int Tt = tile_rows(i);
+    const float* src = p.out + (in_row0 + static_cast<long long>(i) * kTile) * p.H + col0;
+    for (int c = tid; c < Tt * (kBlk / 4); c += NT) {
+      const int r = c / (kBlk / 4), c4 = (c % (kBlk / 4)) * 4;
+      cp_async16(xt + r * kBlk + c4, src + static_cast<long long>(r) * p.H + c4);
     }
-    umma_commit(bar_mc + (c & 1));
+    cp_async_commit();
+  };
+  auto issue_w = [&](int i, int st) {  // one thread
+    mbar_arrive_expect_tx(bar_w + st, 2u * kBlkBytes);
+    bulk_g2s(smb + OutPlan::wb + st * 2 * kBlkBytes, wall + static_cast<long long>(i) * 2 * kBlkBytes,
+             2u * kBlkBytes, bar_w + st);
   };
   if (tid == 0) {
-    issue_sem(0);
-    if (nch > 1) issue_sem(1);
+    mbar_arrive_expect_tx(bar_img, 2u * kBlkBytes);
+    bulk_g2s(smb + OutPlan::img,
+             p.slot_img + (static_cast<size_t>(l) * (p.H / kBlk) + cb) * 2 * kBlkBytes, 2u * kBlkBytes,
+             bar_img);
+    issue_w(0, 0);
   }
-  const float a_l = p.alpha_layer[l];
-  const bool write_ok = !s_bad;
-  if (tid < kSeg) {
-    const int len = max(0, min(Tt, (tid + 1) * (kTile / kSeg)) - tid * (kTile / kSeg));
-    s_gseg[tid] = powf(ge, static_cast<float>(len));
-  }  // read after the first barrier of the chunk loop below
-  float* out = p.out + (in_row0 + (t0 - pos0)) * p.H + rank * HS;
-  for (int c = 0; c < nch; ++c) {
-    const int buf = c & 1;
-    if (!mbar_wait_bounded(bar_mc + buf, (c >> 1) & 1, kMbarPollLimit, p.err)) s_bad = 1;
-    tc_fence_after();
+  issue_x(0, 0);
+  // x of the 15 positions before the call (state ring; zero before position
+  // 0) and the field carried in, for this block's columns.
+  for (int idx = tid; idx < kHalo * kBlk; idx += NT) {
+    const int q = idx / kBlk, c = idx % kBlk;
+    const long long t = pos0 - kHalo + q;
+    halo[idx] = t >= 0 ? ring[static_cast<size_t>(t % kRing) * p.H + col0 + c] : 0.f;
+  }
+  if (tid < kBlk) fcar[tid] = field[col0 + tid];
+  if (tid < kSeg) s_gseg[tid] = powf(ge, static_cast<float>(kSegLen));
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t idesc = umma_idesc_bf16(kTile, kBlk, true);
+  bool ok = true;
+  if (!mbar_wait_bounded(bar_img, 0, kMbarPollLimit, p.err)) ok = false;
+
+  const int cc = tid % kBlk, sg = tid / kBlk;  // column, token segment
+  for (int i = 0; i < tiles; ++i) {
+    const int st = i & 1;
+    const int Tt = tile_rows(i);
+    const long long t0 = pos0 + static_cast<long long>(i) * kTile;
+    if (i + 1 < tiles) {
+      issue_x(i + 1, st ^ 1);  // stage st^1 was released at the end of tile i-1
+      if (tid == 0) issue_w(i + 1, st ^ 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    // sem[T x 64] = w[T x 64 slots] . slot block [64 slots x 64 columns]
+    if (tid == 0) {
+      if (!mbar_wait_bounded(bar_w + st, static_cast<unsigned>((i >> 1) & 1), kMbarPollLimit, p.err)) ok = false;
+      tc_fence_after();
+      const unsigned char* whi = smb + OutPlan::wb + st * 2 * kBlkBytes;
+      const unsigned char* wlo = whi + kBlkBytes;
+      const unsigned char* shi = smb + OutPlan::img;
+      const unsigned char* slo = shi + kBlkBytes;
+#pragma unroll
+      for (int k = 0; k < kSlots / 16; ++k) {
+        const uint64_t ah = umma_desc(whi + k * 2048, 1024, 128), al = umma_desc(wlo + k * 2048, 1024, 128);
+        const uint64_t bh = umma_desc(shi + k * 256, 128, 1024), bl = umma_desc(slo + k * 256, 128, 1024);
+        umma_bf16(tmem, ah, bh, idesc, k > 0);
+        umma_bf16(tmem, ah, bl, idesc, true);
+        umma_bf16(tmem, al, bh, idesc, true);
+      }
+      umma_commit(bar_mma);
+    }
+    __syncthreads();  // x tile i visible to all threads
+    const float* xt = reinterpret_cast<const float*>(smb + OutPlan::xt) + st * kTile * kBlk;
+    auto xat = [&](int r) -> float { return r >= 0 ? xt[r * kBlk + cc] : halo[(r + kHalo) * kBlk + cc]; };
+    // field: segment aggregates from zero, then carries in segment order
+    const int r_lo = sg * kSegLen, r_hi = min(Tt, r_lo + kSegLen);
     {
+      float a = 0.f;
+      for (int r = r_lo; r < r_hi; ++r) a = ewma(ge, a, xt[r * kBlk + cc]);
+      segc[sg * kBlk + cc] = a;
+    }
+    if (!mbar_wait_bounded(bar_mma, static_cast<unsigned>(i & 1), kMbarPollLimit, p.err)) ok = false;
+    tc_fence_after();
+    {  // accumulator row r (token) sits in lane (r%16) + 32*(r/16) for M = 64
       const int sp = warp & 3, colh = (warp >> 2) * 32;
       float v[32];
-      tmem_ld32(tmem + (static_cast<uint32_t>(32 * sp) << 16) + kSlots + buf * kCW + colh, v);
+      tmem_ld32(tmem + (static_cast<uint32_t>(32 * sp) << 16) + colh, v);
       if (lane < 16) {
-        float* dst = semc + (16 * sp + lane) * kSemStride + colh;
+        float* dst = semc + (16 * sp + lane) * kScStride + colh;
 #pragma unroll
-        for (int j = 0; j < 32; j += 4)
-          *reinterpret_cast<float4*>(dst + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+        for (int j = 0; j < 32; ++j) dst[j] = v[j];
       }
     }
     tc_fence_before();
     __syncthreads();
-    if (tid == 0 && c + 2 < nch) issue_sem(c + 2);  // overlaps the epilogue below
-    // field: per-segment aggregates, then carries folded in segment order
-    const int cc = tid % kCW, sg = tid / kCW;  // column, token segment
-    const int e = c * kCW + cc;
-    const int r_lo = sg * (kTile / kSeg), r_hi = min(Tt, r_lo + kTile / kSeg);
-    {
-      float a = 0.f;
-      for (int r = r_lo; r < r_hi; ++r) a = ewma(ge, a, xs[r * XS + e]);
-      segc[sg * kCW + cc] = a;
-    }
-    __syncthreads();
-    float f = fcar[e];
-    for (int s2 = 0; s2 < sg; ++s2) f = fmaf(s_gseg[s2], f, segc[s2 * kCW + cc]);
-    // ring: sum of the 16 positions ending at r, from the x tile and the halo
-    auto xat = [&](int r) -> float { return r >= 0 ? xs[r * XS + e] : halo[(r + kHalo) * HS + e]; };
-    float rs = 0.f;
-    if (r_lo < r_hi)
+    float f = fcar[cc];
+    for (int s2 = 0; s2 < sg; ++s2) f = fmaf(s_gseg[s2], f, segc[s2 * kBlk + cc]);
+    // ring: sum of the 16 positions ending at r [P3 §2.4: mean over all 16
+    // slots]; fusion, clip and scale [P3 §2.2]
+    float* orow = p.out + (in_row0 + (t0 - pos0)) * p.H + col0 + cc;
+    if (r_lo < r_hi) {
+      float rs = 0.f;
       for (int r = r_lo - kHalo; r <= r_lo; ++r) rs += xat(r);
-    for (int r = r_lo; r < r_hi; ++r) {
-      if (r > r_lo) rs += xat(r) - xat(r - kRing);
-      const float x = xs[r * XS + e];
-      f = ewma(ge, f, x);
-      float u = rs * (1.0f / kRing) + 0.5f * f + 0.5f * semc[r * kSemStride + cc];
-      u = fminf(fmaxf(u, -p.clip_eps), p.clip_eps);
-      if (write_ok) out[static_cast<long long>(r) * p.H + e] = fmaf(a_l, u, x);
+      for (int r = r_lo; r < r_hi; ++r) {
+        if (r > r_lo) rs += xat(r) - xat(r - kRing);
+        const float x = xt[r * kBlk + cc];
+        f = ewma(ge, f, x);
+        float u = rs * (1.0f / kRing) + 0.5f * f + 0.5f * semc[r * kScStride + cc];
+        u = fminf(fmaxf(u, -p.clip_eps), p.clip_eps);
+        if (ok) orow[static_cast<long long>(r) * p.H] = fmaf(a_l, u, x);
+      }
     }
-    if (last && write_ok) {
-      const int gi = rank * HS + e;
-      if (r_lo < Tt && r_hi == Tt) field[gi] = f;  // the segment holding the last token
+    const bool seg_last = r_lo < Tt && r_hi == Tt;  // this segment holds the tile's last token
+    if (i == tiles - 1 && ok) {
+      const int gi = col0 + cc;
+      if (seg_last) field[gi] = f;
       if (sg == 0) {
-        // ring slots of the last 16 positions, and their exact sum
+        // ring slots of the last 16 positions that belong to this call, and
+        // the exact sum over all 16
         const long long t_end = t0 + Tt - 1;
         float tot = 0.f;
         for (int r = 0; r < kRing; ++r) {
           const long long q = t_end - (kRing - 1) + r;
           if (q < 0) continue;
           const float v = xat(static_cast<int>(q - t0));
-          ring[static_cast<size_t>(q % kRing) * p.H + gi] = v;
+          if (q >= pos0) ring[static_cast<size_t>(q % kRing) * p.H + gi] = v;
           tot += v;
         }
         ring_sum[gi] = tot;
       }
     }
-    __syncthreads();
-  }
-
-  // ---- (I) last tile: window, S and position of the stream ---------------
-  if (last && write_ok) {
-    for (int idx = tid; idx < NG * D; idx += NT) {
-      const int g = g_lo + idx / D, i = idx % D;
-      if (g >= own_lo) far[g * D + i] = segA[(nseg - 1) * ne + idx];  // S at the tile end
-    }
-    if (own_lo <= g_hi) {
-      const long long t_end = pos0 + p.n - 1;
-      const long long w0 = max(pos0, t_end - K + 1);
-      const int n_own = g_hi - own_lo + 1;
-      const long long cnt = (t_end - w0 + 1) * n_own * D;
-      for (long long idx = tid; idx < cnt; idx += NT) {
-        const long long j = w0 + idx / (n_own * D);
-        const int g = own_lo + static_cast<int>((idx / D) % n_own);
-        const int i = static_cast<int>(idx % D);
-        const long long src = ((j - pos0) * nkv + g) * D + i;
-        const long long dst = (wslot(j) * nkv + g) * D + i;
-        win_k[dst] = kin[src];
-        win_v[dst] = vin[src];
+    __syncthreads();  // segc, fcar and the halo are read above
+    if (seg_last) fcar[cc] = f;
+    if (i + 1 < tiles)  // the last 15 x rows become the next tile's halo (Tt = 64 here)
+      for (int idx = tid; idx < kHalo * kBlk; idx += NT) {
+        const int q = idx / kBlk, c = idx % kBlk;
+        halo[idx] = xt[(kTile - kHalo + q) * kBlk + c];
       }
-    }
-    if (rank == 0 && tid == 0) *reinterpret_cast<long long*>(blk + p.so.pos) = pos0 + p.n;
+    __syncthreads();  // the x stage, halo and carries are ready for the next tile
   }
 
-  // every tensor-core operation has completed (last sem commit waited)
+  // One CTA per stream: window, S and position [P1 §2.2].
+  if (cb == 0 && ok) {
+    unsigned char* b2 = blk;
+    Tin* win_k = reinterpret_cast<Tin*>(b2 + p.so.win_k);
+    Tin* win_v = reinterpret_cast<Tin*>(b2 + p.so.win_v);
+    float* far = reinterpret_cast<float*>(b2 + p.so.far);
+    const int D = p.H / p.nq;
+    const float* sfin = reinterpret_cast<const float*>(p.ws + p.ws_sfin) + static_cast<long long>(s) * p.nkv * D;
+    for (int idx = tid; idx < p.nkv * D; idx += NT) far[idx] = sfin[idx];
+    const long long t_end = pos0 + p.n - 1;
+    const long long w0 = max(pos0, t_end - p.K + 1);
+    const Tin* kin = static_cast<const Tin*>(p.k) + in_row0 * p.nkv * D;
+    const Tin* vin = static_cast<const Tin*>(p.v) + in_row0 * p.nkv * D;
+    const long long row = static_cast<long long>(p.nkv) * D;
+    const long long cnt = (t_end - w0 + 1) * row;
+    for (long long idx = tid; idx < cnt; idx += NT) {
+      const long long j = w0 + idx / row, e = idx % row;
+      win_k[(j % p.K) * row + e] = kin[(j - pos0) * row + e];
+      win_v[(j % p.K) * row + e] = vin[(j - pos0) * row + e];
+    }
+    if (tid == 0) *reinterpret_cast<long long*>(b2 + p.so.pos) = pos0 + p.n;
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
@@ -1028,133 +1014,121 @@ prefill_kernel(const PrefillParams p) {
   }
 }
 
-template <typename Tin, int D>
-cudaError_t prepare_t(int optin) {
+// ---------------------------------------------------------------- host side
+
+template <typename K>
+cudaError_t set_smem(K kernel, int optin) {
   cudaFuncAttributes fa;
-  cudaError_t e = cudaFuncGetAttributes(&fa, prefill_kernel<Tin, D>);
+  cudaError_t e = cudaFuncGetAttributes(&fa, kernel);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(prefill_kernel<Tin, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              optin - static_cast<int>(fa.sharedSizeBytes));
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(prefill_kernel<Tin, D>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   return e;
+}
+
+template <typename K>
+cudaError_t launch_pdl(K kernel, dim3 grid, int smem, cudaStream_t s, const PrefillParams& p) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(NT, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, p);
 }
 
 template <typename Tin, int D>
 cudaError_t launch_t(const PrefillParams& p, cudaStream_t s) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(p.n_tiles * p.CS), 1, 1);
-  cfg.blockDim = dim3(kPrefillThreads, 1, 1);
-  cfg.dynamicSmemBytes = static_cast<size_t>(p.plan.total);
-  cfg.stream = s;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = p.CS;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, prefill_kernel<Tin, D>, p);
-}
-
-template <typename Tin, int D>
-int max_clusters_t(int cs, size_t smem) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(cs * 16), 1, 1);
-  cfg.blockDim = dim3(kPrefillThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = cs;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, prefill_kernel<Tin, D>, &cfg) != cudaSuccess) {
-    cudaGetLastError();
-    return 0;
+  const dim3 g1(static_cast<unsigned>(p.nq), static_cast<unsigned>(p.n_streams), 1);
+  const dim3 g2(static_cast<unsigned>(p.tiles_per_stream), static_cast<unsigned>(p.n_streams), 1);
+  const dim3 g3(static_cast<unsigned>(p.H / kBlk), static_cast<unsigned>(p.n_streams), 1);
+  cudaError_t e;
+  if constexpr (sizeof(Tin) == 2) {
+    if (p.near.tc) e = launch_pdl(near_tc_kernel<D>, g1, p.near.total, s, p);
+    else e = launch_pdl(near_kernel<Tin, D>, g1, p.near.total, s, p);
+  } else {
+    e = launch_pdl(near_kernel<Tin, D>, g1, p.near.total, s, p);
   }
-  return n;
+  if (e == cudaSuccess) e = launch_pdl(pool_kernel, g2, p.pool_smem, s, p);
+  if (e == cudaSuccess) e = launch_pdl(out_kernel<Tin>, g3, p.out_smem, s, p);
+  return e;
 }
 
 }  // namespace
 
-// Shared-memory plan: persistent regions, then a union of the staging
-// buffers (near-field phase) and the pool buffers (pool phase).  The key
-// block is as tall as fits, up to the whole span t0-k .. t0+T-1.  The plan
-// never drops below a third of the SM's shared memory, so at most two CTAs
-// share an SM and their tensor-memory allocations (256 columns each) always
-// fit at once.
-bool plan_prefill(int HPC, int D, int esz, int NGm, int K, size_t budget, bool tc,
-                  PrefillPlan* out) {
-  const int HS = HPC * D, XS = HS + 4;
-  if (HS % kBlk != 0) return false;
-  if (tc && (esz != 2 || K > kSpan - kTile)) return false;
+bool plan_near(int D, int esz, int K, size_t limit, bool tc, NearPlan* out) {
   auto a16 = [](long long x) { return static_cast<int>((x + 15) & ~15LL); };
-  PrefillPlan p;
+  NearPlan p;
   std::memset(&p, 0, sizeof(p));
+  tc = tc && esz == 2 && K <= 16;
   p.tc = tc ? 1 : 0;
+  p.row = D * esz + 16;
+  const int xs = a16(4LL * kTile * (D + kXsPad));
+  const int qb = tc ? kTile * D * 2 : a16(static_cast<long long>(kTile) * p.row);
+  const int kvb = tc ? (D / 8) * kDStr : a16(static_cast<long long>(kTile + K) * p.row);
+  const int fixed = tc ? 2 * (2 * kTile * kNS * 2) : xs;  // P and G blocks, or the x tile
+  const int stage = qb + 2 * kvb;
+  // Two stages where they keep two CTAs per SM, else one, else (CUDA cores)
+  // keys and values from global memory (windows too wide to stage).
+  const long long two_per_sm = static_cast<long long>(limit) / 2 - 1024;
+  int stages = 0;
+  if (2LL * stage + fixed <= two_per_sm) stages = 2;
+  else if (static_cast<long long>(stage) + fixed <= two_per_sm) stages = 1;
+  else if (2LL * stage + fixed <= static_cast<long long>(limit)) stages = 2;
+  else if (static_cast<long long>(stage) + fixed <= static_cast<long long>(limit)) stages = 1;
+  if (tc && stages == 0) return false;
   int off = 0;
-  p.bars = off;                 off += 128;  // mbarriers and the tensor-memory address
-  p.xs = off;                   off += a16(4LL * kTile * XS);
-  p.halo = off;                 off += a16(4LL * kHalo * HS);
-  p.fcar = off;                 off += a16(4LL * HS);
-  p.sst = off;                  off += a16(4LL * NGm * D);
-  p.sagg = off;                 off += a16(4LL * NGm * D);
-  p.sega = off;                 off += a16(4LL * NT);   // far-field scan segments
-  // epilogue carries, then (CUDA-core near field) running max / denominator
-  p.ml = off;                   off += a16(4LL * (kSeg * kCW + (tc ? 0 : 2 * kTile * HPC)));
-  p.u0 = off;
-  // pool phase: slot blocks, partials | sem chunk, x block | w block
-  int q = off;
-  p.sl = q;                     q += a16(static_cast<long long>(HS / kBlk) * 2 * kBlkBytes);
-  p.part = q;                   q += a16(4LL * kTile * std::max(kPartStride, kSemStride));
-  p.wts = q;
-  p.semc = q;                   q += a16(2LL * kBlkBytes);
-  const int pool_end = q;
-  q = off;
   if (tc) {
-    // near-field phase on the tensor cores: one query block, key and value
-    // blocks of every KV head of the CTA, the P block (hi, lo)
-    p.qa = q;                   q += a16(2LL * kTile * D);
-    p.kvp = q;                  q += a16(2LL * 2 * NGm * kSpan * D);
-    p.pa = q;                   q += a16(2LL * 2 * kTile * kSpan);
-    p.KB = kSpan;
+    p.pa = off;
+    off += 2 * kTile * kNS * 2;
+    p.ga = off;
+    off += 2 * kTile * kNS * 2;
   } else {
-    // near-field phase on the CUDA cores: staged queries and key/value rows
-    p.qst = q;                  q += a16(static_cast<long long>(kTile) * HS * esz);
-    const int row_b = NGm * D * esz + 16;
-    const long long room = static_cast<long long>(budget) - q;
-    int kb_rows = static_cast<int>(room / (2LL * row_b));
-    kb_rows = std::min(kb_rows, kTile + K);
-    if (kb_rows < 32) return false;
-    p.KB = kb_rows;
-    p.kb = q;                   q += a16(static_cast<long long>(row_b) * kb_rows);
-    p.vb = q;                   q += a16(static_cast<long long>(row_b) * kb_rows);
+    p.xs = off;
+    off += xs;
   }
-  p.total = std::max(q, pool_end);
-  p.total = std::max<int>(p.total, static_cast<int>((budget + 1024) / 3) + 1);
-  if (static_cast<size_t>(p.total) > budget) return false;
+  for (int st = 0; st < 2; ++st) {
+    if (st < std::max(stages, 1)) {
+      p.q[st] = off;
+      off += qb;
+      if (stages > 0) {
+        p.k[st] = off;
+        off += kvb;
+        p.v[st] = off;
+        off += kvb;
+      }
+    } else {
+      p.q[st] = p.q[0];
+      p.k[st] = p.k[0];
+      p.v[st] = p.v[0];
+    }
+  }
+  p.stages = stages;
+  p.total = off;
+  if (static_cast<size_t>(p.total) > limit) return false;
   *out = p;
   return true;
 }
 
-int prefill_max_active_clusters(int cs, size_t smem, int in_dtype, int head_dim) {
-  if (in_dtype == SFA_F32) return head_dim == 64 ? max_clusters_t<float, 64>(cs, smem) : max_clusters_t<float, 128>(cs, smem);
-  return head_dim == 64 ? max_clusters_t<__nv_bfloat16, 64>(cs, smem)
-                        : max_clusters_t<__nv_bfloat16, 128>(cs, smem);
-}
+int prefill_pool_smem() { return PoolPlan::total; }
+int prefill_out_smem() { return OutPlan::total; }
 
 cudaError_t prefill_prepare(int device) {
   int optin = 0;
   cudaError_t e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device);
-  if (e == cudaSuccess) e = prepare_t<float, 64>(optin);
-  if (e == cudaSuccess) e = prepare_t<float, 128>(optin);
-  if (e == cudaSuccess) e = prepare_t<__nv_bfloat16, 64>(optin);
-  if (e == cudaSuccess) e = prepare_t<__nv_bfloat16, 128>(optin);
+  if (e == cudaSuccess) e = set_smem(near_kernel<float, 64>, optin);
+  if (e == cudaSuccess) e = set_smem(near_kernel<float, 128>, optin);
+  if (e == cudaSuccess) e = set_smem(near_kernel<__nv_bfloat16, 64>, optin);
+  if (e == cudaSuccess) e = set_smem(near_kernel<__nv_bfloat16, 128>, optin);
+  if (e == cudaSuccess) e = set_smem(near_tc_kernel<64>, optin);
+  if (e == cudaSuccess) e = set_smem(near_tc_kernel<128>, optin);
+  if (e == cudaSuccess) e = set_smem(pool_kernel, optin);
+  if (e == cudaSuccess) e = set_smem(out_kernel<float>, optin);
+  if (e == cudaSuccess) e = set_smem(out_kernel<__nv_bfloat16>, optin);
   return e;
 }
 
@@ -1162,7 +1136,7 @@ size_t prefill_smem_limit(int device) {
   int optin = 0;
   if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device) != cudaSuccess)
     return 0;
-  return static_cast<size_t>(optin) - 1024;  // headroom for the kernel's static shared memory
+  return static_cast<size_t>(optin) - 1024;  // headroom for the kernels' static shared memory
 }
 
 cudaError_t launch_prefill(const PrefillParams& p, int in_dtype, int head_dim, cudaStream_t s) {

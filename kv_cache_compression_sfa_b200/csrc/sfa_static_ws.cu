@@ -5,10 +5,11 @@
 // another inference engine may receive only the operator's input and output
 // tensors and no allocator, and a serving loop may forbid cudaMalloc in its
 // steady state because an allocation can synchronise the device.  For them,
-// the prefill's cross-tile scratch (look-back flags, carries and tail rows)
-// lives in one file-scope device array of fixed size, reserved when the
-// library is loaded and held by every GPU that loads it until the process
-// exits.  The caller still passes inputs, outputs and the state.
+// the prefill's scratch (stream positions, the far state at the end of the
+// call and the pool weights of every tile) lives in one file-scope device
+// array of fixed size, reserved when the library is loaded and held by every
+// GPU that loads it until the process exits.  The caller still passes
+// inputs, outputs and the state.
 //
 // The work itself is exactly sfa_prefill's: this entry point only supplies
 // the array's device address as the workspace.
@@ -21,7 +22,7 @@
 namespace {
 
 // Scratch shared by every call on a device (16 MiB: one 512-token prefill of
-// a 24-layer, hidden-896 model needs about 12 MB).
+// a 24-layer, hidden-896 model needs about 3 MB).
 constexpr size_t kStaticWorkspaceBytes = SFA_STATIC_WORKSPACE_BYTES;
 static __device__ __align__(256) unsigned char g_static_ws[kStaticWorkspaceBytes];
 
@@ -62,8 +63,7 @@ int sfa_prefill_static_ws(const sfa_handle* h, const void* q, const void* k, con
   void* ws = nullptr;
   const int rc = static_ws_address(&ws);
   if (rc != SFA_OK) return rc;
-  // sfa_prefill clears the part of the workspace that must start at zero
-  // (ticket counter and look-back flags) on the stream before its kernel.
+  // Nothing in the workspace has to start at zero.
   return sfa_prefill(h, q, k, v, n, batch, state, out, ws, kStaticWorkspaceBytes, stream);
 }
 

@@ -112,11 +112,11 @@ def test_state_snapshot_resumes_exactly():
 
 
 def test_prefill_is_deterministic_across_runs():
-    """The look-back folds carries in a fixed order: repeated runs are bitwise
-    equal, whatever the timing of the tiles."""
+    """Every reduction and carry runs in a fixed order: repeated runs are
+    bitwise equal, whatever the timing of the CTAs."""
     w = WORKLOADS["qwen05b"].replace(name="determinism", n_layers=2, batch=3)
     slots = make_slots(w, "cuda")
-    q, k, v = TokenSource(w, "cuda").get(0, 2100)  # 33 tiles: three look-back groups
+    q, k, v = TokenSource(w, "cuda").get(0, 2100)  # 33 tiles per stream, the last one ragged
     op = _op(w, slots)
     first = op.prefill(q, k, v)
     s1 = op.state.clone()
@@ -128,7 +128,7 @@ def test_prefill_is_deterministic_across_runs():
     assert op.check() == 0
 
 
-def test_chunked_prefill_across_lookback_groups():
+def test_chunked_prefill_across_many_tiles():
     w = WORKLOADS["qwen05b"].replace(name="groups", n_layers=1, batch=2)
     slots = make_slots(w, "cuda")
     q, k, v = TokenSource(w, "cuda").get(0, 2300)

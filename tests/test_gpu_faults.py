@@ -2,9 +2,9 @@
 
 Host-side checks reject bad calls before any launch.  On the device, a state
 built for another configuration is detected from its header and latched;
-the look-back waits of the prefill are bounded, and a test hook withholds
-one tile's publication so that its successor's wait runs out: the kernel
-still finishes, latches SFA_ERR_DEVICE_TIMEOUT, and the context stays usable.
+the prefill's waits are bounded, and a test hook makes one CTA wait on a
+barrier that nothing completes so that its wait runs out: the kernel still
+finishes, latches SFA_ERR_DEVICE_TIMEOUT, and the context stays usable.
 """
 import ctypes
 
@@ -86,11 +86,11 @@ def test_state_of_another_config_is_detected_on_the_device():
     assert a.check() == 0
 
 
-def test_lookback_wait_runs_out_and_the_context_survives():
+def test_bounded_wait_runs_out_and_the_context_survives():
     w = _w()
     op = sfa.SfaOperator(sfa_config(w), make_slots(w, "cuda"), w.batch, max_prefill=256)
     n_streams = w.n_layers * w.batch
-    # withhold tile 1 of stream 0: ticket = tile * n_streams + stream
+    # tile 1 of stream 0: index = tile * n_streams + stream
     sfa.sfa_debug_set_lookback(op.handle, spin_limit=2000, withhold_tile=1 * n_streams + 0)
     q, k, v = TokenSource(w, "cuda").get(0, 256)
     op.prefill(q, k, v)

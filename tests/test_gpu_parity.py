@@ -112,11 +112,9 @@ def test_edge_schedules(name, over, schedule):
     _run_schedule(w, schedule)
 
 
-def test_cuda_core_near_field_on_bf16_inputs(monkeypatch):
-    """bf16 inputs with k <= 16 take the tensor-core near field; the handle's
-    test hook keeps them on the CUDA cores, which must meet the same bar."""
-    monkeypatch.setenv("SFA_CUDA_CORE_NEAR_FIELD", "1")
-    w = _tiny_variant(name="cuda_core_near_bf16", n_layers=2, batch=2, n_q_heads=14,
+def test_gqa7_bf16_chunked_prefill_and_decode():
+    """Seven query heads per KV head, bf16, prefill calls across a decode."""
+    w = _tiny_variant(name="gqa7_bf16_chunks", n_layers=2, batch=2, n_q_heads=14,
                       n_kv_heads=2, head_dim=64, window_k=16, in_dtype="bf16")
     _run_schedule(w, [("p", 130), ("d", 5), ("p", 70)])
 

@@ -49,7 +49,7 @@ def test_static_workspace_rejects_a_call_larger_than_the_array():
     w = WORKLOADS["qwen05b"]
     slots = make_slots(w, "cuda")
     op = sfa.SfaOperator(sfa_config(w), slots, w.batch, device="cuda")
-    n = 4096  # needs ~95 MB of scratch
+    n = 4096  # needs ~25 MB of scratch
     assert sfa.sfa_prefill_workspace_bytes(op.handle, w.batch, n) > sfa.SFA_STATIC_WORKSPACE_BYTES
     q, k, v = TokenSource(w, "cuda").get(0, 1)  # never read: the call is refused first
     out = torch.empty(1, device="cuda")
