@@ -31,9 +31,11 @@ struct sfa_handle {
   float* slot_norm;      // [L][64]
   float* alpha_layer;    // [L]
   unsigned char* slot_img;  // [L][H/64][hi, lo] bf16 blocks for the prefill pool MMAs
+  float* slot_dec;       // [L][cs][64][HS + 4] each decode CTA's slot slice, rows padded
   int* err;              // device error word
   uint64_t cfg_hash;
   int cs;               // CTAs per cluster of the decode kernels
+  int n_sm;              // streaming multiprocessors of the device
   NearPlan near;         // shared-memory plan of the prefill near-field kernel
   int decode_budget;
   unsigned spin_limit;
@@ -110,7 +112,8 @@ std::vector<int> cluster_candidates(int nq, int d) {
 }
 
 // Workspace of a prefill call: the streams' positions, S at the end of the
-// call and the pool weights of every tile (two 8 KB bf16 blocks).
+// call, the pool weights of every tile (two 8 KB bf16 blocks) and S at
+// every tile start.
 PrefillWorkspace prefill_workspace(const sfa_config* c, int layers, int batch, long long n) {
   PrefillWorkspace w;
   const long long streams = static_cast<long long>(layers) * batch;
@@ -119,7 +122,8 @@ PrefillWorkspace prefill_workspace(const sfa_config* c, int layers, int batch, l
   w.pos = 0;
   w.sfin = align256(8 * streams);
   w.w = w.sfin + align256(4 * streams * sdim);
-  w.total = w.w + tiles * 2LL * kBlkBytesHost;
+  w.sst = w.w + tiles * 2LL * kBlkBytesHost;
+  w.total = w.sst + align256(4 * tiles * sdim);
   return w;
 }
 
@@ -149,6 +153,7 @@ void fill_common(P& p, const sfa_handle* h, int batch, void* state) {
   p.slots = h->slots;
   p.slot_norm = h->slot_norm;
   p.slot_img = h->slot_img;
+  if constexpr (std::is_same<P, DecodeParams>::value) p.slot_dec = h->slot_dec;
   p.alpha_layer = h->alpha_layer;
   p.err = h->err;
   p.cfg_hash = h->cfg_hash;
@@ -254,6 +259,7 @@ int sfa_init(const sfa_config* cfg, sfa_handle** out) {
   const int L = cfg->n_layers, H = hidden_of(cfg);
   const size_t slot_bytes = sizeof(float) * static_cast<size_t>(L) * kSlots * H;
   cudaError_t e = cudaGetDevice(&h->device);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&h->n_sm, cudaDevAttrMultiProcessorCount, h->device);
   if (e == cudaSuccess) e = cudaMalloc(&h->slots, slot_bytes);
   if (e == cudaSuccess) e = cudaMalloc(&h->slot_norm, sizeof(float) * L * kSlots);
   if (e == cudaSuccess) e = cudaMalloc(&h->alpha_layer, sizeof(float) * L);
@@ -285,7 +291,7 @@ int sfa_init(const sfa_config* cfg, sfa_handle** out) {
       const int hpc = cfg->n_q_heads / cs;
       const size_t dsm = decode_smem_bytes(hpc, cfg->head_dim, esz,
                                            max_kv_heads_per_cta(cfg->n_q_heads, cfg->n_kv_heads, cs),
-                                           cfg->window_k, decode_budget(limit));
+                                           cfg->n_kv_heads, cfg->window_k, decode_budget(limit));
       if (dsm > limit) continue;
       if (decode_max_active_clusters(cs, dsm, cfg->in_dtype, cfg->head_dim) < 1) continue;
       h->cs = cs;
@@ -297,6 +303,20 @@ int sfa_init(const sfa_config* cfg, sfa_handle** out) {
       break;
     }
     if (e == cudaSuccess && h->cs == 0) e = cudaErrorInvalidConfiguration;
+    if (e == cudaSuccess) {
+      // Each decode CTA's slot slice [64][HS] laid out contiguously with the
+      // rows padded to HS + 4 floats, as in its shared memory: one bulk copy.
+      const int hs = (cfg->n_q_heads / h->cs) * cfg->head_dim;
+      const size_t pitch = static_cast<size_t>(hs + 4) * sizeof(float);
+      const size_t bytes = static_cast<size_t>(L) * h->cs * kSlots * pitch;
+      e = cudaMalloc(&h->slot_dec, bytes);
+      if (e == cudaSuccess) e = cudaMemset(h->slot_dec, 0, bytes);
+      for (int l = 0; l < L && e == cudaSuccess; ++l)
+        for (int r = 0; r < h->cs && e == cudaSuccess; ++r)
+          e = cudaMemcpy2D(h->slot_dec + (static_cast<size_t>(l) * h->cs + r) * kSlots * (hs + 4), pitch,
+                           h->slots + static_cast<size_t>(l) * kSlots * H + static_cast<size_t>(r) * hs,
+                           sizeof(float) * H, sizeof(float) * hs, kSlots, cudaMemcpyDeviceToDevice);
+    }
   }
   if (e == cudaSuccess) e = launch_slot_norms(h->slots, h->slot_norm, L, H, nullptr);
   if (e == cudaSuccess) e = launch_slot_image(h->slots, h->slot_img, L, H, nullptr);
@@ -318,6 +338,7 @@ int sfa_init(const sfa_config* cfg, sfa_handle** out) {
     cudaFree(h->slot_norm);
     cudaFree(h->alpha_layer);
     cudaFree(h->slot_img);
+    cudaFree(h->slot_dec);
     cudaFree(h->err);
     h->magic = 0;
     delete h;
@@ -335,6 +356,7 @@ int sfa_destroy(sfa_handle* h) {
   cudaFree(h->slot_norm);
   cudaFree(h->alpha_layer);
   cudaFree(h->slot_img);
+  cudaFree(h->slot_dec);
   cudaFree(h->err);
   h->magic = 0;
   delete h;
@@ -420,6 +442,19 @@ int sfa_prefill_layers(const sfa_handle* h, int layer_begin, int layer_count, co
   p.ws_pos = w.pos;
   p.ws_sfin = w.sfin;
   p.ws_w = w.w;
+  p.ws_sst = w.sst;
+  {
+    // Near-field segments: about four rounds of two CTAs per SM, each CTA a
+    // run of consecutive tiles of one (stream, head).
+    const long long units = static_cast<long long>(c->n_q_heads) * streams;
+    const long long target = 4LL * 2 * std::max(h->n_sm, 1);
+    long long nseg = std::max(1LL, std::min(tiles_per_stream, (target + units - 1) / units));
+    const long long tps = (tiles_per_stream + nseg - 1) / nseg;
+    nseg = (tiles_per_stream + tps - 1) / tps;
+    if (nseg * c->n_q_heads > 0x7fffffffLL) return SFA_ERR_UNSUPPORTED;
+    p.n_seg = static_cast<int>(nseg);
+    p.tps = static_cast<int>(tps);
+  }
   p.spin_limit = h->spin_limit;
   p.withhold_tile = h->withhold_tile;
   p.near = h->near;

@@ -60,13 +60,14 @@ constexpr int kMaxHeadsCta = kMaxSlice / 64;         // query heads one CTA can 
 // distinct banks.
 struct DecodePlan {
   int bars, sl, xs, red, inbox, wts, pb, mrg, qraw, kc, vc, sg, fld, rsm, wk, wv, total;
-  int rec;         // bytes per staged window slot (NGm heads + pad)
+  int rec;         // bytes per staged window slot
   bool stage_win;  // window staged in shared memory
+  bool whole;      // all KV heads of each slot staged (one copy each for K and V)
 };
 
 __host__ __device__ inline int a16(long long x) { return static_cast<int>((x + 15) & ~15LL); }
 
-__host__ __device__ inline DecodePlan decode_plan(int HPC, int D, int esz, int NGm, int K,
+__host__ __device__ inline DecodePlan decode_plan(int HPC, int D, int esz, int NGm, int nkv, int K,
                                                   int budget) {
   const int HS = HPC * D;
   DecodePlan p;
@@ -85,7 +86,11 @@ __host__ __device__ inline DecodePlan decode_plan(int HPC, int D, int esz, int N
   p.sg = o;    o += a16(4LL * NGm * D);
   p.fld = o;   o += a16(4LL * HS);
   p.rsm = o;   o += a16(4LL * HS);
-  p.rec = NGm * D * esz + 16;
+  // The whole window [k][n_kv][d] in one copy each for K and V where it
+  // fits (few large copies instead of one per slot), else this CTA's heads
+  // of each slot with 16 bytes of padding per slot, else global memory.
+  p.whole = (o + 2LL * K * nkv * D * esz) <= budget;
+  p.rec = p.whole ? nkv * D * esz : NGm * D * esz + 16;
   const long long win = 2LL * K * p.rec;
   p.stage_win = (o + win) <= budget;
   p.wk = o;
@@ -129,7 +134,8 @@ decode_kernel(const DecodeParams p) {
   const int own_lo = (h0 + G - 1) / G;
 
   extern __shared__ __align__(16) unsigned char smb[];
-  const DecodePlan pl = decode_plan(HPC, D, ESZ, p.NGm, K, p.smem_budget);
+  const DecodePlan pl = decode_plan(HPC, D, ESZ, p.NGm, nkv, K, p.smem_budget);
+  const int wb = pl.whole ? g_lo : 0;  // head offset of this CTA's KV heads in a staged slot
   uint64_t* bar_sl = reinterpret_cast<uint64_t*>(smb + pl.bars);
   uint64_t* bar_in = bar_sl + 1;
   uint64_t* bar_red = bar_sl + 2;
@@ -167,12 +173,11 @@ decode_kernel(const DecodeParams p) {
 
   // Slot slice: constant since sfa_init, so it may be fetched before the
   // previous kernel of the stream has finished.
-  const float* slot_base = p.slots + static_cast<size_t>(l) * kSlots * p.H + static_cast<size_t>(rank) * HS;
-  if (warp == 0) {
-    if (lane == 0) mbar_arrive_expect_tx(bar_sl, kSlots * HS * 4u);
-    __syncwarp();
-    for (int j = lane; j < kSlots; j += 32)
-      bulk_g2s(sl + j * (HS + 4), slot_base + static_cast<size_t>(j) * p.H, HS * 4u, bar_sl);
+  // One copy: the slice is stored contiguously with padded rows at init.
+  if (tid == 0) {
+    const unsigned bytes = static_cast<unsigned>(kSlots * (HS + 4) * 4);
+    mbar_arrive_expect_tx(bar_sl, bytes);
+    bulk_g2s(sl, p.slot_dec + (static_cast<size_t>(l) * p.CS + rank) * kSlots * (HS + 4), bytes, bar_sl);
   }
   // Other per-layer constants: slot norms (lane j: slots j, j+32; every
   // warp forms the softmax itself) and alpha_layer.
@@ -216,7 +221,7 @@ decode_kernel(const DecodeParams p) {
     const unsigned hb = static_cast<unsigned>(NG * D * ESZ);
     unsigned bytes = static_cast<unsigned>(HS * ESZ) + 2u * hb + static_cast<unsigned>(NG * D * 4) +
                      2u * static_cast<unsigned>(HS * 4);
-    if (pl.stage_win) bytes += 2u * static_cast<unsigned>(K) * hb;
+    if (pl.stage_win) bytes += 2u * static_cast<unsigned>(K) * (pl.whole ? static_cast<unsigned>(pl.rec) : hb);
     if (lane == 0) mbar_arrive_expect_tx(bar_in, bytes);
     __syncwarp();
     if (lane == 0) bulk_g2s(qraw, qin, static_cast<unsigned>(HS * ESZ), bar_in);
@@ -225,7 +230,10 @@ decode_kernel(const DecodeParams p) {
     if (lane == 3) bulk_g2s(sg, far + g_lo * D, static_cast<unsigned>(NG * D * 4), bar_in);
     if (lane == 4) bulk_g2s(fld, field + rank * HS, static_cast<unsigned>(HS * 4), bar_in);
     if (lane == 5) bulk_g2s(rsm, ring_sum + rank * HS, static_cast<unsigned>(HS * 4), bar_in);
-    if (pl.stage_win)
+    if (pl.whole) {
+      if (lane == 6) bulk_g2s(wk, win_k, static_cast<unsigned>(K * pl.rec), bar_in);
+      if (lane == 7) bulk_g2s(wv, win_v, static_cast<unsigned>(K * pl.rec), bar_in);
+    } else if (pl.stage_win)
       for (int s = lane; s < K; s += 32) {
         const size_t off = (static_cast<size_t>(s) * nkv + g_lo) * D;
         bulk_g2s(wk + s * pl.rec, win_k + off, hb, bar_in);
@@ -291,13 +299,13 @@ decode_kernel(const DecodeParams p) {
     auto krow = [&](int a, int gg) -> const Tin* {
       if (a == nwin - 1) return kc + gg * D;
       const int s2 = wslot(a);
-      if constexpr (STAGED) return reinterpret_cast<const Tin*>(wk + s2 * pl.rec) + gg * D;
+      if constexpr (STAGED) return reinterpret_cast<const Tin*>(wk + s2 * pl.rec) + (wb + gg) * D;
       else return win_k + (static_cast<size_t>(s2) * nkv + g_lo + gg) * D;
     };
     auto vrow = [&](int a, int gg) -> const Tin* {
       if (a == nwin - 1) return vc + gg * D;
       const int s2 = wslot(a);
-      if constexpr (STAGED) return reinterpret_cast<const Tin*>(wv + s2 * pl.rec) + gg * D;
+      if constexpr (STAGED) return reinterpret_cast<const Tin*>(wv + s2 * pl.rec) + (wb + gg) * D;
       else return win_v + (static_cast<size_t>(s2) * nkv + g_lo + gg) * D;
     };
     const int key = lane / LPK, part = lane % LPK;
@@ -397,7 +405,7 @@ decode_kernel(const DecodeParams p) {
     const int gg = (h0 + hh) / G - g_lo;
     float s_new = sg[gg * D + i];
     if (evict) {
-      const Tin* er = pl.stage_win ? reinterpret_cast<const Tin*>(wk + eslot * pl.rec) + gg * D
+      const Tin* er = pl.stage_win ? reinterpret_cast<const Tin*>(wk + eslot * pl.rec) + (wb + gg) * D
                                    : win_k + (static_cast<size_t>(eslot) * nkv + g_lo + gg) * D;
       s_new = ewma(p.gamma_far, s_new, to_f32<Tin>(er[i]));
     }
@@ -527,7 +535,7 @@ decode_kernel(const DecodeParams p) {
       float s = sg[gg * D + i];
       if (evict) {
         const int s2 = eslot;
-        const Tin* er = pl.stage_win ? reinterpret_cast<const Tin*>(wk + s2 * pl.rec) + gg * D
+        const Tin* er = pl.stage_win ? reinterpret_cast<const Tin*>(wk + s2 * pl.rec) + (wb + gg) * D
                                      : win_k + (static_cast<size_t>(s2) * nkv + g_lo + gg) * D;
         s = ewma(p.gamma_far, s, to_f32<Tin>(er[i]));
       }
@@ -542,7 +550,7 @@ decode_kernel(const DecodeParams p) {
 
 template <typename Tin, int D>
 cudaError_t launch_t(const DecodeParams& p, cudaStream_t s) {
-  const DecodePlan pl = decode_plan(p.HPC, D, static_cast<int>(sizeof(Tin)), p.NGm, p.K, p.smem_budget);
+  const DecodePlan pl = decode_plan(p.HPC, D, static_cast<int>(sizeof(Tin)), p.NGm, p.nkv, p.K, p.smem_budget);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.CS, p.n_seq, p.Lc);
   cfg.blockDim = dim3(kDecodeThreads, 1, 1);
@@ -597,8 +605,8 @@ int max_clusters_t(int cs, size_t smem) {
 
 // Shared memory of one decode CTA; the window is staged when it fits in
 // `budget` bytes together with everything else.
-size_t decode_smem_bytes(int HPC, int head_dim, int esz, int NGm, int K, int budget) {
-  return static_cast<size_t>(decode_plan(HPC, head_dim, esz, NGm, K, budget).total);
+size_t decode_smem_bytes(int HPC, int head_dim, int esz, int NGm, int nkv, int K, int budget) {
+  return static_cast<size_t>(decode_plan(HPC, head_dim, esz, NGm, nkv, K, budget).total);
 }
 
 int decode_max_active_clusters(int cs, size_t smem, int in_dtype, int head_dim) {

@@ -63,6 +63,7 @@ struct DecodeParams {
   const float* slot_norm;   // [L][64], clamped at kNormFloor
   const float* alpha_layer; // [L]
   const unsigned char* slot_img;  // pre-split bf16 slot blocks (batch-tiled decode)
+  const float* slot_dec;          // [L][CS][64][HS + 4] slot slice of every decode CTA
   int* err;
   uint64_t cfg_hash;
   StreamOffsets so;
@@ -110,8 +111,10 @@ struct PrefillParams {
   int L, B, nq, nkv, K, H, G;
   int l0;                   // first layer of the state served (streams are l0*B + ...)
   int tiles_per_stream, n_streams;
-  // workspace byte offsets: stream positions, S at the end of the call, pool weights
-  long long ws_pos, ws_sfin, ws_w;
+  int n_seg, tps;           // near field: segments per stream, tiles per segment
+  // workspace byte offsets: stream positions, S at the end of the call, pool
+  // weights, far-field state at every tile start
+  long long ws_pos, ws_sfin, ws_w, ws_sst;
   float gamma_far, alpha_far, ema_gamma, inv_temp, clip_eps, score_scale;
   unsigned spin_limit;      // polls of a bounded wait before it gives up
   long long withhold_tile;  // test hook: this tile's pool CTA waits on a barrier nothing completes
@@ -124,6 +127,7 @@ struct PrefillWorkspace {
   long long pos;    // [streams] int64 position at the start of the call
   long long sfin;   // [streams][n_kv][d] fp32 far state at the end of the call
   long long w;      // [streams * tiles][hi, lo] 64 x 64 bf16 pool-weight blocks
+  long long sst;    // [streams][tiles][n_kv][d] fp32 far state at every tile start
   long long total;
 };
 
@@ -144,7 +148,7 @@ int prefill_pool_smem();
 int prefill_out_smem();
 cudaError_t prefill_prepare(int device);
 cudaError_t decode_prepare(int device);
-size_t decode_smem_bytes(int HPC, int head_dim, int esz, int NGm, int K, int budget);
+size_t decode_smem_bytes(int HPC, int head_dim, int esz, int NGm, int nkv, int K, int budget);
 int decode_max_active_clusters(int cs, size_t smem, int in_dtype, int head_dim);
 size_t prefill_smem_limit(int device);
 cudaError_t launch_write_header(unsigned char* state, StateHeader h, cudaStream_t s);

@@ -1,5 +1,5 @@
 // sfa_prefill.cu — SFA prefill: n tokens per (layer, sequence) stream in
-// three kernels, each parallel over independent work units with no waits
+// five kernels, each parallel over independent work units with no waits
 // between CTAs.
 //
 // Sources (web pages):
@@ -8,14 +8,17 @@
 //   [P3] "Dalin Soma SFA基于信号场注意力机制的神经网络推理加速框架"
 //        §2.1 channels 1–3, §2.2 fusion, clip and alpha_layer, §2.4 ring mean.
 //
-// 1. near_kernel, one CTA per (stream, query head), walks the stream's
-//    tiles of kTile tokens in order.  Per tile: queries and the key/value
-//    span (positions t0-k .. t0+T-1) staged in shared memory by cp.async,
-//    the next tile's copy in flight during this one's arithmetic; the
-//    far-field EWMA S of the head's KV group carried in registers across
-//    tiles [P1 §2.1 eq. S_t]; the near field as an online softmax per token
-//    on the CUDA cores [P1 §2.1 eq. O_near]; x = O_near + alpha_far * S
-//    [P1 §2.1 eq. O] written into `out`, which holds x until step 3.
+// 0. far_agg_kernel / far_carry_kernel: the far-field EWMA S [P1 §2.1 eq.
+//    S_t] at every tile start of kTile tokens, as a two-level scan: one
+//    aggregate of the evicted keys per tile (independent terms), then one
+//    fold in tile order per (stream, KV head, dim).
+// 1. near_tc_kernel (bf16, k <= 16) or near_kernel (CUDA cores), one CTA per
+//    (stream, query head, segment of consecutive tiles).  Per tile: queries
+//    and the key/value span staged in shared memory by cp.async, the next
+//    tile's copy in flight during this one's arithmetic; the near field as a
+//    softmax over each token's window [P1 §2.1 eq. O_near] and
+//    x = O_near + alpha_far * S [P1 §2.1 eq. O] written into `out`, which
+//    holds x until step 3.
 // 2. pool_kernel, one CTA per (stream, tile): the cosine scores of the
 //    tile's tokens against the 64 slots, x[T x H] . slot^T on the tcgen05
 //    tensor cores (three bf16 MMAs per 64-column chunk, hi*hi + hi*lo +
@@ -69,6 +72,125 @@ __device__ __forceinline__ bool header_matches(const PrefillParams& p) {
 
 __device__ __forceinline__ unsigned char* stream_block(const PrefillParams& p, int s) {
   return p.state + kHeaderBytes + (static_cast<long long>(p.l0) * p.B + s) * p.so.stride;
+}
+
+// ======================================================================
+// 0. far-field state at every tile start [P1 §2.1 eq. S_t]
+// ======================================================================
+// S folds one evicted key per token once the position reaches k, so over a
+// tile of Tt tokens S_end = gamma^ev S_start + agg with
+//   agg = sum over evicting tokens r of (1-gamma) gamma^(Tt-1-r) K_{t0+r-k},
+// ev the number of evicting tokens.  far_agg_kernel forms agg for every
+// tile in parallel (independent terms); far_carry_kernel folds them in tile
+// order per (stream, KV head, dim) and stores S at every tile start (in
+// place of agg) and at the end of the call.
+
+template <typename Tin, int D>
+__global__ void __launch_bounds__(NT) far_agg_kernel(const PrefillParams p) {
+  constexpr int VE = Load16<Tin>::N;  // dims per 16-byte load
+  constexpr int kQ = 4;               // token quarters of a tile
+  constexpr int kQLen = kTile / kQ;
+  const int tile = blockIdx.x, s = blockIdx.y, tid = threadIdx.x;
+  __shared__ int s_ok;
+  __shared__ long long s_pos;
+  __shared__ float s_w[kTile];
+  extern __shared__ __align__(16) unsigned char smb[];  // [kQ][n_kv * D] quarter sums
+
+  pdl_trigger();
+  pdl_wait();  // the state may be written by the previous kernel of the stream
+  unsigned char* blk = stream_block(p, s);
+  if (tid == 0) {
+    s_ok = header_matches(p);
+    s_pos = __ldcg(reinterpret_cast<const long long*>(blk + p.so.pos));
+  }
+  __syncthreads();
+  if (!s_ok) {  // uniform over the grid; every later kernel of the call sees it too
+    if (tid == 0 && tile == 0 && s == 0) latch_error(p.err, SFA_ERR_STATE_MISMATCH);
+    return;
+  }
+  const long long pos0 = s_pos;
+  if (tid == 0 && tile == 0) reinterpret_cast<long long*>(p.ws + p.ws_pos)[s] = pos0;
+  const int K = p.K, nkv = p.nkv;
+  const long long t0 = pos0 + static_cast<long long>(tile) * kTile;
+  const int Tt = static_cast<int>(min(static_cast<long long>(kTile), p.n - static_cast<long long>(tile) * kTile));
+  if (tid < kTile)
+    s_w[tid] = (tid < Tt && t0 + tid >= K) ? (1.0f - p.gamma_far) * powf(p.gamma_far, static_cast<float>(Tt - 1 - tid)) : 0.f;
+  __syncthreads();
+  const Tin* win_k = reinterpret_cast<const Tin*>(blk + p.so.win_k);
+  const Tin* kin = static_cast<const Tin*>(p.k) + static_cast<long long>(s) * p.n * nkv * D;
+  const int ne = nkv * D, nv = ne / VE;
+  float* part = reinterpret_cast<float*>(smb);
+  // Work item (16-byte dim group v, token quarter q): the quarter's 16 keys
+  // all in flight at once.
+  for (int it = tid; it < nv * kQ; it += NT) {
+    const int v = it % nv, q = it / nv;
+    const int g = (v * VE) / D, d0 = (v * VE) % D;
+    uint4 raw[kQLen];  // raw 16-byte loads, all in flight; unpacked at the multiply-add
+#pragma unroll
+    for (int u = 0; u < kQLen; ++u) {
+      const int r = q * kQLen + u;
+      const long long t = t0 + r;
+      // evicted position; tokens that evict nothing read their own key (weight 0)
+      const long long j = (r < Tt && t >= K) ? t - K : t0;
+      const Tin* row = j >= pos0 ? kin + ((j - pos0) * nkv + g) * D : win_k + ((j % K) * nkv + g) * D;
+      raw[u] = *reinterpret_cast<const uint4*>(row + d0);
+    }
+    float acc[VE];
+#pragma unroll
+    for (int e = 0; e < VE; ++e) acc[e] = 0.f;
+#pragma unroll
+    for (int u = 0; u < kQLen; ++u) {
+      const float w = s_w[q * kQLen + u];
+      float kv[VE];
+      Load16<Tin>::run(reinterpret_cast<const Tin*>(&raw[u]), kv);
+#pragma unroll
+      for (int e = 0; e < VE; ++e) acc[e] = fmaf(w, kv[e], acc[e]);
+    }
+#pragma unroll
+    for (int e = 0; e < VE; ++e) part[q * ne + v * VE + e] = acc[e];
+  }
+  __syncthreads();
+  float* agg = reinterpret_cast<float*>(p.ws + p.ws_sst) +
+               (static_cast<long long>(s) * p.tiles_per_stream + tile) * ne;
+  for (int e = tid; e < ne; e += NT)  // quarters added in order
+    agg[e] = ((part[e] + part[ne + e]) + part[2 * ne + e]) + part[3 * ne + e];
+}
+
+__global__ void __launch_bounds__(NT) far_carry_kernel(const PrefillParams p) {
+  const int s = blockIdx.y;
+  const int e = blockIdx.x * NT + threadIdx.x;
+  __shared__ int s_ok;
+  pdl_trigger();
+  pdl_wait();  // tile aggregates from far_agg_kernel
+  if (threadIdx.x == 0) s_ok = header_matches(p);
+  __syncthreads();
+  const int ne = p.nkv * (p.H / p.nq);
+  if (!s_ok || e >= ne) return;
+  const long long pos0 = reinterpret_cast<const long long*>(p.ws + p.ws_pos)[s];
+  const float* far = reinterpret_cast<const float*>(stream_block(p, s) + p.so.far);
+  float S = far[e];
+  float* a = reinterpret_cast<float*>(p.ws + p.ws_sst) + static_cast<long long>(s) * p.tiles_per_stream * ne + e;
+  const float gf = p.gamma_far, g64 = powf(gf, static_cast<float>(kTile));
+  const int tiles = p.tiles_per_stream, K = p.K;
+  constexpr int kChunk = 8;  // aggregates in flight per thread
+  for (int t8 = 0; t8 < tiles; t8 += kChunk) {
+    float av[kChunk];
+#pragma unroll
+    for (int u = 0; u < kChunk; ++u) av[u] = (t8 + u < tiles) ? a[static_cast<long long>(t8 + u) * ne] : 0.f;
+#pragma unroll
+    for (int u = 0; u < kChunk; ++u) {
+      const int i = t8 + u;
+      if (i < tiles) {
+        const long long t0 = pos0 + static_cast<long long>(i) * kTile;
+        const long long Tt = min(static_cast<long long>(kTile), p.n - static_cast<long long>(i) * kTile);
+        const long long ev = max(0LL, t0 + Tt - max(t0, static_cast<long long>(K)));
+        const float gev = ev == kTile ? g64 : powf(gf, static_cast<float>(ev));
+        a[static_cast<long long>(i) * ne] = S;
+        S = fmaf(gev, S, av[u]);
+      }
+    }
+  }
+  reinterpret_cast<float*>(p.ws + p.ws_sfin)[static_cast<long long>(s) * ne + e] = S;
 }
 
 // ======================================================================
@@ -156,7 +278,8 @@ __global__ void __launch_bounds__(NT, 2) near_kernel(const PrefillParams p) {
   constexpr int ESZ = static_cast<int>(sizeof(Tin));
   constexpr int C16 = D * ESZ / 16;  // 16-byte chunks of one head row
   constexpr int XS = D + kXsPad;
-  const int h = blockIdx.x, s = blockIdx.y;  // query head, call-relative stream
+  const int h = blockIdx.x % p.nq, seg = blockIdx.x / p.nq;  // query head, segment of tiles
+  const int s = blockIdx.y;                                   // call-relative stream
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   extern __shared__ __align__(16) unsigned char smb[];
   const NearPlan& np = p.near;
@@ -164,23 +287,20 @@ __global__ void __launch_bounds__(NT, 2) near_kernel(const PrefillParams p) {
   __shared__ long long s_pos;
 
   pdl_trigger();
-  pdl_wait();  // the state may be written by the previous kernel of the stream
+  pdl_wait();  // far state at the tile starts from far_carry_kernel
   unsigned char* blk = stream_block(p, s);
   if (tid == 0) {
     s_ok = header_matches(p);
-    s_pos = __ldcg(reinterpret_cast<const long long*>(blk + p.so.pos));
+    s_pos = reinterpret_cast<const long long*>(p.ws + p.ws_pos)[s];
   }
   __syncthreads();
-  if (!s_ok) {  // uniform over the grid
-    if (tid == 0 && h == 0 && s == 0) latch_error(p.err, SFA_ERR_STATE_MISMATCH);
-    return;
-  }
+  if (!s_ok) return;  // latched by far_agg_kernel
   const long long pos0 = s_pos;
-  if (tid == 0 && h == 0) reinterpret_cast<long long*>(p.ws + p.ws_pos)[s] = pos0;
   const int K = p.K, nkv = p.nkv, g = h / p.G;
   const Tin* win_k = reinterpret_cast<const Tin*>(blk + p.so.win_k);
   const Tin* win_v = reinterpret_cast<const Tin*>(blk + p.so.win_v);
-  const float* far = reinterpret_cast<const float*>(blk + p.so.far);
+  const float* sst = reinterpret_cast<const float*>(p.ws + p.ws_sst) +
+                     static_cast<long long>(s) * p.tiles_per_stream * nkv * D + g * D;
   const long long in_row0 = static_cast<long long>(s) * p.n;  // first input row of the stream
   const Tin* qin = static_cast<const Tin*>(p.q) + in_row0 * p.nq * D;
   const Tin* kin = static_cast<const Tin*>(p.k) + in_row0 * nkv * D;
@@ -224,12 +344,13 @@ __global__ void __launch_bounds__(NT, 2) near_kernel(const PrefillParams p) {
     cp_async_commit();
   };
 
-  float sreg = (tid < D) ? far[g * D + tid] : 0.f;  // S of KV head g, dim tid, carried across tiles
   const float gf = p.gamma_far, af = p.alpha_far;
-  const int tiles = p.tiles_per_stream;
-  issue(0, 0);
-  for (int i = 0; i < tiles; ++i) {
-    const int st = (np.stages == 2) ? (i & 1) : 0;
+  const int i0 = seg * p.tps, tiles = min(p.tiles_per_stream, i0 + p.tps);  // this CTA's tiles
+  issue(i0, 0);
+  for (int i = i0; i < tiles; ++i) {
+    const int st = (np.stages == 2) ? ((i - i0) & 1) : 0;
+    // S of KV head g, dim tid, at the tile start
+    float sreg = (tid < D) ? sst[static_cast<long long>(i) * nkv * D + tid] : 0.f;
     if (np.stages == 2 && i + 1 < tiles) {
       issue(i + 1, st ^ 1);  // that stage was released at the end of tile i-1
       cp_async_wait<1>();
@@ -292,9 +413,6 @@ __global__ void __launch_bounds__(NT, 2) near_kernel(const PrefillParams p) {
     __syncthreads();  // the stage and the x tile are free again
     if (np.stages != 2 && i + 1 < tiles) issue(i + 1, 0);
   }
-  // S at the end of the call, from the group's first query head.
-  if (tid < D && h % p.G == 0)
-    reinterpret_cast<float*>(p.ws + p.ws_sfin)[(static_cast<long long>(s) * nkv + g) * D + tid] = sreg;
 }
 
 // Near field and far field on the tensor cores (bf16 inputs, k <= 16).
@@ -312,8 +430,7 @@ __global__ void __launch_bounds__(NT, 2) near_kernel(const PrefillParams p) {
 // m(r) = max(0, r - r_ev + 1).  G[r][c] = alpha_far (1-gamma) gamma^(r-j)
 // for span row c = j+16-k holds the second term, so X = O_near + alpha_far
 // (S_r - gamma^m(r) S0) and the epilogue adds alpha_far gamma^m(r) S0
-// [P1 §2.1 eq. O].  S at the tile end (the next tile's S0) is one dot
-// product per dim over the evicted keys, with no chain from token to token.
+// [P1 §2.1 eq. O]; S0 comes from far_carry_kernel.
 // Operand blocks use the core-matrix layout of sfa_umma.cuh; the key and
 // value blocks put 8-dim groups kDStr bytes apart (16 bytes of padding) so
 // that threads reading one key row hit distinct banks.  The key and value
@@ -332,7 +449,8 @@ __global__ void __launch_bounds__(NT, 2) near_tc_kernel(const PrefillParams p) {
   using Tin = __nv_bfloat16;
   constexpr int C16 = D / 8;  // 16-byte chunks of one head row
   constexpr int kBlkKV = (D / 8) * kDStr;
-  const int h = blockIdx.x, s = blockIdx.y;
+  const int h = blockIdx.x % p.nq, seg = blockIdx.x / p.nq;  // query head, segment of tiles
+  const int s = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   extern __shared__ __align__(16) unsigned char smb[];
   const NearPlan& np = p.near;
@@ -340,31 +458,28 @@ __global__ void __launch_bounds__(NT, 2) near_tc_kernel(const PrefillParams p) {
   __shared__ uint32_t s_tmem;
   __shared__ int s_ok;
   __shared__ long long s_pos;
-  __shared__ float s_s0[128];        // S at the tile start (this head's KV group)
+  __shared__ __align__(16) float s_s0[2][128];  // S at the tile start, per stage
   __shared__ float s_gpow[kTile + 1];  // gamma_far^m
 
   pdl_trigger();
-  pdl_wait();
+  pdl_wait();  // far state at the tile starts from far_carry_kernel
   unsigned char* blk = stream_block(p, s);
   if (tid <= kTile) s_gpow[tid] = powf(p.gamma_far, static_cast<float>(tid));
   if (tid == 0) {
     s_ok = header_matches(p);
-    s_pos = __ldcg(reinterpret_cast<const long long*>(blk + p.so.pos));
+    s_pos = reinterpret_cast<const long long*>(p.ws + p.ws_pos)[s];
     mbar_init(&s_bar, 1);
     mbar_fence_init();
   }
   __syncthreads();
-  if (!s_ok) {
-    if (tid == 0 && h == 0 && s == 0) latch_error(p.err, SFA_ERR_STATE_MISMATCH);
-    return;
-  }
+  if (!s_ok) return;  // latched by far_agg_kernel
   if (warp == 0) tmem_alloc(&s_tmem, kTmemNear);
   const long long pos0 = s_pos;
-  if (tid == 0 && h == 0) reinterpret_cast<long long*>(p.ws + p.ws_pos)[s] = pos0;
   const int K = p.K, nkv = p.nkv, g = h / p.G;
   const Tin* win_k = reinterpret_cast<const Tin*>(blk + p.so.win_k);
   const Tin* win_v = reinterpret_cast<const Tin*>(blk + p.so.win_v);
-  const float* far = reinterpret_cast<const float*>(blk + p.so.far);
+  const float* sst = reinterpret_cast<const float*>(p.ws + p.ws_sst) +
+                     static_cast<long long>(s) * p.tiles_per_stream * nkv * D + g * D;
   const long long in_row0 = static_cast<long long>(s) * p.n;
   const Tin* qin = static_cast<const Tin*>(p.q) + in_row0 * p.nq * D;
   const Tin* kin = static_cast<const Tin*>(p.k) + in_row0 * nkv * D;
@@ -396,8 +511,7 @@ __global__ void __launch_bounds__(NT, 2) near_tc_kernel(const PrefillParams p) {
       *reinterpret_cast<__nv_bfloat16*>(ga_lo + off) = lb;
     }
   };
-  if (tid < D) s_s0[tid] = far[g * D + tid];
-  __syncthreads();  // s_gpow, s_s0
+  __syncthreads();  // s_gpow
   int g_built = -1;
 
   // Copies of tile i into stage st: queries (rows past the tile zero) and
@@ -408,6 +522,7 @@ __global__ void __launch_bounds__(NT, 2) near_tc_kernel(const PrefillParams p) {
     unsigned char* qa = smb + np.q[st];
     unsigned char* kb = smb + np.k[st];
     unsigned char* vb = smb + np.v[st];
+    if (tid < D / 4) cp_async16(&s_s0[st][4 * tid], sst + static_cast<long long>(i) * nkv * D + 4 * tid);
     for (int c = tid; c < kTile * C16; c += NT) {
       const int r = c / C16, u = c % C16;
       unsigned char* dst = qa + blk_off(r, 8 * u);
@@ -435,13 +550,12 @@ __global__ void __launch_bounds__(NT, 2) near_tc_kernel(const PrefillParams p) {
   const uint32_t tmem = s_tmem;
   const uint32_t idesc_qk = umma_idesc_bf16(kTile, kNS, false);
   const uint32_t idesc_pv = umma_idesc_bf16(kTile, D, true);
-  float sreg = 0.f;  // S at the tile end (threads tid < D, dim tid)
-  const int tiles = p.tiles_per_stream;
+  const int i0 = seg * p.tps, tiles = min(p.tiles_per_stream, i0 + p.tps);  // this CTA's tiles
   unsigned par = 0;
   bool ok = true;
-  issue(0, 0);
-  for (int i = 0; i < tiles; ++i) {
-    const int st = (np.stages == 2) ? (i & 1) : 0;
+  issue(i0, 0);
+  for (int i = i0; i < tiles; ++i) {
+    const int st = (np.stages == 2) ? ((i - i0) & 1) : 0;
     if (np.stages == 2 && i + 1 < tiles) {
       issue(i + 1, st ^ 1);
       cp_async_wait<1>();
@@ -467,18 +581,6 @@ __global__ void __launch_bounds__(NT, 2) near_tc_kernel(const PrefillParams p) {
         umma_bf16(tmem, umma_desc(qa + k2 * 2048, 1024, 128), umma_desc(kb + 2 * k2 * kDStr, kDStr, 128),
                   idesc_qk, k2 > 0);
       umma_commit(&s_bar);
-    }
-    // S at the tile end while the scores form: gamma^m S0 plus the evicted
-    // keys' weighted sum (independent terms, four accumulators).
-    if (tid < D) {
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int j = 0; j < kTile; ++j) {
-        const float e = __bfloat162float(*reinterpret_cast<const Tin*>(kb + kv_off(j + 16 - K, tid)));
-        const float w = (j >= r_ev && j < Tt) ? (1.0f - gf) * s_gpow[max(0, Tt - 1 - j)] : 0.f;
-        acc[j & 3] = fmaf(w, e, acc[j & 3]);
-      }
-      sreg = fmaf(s_gpow[max(0, Tt - r_ev)], s_s0[tid], (acc[0] + acc[1]) + (acc[2] + acc[3]));
     }
     if (!mbar_wait_bounded(&s_bar, par, kMbarPollLimit, p.err)) ok = false;
     par ^= 1u;
@@ -556,7 +658,7 @@ __global__ void __launch_bounds__(NT, 2) near_tc_kernel(const PrefillParams p) {
         float v[32];
         tmem_ld32(tmem + (static_cast<uint32_t>(32 * sp) << 16) + kTmemO + colh + c0, v);
         if (lane < 16 && r < Tt && ok) {
-          const float* s0 = s_s0 + colh + c0;
+          const float* s0 = s_s0[st] + colh + c0;
 #pragma unroll
           for (int j = 0; j < 32; j += 4)
             *reinterpret_cast<float4*>(orow + c0 + j) =
@@ -566,12 +668,9 @@ __global__ void __launch_bounds__(NT, 2) near_tc_kernel(const PrefillParams p) {
       }
     }
     tc_fence_before();
-    __syncthreads();  // stage, P, S0 and accumulators free again
-    if (tid < D) s_s0[tid] = sreg;  // read after the next tile's barriers
+    __syncthreads();  // stage, P and accumulators free again
     if (np.stages != 2 && i + 1 < tiles) issue(i + 1, 0);
   }
-  if (tid < D && h % p.G == 0)
-    reinterpret_cast<float*>(p.ws + p.ws_sfin)[(static_cast<long long>(s) * nkv + g) * D + tid] = sreg;
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
@@ -791,9 +890,9 @@ struct OutPlan {
   static constexpr int tmem = 64;
   static constexpr int img = 128;                         // [hi, lo] slot block of the columns
   static constexpr int wb = img + 2 * kBlkBytes;          // [2][hi, lo] weight blocks
-  static constexpr int xt = wb + 2 * 2 * kBlkBytes;       // [2][64][64] fp32 x tiles
-  static constexpr int halo = xt + 2 * kTile * kBlk * 4;  // [15][64] x before the tile
-  static constexpr int sem = halo + kHalo * kBlk * 4;     // [64][65] sem
+  // [2][15 + 64][64] fp32: x of the 15 positions before the tile, then the tile
+  static constexpr int xt = wb + 2 * 2 * kBlkBytes;
+  static constexpr int sem = xt + 2 * (kHalo + kTile) * kBlk * 4;  // [64][65] sem
   static constexpr int segc = sem + kTile * kScStride * 4;  // [kSeg][64] field segment aggregates
   static constexpr int fcar = segc + kSeg * kBlk * 4;     // [64] field at the tile start
   static constexpr int total = fcar + kBlk * 4;
@@ -808,7 +907,6 @@ __global__ void __launch_bounds__(NT, 2) out_kernel(const PrefillParams p) {
   uint64_t* bar_w = bar_img + 1;    // [2] weight blocks landed
   uint64_t* bar_mma = bar_img + 3;  // sem MMAs done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smb + OutPlan::tmem);
-  float* halo = reinterpret_cast<float*>(smb + OutPlan::halo);
   float* semc = reinterpret_cast<float*>(smb + OutPlan::sem);
   float* segc = reinterpret_cast<float*>(smb + OutPlan::segc);
   float* fcar = reinterpret_cast<float*>(smb + OutPlan::fcar);
@@ -844,8 +942,10 @@ __global__ void __launch_bounds__(NT, 2) out_kernel(const PrefillParams p) {
   auto tile_rows = [&](int i) -> int {
     return static_cast<int>(min(static_cast<long long>(kTile), p.n - static_cast<long long>(i) * kTile));
   };
+  constexpr int XR = kHalo + kTile;  // rows of an x stage
+  auto xstage = [&](int st) -> float* { return reinterpret_cast<float*>(smb + OutPlan::xt) + st * XR * kBlk; };
   auto issue_x = [&](int i, int st) {
-    float* xt = reinterpret_cast<float*>(smb + OutPlan::xt) + st * kTile * kBlk;
+    float* xt = xstage(st) + kHalo * kBlk;
     const int Tt = tile_rows(i);
     const float* src = p.out + (in_row0 + static_cast<long long>(i) * kTile) * p.H + col0;
     for (int c = tid; c < Tt * (kBlk / 4); c += NT) {
@@ -872,7 +972,7 @@ __global__ void __launch_bounds__(NT, 2) out_kernel(const PrefillParams p) {
   for (int idx = tid; idx < kHalo * kBlk; idx += NT) {
     const int q = idx / kBlk, c = idx % kBlk;
     const long long t = pos0 - kHalo + q;
-    halo[idx] = t >= 0 ? ring[static_cast<size_t>(t % kRing) * p.H + col0 + c] : 0.f;
+    xstage(0)[idx] = t >= 0 ? ring[static_cast<size_t>(t % kRing) * p.H + col0 + c] : 0.f;
   }
   if (tid < kBlk) fcar[tid] = field[col0 + tid];
   if (tid < kSeg) s_gseg[tid] = powf(ge, static_cast<float>(kSegLen));
@@ -915,13 +1015,23 @@ __global__ void __launch_bounds__(NT, 2) out_kernel(const PrefillParams p) {
       umma_commit(bar_mma);
     }
     __syncthreads();  // x tile i visible to all threads
-    const float* xt = reinterpret_cast<const float*>(smb + OutPlan::xt) + st * kTile * kBlk;
-    auto xat = [&](int r) -> float { return r >= 0 ? xt[r * kBlk + cc] : halo[(r + kHalo) * kBlk + cc]; };
-    // field: segment aggregates from zero, then carries in segment order
-    const int r_lo = sg * kSegLen, r_hi = min(Tt, r_lo + kSegLen);
+    // Thread (column cc, segment sg) owns tokens r_lo .. r_lo+15 of its
+    // column.  Its x values for positions t0+r_lo-15 .. t0+r_lo+15 (stage
+    // rows r_lo .. r_lo+30; rows past the tile hold stale values that no
+    // result uses) go to registers in one batch.
+    const float* xb = xstage(st);
+    const int r_lo = sg * kSegLen;
+    float xv[kSegLen + kHalo];
+#pragma unroll
+    for (int u = 0; u < kSegLen + kHalo; ++u) xv[u] = xb[(r_lo + u) * kBlk + cc];
+    // field: this segment's aggregate from zero [P3 §2.1 channel 2]
     {
       float a = 0.f;
-      for (int r = r_lo; r < r_hi; ++r) a = ewma(ge, a, xt[r * kBlk + cc]);
+#pragma unroll
+      for (int u = 0; u < kSegLen; ++u) {
+        const float an = ewma(ge, a, xv[kHalo + u]);
+        a = (r_lo + u < Tt) ? an : a;
+      }
       segc[sg * kBlk + cc] = a;
     }
     if (!mbar_wait_bounded(bar_mma, static_cast<unsigned>(i & 1), kMbarPollLimit, p.err)) ok = false;
@@ -940,48 +1050,50 @@ __global__ void __launch_bounds__(NT, 2) out_kernel(const PrefillParams p) {
     __syncthreads();
     float f = fcar[cc];
     for (int s2 = 0; s2 < sg; ++s2) f = fmaf(s_gseg[s2], f, segc[s2 * kBlk + cc]);
-    // ring: sum of the 16 positions ending at r [P3 §2.4: mean over all 16
-    // slots]; fusion, clip and scale [P3 §2.2]
-    float* orow = p.out + (in_row0 + (t0 - pos0)) * p.H + col0 + cc;
-    if (r_lo < r_hi) {
-      float rs = 0.f;
-      for (int r = r_lo - kHalo; r <= r_lo; ++r) rs += xat(r);
-      for (int r = r_lo; r < r_hi; ++r) {
-        if (r > r_lo) rs += xat(r) - xat(r - kRing);
-        const float x = xt[r * kBlk + cc];
-        f = ewma(ge, f, x);
-        float u = rs * (1.0f / kRing) + 0.5f * f + 0.5f * semc[r * kScStride + cc];
-        u = fminf(fmaxf(u, -p.clip_eps), p.clip_eps);
-        if (ok) orow[static_cast<long long>(r) * p.H] = fmaf(a_l, u, x);
-      }
+    float sv[kSegLen];
+#pragma unroll
+    for (int u = 0; u < kSegLen; ++u) sv[u] = semc[(r_lo + u) * kScStride + cc];
+    // ring: sum of the 16 positions ending at token r [P3 §2.4: mean over all
+    // 16 slots], sliding; fusion, clip and scale [P3 §2.2]
+    float rs = 0.f;
+#pragma unroll
+    for (int u = 0; u < kRing; ++u) rs += xv[u];
+    float* orow = p.out + (in_row0 + (t0 - pos0) + r_lo) * p.H + col0 + cc;
+#pragma unroll
+    for (int u = 0; u < kSegLen; ++u) {
+      if (u > 0) rs += xv[kHalo + u] - xv[u - 1];
+      const float x = xv[kHalo + u];
+      const bool live = r_lo + u < Tt;
+      const float fn = ewma(ge, f, x);
+      f = live ? fn : f;
+      float uu = rs * (1.0f / kRing) + 0.5f * f + 0.5f * sv[u];
+      uu = fminf(fmaxf(uu, -p.clip_eps), p.clip_eps);
+      if (live && ok) orow[static_cast<long long>(u) * p.H] = fmaf(a_l, uu, x);
     }
-    const bool seg_last = r_lo < Tt && r_hi == Tt;  // this segment holds the tile's last token
+    const bool seg_last = r_lo < Tt && r_lo + kSegLen >= Tt;  // this segment holds the tile's last token
     if (i == tiles - 1 && ok) {
       const int gi = col0 + cc;
       if (seg_last) field[gi] = f;
       if (sg == 0) {
         // ring slots of the last 16 positions that belong to this call, and
-        // the exact sum over all 16
+        // the exact sum over all 16 (position q is stage row q - t0 + 15)
         const long long t_end = t0 + Tt - 1;
         float tot = 0.f;
         for (int r = 0; r < kRing; ++r) {
           const long long q = t_end - (kRing - 1) + r;
           if (q < 0) continue;
-          const float v = xat(static_cast<int>(q - t0));
+          const float v = xb[static_cast<int>(q - t0 + kHalo) * kBlk + cc];
           if (q >= pos0) ring[static_cast<size_t>(q % kRing) * p.H + gi] = v;
           tot += v;
         }
         ring_sum[gi] = tot;
       }
     }
-    __syncthreads();  // segc, fcar and the halo are read above
+    __syncthreads();  // segc and fcar are read above
     if (seg_last) fcar[cc] = f;
-    if (i + 1 < tiles)  // the last 15 x rows become the next tile's halo (Tt = 64 here)
-      for (int idx = tid; idx < kHalo * kBlk; idx += NT) {
-        const int q = idx / kBlk, c = idx % kBlk;
-        halo[idx] = xt[(kTile - kHalo + q) * kBlk + c];
-      }
-    __syncthreads();  // the x stage, halo and carries are ready for the next tile
+    if (i + 1 < tiles)  // the tile's last 15 x rows lead the next stage (Tt = 64 here)
+      for (int idx = tid; idx < kHalo * kBlk; idx += NT) xstage(st ^ 1)[idx] = xb[kTile * kBlk + idx];
+    __syncthreads();  // the x stage, halo rows and carries are ready for the next tile
   }
 
   // One CTA per stream: window, S and position [P1 §2.2].
@@ -1043,10 +1155,16 @@ cudaError_t launch_pdl(K kernel, dim3 grid, int smem, cudaStream_t s, const Pref
 
 template <typename Tin, int D>
 cudaError_t launch_t(const PrefillParams& p, cudaStream_t s) {
-  const dim3 g1(static_cast<unsigned>(p.nq), static_cast<unsigned>(p.n_streams), 1);
-  const dim3 g2(static_cast<unsigned>(p.tiles_per_stream), static_cast<unsigned>(p.n_streams), 1);
-  const dim3 g3(static_cast<unsigned>(p.H / kBlk), static_cast<unsigned>(p.n_streams), 1);
-  cudaError_t e;
+  const unsigned ns = static_cast<unsigned>(p.n_streams);
+  const int ne = p.nkv * D;
+  const dim3 g0(static_cast<unsigned>(p.tiles_per_stream), ns, 1);
+  const dim3 gc(static_cast<unsigned>((ne + NT - 1) / NT), ns, 1);
+  const dim3 g1(static_cast<unsigned>(p.nq * p.n_seg), ns, 1);
+  const dim3 g2(static_cast<unsigned>(p.tiles_per_stream), ns, 1);
+  const dim3 g3(static_cast<unsigned>(p.H / kBlk), ns, 1);
+  cudaError_t e = launch_pdl(far_agg_kernel<Tin, D>, g0, 4 * ne * 4, s, p);
+  if (e == cudaSuccess) e = launch_pdl(far_carry_kernel, gc, 0, s, p);
+  if (e != cudaSuccess) return e;
   if constexpr (sizeof(Tin) == 2) {
     if (p.near.tc) e = launch_pdl(near_tc_kernel<D>, g1, p.near.total, s, p);
     else e = launch_pdl(near_kernel<Tin, D>, g1, p.near.total, s, p);
@@ -1126,6 +1244,10 @@ cudaError_t prefill_prepare(int device) {
   if (e == cudaSuccess) e = set_smem(near_kernel<__nv_bfloat16, 128>, optin);
   if (e == cudaSuccess) e = set_smem(near_tc_kernel<64>, optin);
   if (e == cudaSuccess) e = set_smem(near_tc_kernel<128>, optin);
+  if (e == cudaSuccess) e = set_smem(far_agg_kernel<float, 64>, optin);
+  if (e == cudaSuccess) e = set_smem(far_agg_kernel<float, 128>, optin);
+  if (e == cudaSuccess) e = set_smem(far_agg_kernel<__nv_bfloat16, 64>, optin);
+  if (e == cudaSuccess) e = set_smem(far_agg_kernel<__nv_bfloat16, 128>, optin);
   if (e == cudaSuccess) e = set_smem(pool_kernel, optin);
   if (e == cudaSuccess) e = set_smem(out_kernel<float>, optin);
   if (e == cudaSuccess) e = set_smem(out_kernel<__nv_bfloat16>, optin);
