@@ -160,7 +160,12 @@ SFA_API int sfa_prefill(const sfa_handle* h, const void* q, const void* k, const
                 size_t workspace_bytes, void* stream);
 
 /* Folds one token per sequence into the state and writes its output.
- * One kernel launch covers all layers and sequences; no workspace. */
+ * One kernel launch covers all layers and sequences; no workspace.
+ * The kernel may start, and read q, k and v, while the previous SFA call on
+ * the same stream is still running (programmatic dependent launch; the
+ * state is read only after that call has finished).  So q, k and v must not
+ * be memory that an earlier SFA call on the stream writes (its out or
+ * state); inputs written by any other kernel are safe. */
 SFA_API int sfa_decode_step(const sfa_handle* h, const void* q, const void* k, const void* v,
                     int batch, void* state, float* out, void* stream);
 
@@ -193,7 +198,8 @@ SFA_API int sfa_prefill_layers(const sfa_handle* h, int layer_begin, int layer_c
  * [layer_count][n_seq][n_kv][d], out [layer_count][n_seq][hidden] fp32.
  * Sequences not listed keep their state and position.  An index out of range
  * is skipped on the device and latched as SFA_ERR_INVALID_ARG for
- * sfa_check_device_status; host-visible errors as for sfa_decode_step. */
+ * sfa_check_device_status; host-visible errors, and the condition on q, k
+ * and v, as for sfa_decode_step. */
 SFA_API int sfa_decode_step_ex(const sfa_handle* h, int layer_begin, int layer_count,
                                const int* seq_ids, int n_seq, const void* q, const void* k,
                                const void* v, int batch, void* state, float* out, void* stream);

@@ -20,13 +20,15 @@
 //
 // Latency.  A decode step of a small batch is bound by memory latency, not
 // bandwidth.  Every operand a CTA needs is brought into shared memory by the
-// bulk-copy engine in one batch: the slot slice before the kernel waits on
-// its predecessor (programmatic dependent launch; slots are constant), the
-// query slice, the new key/value, the window, S, field and ring sum right
-// after.  Only the ring slot t mod 16 depends on the position and follows
-// one round trip later, overlapped with the near field.  All arithmetic
-// then runs from shared memory.  A window too large for the shared-memory
-// budget is read from global memory instead.
+// bulk-copy engine in a few large copies: before the kernel waits on its
+// predecessor (programmatic dependent launch), the slot slice (constant;
+// stored per CTA with padded rows at init) and this call's q, K_t and V_t
+// (which no earlier SFA call on the stream writes); right after, S, field,
+// ring sum and the window (all KV heads of every slot in one copy each for
+// K and V where it fits).  Only the ring slot t mod 16 depends on the
+// position and follows one round trip later, overlapped with the near field.
+// All arithmetic then runs from shared memory.  A window too large for the
+// shared-memory budget is read from global memory instead.
 //
 // Ordering.  The window slot t mod k and the far state S are read by every
 // CTA that needs that KV head and written by one owner CTA (the one holding
@@ -139,6 +141,7 @@ decode_kernel(const DecodeParams p) {
   uint64_t* bar_sl = reinterpret_cast<uint64_t*>(smb + pl.bars);
   uint64_t* bar_in = bar_sl + 1;
   uint64_t* bar_red = bar_sl + 2;
+  uint64_t* bar_q = bar_sl + 3;     // this call's q, K_t, V_t
   float* sl = reinterpret_cast<float*>(smb + pl.sl);        // [64][HS+4] slot slice
   float* xs = reinterpret_cast<float*>(smb + pl.xs);        // [HS] x_t
   float* red = reinterpret_cast<float*>(smb + pl.red);      // [NW][68] per-warp pool partials
@@ -161,6 +164,7 @@ decode_kernel(const DecodeParams p) {
     mbar_init(bar_sl, 1);
     mbar_init(bar_in, 1);
     mbar_init(bar_red, 1);
+    mbar_init(bar_q, 1);
     mbar_fence_init();
     // the partials of all CS ranks (this one included) complete the phase
     mbar_arrive_expect_tx(bar_red, static_cast<unsigned>(p.CS) * kRedBytes);
@@ -185,7 +189,23 @@ decode_kernel(const DecodeParams p) {
   const float inrm0 = 1.f / nrm[lane], inrm1 = 1.f / nrm[lane + 32];
   const float a_l = p.alpha_layer[l];
 
-  pdl_wait();  // state and inputs may be written by the previous kernel
+  // This call's query slice and K_t, V_t of the CTA's KV heads.  No earlier
+  // SFA call on the stream writes them (a condition of the C ABI), so they
+  // are fetched before the wait below; decode inputs usually come from HBM,
+  // and this takes that latency off the critical path.
+  const long long io = static_cast<long long>(li) * p.n_seq + bi;  // input / output row
+  const Tin* qin = static_cast<const Tin*>(p.q) + (io * p.nq + h0) * D;
+  const Tin* kin = static_cast<const Tin*>(p.k) + io * nkv * D;
+  const Tin* vin = static_cast<const Tin*>(p.v) + io * nkv * D;
+  if (tid == 32) {
+    const unsigned hb = static_cast<unsigned>(NG * D * ESZ);
+    mbar_arrive_expect_tx(bar_q, static_cast<unsigned>(HS * ESZ) + 2u * hb);
+    bulk_g2s(qraw, qin, static_cast<unsigned>(HS * ESZ), bar_q);
+    bulk_g2s(kc, kin + g_lo * D, hb, bar_q);
+    bulk_g2s(vc, vin + g_lo * D, hb, bar_q);
+  }
+
+  pdl_wait();  // the state may be written by the previous kernel
 
   // Sequence served: from the caller's list, checked against the batch (an
   // index out of range leaves the cluster without touching the state).
@@ -194,7 +214,6 @@ decode_kernel(const DecodeParams p) {
   const bool b_ok = b >= 0 && b < p.B;
   if (!b_ok) b = 0;
   const long long stream = static_cast<long long>(l) * p.B + b;  // state stream
-  const long long io = static_cast<long long>(li) * p.n_seq + bi;  // input / output row
   unsigned char* blk = p.state + kHeaderBytes + stream * p.so.stride;
   Tin* win_k = reinterpret_cast<Tin*>(blk + p.so.win_k);
   Tin* win_v = reinterpret_cast<Tin*>(blk + p.so.win_v);
@@ -202,9 +221,6 @@ decode_kernel(const DecodeParams p) {
   float* field = reinterpret_cast<float*>(blk + p.so.field);
   float* ring_sum = reinterpret_cast<float*>(blk + p.so.ring_sum);
   float* ring = reinterpret_cast<float*>(blk + p.so.ring);
-  const Tin* qin = static_cast<const Tin*>(p.q) + (io * p.nq + h0) * D;
-  const Tin* kin = static_cast<const Tin*>(p.k) + io * nkv * D;
-  const Tin* vin = static_cast<const Tin*>(p.v) + io * nkv * D;
 
   if (tid == 0) {  // header and position: independent loads, one round trip
     const uint4 h0v = __ldcg(reinterpret_cast<const uint4*>(p.state));
@@ -217,16 +233,12 @@ decode_kernel(const DecodeParams p) {
            (hd.n_layers == p.L);
     s_pos = pos;
   }
-  if (warp == 1) {  // everything else of this stream, one batch of copies
+  if (warp == 1) {  // the rest of this stream's state, one batch of copies
     const unsigned hb = static_cast<unsigned>(NG * D * ESZ);
-    unsigned bytes = static_cast<unsigned>(HS * ESZ) + 2u * hb + static_cast<unsigned>(NG * D * 4) +
-                     2u * static_cast<unsigned>(HS * 4);
+    unsigned bytes = static_cast<unsigned>(NG * D * 4) + 2u * static_cast<unsigned>(HS * 4);
     if (pl.stage_win) bytes += 2u * static_cast<unsigned>(K) * (pl.whole ? static_cast<unsigned>(pl.rec) : hb);
     if (lane == 0) mbar_arrive_expect_tx(bar_in, bytes);
     __syncwarp();
-    if (lane == 0) bulk_g2s(qraw, qin, static_cast<unsigned>(HS * ESZ), bar_in);
-    if (lane == 1) bulk_g2s(kc, kin + g_lo * D, hb, bar_in);
-    if (lane == 2) bulk_g2s(vc, vin + g_lo * D, hb, bar_in);
     if (lane == 3) bulk_g2s(sg, far + g_lo * D, static_cast<unsigned>(NG * D * 4), bar_in);
     if (lane == 4) bulk_g2s(fld, field + rank * HS, static_cast<unsigned>(HS * 4), bar_in);
     if (lane == 5) bulk_g2s(rsm, ring_sum + rank * HS, static_cast<unsigned>(HS * 4), bar_in);
@@ -243,6 +255,7 @@ decode_kernel(const DecodeParams p) {
   __syncthreads();
   if (!s_ok || !b_ok) {  // uniform over the cluster (same header, same sequence)
     mbar_wait_bounded(bar_sl, 0, kMbarPollLimit, p.err);  // no copy may land after exit
+    mbar_wait_bounded(bar_q, 0, kMbarPollLimit, p.err);
     mbar_wait_bounded(bar_in, 0, kMbarPollLimit, p.err);
     cluster_wait();
     if (tid == 0 && rank == 0) {
@@ -272,6 +285,7 @@ decode_kernel(const DecodeParams p) {
     ring_old[m] = (m < ncol && ehalf == 0) ? ring_row[ecol + m * kColsPerPass] : 0.f;
 
   bool ok = mbar_wait_bounded(bar_in, 0, kMbarPollLimit, p.err);
+  ok = mbar_wait_bounded(bar_q, 0, kMbarPollLimit, p.err) && ok;
 
   // Window slot of the a-th window position (a = 0 .. nwin-1 is position
   // j0+a).
