@@ -200,6 +200,15 @@ decode_tile_kernel(const DecodeParams p) {
       float m = -INFINITY, den = 0.f, o[EPL];
 #pragma unroll
       for (int e = 0; e < EPL; ++e) o[e] = 0.f;
+      // A window of one chunk (k <= 16): its value rows are loaded together
+      // with the key rows, one round trip instead of two.
+      constexpr int kPre = KPC <= 16 ? KPC : 1;
+      float vpre[kPre][EPL];
+      if (KPC <= 16 && nwin <= KPC) {
+#pragma unroll
+        for (int u = 0; u < kPre; ++u)
+          VecLoad<Tin, EPL>::run(wrow(win_v, vt, min(u, nwin - 1)) + lane * EPL, vpre[u]);
+      }
       for (int base = 0; base < nwin; base += KPC) {
         const int cnt = min(KPC, nwin - base);
         float s;
@@ -228,6 +237,14 @@ decode_tile_kernel(const DecodeParams p) {
         den = fmaf(den, corr, ps);
 #pragma unroll
         for (int e = 0; e < EPL; ++e) o[e] *= corr;
+        if (KPC <= 16 && nwin <= KPC) {
+#pragma unroll
+          for (int u = 0; u < kPre; ++u) {
+            const float pc = __shfl_sync(0xffffffffu, pj, (u * LPK) & 31);  // 0 past cnt
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) o[e] = fmaf(pc, vpre[u][e], o[e]);
+          }
+        } else
         for (int c0 = 0; c0 < cnt; c0 += 8) {
           float vv[8][EPL];
 #pragma unroll

@@ -687,31 +687,31 @@ __global__ void __launch_bounds__(NT, 2) near_tc_kernel(const PrefillParams p) {
 struct PoolPlan {
   static constexpr int bars = 0;                        // 6 mbarriers
   static constexpr int tmem = 64;                       // tensor-memory address
-  static constexpr int xf = 128;                        // [2][64][64] fp32 x chunks
-  static constexpr int img = xf + 2 * kBlk * kBlk * 4;  // [2][hi, lo] slot blocks
-  static constexpr int xsp = img + 2 * 2 * kBlkBytes;   // [2][hi, lo] split x blocks
+  static constexpr int img = 128;                       // [3][hi, lo] slot blocks
+  static constexpr int xsp = img + 3 * 2 * kBlkBytes;   // [2][hi, lo] split x blocks
   static constexpr int sc = xsp + 2 * 2 * kBlkBytes;    // [64][65] fp32 scores
-  static constexpr int ss = sc + kTile * kScStride * 4; // [64] |x|^2
-  static constexpr int total = ss + kTile * 4;
+  static constexpr int ss = sc + kTile * kScStride * 4; // [16][64] |x|^2 partials
+  static constexpr int total = ss + 16 * kTile * 4;
 };
 
 __global__ void __launch_bounds__(NT, 2) pool_kernel(const PrefillParams p) {
   const int tile = blockIdx.x, s = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   extern __shared__ __align__(16) unsigned char smb[];
-  uint64_t* bar_img = reinterpret_cast<uint64_t*>(smb + PoolPlan::bars);  // [2] slot blocks landed
-  uint64_t* bar_mma = bar_img + 2;                                       // [2] MMAs of a stage done
-  uint64_t* bar_probe = bar_img + 4;                                     // test hook only
+  uint64_t* bar_img = reinterpret_cast<uint64_t*>(smb + PoolPlan::bars);  // [3] slot blocks landed
+  uint64_t* bar_mma = bar_img + 3;                                       // [2] MMAs of a split stage done
+  uint64_t* bar_probe = bar_img + 5;                                     // test hook only
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smb + PoolPlan::tmem);
   float* sc = reinterpret_cast<float*>(smb + PoolPlan::sc);
-  float* ssq = reinterpret_cast<float*>(smb + PoolPlan::ss);
+  float* sqp = reinterpret_cast<float*>(smb + PoolPlan::ss);
   __shared__ int s_ok;
+  __shared__ float ssq[kTile];
 
   pdl_trigger();
   pdl_wait();  // x is written by near_kernel
   if (tid == 0) {
     s_ok = header_matches(p);
-    for (int b = 0; b < 5; ++b) mbar_init(bar_img + b, 1);
+    for (int b = 0; b < 6; ++b) mbar_init(bar_img + b, 1);
     mbar_fence_init();
   }
   __syncthreads();
@@ -725,70 +725,72 @@ __global__ void __launch_bounds__(NT, 2) pool_kernel(const PrefillParams p) {
   const unsigned char* img_l = p.slot_img + static_cast<size_t>(l) * nch * 2 * kBlkBytes;
   bool ok = true;
 
-  // Copies of chunk c into stage st: x columns 64c .. 64c+63 of the tile's
-  // rows (rows past the tile are zero) and the slot blocks of the chunk.
-  auto issue_x = [&](int c, int st) {
-    float* xf = reinterpret_cast<float*>(smb + PoolPlan::xf) + st * kBlk * kBlk;
-    for (int i = tid; i < kBlk * kBlk / 4; i += NT) {
-      const int r = i / (kBlk / 4), c4 = (i % (kBlk / 4)) * 4;
-      if (r < Tt) cp_async16(xf + r * kBlk + c4, xrow0 + static_cast<long long>(r) * p.H + c * kBlk + c4);
-      else *reinterpret_cast<float4*>(xf + r * kBlk + c4) = make_float4(0.f, 0.f, 0.f, 0.f);
+  // Thread tid handles 4 columns c4 .. c4+3 of rows r_m (m = 0..3) of every
+  // chunk.  The mapping makes a warp's split stores cover whole 128-byte
+  // lines of the core-matrix layout (row r & 7 in lane bits 0-2, column bit
+  // 2 in lane bit 3).
+  const int c4 = ((tid >> 4) & 7) * 8 + ((tid >> 3) & 1) * 4;
+  auto row_of = [&](int m) { return (2 * m + (tid >> 7)) * 8 + (tid & 7); };
+  // x chunk c (columns 64c ..) into registers, rows past the tile zero.
+  auto load_x = [&](int c, float4 (&v)[4]) {
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int r = row_of(m);
+      v[m] = r < Tt ? __ldcg(reinterpret_cast<const float4*>(xrow0 + static_cast<long long>(r) * p.H + c * kBlk + c4))
+                    : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    cp_async_commit();
   };
-  auto issue_img = [&](int c, int st) {  // one thread
+  auto issue_img = [&](int c) {  // one thread; stage c % 3
+    const int st = c % 3;
     mbar_arrive_expect_tx(bar_img + st, 2u * kBlkBytes);
     bulk_g2s(smb + PoolPlan::img + st * 2 * kBlkBytes, img_l + static_cast<size_t>(c) * 2 * kBlkBytes,
              2u * kBlkBytes, bar_img + st);
   };
   if (tid == 0) {
-    issue_img(0, 0);
-    if (nch > 1) issue_img(1, 1);
+    issue_img(0);
+    if (nch > 1) issue_img(1);
   }
-  issue_x(0, 0);
-  if (nch > 1) issue_x(1, 1);
+  float4 nxt[4];
+  load_x(0, nxt);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t idesc = umma_idesc_bf16(kBlk, kSlots, false);
 
-  // |x|^2: thread tid covers columns 4*(tid%16) .. +3 of rows tid/16 + 16m.
-  float sq[4] = {0.f, 0.f, 0.f, 0.f};
+  float sq[4] = {0.f, 0.f, 0.f, 0.f};  // |x|^2 of rows r_m over this thread's columns
   for (int c = 0; c < nch; ++c) {
+    float4 cur[4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) cur[m] = nxt[m];
+    if (c + 1 < nch) load_x(c + 1, nxt);  // in flight during this chunk
     const int st = c & 1;
-    const unsigned ph = static_cast<unsigned>((c >> 1) & 1);
-    if (c + 1 < nch) cp_async_wait<1>();
-    else cp_async_wait<0>();
-    __syncthreads();  // x chunk c visible to all threads
     // The split blocks of stage st were read by the MMAs of chunk c-2.
-    if (c >= 2 && !mbar_wait_bounded(bar_mma + st, ph ^ 1u, kMbarPollLimit, p.err)) ok = false;
-    const float* xf = reinterpret_cast<const float*>(smb + PoolPlan::xf) + st * kBlk * kBlk;
+    if (c >= 2 && !mbar_wait_bounded(bar_mma + st, static_cast<unsigned>(((c - 2) >> 1) & 1), kMbarPollLimit, p.err))
+      ok = false;
     unsigned char* xhi = smb + PoolPlan::xsp + st * 2 * kBlkBytes;
     unsigned char* xlo = xhi + kBlkBytes;
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
-      const int i = m * NT + tid;
-      const int r = i / (kBlk / 4), c4 = (i % (kBlk / 4)) * 4;
-      const float4 v = *reinterpret_cast<const float4*>(xf + r * kBlk + c4);
+      const float4 v = cur[m];
       sq[m] = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, sq[m]))));
       __nv_bfloat16 hh[4], ll[4];
       split_bf16(v.x, hh[0], ll[0]);
       split_bf16(v.y, hh[1], ll[1]);
       split_bf16(v.z, hh[2], ll[2]);
       split_bf16(v.w, hh[3], ll[3]);
-      const int off = blk_off(r, c4);
+      const int off = blk_off(row_of(m), c4);
       *reinterpret_cast<uint2*>(xhi + off) = *reinterpret_cast<const uint2*>(hh);
       *reinterpret_cast<uint2*>(xlo + off) = *reinterpret_cast<const uint2*>(ll);
     }
     fence_proxy_async_smem();
     tc_fence_before();
-    __syncthreads();  // split blocks written; x chunk c consumed
-    if (c + 2 < nch) issue_x(c + 2, st);
+    __syncthreads();  // split blocks of chunk c written
     if (tid == 0) {
-      if (!mbar_wait_bounded(bar_img + st, ph, kMbarPollLimit, p.err)) ok = false;
+      const int si = c % 3;
+      if (!mbar_wait_bounded(bar_img + si, static_cast<unsigned>((c / 3) & 1), kMbarPollLimit, p.err)) ok = false;
       tc_fence_after();
-      const unsigned char* shi = smb + PoolPlan::img + st * 2 * kBlkBytes;
+      const unsigned char* shi = smb + PoolPlan::img + si * 2 * kBlkBytes;
       const unsigned char* slo = shi + kBlkBytes;
 #pragma unroll
       for (int k = 0; k < kBlk / 16; ++k) {
@@ -799,21 +801,25 @@ __global__ void __launch_bounds__(NT, 2) pool_kernel(const PrefillParams p) {
         umma_bf16(tmem, al, bh, idesc, true);
       }
       umma_commit(bar_mma + st);
-      if (c + 2 < nch) {  // the slot blocks of stage st are free once these MMAs finish
-        if (!mbar_wait_bounded(bar_mma + st, ph, kMbarPollLimit, p.err)) ok = false;
-        issue_img(c + 2, st);
+      if (c + 2 < nch) {
+        // stage (c+2) % 3 held chunk c-1's slot blocks: wait for its MMAs
+        // (committed one chunk ago), then reload it
+        if (c >= 1 && !mbar_wait_bounded(bar_mma + ((c - 1) & 1), static_cast<unsigned>(((c - 1) >> 1) & 1),
+                                         kMbarPollLimit, p.err))
+          ok = false;
+        issue_img(c + 2);
       }
     }
   }
-  // |x|^2 per row: 16 threads (half a warp) share a row.
+  // |x|^2 per row: the 16 threads sharing a row add their partials in order.
 #pragma unroll
-  for (int m = 0; m < 4; ++m) {
-    float v = sq[m];
-    v += __shfl_xor_sync(0xffffffffu, v, 8);
-    v += __shfl_xor_sync(0xffffffffu, v, 4);
-    v += __shfl_xor_sync(0xffffffffu, v, 2);
-    v += __shfl_xor_sync(0xffffffffu, v, 1);
-    if ((tid & 15) == 0) ssq[m * (NT / 16) + tid / 16] = v;
+  for (int m = 0; m < 4; ++m) sqp[((tid >> 3) & 15) * kTile + row_of(m)] = sq[m];
+  __syncthreads();
+  if (tid < kTile) {
+    float v = 0.f;
+#pragma unroll
+    for (int q = 0; q < 16; ++q) v += sqp[q * kTile + tid];
+    ssq[tid] = v;
   }
   // Test hook: a bounded wait on a barrier that nothing completes.
   if (tid == 0 && static_cast<long long>(tile) * p.n_streams + s == p.withhold_tile) {
