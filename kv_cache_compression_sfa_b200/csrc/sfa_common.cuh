@@ -194,6 +194,17 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// 3-D tiled bulk tensor load (no multicast) of the box at coordinates
+// (x, y, z) of `map` into shared memory, completion counted in bytes on
+// `bar`.  x times the element size must be a multiple of 16 bytes; other
+// coordinates may lie outside the tensor (those elements read as zero).
+__device__ __forceinline__ void tma_load_3d(void* dst, const void* map, int x, int y, int z, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::
+          "r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // Orders this thread's earlier generic-proxy shared-memory accesses before
 // later bulk copies (async proxy) into the same bytes.
 __device__ __forceinline__ void fence_proxy_async_smem() {

@@ -7,6 +7,7 @@
 //   [P3] "Dalin Soma SFA基于信号场注意力机制的神经网络推理加速框架"
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cstddef>
 #include <cstdint>
@@ -120,6 +121,13 @@ struct PrefillParams {
   long long withhold_tile;  // test hook: this tile's pool CTA waits on a barrier nothing completes
   NearPlan near;
   int pool_smem, out_smem;
+};
+
+// Tensor maps of one prefill call's q, k and v for the tensor-core near field:
+// 3-D views (head dim, head, token row over all streams of the call) whose
+// 8-element x 1 x T-row boxes land as one column of core matrices.
+struct NearMaps {
+  CUtensorMap q, k, v;
 };
 
 // Workspace layout for a prefill call (bytes); nothing in it needs clearing.

@@ -40,6 +40,7 @@
 // is on its own copies or MMAs and is bounded; a wait that runs out latches
 // SFA_ERR_DEVICE_TIMEOUT and the kernel still finishes.
 #include <cuda_bf16.h>
+#include <cudaTypedefs.h>
 
 #include <algorithm>
 #include <cstring>
@@ -431,12 +432,13 @@ __global__ void __launch_bounds__(NT, 2) near_kernel(const PrefillParams p) {
 // for span row c = j+16-k holds the second term, so X = O_near + alpha_far
 // (S_r - gamma^m(r) S0) and the epilogue adds alpha_far gamma^m(r) S0
 // [P1 §2.1 eq. O]; S0 comes from far_carry_kernel.
-// Operand blocks use the core-matrix layout of sfa_umma.cuh; the key and
-// value blocks put 8-dim groups kDStr bytes apart (16 bytes of padding) so
-// that threads reading one key row hit distinct banks.  The key and value
-// blocks are the MN-major B of G.K and P.V.
+// Operand blocks use the core-matrix layout of sfa_umma.cuh; in the key and
+// value blocks the 8-dim groups are kDStr bytes apart, each a column of
+// kNS core-matrix rows that one tensor copy fills.  The key and value
+// blocks are the MN-major B of G.K and P.V.  Tensor copies need 128-byte
+// aligned shared-memory destinations: the blocks start at multiples of 128.
 constexpr int kNS = kTile + 16;
-constexpr int kDStr = (kNS / 8) * 128 + 16;
+constexpr int kDStr = (kNS / 8) * 128;
 constexpr int kTmemNear = 256;
 constexpr int kTmemO = 128;
 
@@ -445,16 +447,20 @@ __device__ __forceinline__ int kv_off(int c, int d) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(NT, 2) near_tc_kernel(const PrefillParams p) {
+__global__ void __launch_bounds__(NT, 2)
+near_tc_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ NearMaps maps) {
   using Tin = __nv_bfloat16;
   constexpr int C16 = D / 8;  // 16-byte chunks of one head row
   constexpr int kBlkKV = (D / 8) * kDStr;
   const int h = blockIdx.x % p.nq, seg = blockIdx.x / p.nq;  // query head, segment of tiles
   const int s = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  extern __shared__ __align__(16) unsigned char smb[];
+  extern __shared__ __align__(128) unsigned char smb_raw[];
+  // 128-byte aligned base (the plan leaves 128 bytes of slack)
+  unsigned char* smb = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smb_raw) + 127) & ~static_cast<uintptr_t>(127));
   const NearPlan& np = p.near;
   __shared__ __align__(8) uint64_t s_bar;
+  __shared__ __align__(8) uint64_t s_ld[2];  // tensor copies of a stage landed
   __shared__ uint32_t s_tmem;
   __shared__ int s_ok;
   __shared__ long long s_pos;
@@ -469,6 +475,8 @@ __global__ void __launch_bounds__(NT, 2) near_tc_kernel(const PrefillParams p) {
     s_ok = header_matches(p);
     s_pos = reinterpret_cast<const long long*>(p.ws + p.ws_pos)[s];
     mbar_init(&s_bar, 1);
+    mbar_init(&s_ld[0], 1);
+    mbar_init(&s_ld[1], 1);
     mbar_fence_init();
   }
   __syncthreads();
@@ -514,34 +522,49 @@ __global__ void __launch_bounds__(NT, 2) near_tc_kernel(const PrefillParams p) {
   __syncthreads();  // s_gpow
   int g_built = -1;
 
-  // Copies of tile i into stage st: queries (rows past the tile zero) and
-  // the span rows of positions t0-16 .. t0+Tt-1 (others zero).
+  // Copies of tile i into stage st by the tensor-copy engine: D/8 boxes of
+  // [64 tokens x 8 dims] for the queries and of [kNS rows x 8 dims] for the
+  // key and value span (positions t0-16 .. t0+63), each landing as one
+  // column of core matrices.  Token rows count over all streams of the
+  // call, so rows past the stream hold another stream's inputs (finite,
+  // masked out) and rows past the call read as zero; the first tile's rows
+  // before the call are replaced from the state window (fix_history).
+  constexpr unsigned kTileBytes = static_cast<unsigned>((D / 8) * (kTile + 2 * kNS) * 16);
+  const int row0 = static_cast<int>(static_cast<long long>(s) * p.n);  // first token row of the stream
   auto issue = [&](int i, int st) {
-    const long long t0 = pos0 + static_cast<long long>(i) * kTile;
-    const int Tt = static_cast<int>(min(static_cast<long long>(kTile), p.n - static_cast<long long>(i) * kTile));
     unsigned char* qa = smb + np.q[st];
     unsigned char* kb = smb + np.k[st];
     unsigned char* vb = smb + np.v[st];
     if (tid < D / 4) cp_async16(&s_s0[st][4 * tid], sst + static_cast<long long>(i) * nkv * D + 4 * tid);
-    for (int c = tid; c < kTile * C16; c += NT) {
-      const int r = c / C16, u = c % C16;
-      unsigned char* dst = qa + blk_off(r, 8 * u);
-      if (r < Tt) cp_async16(dst, qin + ((t0 - pos0 + r) * p.nq + h) * D + 8 * u);
-      else *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
-    }
-    for (int c = tid; c < kNS * C16; c += NT) {
-      const int r = c / C16, u = c % C16;
-      const long long j = t0 - 16 + r;
-      const int off = kv_off(r, 8 * u);
-      if (j >= 0 && r < 16 + Tt) {
-        cp_async16(kb + off, krow_g(j) + 8 * u);
-        cp_async16(vb + off, vrow_g(j) + 8 * u);
-      } else {
-        *reinterpret_cast<uint4*>(kb + off) = make_uint4(0u, 0u, 0u, 0u);
-        *reinterpret_cast<uint4*>(vb + off) = make_uint4(0u, 0u, 0u, 0u);
+    cp_async_commit();
+    if (tid == 0) {
+      const int rq = row0 + i * kTile, rkv = rq - 16;
+      mbar_arrive_expect_tx(&s_ld[st], kTileBytes);
+#pragma unroll
+      for (int u = 0; u < D / 8; ++u) {
+        tma_load_3d(qa + u * 1024, &maps.q, 8 * u, h, rq, &s_ld[st]);
+        tma_load_3d(kb + u * kDStr, &maps.k, 8 * u, g, rkv, &s_ld[st]);
+        tma_load_3d(vb + u * kDStr, &maps.v, 8 * u, g, rkv, &s_ld[st]);
       }
     }
-    cp_async_commit();
+  };
+  // Span rows 0..15 of the call's first tile: positions before the call
+  // from the state window, before position 0 zero.
+  auto fix_history = [&](int st) {
+    unsigned char* kb = smb + np.k[st];
+    unsigned char* vb = smb + np.v[st];
+    for (int c = tid; c < 16 * C16; c += NT) {
+      const int r = c / C16, u = c % C16;
+      const long long j = pos0 - 16 + r;
+      const int off = kv_off(r, 8 * u);
+      uint4 kv = make_uint4(0u, 0u, 0u, 0u), vv = kv;
+      if (j >= 0) {
+        kv = *reinterpret_cast<const uint4*>(krow_g(j) + 8 * u);
+        vv = *reinterpret_cast<const uint4*>(vrow_g(j) + 8 * u);
+      }
+      *reinterpret_cast<uint4*>(kb + off) = kv;
+      *reinterpret_cast<uint4*>(vb + off) = vv;
+    }
   };
 
   tc_fence_before();
@@ -556,12 +579,15 @@ __global__ void __launch_bounds__(NT, 2) near_tc_kernel(const PrefillParams p) {
   issue(i0, 0);
   for (int i = i0; i < tiles; ++i) {
     const int st = (np.stages == 2) ? ((i - i0) & 1) : 0;
+    const unsigned ld_par = static_cast<unsigned>(((np.stages == 2) ? ((i - i0) >> 1) : (i - i0)) & 1);
     if (np.stages == 2 && i + 1 < tiles) {
       issue(i + 1, st ^ 1);
       cp_async_wait<1>();
     } else {
       cp_async_wait<0>();
     }
+    if (!mbar_wait_bounded(&s_ld[st], ld_par, kMbarPollLimit, p.err)) ok = false;
+    if (i == 0) fix_history(st);  // the call's first tile (the copies above have landed)
     const long long t0 = pos0 + static_cast<long long>(i) * kTile;
     const int Tt = static_cast<int>(min(static_cast<long long>(kTile), p.n - static_cast<long long>(i) * kTile));
     const int r_ev = static_cast<int>(max(0LL, min(static_cast<long long>(Tt), K - t0)));
@@ -1159,6 +1185,41 @@ cudaError_t launch_pdl(K kernel, dim3 grid, int smem, cudaStream_t s, const Pref
   return cudaLaunchKernelEx(&cfg, kernel, p);
 }
 
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// against the driver library).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// q as (D, n_q, rows) and k, v as (D, n_kv, rows) bf16 tensors, rows = every
+// token of every stream of the call; boxes of 8 x 1 x T.
+cudaError_t encode_near_maps(const PrefillParams& p, int D, NearMaps* m) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return cudaErrorNotSupported;
+  const cuuint64_t rows = static_cast<cuuint64_t>(p.n_streams) * static_cast<cuuint64_t>(p.n);
+  if (rows > 0x7fffffffULL) return cudaErrorInvalidValue;  // 32-bit coordinates
+  const cuuint32_t estr[3] = {1, 1, 1};
+  auto one = [&](CUtensorMap* map, const void* base, int heads, int box_rows) -> bool {
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(heads), rows};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(heads) * D * 2};
+    const cuuint32_t box[3] = {8, 1, static_cast<cuuint32_t>(box_rows)};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  };
+  if (!one(&m->q, p.q, p.nq, kTile) || !one(&m->k, p.k, p.nkv, kNS) || !one(&m->v, p.v, p.nkv, kNS))
+    return cudaErrorInvalidValue;
+  return cudaSuccess;
+}
+
 template <typename Tin, int D>
 cudaError_t launch_t(const PrefillParams& p, cudaStream_t s) {
   const unsigned ns = static_cast<unsigned>(p.n_streams);
@@ -1172,8 +1233,25 @@ cudaError_t launch_t(const PrefillParams& p, cudaStream_t s) {
   if (e == cudaSuccess) e = launch_pdl(far_carry_kernel, gc, 0, s, p);
   if (e != cudaSuccess) return e;
   if constexpr (sizeof(Tin) == 2) {
-    if (p.near.tc) e = launch_pdl(near_tc_kernel<D>, g1, p.near.total, s, p);
-    else e = launch_pdl(near_kernel<Tin, D>, g1, p.near.total, s, p);
+    if (p.near.tc) {
+      NearMaps maps;
+      e = encode_near_maps(p, D, &maps);
+      if (e == cudaSuccess) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = g1;
+        cfg.blockDim = dim3(NT, 1, 1);
+        cfg.dynamicSmemBytes = static_cast<size_t>(p.near.total);
+        cfg.stream = s;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, near_tc_kernel<D>, p, maps);
+      }
+    } else {
+      e = launch_pdl(near_kernel<Tin, D>, g1, p.near.total, s, p);
+    }
   } else {
     e = launch_pdl(near_kernel<Tin, D>, g1, p.near.total, s, p);
   }
@@ -1232,7 +1310,7 @@ bool plan_near(int D, int esz, int K, size_t limit, bool tc, NearPlan* out) {
     }
   }
   p.stages = stages;
-  p.total = off;
+  p.total = off + (tc ? 128 : 0);  // tensor cores: slack to align the base to 128 bytes
   if (static_cast<size_t>(p.total) > limit) return false;
   *out = p;
   return true;
