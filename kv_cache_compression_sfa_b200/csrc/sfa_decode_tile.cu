@@ -81,7 +81,7 @@ decode_tile_kernel(const DecodeParams p) {
   const int HPC = p.HPC, HS = HPC * D, XS = HS + 4, nch = HS / kBlk;
   const int K = p.K, G = p.G, nkv = p.nkv;
   const int h0 = rank * HPC;
-  const int g_lo = h0 / G, g_hi = (h0 + HPC - 1) / G;
+  const int g_hi = (h0 + HPC - 1) / G;
   const int own_lo = (h0 + G - 1) / G;  // KV heads whose window and S this CTA writes
   const int tiles_per_layer = (p.n_seq + TB - 1) / TB;
   const int ti = static_cast<int>(blockIdx.x) / p.CS;

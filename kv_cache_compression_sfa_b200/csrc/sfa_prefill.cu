@@ -451,7 +451,6 @@ __global__ void __launch_bounds__(NT, 2)
 near_tc_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ NearMaps maps) {
   using Tin = __nv_bfloat16;
   constexpr int C16 = D / 8;  // 16-byte chunks of one head row
-  constexpr int kBlkKV = (D / 8) * kDStr;
   const int h = blockIdx.x % p.nq, seg = blockIdx.x / p.nq;  // query head, segment of tiles
   const int s = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -489,7 +488,6 @@ near_tc_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ 
   const float* sst = reinterpret_cast<const float*>(p.ws + p.ws_sst) +
                      static_cast<long long>(s) * p.tiles_per_stream * nkv * D + g * D;
   const long long in_row0 = static_cast<long long>(s) * p.n;
-  const Tin* qin = static_cast<const Tin*>(p.q) + in_row0 * p.nq * D;
   const Tin* kin = static_cast<const Tin*>(p.k) + in_row0 * nkv * D;
   const Tin* vin = static_cast<const Tin*>(p.v) + in_row0 * nkv * D;
   auto krow_g = [&](long long j) -> const Tin* {
