@@ -103,6 +103,15 @@ EDGE = [
      [("p", 77), ("d", 9)]),
     ("eight_heads_per_cta", dict(n_q_heads=16, n_kv_heads=16, head_dim=64, window_k=3),
      [("p", 66), ("d", 2)]),
+    # bf16, k <= 16: the tensor-core near field with tensor copies; short and
+    # ragged calls put a call's first tile (rows before the call from the
+    # state window) next to stream boundaries
+    ("bf16_small_chunks", dict(n_layers=2, batch=2, n_q_heads=4, n_kv_heads=2, head_dim=64,
+                               window_k=12, in_dtype="bf16"),
+     [("p", 3), ("p", 17), ("d", 2), ("p", 64), ("p", 1), ("p", 130), ("d", 3)]),
+    ("bf16_d128_small_chunks", dict(n_layers=1, batch=3, n_q_heads=4, n_kv_heads=1, head_dim=128,
+                                    window_k=16, in_dtype="bf16"),
+     [("p", 15), ("p", 16), ("p", 65), ("d", 1), ("p", 2)]),
 ]
 
 
@@ -110,6 +119,15 @@ EDGE = [
 def test_edge_schedules(name, over, schedule):
     w = _tiny_variant(name=name, **over)
     _run_schedule(w, schedule)
+
+
+def test_cuda_core_near_field_on_bf16_inputs(monkeypatch):
+    """bf16 inputs with k <= 16 take the tensor-core near field; the handle's
+    test hook keeps them on the CUDA cores, which must meet the same bar."""
+    monkeypatch.setenv("SFA_CUDA_CORE_NEAR_FIELD", "1")
+    w = _tiny_variant(name="cuda_core_near_bf16", n_layers=2, batch=2, n_q_heads=14,
+                      n_kv_heads=2, head_dim=64, window_k=16, in_dtype="bf16")
+    _run_schedule(w, [("p", 130), ("d", 5), ("p", 70)])
 
 
 def test_gqa7_bf16_chunked_prefill_and_decode():
