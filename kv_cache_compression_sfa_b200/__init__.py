@@ -340,6 +340,10 @@ def sfa_prefill_static_ws(h: Handle, q, k, v, n: int, batch: int, state: torch.T
 
 def sfa_decode_step(h: Handle, q, k, v, batch: int, state: torch.Tensor, out: torch.Tensor,
                     stream=None) -> None:
+    """One token per sequence, all layers.  The kernel may read q, k and v
+    before the previous SFA call on the stream has finished, so they must not
+    be memory that an earlier SFA call writes (its out or state); inputs
+    written by any other kernel are safe."""
     qp, kp, vp = _qkv_checks(h, q, k, v, 1, batch)
     sp = _dev(state, "state", torch.uint8, sfa_state_bytes(h, batch))
     op = _dev(out, "out", torch.float32, h.cfg.n_layers * batch * h.cfg.hidden)
@@ -353,6 +357,9 @@ def sfa_check_device_status(h: Handle, stream=None) -> int:
 
 
 def sfa_debug_set_lookback(h: Handle, spin_limit: int = 0, withhold_tile: int = -1) -> None:
+    """Test hook of the prefill's bounded waits: the pool CTA of tile
+    `withhold_tile` (tile * streams + stream) waits on a barrier that nothing
+    completes, giving up after `spin_limit` polls (0: default); -1 disables."""
     rc = load_library().sfa_debug_set_lookback(h.ptr, spin_limit, withhold_tile)
     if rc != SFA_OK:
         raise SfaError(rc, "sfa_debug_set_lookback")
