@@ -153,6 +153,9 @@ SFA_API int sfa_state_reset(const sfa_handle* h, void* state, int batch, void* s
 /* Folds n >= 0 tokens per sequence into the state and writes their outputs.
  * Equivalent to n calls of sfa_decode_step (same results within rounding).
  * Continues from each stream's current position.  n == 0 enqueues nothing.
+ * SFA_ERR_UNSUPPORTED when layers x batch x n exceeds 2^31 - 1 (bf16 inputs
+ * with k <= 16: the tensor copies use 32-bit row coordinates; split the
+ * call) or layers x batch exceeds 65535.
  * workspace: sfa_prefill_workspace_bytes(h, batch, n) bytes (may be NULL if
  * that is 0); workspace_bytes is its size, checked. */
 SFA_API int sfa_prefill(const sfa_handle* h, const void* q, const void* k, const void* v,

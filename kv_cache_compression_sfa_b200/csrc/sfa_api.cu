@@ -426,6 +426,8 @@ int sfa_prefill_layers(const sfa_handle* h, int layer_begin, int layer_count, co
   const long long streams = static_cast<long long>(layer_count) * batch;
   const long long tiles_per_stream = (n + kTile - 1) / kTile;
   if (streams > 65535 || tiles_per_stream > 0x7fffffffLL) return SFA_ERR_UNSUPPORTED;
+  // the tensor copies of the near field address token rows with 32-bit coordinates
+  if (h->near.tc && streams * n > 0x7fffffffLL) return SFA_ERR_UNSUPPORTED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   PrefillParams p;
   std::memset(&p, 0, sizeof(p));
