@@ -118,7 +118,12 @@ __device__ __forceinline__ void st_async_v4(unsigned addr, float4 v, unsigned ba
       : "memory");
 }
 
-template <typename Tin, int D>
+// Near-field variants, chosen on the host per launch so that each kernel
+// holds one copy of the near-field loop: window staged in shared memory or
+// read from global memory, and window positions a warp scores at a time.
+constexpr int kVarT4 = 0, kVarT8 = 1, kVarT16 = 2, kVarT32 = 3, kVarF8 = 4, kVarF32 = 5;
+
+template <typename Tin, int D, int VAR>
 __global__ void __launch_bounds__(kDecodeThreads, 2)
 decode_kernel(const DecodeParams p) {
   constexpr int EPL = D / 32;  // elements of a head row per lane in P·V
@@ -383,23 +388,10 @@ decode_kernel(const DecodeParams p) {
       }
     }
   };
-  using T_ = std::true_type;
-  using F_ = std::false_type;
-  using K4 = std::integral_constant<int, 4>;
-  using K8 = std::integral_constant<int, 8>;
-  using K16 = std::integral_constant<int, 16>;
-  using K32 = std::integral_constant<int, 32>;
   {
-    const int pmax = (K + wph - 1) / wph;  // most positions a warp ever takes
-    if (pl.stage_win) {
-      if (pmax <= 4) near_part(T_{}, K4{});
-      else if (pmax <= 8) near_part(T_{}, K8{});
-      else if (pmax <= 16) near_part(T_{}, K16{});
-      else near_part(T_{}, K32{});
-    } else {
-      if (pmax <= 8) near_part(F_{}, K8{});
-      else near_part(F_{}, K32{});
-    }
+    constexpr bool kStaged = VAR < kVarF8;
+    constexpr int kKpc = (VAR == kVarT4) ? 4 : (VAR == kVarT8 || VAR == kVarF8) ? 8 : (VAR == kVarT16) ? 16 : 32;
+    near_part(std::integral_constant<bool, kStaged>{}, std::integral_constant<int, kKpc>{});
   }
   __syncthreads();
 
@@ -562,9 +554,18 @@ decode_kernel(const DecodeParams p) {
   }
 }
 
-template <typename Tin, int D>
-cudaError_t launch_t(const DecodeParams& p, cudaStream_t s) {
-  const DecodePlan pl = decode_plan(p.HPC, D, static_cast<int>(sizeof(Tin)), p.NGm, p.nkv, p.K, p.smem_budget);
+// The near-field variant a launch needs (the kernel's own choice of warps
+// per head and window staging, made on the host).
+int decode_variant(const DecodeParams& p, const DecodePlan& pl) {
+  int wph = 1;
+  while (wph * 2 * p.HPC <= NW) wph *= 2;
+  const int pmax = (p.K + wph - 1) / wph;  // most positions a warp ever takes
+  if (pl.stage_win) return pmax <= 4 ? kVarT4 : pmax <= 8 ? kVarT8 : pmax <= 16 ? kVarT16 : kVarT32;
+  return pmax <= 8 ? kVarF8 : kVarF32;
+}
+
+template <typename Tin, int D, int VAR>
+cudaError_t launch_v(const DecodeParams& p, const DecodePlan& pl, cudaStream_t s) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.CS, p.n_seq, p.Lc);
   cfg.blockDim = dim3(kDecodeThreads, 1, 1);
@@ -579,21 +580,47 @@ cudaError_t launch_t(const DecodeParams& p, cudaStream_t s) {
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, decode_kernel<Tin, D>, p);
+  return cudaLaunchKernelEx(&cfg, decode_kernel<Tin, D, VAR>, p);
+}
+
+template <typename Tin, int D>
+cudaError_t launch_t(const DecodeParams& p, cudaStream_t s) {
+  const DecodePlan pl = decode_plan(p.HPC, D, static_cast<int>(sizeof(Tin)), p.NGm, p.nkv, p.K, p.smem_budget);
+  switch (decode_variant(p, pl)) {
+    case kVarT4: return launch_v<Tin, D, kVarT4>(p, pl, s);
+    case kVarT8: return launch_v<Tin, D, kVarT8>(p, pl, s);
+    case kVarT16: return launch_v<Tin, D, kVarT16>(p, pl, s);
+    case kVarT32: return launch_v<Tin, D, kVarT32>(p, pl, s);
+    case kVarF8: return launch_v<Tin, D, kVarF8>(p, pl, s);
+    default: return launch_v<Tin, D, kVarF32>(p, pl, s);
+  }
+}
+
+template <typename Tin, int D, int VAR>
+cudaError_t prepare_v(int optin) {
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, decode_kernel<Tin, D, VAR>);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(decode_kernel<Tin, D, VAR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             optin - static_cast<int>(fa.sharedSizeBytes));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(decode_kernel<Tin, D, VAR>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  return e;
 }
 
 template <typename Tin, int D>
 cudaError_t prepare_t(int optin) {
-  cudaFuncAttributes fa;
-  cudaError_t e = cudaFuncGetAttributes(&fa, decode_kernel<Tin, D>);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(decode_kernel<Tin, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             optin - static_cast<int>(fa.sharedSizeBytes));
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(decode_kernel<Tin, D>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  cudaError_t e = prepare_v<Tin, D, kVarT4>(optin);
+  if (e == cudaSuccess) e = prepare_v<Tin, D, kVarT8>(optin);
+  if (e == cudaSuccess) e = prepare_v<Tin, D, kVarT16>(optin);
+  if (e == cudaSuccess) e = prepare_v<Tin, D, kVarT32>(optin);
+  if (e == cudaSuccess) e = prepare_v<Tin, D, kVarF8>(optin);
+  if (e == cudaSuccess) e = prepare_v<Tin, D, kVarF32>(optin);
   return e;
 }
 
+// Clusters of `cs` CTAs resident at once (shared memory bounds it; the
+// variants differ only in the near-field loop).
 template <typename Tin, int D>
 int max_clusters_t(int cs, size_t smem) {
   cudaLaunchConfig_t cfg = {};
@@ -608,7 +635,7 @@ int max_clusters_t(int cs, size_t smem) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, decode_kernel<Tin, D>, &cfg) != cudaSuccess) {
+  if (cudaOccupancyMaxActiveClusters(&n, decode_kernel<Tin, D, kVarT32>, &cfg) != cudaSuccess) {
     cudaGetLastError();
     return 0;
   }
