@@ -83,7 +83,7 @@ typedef struct sfa_config {
   int ring_size;       /* must be 16                       [P3 §2.1 ch. 1]   */
   float ema_gamma;     /* EMA field decay (0.98)           [P3 §2.1 ch. 2]   */
   int n_slots;         /* must be 64                       [P3 §2.1 ch. 3]   */
-  float temperature;   /* pool temperature (0.07), > 0     [P3 §2.1 ch. 3]   */
+  float temperature;   /* pool temperature (0.07), > 0, 1/T finite [P3 §2.1] */
   float clip_eps;      /* enhancement clip ε (0.5), >= 0   [P3 §2.2]         */
   float alpha_base;    /* base strength (0.1)              [P3 §2.2]         */
   float cross_decay;   /* per-layer decay (0.8)            [P3 §2.2]         */
@@ -130,7 +130,10 @@ SFA_API int sfa_state_layout_for(const sfa_config* cfg, int batch, sfa_state_lay
 
 /* Creates a handle on the current device: validates cfg, copies the slots,
  * precomputes slot norms and the alpha_layer table, allocates the device
- * error word.  *out receives the handle, or NULL on error. */
+ * error word.  *out receives the handle, or NULL on error.  Returns the
+ * status of sfa_config_validate for a bad configuration, SFA_ERR_UNSUPPORTED
+ * when a kernel's shared-memory plan does not fit the current device, and
+ * SFA_ERR_CUDA when a CUDA call fails (no device, out of memory). */
 SFA_API int sfa_init(const sfa_config* cfg, sfa_handle** out);
 
 /* Frees the handle's device memory (synchronises the device first). */
@@ -140,10 +143,11 @@ SFA_API int sfa_destroy(sfa_handle* h);
 SFA_API size_t sfa_state_bytes(const sfa_handle* h, int batch);
 
 /* Bytes of prefill workspace for a call of n tokens x `batch`; 0 on invalid
- * input.  The workspace holds each stream's position at the start of the
- * call, the far-field state at its end and the pool weights of every
- * 64-token tile (16 KB per tile and stream); its content need not be
- * initialised. */
+ * input or a call beyond sfa_prefill's limits (below).  The workspace holds
+ * each stream's position at the start of the call, the far-field state at its
+ * end, and per 64-token tile and stream the pool weights (16 KB) and the
+ * far-field state at the tile's start (n_kv x d fp32); its content need not
+ * be initialised. */
 SFA_API size_t sfa_prefill_workspace_bytes(const sfa_handle* h, int batch, long long n);
 
 /* Zeroes `state` (state_bytes(h, batch) bytes) and writes its header for
@@ -153,9 +157,10 @@ SFA_API int sfa_state_reset(const sfa_handle* h, void* state, int batch, void* s
 /* Folds n >= 0 tokens per sequence into the state and writes their outputs.
  * Equivalent to n calls of sfa_decode_step (same results within rounding).
  * Continues from each stream's current position.  n == 0 enqueues nothing.
- * SFA_ERR_UNSUPPORTED when layers x batch x n exceeds 2^31 - 1 (bf16 inputs
- * with k <= 16: the tensor copies use 32-bit row coordinates; split the
- * call) or layers x batch exceeds 65535.
+ * SFA_ERR_UNSUPPORTED when layers x batch exceeds 65535, n exceeds
+ * 64 x (2^31 - 1), or layers x batch x n exceeds 2^31 - 1 with bf16 inputs
+ * and k <= 16 (the tensor copies use 32-bit row coordinates; split the
+ * call).
  * workspace: sfa_prefill_workspace_bytes(h, batch, n) bytes (may be NULL if
  * that is 0); workspace_bytes is its size, checked. */
 SFA_API int sfa_prefill(const sfa_handle* h, const void* q, const void* k, const void* v,
@@ -179,7 +184,8 @@ SFA_API int sfa_decode_step(const sfa_handle* h, const void* q, const void* k, c
  * sequences; the arithmetic is exactly that of the full calls.
  *
  * Bytes of prefill workspace for a sfa_prefill_layers call of layer_count
- * layers; 0 on invalid input (layer_count outside 1 .. n_layers). */
+ * layers; 0 on invalid input (layer_count outside 1 .. n_layers) or a call
+ * beyond sfa_prefill's limits. */
 SFA_API size_t sfa_prefill_layers_workspace_bytes(const sfa_handle* h, int layer_count, int batch,
                                                   long long n);
 

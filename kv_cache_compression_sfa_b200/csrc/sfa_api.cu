@@ -127,6 +127,15 @@ PrefillWorkspace prefill_workspace(const sfa_config* c, int layers, int batch, l
   return w;
 }
 
+// Limits of one prefill call: its kernels put the layers x batch streams in
+// gridDim.y (at most 65535) and count a stream's tiles in 32 bits.  Checked
+// before any size arithmetic, which these bounds keep below 2^63.
+int prefill_shape_status(int layers, int batch, long long n) {
+  if (static_cast<long long>(layers) * batch > 65535) return SFA_ERR_UNSUPPORTED;
+  if (n > 0x7fffffffLL * kTile) return SFA_ERR_UNSUPPORTED;
+  return SFA_OK;
+}
+
 // Most KV heads any CTA of a cluster of `cs` needs.
 int max_kv_heads_per_cta(int nq, int nkv, int cs) {
   const int hpc = nq / cs, g = nq / nkv;
@@ -206,7 +215,8 @@ int sfa_config_validate(const sfa_config* c) {
     if (!std::isfinite(s)) return SFA_ERR_INVALID_ARG;
   if (c->gamma_far < 0.f || c->gamma_far > 1.f || c->ema_gamma < 0.f || c->ema_gamma > 1.f)
     return SFA_ERR_INVALID_ARG;
-  if (!(c->temperature > 0.f) || c->clip_eps < 0.f) return SFA_ERR_INVALID_ARG;
+  if (!(c->temperature > 0.f) || !std::isfinite(1.0f / c->temperature) || c->clip_eps < 0.f)
+    return SFA_ERR_INVALID_ARG;
   if (c->in_dtype != SFA_F32 && c->in_dtype != SFA_BF16) return SFA_ERR_INVALID_ARG;
   if (c->slots == nullptr) return SFA_ERR_INVALID_ARG;
   if (!aligned16(c->slots)) return SFA_ERR_ALIGNMENT;
@@ -257,6 +267,7 @@ int sfa_init(const sfa_config* cfg, sfa_handle** out) {
     h->tile_mode = (tenv && tenv[0] == '0') ? 0 : (tenv && tenv[0] == '1') ? 1 : -1;
   }
   const int L = cfg->n_layers, H = hidden_of(cfg);
+  bool no_fit = false;  // a kernel's shared-memory plan does not fit this device
   const size_t slot_bytes = sizeof(float) * static_cast<size_t>(L) * kSlots * H;
   cudaError_t e = cudaGetDevice(&h->device);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&h->n_sm, cudaDevAttrMultiProcessorCount, h->device);
@@ -283,9 +294,10 @@ int sfa_init(const sfa_config* cfg, sfa_handle** out) {
     const bool tc = !(nenv && nenv[0] == '1');
     if (!(tc && plan_near(cfg->head_dim, esz, cfg->window_k, limit, true, &h->near)) &&
         !plan_near(cfg->head_dim, esz, cfg->window_k, limit, false, &h->near))
-      e = cudaErrorInvalidConfiguration;
+      no_fit = true;
     if (static_cast<size_t>(std::max(prefill_pool_smem(), prefill_out_smem())) > limit)
-      e = cudaErrorInvalidConfiguration;
+      no_fit = true;
+    if (no_fit) e = cudaErrorInvalidConfiguration;
     for (int cs : cluster_candidates(cfg->n_q_heads, cfg->head_dim)) {
       if (e != cudaSuccess) break;
       const int hpc = cfg->n_q_heads / cs;
@@ -302,7 +314,10 @@ int sfa_init(const sfa_config* cfg, sfa_handle** out) {
                    decode_tile_max_active_clusters(cs, tsm, cfg->in_dtype, cfg->head_dim) >= 1;
       break;
     }
-    if (e == cudaSuccess && h->cs == 0) e = cudaErrorInvalidConfiguration;
+    if (e == cudaSuccess && h->cs == 0) {
+      no_fit = true;
+      e = cudaErrorInvalidConfiguration;
+    }
     if (e == cudaSuccess) {
       // Each decode CTA's slot slice [64][HS] laid out contiguously with the
       // rows padded to HS + 4 floats, as in its shared memory: one bulk copy.
@@ -342,7 +357,7 @@ int sfa_init(const sfa_config* cfg, sfa_handle** out) {
     cudaFree(h->err);
     h->magic = 0;
     delete h;
-    return SFA_ERR_CUDA;
+    return no_fit ? SFA_ERR_UNSUPPORTED : SFA_ERR_CUDA;
   }
   h->cfg.slots = h->slots;
   *out = h;
@@ -380,6 +395,7 @@ size_t sfa_prefill_layers_workspace_bytes(const sfa_handle* h, int layer_count, 
   if (!handle_ok(h) || batch <= 0 || n <= 0 || layer_count <= 0 ||
       layer_count > h->cfg.n_layers)
     return 0;
+  if (prefill_shape_status(layer_count, batch, n) != SFA_OK) return 0;
   return static_cast<size_t>(prefill_workspace(&h->cfg, layer_count, batch, n).total);
 }
 
@@ -420,12 +436,13 @@ int sfa_prefill_layers(const sfa_handle* h, int layer_begin, int layer_count, co
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(state) || !aligned16(out) ||
       !aligned16(workspace))
     return SFA_ERR_ALIGNMENT;
+  const int shape = prefill_shape_status(layer_count, batch, n);
+  if (shape != SFA_OK) return shape;
   const sfa_config* c = &h->cfg;
   const PrefillWorkspace w = prefill_workspace(c, layer_count, batch, n);
   if (!workspace || workspace_bytes < static_cast<size_t>(w.total)) return SFA_ERR_WORKSPACE;
   const long long streams = static_cast<long long>(layer_count) * batch;
   const long long tiles_per_stream = (n + kTile - 1) / kTile;
-  if (streams > 65535 || tiles_per_stream > 0x7fffffffLL) return SFA_ERR_UNSUPPORTED;
   // the tensor copies of the near field address token rows with 32-bit coordinates
   if (h->near.tc && streams * n > 0x7fffffffLL) return SFA_ERR_UNSUPPORTED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

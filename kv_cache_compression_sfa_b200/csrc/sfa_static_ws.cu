@@ -58,7 +58,9 @@ int sfa_prefill_static_ws(const sfa_handle* h, const void* q, const void* k, con
   if (n < 0 || batch <= 0) return SFA_ERR_INVALID_ARG;
   if (n == 0) return SFA_OK;
   const size_t need = sfa_prefill_workspace_bytes(h, batch, n);
-  if (need == 0) return SFA_ERR_INVALID_ARG;
+  // 0: a bad handle or a call beyond sfa_prefill's limits; sfa_prefill
+  // returns that status without launching anything.
+  if (need == 0) return sfa_prefill(h, q, k, v, n, batch, state, out, nullptr, 0, stream);
   if (need > kStaticWorkspaceBytes) return SFA_ERR_WORKSPACE;  // call exceeds the fixed scratch
   void* ws = nullptr;
   const int rc = static_ws_address(&ws);

@@ -83,6 +83,7 @@ def _cfg(**kw):
     ({"ring_size": 8}, sfa.SFA_ERR_UNSUPPORTED),
     ({"n_slots": 32}, sfa.SFA_ERR_UNSUPPORTED),
     ({"temperature": 0.0}, sfa.SFA_ERR_INVALID_ARG),
+    ({"temperature": 1e-45}, sfa.SFA_ERR_INVALID_ARG),   # 1/T overflows to inf
     ({"gamma_far": 1.5}, sfa.SFA_ERR_INVALID_ARG),
     ({"ema_gamma": float("nan")}, sfa.SFA_ERR_INVALID_ARG),
     ({"clip_eps": -1.0}, sfa.SFA_ERR_INVALID_ARG),

@@ -46,6 +46,14 @@ def test_host_rejects_bad_arguments_without_launching():
     assert lib.sfa_prefill(*bad) == sfa.SFA_ERR_WORKSPACE
     bad = list(args); bad[0] = None
     assert lib.sfa_prefill(*bad) == sfa.SFA_ERR_INVALID_ARG
+    # beyond the call limits: 2 layers x 40000 sequences > 65535 streams, and
+    # n > 64 x (2^31 - 1) tokens; no workspace size, refused before any launch
+    for n, b in [(8, 40000), (1 << 40, 2)]:
+        assert lib.sfa_prefill_workspace_bytes(h, b, n) == 0
+        bad = list(args); bad[4] = n; bad[5] = b
+        assert lib.sfa_prefill(*bad) == sfa.SFA_ERR_UNSUPPORTED
+        assert lib.sfa_prefill_static_ws(h, *args[1:4], n, b, st, out.data_ptr(), s) == \
+            sfa.SFA_ERR_UNSUPPORTED
     assert lib.sfa_decode_step(h, q.data_ptr() + 2, k.data_ptr(), v.data_ptr(), 2, st,
                                out.data_ptr(), s) == sfa.SFA_ERR_ALIGNMENT
     torch.cuda.synchronize()
