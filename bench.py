@@ -70,6 +70,23 @@ def dist_env():
             int(os.environ.get("LOCAL_RANK", "0")))
 
 
+def max_over_ranks(values, world, device):
+    """Per-rank times (ms) reduced with MAX over the ranks, so the slowest
+    replica sets the job's time; every rank receives the result."""
+    import torch
+    t = torch.tensor([float(x) for x in values], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def job_rate(world, units_per_rank, ms):
+    """Whole-job throughput: the units all `world` replicas processed (each
+    the same amount) over the max-over-ranks time in ms."""
+    return world * units_per_rank / (ms / 1e3)
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -428,14 +445,11 @@ def main():
     rc = op.check()
     if rc != 0:
         raise SystemExit(f"device error in the timed region: {sfa.sfa_status_string(rc)}")
-    t = torch.tensor([sum(pre_ms) + sum(dec_ms), sum(pre_ms), sum(dec_ms)], dtype=torch.float64,
-                     device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms, pre_tot, dec_tot = (float(x) for x in t.tolist())
+    total_ms, pre_tot, dec_tot = max_over_ranks(
+        [sum(pre_ms) + sum(dec_ms), sum(pre_ms), sum(dec_ms)], world, dev)
     timed_pre = n_pre if has_a else 0
     tokens_per_step = B * (timed_pre + (n_dec if has_b else 0))
-    value = world * tokens_per_step * args.steps / (total_ms / 1e3)
+    value = job_rate(world, tokens_per_step * args.steps, total_ms)
     ms_per_step = total_ms / args.steps
 
     # ---- roofline of the dominant kernel
@@ -445,13 +459,13 @@ def main():
     if has_a:
         pre_ms_avg = pre_tot / args.steps
         pre_gbs = pre_bytes / (pre_ms_avg / 1e3) / 1e9
-        section["prefill"] = {"tokens_per_s": world * B * n_pre * args.steps / (pre_tot / 1e3),
+        section["prefill"] = {"tokens_per_s": job_rate(world, B * n_pre * args.steps, pre_tot),
                               "ms": pre_ms_avg, "algorithmic_bytes": pre_bytes,
                               "achieved_gbs": pre_gbs, "frac": pre_gbs / peak}
     if has_b:
         dec_launch_ms = dec_tot / (args.steps * n_dec)
         dec_gbs = dec_bytes / (dec_launch_ms / 1e3) / 1e9
-        section["decode"] = {"tokens_per_s": world * B * n_dec * args.steps / (dec_tot / 1e3),
+        section["decode"] = {"tokens_per_s": job_rate(world, B * n_dec * args.steps, dec_tot),
                              "us_per_step": 1e3 * dec_launch_ms, "algorithmic_bytes": dec_bytes,
                              "achieved_gbs": dec_gbs, "frac": dec_gbs / peak}
     dominant = "decode" if has_b and (not has_a or dec_tot >= pre_tot) else "prefill"
@@ -578,12 +592,8 @@ def measure_e2e(args, w, op, qp, kp, vp, qd, kd, vd, n_pre, n_dec, world, dev):
         dist.barrier()
     e0, e1 = run(steps)
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1)
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms = float(t.item())
-    value = world * B * (n_pre + n_dec) * steps / (ms / 1e3)
+    ms = max_over_ranks([e0.elapsed_time(e1)], world, dev)[0]
+    value = job_rate(world, B * (n_pre + n_dec) * steps, ms)
     return {"value": value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "steps": steps, "l2": "not flushed (host copies between steps)",
             "overlap": "copies on two streams overlap the neighbouring steps' compute"}
@@ -612,7 +622,7 @@ def measure_e2e_decode(args, w, op, qd, kd, vd, n_dec, world, dev):
             h_out[t].copy_(d_out, non_blocking=True)
 
     ms = _time_e2e(one, steps, world, dev)
-    value = world * B * n_dec * steps / (ms / 1e3)
+    value = job_rate(world, B * n_dec * steps, ms)
     return {"value": value, "unit": UNIT, "h2d_bytes_per_step": per * n_dec,
             "d2h_bytes_per_step": n_dec * L * B * H * 4, "steps": steps,
             "l2": "not flushed"}
@@ -632,11 +642,7 @@ def _time_e2e(one, steps, world, dev):
         one()
     e1.record()
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1)
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    return max_over_ranks([e0.elapsed_time(e1)], world, dev)[0]
 
 
 def cpu_baseline(w, n_pre):
