@@ -27,6 +27,21 @@
  *   - the vector fed to ring, field and pool is x = O_near + alpha_far * S;
  *   - each cosine norm is clamped below at 1e-12;
  *   - slots are fixed inputs and the pool mixes the raw slots.
+ *
+ * Pins (tests/test_oracle_pins.py; tests/test_oracle_mutations.py plants
+ * mistakes in copies of this file and checks that a pin catches each):
+ *   - near field: library softmax attention (full causal while n <= k, and
+ *     sliding-window), with GQA;
+ *   - far field: the evicted key when gamma_far = 0, and c(1 - gamma^m) for a
+ *     constant key stream;
+ *   - ring mean, field and fusion: closed forms on a constant value stream;
+ *   - pool: basis-vector slots (closed-form softmax), equal slots, zero x, and
+ *     generic inputs against library attention with normalised query and keys;
+ *   - the whole path against an unrolled formulation (sums over the history
+ *     in place of every recurrence) on generic inputs;
+ *   - alpha_layer: hand-worked values and both endpoints;
+ *   - the printed constants and the calibration table (tests/golden/).
+ * No function here is left "parity unpinned".
  */
 #include "sfa_oracle.h"
 
