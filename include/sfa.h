@@ -169,11 +169,11 @@ SFA_API int sfa_prefill(const sfa_handle* h, const void* q, const void* k, const
 
 /* Folds one token per sequence into the state and writes its output.
  * One kernel launch covers all layers and sequences; no workspace.
- * The kernel may start, and read q, k and v, while the previous SFA call on
- * the same stream is still running (programmatic dependent launch; the
- * state is read only after that call has finished).  So q, k and v must not
- * be memory that an earlier SFA call on the stream writes (its out or
- * state); inputs written by any other kernel are safe. */
+ * The kernel may start while the previous kernel on the stream is still
+ * running (programmatic dependent launch): it fetches the handle's
+ * constants at once, and the state, q, k and v only once that kernel has
+ * finished, so inputs produced by the kernel just before are safe.  See
+ * sfa_set_decode_input_prefetch for fetching q, k and v earlier. */
 SFA_API int sfa_decode_step(const sfa_handle* h, const void* q, const void* k, const void* v,
                     int batch, void* state, float* out, void* stream);
 
@@ -207,11 +207,25 @@ SFA_API int sfa_prefill_layers(const sfa_handle* h, int layer_begin, int layer_c
  * [layer_count][n_seq][n_kv][d], out [layer_count][n_seq][hidden] fp32.
  * Sequences not listed keep their state and position.  An index out of range
  * is skipped on the device and latched as SFA_ERR_INVALID_ARG for
- * sfa_check_device_status; host-visible errors, and the condition on q, k
- * and v, as for sfa_decode_step. */
+ * sfa_check_device_status; host-visible errors, and the input prefetch
+ * option, as for sfa_decode_step. */
 SFA_API int sfa_decode_step_ex(const sfa_handle* h, int layer_begin, int layer_count,
                                const int* seq_ids, int n_seq, const void* q, const void* k,
                                const void* v, int batch, void* state, float* out, void* stream);
+
+/* Decode input prefetch (default off).  enable = 1 declares that, for every
+ * later decode call on this handle, q, k and v are complete when the call is
+ * enqueued and nothing that may still be running on the stream writes them:
+ * for example inputs written before a synchronisation, copied in by
+ * cudaMemcpyAsync, or written by a kernel on another stream that the call's
+ * stream waits for through an event.  The per-sequence decode kernel then
+ * fetches them before the previous kernel on the stream has finished, which
+ * takes one memory round trip off each call.  With enable = 1, inputs
+ * written by a kernel still running on the stream (a projection launched
+ * just before the call, or an earlier SFA call's out) may be read before
+ * they are written.  enable = 0 restores the default.  SFA_ERR_INVALID_ARG
+ * for another value.  Results are identical either way. */
+SFA_API int sfa_set_decode_input_prefetch(sfa_handle* h, int enable);
 
 /* Synchronises `stream`, then returns and clears the first error latched on
  * the device since the last check (SFA_OK if none), or SFA_ERR_CUDA if the

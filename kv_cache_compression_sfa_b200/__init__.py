@@ -45,6 +45,7 @@ EXPORTED = (
     "sfa_prefill", "sfa_decode_step", "sfa_check_device_status", "sfa_status_string",
     "sfa_abi_version", "sfa_debug_set_lookback", "sfa_prefill_static_ws",
     "sfa_prefill_layers_workspace_bytes", "sfa_prefill_layers", "sfa_decode_step_ex",
+    "sfa_set_decode_input_prefetch",
 )
 
 
@@ -109,6 +110,7 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
             "sfa_prefill_layers_workspace_bytes": (sz, [vp, i, i, ll]),
             "sfa_prefill_layers": (i, [vp, i, i, vp, vp, vp, ll, i, vp, vp, vp, sz, vp]),
             "sfa_decode_step_ex": (i, [vp, i, i, vp, i, vp, vp, vp, i, vp, vp, vp]),
+            "sfa_set_decode_input_prefetch": (i, [vp, i]),
         }
         for name, (res, args) in sigs.items():
             fn = getattr(lib, name)
@@ -340,16 +342,26 @@ def sfa_prefill_static_ws(h: Handle, q, k, v, n: int, batch: int, state: torch.T
 
 def sfa_decode_step(h: Handle, q, k, v, batch: int, state: torch.Tensor, out: torch.Tensor,
                     stream=None) -> None:
-    """One token per sequence, all layers.  The kernel may read q, k and v
-    before the previous SFA call on the stream has finished, so they must not
-    be memory that an earlier SFA call writes (its out or state); inputs
-    written by any other kernel are safe."""
+    """One token per sequence, all layers.  q, k and v are read once the
+    previous kernel on the stream has finished, unless the handle's input
+    prefetch is on (sfa_set_decode_input_prefetch)."""
     qp, kp, vp = _qkv_checks(h, q, k, v, 1, batch)
     sp = _dev(state, "state", torch.uint8, sfa_state_bytes(h, batch))
     op = _dev(out, "out", torch.float32, h.cfg.n_layers * batch * h.cfg.hidden)
     rc = load_library().sfa_decode_step(h.ptr, qp, kp, vp, batch, sp, op, _stream_ptr(stream))
     if rc != SFA_OK:
         raise SfaError(rc, "sfa_decode_step")
+
+
+def sfa_set_decode_input_prefetch(h: Handle, enable: bool) -> None:
+    """Declare (True) that every later decode call's q, k and v are complete
+    when the call is enqueued and that nothing still running on the stream
+    writes them; the decode kernel then fetches them before the previous
+    kernel on the stream has finished.  False (the default) fetches them
+    after it.  Results are identical either way."""
+    rc = load_library().sfa_set_decode_input_prefetch(h.ptr, 1 if enable else 0)
+    if rc != SFA_OK:
+        raise SfaError(rc, "sfa_set_decode_input_prefetch")
 
 
 def sfa_check_device_status(h: Handle, stream=None) -> int:

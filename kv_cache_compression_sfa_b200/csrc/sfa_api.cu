@@ -43,6 +43,7 @@ struct sfa_handle {
   bool tile_ok;          // the batch-tiled decode fits this configuration
   int tile_smem;         // its dynamic shared memory per CTA
   int tile_mode;         // -1: by batch size; 0: never; 1: always (test hook)
+  bool inputs_early;     // decode inputs declared complete before each call
 };
 
 namespace {
@@ -259,6 +260,7 @@ int sfa_init(const sfa_config* cfg, sfa_handle** out) {
   h->cs = 0;
   h->spin_limit = kDefaultSpinLimit;
   h->withhold_tile = -1;
+  h->inputs_early = false;
   {
     // Test hook (environment, read once per handle): SFA_DECODE_TILE=0 / 1
     // turns the batch-tiled decode off / on for every batch size (default:
@@ -517,6 +519,7 @@ int sfa_decode_step_ex(const sfa_handle* h, int layer_begin, int layer_count, co
   p.NGm = max_kv_heads_per_cta(c->n_q_heads, c->n_kv_heads, p.CS);
   p.smem_budget = h->decode_budget;
   p.tile_smem = h->tile_smem;
+  p.inputs_early = h->inputs_early ? 1 : 0;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // Batch-tiled decode from kDecodeTileMinSeqs sequences with windows of at
   // most kDecodeTileMaxWindow positions (longer windows: each warp walks its
@@ -558,6 +561,12 @@ const char* sfa_status_string(int status) {
 }
 
 int sfa_abi_version(void) { return SFA_ABI_VERSION; }
+
+int sfa_set_decode_input_prefetch(sfa_handle* h, int enable) {
+  if (!handle_ok(h) || (enable != 0 && enable != 1)) return SFA_ERR_INVALID_ARG;
+  h->inputs_early = enable == 1;
+  return SFA_OK;
+}
 
 int sfa_debug_set_lookback(sfa_handle* h, unsigned int spin_limit, long long withhold_tile) {
   if (!handle_ok(h)) return SFA_ERR_INVALID_ARG;

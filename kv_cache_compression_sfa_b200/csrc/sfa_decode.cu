@@ -194,23 +194,29 @@ decode_kernel(const DecodeParams p) {
   const float inrm0 = 1.f / nrm[lane], inrm1 = 1.f / nrm[lane + 32];
   const float a_l = p.alpha_layer[l];
 
-  // This call's query slice and K_t, V_t of the CTA's KV heads.  No earlier
-  // SFA call on the stream writes them (a condition of the C ABI), so they
-  // are fetched before the wait below; decode inputs usually come from HBM,
-  // and this takes that latency off the critical path.
+  // This call's query slice and K_t, V_t of the CTA's KV heads.  A kernel
+  // still running on the stream may be writing them, so by default they are
+  // fetched after the wait below.  When the caller has declared them
+  // complete before the call (sfa_set_decode_input_prefetch), they are
+  // fetched before it: decode inputs usually come from HBM, and that takes
+  // their latency off the critical path.
   const long long io = static_cast<long long>(li) * p.n_seq + bi;  // input / output row
   const Tin* qin = static_cast<const Tin*>(p.q) + (io * p.nq + h0) * D;
   const Tin* kin = static_cast<const Tin*>(p.k) + io * nkv * D;
   const Tin* vin = static_cast<const Tin*>(p.v) + io * nkv * D;
-  if (tid == 32) {
-    const unsigned hb = static_cast<unsigned>(NG * D * ESZ);
-    mbar_arrive_expect_tx(bar_q, static_cast<unsigned>(HS * ESZ) + 2u * hb);
-    bulk_g2s(qraw, qin, static_cast<unsigned>(HS * ESZ), bar_q);
-    bulk_g2s(kc, kin + g_lo * D, hb, bar_q);
-    bulk_g2s(vc, vin + g_lo * D, hb, bar_q);
-  }
+  auto fetch_inputs = [&]() {
+    if (tid == 32) {
+      const unsigned hb = static_cast<unsigned>(NG * D * ESZ);
+      mbar_arrive_expect_tx(bar_q, static_cast<unsigned>(HS * ESZ) + 2u * hb);
+      bulk_g2s(qraw, qin, static_cast<unsigned>(HS * ESZ), bar_q);
+      bulk_g2s(kc, kin + g_lo * D, hb, bar_q);
+      bulk_g2s(vc, vin + g_lo * D, hb, bar_q);
+    }
+  };
+  if (p.inputs_early) fetch_inputs();
 
-  pdl_wait();  // the state may be written by the previous kernel
+  pdl_wait();  // the state (and, by default, the inputs) may be written by the previous kernel
+  if (!p.inputs_early) fetch_inputs();
 
   // Sequence served: from the caller's list, checked against the batch (an
   // index out of range leaves the cluster without touching the state).

@@ -75,6 +75,7 @@ struct DecodeParams {
   int NGm;          // most KV heads any CTA needs
   int smem_budget;  // shared-memory bytes the plan may use (window staged if it fits)
   int tile_smem;    // dynamic shared memory of the batch-tiled decode
+  int inputs_early; // q, K_t, V_t may be fetched before the wait for the previous kernel
   float gamma_far, alpha_far, ema_gamma, inv_temp, clip_eps, score_scale;
 };
 

@@ -5,7 +5,8 @@
   * n = 0 is a no-op;
   * sequences are independent: permuting the batch permutes the outputs
     bit for bit;
-  * a state copied out and restored resumes exactly (checkpoint/resume).
+  * a state copied out and restored resumes exactly (checkpoint/resume);
+  * the decode input-prefetch option does not change any bit.
 """
 import numpy as np
 import pytest
@@ -49,6 +50,26 @@ def test_prefill_equals_decode_steps():
         assert torch.equal(sa[key], sb[key]), key
     for key in ("far", "field", "ring", "ring_sum"):
         assert _rel(sa[key], sb[key]) < 2e-5, key
+
+
+def test_decode_input_prefetch_gives_identical_results():
+    """The input-prefetch option only moves the point where the decode kernel
+    fetches q, k and v (before or after the previous kernel on the stream
+    ends); outputs and state are bit-identical with and without it."""
+    w = _w()
+    slots = make_slots(w, "cuda")
+    q, k, v = TokenSource(w, "cuda").get(0, 40)
+    steps = [tuple(x[:, :, t].contiguous() for x in (q, k, v)) for t in range(40)]
+    torch.cuda.synchronize()  # every input is complete before the calls
+    runs = []
+    for prefetch in (False, True):
+        op = _op(w, slots)
+        sfa.sfa_set_decode_input_prefetch(op.handle, prefetch)
+        outs = [op.decode(*s) for s in steps]
+        assert op.check() == 0
+        runs.append((torch.stack(outs), op.state.clone()))
+    assert torch.equal(runs[0][0], runs[1][0])
+    assert torch.equal(runs[0][1], runs[1][1])
 
 
 @pytest.mark.parametrize("cuts", [[64], [1, 63], [15, 16, 17], [100, 7, 43]])
