@@ -37,8 +37,9 @@
  *   - One state buffer serves `batch` sequences for all layers.  A state is
  *     used by one stream at a time; stream order serialises calls.  The
  *     compute calls never modify the handle, so it may be shared across
- *     streams and host threads (only sfa_debug_set_lookback and
- *     sfa_destroy modify it).
+ *     streams and host threads (only sfa_set_decode_input_prefetch,
+ *     sfa_debug_set_lookback and sfa_destroy modify it: call those while no
+ *     other host thread uses the handle).
  */
 #ifndef SFA_H
 #define SFA_H

@@ -39,6 +39,26 @@ def test_library_exports_every_declared_symbol(lib):
     assert exported == _declared()
 
 
+def test_plain_c_client_compiles_links_and_runs(lib, tmp_path):
+    """The header is plain C99 and the library is enough to link against: a C
+    program that includes only sfa.h builds with gcc -std=c99 -Wall -Wextra
+    -Werror, links libsfa.so and runs the host-only calls without a GPU."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc not found")
+    exe = str(tmp_path / "c_abi_client")
+    libdir = os.path.dirname(sfa.LIB_PATH)
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic",
+                    "-I", os.path.join(ROOT, "include"),
+                    os.path.join(ROOT, "tests", "c_abi_client.c"), "-o", exe,
+                    "-L", libdir, "-lsfa", f"-Wl,-rpath,{libdir}"], check=True)
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0, r.stderr
+    assert r.stdout.strip() == "ok"
+
+
 def test_abi_version(lib):
     assert sfa.sfa_abi_version() == 1
 
