@@ -22,10 +22,10 @@
 // bandwidth.  Every operand a CTA needs is brought into shared memory by the
 // bulk-copy engine in a few large copies: before the kernel waits on its
 // predecessor (programmatic dependent launch), the slot slice (constant;
-// stored per CTA with padded rows at init) and this call's q, K_t and V_t
-// (which no earlier SFA call on the stream writes); right after, S, field,
-// ring sum and the window (all KV heads of every slot in one copy each for
-// K and V where it fits).  Only the ring slot t mod 16 depends on the
+// stored per CTA with padded rows at init), and this call's q, K_t and V_t
+// too when the caller has declared them complete before the call; right
+// after, the inputs otherwise, then S, field, ring sum and the window (all
+// KV heads of every slot in one copy each for K and V where it fits).  Only the ring slot t mod 16 depends on the
 // position and follows one round trip later, overlapped with the near field.
 // All arithmetic then runs from shared memory.  A window too large for the
 // shared-memory budget is read from global memory instead.
