@@ -292,6 +292,32 @@ def test_whole_path_matches_unrolled_definition(nq, nkv, d, K, gf):
             np.testing.assert_allclose(out[l, b], ref, rtol=1e-9, atol=1e-11)
 
 
+try:
+    from hypothesis import HealthCheck, given, settings, strategies as st
+except ImportError:  # pragma: no cover
+    given = None
+
+if given is not None:
+    @settings(max_examples=30, deadline=None, derandomize=True,
+              suppress_health_check=[HealthCheck.too_slow])
+    @given(grp=st.sampled_from([(1, 1), (2, 1), (2, 2), (4, 2), (3, 1)]),
+           d=st.sampled_from([2, 4, 8]), K=st.integers(1, 6), n=st.integers(1, 21),
+           gf=st.floats(0.0, 0.99), af=st.floats(0.0, 1.0), ab=st.floats(0.0, 3.0),
+           eps=st.floats(0.05, 2.0), seed=st.integers(0, 2**16))
+    def test_whole_path_matches_unrolled_definition_on_random_shapes(grp, d, K, n, gf, af, ab,
+                                                                     eps, seed):
+        """The unrolled pin above, drawn over small shapes, GQA groupings,
+        windows longer and shorter than the sequence, and the scalar ranges."""
+        nq, nkv = grp
+        f32 = lambda x: float(np.float32(x))
+        gf, af, ab, eps = f32(gf), f32(af), f32(ab), f32(eps)
+        q, k, v, slots = _inputs(seed, 1, 1, n, nq, nkv, d)
+        p = OracleParams(nq, nkv, d, K, gamma_far=gf, alpha_far=af, clip_eps=eps)
+        out = _run(p, ab, 0.9, slots, q, k, v)[0, 0]
+        ref = _unrolled_reference(q[0, 0], k[0, 0], v[0, 0], slots[0], p, 0.3 * ab)
+        np.testing.assert_allclose(out, ref, rtol=1e-9, atol=1e-11)
+
+
 # ------------------------------------------------------------- alpha_layer
 
 def test_alpha_layer_endpoints_and_worked_values():
