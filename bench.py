@@ -87,6 +87,14 @@ def job_rate(world, units_per_rank, ms):
     return world * units_per_rank / (ms / 1e3)
 
 
+def step_medians(pre_ms, dec_ms):
+    """Median over the timed steps of this rank's per-step times (ms): the
+    whole step, its prefill part and its decode part."""
+    tot = [a + b for a, b in zip(pre_ms, dec_ms)]
+    return {"step_ms": statistics.median(tot), "prefill_ms": statistics.median(pre_ms),
+            "decode_ms": statistics.median(dec_ms), "steps": len(tot)}
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -447,6 +455,7 @@ def main():
     clocks = sampler.stop() if sampler else None
     pre_ms = [e[0].elapsed_time(e[1]) for e in ev]
     dec_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    medians = step_medians(pre_ms, dec_ms)
     rc = op.check()
     if rc != 0:
         raise SystemExit(f"device error in the timed region: {sfa.sfa_status_string(rc)}")
@@ -504,7 +513,8 @@ def main():
     launches_per_step = (1 + 5 if has_a else 0) + (n_dec if has_b else 0)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "median": medians,
+        "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {**workload_config(w, n_pre),
                    "decode_inputs": "prefetched: complete before each call "

@@ -99,3 +99,11 @@ def test_enhancement_stats_closed_forms():
     assert st["abs_cos_p90"] < 1e-12
     share = np.linalg.norm(e, axis=1) / np.linalg.norm(x + e, axis=1)
     assert abs(st["share_median"] - np.median(share)) < 1e-12
+
+
+def test_step_medians():
+    m = bench.step_medians([1.0, 3.0, 2.0], [10.0, 30.0, 20.0])
+    assert m == {"step_ms": 22.0, "prefill_ms": 2.0, "decode_ms": 20.0, "steps": 3}
+    # medians are per part, so they need not add up to the step median
+    m = bench.step_medians([1.0, 9.0, 2.0, 8.0], [9.0, 1.0, 8.0, 2.0])
+    assert m["step_ms"] == 10.0 and m["prefill_ms"] == 5.0 and m["decode_ms"] == 5.0
