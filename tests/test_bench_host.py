@@ -107,3 +107,122 @@ def test_step_medians():
     # medians are per part, so they need not add up to the step median
     m = bench.step_medians([1.0, 9.0, 2.0, 8.0], [9.0, 1.0, 8.0, 2.0])
     assert m["step_ms"] == 10.0 and m["prefill_ms"] == 5.0 and m["decode_ms"] == 5.0
+
+
+class _FakeEvent:
+    def __init__(self, enable_timing=False):
+        pass
+
+    def record(self, stream=None):
+        pass
+
+    def elapsed_time(self, other):
+        return 2.0
+
+
+class _FakeStream:
+    def __init__(self, device=None):
+        pass
+
+    def wait_event(self, e):
+        pass
+
+    def wait_stream(self, s):
+        pass
+
+
+class _RecordingOp:
+    """Stands in for SfaOperator: records what every call received."""
+
+    def __init__(self):
+        self.calls = []
+
+    def reset(self, stream=None):
+        self.calls.append(("reset",))
+
+    def prefill(self, q, k, v, out=None, stream=None):
+        self.calls.append(("prefill", q.clone(), k.clone(), v.clone(), out))
+        out.fill_(1.0)
+        return out
+
+    def decode(self, q, k, v, out=None, stream=None):
+        self.calls.append(("decode", q.clone(), k.clone(), v.clone(), out))
+        out.fill_(2.0)
+        return out
+
+
+def _fake_cuda(monkeypatch):
+    import contextlib
+    import torch
+    monkeypatch.setattr(torch.cuda, "Event", _FakeEvent)
+    monkeypatch.setattr(torch.cuda, "Stream", _FakeStream)
+    monkeypatch.setattr(torch.cuda, "current_stream", lambda device=None: _FakeStream())
+    monkeypatch.setattr(torch.cuda, "stream", lambda s: contextlib.nullcontext())
+    monkeypatch.setattr(torch.cuda, "synchronize", lambda device=None: None)
+    monkeypatch.setattr(torch.Tensor, "pin_memory", lambda self: self)
+
+
+@pytest.mark.parametrize("n_dec", [0, 3])
+def test_e2e_step_loop_feeds_every_call_its_own_inputs(monkeypatch, n_dec):
+    """measure_e2e on CPU with fake streams and events: each step resets,
+    prefills with that step's inputs and runs every decode call on its own
+    token's q/k/v and output slice, alternating the two buffer sets."""
+    import types
+    import torch
+    _fake_cuda(monkeypatch)
+    w = types.SimpleNamespace(n_layers=2, batch=1, hidden=8)
+    g = torch.Generator().manual_seed(0)
+    mk = lambda *s: torch.randn(*s, generator=g).to(torch.bfloat16)
+    n_pre = 5
+    qp, kp, vp = mk(2, 1, n_pre, 2, 4), mk(2, 1, n_pre, 1, 4), mk(2, 1, n_pre, 1, 4)
+    qd = [mk(2, 1, 2, 4) for _ in range(n_dec)]
+    kd = [mk(2, 1, 1, 4) for _ in range(n_dec)]
+    vd = [mk(2, 1, 1, 4) for _ in range(n_dec)]
+    op = _RecordingOp()
+    args = types.SimpleNamespace(steps=4)
+    e2e = bench.measure_e2e(args, w, op, qp, kp, vp, qd, kd, vd, n_pre, n_dec, 1, "cpu")
+    steps = 3 + max(3, min(args.steps, 200))  # untimed run(3), then the timed run
+    per_step = 2 + n_dec
+    assert len(op.calls) == steps * per_step
+    outs = set()
+    for s in range(steps):
+        c = op.calls[s * per_step:(s + 1) * per_step]
+        assert c[0] == ("reset",)
+        assert c[1][0] == "prefill" and all(torch.equal(a, b) for a, b in zip(c[1][1:4], (qp, kp, vp)))
+        for t in range(n_dec):
+            name, q, k, v, out = c[2 + t]
+            assert name == "decode"
+            assert torch.equal(q, qd[t]) and torch.equal(k, kd[t]) and torch.equal(v, vd[t])
+            assert out.shape == (2, 1, 8) and out.is_contiguous()
+            outs.add(out.data_ptr())
+    assert len(outs) == 2 * n_dec  # one output slice per token and buffer set
+    dec_elems = sum(x.numel() for x in qd + kd + vd)
+    assert e2e["h2d_bytes_per_step"] == 2 * (qp.numel() + kp.numel() + vp.numel() + dec_elems)
+    assert e2e["d2h_bytes_per_step"] == 4 * 2 * 8 * (n_pre + n_dec)
+    assert e2e["value"] == pytest.approx(1 * (n_pre + n_dec) * 4 / 2e-3)
+
+
+def test_e2e_decode_only_loop_copies_each_token(monkeypatch):
+    """measure_e2e_decode on CPU with fake streams and events: every call
+    copies in its token's inputs (cycling the input ring) and decodes them."""
+    import types
+    import torch
+    _fake_cuda(monkeypatch)
+    w = types.SimpleNamespace(n_layers=2, batch=3, hidden=8)
+    g = torch.Generator().manual_seed(1)
+    mk = lambda *s: torch.randn(*s, generator=g).to(torch.bfloat16)
+    n_ring, n_dec = 2, 5
+    qd = [mk(2, 3, 2, 4) for _ in range(n_ring)]
+    kd = [mk(2, 3, 1, 4) for _ in range(n_ring)]
+    vd = [mk(2, 3, 1, 4) for _ in range(n_ring)]
+    op = _RecordingOp()
+    args = types.SimpleNamespace(steps=3)
+    e2e = bench.measure_e2e_decode(args, w, op, qd, kd, vd, n_dec, 1, "cpu")
+    runs = 3 + 3  # three untimed, then max(3, min(steps, 5)) timed
+    assert len(op.calls) == runs * n_dec
+    for i, c in enumerate(op.calls):
+        r = (i % n_dec) % n_ring
+        assert c[0] == "decode" and torch.equal(c[1], qd[r]) and torch.equal(c[3], vd[r])
+    assert e2e["h2d_bytes_per_step"] == n_dec * 2 * (qd[0].numel() + kd[0].numel() + vd[0].numel())
+    assert e2e["d2h_bytes_per_step"] == n_dec * 2 * 3 * 8 * 4
+    assert e2e["value"] == pytest.approx(3 * n_dec * 3 / 2e-3)
