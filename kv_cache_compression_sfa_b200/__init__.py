@@ -195,8 +195,12 @@ def _stream_ptr(stream) -> int:
     return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
 
 
+def _is_cuda_tensor(t) -> bool:
+    return isinstance(t, torch.Tensor) and t.is_cuda
+
+
 def _dev(t: torch.Tensor, name: str, dtype=None, min_numel: int = 0) -> int:
-    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+    if not _is_cuda_tensor(t):
         raise ValueError(f"{name} must be a CUDA tensor")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
@@ -391,8 +395,15 @@ class SfaOperator:
         self.batch = batch
         self.device = torch.device(device or slots.device)
         self.handle = sfa_init(cfg, slots)
-        self.state = torch.empty(sfa_state_bytes(self.handle, batch), dtype=torch.uint8,
-                                 device=self.device)
+        self._state_bytes = sfa_state_bytes(self.handle, batch)
+        self.state = torch.empty(self._state_bytes, dtype=torch.uint8, device=self.device)
+        # Per-call constants of decode(), which a serving loop calls once per
+        # token: the C entry point, the element counts and the input dtype.
+        rows = cfg.n_layers * batch
+        self._dec_numel = (rows * cfg.n_q_heads * cfg.head_dim, rows * cfg.n_kv_heads * cfg.head_dim,
+                           rows * cfg.hidden)
+        self._in_dtype = cfg.torch_dtype
+        self._decode_fn = load_library().sfa_decode_step
         self.workspace = None
         if max_prefill > 0:
             self._ensure_workspace(max_prefill)
@@ -419,11 +430,20 @@ class SfaOperator:
         return out
 
     def decode(self, q, k, v, out: Optional[torch.Tensor] = None, stream=None):
-        c = self.cfg
+        """One token per sequence, all layers: the checks and the call of
+        sfa_decode_step, with the per-operator constants looked up once."""
         if out is None:
+            c = self.cfg
             out = torch.empty((c.n_layers, self.batch, c.hidden), dtype=torch.float32,
                               device=self.device)
-        sfa_decode_step(self.handle, q, k, v, self.batch, self.state, out, stream)
+        nq, nkv, nout = self._dec_numel
+        dt = self._in_dtype
+        rc = self._decode_fn(self.handle.ptr, _dev(q, "q", dt, nq), _dev(k, "k", dt, nkv),
+                             _dev(v, "v", dt, nkv),
+                             self.batch, _dev(self.state, "state", torch.uint8, self._state_bytes),
+                             _dev(out, "out", torch.float32, nout), _stream_ptr(stream))
+        if rc != SFA_OK:
+            raise SfaError(rc, "sfa_decode_step")
         return out
 
     def prefill_layers(self, layer_begin: int, q, k, v, out: Optional[torch.Tensor] = None,
