@@ -614,9 +614,16 @@ def measure_e2e(args, w, op, qp, kp, vp, qd, kd, vd, n_pre, n_dec, world, dev):
     e0, e1 = run(steps)
     torch.cuda.synchronize()
     ms = max_over_ranks([e0.elapsed_time(e1)], world, dev)[0]
+    # Host time to issue one step into empty queues (outside the timed run):
+    # when it is close to the step time, the e2e figure is bound by the host.
+    h0 = time.perf_counter()
+    run(1)
+    host_ms = 1e3 * (time.perf_counter() - h0)
+    torch.cuda.synchronize()
     value = job_rate(world, B * (n_pre + n_dec) * steps, ms)
     return {"value": value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "steps": steps, "l2": "not flushed (host copies between steps)",
+            "steps": steps, "ms_per_step": ms / steps, "host_issue_ms_per_step": host_ms,
+            "l2": "not flushed (host copies between steps)",
             "overlap": "copies on two streams overlap the neighbouring steps' compute"}
 
 

@@ -181,7 +181,7 @@ def test_e2e_step_loop_feeds_every_call_its_own_inputs(monkeypatch, n_dec):
     op = _RecordingOp()
     args = types.SimpleNamespace(steps=4)
     e2e = bench.measure_e2e(args, w, op, qp, kp, vp, qd, kd, vd, n_pre, n_dec, 1, "cpu")
-    steps = 3 + max(3, min(args.steps, 200))  # untimed run(3), then the timed run
+    steps = 3 + max(3, min(args.steps, 200)) + 1  # run(3), the timed run, the host-cost run(1)
     per_step = 2 + n_dec
     assert len(op.calls) == steps * per_step
     outs = set()
@@ -200,6 +200,7 @@ def test_e2e_step_loop_feeds_every_call_its_own_inputs(monkeypatch, n_dec):
     assert e2e["h2d_bytes_per_step"] == 2 * (qp.numel() + kp.numel() + vp.numel() + dec_elems)
     assert e2e["d2h_bytes_per_step"] == 4 * 2 * 8 * (n_pre + n_dec)
     assert e2e["value"] == pytest.approx(1 * (n_pre + n_dec) * 4 / 2e-3)
+    assert e2e["ms_per_step"] == pytest.approx(2.0 / 4) and e2e["host_issue_ms_per_step"] > 0
 
 
 def test_e2e_decode_only_loop_copies_each_token(monkeypatch):
