@@ -28,6 +28,7 @@ operator has no cross-stream exchange), timed per rank and reduced with MAX.
 from __future__ import annotations
 
 import argparse
+import contextlib
 import hashlib
 import json
 import os
@@ -68,6 +69,27 @@ def parse():
 def dist_env():
     return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
             int(os.environ.get("LOCAL_RANK", "0")))
+
+
+@contextlib.contextmanager
+def nvtx_range(name: str):
+    """NVTX range around a phase of the bench, for Nsight timelines; a no-op
+    where NVTX is unavailable."""
+    pushed = False
+    try:
+        import torch
+        torch.cuda.nvtx.range_push(name)
+        pushed = True
+    except Exception:
+        pass
+    try:
+        yield
+    finally:
+        if pushed:
+            try:
+                torch.cuda.nvtx.range_pop()
+            except Exception:
+                pass
 
 
 def max_over_ranks(values, world, device):
@@ -433,9 +455,10 @@ def main():
         if ev:
             ev[2].record()
 
-    for _ in range(args.warmup):
-        one_step()
-    torch.cuda.synchronize()
+    with nvtx_range("sfa warm-up"):
+        for _ in range(args.warmup):
+            one_step()
+        torch.cuda.synchronize()
     if op.check() != 0:
         raise SystemExit("device error during warm-up")
 
@@ -447,9 +470,10 @@ def main():
     if sampler:
         sampler.start()
         time.sleep(0.1)
-    for s in range(args.steps):
-        one_step(ev[s])
-    torch.cuda.synchronize()
+    with nvtx_range("sfa timed steps"):
+        for s in range(args.steps):
+            one_step(ev[s])
+        torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     clocks = sampler.stop() if sampler else None
@@ -493,10 +517,11 @@ def main():
     # ---- e2e through the public API with host buffers
     e2e = None
     if not args.no_e2e:
-        if kind == "decode":
-            e2e = measure_e2e_decode(args, w, op, qd, kd, vd, n_dec, world, dev)
-        else:
-            e2e = measure_e2e(args, w, op, qp, kp, vp, qd, kd, vd, n_pre, n_dec, world, dev)
+        with nvtx_range("sfa e2e"):
+            if kind == "decode":
+                e2e = measure_e2e_decode(args, w, op, qd, kd, vd, n_dec, world, dev)
+            else:
+                e2e = measure_e2e(args, w, op, qp, kp, vp, qd, kd, vd, n_pre, n_dec, world, dev)
 
     # ---- oracle on the host cores (rank 0, N = 1 only)
     cpu = None

@@ -227,3 +227,11 @@ def test_e2e_decode_only_loop_copies_each_token(monkeypatch):
     assert e2e["h2d_bytes_per_step"] == n_dec * 2 * (qd[0].numel() + kd[0].numel() + vd[0].numel())
     assert e2e["d2h_bytes_per_step"] == n_dec * 2 * 3 * 8 * 4
     assert e2e["value"] == pytest.approx(3 * n_dec * 3 / 2e-3)
+
+
+def test_nvtx_range_wraps_and_reraises():
+    with bench.nvtx_range("test range"):
+        pass
+    with pytest.raises(KeyError):
+        with bench.nvtx_range("test range"):
+            raise KeyError("inside")
