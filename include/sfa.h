@@ -79,7 +79,7 @@ typedef struct sfa_config {
   int n_kv_heads;      /* KV heads, divides n_q_heads (GQA)                  */
   int head_dim;        /* 64 or 128                                          */
   int window_k;        /* near window k, 1..256            [P1 §2.1, §2.2]   */
-  float gamma_far;     /* far-field EWMA decay, [0, 1)     [P1 eq. S_t]      */
+  float gamma_far;     /* far-field EWMA decay, [0, 1]     [P1 eq. S_t]      */
   float alpha_far;     /* far-field mixing coefficient     [P1 eq. O]        */
   int ring_size;       /* must be 16                       [P3 §2.1 ch. 1]   */
   float ema_gamma;     /* EMA field decay (0.98)           [P3 §2.1 ch. 2]   */
@@ -122,8 +122,10 @@ SFA_API void sfa_config_default(sfa_config* cfg);
 /* Validates a configuration without touching the GPU: SFA_OK,
  * SFA_ERR_INVALID_ARG (null, non-positive sizes, non-finite or out-of-range
  * scalars, n_q % n_kv != 0) or SFA_ERR_UNSUPPORTED (head_dim not 64/128,
- * window_k > 256, ring_size != 16, n_slots != 64, hidden > 8192).  The slots
- * pointer is checked for NULL and alignment only. */
+ * window_k > 256, ring_size != 16, n_slots != 64, hidden > 8192, or no
+ * divisor cs <= 16 of n_q_heads with (n_q_heads / cs) * head_dim <= 512:
+ * the decode kernel splits the hidden vector over a cluster of cs CTAs).
+ * The slots pointer is checked for NULL and alignment only. */
 SFA_API int sfa_config_validate(const sfa_config* cfg);
 
 /* State layout for `batch` sequences of `cfg` (host arithmetic, no CUDA). */

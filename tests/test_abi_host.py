@@ -109,6 +109,9 @@ def _cfg(**kw):
     ({"clip_eps": -1.0}, sfa.SFA_ERR_INVALID_ARG),
     ({"in_dtype": 7}, sfa.SFA_ERR_INVALID_ARG),
     ({"n_q_heads": 128, "n_kv_heads": 8, "head_dim": 128}, sfa.SFA_ERR_UNSUPPORTED),
+    ({"n_q_heads": 17, "n_kv_heads": 1}, sfa.SFA_ERR_UNSUPPORTED),   # no cluster split of 17 heads
+    ({"gamma_far": 1.0}, sfa.SFA_OK),                                # S stays as it is
+    ({"gamma_far": -0.1}, sfa.SFA_ERR_INVALID_ARG),
 ])
 def test_config_validate_codes(lib, kw, code):
     assert sfa.sfa_config_validate(_cfg(**kw).to_c(256)) == code
