@@ -164,8 +164,12 @@ SFA_API int sfa_state_reset(const sfa_handle* h, void* state, int batch, void* s
  * 64 x (2^31 - 1), or layers x batch x n exceeds 2^31 - 1 with bf16 inputs
  * and k <= 16 (the tensor copies use 32-bit row coordinates; split the
  * call).
- * workspace: sfa_prefill_workspace_bytes(h, batch, n) bytes (may be NULL if
- * that is 0); workspace_bytes is its size, checked. */
+ * workspace: sfa_prefill_workspace_bytes(h, batch, n) bytes (may be NULL
+ * when n == 0); workspace_bytes is its size, checked.
+ * Before any launch: SFA_ERR_INVALID_ARG (bad handle, n < 0, batch <= 0, a
+ * NULL tensor), SFA_ERR_ALIGNMENT, SFA_ERR_WORKSPACE, SFA_ERR_UNSUPPORTED.
+ * A state whose header does not match the handle or batch is left untouched
+ * and latched as SFA_ERR_STATE_MISMATCH for sfa_check_device_status. */
 SFA_API int sfa_prefill(const sfa_handle* h, const void* q, const void* k, const void* v,
                 long long n, int batch, void* state, float* out, void* workspace,
                 size_t workspace_bytes, void* stream);
@@ -176,15 +180,20 @@ SFA_API int sfa_prefill(const sfa_handle* h, const void* q, const void* k, const
  * running (programmatic dependent launch): it fetches the handle's
  * constants at once, and the state, q, k and v only once that kernel has
  * finished, so inputs produced by the kernel just before are safe.  See
- * sfa_set_decode_input_prefetch for fetching q, k and v earlier. */
+ * sfa_set_decode_input_prefetch for fetching q, k and v earlier.
+ * Before any launch: SFA_ERR_INVALID_ARG (bad handle, batch <= 0, a NULL
+ * tensor), SFA_ERR_ALIGNMENT, SFA_ERR_UNSUPPORTED (batch > 65535).  A state
+ * whose header does not match is left untouched and latched as
+ * SFA_ERR_STATE_MISMATCH, as for sfa_prefill. */
 SFA_API int sfa_decode_step(const sfa_handle* h, const void* q, const void* k, const void* v,
                     int batch, void* state, float* out, void* stream);
 
 /* Serving variants.  The pages call the enhancement once per layer from
  * inside the model's attention ([P2] usage example and llama.cpp
  * integration: one call per layer with that layer's attention output); a
- * serving loop also drops finished sequences from a decode step.  These calls serve a range of layers and, for decode, a list of
- * sequences; the arithmetic is exactly that of the full calls.
+ * serving loop also drops finished sequences from a decode step.  These
+ * calls serve a range of layers and, for decode, a list of sequences; the
+ * arithmetic is exactly that of the full calls.
  *
  * Bytes of prefill workspace for a sfa_prefill_layers call of layer_count
  * layers; 0 on invalid input (layer_count outside 1 .. n_layers) or a call
