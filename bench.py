@@ -5,21 +5,26 @@ One step is one pass of the whole hot path over one batch of synthetic
 input; a token is one sequence position through all layers.  Three kinds of
 step, chosen by the workload:
 
-  * prefill + decode (default; tiny, qwen05b, qwen7b_decode): state reset,
-    prefill of the prompt, then the decode steps, every layer and sequence;
+  * decode only (batched_decode, the default, and the k x gamma_far x alpha
+    sweep points): the prompt is prefilled once, untimed; a step is the
+    workload's decode steps over all layers and sequences (each decode call
+    moves more than the L2, so nothing is flushed).
+  * prefill only (long_prefill): state reset and one prefill of the batch;
     L2 is flushed (256 MB write) before every timed step, outside its events.
-  * prefill only (long_prefill): state reset and one prefill of the batch.
-  * decode only (batched_decode and the k x gamma_far x alpha sweep points):
-    the prompt is prefilled once, untimed; a step is the workload's decode
-    steps over all layers and sequences (each decode call moves more than
-    the L2, so nothing is flushed).
+  * prefill + decode (tiny, qwen05b, qwen7b_decode): state reset, prefill of
+    the prompt, then the decode steps, every layer and sequence; L2 flushed
+    as for prefill.
 
-Default workload: the Qwen2.5-0.5B attention shape (24 layers, 14 query / 2
-KV heads, head_dim 64, batch 1, prefill 512 + 128 decode steps, k = 16,
-bf16 inputs).
+Default line: the batched decode of the Qwen2.5-7B attention shape (28
+layers, 28 query / 4 KV heads, head_dim 128, 256 sequences, k = 16, 1,024
+prefilled tokens, 512 timed decode steps, Student-t inputs in bf16) is the
+headline; the same run adds one object each for the long prefill (4 x 65,536
+tokens of one 7B-shaped layer), the Qwen2.5-0.5B step (512 + 128 tokens, 24
+layers, batch 1) and the decode time after 1K / 4K / 8K-token prompts
+(context flatness), each with its own roofline fraction.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                  [--workload NAME] [--context N]
+                  [--workload NAME] [--context N] [--no-extras]
 
 N > 1 runs under torch.distributed.run as independent replicas (the
 operator has no cross-stream exchange), timed per rank and reduced with MAX.
@@ -46,15 +51,21 @@ METRIC = "SFA prefill & decode tokens/s on 1 B200; achieved HBM GB/s vs ~8 TB/s 
 UNIT = "tokens/s"
 L2_FLUSH_BYTES = 256 << 20
 FALLBACK_HBM_GBS = 6650.0
+HEADLINE = "batched_decode"  # default workload of the bench line
+EXTRAS = ("long_prefill", "qwen05b")  # timed in the same run, each in its own object
+CONTEXTS = (1024, 4096, 8192)  # context-flatness object: decode after these prompt lengths
 
 
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="qwen05b")
+    ap.add_argument("--workload", default=HEADLINE)
+    ap.add_argument("--no-extras", action="store_true",
+                    help="time the headline workload only (no long_prefill, qwen05b and "
+                         "context-flatness objects)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--context", type=int, default=0,
@@ -235,42 +246,82 @@ def kernel_traffic(kernel_src: str, name: str, workload: str):
 # ------------------------------------------------------------------ oracle
 
 
-def oracle_tokens_per_s(w, layers, n_tokens, src, slots_np, seqs=None):
-    """Times the fp64 oracle on `layers` x `seqs` streams over n_tokens."""
+def sample_streams(w):
+    """The (layer, sequence) streams the oracle times: first, middle and last
+    layer and sequence (for the batched-decode sweep: layers 0, 14, 27 x
+    sequences 0, 128, 255)."""
+    pick = lambda n: sorted({0, n // 2, n - 1})
+    return pick(w.n_layers), pick(w.batch)
+
+
+def oracle_inputs(w, layers, seqs, n_tokens, dev):
+    """q, k, v of the chosen streams for positions 0 .. n_tokens-1, float32
+    numpy [len(layers), len(seqs), n, heads, d].  Drawn with the workload's
+    own generator on `dev` (the bench's GPU when there is one, so the oracle
+    sees exactly the values the GPU arm uses) one token block at a time, and
+    only the chosen streams are copied to the host."""
+    import torch
+    from workloads import TOKEN_BLOCK, TokenSource
+    src = TokenSource(w, dev)
+    li = torch.tensor(layers, device=dev)
+    si = torch.tensor(seqs, device=dev)
+    parts = ([], [], [])
+    for t0 in range(0, n_tokens, TOKEN_BLOCK):
+        blk = src.get(t0, min(n_tokens, t0 + TOKEN_BLOCK))
+        for i, x in enumerate(blk):
+            parts[i].append(x.index_select(0, li).index_select(1, si).float().cpu())
+        del blk
+    return tuple(torch.cat(p, dim=2).numpy() for p in parts)
+
+
+def oracle_tokens_per_s(w, layers, seqs, qn, kn, vn, slots_np):
+    """Times the fp64 oracle from position 0 on the streams layers x seqs
+    (inputs from oracle_inputs); returns (tokens/s as positions through all
+    layers, threads used, seconds)."""
     import numpy as np
     import oracle
     f = lambda x: float(np.float32(x))
     v = w.values
-    seqs = list(range(w.batch)) if seqs is None else list(seqs)
     p = oracle.OracleParams(w.n_q_heads, w.n_kv_heads, w.head_dim, w.window_k,
                             gamma_far=f(v.gamma_far), alpha_far=f(v.alpha_far))
-    q, k, vv = src.get(0, n_tokens)
-    sel = lambda x: x[layers][:, seqs].float().cpu().numpy()
-    qn, kn, vn = sel(q), sel(k), sel(vv)
-    st = oracle.OracleState(p, len(layers) * len(seqs))
-    slots = slots_np[layers]
+    pairs = [(a, b) for a in range(len(layers)) for b in range(len(seqs))]
+    n = qn.shape[2]
+    alpha = [oracle.alpha_layer(f(v.alpha_base), f(v.cross_decay), layers[a], w.n_layers)
+             for a, _ in pairs]
+    sl = np.stack([slots_np[layers[a]] for a, _ in pairs]).astype(np.float32)
+    qq = np.stack([qn[a, b] for a, b in pairs])
+    kk = np.stack([kn[a, b] for a, b in pairs])
+    vv = np.stack([vn[a, b] for a, b in pairs])
+    st = oracle.OracleState(p, len(pairs))
     t0 = time.perf_counter()
-    _, used = oracle.run_layers(p, f(v.alpha_base), f(v.cross_decay), slots, qn, kn, vn, st,
-                                n_layers=w.n_layers)
+    _, used = oracle.run_streams(p, alpha, sl, qq, kk, vv, st)
     dt = time.perf_counter() - t0
-    tokens = len(seqs) * n_tokens * len(layers) / w.n_layers  # positions through all layers
+    tokens = len(pairs) * n / w.n_layers  # positions through all layers
     return tokens / dt, used, dt
+
+
+def input_device():
+    """Where inputs for the oracle are drawn: the GPU when present."""
+    import torch
+    return torch.device("cuda", 0) if torch.cuda.is_available() else torch.device("cpu")
 
 
 def run_reference(args, w, n_pre):
     rank, world, _ = dist_env()
     if rank != 0:
         return
-    from workloads import TokenSource, make_slots
-    src = TokenSource(w, "cpu")
-    slots_np = make_slots(w, "cpu").numpy()
+    from workloads import make_slots
+    dev = input_device()
+    slots_np = make_slots(w, dev).cpu().numpy()
     n_tok = 64  # bounded sample per step: one layer, a few sequences, 64 positions
     seqs = list(range(min(w.batch, 4)))
+    steps = [s % w.n_layers for s in range(args.steps)]
+    inputs = {l: oracle_inputs(w, [l], seqs, n_tok, dev) for l in sorted(set(steps) | {0})}
     for _ in range(args.warmup):
-        oracle_tokens_per_s(w, [0], n_tok, src, slots_np, seqs)
+        oracle_tokens_per_s(w, [0], seqs, *inputs[0], slots_np)
     times, used = [], 1
-    for s in range(args.steps):
-        _, used, dt = oracle_tokens_per_s(w, [s % w.n_layers], n_tok, src, slots_np, seqs)
+    for l in steps:
+        _, used, dt = oracle_tokens_per_s(w, [l], seqs, *inputs[l], slots_np)
         times.append(dt)
     total = sum(times)
     tokens = args.steps * len(seqs) * n_tok / w.n_layers
@@ -334,12 +385,305 @@ def sfa_config_for(sfa, w):
 DECODE_RING = 64  # distinct decode inputs cycled by the decode-only step
 
 
+class Run:
+    """One workload's operator, inputs and captured CUDA graphs.
+
+    ``one_step(ev)`` replays one step (prefill part a, decode part b); with
+    ``ev`` it records three events around the parts."""
+
+    def __init__(self, w, n_pre, dev, rank, sfa):
+        import torch
+        from workloads import TokenSource, make_slots
+        self.w, self.n_pre = w, n_pre
+        self.kind = kind = step_kind(w)
+        n_dec = w.decode_steps
+        L, B, H = w.n_layers, w.batch, w.hidden
+        src = TokenSource(w, dev, salt=rank)
+        slots = make_slots(w, dev)
+        chunk = 128 if kind == "decode" else n_pre
+        op = sfa.SfaOperator(sfa_config_for(sfa, w), slots, B, max_prefill=chunk, device=dev)
+        self.op = op
+        # Every decode input is complete before its call: the timed steps
+        # replay inputs written before the timed region, and the e2e steps copy
+        # them in with cudaMemcpyAsync ordered by events.  So the decode kernel
+        # may fetch them before the previous kernel on the stream ends.
+        sfa.sfa_set_decode_input_prefetch(op.handle, True)
+        self.flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        self.qp = self.kp = self.vp = None
+        if kind == "decode":
+            # untimed prompt, in chunks; then a ring of distinct decode inputs
+            n_ring = min(DECODE_RING, n_dec)
+            out_c = torch.empty((L, B, chunk, H), dtype=torch.float32, device=dev)
+            for t0 in range(0, n_pre, chunk):
+                q, k, v = src.get(t0, min(n_pre, t0 + chunk))
+                op.prefill(q, k, v, out=out_c[:, :, :q.shape[2]])
+                del q, k, v
+            del out_c
+            qa, ka, va = src.get(n_pre, n_pre + n_ring)
+            qd = [qa[:, :, t].contiguous() for t in range(n_ring)]
+            kd = [ka[:, :, t].contiguous() for t in range(n_ring)]
+            vd = [va[:, :, t].contiguous() for t in range(n_ring)]
+            del qa, ka, va
+            out_d = torch.empty((n_ring, L, B, H), dtype=torch.float32, device=dev)
+            self.replays = max(1, n_dec // n_ring)
+            self.n_dec = self.replays * n_ring
+
+            def part_a():
+                pass
+
+            def part_b():
+                for t in range(n_ring):
+                    op.decode(qd[t], kd[t], vd[t], out=out_d[t])
+        else:
+            qp, kp, vp = src.get(0, n_pre)
+            self.qp, self.kp, self.vp = qp, kp, vp
+            qa, ka, va = src.get(n_pre, n_pre + n_dec)
+            qd = [qa[:, :, t].contiguous() for t in range(n_dec)]
+            kd = [ka[:, :, t].contiguous() for t in range(n_dec)]
+            vd = [va[:, :, t].contiguous() for t in range(n_dec)]
+            del qa, ka, va
+            out_p = torch.empty((L, B, n_pre, H), dtype=torch.float32, device=dev)
+            out_d = torch.empty((n_dec, L, B, H), dtype=torch.float32, device=dev)
+            self.replays = 1
+            self.n_dec = n_dec
+
+            def part_a():
+                op.reset()
+                op.prefill(qp, kp, vp, out=out_p)
+
+            def part_b():
+                for t in range(n_dec):
+                    op.decode(qd[t], kd[t], vd[t], out=out_d[t])
+        self.qd, self.kd, self.vd = qd, kd, vd
+        del src
+
+        # eager warm-up, then capture both halves as CUDA graphs
+        part_a()
+        part_b()
+        torch.cuda.synchronize()
+        rc = op.check()
+        if rc != 0:
+            raise SystemExit(f"{w.name}: device error during warm-up: {sfa.sfa_status_string(rc)}")
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        self.g_a, self.g_b = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        self.has_a, self.has_b = kind != "decode", kind != "prefill"
+        with torch.cuda.stream(side):
+            if self.has_a:
+                with torch.cuda.graph(self.g_a, stream=side):
+                    part_a()
+            if self.has_b:
+                with torch.cuda.graph(self.g_b, stream=side):
+                    part_b()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        self.flush_each = kind != "decode"
+        # our kernels per step: state header write + five prefill kernels;
+        # one per decode call
+        self.launches_per_step = (1 + 5 if self.has_a else 0) + (self.n_dec if self.has_b else 0)
+
+    def one_step(self, ev=None):
+        if self.flush_each:
+            self.flush.zero_()
+        if ev:
+            ev[0].record()
+        if self.has_a:
+            self.g_a.replay()
+        if ev:
+            ev[1].record()
+        for _ in range(self.replays if self.has_b else 0):
+            self.g_b.replay()
+        if ev:
+            ev[2].record()
+
+    def tokens_per_step(self):
+        return self.w.batch * ((self.n_pre if self.has_a else 0) + (self.n_dec if self.has_b else 0))
+
+    def release(self):
+        import torch
+        for name in ("g_a", "g_b", "op", "flush", "qd", "kd", "vd", "qp", "kp", "vp"):
+            if hasattr(self, name):
+                delattr(self, name)
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+
+
+def time_run(run, sfa, steps, warmup, world, dev, sampler=None):
+    """W untimed steps, then exactly K steps between barriers and device
+    synchronisations; per-step CUDA-event times of the prefill and decode
+    parts (ms) and the clock record of the timed region."""
+    import torch
+    import torch.distributed as dist
+    with nvtx_range(f"sfa {run.w.name} warm-up"):
+        for _ in range(warmup):
+            run.one_step()
+        torch.cuda.synchronize()
+    if run.op.check() != 0:
+        raise SystemExit(f"{run.w.name}: device error during warm-up")
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+        time.sleep(0.1)
+    with nvtx_range(f"sfa {run.w.name} timed steps"):
+        for s in range(steps):
+            run.one_step(ev[s])
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop() if sampler else None
+    pre_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    dec_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    rc = run.op.check()
+    if rc != 0:
+        raise SystemExit(f"{run.w.name}: device error in the timed region: "
+                         f"{sfa.sfa_status_string(rc)}")
+    return pre_ms, dec_ms, clocks
+
+
+def roofline_sections(run, pre_tot, dec_tot, steps, world, peak):
+    """Per part (prefill, decode): tokens/s, time, algorithmic bytes per
+    launch, achieved GB/s and the fraction of the HBM peak."""
+    w, B = run.w, run.w.batch
+    dec_bytes, pre_bytes = workload_bytes(w, run.n_pre)
+    section = {}
+    if run.has_a:
+        pre_ms_avg = pre_tot / steps
+        pre_gbs = pre_bytes / (pre_ms_avg / 1e3) / 1e9
+        section["prefill"] = {"tokens_per_s": job_rate(world, B * run.n_pre * steps, pre_tot),
+                              "ms": pre_ms_avg, "algorithmic_bytes": pre_bytes,
+                              "achieved_gbs": pre_gbs, "frac": pre_gbs / peak}
+    if run.has_b:
+        dec_launch_ms = dec_tot / (steps * run.n_dec)
+        dec_gbs = dec_bytes / (dec_launch_ms / 1e3) / 1e9
+        section["decode"] = {"tokens_per_s": job_rate(world, B * run.n_dec * steps, dec_tot),
+                             "us_per_step": 1e3 * dec_launch_ms, "algorithmic_bytes": dec_bytes,
+                             "achieved_gbs": dec_gbs, "frac": dec_gbs / peak}
+    return section
+
+
+def dominant_kernel(run):
+    """(part, kernel name, source file) of the kernel that dominates a step."""
+    if run.has_b and (not run.has_a or run.kind == "decode"):
+        if run.w.batch >= 64 and run.w.window_k <= 64:
+            return "decode", "decode_tile_kernel", "sfa_decode_tile.cu"
+        return "decode", "decode_kernel", "sfa_decode.cu"
+    return "prefill", "prefill", "sfa_prefill.cu"
+
+
+def roofline_for(run, section, peak, peak_src):
+    part, kernel, src = dominant_kernel(run)
+    if part not in section:  # a prefill-and-decode step whose prefill dominates
+        part = "prefill" if "prefill" in section else "decode"
+    dom = section[part]
+    traffic, traffic_wl = kernel_traffic(
+        os.path.join(ROOT, "kv_cache_compression_sfa_b200", "csrc", src), kernel, run.w.name)
+    return {"bound": "hbm", "kernel": kernel, "part": part, "achieved": dom["achieved_gbs"],
+            "peak": peak, "unit": "GB/s", "frac": dom["achieved_gbs"] / peak,
+            "peak_source": peak_src, "traffic": traffic,
+            "traffic_source": traffic_wl}
+
+
+def extra_object(args, name, sfa, world, dev, rank, peak, peak_src):
+    """A further workload timed in the same run: its own tokens/s, bytes,
+    GB/s and roofline fraction (steps and warm-up bounded to keep the run
+    short)."""
+    from workloads import get_workload
+    w = get_workload(name)
+    n_pre = w.prefill_n[0]
+    run = Run(w, n_pre, dev, rank, sfa)
+    steps = max(3, min(args.steps, 10))
+    pre_ms, dec_ms, _ = time_run(run, sfa, steps, max(3, args.warmup), world, dev)
+    total, pre_tot, dec_tot = max_over_ranks(
+        [sum(pre_ms) + sum(dec_ms), sum(pre_ms), sum(dec_ms)], world, dev)
+    section = roofline_sections(run, pre_tot, dec_tot, steps, world, peak)
+    obj = {"workload": workload_config(w, n_pre)["workload"],
+           "value": job_rate(world, run.tokens_per_step() * steps, total), "unit": UNIT,
+           "steps": steps, "ms_per_step": total / steps,
+           "median": step_medians(pre_ms, dec_ms), **section,
+           "roofline": roofline_for(run, section, peak, peak_src),
+           "gpu_launches": steps * run.launches_per_step,
+           "l2": workload_config(w, n_pre)["l2"]}
+    run.release()
+    return obj
+
+
+def context_rows(w, sfa, dev, contexts, n_dec=64, reps=4):
+    """Decode time per step after prompts of each length, with the SFA state
+    per sequence against a full K/V cache [P1 §2.2, §3.3, §3.4]: the prompt is
+    prefilled in 4,096-token calls, then n_dec decode steps are captured in a
+    CUDA graph and replayed `reps` times."""
+    import torch
+    from workloads import TokenSource, make_slots
+    src = TokenSource(w, dev)
+    op = sfa.SfaOperator(sfa_config_for(sfa, w), make_slots(w, dev), w.batch,
+                         max_prefill=4096, device=dev)
+    lay = op.layout()
+    state_per_seq = lay.stream_stride * w.n_layers
+    rows = []
+    for ctx in contexts:
+        op.reset()
+        for t0 in range(0, ctx, 4096):
+            q, k, v = src.get(t0, min(ctx, t0 + 4096))
+            op.prefill(q, k, v)
+            del q, k, v
+        qa, ka, va = src.get(ctx, ctx + n_dec)
+        qd = [qa[:, :, t].contiguous() for t in range(n_dec)]
+        kd = [ka[:, :, t].contiguous() for t in range(n_dec)]
+        vd = [va[:, :, t].contiguous() for t in range(n_dec)]
+        out_d = torch.empty((n_dec, w.n_layers, w.batch, w.hidden), dtype=torch.float32,
+                            device=dev)
+        for t in range(n_dec):  # warm-up (advances the state; cost is flat in t)
+            op.decode(qd[t], kd[t], vd[t], out=out_d[t])
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(g, stream=side):
+                for t in range(n_dec):
+                    op.decode(qd[t], kd[t], vd[t], out=out_d[t])
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        if op.check() != 0:
+            raise SystemExit("device error in the context report")
+        us = 1e3 * e0.elapsed_time(e1) / (reps * n_dec)
+        rows.append({"context": ctx, "decode_us_per_step": us,
+                     "sfa_state_bytes_per_seq": state_per_seq,
+                     "full_kv_bytes_per_seq": full_kv_bytes(w, ctx),
+                     "compression": full_kv_bytes(w, ctx) / state_per_seq})
+        del g, qd, kd, vd, out_d, qa, ka, va
+    del op
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return rows
+
+
+def flatness_object(sfa, dev):
+    from workloads import get_workload
+    w = get_workload("qwen7b_decode")
+    rows = context_rows(w, sfa, dev, CONTEXTS)
+    us = [r["decode_us_per_step"] for r in rows]
+    return {"workload": (f"{w.name}: {w.n_layers} layers, {w.n_q_heads}q/{w.n_kv_heads}kv heads, "
+                         f"head_dim {w.head_dim}, batch {w.batch}, k={w.window_k}; 64 decode "
+                         f"steps after each prompt"),
+            "rows": rows, "decode_us_spread": (max(us) - min(us)) / min(us)}
+
+
 def main():
     args = parse()
     from workloads import get_workload
     if args.report:
         run_report(args)
         return
+    headline_default = args.workload == HEADLINE
     w = get_workload(args.workload)
     n_pre = args.context or w.prefill_n[0]
     if args.impl == "reference":
@@ -350,7 +694,6 @@ def main():
     import torch.distributed as dist
     import kv_cache_compression_sfa_b200 as sfa
     from kv_cache_compression_sfa_b200 import build as sfa_build
-    from workloads import TokenSource, make_slots
 
     rank, world, local = dist_env()
     if not torch.cuda.is_available():
@@ -363,179 +706,54 @@ def main():
                                 device_id=dev)
     sfa_build.build()
 
-    kind = step_kind(w)
-    n_dec = w.decode_steps
-    L, B, H = w.n_layers, w.batch, w.hidden
-    src = TokenSource(w, dev, salt=rank)
-    slots = make_slots(w, dev)
-    chunk = 128 if kind == "decode" else n_pre
-    op = sfa.SfaOperator(sfa_config_for(sfa, w), slots, B, max_prefill=chunk, device=dev)
-    # Every decode input is complete before its call: the timed steps replay
-    # inputs written before the timed region, and the e2e steps copy them in
-    # with cudaMemcpyAsync ordered by events.  So the decode kernel may fetch
-    # them before the previous kernel on the stream ends.
-    sfa.sfa_set_decode_input_prefetch(op.handle, True)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-
-    if kind == "decode":
-        # untimed prompt, in chunks; then a ring of distinct decode inputs
-        n_ring = min(DECODE_RING, n_dec)
-        out_c = torch.empty((L, B, chunk, H), dtype=torch.float32, device=dev)
-        for t0 in range(0, n_pre, chunk):
-            q, k, v = src.get(t0, min(n_pre, t0 + chunk))
-            op.prefill(q, k, v, out=out_c[:, :, :q.shape[2]])
-            del q, k, v
-        del out_c
-        qa, ka, va = src.get(n_pre, n_pre + n_ring)
-        qd = [qa[:, :, t].contiguous() for t in range(n_ring)]
-        kd = [ka[:, :, t].contiguous() for t in range(n_ring)]
-        vd = [va[:, :, t].contiguous() for t in range(n_ring)]
-        del qa, ka, va
-        out_d = torch.empty((n_ring, L, B, H), dtype=torch.float32, device=dev)
-        replays = max(1, n_dec // n_ring)
-        n_dec = replays * n_ring
-
-        def part_a():
-            pass
-
-        def part_b():
-            for t in range(n_ring):
-                op.decode(qd[t], kd[t], vd[t], out=out_d[t])
-    else:
-        qp, kp, vp = src.get(0, n_pre)
-        qa, ka, va = src.get(n_pre, n_pre + n_dec)
-        qd = [qa[:, :, t].contiguous() for t in range(n_dec)]
-        kd = [ka[:, :, t].contiguous() for t in range(n_dec)]
-        vd = [va[:, :, t].contiguous() for t in range(n_dec)]
-        out_p = torch.empty((L, B, n_pre, H), dtype=torch.float32, device=dev)
-        out_d = torch.empty((n_dec, L, B, H), dtype=torch.float32, device=dev)
-        replays = 1
-
-        def part_a():
-            op.reset()
-            op.prefill(qp, kp, vp, out=out_p)
-
-        def part_b():
-            for t in range(n_dec):
-                op.decode(qd[t], kd[t], vd[t], out=out_d[t])
-
-    # eager warm-up, then capture both halves as CUDA graphs
-    part_a()
-    part_b()
-    torch.cuda.synchronize()
-    rc = op.check()
-    if rc != 0:
-        raise SystemExit(f"device error during warm-up: {sfa.sfa_status_string(rc)}")
-    side = torch.cuda.Stream()
-    side.wait_stream(torch.cuda.current_stream())
-    g_a, g_b = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-    has_a, has_b = kind != "decode", kind != "prefill"
-    with torch.cuda.stream(side):
-        if has_a:
-            with torch.cuda.graph(g_a, stream=side):
-                part_a()
-        if has_b:
-            with torch.cuda.graph(g_b, stream=side):
-                part_b()
-    torch.cuda.current_stream().wait_stream(side)
-    torch.cuda.synchronize()
-    flush_each = kind != "decode"
-
-    def one_step(ev=None):
-        if flush_each:
-            flush.zero_()
-        if ev:
-            ev[0].record()
-        if has_a:
-            g_a.replay()
-        if ev:
-            ev[1].record()
-        for _ in range(replays if has_b else 0):
-            g_b.replay()
-        if ev:
-            ev[2].record()
-
-    with nvtx_range("sfa warm-up"):
-        for _ in range(args.warmup):
-            one_step()
-        torch.cuda.synchronize()
-    if op.check() != 0:
-        raise SystemExit("device error during warm-up")
-
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    run = Run(w, n_pre, dev, rank, sfa)
     sampler = ClockSampler(gpu_index_for(dev)) if rank == 0 else None
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    if sampler:
-        sampler.start()
-        time.sleep(0.1)
-    with nvtx_range("sfa timed steps"):
-        for s in range(args.steps):
-            one_step(ev[s])
-        torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    clocks = sampler.stop() if sampler else None
-    pre_ms = [e[0].elapsed_time(e[1]) for e in ev]
-    dec_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    pre_ms, dec_ms, clocks = time_run(run, sfa, args.steps, args.warmup, world, dev, sampler)
     medians = step_medians(pre_ms, dec_ms)
-    rc = op.check()
-    if rc != 0:
-        raise SystemExit(f"device error in the timed region: {sfa.sfa_status_string(rc)}")
     total_ms, pre_tot, dec_tot = max_over_ranks(
         [sum(pre_ms) + sum(dec_ms), sum(pre_ms), sum(dec_ms)], world, dev)
-    timed_pre = n_pre if has_a else 0
-    tokens_per_step = B * (timed_pre + (n_dec if has_b else 0))
-    value = job_rate(world, tokens_per_step * args.steps, total_ms)
+    value = job_rate(world, run.tokens_per_step() * args.steps, total_ms)
     ms_per_step = total_ms / args.steps
 
-    # ---- roofline of the dominant kernel
     peak, peak_kind = measured_peaks()
-    dec_bytes, pre_bytes = workload_bytes(w, n_pre)
-    section = {}
-    if has_a:
-        pre_ms_avg = pre_tot / args.steps
-        pre_gbs = pre_bytes / (pre_ms_avg / 1e3) / 1e9
-        section["prefill"] = {"tokens_per_s": job_rate(world, B * n_pre * args.steps, pre_tot),
-                              "ms": pre_ms_avg, "algorithmic_bytes": pre_bytes,
-                              "achieved_gbs": pre_gbs, "frac": pre_gbs / peak}
-    if has_b:
-        dec_launch_ms = dec_tot / (args.steps * n_dec)
-        dec_gbs = dec_bytes / (dec_launch_ms / 1e3) / 1e9
-        section["decode"] = {"tokens_per_s": job_rate(world, B * n_dec * args.steps, dec_tot),
-                             "us_per_step": 1e3 * dec_launch_ms, "algorithmic_bytes": dec_bytes,
-                             "achieved_gbs": dec_gbs, "frac": dec_gbs / peak}
-    dominant = "decode" if has_b and (not has_a or dec_tot >= pre_tot) else "prefill"
-    dom = section[dominant]
-    traffic, _ = kernel_traffic(
-        os.path.join(ROOT, "kv_cache_compression_sfa_b200", "csrc", f"sfa_{dominant}.cu"),
-        dominant, w.name)
     peak_src = (f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
                 if peak_kind == "measured" else "fallback 6.65 TB/s")
+    section = roofline_sections(run, pre_tot, dec_tot, args.steps, world, peak)
+    roofline = roofline_for(run, section, peak, peak_src)
 
     # ---- e2e through the public API with host buffers
     e2e = None
     if not args.no_e2e:
         with nvtx_range("sfa e2e"):
-            if kind == "decode":
-                e2e = measure_e2e_decode(args, w, op, qd, kd, vd, n_dec, world, dev)
+            if run.kind == "decode":
+                e2e = measure_e2e_decode(args, w, run.op, run.qd, run.kd, run.vd, run.n_dec,
+                                         world, dev)
             else:
-                e2e = measure_e2e(args, w, op, qp, kp, vp, qd, kd, vd, n_pre, n_dec, world, dev)
+                e2e = measure_e2e(args, w, run.op, run.qp, run.kp, run.vp, run.qd, run.kd,
+                                  run.vd, n_pre, run.n_dec, world, dev)
+    launches = args.steps * run.launches_per_step
+    run.release()
+
+    # ---- further workloads in the same run (one GPU only: every replica of
+    # a multi-GPU run would repeat them)
+    extras = {}
+    if headline_default and not args.no_extras and world == 1:
+        for name in EXTRAS:
+            with nvtx_range(f"sfa extra {name}"):
+                extras[name] = extra_object(args, name, sfa, world, dev, rank, peak, peak_src)
+        with nvtx_range("sfa context flatness"):
+            extras["context_flatness"] = flatness_object(sfa, dev)
 
     # ---- oracle on the host cores (rank 0, N = 1 only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(w, n_pre)
+        cpu = cpu_baseline(w, n_pre, dev)
 
     if world > 1:
         dist.barrier()
-        del g_a, g_b
         dist.destroy_process_group()
     if rank != 0:
         return
-    # our kernels per step: state header write + five prefill kernels; one per decode call
-    launches_per_step = (1 + 5 if has_a else 0) + (n_dec if has_b else 0)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "median": medians,
@@ -545,13 +763,12 @@ def main():
                    "decode_inputs": "prefetched: complete before each call "
                                     "(sfa_set_decode_input_prefetch)"},
         **section,
-        "roofline": {"bound": "hbm", "kernel": f"sfa {dominant}", "achieved": dom["achieved_gbs"],
-                     "peak": peak, "unit": "GB/s", "frac": dom["achieved_gbs"] / peak,
-                     "peak_source": peak_src, "traffic": traffic},
+        "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": args.steps * launches_per_step,
+        "gpu_launches": launches,
         "clocks": clocks,
+        **extras,
     }
     print(json.dumps(line), flush=True)
 
@@ -699,29 +916,30 @@ def _time_e2e(one, steps, world, dev):
     return max_over_ranks([e0.elapsed_time(e1)], world, dev)[0]
 
 
-def cpu_baseline(w, n_pre):
-    import numpy as np
-    from workloads import TokenSource, make_slots
-    src = TokenSource(w, "cpu")
-    slots_np = make_slots(w, "cpu").numpy()
-    n_tok = n_pre + w.decode_steps
-    # bounded sample: positions 0 .. n_tok-1 of as many (layer, sequence)
-    # streams as fit in ~15 s, estimated from one layer of a few sequences
-    seqs = list(range(min(w.batch, 4)))
-    rate1, used1, dt1 = oracle_tokens_per_s(w, [0], n_tok, src, slots_np, seqs)
-    n_layers = max(1, min(w.n_layers, int(15.0 / max(dt1, 1e-3))))
-    layers = list(range(n_layers))
-    # repeat the sample (from a fresh state each time) until ~10 s of work
+def cpu_baseline(w, n_pre, dev):
+    """The fp64 oracle on the host cores, from position 0 over the workload's
+    prompt and decode steps, on the streams of sample_streams(w); the token
+    count is capped so one pass stays near 15 s, and the pass is repeated
+    (from a fresh state) until about 10 s of work."""
+    from workloads import make_slots
+    slots_np = make_slots(w, dev).cpu().numpy()
+    layers, seqs = sample_streams(w)
+    n_full = n_pre + w.decode_steps
+    q, k, v = oracle_inputs(w, layers, seqs, min(64, n_full), dev)
+    _, _, dt64 = oracle_tokens_per_s(w, layers, seqs, q, k, v, slots_np)
+    n_tok = max(64, min(n_full, int(64 * 15.0 / max(dt64, 1e-3))))
+    q, k, v = oracle_inputs(w, layers, seqs, n_tok, dev)
     total_tok, total_dt, reps, used = 0.0, 0.0, 0, 1
     while reps < 1 or (total_dt < 10.0 and reps < 100):
-        rate, used, dt = oracle_tokens_per_s(w, layers, n_tok, src, slots_np, seqs)
+        rate, used, dt = oracle_tokens_per_s(w, layers, seqs, q, k, v, slots_np)
         total_tok += rate * dt
         total_dt += dt
         reps += 1
     return {"value": total_tok / total_dt, "unit": UNIT, "cores": used, "kind": "oracle",
-            "sample": (f"{n_layers} of {w.n_layers} layers x {len(seqs)} of {w.batch} seq x "
-                       f"{n_tok} positions, repeated {reps} times ({total_dt:.1f} s); tokens "
-                       f"scaled to positions through all layers")}
+            "sample": (f"layers {layers} x sequences {seqs} of {w.name} ({w.n_layers} layers x "
+                       f"{w.batch} seq), positions 0..{n_tok - 1} of {n_full}, repeated {reps} "
+                       f"times ({total_dt:.1f} s); tokens scaled to positions through all "
+                       f"layers")}
 
 
 # ------------------------------------------------------------------ reports
@@ -767,60 +985,18 @@ def run_report(args):
     if args.report == "context":
         # state bytes per sequence vs a full K/V cache, and decode time per
         # step after prompts of growing length [P1 §2.2, §3.4]
-        w = get_workload(args.workload if args.workload != "qwen05b" else "qwen7b_decode")
-        src = TokenSource(w, dev)
-        op = sfa.SfaOperator(sfa_config_for(sfa, w), make_slots(w, dev), w.batch,
-                             max_prefill=4096, device=dev)
-        lay = op.layout()
-        state_per_seq = lay.stream_stride * w.n_layers
-        n_dec = 64
-        rows = []
-        ctx = 1024
+        w = get_workload(args.workload if args.workload != HEADLINE else "qwen7b_decode")
+        ctxs, ctx = [], 1024
         while ctx <= args.max_context:
-            op.reset()
-            for t0 in range(0, ctx, 4096):
-                q, k, v = src.get(t0, min(ctx, t0 + 4096))
-                op.prefill(q, k, v)
-                del q, k, v
-            qa, ka, va = src.get(ctx, ctx + n_dec)
-            qd = [qa[:, :, t].contiguous() for t in range(n_dec)]
-            kd = [ka[:, :, t].contiguous() for t in range(n_dec)]
-            vd = [va[:, :, t].contiguous() for t in range(n_dec)]
-            out_d = torch.empty((n_dec, w.n_layers, w.batch, w.hidden), dtype=torch.float32,
-                                device=dev)
-            for t in range(n_dec):  # warm-up (advances the state; cost is flat in t)
-                op.decode(qd[t], kd[t], vd[t], out=out_d[t])
-            g = torch.cuda.CUDAGraph()
-            side = torch.cuda.Stream()
-            side.wait_stream(torch.cuda.current_stream())
-            with torch.cuda.stream(side):
-                with torch.cuda.graph(g, stream=side):
-                    for t in range(n_dec):
-                        op.decode(qd[t], kd[t], vd[t], out=out_d[t])
-            torch.cuda.current_stream().wait_stream(side)
-            torch.cuda.synchronize()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            reps = 4
-            e0.record()
-            for _ in range(reps):
-                g.replay()
-            e1.record()
-            torch.cuda.synchronize()
-            if op.check() != 0:
-                raise SystemExit("device error in the context report")
-            us = 1e3 * e0.elapsed_time(e1) / (reps * n_dec)
-            rows.append({"context": ctx, "decode_us_per_step": us,
-                         "sfa_state_bytes_per_seq": state_per_seq,
-                         "full_kv_bytes_per_seq": full_kv_bytes(w, ctx),
-                         "compression": full_kv_bytes(w, ctx) / state_per_seq})
-            del g, qd, kd, vd, out_d, qa, ka, va
+            ctxs.append(ctx)
             ctx *= 2
+        rows = context_rows(w, sfa, dev, ctxs)
         print(json.dumps({"report": "context", "workload": w.name, "n_layers": w.n_layers,
                           "window_k": w.window_k, "rows": rows}), flush=True)
         return
 
     # enhancement share and its angle to x against alpha_base [P2 calibration]
-    w = get_workload(args.workload)
+    w = get_workload(args.workload if args.workload != HEADLINE else "qwen05b")
     n = args.context or w.prefill_n[0]
     src = TokenSource(w, dev)
     slots = make_slots(w, dev)
