@@ -567,7 +567,7 @@ def roofline_sections(run, pre_tot, dec_tot, steps, world, peak):
 def dominant_kernel(run):
     """(part, kernel name, source file) of the kernel that dominates a step."""
     if run.has_b and (not run.has_a or run.kind == "decode"):
-        if run.w.batch >= 64 and run.w.window_k <= 64:
+        if run.w.batch >= 64 and run.w.window_k <= 64:  # the library's batch-tiled rule
             return "decode", "decode_tile_kernel", "sfa_decode_tile.cu"
         return "decode", "decode_kernel", "sfa_decode.cu"
     return "prefill", "prefill", "sfa_prefill.cu"

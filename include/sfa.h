@@ -37,9 +37,9 @@
  *   - One state buffer serves `batch` sequences for all layers.  A state is
  *     used by one stream at a time; stream order serialises calls.  The
  *     compute calls never modify the handle, so it may be shared across
- *     streams and host threads (only sfa_set_decode_input_prefetch,
- *     sfa_debug_set_lookback and sfa_destroy modify it: call those while no
- *     other host thread uses the handle).
+ *     streams and host threads (only sfa_set_decode_input_prefetch, the
+ *     sfa_debug_* hooks and sfa_destroy modify it: call those while no other
+ *     host thread uses the handle).
  */
 #ifndef SFA_H
 #define SFA_H
@@ -57,7 +57,7 @@
 extern "C" {
 #endif
 
-#define SFA_ABI_VERSION 1
+#define SFA_ABI_VERSION 2
 
 typedef enum sfa_status {
   SFA_OK = 0,
@@ -131,7 +131,8 @@ SFA_API int sfa_config_validate(const sfa_config* cfg);
 /* State layout for `batch` sequences of `cfg` (host arithmetic, no CUDA). */
 SFA_API int sfa_state_layout_for(const sfa_config* cfg, int batch, sfa_state_layout* out);
 
-/* Creates a handle on the current device: validates cfg, copies the slots,
+/* [P2] engine init(n_layers, hidden): the operator's constants for one model.
+ * Creates a handle on the current device: validates cfg, copies the slots,
  * precomputes slot norms and the alpha_layer table, allocates the device
  * error word.  *out receives the handle, or NULL on error.  Returns the
  * status of sfa_config_validate for a bad configuration, SFA_ERR_UNSUPPORTED
@@ -139,10 +140,13 @@ SFA_API int sfa_state_layout_for(const sfa_config* cfg, int batch, sfa_state_lay
  * SFA_ERR_CUDA when a CUDA call fails (no device, out of memory). */
 SFA_API int sfa_init(const sfa_config* cfg, sfa_handle** out);
 
-/* Frees the handle's device memory (synchronises the device first). */
+/* [P2] engine lifetime: the counterpart of sfa_init.
+ * Frees the handle's device memory (synchronises the device first). */
 SFA_API int sfa_destroy(sfa_handle* h);
 
-/* Bytes of a state buffer for `batch` sequences; 0 on invalid input. */
+/* [P1 §2.2] O(k·d) state: its size depends on the window, the heads and
+ * the hidden size, never on the context length.
+ * Bytes of a state buffer for `batch` sequences; 0 on invalid input. */
 SFA_API size_t sfa_state_bytes(const sfa_handle* h, int batch);
 
 /* Bytes of prefill workspace for a call of n tokens x `batch`; 0 on invalid
@@ -153,11 +157,16 @@ SFA_API size_t sfa_state_bytes(const sfa_handle* h, int batch);
  * be initialised. */
 SFA_API size_t sfa_prefill_workspace_bytes(const sfa_handle* h, int batch, long long n);
 
-/* Zeroes `state` (state_bytes(h, batch) bytes) and writes its header for
+/* [P1 §2.2] state of the window, the far field and [P3 §2.1] the ring,
+ * field and position, all back to their empty values.
+ * Zeroes `state` (state_bytes(h, batch) bytes) and writes its header for
  * this handle and batch: every stream back to position 0. */
 SFA_API int sfa_state_reset(const sfa_handle* h, void* state, int batch, void* stream);
 
-/* Folds n >= 0 tokens per sequence into the state and writes their outputs.
+/* [P1 §2.1] near field (eq. O_near), far field (eq. S_t) and their sum
+ * (eq. O); [P3 §2.1] ring, field and semantic pool; [P3 §2.2] fusion, clip
+ * and alpha_layer, for n consecutive tokens of every sequence.
+ * Folds n >= 0 tokens per sequence into the state and writes their outputs.
  * Equivalent to n calls of sfa_decode_step (same results within rounding).
  * Continues from each stream's current position.  n == 0 enqueues nothing.
  * SFA_ERR_UNSUPPORTED when layers x batch exceeds 65535, n exceeds
@@ -174,7 +183,10 @@ SFA_API int sfa_prefill(const sfa_handle* h, const void* q, const void* k, const
                 long long n, int batch, void* state, float* out, void* workspace,
                 size_t workspace_bytes, void* stream);
 
-/* Folds one token per sequence into the state and writes its output.
+/* [P1 §2.1] and [P3 §2.1–2.2] for one token of every sequence: the
+ * per-step form of [P2]'s compute_enhancement(layer, attn_output), over all
+ * layers at once.
+ * Folds one token per sequence into the state and writes its output.
  * One kernel launch covers all layers and sequences; no workspace.
  * The kernel may start while the previous kernel on the stream is still
  * running (programmatic dependent launch): it fetches the handle's
@@ -279,7 +291,19 @@ SFA_API int sfa_prefill_static_ws(const sfa_handle* h, const void* q, const void
  * up and latches SFA_ERR_DEVICE_TIMEOUT (0 restores the default).  The
  * kernel still finishes and the context stays usable.  Affects later calls
  * on this handle only. */
-SFA_API int sfa_debug_set_lookback(sfa_handle* h, unsigned int spin_limit, long long withhold_tile);
+SFA_API int sfa_debug_set_wait_limit(sfa_handle* h, unsigned int spin_limit, long long withhold_tile);
+
+/* Test hook that pins the kernel variants, so that every variant can be
+ * checked on one workload (not needed in normal use; results agree within
+ * the operator's tolerance whichever runs).  decode_tile: -1 chooses the
+ * decode kernel by the number of sequences per call (the default), 0 always
+ * the per-sequence kernel, 1 always the batch-tiled kernel.
+ * prefill_near_tc: 1 runs the prefill near field on the tensor cores where
+ * they apply (bf16 inputs, k <= 16; the default), 0 on the CUDA cores.
+ * SFA_ERR_INVALID_ARG for other values, SFA_ERR_UNSUPPORTED if the requested
+ * kernel does not fit this configuration (nothing changes then).  Affects
+ * later calls on this handle only. */
+SFA_API int sfa_debug_set_paths(sfa_handle* h, int decode_tile, int prefill_near_tc);
 
 #ifdef __cplusplus
 }

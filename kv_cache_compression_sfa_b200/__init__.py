@@ -43,7 +43,7 @@ EXPORTED = (
     "sfa_config_default", "sfa_config_validate", "sfa_state_layout_for", "sfa_init",
     "sfa_destroy", "sfa_state_bytes", "sfa_prefill_workspace_bytes", "sfa_state_reset",
     "sfa_prefill", "sfa_decode_step", "sfa_check_device_status", "sfa_status_string",
-    "sfa_abi_version", "sfa_debug_set_lookback", "sfa_prefill_static_ws",
+    "sfa_abi_version", "sfa_debug_set_wait_limit", "sfa_debug_set_paths", "sfa_prefill_static_ws",
     "sfa_prefill_layers_workspace_bytes", "sfa_prefill_layers", "sfa_decode_step_ex",
     "sfa_set_decode_input_prefetch",
 )
@@ -105,7 +105,8 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
             "sfa_check_device_status": (i, [vp, vp]),
             "sfa_status_string": (ctypes.c_char_p, [i]),
             "sfa_abi_version": (i, []),
-            "sfa_debug_set_lookback": (i, [vp, ctypes.c_uint, ll]),
+            "sfa_debug_set_wait_limit": (i, [vp, ctypes.c_uint, ll]),
+            "sfa_debug_set_paths": (i, [vp, i, i]),
             "sfa_prefill_static_ws": (i, [vp, vp, vp, vp, ll, i, vp, vp, vp]),
             "sfa_prefill_layers_workspace_bytes": (sz, [vp, i, i, ll]),
             "sfa_prefill_layers": (i, [vp, i, i, vp, vp, vp, ll, i, vp, vp, vp, sz, vp]),
@@ -372,13 +373,22 @@ def sfa_check_device_status(h: Handle, stream=None) -> int:
     return int(load_library().sfa_check_device_status(h.ptr, _stream_ptr(stream)))
 
 
-def sfa_debug_set_lookback(h: Handle, spin_limit: int = 0, withhold_tile: int = -1) -> None:
+def sfa_debug_set_wait_limit(h: Handle, spin_limit: int = 0, withhold_tile: int = -1) -> None:
     """Test hook of the prefill's bounded waits: the pool CTA of tile
     `withhold_tile` (tile * streams + stream) waits on a barrier that nothing
     completes, giving up after `spin_limit` polls (0: default); -1 disables."""
-    rc = load_library().sfa_debug_set_lookback(h.ptr, spin_limit, withhold_tile)
+    rc = load_library().sfa_debug_set_wait_limit(h.ptr, spin_limit, withhold_tile)
     if rc != SFA_OK:
-        raise SfaError(rc, "sfa_debug_set_lookback")
+        raise SfaError(rc, "sfa_debug_set_wait_limit")
+
+
+def sfa_debug_set_paths(h: Handle, decode_tile: int = -1, prefill_near_tc: bool = True) -> None:
+    """Test hook that pins the kernel variants: decode_tile -1 (by batch
+    size), 0 (per-sequence kernel) or 1 (batch-tiled kernel); prefill near
+    field on the tensor cores (True, where they apply) or CUDA cores."""
+    rc = load_library().sfa_debug_set_paths(h.ptr, int(decode_tile), 1 if prefill_near_tc else 0)
+    if rc != SFA_OK:
+        raise SfaError(rc, "sfa_debug_set_paths")
 
 
 class SfaOperator:

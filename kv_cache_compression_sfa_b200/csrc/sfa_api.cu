@@ -14,7 +14,6 @@
 #include <cstdint>
 #include <algorithm>
 #include <type_traits>
-#include <cstdlib>
 #include <cstring>
 #include <new>
 #include <vector>
@@ -41,8 +40,9 @@ struct sfa_handle {
   unsigned spin_limit;
   long long withhold_tile;
   bool tile_ok;          // the batch-tiled decode fits this configuration
-  int tile_smem;         // its dynamic shared memory per CTA
-  int tile_mode;         // -1: by batch size; 0: never; 1: always (test hook)
+  TilePlan tile_plan;    // its shared-memory plan
+  int tile_mode;         // -1: by batch size; 0: never; 1: always (sfa_debug_set_paths)
+  bool near_tc;          // prefill near field on the tensor cores where it applies
   bool inputs_early;     // decode inputs declared complete before each call
 };
 
@@ -156,6 +156,15 @@ bool handle_ok(const sfa_handle* h) { return h != nullptr && h->magic == kHandle
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? SFA_OK : SFA_ERR_CUDA; }
 
+// Near-field plan of the prefill: on the tensor cores where they apply (bf16
+// inputs, k <= 16) unless h->near_tc is off, else on the CUDA cores.
+bool plan_near_field(sfa_handle* h, size_t limit) {
+  const sfa_config* c = &h->cfg;
+  const int esz = static_cast<int>(in_bytes(c->in_dtype));
+  return (h->near_tc && plan_near(c->head_dim, esz, c->window_k, limit, true, &h->near)) ||
+         plan_near(c->head_dim, esz, c->window_k, limit, false, &h->near);
+}
+
 template <typename P>
 void fill_common(P& p, const sfa_handle* h, int batch, void* state) {
   const sfa_config* c = &h->cfg;
@@ -261,13 +270,8 @@ int sfa_init(const sfa_config* cfg, sfa_handle** out) {
   h->spin_limit = kDefaultSpinLimit;
   h->withhold_tile = -1;
   h->inputs_early = false;
-  {
-    // Test hook (environment, read once per handle): SFA_DECODE_TILE=0 / 1
-    // turns the batch-tiled decode off / on for every batch size (default:
-    // from kDecodeTileMinSeqs sequences per call).
-    const char* tenv = std::getenv("SFA_DECODE_TILE");
-    h->tile_mode = (tenv && tenv[0] == '0') ? 0 : (tenv && tenv[0] == '1') ? 1 : -1;
-  }
+  h->tile_mode = -1;
+  h->near_tc = true;
   const int L = cfg->n_layers, H = hidden_of(cfg);
   bool no_fit = false;  // a kernel's shared-memory plan does not fit this device
   const size_t slot_bytes = sizeof(float) * static_cast<size_t>(L) * kSlots * H;
@@ -289,14 +293,7 @@ int sfa_init(const sfa_config* cfg, sfa_handle** out) {
     // device.
     const size_t limit = prefill_smem_limit(h->device);
     const int esz = static_cast<int>(in_bytes(cfg->in_dtype));
-    // Test hook (environment, read once per handle): SFA_CUDA_CORE_NEAR_FIELD=1
-    // keeps the prefill near field on the CUDA cores where the tensor-core
-    // one applies (bf16, k <= 16), so both can be checked on one workload.
-    const char* nenv = std::getenv("SFA_CUDA_CORE_NEAR_FIELD");
-    const bool tc = !(nenv && nenv[0] == '1');
-    if (!(tc && plan_near(cfg->head_dim, esz, cfg->window_k, limit, true, &h->near)) &&
-        !plan_near(cfg->head_dim, esz, cfg->window_k, limit, false, &h->near))
-      no_fit = true;
+    if (!plan_near_field(h, limit)) no_fit = true;
     if (static_cast<size_t>(std::max(prefill_pool_smem(), prefill_out_smem())) > limit)
       no_fit = true;
     if (no_fit) e = cudaErrorInvalidConfiguration;
@@ -310,10 +307,10 @@ int sfa_init(const sfa_config* cfg, sfa_handle** out) {
       if (decode_max_active_clusters(cs, dsm, cfg->in_dtype, cfg->head_dim) < 1) continue;
       h->cs = cs;
       h->decode_budget = decode_budget(limit);
-      const size_t tsm = decode_tile_smem_bytes(hpc, cfg->head_dim, limit);
-      h->tile_smem = static_cast<int>(tsm);
-      h->tile_ok = tsm <= limit &&
-                   decode_tile_max_active_clusters(cs, tsm, cfg->in_dtype, cfg->head_dim) >= 1;
+      h->tile_ok = plan_decode_tile(hpc, cfg->head_dim, esz, cfg->n_q_heads / cfg->n_kv_heads,
+                                     cfg->window_k, limit, &h->tile_plan) &&
+                   decode_tile_max_active_clusters(cs, static_cast<size_t>(h->tile_plan.total),
+                                                   cfg->in_dtype, cfg->head_dim) >= 1;
       break;
     }
     if (e == cudaSuccess && h->cs == 0) {
@@ -518,12 +515,12 @@ int sfa_decode_step_ex(const sfa_handle* h, int layer_begin, int layer_count, co
   p.HPC = c->n_q_heads / p.CS;
   p.NGm = max_kv_heads_per_cta(c->n_q_heads, c->n_kv_heads, p.CS);
   p.smem_budget = h->decode_budget;
-  p.tile_smem = h->tile_smem;
+  p.tp = h->tile_plan;
   p.inputs_early = h->inputs_early ? 1 : 0;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // Batch-tiled decode from kDecodeTileMinSeqs sequences with windows of at
-  // most kDecodeTileMaxWindow positions (longer windows: each warp walks its
-  // window serially and the per-stream kernel, which splits it, is faster).
+  // Batch-tiled decode from kDecodeTileMinSeqs sequences per call with
+  // windows of at most kDecodeTileMaxWindow positions (longer windows: the
+  // per-sequence kernel, which splits a head's window over warps, is faster).
   const bool tile = h->tile_ok &&
                     (h->tile_mode == 1 || (h->tile_mode < 0 && n_seq >= kDecodeTileMinSeqs &&
                                            c->window_k <= kDecodeTileMaxWindow));
@@ -568,10 +565,27 @@ int sfa_set_decode_input_prefetch(sfa_handle* h, int enable) {
   return SFA_OK;
 }
 
-int sfa_debug_set_lookback(sfa_handle* h, unsigned int spin_limit, long long withhold_tile) {
+int sfa_debug_set_wait_limit(sfa_handle* h, unsigned int spin_limit, long long withhold_tile) {
   if (!handle_ok(h)) return SFA_ERR_INVALID_ARG;
   h->spin_limit = spin_limit ? spin_limit : kDefaultSpinLimit;
   h->withhold_tile = withhold_tile < 0 ? -1 : withhold_tile;
+  return SFA_OK;
+}
+
+int sfa_debug_set_paths(sfa_handle* h, int decode_tile, int prefill_near_tc) {
+  if (!handle_ok(h) || decode_tile < -1 || decode_tile > 1 || prefill_near_tc < 0 ||
+      prefill_near_tc > 1)
+    return SFA_ERR_INVALID_ARG;
+  if (decode_tile == 1 && !h->tile_ok) return SFA_ERR_UNSUPPORTED;
+  const bool old_tc = h->near_tc;
+  const NearPlan old_plan = h->near;
+  h->near_tc = prefill_near_tc == 1;
+  if (!plan_near_field(h, prefill_smem_limit(h->device))) {
+    h->near_tc = old_tc;
+    h->near = old_plan;
+    return SFA_ERR_UNSUPPORTED;
+  }
+  h->tile_mode = decode_tile;
   return SFA_OK;
 }
 

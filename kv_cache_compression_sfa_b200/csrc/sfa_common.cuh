@@ -205,6 +205,21 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const void* map, int x, i
       : "memory");
 }
 
+// 4-D tiled bulk tensor load (no multicast), as tma_load_3d.
+__device__ __forceinline__ void tma_load_4d(void* dst, const void* map, int x, int y, int z, int w,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], [%6];" ::
+          "r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w),
+          "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Plain arrive (count 1, no transaction bytes) on a barrier of this CTA.
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 // Orders this thread's earlier generic-proxy shared-memory accesses before
 // later bulk copies (async proxy) into the same bytes.
 __device__ __forceinline__ void fence_proxy_async_smem() {

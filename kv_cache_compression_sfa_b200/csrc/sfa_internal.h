@@ -31,9 +31,12 @@ constexpr int kTile = 64;                 // tokens per prefill tile
 constexpr int kHalo = kRing - 1;          // x rows a token needs from before its tile
 constexpr int kPrefillThreads = 256;
 constexpr int kDecodeThreads = 256;
-constexpr int kDecodeTileThreads = 256;     // batch-tiled decode (64 sequences per tile)
+constexpr int kDecodeTileThreads = 256;     // batch-tiled decode: compute threads (plus one copy warp)
 constexpr int kDecodeTileMinSeqs = 64;      // batch-tiled decode from this many sequences per call
 constexpr int kDecodeTileMaxWindow = 64;    // ... and windows of at most this many positions
+constexpr int kDecodeTileHeads = 8;         // query heads of one near-field work item
+constexpr int kDecodeTileChunk = 16;        // window slots per staged chunk
+constexpr int kDecodeTileMaxStages = 12;
 
 constexpr unsigned kDefaultSpinLimit = 1u << 21;  // polls of a bounded wait
 
@@ -52,6 +55,25 @@ static_assert(sizeof(StateHeader) <= kHeaderBytes, "header too large");
 struct StreamOffsets {
   long long pos, win_k, win_v, far, field, ring_sum, ring;
   long long stride;
+};
+
+// Shared-memory plan of the batch-tiled decode (byte offsets; see
+// sfa_decode_tile.cu).
+struct TilePlan {
+  int bars;       // mbarriers and the tensor-memory address
+  int xs;         // [64][HS + 4] fp32 x of the tile's sequences
+  int rows;       // [64] positions, then [64] stream indices (int64)
+  int sl;         // [HS / 64][hi, lo] slot blocks of the slice
+  int xw;         // [hi, lo] split x block, then the pool-weight block
+  int pb;         // per compute warp: P [8][16], corrections [8], denominators [8]
+  int hdr;        // per compute warp: q of up to 8 heads, K_t, V_t, S of one KV head
+  int hdr_bytes;  // bytes of one warp's header
+  int hq, hkt, hvt, hs;  // offsets inside a header
+  int stg;        // ring of staged window chunks; after the near field the pool partials
+  int stage;      // bytes per stage (keys, then values)
+  int kcb;        // window slots per chunk
+  int ns;         // stages
+  int total;      // dynamic shared memory
 };
 
 struct DecodeParams {
@@ -74,7 +96,7 @@ struct DecodeParams {
   int n_seq;
   int NGm;          // most KV heads any CTA needs
   int smem_budget;  // shared-memory bytes the plan may use (window staged if it fits)
-  int tile_smem;    // dynamic shared memory of the batch-tiled decode
+  TilePlan tp;      // shared-memory plan of the batch-tiled decode
   int inputs_early; // q, K_t, V_t may be fetched before the wait for the previous kernel
   float gamma_far, alpha_far, ema_gamma, inv_temp, clip_eps, score_scale;
 };
@@ -146,7 +168,9 @@ inline long long align256(long long x) { return (x + 255) & ~255LL; }
 cudaError_t launch_decode(const DecodeParams& p, int in_dtype, int head_dim, cudaStream_t s);
 cudaError_t launch_decode_tile(const DecodeParams& p, int in_dtype, int head_dim, cudaStream_t s);
 cudaError_t decode_tile_prepare(int device);
-size_t decode_tile_smem_bytes(int HPC, int head_dim, size_t limit);
+// Plan of the batch-tiled decode within `limit` bytes of shared memory;
+// false if none fits.
+bool plan_decode_tile(int HPC, int head_dim, int esz, int G, int K, size_t limit, TilePlan* out);
 int decode_tile_max_active_clusters(int cs, size_t smem, int in_dtype, int head_dim);
 cudaError_t launch_prefill(const PrefillParams& p, int in_dtype, int head_dim, cudaStream_t s);
 // Near-field plan for head_dim D, input element size esz and window K within

@@ -66,7 +66,8 @@ int main(void) {
                            dummy_input, (float*)dummy_input, NULL) == SFA_ERR_INVALID_ARG);
   CHECK(sfa_set_decode_input_prefetch(NULL, 1) == SFA_ERR_INVALID_ARG);
   CHECK(sfa_check_device_status(NULL, NULL) == SFA_ERR_INVALID_ARG);
-  CHECK(sfa_debug_set_lookback(NULL, 0, -1) == SFA_ERR_INVALID_ARG);
+  CHECK(sfa_debug_set_wait_limit(NULL, 0, -1) == SFA_ERR_INVALID_ARG);
+  CHECK(sfa_debug_set_paths(NULL, -1, 1) == SFA_ERR_INVALID_ARG);
 
   printf("ok\n");
   return 0;

@@ -99,13 +99,13 @@ def test_bounded_wait_runs_out_and_the_context_survives():
     op = sfa.SfaOperator(sfa_config(w), make_slots(w, "cuda"), w.batch, max_prefill=256)
     n_streams = w.n_layers * w.batch
     # tile 1 of stream 0: index = tile * n_streams + stream
-    sfa.sfa_debug_set_lookback(op.handle, spin_limit=2000, withhold_tile=1 * n_streams + 0)
+    sfa.sfa_debug_set_wait_limit(op.handle, spin_limit=2000, withhold_tile=1 * n_streams + 0)
     q, k, v = TokenSource(w, "cuda").get(0, 256)
     op.prefill(q, k, v)
     assert op.check() == sfa.SFA_ERR_DEVICE_TIMEOUT
     # back to normal: the same call on a fresh state succeeds and matches a
     # fresh operator
-    sfa.sfa_debug_set_lookback(op.handle, 0, -1)
+    sfa.sfa_debug_set_wait_limit(op.handle, 0, -1)
     op.reset()
     got = op.prefill(q, k, v)
     assert op.check() == 0

@@ -12,6 +12,7 @@ import numpy as np
 import pytest
 import torch
 
+import kv_cache_compression_sfa_b200 as sfa
 from sfa_harness import TOL, Pair, assert_close
 from workloads import WORKLOADS, SfaConfigValues, Workload, sweep_c5
 
@@ -24,9 +25,12 @@ def _tiny_variant(**kw) -> Workload:
     return base.replace(values=dataclasses.replace(base.values, **vals), **kw)
 
 
-def _run_schedule(w: Workload, schedule, layers=None, seqs=None, check_state=True):
-    """schedule: list of ("p", n) prefill calls and ("d", steps) decode runs."""
+def _run_schedule(w: Workload, schedule, layers=None, seqs=None, check_state=True, paths=None):
+    """schedule: list of ("p", n) prefill calls and ("d", steps) decode runs;
+    paths: (decode_tile, prefill_near_tc) for sfa_debug_set_paths."""
     pair = Pair(w, layers=layers, seqs=seqs)
+    if paths is not None:
+        sfa.sfa_debug_set_paths(pair.op.handle, *paths)
     tol = TOL[w.in_dtype]
     for kind, n in schedule:
         if kind == "p":
@@ -121,13 +125,12 @@ def test_edge_schedules(name, over, schedule):
     _run_schedule(w, schedule)
 
 
-def test_cuda_core_near_field_on_bf16_inputs(monkeypatch):
+def test_cuda_core_near_field_on_bf16_inputs():
     """bf16 inputs with k <= 16 take the tensor-core near field; the handle's
     test hook keeps them on the CUDA cores, which must meet the same bar."""
-    monkeypatch.setenv("SFA_CUDA_CORE_NEAR_FIELD", "1")
     w = _tiny_variant(name="cuda_core_near_bf16", n_layers=2, batch=2, n_q_heads=14,
                       n_kv_heads=2, head_dim=64, window_k=16, in_dtype="bf16")
-    _run_schedule(w, [("p", 130), ("d", 5), ("p", 70)])
+    _run_schedule(w, [("p", 130), ("d", 5), ("p", 70)], paths=(-1, False))
 
 
 def test_gqa7_bf16_chunked_prefill_and_decode():
@@ -137,20 +140,16 @@ def test_gqa7_bf16_chunked_prefill_and_decode():
     _run_schedule(w, [("p", 130), ("d", 5), ("p", 70)])
 
 
-@pytest.mark.parametrize("name,over,schedule",
-                         [e for e in EDGE if e[0] in ("gqa_f32_d64", "mha_k1", "k256_spans_tiles",
-                                                      "d128_f32_multilayer", "gqa7_bf16",
-                                                      "decode_from_empty", "eight_heads_per_cta")],
-                         ids=lambda x: x if isinstance(x, str) else "")
-def test_batch_tiled_decode_on_edge_schedules(monkeypatch, name, over, schedule):
+@pytest.mark.parametrize("name,over,schedule", EDGE, ids=[e[0] for e in EDGE])
+def test_batch_tiled_decode_on_edge_schedules(name, over, schedule):
     """The batch-tiled decode (64 sequences per cluster, pool on the tensor
-    cores) serves every batch when SFA_DECODE_TILE=1; same bar as above."""
-    monkeypatch.setenv("SFA_DECODE_TILE", "1")
+    cores) serves every batch when the handle's test hook pins it; same bar
+    as above."""
     w = _tiny_variant(name=name + "_tiled", **over)
-    _run_schedule(w, schedule)
+    _run_schedule(w, schedule, paths=(1, True))
 
 
-def test_batch_tiled_decode_partial_tile_and_sequence_list(monkeypatch):
+def test_batch_tiled_decode_partial_tile_and_sequence_list():
     """70 sequences (a full and a partial tile), then a permuted subset."""
     w = _tiny_variant(name="tiled_70", n_layers=2, batch=70, n_q_heads=14, n_kv_heads=2,
                       head_dim=64, window_k=16, in_dtype="bf16")

@@ -19,8 +19,10 @@ def _w(**kw):
     return WORKLOADS["qwen05b"].replace(**base)
 
 
-def _op(w, slots):
-    return sfa.SfaOperator(sfa_config(w), slots, w.batch, device="cuda")
+def _op(w, slots, decode_tile=-1):
+    op = sfa.SfaOperator(sfa_config(w), slots, w.batch, device="cuda")
+    sfa.sfa_debug_set_paths(op.handle, decode_tile, True)
+    return op
 
 
 def _state_equal(a, b):
@@ -58,19 +60,20 @@ def test_layer_range_calls_equal_the_full_calls(split):
     _state_equal(full, part)
 
 
-def test_decode_of_a_subset_of_the_batch():
+@pytest.mark.parametrize("decode_tile", [0, 1], ids=["per_sequence", "batch_tiled"])
+def test_decode_of_a_subset_of_the_batch(decode_tile):
     w = _w(n_layers=2, batch=4)
     slots = make_slots(w, "cuda")
     src = TokenSource(w, "cuda")
     q, k, v = src.get(0, 70)
-    op = _op(w, slots)
+    op = _op(w, slots, decode_tile)
     op.prefill(q, k, v)
     keep = [1, 3]
     before = sfa.read_state(op)
     # reference: a batch holding only sequences 2 and 0, in that order
     sel = torch.tensor([2, 0], device="cuda")
     wr = w.replace(batch=2)
-    ref = _op(wr, slots)
+    ref = _op(wr, slots, decode_tile)
     ref.prefill(*(x.index_select(1, sel).contiguous() for x in (q, k, v)))
     ids = torch.tensor([2, 0], dtype=torch.int32, device="cuda")
     for t in range(70, 75):
@@ -107,11 +110,12 @@ def test_subset_decode_matches_the_oracle():
     pair.compare_state(TOL[w.in_dtype])
 
 
-def test_out_of_range_sequence_is_skipped_and_latched():
+@pytest.mark.parametrize("decode_tile", [0, 1], ids=["per_sequence", "batch_tiled"])
+def test_out_of_range_sequence_is_skipped_and_latched(decode_tile):
     w = _w(n_layers=1, batch=2)
     slots = make_slots(w, "cuda")
     src = TokenSource(w, "cuda")
-    op = _op(w, slots)
+    op = _op(w, slots, decode_tile)
     op.prefill(*src.get(0, 20))
     assert op.check() == 0
     before = sfa.read_state(op)
