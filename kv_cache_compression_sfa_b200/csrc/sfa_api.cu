@@ -307,10 +307,8 @@ int sfa_init(const sfa_config* cfg, sfa_handle** out) {
       if (decode_max_active_clusters(cs, dsm, cfg->in_dtype, cfg->head_dim) < 1) continue;
       h->cs = cs;
       h->decode_budget = decode_budget(limit);
-      h->tile_ok = plan_decode_tile(hpc, cfg->head_dim, esz, cfg->n_q_heads / cfg->n_kv_heads,
-                                     cfg->window_k, limit, &h->tile_plan) &&
-                   decode_tile_max_active_clusters(cs, static_cast<size_t>(h->tile_plan.total),
-                                                   cfg->in_dtype, cfg->head_dim) >= 1;
+      h->tile_ok = plan_decode_tile(hidden_of(cfg), cfg->head_dim, esz, cfg->n_q_heads / cfg->n_kv_heads,
+                                    cfg->window_k, limit, &h->tile_plan);
       break;
     }
     if (e == cudaSuccess && h->cs == 0) {
@@ -518,12 +516,9 @@ int sfa_decode_step_ex(const sfa_handle* h, int layer_begin, int layer_count, co
   p.tp = h->tile_plan;
   p.inputs_early = h->inputs_early ? 1 : 0;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // Batch-tiled decode from kDecodeTileMinSeqs sequences per call with
-  // windows of at most kDecodeTileMaxWindow positions (longer windows: the
-  // per-sequence kernel, which splits a head's window over warps, is faster).
+  // Batch-tiled decode from kDecodeTileMinSeqs sequences per call.
   const bool tile = h->tile_ok &&
-                    (h->tile_mode == 1 || (h->tile_mode < 0 && n_seq >= kDecodeTileMinSeqs &&
-                                           c->window_k <= kDecodeTileMaxWindow));
+                    (h->tile_mode == 1 || (h->tile_mode < 0 && n_seq >= kDecodeTileMinSeqs));
   if (tile) return cuda_status(launch_decode_tile(p, c->in_dtype, c->head_dim, s));
   return cuda_status(launch_decode(p, c->in_dtype, c->head_dim, s));
 }

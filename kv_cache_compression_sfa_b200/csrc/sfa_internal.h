@@ -31,12 +31,9 @@ constexpr int kTile = 64;                 // tokens per prefill tile
 constexpr int kHalo = kRing - 1;          // x rows a token needs from before its tile
 constexpr int kPrefillThreads = 256;
 constexpr int kDecodeThreads = 256;
-constexpr int kDecodeTileThreads = 256;     // batch-tiled decode: compute threads (plus one copy warp)
 constexpr int kDecodeTileMinSeqs = 64;      // batch-tiled decode from this many sequences per call
-constexpr int kDecodeTileMaxWindow = 64;    // ... and windows of at most this many positions
-constexpr int kDecodeTileHeads = 8;         // query heads of one near-field work item
+constexpr int kDecodeTileHeads = 8;         // most query heads per KV head it serves
 constexpr int kDecodeTileChunk = 16;        // window slots per staged chunk
-constexpr int kDecodeTileMaxStages = 12;
 
 constexpr unsigned kDefaultSpinLimit = 1u << 21;  // polls of a bounded wait
 
@@ -57,23 +54,17 @@ struct StreamOffsets {
   long long stride;
 };
 
-// Shared-memory plan of the batch-tiled decode (byte offsets; see
-// sfa_decode_tile.cu).
+// Plans of the batch-tiled decode (byte offsets and sizes; see
+// sfa_decode_tile.cu): its near-field kernel and its pool kernel.
 struct TilePlan {
-  int bars;       // mbarriers and the tensor-memory address
-  int xs;         // [64][HS + 4] fp32 x of the tile's sequences
-  int rows;       // [64] positions, then [64] stream indices (int64)
-  int sl;         // [HS / 64][hi, lo] slot blocks of the slice
-  int xw;         // [hi, lo] split x block, then the pool-weight block
-  int pb;         // per compute warp: P [8][16], corrections [8], denominators [8]
-  int hdr;        // per compute warp: q of up to 8 heads, K_t, V_t, S of one KV head
-  int hdr_bytes;  // bytes of one warp's header
-  int hq, hkt, hvt, hs;  // offsets inside a header
-  int stg;        // ring of staged window chunks; after the near field the pool partials
-  int stage;      // bytes per stage (keys, then values)
-  int kcb;        // window slots per chunk
-  int ns;         // stages
-  int total;      // dynamic shared memory
+  int kcb;          // window slots per staged chunk
+  int hq, hkt, hvt, hs, hdr_bytes;  // per-warp header: q of the KV head's query heads, K_t, V_t, S
+  int chunk_bytes;  // a staged window chunk: keys, then values
+  int warp_bytes;   // per warp: two headers and two chunks
+  int near_warps;   // warps of a near-field CTA
+  int near_rows;    // sequences of a near-field CTA
+  int near_smem;    // its dynamic shared memory
+  int pool_smem;    // dynamic shared memory of the pool kernel
 };
 
 struct DecodeParams {
@@ -169,9 +160,9 @@ cudaError_t launch_decode(const DecodeParams& p, int in_dtype, int head_dim, cud
 cudaError_t launch_decode_tile(const DecodeParams& p, int in_dtype, int head_dim, cudaStream_t s);
 cudaError_t decode_tile_prepare(int device);
 // Plan of the batch-tiled decode within `limit` bytes of shared memory;
-// false if none fits.
-bool plan_decode_tile(int HPC, int head_dim, int esz, int G, int K, size_t limit, TilePlan* out);
-int decode_tile_max_active_clusters(int cs, size_t smem, int in_dtype, int head_dim);
+// false if none fits or the configuration is outside it (more than
+// kDecodeTileHeads query heads per KV head, hidden not a multiple of 64).
+bool plan_decode_tile(int H, int head_dim, int esz, int G, int K, size_t limit, TilePlan* out);
 cudaError_t launch_prefill(const PrefillParams& p, int in_dtype, int head_dim, cudaStream_t s);
 // Near-field plan for head_dim D, input element size esz and window K within
 // `limit` bytes of shared memory, on the tensor cores if tc (bf16, K <= 16);
