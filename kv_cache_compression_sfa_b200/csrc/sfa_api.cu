@@ -516,8 +516,9 @@ int sfa_decode_step_ex(const sfa_handle* h, int layer_begin, int layer_count, co
   p.tp = h->tile_plan;
   p.inputs_early = h->inputs_early ? 1 : 0;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // Batch-tiled decode from kDecodeTileMinSeqs sequences per call.
-  const bool tile = h->tile_ok &&
+  // Batch-tiled decode from kDecodeTileMinSeqs sequences per call (its
+  // tensor copies address input rows with 32-bit coordinates).
+  const bool tile = h->tile_ok && static_cast<long long>(layer_count) * n_seq <= 0x7fffffffLL &&
                     (h->tile_mode == 1 || (h->tile_mode < 0 && n_seq >= kDecodeTileMinSeqs));
   if (tile) return cuda_status(launch_decode_tile(p, c->in_dtype, c->head_dim, s));
   return cuda_status(launch_decode(p, c->in_dtype, c->head_dim, s));

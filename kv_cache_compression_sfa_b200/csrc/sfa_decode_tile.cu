@@ -56,11 +56,13 @@ constexpr int kPbFloats = HB * KCB + 2 * HB;  // per warp: P, corrections, denom
 constexpr int kNearRows = 16;           // sequences per near-field CTA
 static_assert(HB <= 8 && KCB == 16, "near-field lane mapping: 2 x 16 lanes, 4 heads each");
 
-// Tensor maps of the state's window rings (keys, values) for one call:
+// Tensor maps of one call: the state's window rings (keys, values) as
 // (head dim, KV head, slot, stream) views with boxes of one KV head x kcb
-// slots.
+// slots; for bf16 inputs also q as (head dim, query head, input row) with
+// boxes of one KV head's query heads, both in 64-dim halves with 128-byte
+// swizzling.
 struct WinMaps {
-  CUtensorMap k, v;
+  CUtensorMap k, v, q;
 };
 
 __host__ __device__ inline int a128(long long x) { return static_cast<int>((x + 127) & ~127LL); }
@@ -341,37 +343,369 @@ decode_near_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
   }
 }
 
+// ---------------------------------------------------- near field, bf16 MMAs
+
+// Warp-level bf16 matrix ops: ldmatrix (four 8 x 8 b16 matrices, optionally
+// transposed) and mma.sync m16n8k16 with fp32 accumulation.
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo_col, float hi_col) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo_col, hi_col);  // .x = first (lower) column
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// Shared-memory layout of the MMA near field, per warp (bytes): two headers
+// then two window chunks.  A header holds the q rows of the item's query
+// heads as (head dim / 64) swizzled 1 KB blocks of 8 rows x 128 bytes, then
+// K_t, V_t (plain) and S (fp32).  A chunk holds keys then values, each as
+// (head dim / 64) swizzled blocks of 16 slots x 128 bytes.  Tensor copies
+// with 128-byte swizzling put the 16-byte group j of row r at group
+// j ^ (r % 8); every block starts on a 1 KB boundary.
+template <int D>
+struct MmaNear {
+  static constexpr int NH = D / 64;              // 64-dim halves of a head row
+  static constexpr int qblk = 1024;              // 8 rows x 128 B
+  static constexpr int hq = 0;
+  static constexpr int hkt = NH * qblk;
+  static constexpr int hvt = hkt + D * 2;
+  static constexpr int hs = hvt + D * 2;
+  static constexpr int hdr = ((hs + 4 * D + 1023) / 1024) * 1024;
+  static constexpr int kblk = KCB * 128;         // 16 rows x 128 B
+  static constexpr int chunk = 2 * NH * kblk;    // keys, then values
+  static constexpr int warp = 2 * hdr + 2 * chunk;
+};
+
+template <int D>
+__global__ void __launch_bounds__(NTN, 1)
+decode_near_mma_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ WinMaps maps) {
+  using L = MmaNear<D>;
+  constexpr int NT16 = D / 8;  // n-tiles of 8 head dims
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int K = p.K, G = p.G, nkv = p.nkv;
+  const int blocks_per_layer = (p.n_seq + kNearRows - 1) / kNearRows;
+  const int li = static_cast<int>(blockIdx.x) / blocks_per_layer;
+  const int rb = static_cast<int>(blockIdx.x) % blocks_per_layer;
+  const int l = p.l0 + li;
+  const int kcb = p.tp.kcb;
+  const int nck = (K + kcb - 1) / kcb;
+
+  extern __shared__ __align__(128) unsigned char smb_mma[];
+  // 1 KB aligned base (the plan leaves 1 KB of slack) for the swizzled blocks
+  unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smb_mma) + 1023) &
+                                                       ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm) + warp * 4;  // hdr full [2], chunk full [2]
+  unsigned char* wbase = sm + 1024 + warp * L::warp;
+  auto hdr = [&](int i) { return wbase + i * L::hdr; };
+  auto chk = [&](int i) { return wbase + 2 * L::hdr + i * L::chunk; };
+  __shared__ long long s_st[kNearRows], s_pos[kNearRows];
+
+  if (lane == 0) {
+    for (int i = 0; i < 4; ++i) mbar_init(bars + i, 1);
+    mbar_fence_init();
+  }
+  if (kcb < KCB) {  // slots past kcb are never copied: keep them finite (zero)
+    for (int b = 0; b < 2; ++b)
+      for (int i = lane; i < 2 * L::NH * (KCB - kcb) * 8; i += 32) {
+        const int blk = i / ((KCB - kcb) * 8), rem = i % ((KCB - kcb) * 8);
+        reinterpret_cast<uint4*>(chk(b) + blk * L::kblk + kcb * 128)[rem] = make_uint4(0u, 0u, 0u, 0u);
+      }
+  }
+  pdl_trigger();
+  pdl_wait();  // state and inputs may be written by the previous kernel
+  if (tid < kNearRows) {
+    const int bi = rb * kNearRows + tid;
+    long long st = -1, ps = 0;
+    if (bi < p.n_seq) {
+      const int b = p.seq_ids ? __ldcg(p.seq_ids + bi) : bi;
+      if (b >= 0 && b < p.B) {
+        st = static_cast<long long>(l) * p.B + b;
+        ps = __ldcg(reinterpret_cast<const long long*>(p.state + kHeaderBytes + st * p.so.stride + p.so.pos));
+      } else {
+        latch_error(p.err, SFA_ERR_INVALID_ARG);
+      }
+    }
+    s_st[tid] = st;
+    s_pos[tid] = ps;
+  }
+  __syncthreads();
+  {
+    const uint4 h0v = __ldcg(reinterpret_cast<const uint4*>(p.state));
+    const uint4 h1v = __ldcg(reinterpret_cast<const uint4*>(p.state + 16));
+    StateHeader hd;
+    reinterpret_cast<uint4*>(&hd)[0] = h0v;
+    reinterpret_cast<uint4*>(&hd)[1] = h1v;
+    if (!(hd.magic == kMagic && hd.cfg_hash == p.cfg_hash && hd.batch == p.B && hd.n_layers == p.L)) {
+      if (tid == 0 && blockIdx.x == 0) latch_error(p.err, SFA_ERR_STATE_MISMATCH);
+      return;
+    }
+  }
+
+  const int n_items = kNearRows * nkv;
+  const long long in_row0 = static_cast<long long>(li) * p.n_seq + static_cast<long long>(rb) * kNearRows;
+  // Copies of one unit into chunk buffer b (header buffer hb with piece 0);
+  // lane 0.  Absent sequences: plain arrivals, so phases stay in step.
+  auto issue = [&](int it, int piece, int b, int hb) {
+    const int r = it / nkv, g = it - r * nkv;
+    const long long st = s_st[r];
+    if (st < 0) {
+      if (piece == 0) mbar_arrive(bars + hb);
+      mbar_arrive(bars + 2 + b);
+      return;
+    }
+    fence_proxy_async_smem();  // this warp's accesses of the buffers came first
+    if (piece == 0) {
+      uint64_t* hf = bars + hb;
+      const long long io = in_row0 + r;
+      unsigned char* h = hdr(hb);
+      mbar_arrive_expect_tx(hf, static_cast<unsigned>((G + 2) * D * 2 + 4 * D));
+#pragma unroll
+      for (int hh = 0; hh < L::NH; ++hh)
+        tma_load_3d(h + L::hq + hh * L::qblk, &maps.q, 64 * hh, g * G, static_cast<int>(io), hf);
+      bulk_g2s(h + L::hkt, static_cast<const __nv_bfloat16*>(p.k) + (io * nkv + g) * D, D * 2, hf);
+      bulk_g2s(h + L::hvt, static_cast<const __nv_bfloat16*>(p.v) + (io * nkv + g) * D, D * 2, hf);
+      bulk_g2s(h + L::hs, p.state + kHeaderBytes + st * p.so.stride + p.so.far + static_cast<long long>(g) * D * 4,
+               D * 4, hf);
+    }
+    uint64_t* cf = bars + 2 + b;
+    unsigned char* c = chk(b);
+    mbar_arrive_expect_tx(cf, static_cast<unsigned>(2 * kcb * D * 2));
+#pragma unroll
+    for (int hh = 0; hh < L::NH; ++hh) {
+      tma_load_4d(c + hh * L::kblk, &maps.k, 64 * hh, g, piece * kcb, static_cast<int>(st), cf);
+      tma_load_4d(c + (L::NH + hh) * L::kblk, &maps.v, 64 * hh, g, piece * kcb, static_cast<int>(st), cf);
+    }
+  };
+
+  const int g8 = lane >> 2, tig = lane & 3;  // MMA fragment row / column pair
+  const int mi = lane >> 3, rr = lane & 7;   // ldmatrix: matrix and row this lane addresses
+  bool ok = true;
+  int unit = 0;
+  int k_item = 0;
+  if (lane == 0 && warp < n_items) issue(warp, 0, 0, 0);
+  for (int it = warp; it < n_items; it += NWN, ++k_item) {
+    const int r = it / nkv, g = it - r * nkv;
+    const long long st = s_st[r];
+    const long long t = s_pos[r];
+    const int es = static_cast<int>(t % K);  // slot of token t: holds the evicted key t-k
+    const bool full_win = t >= K - 1;
+    const int hb = k_item & 1;
+    unsigned char* h = hdr(hb);
+    const uint32_t qb = smem_u32(h + L::hq);
+    const __nv_bfloat16* ktr = reinterpret_cast<const __nv_bfloat16*>(h + L::hkt);
+    const __nv_bfloat16* vtr = reinterpret_cast<const __nv_bfloat16*>(h + L::hvt);
+    const float* s_old = reinterpret_cast<const float*>(h + L::hs);
+    float o[NT16][4], kev[NT16][2];
+#pragma unroll
+    for (int n = 0; n < NT16; ++n) {
+      o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+      kev[n][0] = kev[n][1] = 0.f;
+    }
+    float m_run = -INFINITY, l_run = 0.f;  // row g8 of the item (query head g8)
+    if (!mbar_wait_bounded(bars + hb, static_cast<unsigned>((k_item >> 1) & 1), kMbarPollLimit, p.err)) ok = false;
+    for (int piece = 0; piece < nck; ++piece) {
+      const int b = unit & 1;
+      if (lane == 0) {
+        if (piece + 1 < nck) issue(it, piece + 1, b ^ 1, hb);
+        else if (it + NWN < n_items) issue(it + NWN, 0, b ^ 1, hb ^ 1);
+      }
+      if (!mbar_wait_bounded(bars + 2 + b, static_cast<unsigned>((unit >> 1) & 1), kMbarPollLimit, p.err))
+        ok = false;
+      ++unit;
+      if (st < 0) continue;
+      unsigned char* c = chk(b);
+      const uint32_t kb = smem_u32(c), vb = smem_u32(c + L::NH * L::kblk);
+      const int base = piece * kcb;
+      if (piece == es / kcb) {
+        // slot es holds the key token t evicts: keep it for S, then put
+        // token t's own key and value in its place
+        const int er = es - base;
+#pragma unroll
+        for (int n = 0; n < NT16; ++n) {
+          const __nv_bfloat162 e2 = *reinterpret_cast<const __nv_bfloat162*>(
+              c + (n >> 3) * L::kblk + er * 128 + (((n & 7) ^ (er & 7)) << 4) + 4 * tig);
+          const float2 f = __bfloat1622float2(e2);
+          kev[n][0] = f.x;
+          kev[n][1] = f.y;
+        }
+        __syncwarp();
+        if (lane < 2 * NT16) {  // 16-byte groups of K_t (lanes < NT16) and V_t
+          const int grp = lane % NT16;
+          const bool is_v = lane >= NT16;
+          const uint4 src = *reinterpret_cast<const uint4*>((is_v ? vtr : ktr) + 8 * grp);
+          *reinterpret_cast<uint4*>(c + ((is_v ? L::NH : 0) + (grp >> 3)) * L::kblk + er * 128 +
+                                    (((grp & 7) ^ (er & 7)) << 4)) = src;
+        }
+        __syncwarp();
+      }
+      // S[16 heads x 16 slots] = q . K^T; heads >= G read head 0 (discarded)
+      float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks) {
+        uint32_t a[4], bk[4];
+        int qrow = rr + 8 * (mi & 1);
+        if (qrow >= G) qrow = 0;
+        const int qg = 2 * ks + (mi >> 1);
+        ldsm_x4(qb + (qg >> 3) * L::qblk + qrow * 128 + (((qg & 7) ^ (qrow & 7)) << 4), a);
+        const int krow = rr + 8 * (mi >> 1);
+        const int kg = 2 * ks + (mi & 1);
+        ldsm_x4(kb + (kg >> 3) * L::kblk + krow * 128 + (((kg & 7) ^ (krow & 7)) << 4), bk);
+        mma16816(s0, a, bk[0], bk[1]);
+        mma16816(s1, a, bk[2], bk[3]);
+      }
+      // online softmax for row g8 over the chunk's valid slots
+      float v[4] = {s0[0], s0[1], s1[0], s1[1]};
+      float cm = -INFINITY;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int kk = (e >> 1) * 8 + 2 * tig + (e & 1);
+        const int s = base + kk;
+        const bool valid = kk < kcb && s < K && (full_win || s <= t);
+        v[e] = valid ? v[e] * p.score_scale : -INFINITY;
+        cm = fmaxf(cm, v[e]);
+      }
+      cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 1));
+      cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 2));
+      const float mn = fmaxf(m_run, cm);
+      const float corr = mn == -INFINITY ? 1.f : expf(m_run - mn);
+      float pr[4], ps = 0.f;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        pr[e] = v[e] == -INFINITY ? 0.f : expf(v[e] - mn);
+        ps += pr[e];
+      }
+      ps += __shfl_xor_sync(0xffffffffu, ps, 1);
+      ps += __shfl_xor_sync(0xffffffffu, ps, 2);
+      l_run = fmaf(l_run, corr, ps);
+      m_run = mn;
+      if (piece > 0) {
+#pragma unroll
+        for (int n = 0; n < NT16; ++n) {
+          o[n][0] *= corr;
+          o[n][1] *= corr;
+        }
+      }
+      // P as split bf16 A operands (rows 8..15 zero): P = P_hi + P_lo
+      uint32_t ah[4], al[4];
+      {
+        float hi[4], lo[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          hi[e] = __bfloat162float(__float2bfloat16_rn(pr[e]));
+          lo[e] = pr[e] - hi[e];
+        }
+        ah[0] = pack_bf16(hi[0], hi[1]);
+        ah[1] = 0u;
+        ah[2] = pack_bf16(hi[2], hi[3]);
+        ah[3] = 0u;
+        al[0] = pack_bf16(lo[0], lo[1]);
+        al[1] = 0u;
+        al[2] = pack_bf16(lo[2], lo[3]);
+        al[3] = 0u;
+      }
+      // O[16 x D] += P . V over the chunk's 16 slots
+#pragma unroll
+      for (int n2 = 0; n2 < NT16 / 2; ++n2) {
+        uint32_t bv[4];
+        const int vrow = rr + 8 * (mi & 1);
+        const int vg = 2 * n2 + (mi >> 1);
+        ldsm_x4_t(vb + (vg >> 3) * L::kblk + vrow * 128 + (((vg & 7) ^ (vrow & 7)) << 4), bv);
+        mma16816(o[2 * n2], ah, bv[0], bv[1]);
+        mma16816(o[2 * n2], al, bv[0], bv[1]);
+        mma16816(o[2 * n2 + 1], ah, bv[2], bv[3]);
+        mma16816(o[2 * n2 + 1], al, bv[2], bv[3]);
+      }
+      __syncwarp();
+    }
+    if (st < 0) continue;
+    // x = O_near + alpha_far * S_t for the item's heads; then S and slot es
+    const long long io = in_row0 + r;
+    const float inv = 1.f / l_run;
+    float* far = reinterpret_cast<float*>(p.state + kHeaderBytes + st * p.so.stride + p.so.far) + g * D;
+    float* xrow = p.out + io * p.H + (static_cast<long long>(g) * G + g8) * D;
+#pragma unroll
+    for (int n = 0; n < NT16; ++n) {
+      const int d = 8 * n + 2 * tig;
+      float sn0 = s_old[d], sn1 = s_old[d + 1];
+      if (t >= K) {
+        sn0 = ewma(p.gamma_far, sn0, kev[n][0]);
+        sn1 = ewma(p.gamma_far, sn1, kev[n][1]);
+      }
+      if (g8 < G)
+        *reinterpret_cast<float2*>(xrow + d) =
+            make_float2(fmaf(p.alpha_far, sn0, o[n][0] * inv), fmaf(p.alpha_far, sn1, o[n][1] * inv));
+      if (g8 == 0 && ok) *reinterpret_cast<float2*>(far + d) = make_float2(sn0, sn1);
+    }
+    if (ok && lane < 2 * NT16) {
+      const int grp = lane % NT16;
+      const bool is_v = lane >= NT16;
+      const size_t wo = (static_cast<size_t>(es) * nkv + g) * D + 8 * grp;
+      unsigned char* blk = p.state + kHeaderBytes + st * p.so.stride;
+      __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(blk + (is_v ? p.so.win_v : p.so.win_k)) + wo;
+      *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>((is_v ? vtr : ktr) + 8 * grp);
+    }
+    __syncwarp();  // the header is reused two items later
+  }
+}
+
 // ---------------------------------------------------------------- pool kernel
 
-constexpr int NTP = 256;
-constexpr int NWP = NTP / 32;
+constexpr int NTC = 256;                // pool kernel: compute threads (8 warps)
+constexpr int NWC = NTC / 32;
+constexpr int NTP = NTC + 32;           // plus the MMA warp
 constexpr int TR = 16;                  // sequences per pool CTA (rows of the MMAs' M = 64)
 constexpr int kSlotStages = 3;
+constexpr int kABufs = 2;               // split x blocks
+constexpr int kSemBufs = 2;             // sem accumulators in tensor memory and their staging
 constexpr int kScStride = kSlots + 1;
 constexpr int kSemStride = kBlk + 4;
 constexpr int kTmemCols = 256;          // scores (64) + two 64-column sem buffers
-static_assert(TR * 16 == NTP, "pool kernel: 16 threads per row, 4 columns each");
+static_assert(TR * 16 == NTC, "pool kernel: 16 threads per row, 4 columns each");
 
 // Pool CTA shared memory (byte offsets).
 struct PoolTilePlan {
-  static constexpr int bars = 0;                                  // mbarriers, tmem address
-  static constexpr int a = 256;                                   // [2][hi, lo] x blocks
-  static constexpr int w = a + 2 * 2 * kBlkBytes;                 // [hi, lo] weight block
-  static constexpr int sl = w + 2 * kBlkBytes;                    // [3][hi, lo] slot blocks
-  static constexpr int sc = sl + kSlotStages * 2 * kBlkBytes;     // [16][65] scores, then
-  static constexpr int sem = sc;                                  // [16][68] sem chunk
-  static constexpr int total = sc + TR * kSemStride * 4;
+  static constexpr int bars = 0;                                     // mbarriers, tmem address
+  static constexpr int a = 512;                                      // [2][hi, lo] x blocks
+  static constexpr int w = a + kABufs * 2 * kBlkBytes;               // [hi, lo] weight block
+  static constexpr int sl = w + 2 * kBlkBytes;                       // [3][hi, lo] slot blocks
+  static constexpr int sem = sl + kSlotStages * 2 * kBlkBytes;       // [2][16][68] sem chunks
+  static constexpr int sc = sem + kSemBufs * TR * kSemStride * 4;    // [16][65] scores
+  static constexpr int total = sc + TR * kScStride * 4;
 };
-static_assert(TR * kScStride <= TR * kSemStride, "scores fit the sem staging");
-// barrier slots
-constexpr int kPbSlFull = 0;                         // [3] slot block landed
-constexpr int kPbSlEmpty = kPbSlFull + kSlotStages;  // [3] MMAs done with the slot block
-constexpr int kPbAEmpty = kPbSlEmpty + kSlotStages;  // [2] MMAs done with the x block
-constexpr int kPbSem = kPbAEmpty + 2;                // [2] sem MMAs done
-constexpr int kPbScores = kPbSem + 2;                // all score MMAs done
-constexpr int kPbCount = kPbScores + 1;
+// barrier slots (arrival counts in brackets)
+constexpr int kPbSlFull = 0;                           // [3] slot block landed (1 + bytes)
+constexpr int kPbSlEmpty = kPbSlFull + kSlotStages;    // [3] MMAs done with a slot block (commit)
+constexpr int kPbAFull = kPbSlEmpty + kSlotStages;     // [2] x block written (8 warps)
+constexpr int kPbAEmpty = kPbAFull + kABufs;           // [2] MMAs done with an x block (commit)
+constexpr int kPbScores = kPbAEmpty + kABufs;          // all score MMAs done (commit)
+constexpr int kPbWFull = kPbScores + 1;                // weight block written (8 warps)
+constexpr int kPbSemFull = kPbWFull + 1;               // [2] sem accumulator ready (commit)
+constexpr int kPbSemEmpty = kPbSemFull + kSemBufs;     // [2] sem accumulator read (2 warps)
+constexpr int kPbStFull = kPbSemEmpty + kSemBufs;      // [2] sem chunk staged (2 warps)
+constexpr int kPbStEmpty = kPbStFull + kSemBufs;       // [2] staged chunk used (8 warps)
+constexpr int kPbCount = kPbStEmpty + kSemBufs;
 static_assert(kPbCount * 8 + 4 <= PoolTilePlan::a, "barriers fit");
 
+// Pass 1 and pass 2 run as a pipeline without CTA-wide barriers: warp 8
+// (one lane) loads the slot blocks and issues every MMA; warps 0-7 split x
+// into the MMA blocks, then run the epilogue; warps 0 and 4, which can read
+// tensor-memory lanes 0-15 (rows 0-15 of an M = 64 accumulator), stage each
+// sem chunk in shared memory for the others.  mbarriers carry every
+// hand-off.
 __global__ void __launch_bounds__(NTP, 2) decode_pool_kernel(const __grid_constant__ DecodeParams p) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int tiles_per_layer = (p.n_seq + TR - 1) / TR;
@@ -387,49 +721,46 @@ __global__ void __launch_bounds__(NTP, 2) decode_pool_kernel(const __grid_consta
   unsigned char* wblk = sm + PoolTilePlan::w;
   unsigned char* slb = sm + PoolTilePlan::sl;
   float* sc = reinterpret_cast<float*>(sm + PoolTilePlan::sc);
-  float* semc = reinterpret_cast<float*>(sm + PoolTilePlan::sem);
+  float* semst = reinterpret_cast<float*>(sm + PoolTilePlan::sem);
   __shared__ long long s_st[TR], s_pos[TR];
-  __shared__ float s_ssq[TR];
+  __shared__ float s_ssq[TR][2];
   __shared__ int s_ok;
 
   const unsigned char* img_l = p.slot_img + static_cast<size_t>(l) * nch * 2 * kBlkBytes;
   // Slot block loads q = 0 .. 2*nch-1 (pass 1, then pass 2) through the
   // three stages: load q is block q % nch in stage q % 3.
-  auto issue_slot = [&](int q) {  // tid 0
+  auto issue_slot = [&](int q) {  // the MMA lane
     const int st = q % kSlotStages;
     mbar_arrive_expect_tx(bars + kPbSlFull + st, 2u * kBlkBytes);
     bulk_g2s(slb + st * 2 * kBlkBytes, img_l + static_cast<size_t>(q % nch) * 2 * kBlkBytes, 2u * kBlkBytes,
              bars + kPbSlFull + st);
   };
-  bool ok_slot = true;
-  // After the MMAs of load q are issued: the stage of load q-1 (its MMAs
-  // committed one chunk earlier) takes load q+2.  tid 0.
-  auto refill_slot = [&](int q) {
-    if (q < 1 || q + kSlotStages - 1 >= 2 * nch) return;
-    const int st = (q - 1) % kSlotStages;
-    if (!mbar_wait_bounded(bars + kPbSlEmpty + st, static_cast<unsigned>(((q - 1) / kSlotStages) & 1), kMbarPollLimit,
-                           p.err))
-      ok_slot = false;
-    issue_slot(q + kSlotStages - 1);
-  };
   if (tid == 0) {
-    for (int i = 0; i < kPbCount; ++i) mbar_init(bars + i, 1);
+    for (int i = 0; i < kPbCount; ++i) {
+      const bool by_warps = i == kPbWFull || (i >= kPbAFull && i < kPbAFull + kABufs) ||
+                            (i >= kPbStEmpty && i < kPbStEmpty + kSemBufs);
+      const bool by_readers = (i >= kPbSemEmpty && i < kPbSemEmpty + kSemBufs) ||
+                              (i >= kPbStFull && i < kPbStFull + kSemBufs);
+      mbar_init(bars + i, by_warps ? NWC : by_readers ? 2 : 1);
+    }
     mbar_fence_init();
-    // the slot blocks are constant since sfa_init: the first loads go out
-    // before the wait for the previous kernel
-    for (int q = 0; q < kSlotStages && q < 2 * nch; ++q) issue_slot(q);
   }
   if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);  // at most two CTAs per SM: never waits
   // rows 16..63 of the x and weight blocks stay zero
-  for (int i = tid; i < (2 * 2 + 2) * kBlkBytes / 16; i += NTP) {
+  for (int i = tid; i < (kABufs * 2 + 2) * kBlkBytes / 16; i += NTP) {
     const int bi = i / (kBlkBytes / 16), rem = i % (kBlkBytes / 16);
-    unsigned char* base = (bi < 4 ? ablk + bi * kBlkBytes : wblk + (bi - 4) * kBlkBytes);
+    unsigned char* base = (bi < kABufs * 2 ? ablk + bi * kBlkBytes : wblk + (bi - kABufs * 2) * kBlkBytes);
     reinterpret_cast<uint4*>(base)[rem] = make_uint4(0u, 0u, 0u, 0u);
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if (tid == NTC) {
+    // the slot blocks are constant since sfa_init: the first loads go out
+    // before the wait for the previous kernel
+    for (int q = 0; q < kSlotStages && q < 2 * nch; ++q) issue_slot(q);
+  }
   pdl_trigger();
   pdl_wait();  // x from decode_near_kernel; the state
 
@@ -456,33 +787,98 @@ __global__ void __launch_bounds__(NTP, 2) decode_pool_kernel(const __grid_consta
   }
   __syncthreads();
   bool ok = s_ok != 0;  // a mismatch was latched by decode_near_kernel
-
-  // Thread tid: row r = tid / 16, columns c4 .. c4+3 of every chunk.
-  const int r = tid >> 4, c4 = (tid & 15) * 4;
-  const long long st = s_st[r];
-  const long long io = static_cast<long long>(li) * p.n_seq + static_cast<long long>(tb) * TR + r;
-  const bool live = st >= 0 && ok;
-  const float* xrow = p.out + (live ? io : 0) * p.H + c4;
-  auto load_x = [&](int c) -> float4 {
-    return live ? __ldcg(reinterpret_cast<const float4*>(xrow + c * kBlk)) : make_float4(0.f, 0.f, 0.f, 0.f);
-  };
-
-  // ---- pass 1: scores[16 x 64] = x . slot^T and |x|^2 ----------------------
   const uint32_t idesc_s = umma_idesc_bf16(kBlk, kSlots, false);
-  float4 xn0 = load_x(0);  // chunks c and c+1 in flight
-  float4 xn1 = nch > 1 ? load_x(1) : make_float4(0.f, 0.f, 0.f, 0.f);
-  float sq = 0.f;
-  for (int c = 0; c < nch; ++c) {
-    const int b = c & 1;
-    const float4 v = xn0;
-    xn0 = xn1;
-    if (c + 2 < nch) xn1 = load_x(c + 2);
-    sq = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, sq))));
-    // x block b was read by the MMAs of chunk c-2
-    if (c >= 2 && !mbar_wait_bounded(bars + kPbAEmpty + b, static_cast<unsigned>(((c - 2) >> 1) & 1), kMbarPollLimit, p.err))
-      ok = false;
-    unsigned char* xhi = ablk + b * 2 * kBlkBytes;
-    {
+  const uint32_t idesc_c = umma_idesc_bf16(kBlk, kBlk, true);
+
+  if (warp == NWC) {
+    // ---- MMA warp: slot loads and every MMA -------------------------------
+    if (lane == 0) {
+      // After the MMAs of load q: the stage of load q-1 (its MMAs committed
+      // one chunk earlier) takes load q+2.
+      auto refill_slot = [&](int q) {
+        if (q < 1 || q + kSlotStages - 1 >= 2 * nch) return;
+        const int st = (q - 1) % kSlotStages;
+        if (!mbar_wait_bounded(bars + kPbSlEmpty + st, static_cast<unsigned>(((q - 1) / kSlotStages) & 1),
+                               kMbarPollLimit, p.err))
+          ok = false;
+        issue_slot(q + kSlotStages - 1);
+      };
+      // pass 1: scores[16 x 64] += x_c . slot_c^T
+      for (int c = 0; c < nch; ++c) {
+        const int stg = c % kSlotStages, b = c % kABufs;
+        if (!mbar_wait_bounded(bars + kPbSlFull + stg, static_cast<unsigned>((c / kSlotStages) & 1), kMbarPollLimit, p.err))
+          ok = false;
+        if (!mbar_wait_bounded(bars + kPbAFull + b, static_cast<unsigned>((c / kABufs) & 1), kMbarPollLimit, p.err))
+          ok = false;
+        tc_fence_after();
+        const unsigned char* xhi = ablk + b * 2 * kBlkBytes;
+        const unsigned char* shi = slb + stg * 2 * kBlkBytes;
+#pragma unroll
+        for (int k = 0; k < kBlk / 16; ++k) {
+          const uint64_t ah = umma_desc(xhi + k * 2048, 1024, 128), al = umma_desc(xhi + kBlkBytes + k * 2048, 1024, 128);
+          const uint64_t bh = umma_desc(shi + k * 2048, 1024, 128), bl = umma_desc(shi + kBlkBytes + k * 2048, 1024, 128);
+          umma_bf16(tmem, ah, bh, idesc_s, c > 0 || k > 0);
+          umma_bf16(tmem, ah, bl, idesc_s, true);
+          umma_bf16(tmem, al, bh, idesc_s, true);
+        }
+        umma_commit(bars + kPbAEmpty + b);
+        umma_commit(bars + kPbSlEmpty + stg);
+        refill_slot(c);
+      }
+      umma_commit(bars + kPbScores);
+      // pass 2: sem chunk c = w . slot_c into accumulator c % 2
+      if (!mbar_wait_bounded(bars + kPbWFull, 0, kMbarPollLimit, p.err)) ok = false;
+      for (int c = 0; c < nch; ++c) {
+        const int q = nch + c, stg = q % kSlotStages, b = c % kSemBufs;
+        if (!mbar_wait_bounded(bars + kPbSlFull + stg, static_cast<unsigned>((q / kSlotStages) & 1), kMbarPollLimit, p.err))
+          ok = false;
+        if (c >= kSemBufs &&
+            !mbar_wait_bounded(bars + kPbSemEmpty + b, static_cast<unsigned>(((c / kSemBufs) - 1) & 1), kMbarPollLimit, p.err))
+          ok = false;
+        tc_fence_after();
+        const uint32_t dst = tmem + kSlots + b * kBlk;
+        const unsigned char* shi = slb + stg * 2 * kBlkBytes;
+#pragma unroll
+        for (int k = 0; k < kSlots / 16; ++k) {
+          const uint64_t ah = umma_desc(wblk + k * 2048, 1024, 128), al = umma_desc(wblk + kBlkBytes + k * 2048, 1024, 128);
+          const uint64_t bh = umma_desc(shi + k * 256, 128, 1024), bl = umma_desc(shi + kBlkBytes + k * 256, 128, 1024);
+          umma_bf16(dst, ah, bh, idesc_c, k > 0);
+          umma_bf16(dst, ah, bl, idesc_c, true);
+          umma_bf16(dst, al, bh, idesc_c, true);
+        }
+        umma_commit(bars + kPbSemFull + b);
+        umma_commit(bars + kPbSlEmpty + stg);
+        refill_slot(q);
+      }
+      // the last slot loads have landed and been read: nothing in flight
+      if (!ok) latch_error(p.err, SFA_ERR_DEVICE_TIMEOUT);
+    }
+    __syncwarp();
+  } else {
+    // ---- compute warps --------------------------------------------------
+    // Thread tid: row r = tid / 16, columns c4 .. c4+3 of every chunk.
+    const int r = tid >> 4, c4 = (tid & 15) * 4;
+    const long long st = s_st[r];
+    const long long io = static_cast<long long>(li) * p.n_seq + static_cast<long long>(tb) * TR + r;
+    const bool live = st >= 0 && ok;
+    const float* xrow = p.out + (live ? io : 0) * p.H + c4;
+    auto load_x = [&](int c) -> float4 {
+      return (live && c < nch) ? __ldcg(reinterpret_cast<const float4*>(xrow + c * kBlk))
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+    };
+    // pass 1: split x chunk c into x block c % 2; |x|^2
+    float4 xn0 = load_x(0), xn1 = load_x(1);  // chunks c and c+1 in flight
+    float sq = 0.f;
+    for (int c = 0; c < nch; ++c) {
+      const int b = c % kABufs;
+      const float4 v = xn0;
+      xn0 = xn1;
+      xn1 = load_x(c + 2);
+      sq = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, sq))));
+      if (c >= kABufs &&
+          !mbar_wait_bounded(bars + kPbAEmpty + b, static_cast<unsigned>(((c / kABufs) - 1) & 1), kMbarPollLimit, p.err))
+        ok = false;
+      unsigned char* xhi = ablk + b * 2 * kBlkBytes;
       __nv_bfloat16 hh[4], ll[4];
       split_bf16(v.x, hh[0], ll[0]);
       split_bf16(v.y, hh[1], ll[1]);
@@ -491,170 +887,135 @@ __global__ void __launch_bounds__(NTP, 2) decode_pool_kernel(const __grid_consta
       const int off = blk_off(r, c4);
       *reinterpret_cast<uint2*>(xhi + off) = *reinterpret_cast<const uint2*>(hh);
       *reinterpret_cast<uint2*>(xhi + kBlkBytes + off) = *reinterpret_cast<const uint2*>(ll);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bars + kPbAFull + b);
     }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0) {
-      const int stg = c % kSlotStages;
-      if (!mbar_wait_bounded(bars + kPbSlFull + stg, static_cast<unsigned>((c / kSlotStages) & 1), kMbarPollLimit, p.err))
-        ok = false;
+    // |x|^2 per row: the 16 threads of a row (one half-warp) add their partials
+#pragma unroll
+    for (int off = 8; off > 0; off >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, off);
+    if ((tid & 15) == 0) s_ssq[r][0] = sq;
+    if ((warp & 3) == 0) {  // rows 0..15 sit in lanes 0..15 of the first lane quarter (M = 64)
+      if (!mbar_wait_bounded(bars + kPbScores, 0, kMbarPollLimit, p.err)) ok = false;
       tc_fence_after();
-      const unsigned char* shi = slb + stg * 2 * kBlkBytes;
-#pragma unroll
-      for (int k = 0; k < kBlk / 16; ++k) {
-        const uint64_t ah = umma_desc(xhi + k * 2048, 1024, 128), al = umma_desc(xhi + kBlkBytes + k * 2048, 1024, 128);
-        const uint64_t bh = umma_desc(shi + k * 2048, 1024, 128), bl = umma_desc(shi + kBlkBytes + k * 2048, 1024, 128);
-        umma_bf16(tmem, ah, bh, idesc_s, c > 0 || k > 0);
-        umma_bf16(tmem, ah, bl, idesc_s, true);
-        umma_bf16(tmem, al, bh, idesc_s, true);
-      }
-      umma_commit(bars + kPbAEmpty + b);
-      umma_commit(bars + kPbSlEmpty + stg);
-      refill_slot(c);
-    }
-  }
-  if (tid == 0) umma_commit(bars + kPbScores);
-  // |x|^2 per row: the 16 threads of a row (one half-warp) add their partials
-#pragma unroll
-  for (int off = 8; off > 0; off >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, off);
-  if ((tid & 15) == 0) s_ssq[r] = sq;
-  if (!mbar_wait_bounded(bars + kPbScores, 0, kMbarPollLimit, p.err)) ok = false;
-  tc_fence_after();
-  if ((warp & 3) == 0) {  // rows 0..15 sit in lanes 0..15 of the first lane quarter (M = 64)
-    const int colh = (warp >> 2) * 32;
-    float v[32];
-    tmem_ld32(tmem + colh, v);
-    if (lane < TR) {
-#pragma unroll
-      for (int jj = 0; jj < 32; ++jj) sc[lane * kScStride + colh + jj] = v[jj];
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-
-  // ---- softmax(cos/T) per row [P3 §2.1 channel 3]; weights as split bf16 ---
-  {
-    const float* nrm = p.slot_norm + static_cast<size_t>(l) * kSlots;
-    const float n0 = nrm[lane], n1 = nrm[lane + 32];
-    for (int rr = warp; rr < TR; rr += NWP) {
-      const float nx = fmaxf(sqrtf(s_ssq[rr]), kNormFloor);
-      const float c0 = sc[rr * kScStride + lane] / (nx * n0) * p.inv_temp;
-      const float c1 = sc[rr * kScStride + lane + 32] / (nx * n1) * p.inv_temp;
-      const float mx = warp_max_redux(fmaxf(c0, c1));
-      const float e0 = expf(c0 - mx), e1 = expf(c1 - mx);
-      const float inv = 1.f / warp_sum(e0 + e1);
-      __nv_bfloat16 h0, l0, h1, l1;
-      split_bf16(e0 * inv, h0, l0);
-      split_bf16(e1 * inv, h1, l1);
-      const int o0 = blk_off(rr, lane), o1 = blk_off(rr, lane + 32);
-      *reinterpret_cast<__nv_bfloat16*>(wblk + o0) = h0;
-      *reinterpret_cast<__nv_bfloat16*>(wblk + kBlkBytes + o0) = l0;
-      *reinterpret_cast<__nv_bfloat16*>(wblk + o1) = h1;
-      *reinterpret_cast<__nv_bfloat16*>(wblk + kBlkBytes + o1) = l1;
-    }
-  }
-  fence_proxy_async_smem();
-  tc_fence_before();
-  __syncthreads();
-
-  // ---- pass 2: sem chunk c [16 x 64] = w . slot_c on the tensor cores; ring,
-  // field, fusion, clip, output [P3 §2.1 channels 1-2, §2.2]
-  const uint32_t idesc_c = umma_idesc_bf16(kBlk, kBlk, true);
-  auto issue_sem = [&](int c) {  // tid 0: slot load nch + c
-    const int q = nch + c, stg = q % kSlotStages;
-    if (!mbar_wait_bounded(bars + kPbSlFull + stg, static_cast<unsigned>((q / kSlotStages) & 1), kMbarPollLimit, p.err))
-      ok = false;
-    tc_fence_after();
-    const uint32_t dst = tmem + kSlots + (c & 1) * kBlk;
-    const unsigned char* shi = slb + stg * 2 * kBlkBytes;
-#pragma unroll
-    for (int k = 0; k < kSlots / 16; ++k) {
-      const uint64_t ah = umma_desc(wblk + k * 2048, 1024, 128), al = umma_desc(wblk + kBlkBytes + k * 2048, 1024, 128);
-      const uint64_t bh = umma_desc(shi + k * 256, 128, 1024), bl = umma_desc(shi + kBlkBytes + k * 256, 128, 1024);
-      umma_bf16(dst, ah, bh, idesc_c, k > 0);
-      umma_bf16(dst, ah, bl, idesc_c, true);
-      umma_bf16(dst, al, bh, idesc_c, true);
-    }
-    umma_commit(bars + kPbSem + (c & 1));
-    umma_commit(bars + kPbSlEmpty + stg);
-    refill_slot(q);
-  };
-  if (tid == 0) {
-    issue_sem(0);
-    if (nch > 1) issue_sem(1);
-  }
-  const int slot_r = static_cast<int>(s_pos[r] & (kRing - 1));
-  unsigned char* blk = p.state + kHeaderBytes + (live ? st : 0) * p.so.stride;
-  float* ring_r = reinterpret_cast<float*>(blk + p.so.ring) + static_cast<size_t>(slot_r) * p.H + c4;
-  float* rsum_r = reinterpret_cast<float*>(blk + p.so.ring_sum) + c4;
-  float* fld_r = reinterpret_cast<float*>(blk + p.so.field) + c4;
-  float* out_r = p.out + (live ? io : 0) * p.H + c4;
-  // x and state of chunks c and c+1 in flight
-  struct Row4 {
-    float4 x, old, rs, fl;
-  };
-  auto load_row = [&](int c) -> Row4 {
-    Row4 v;
-    if (live && c < nch) {
-      v.x = __ldcg(reinterpret_cast<const float4*>(out_r + c * kBlk));
-      v.old = __ldcg(reinterpret_cast<const float4*>(ring_r + c * kBlk));
-      v.rs = __ldcg(reinterpret_cast<const float4*>(rsum_r + c * kBlk));
-      v.fl = __ldcg(reinterpret_cast<const float4*>(fld_r + c * kBlk));
-    } else {
-      v.x = v.old = v.rs = v.fl = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    return v;
-  };
-  Row4 rn0 = load_row(0), rn1 = load_row(1);
-  const float a_l = p.alpha_layer[l];
-  for (int c = 0; c < nch; ++c) {
-    const int b = c & 1;
-    if (!mbar_wait_bounded(bars + kPbSem + b, static_cast<unsigned>((c >> 1) & 1), kMbarPollLimit, p.err)) ok = false;
-    tc_fence_after();
-    if ((warp & 3) == 0) {
       const int colh = (warp >> 2) * 32;
       float v[32];
-      tmem_ld32(tmem + kSlots + b * kBlk + colh, v);
+      tmem_ld32(tmem + colh, v);
       if (lane < TR) {
-        float* dst = semc + lane * kSemStride + colh;
 #pragma unroll
-        for (int jj = 0; jj < 32; jj += 4)
-          *reinterpret_cast<float4*>(dst + jj) = make_float4(v[jj], v[jj + 1], v[jj + 2], v[jj + 3]);
+        for (int jj = 0; jj < 32; ++jj) sc[lane * kScStride + colh + jj] = v[jj];
       }
     }
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0 && c + 2 < nch) issue_sem(c + 2);  // its buffer was read just above
-    const float4 x = rn0.x, ro = rn0.old, rs = rn0.rs, fl = rn0.fl;
-    const float4 sv = *reinterpret_cast<const float4*>(semc + r * kSemStride + c4);
-    rn0 = rn1;
-    rn1 = load_row(c + 2);
-    if (live && ok) {
-      const float xa[4] = {x.x, x.y, x.z, x.w}, roa[4] = {ro.x, ro.y, ro.z, ro.w};
-      const float rsa[4] = {rs.x, rs.y, rs.z, rs.w}, fla[4] = {fl.x, fl.y, fl.z, fl.w};
-      const float sva[4] = {sv.x, sv.y, sv.z, sv.w};
-      float rv[4], fv[4], ov[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        rv[e] = (rsa[e] - roa[e]) + xa[e];        // ring sum after storing x_t
-        fv[e] = ewma(p.ema_gamma, fla[e], xa[e]);  // EMA field
-        float uu = rv[e] * (1.0f / kRing) + 0.5f * fv[e] + 0.5f * sva[e];
-        uu = fminf(fmaxf(uu, -p.clip_eps), p.clip_eps);
-        ov[e] = fmaf(a_l, uu, xa[e]);
+    // scores and |x|^2 of every row in shared memory (compute warps only)
+    asm volatile("bar.sync 1, %0;" ::"n"(NTC) : "memory");
+    // softmax(cos/T) per row [P3 §2.1 channel 3]; weights as split bf16
+    {
+      const float* nrm = p.slot_norm + static_cast<size_t>(l) * kSlots;
+      const float n0 = nrm[lane], n1 = nrm[lane + 32];
+      for (int rr = warp; rr < TR; rr += NWC) {
+        const float nx = fmaxf(sqrtf(s_ssq[rr][0]), kNormFloor);
+        const float c0 = sc[rr * kScStride + lane] / (nx * n0) * p.inv_temp;
+        const float c1 = sc[rr * kScStride + lane + 32] / (nx * n1) * p.inv_temp;
+        const float mx = warp_max_redux(fmaxf(c0, c1));
+        const float e0 = expf(c0 - mx), e1 = expf(c1 - mx);
+        const float inv = 1.f / warp_sum(e0 + e1);
+        __nv_bfloat16 h0, l0, h1, l1;
+        split_bf16(e0 * inv, h0, l0);
+        split_bf16(e1 * inv, h1, l1);
+        const int o0 = blk_off(rr, lane), o1 = blk_off(rr, lane + 32);
+        *reinterpret_cast<__nv_bfloat16*>(wblk + o0) = h0;
+        *reinterpret_cast<__nv_bfloat16*>(wblk + kBlkBytes + o0) = l0;
+        *reinterpret_cast<__nv_bfloat16*>(wblk + o1) = h1;
+        *reinterpret_cast<__nv_bfloat16*>(wblk + kBlkBytes + o1) = l1;
       }
-      *reinterpret_cast<float4*>(ring_r + c * kBlk) = x;
-      *reinterpret_cast<float4*>(rsum_r + c * kBlk) = make_float4(rv[0], rv[1], rv[2], rv[3]);
-      *reinterpret_cast<float4*>(fld_r + c * kBlk) = make_float4(fv[0], fv[1], fv[2], fv[3]);
-      *reinterpret_cast<float4*>(out_r + c * kBlk) = make_float4(ov[0], ov[1], ov[2], ov[3]);
     }
-    __syncthreads();  // semc is rewritten by the next chunk
-  }
-  if (!ok_slot) ok = false;  // tid 0's waits
-  if (live && ok && (tid & 15) == 0)
-    *reinterpret_cast<long long*>(p.state + kHeaderBytes + st * p.so.stride + p.so.pos) = s_pos[r] + 1;
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bars + kPbWFull);
 
-  // every tensor-core operation has completed (last sem commit waited)
+    // pass 2: ring, field, fusion, clip, output [P3 §2.1 channels 1-2, §2.2]
+    const int slot_r = static_cast<int>(s_pos[r] & (kRing - 1));
+    unsigned char* blk = p.state + kHeaderBytes + (live ? st : 0) * p.so.stride;
+    float* ring_r = reinterpret_cast<float*>(blk + p.so.ring) + static_cast<size_t>(slot_r) * p.H + c4;
+    float* rsum_r = reinterpret_cast<float*>(blk + p.so.ring_sum) + c4;
+    float* fld_r = reinterpret_cast<float*>(blk + p.so.field) + c4;
+    float* out_r = p.out + (live ? io : 0) * p.H + c4;
+    struct Row4 {
+      float4 x, old, rs, fl;
+    };
+    auto load_row = [&](int c) -> Row4 {
+      Row4 v;
+      if (live && c < nch) {
+        v.x = __ldcg(reinterpret_cast<const float4*>(out_r + c * kBlk));
+        v.old = __ldcg(reinterpret_cast<const float4*>(ring_r + c * kBlk));
+        v.rs = __ldcg(reinterpret_cast<const float4*>(rsum_r + c * kBlk));
+        v.fl = __ldcg(reinterpret_cast<const float4*>(fld_r + c * kBlk));
+      } else {
+        v.x = v.old = v.rs = v.fl = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      return v;
+    };
+    Row4 rn0 = load_row(0), rn1 = load_row(1);  // chunks c and c+1 in flight
+    const float a_l = p.alpha_layer[l];
+    const bool reader = (warp & 3) == 0;
+    for (int c = 0; c < nch; ++c) {
+      const int b = c % kSemBufs;
+      const unsigned ph = static_cast<unsigned>((c / kSemBufs) & 1);
+      float* stg = semst + b * TR * kSemStride;
+      if (reader) {
+        // accumulator b -> staging b (once the compute warps are done with it)
+        if (!mbar_wait_bounded(bars + kPbSemFull + b, ph, kMbarPollLimit, p.err)) ok = false;
+        tc_fence_after();
+        const int colh = (warp >> 2) * 32;
+        float v[32];
+        tmem_ld32(tmem + kSlots + b * kBlk + colh, v);
+        tc_fence_before();
+        if (lane == 0) mbar_arrive(bars + kPbSemEmpty + b);
+        if (c >= kSemBufs &&
+            !mbar_wait_bounded(bars + kPbStEmpty + b, static_cast<unsigned>(((c / kSemBufs) - 1) & 1), kMbarPollLimit, p.err))
+          ok = false;
+        if (lane < TR) {
+          float* dst = stg + lane * kSemStride + colh;
+#pragma unroll
+          for (int jj = 0; jj < 32; jj += 4)
+            *reinterpret_cast<float4*>(dst + jj) = make_float4(v[jj], v[jj + 1], v[jj + 2], v[jj + 3]);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bars + kPbStFull + b);
+      }
+      const Row4 cur = rn0;
+      rn0 = rn1;
+      rn1 = load_row(c + 2);
+      if (!mbar_wait_bounded(bars + kPbStFull + b, ph, kMbarPollLimit, p.err)) ok = false;
+      const float4 sv = *reinterpret_cast<const float4*>(stg + r * kSemStride + c4);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bars + kPbStEmpty + b);
+      if (live && ok) {
+        const float xa[4] = {cur.x.x, cur.x.y, cur.x.z, cur.x.w};
+        const float roa[4] = {cur.old.x, cur.old.y, cur.old.z, cur.old.w};
+        const float rsa[4] = {cur.rs.x, cur.rs.y, cur.rs.z, cur.rs.w};
+        const float fla[4] = {cur.fl.x, cur.fl.y, cur.fl.z, cur.fl.w};
+        const float sva[4] = {sv.x, sv.y, sv.z, sv.w};
+        float rv[4], fv[4], ov[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          rv[e] = (rsa[e] - roa[e]) + xa[e];        // ring sum after storing x_t
+          fv[e] = ewma(p.ema_gamma, fla[e], xa[e]);  // EMA field
+          float uu = rv[e] * (1.0f / kRing) + 0.5f * fv[e] + 0.5f * sva[e];
+          uu = fminf(fmaxf(uu, -p.clip_eps), p.clip_eps);
+          ov[e] = fmaf(a_l, uu, xa[e]);
+        }
+        *reinterpret_cast<float4*>(ring_r + c * kBlk) = cur.x;
+        *reinterpret_cast<float4*>(rsum_r + c * kBlk) = make_float4(rv[0], rv[1], rv[2], rv[3]);
+        *reinterpret_cast<float4*>(fld_r + c * kBlk) = make_float4(fv[0], fv[1], fv[2], fv[3]);
+        *reinterpret_cast<float4*>(out_r + c * kBlk) = make_float4(ov[0], ov[1], ov[2], ov[3]);
+      }
+    }
+    if (live && ok && (tid & 15) == 0)
+      *reinterpret_cast<long long*>(p.state + kHeaderBytes + st * p.so.stride + p.so.pos) = s_pos[r] + 1;
+  }
+
+  // every tensor-core operation has completed (the last sem chunk was read)
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
@@ -690,25 +1051,39 @@ PFN_cuTensorMapEncodeTiled_v12000 tile_map_encoder() {
 }
 
 // The window rings of every stream of the state as (head dim, KV head,
-// slot, stream) tensors; boxes of head_dim x 1 x kcb x 1.
+// slot, stream) tensors: boxes of head_dim x 1 x kcb x 1 (fp32 inputs), or
+// of 64 x 1 x kcb x 1 with 128-byte swizzling (bf16 inputs, warp MMAs),
+// which then also get q as a (head dim, query head, input row) tensor.
 cudaError_t encode_win_maps(const DecodeParams& p, int D, int esz, WinMaps* m) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = tile_map_encoder();
   if (!enc) return cudaErrorNotSupported;
+  const bool mma = esz == 2;
   const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(p.nkv),
                               static_cast<cuuint64_t>(p.K),
                               static_cast<cuuint64_t>(p.L) * static_cast<cuuint64_t>(p.B)};
   const cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * esz, static_cast<cuuint64_t>(p.nkv) * D * esz,
                                  static_cast<cuuint64_t>(p.so.stride)};
-  const cuuint32_t box[4] = {static_cast<cuuint32_t>(D), 1, static_cast<cuuint32_t>(p.tp.kcb), 1};
+  const cuuint32_t box[4] = {static_cast<cuuint32_t>(mma ? 64 : D), 1, static_cast<cuuint32_t>(p.tp.kcb), 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   const CUtensorMapDataType dt = esz == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const CUtensorMapSwizzle sw = mma ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE;
   auto one = [&](CUtensorMap* map, long long off) -> bool {
     void* base = p.state + kHeaderBytes + off;
-    return enc(map, dt, 4, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-               CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return enc(map, dt, 4, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
   };
   if (!one(&m->k, p.so.win_k) || !one(&m->v, p.so.win_v)) return cudaErrorInvalidValue;
+  std::memset(&m->q, 0, sizeof(m->q));
+  if (mma) {
+    const cuuint64_t qdims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(p.nq),
+                                 static_cast<cuuint64_t>(p.Lc) * static_cast<cuuint64_t>(p.n_seq)};
+    const cuuint64_t qstr[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(p.nq) * D * 2};
+    const cuuint32_t qbox[3] = {64, static_cast<cuuint32_t>(p.G), 1};
+    if (enc(&m->q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(p.q), qdims, qstr, qbox, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
   return cudaSuccess;
 }
 
@@ -727,10 +1102,14 @@ cudaError_t launch_t(const DecodeParams& p, cudaStream_t s) {
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, decode_near_kernel<Tin, D>, p, maps);
+  if constexpr (sizeof(Tin) == 2) {
+    e = cudaLaunchKernelEx(&cfg, decode_near_mma_kernel<D>, p, maps);
+  } else {
+    e = cudaLaunchKernelEx(&cfg, decode_near_kernel<Tin, D>, p, maps);
+  }
   if (e != cudaSuccess) return e;
   cfg.gridDim = dim3(static_cast<unsigned>(p.Lc * ((p.n_seq + TR - 1) / TR)), 1, 1);
-  cfg.blockDim = dim3(NTP, 1, 1);
+  cfg.blockDim = dim3(NTP, 1, 1);  // compute warps + the MMA warp
   cfg.dynamicSmemBytes = static_cast<size_t>(p.tp.pool_smem);
   return cudaLaunchKernelEx(&cfg, decode_pool_kernel, p);
 }
@@ -750,6 +1129,14 @@ bool plan_decode_tile(int H, int D, int esz, int G, int K, size_t limit, TilePla
   p.hvt = p.hkt + D * esz;
   p.hs = p.hvt + D * esz;
   p.hdr_bytes = a128(p.hs + 4LL * D);
+  if (esz == 2) {  // warp-MMA near field: fixed layout, chunks of 16 slots
+    p.kcb = std::min(KCB, K);
+    p.warp_bytes = D == 64 ? MmaNear<64>::warp : MmaNear<128>::warp;
+    p.near_smem = 2048 + NWN * p.warp_bytes;  // barriers (1 KB) + 1 KB alignment slack
+    if (static_cast<size_t>(p.near_smem) > limit) return false;
+    *out = p;
+    return true;
+  }
   // Window chunks of 16 slots, fewer where a plan of 16 does not fit.
   for (int kcb = std::min(KCB, K); kcb >= 1; kcb /= 2) {
     p.kcb = kcb;
@@ -769,8 +1156,8 @@ cudaError_t decode_tile_prepare(int device) {
   cudaError_t e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device);
   if (e == cudaSuccess) e = set_smem_t(decode_near_kernel<float, 64>, optin);
   if (e == cudaSuccess) e = set_smem_t(decode_near_kernel<float, 128>, optin);
-  if (e == cudaSuccess) e = set_smem_t(decode_near_kernel<__nv_bfloat16, 64>, optin);
-  if (e == cudaSuccess) e = set_smem_t(decode_near_kernel<__nv_bfloat16, 128>, optin);
+  if (e == cudaSuccess) e = set_smem_t(decode_near_mma_kernel<64>, optin);
+  if (e == cudaSuccess) e = set_smem_t(decode_near_mma_kernel<128>, optin);
   if (e == cudaSuccess) e = set_smem_t(decode_pool_kernel, optin);
   return e;
 }
