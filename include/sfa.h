@@ -31,7 +31,8 @@
  *   - Layer-major, token-major layouts (d = head_dim, H = n_q_heads·d):
  *       prefill q   [L][batch][n][n_q_heads][d]    in_dtype
  *               k,v [L][batch][n][n_kv_heads][d]   in_dtype
- *               out [L][batch][n][H]               fp32
+ *               out [L][batch][n][H]               fp32 (bf16 in the bf16 output
+ *                                                  modes, sfa_set_output_mode)
  *       decode  q   [L][batch][n_q_heads][d], k,v [L][batch][n_kv_heads][d],
  *               out [L][batch][H].
  *   - One state buffer serves `batch` sequences for all layers.  A state is
@@ -71,6 +72,18 @@ typedef enum sfa_status {
 } sfa_status;
 
 typedef enum sfa_dtype { SFA_F32 = 0, SFA_BF16 = 1 } sfa_dtype;
+
+/* What the compute calls write into `out` ([P3 §2.2]: output = attention
+ * output + enhancement, with enhancement = alpha_layer * clip(ring_mean +
+ * 0.5*field + 0.5*semantic, -eps, eps) and the attention output x = O_near +
+ * alpha_far*S [P1 §2.1 eq. O]).  Set per handle by sfa_set_output_mode. */
+typedef enum sfa_out_mode {
+  SFA_OUT_F32 = 0,      /* out fp32 = x + enhancement (default)                       */
+  SFA_OUT_BF16 = 1,     /* out bf16 = x + enhancement, rounded to nearest              */
+  SFA_OUT_ADD_F32 = 2,  /* out fp32 += enhancement: out holds the caller's attention
+                           output on entry ([P2] compute_enhancement(layer, attn_output)) */
+  SFA_OUT_ADD_BF16 = 3  /* out bf16 += enhancement, rounded to nearest                 */
+} sfa_out_mode;
 
 /* Operator configuration.  Field names follow the pages' SFA_Config. */
 typedef struct sfa_config {
@@ -180,7 +193,7 @@ SFA_API int sfa_state_reset(const sfa_handle* h, void* state, int batch, void* s
  * A state whose header does not match the handle or batch is left untouched
  * and latched as SFA_ERR_STATE_MISMATCH for sfa_check_device_status. */
 SFA_API int sfa_prefill(const sfa_handle* h, const void* q, const void* k, const void* v,
-                long long n, int batch, void* state, float* out, void* workspace,
+                long long n, int batch, void* state, void* out, void* workspace,
                 size_t workspace_bytes, void* stream);
 
 /* [P1 §2.1] and [P3 §2.1–2.2] for one token of every sequence: the
@@ -198,7 +211,7 @@ SFA_API int sfa_prefill(const sfa_handle* h, const void* q, const void* k, const
  * whose header does not match is left untouched and latched as
  * SFA_ERR_STATE_MISMATCH, as for sfa_prefill. */
 SFA_API int sfa_decode_step(const sfa_handle* h, const void* q, const void* k, const void* v,
-                    int batch, void* state, float* out, void* stream);
+                    int batch, void* state, void* out, void* stream);
 
 /* Serving variants.  The pages call the enhancement once per layer from
  * inside the model's attention ([P2] usage example and llama.cpp
@@ -220,7 +233,7 @@ SFA_API size_t sfa_prefill_layers_workspace_bytes(const sfa_handle* h, int layer
  * streams are untouched.  SFA_ERR_INVALID_ARG for a range outside 0 .. L-1. */
 SFA_API int sfa_prefill_layers(const sfa_handle* h, int layer_begin, int layer_count,
                                const void* q, const void* k, const void* v, long long n, int batch,
-                               void* state, float* out, void* workspace, size_t workspace_bytes,
+                               void* state, void* out, void* workspace, size_t workspace_bytes,
                                void* stream);
 
 /* sfa_decode_step for layers layer_begin .. layer_begin + layer_count - 1 and
@@ -235,7 +248,7 @@ SFA_API int sfa_prefill_layers(const sfa_handle* h, int layer_begin, int layer_c
  * option, as for sfa_decode_step. */
 SFA_API int sfa_decode_step_ex(const sfa_handle* h, int layer_begin, int layer_count,
                                const int* seq_ids, int n_seq, const void* q, const void* k,
-                               const void* v, int batch, void* state, float* out, void* stream);
+                               const void* v, int batch, void* state, void* out, void* stream);
 
 /* Decode input prefetch (default off).  enable = 1 declares that, for every
  * later decode call on this handle, q, k and v are complete when the call is
@@ -251,6 +264,16 @@ SFA_API int sfa_decode_step_ex(const sfa_handle* h, int layer_begin, int layer_c
  * for another value.  Results are identical either way. */
 SFA_API int sfa_set_decode_input_prefetch(sfa_handle* h, int enable);
 
+/* Output mode of later compute calls on this handle (sfa_out_mode; default
+ * SFA_OUT_F32).  In the bf16 modes `out` points at bf16 elements; in the
+ * add modes the calls read out (the caller's attention output, in the
+ * mode's dtype) and add the enhancement to it in place.  Outside
+ * SFA_OUT_F32 the prefill keeps x in its workspace instead of in out, so
+ * sfa_prefill_workspace_bytes grows by layers x batch x n x hidden x 4
+ * bytes, and decode calls of many sequences run the per-sequence kernel.
+ * SFA_ERR_INVALID_ARG for another value. */
+SFA_API int sfa_set_output_mode(sfa_handle* h, int mode);
+
 /* Synchronises `stream`, then returns and clears the first error latched on
  * the device since the last check (SFA_OK if none), or SFA_ERR_CUDA if the
  * stream reports a CUDA error. */
@@ -261,6 +284,24 @@ SFA_API const char* sfa_status_string(int status);
 
 /* ABI version of the loaded library (SFA_ABI_VERSION it was built with). */
 SFA_API int sfa_abi_version(void);
+
+/* Ragged prefill.  A serving engine's batch holds prompts of different
+ * lengths, and [P2]'s engine is called per layer with whatever tokens each
+ * sequence has; this call folds lens[b] tokens into sequence b (0 <= lens[b]
+ * <= n_max), every sequence from its own position, with the arithmetic of
+ * sfa_prefill.  q, k, v and out keep the layouts of sfa_prefill with n =
+ * n_max: sequence b's tokens are its rows 0 .. lens[b]-1; the rows past
+ * lens[b] take no part in any result, and out keeps what it held there.
+ * lens: DEVICE array of `batch` int32, read by the kernels, so an earlier
+ * kernel on the stream may write it.  workspace:
+ * sfa_prefill_workspace_bytes(h, batch, n_max) bytes.  A count outside
+ * 0 .. n_max leaves that sequence's state and output untouched and is
+ * latched as SFA_ERR_INVALID_ARG for sfa_check_device_status; lens == NULL
+ * is SFA_ERR_INVALID_ARG.  Otherwise the returns of sfa_prefill; n_max == 0
+ * enqueues nothing. */
+SFA_API int sfa_prefill_ragged(const sfa_handle* h, const void* q, const void* k, const void* v,
+                               long long n_max, const int* lens, int batch, void* state, void* out,
+                               void* workspace, size_t workspace_bytes, void* stream);
 
 /* Bytes of the fixed device scratch behind sfa_prefill_static_ws. */
 #define SFA_STATIC_WORKSPACE_BYTES (16u << 20)
@@ -282,7 +323,7 @@ SFA_API int sfa_abi_version(void);
  * prefill into smaller chunks), otherwise exactly what sfa_prefill returns;
  * results equal sfa_prefill's. */
 SFA_API int sfa_prefill_static_ws(const sfa_handle* h, const void* q, const void* k, const void* v,
-                                  long long n, int batch, void* state, float* out, void* stream);
+                                  long long n, int batch, void* state, void* out, void* stream);
 
 /* Test hook for the device-side bounded waits of sfa_prefill (not needed in
  * normal use).  withhold_tile: tile index (tile * streams + stream, streams =

@@ -39,13 +39,18 @@ SFA_ERR_WORKSPACE = -7
 SFA_F32 = 0
 SFA_BF16 = 1
 
+SFA_OUT_F32 = 0       # out fp32 = x + enhancement (default)
+SFA_OUT_BF16 = 1      # out bf16 = x + enhancement
+SFA_OUT_ADD_F32 = 2   # out fp32 += enhancement (out holds the caller's attention output)
+SFA_OUT_ADD_BF16 = 3  # out bf16 += enhancement
+
 EXPORTED = (
     "sfa_config_default", "sfa_config_validate", "sfa_state_layout_for", "sfa_init",
     "sfa_destroy", "sfa_state_bytes", "sfa_prefill_workspace_bytes", "sfa_state_reset",
     "sfa_prefill", "sfa_decode_step", "sfa_check_device_status", "sfa_status_string",
     "sfa_abi_version", "sfa_debug_set_wait_limit", "sfa_debug_set_paths", "sfa_prefill_static_ws",
     "sfa_prefill_layers_workspace_bytes", "sfa_prefill_layers", "sfa_decode_step_ex",
-    "sfa_set_decode_input_prefetch",
+    "sfa_set_decode_input_prefetch", "sfa_prefill_ragged", "sfa_set_output_mode",
 )
 
 
@@ -112,6 +117,8 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
             "sfa_prefill_layers": (i, [vp, i, i, vp, vp, vp, ll, i, vp, vp, vp, sz, vp]),
             "sfa_decode_step_ex": (i, [vp, i, i, vp, i, vp, vp, vp, i, vp, vp, vp]),
             "sfa_set_decode_input_prefetch": (i, [vp, i]),
+            "sfa_prefill_ragged": (i, [vp, vp, vp, vp, ll, vp, i, vp, vp, vp, sz, vp]),
+            "sfa_set_output_mode": (i, [vp, i]),
         }
         for name, (res, args) in sigs.items():
             fn = getattr(lib, name)
@@ -218,6 +225,12 @@ class Handle:
     def __init__(self, ptr: int, cfg: SfaConfig):
         self.ptr = ptr
         self.cfg = cfg
+        self.out_mode = SFA_OUT_F32
+
+    @property
+    def out_dtype(self) -> torch.dtype:
+        """dtype of `out` in the handle's output mode."""
+        return torch.bfloat16 if self.out_mode in (SFA_OUT_BF16, SFA_OUT_ADD_BF16) else torch.float32
 
     def __del__(self):
         if getattr(self, "ptr", None):
@@ -276,7 +289,7 @@ def sfa_prefill(h: Handle, q, k, v, n: int, batch: int, state: torch.Tensor, out
         return
     qp, kp, vp = _qkv_checks(h, q, k, v, n, batch)
     sp = _dev(state, "state", torch.uint8, sfa_state_bytes(h, batch))
-    op = _dev(out, "out", torch.float32, h.cfg.n_layers * batch * n * h.cfg.hidden)
+    op = _dev(out, "out", h.out_dtype, h.cfg.n_layers * batch * n * h.cfg.hidden)
     need = sfa_prefill_workspace_bytes(h, batch, n)
     if workspace is None or workspace.numel() < need:
         raise SfaError(SFA_ERR_WORKSPACE, "sfa_prefill")
@@ -285,6 +298,28 @@ def sfa_prefill(h: Handle, q, k, v, n: int, batch: int, state: torch.Tensor, out
                                     workspace.numel(), _stream_ptr(stream))
     if rc != SFA_OK:
         raise SfaError(rc, "sfa_prefill")
+
+
+def sfa_prefill_ragged(h: Handle, q, k, v, n_max: int, lens: torch.Tensor, batch: int,
+                       state: torch.Tensor, out: torch.Tensor, workspace: Optional[torch.Tensor],
+                       stream=None) -> None:
+    """sfa_prefill where sequence b folds in lens[b] (device int32) tokens of
+    its rows 0 .. lens[b]-1 of the n_max-row inputs; out rows past lens[b]
+    are left as they were."""
+    if n_max == 0:
+        return
+    qp, kp, vp = _qkv_checks(h, q, k, v, n_max, batch)
+    sp = _dev(state, "state", torch.uint8, sfa_state_bytes(h, batch))
+    op = _dev(out, "out", h.out_dtype, h.cfg.n_layers * batch * n_max * h.cfg.hidden)
+    lp = _dev(lens, "lens", torch.int32, batch)
+    need = sfa_prefill_workspace_bytes(h, batch, n_max)
+    if workspace is None or workspace.numel() < need:
+        raise SfaError(SFA_ERR_WORKSPACE, "sfa_prefill_ragged")
+    wp = _dev(workspace, "workspace", torch.uint8)
+    rc = load_library().sfa_prefill_ragged(h.ptr, qp, kp, vp, n_max, lp, batch, sp, op, wp,
+                                           workspace.numel(), _stream_ptr(stream))
+    if rc != SFA_OK:
+        raise SfaError(rc, "sfa_prefill_ragged")
 
 
 def sfa_prefill_layers_workspace_bytes(h: Handle, layer_count: int, batch: int, n: int) -> int:
@@ -300,7 +335,7 @@ def sfa_prefill_layers(h: Handle, layer_begin: int, layer_count: int, q, k, v, n
         return
     qp, kp, vp = _qkv_checks(h, q, k, v, n, batch, layer_count)
     sp = _dev(state, "state", torch.uint8, sfa_state_bytes(h, batch))
-    op = _dev(out, "out", torch.float32, layer_count * batch * n * h.cfg.hidden)
+    op = _dev(out, "out", h.out_dtype, layer_count * batch * n * h.cfg.hidden)
     need = sfa_prefill_layers_workspace_bytes(h, layer_count, batch, n)
     if workspace is None or workspace.numel() < need:
         raise SfaError(SFA_ERR_WORKSPACE, "sfa_prefill_layers")
@@ -319,7 +354,7 @@ def sfa_decode_step_ex(h: Handle, layer_begin: int, layer_count: int,
     n_seq = batch if seq_ids is None else int(seq_ids.numel())
     qp, kp, vp = _qkv_checks(h, q, k, v, 1, n_seq, layer_count)
     sp = _dev(state, "state", torch.uint8, sfa_state_bytes(h, batch))
-    op = _dev(out, "out", torch.float32, layer_count * n_seq * h.cfg.hidden)
+    op = _dev(out, "out", h.out_dtype, layer_count * n_seq * h.cfg.hidden)
     ip = None if seq_ids is None else _dev(seq_ids, "seq_ids", torch.int32, n_seq)
     rc = load_library().sfa_decode_step_ex(h.ptr, layer_begin, layer_count, ip, n_seq, qp, kp, vp,
                                            batch, sp, op, _stream_ptr(stream))
@@ -338,7 +373,7 @@ def sfa_prefill_static_ws(h: Handle, q, k, v, n: int, batch: int, state: torch.T
         return
     qp, kp, vp = _qkv_checks(h, q, k, v, n, batch)
     sp = _dev(state, "state", torch.uint8, sfa_state_bytes(h, batch))
-    op = _dev(out, "out", torch.float32, h.cfg.n_layers * batch * n * h.cfg.hidden)
+    op = _dev(out, "out", h.out_dtype, h.cfg.n_layers * batch * n * h.cfg.hidden)
     rc = load_library().sfa_prefill_static_ws(h.ptr, qp, kp, vp, n, batch, sp, op,
                                               _stream_ptr(stream))
     if rc != SFA_OK:
@@ -352,7 +387,7 @@ def sfa_decode_step(h: Handle, q, k, v, batch: int, state: torch.Tensor, out: to
     prefetch is on (sfa_set_decode_input_prefetch)."""
     qp, kp, vp = _qkv_checks(h, q, k, v, 1, batch)
     sp = _dev(state, "state", torch.uint8, sfa_state_bytes(h, batch))
-    op = _dev(out, "out", torch.float32, h.cfg.n_layers * batch * h.cfg.hidden)
+    op = _dev(out, "out", h.out_dtype, h.cfg.n_layers * batch * h.cfg.hidden)
     rc = load_library().sfa_decode_step(h.ptr, qp, kp, vp, batch, sp, op, _stream_ptr(stream))
     if rc != SFA_OK:
         raise SfaError(rc, "sfa_decode_step")
@@ -367,6 +402,16 @@ def sfa_set_decode_input_prefetch(h: Handle, enable: bool) -> None:
     rc = load_library().sfa_set_decode_input_prefetch(h.ptr, 1 if enable else 0)
     if rc != SFA_OK:
         raise SfaError(rc, "sfa_set_decode_input_prefetch")
+
+
+def sfa_set_output_mode(h: Handle, mode: int) -> None:
+    """What later compute calls write into out: SFA_OUT_F32 / SFA_OUT_BF16
+    (x + enhancement) or SFA_OUT_ADD_F32 / SFA_OUT_ADD_BF16 (out, holding
+    the caller's attention output, plus the enhancement in place)."""
+    rc = load_library().sfa_set_output_mode(h.ptr, int(mode))
+    if rc != SFA_OK:
+        raise SfaError(rc, "sfa_set_output_mode")
+    h.out_mode = int(mode)
 
 
 def sfa_check_device_status(h: Handle, stream=None) -> int:
@@ -427,16 +472,38 @@ class SfaOperator:
     def reset(self, stream=None):
         sfa_state_reset(self.handle, self.state, self.batch, stream)
 
+    def set_output_mode(self, mode: int) -> None:
+        sfa_set_output_mode(self.handle, mode)
+
+    def _new_out(self, shape):
+        if self.handle.out_mode in (SFA_OUT_ADD_F32, SFA_OUT_ADD_BF16):
+            raise ValueError("the add output modes need out: it holds the attention output")
+        return torch.empty(shape, dtype=self.handle.out_dtype, device=self.device)
+
     def prefill(self, q, k, v, out: Optional[torch.Tensor] = None, stream=None):
         n = q.shape[2]
         c = self.cfg
         if out is None:
-            out = torch.empty((c.n_layers, self.batch, n, c.hidden), dtype=torch.float32,
-                              device=self.device)
+            out = self._new_out((c.n_layers, self.batch, n, c.hidden))
         if n > 0:
             self._ensure_workspace(n)
             sfa_prefill(self.handle, q, k, v, n, self.batch, self.state, out, self.workspace,
                         stream)
+        return out
+
+    def prefill_ragged(self, q, k, v, lens: torch.Tensor, out: Optional[torch.Tensor] = None,
+                       stream=None):
+        """Prefill where sequence b takes lens[b] (device int32) of the n_max
+        rows of q, k, v ([L, B, n_max, heads, d]); out rows past lens[b] keep
+        their contents (a new out starts as NaN there)."""
+        n = q.shape[2]
+        c = self.cfg
+        if out is None:
+            out = self._new_out((c.n_layers, self.batch, n, c.hidden)).fill_(float("nan"))
+        if n > 0:
+            self._ensure_workspace(n)
+            sfa_prefill_ragged(self.handle, q, k, v, n, lens, self.batch, self.state, out,
+                               self.workspace, stream)
         return out
 
     def decode(self, q, k, v, out: Optional[torch.Tensor] = None, stream=None):
@@ -444,14 +511,13 @@ class SfaOperator:
         sfa_decode_step, with the per-operator constants looked up once."""
         if out is None:
             c = self.cfg
-            out = torch.empty((c.n_layers, self.batch, c.hidden), dtype=torch.float32,
-                              device=self.device)
+            out = self._new_out((c.n_layers, self.batch, c.hidden))
         nq, nkv, nout = self._dec_numel
         dt = self._in_dtype
         rc = self._decode_fn(self.handle.ptr, _dev(q, "q", dt, nq), _dev(k, "k", dt, nkv),
                              _dev(v, "v", dt, nkv),
                              self.batch, _dev(self.state, "state", torch.uint8, self._state_bytes),
-                             _dev(out, "out", torch.float32, nout), _stream_ptr(stream))
+                             _dev(out, "out", self.handle.out_dtype, nout), _stream_ptr(stream))
         if rc != SFA_OK:
             raise SfaError(rc, "sfa_decode_step")
         return out
@@ -461,8 +527,7 @@ class SfaOperator:
         """Prefill of layers layer_begin .. layer_begin + q.shape[0] - 1."""
         lc, n = q.shape[0], q.shape[2]
         if out is None:
-            out = torch.empty((lc, self.batch, n, self.cfg.hidden), dtype=torch.float32,
-                              device=self.device)
+            out = self._new_out((lc, self.batch, n, self.cfg.hidden))
         if n > 0:
             need = sfa_prefill_layers_workspace_bytes(self.handle, lc, self.batch, n)
             if self.workspace is None or self.workspace.numel() < need:
@@ -477,7 +542,7 @@ class SfaOperator:
         sequences in seq_ids (int32, on the device; None = all)."""
         lc, ns = q.shape[0], q.shape[1]
         if out is None:
-            out = torch.empty((lc, ns, self.cfg.hidden), dtype=torch.float32, device=self.device)
+            out = self._new_out((lc, ns, self.cfg.hidden))
         sfa_decode_step_ex(self.handle, layer_begin, lc, seq_ids, q, k, v, self.batch,
                            self.state, out, stream)
         return out

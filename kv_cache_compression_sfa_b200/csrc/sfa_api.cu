@@ -44,6 +44,7 @@ struct sfa_handle {
   int tile_mode;         // -1: by batch size; 0: never; 1: always (sfa_debug_set_paths)
   bool near_tc;          // prefill near field on the tensor cores where it applies
   bool inputs_early;     // decode inputs declared complete before each call
+  int out_mode;          // sfa_out_mode of the compute calls
 };
 
 namespace {
@@ -115,7 +116,7 @@ std::vector<int> cluster_candidates(int nq, int d) {
 // Workspace of a prefill call: the streams' positions, S at the end of the
 // call, the pool weights of every tile (two 8 KB bf16 blocks) and S at
 // every tile start.
-PrefillWorkspace prefill_workspace(const sfa_config* c, int layers, int batch, long long n) {
+PrefillWorkspace prefill_workspace(const sfa_config* c, int layers, int batch, long long n, int out_mode) {
   PrefillWorkspace w;
   const long long streams = static_cast<long long>(layers) * batch;
   const long long tiles = streams * ((n + kTile - 1) / kTile);
@@ -124,7 +125,10 @@ PrefillWorkspace prefill_workspace(const sfa_config* c, int layers, int batch, l
   w.sfin = align256(8 * streams);
   w.w = w.sfin + align256(4 * streams * sdim);
   w.sst = w.w + tiles * 2LL * kBlkBytesHost;
-  w.total = w.sst + align256(4 * tiles * sdim);
+  w.x = w.sst + align256(4 * tiles * sdim);
+  // x between the kernels, where the result buffer cannot hold it
+  const long long xb = out_mode == SFA_OUT_F32 ? 0 : align256(4LL * streams * n * hidden_of(c));
+  w.total = w.x + xb;
   return w;
 }
 
@@ -191,6 +195,10 @@ void fill_common(P& p, const sfa_handle* h, int batch, void* state) {
   p.clip_eps = c->clip_eps;
   p.score_scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(c->head_dim)));
 }
+
+int prefill_impl(const sfa_handle* h, int layer_begin, int layer_count, const void* q, const void* k,
+                 const void* v, long long n, const int* lens, int batch, void* state, void* out,
+                 void* workspace, size_t workspace_bytes, void* stream);
 
 }  // namespace
 
@@ -272,6 +280,7 @@ int sfa_init(const sfa_config* cfg, sfa_handle** out) {
   h->inputs_early = false;
   h->tile_mode = -1;
   h->near_tc = true;
+  h->out_mode = SFA_OUT_F32;
   const int L = cfg->n_layers, H = hidden_of(cfg);
   bool no_fit = false;  // a kernel's shared-memory plan does not fit this device
   const size_t slot_bytes = sizeof(float) * static_cast<size_t>(L) * kSlots * H;
@@ -393,7 +402,7 @@ size_t sfa_prefill_layers_workspace_bytes(const sfa_handle* h, int layer_count, 
       layer_count > h->cfg.n_layers)
     return 0;
   if (prefill_shape_status(layer_count, batch, n) != SFA_OK) return 0;
-  return static_cast<size_t>(prefill_workspace(&h->cfg, layer_count, batch, n).total);
+  return static_cast<size_t>(prefill_workspace(&h->cfg, layer_count, batch, n, h->out_mode).total);
 }
 
 int sfa_state_reset(const sfa_handle* h, void* state, int batch, void* stream) {
@@ -415,7 +424,7 @@ int sfa_state_reset(const sfa_handle* h, void* state, int batch, void* stream) {
 }
 
 int sfa_prefill(const sfa_handle* h, const void* q, const void* k, const void* v, long long n,
-                int batch, void* state, float* out, void* workspace, size_t workspace_bytes,
+                int batch, void* state, void* out, void* workspace, size_t workspace_bytes,
                 void* stream) {
   if (!handle_ok(h)) return SFA_ERR_INVALID_ARG;
   return sfa_prefill_layers(h, 0, h->cfg.n_layers, q, k, v, n, batch, state, out, workspace,
@@ -424,7 +433,26 @@ int sfa_prefill(const sfa_handle* h, const void* q, const void* k, const void* v
 
 int sfa_prefill_layers(const sfa_handle* h, int layer_begin, int layer_count, const void* q,
                        const void* k, const void* v, long long n, int batch, void* state,
-                       float* out, void* workspace, size_t workspace_bytes, void* stream) {
+                       void* out, void* workspace, size_t workspace_bytes, void* stream) {
+  return prefill_impl(h, layer_begin, layer_count, q, k, v, n, nullptr, batch, state, out, workspace,
+                      workspace_bytes, stream);
+}
+
+int sfa_prefill_ragged(const sfa_handle* h, const void* q, const void* k, const void* v, long long n_max,
+                       const int* lens, int batch, void* state, void* out, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  if (!handle_ok(h) || !lens) return SFA_ERR_INVALID_ARG;
+  return prefill_impl(h, 0, h->cfg.n_layers, q, k, v, n_max, lens, batch, state, out, workspace,
+                      workspace_bytes, stream);
+}
+
+}  // extern "C"
+
+namespace {
+
+int prefill_impl(const sfa_handle* h, int layer_begin, int layer_count, const void* q, const void* k,
+                 const void* v, long long n, const int* lens, int batch, void* state, void* out,
+                 void* workspace, size_t workspace_bytes, void* stream) {
   if (!handle_ok(h) || n < 0 || batch <= 0) return SFA_ERR_INVALID_ARG;
   if (layer_begin < 0 || layer_count <= 0 || layer_begin + layer_count > h->cfg.n_layers)
     return SFA_ERR_INVALID_ARG;
@@ -436,7 +464,7 @@ int sfa_prefill_layers(const sfa_handle* h, int layer_begin, int layer_count, co
   const int shape = prefill_shape_status(layer_count, batch, n);
   if (shape != SFA_OK) return shape;
   const sfa_config* c = &h->cfg;
-  const PrefillWorkspace w = prefill_workspace(c, layer_count, batch, n);
+  const PrefillWorkspace w = prefill_workspace(c, layer_count, batch, n, h->out_mode);
   if (!workspace || workspace_bytes < static_cast<size_t>(w.total)) return SFA_ERR_WORKSPACE;
   const long long streams = static_cast<long long>(layer_count) * batch;
   const long long tiles_per_stream = (n + kTile - 1) / kTile;
@@ -449,9 +477,14 @@ int sfa_prefill_layers(const sfa_handle* h, int layer_begin, int layer_count, co
   p.q = q;
   p.k = k;
   p.v = v;
-  p.out = out;
   p.ws = static_cast<unsigned char*>(workspace);
+  p.res = out;
+  p.out_mode = h->out_mode;
+  // x between the kernels: in the result buffer itself (fp32 x + enhancement
+  // overwrites it row by row) or in the workspace
+  p.out = h->out_mode == SFA_OUT_F32 ? static_cast<float*>(out) : reinterpret_cast<float*>(p.ws + w.x);
   p.n = n;
+  p.lens = lens;
   p.l0 = layer_begin;
   p.tiles_per_stream = static_cast<int>(tiles_per_stream);
   p.n_streams = static_cast<int>(streams);
@@ -459,6 +492,7 @@ int sfa_prefill_layers(const sfa_handle* h, int layer_begin, int layer_count, co
   p.ws_sfin = w.sfin;
   p.ws_w = w.w;
   p.ws_sst = w.sst;
+  p.ws_x = w.x;
   {
     // Near-field segments: about four rounds of two CTAs per SM, each CTA a
     // run of consecutive tiles of one (stream, head).
@@ -479,8 +513,12 @@ int sfa_prefill_layers(const sfa_handle* h, int layer_begin, int layer_count, co
   return cuda_status(launch_prefill(p, c->in_dtype, c->head_dim, s));
 }
 
+}  // namespace
+
+extern "C" {
+
 int sfa_decode_step(const sfa_handle* h, const void* q, const void* k, const void* v, int batch,
-                    void* state, float* out, void* stream) {
+                    void* state, void* out, void* stream) {
   if (!handle_ok(h)) return SFA_ERR_INVALID_ARG;
   return sfa_decode_step_ex(h, 0, h->cfg.n_layers, nullptr, batch, q, k, v, batch, state, out,
                             stream);
@@ -488,7 +526,7 @@ int sfa_decode_step(const sfa_handle* h, const void* q, const void* k, const voi
 
 int sfa_decode_step_ex(const sfa_handle* h, int layer_begin, int layer_count, const int* seq_ids,
                        int n_seq, const void* q, const void* k, const void* v, int batch,
-                       void* state, float* out, void* stream) {
+                       void* state, void* out, void* stream) {
   if (!handle_ok(h) || batch <= 0 || !q || !k || !v || !state || !out) return SFA_ERR_INVALID_ARG;
   if (layer_begin < 0 || layer_count <= 0 || layer_begin + layer_count > h->cfg.n_layers)
     return SFA_ERR_INVALID_ARG;
@@ -508,7 +546,9 @@ int sfa_decode_step_ex(const sfa_handle* h, int layer_begin, int layer_count, co
   p.q = q;
   p.k = k;
   p.v = v;
-  p.out = out;
+  p.out = static_cast<float*>(out);  // the batch-tiled decode keeps x here (SFA_OUT_F32 only)
+  p.res = out;
+  p.out_mode = h->out_mode;
   p.CS = h->cs;
   p.HPC = c->n_q_heads / p.CS;
   p.NGm = max_kv_heads_per_cta(c->n_q_heads, c->n_kv_heads, p.CS);
@@ -517,8 +557,10 @@ int sfa_decode_step_ex(const sfa_handle* h, int layer_begin, int layer_count, co
   p.inputs_early = h->inputs_early ? 1 : 0;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // Batch-tiled decode from kDecodeTileMinSeqs sequences per call (its
-  // tensor copies address input rows with 32-bit coordinates).
+  // tensor copies address input rows with 32-bit coordinates; it keeps x in
+  // out, so only for fp32 x + enhancement results).
   const bool tile = h->tile_ok && static_cast<long long>(layer_count) * n_seq <= 0x7fffffffLL &&
+                    h->out_mode == SFA_OUT_F32 &&
                     (h->tile_mode == 1 || (h->tile_mode < 0 && n_seq >= kDecodeTileMinSeqs));
   if (tile) return cuda_status(launch_decode_tile(p, c->in_dtype, c->head_dim, s));
   return cuda_status(launch_decode(p, c->in_dtype, c->head_dim, s));
@@ -554,6 +596,12 @@ const char* sfa_status_string(int status) {
 }
 
 int sfa_abi_version(void) { return SFA_ABI_VERSION; }
+
+int sfa_set_output_mode(sfa_handle* h, int mode) {
+  if (!handle_ok(h) || mode < SFA_OUT_F32 || mode > SFA_OUT_ADD_BF16) return SFA_ERR_INVALID_ARG;
+  h->out_mode = mode;
+  return SFA_OK;
+}
 
 int sfa_set_decode_input_prefetch(sfa_handle* h, int enable) {
   if (!handle_ok(h) || (enable != 0 && enable != 1)) return SFA_ERR_INVALID_ARG;

@@ -41,6 +41,24 @@ __device__ __forceinline__ float ewma(float g, float s, float e) {
   return fmaf(g, s, (1.0f - g) * e);
 }
 
+// Result element i of the enhancement alpha_layer * u for attention output
+// x, in the output mode [P3 §2.2]: fp32 or bf16 x + enhancement, or the
+// enhancement added to the caller's attention output already in res.  The
+// fp32 mode rounds once: fmaf(alpha_layer, u, x).
+__device__ __forceinline__ void store_result(int mode, void* res, long long i, float a_l, float u, float x) {
+  if (mode == SFA_OUT_F32) {
+    static_cast<float*>(res)[i] = fmaf(a_l, u, x);
+  } else if (mode == SFA_OUT_BF16) {
+    static_cast<__nv_bfloat16*>(res)[i] = __float2bfloat16_rn(fmaf(a_l, u, x));
+  } else if (mode == SFA_OUT_ADD_F32) {
+    float* r = static_cast<float*>(res) + i;
+    *r = fmaf(a_l, u, *r);
+  } else {
+    __nv_bfloat16* r = static_cast<__nv_bfloat16*>(res) + i;
+    *r = __float2bfloat16_rn(fmaf(a_l, u, __bfloat162float(*r)));
+  }
+}
+
 // Loads N consecutive elements of the input dtype and widens them to fp32.
 template <typename T, int N>
 struct VecLoad;

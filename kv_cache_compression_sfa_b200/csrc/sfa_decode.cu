@@ -531,7 +531,7 @@ decode_kernel(const DecodeParams p) {
         ring_row[c] = x;
         ring_sum[gi] = rv;
         field[gi] = fv;
-        p.out[io * p.H + gi] = fmaf(a_l, u, x);
+        store_result(p.out_mode, p.res, io * p.H + gi, a_l, u, x);
       }
     }
   }

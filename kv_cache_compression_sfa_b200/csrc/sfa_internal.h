@@ -71,7 +71,9 @@ struct DecodeParams {
   const void* q;
   const void* k;
   const void* v;
-  float* out;
+  float* out;               // fp32 result (SFA_OUT_F32), where the batch-tiled decode keeps x
+  void* res;                // result in the output mode's dtype
+  int out_mode;             // sfa_out_mode
   unsigned char* state;
   const float* slots;       // [L][64][H]
   const float* slot_norm;   // [L][64], clamped at kNormFloor
@@ -112,7 +114,9 @@ struct PrefillParams {
   const void* q;
   const void* k;
   const void* v;
-  float* out;
+  float* out;               // x between the kernels: the result buffer (SFA_OUT_F32) or workspace
+  void* res;                // result in the output mode's dtype
+  int out_mode;             // sfa_out_mode
   unsigned char* state;
   unsigned char* ws;
   const float* slots;
@@ -122,14 +126,16 @@ struct PrefillParams {
   int* err;
   uint64_t cfg_hash;
   StreamOffsets so;
-  long long n;              // tokens per stream in this call
+  long long n;              // tokens per stream in this call (row pitch of q, k, v, out)
+  const int* lens;          // [B] tokens of each sequence (ragged call, device), or null: all n
   int L, B, nq, nkv, K, H, G;
   int l0;                   // first layer of the state served (streams are l0*B + ...)
   int tiles_per_stream, n_streams;
   int n_seg, tps;           // near field: segments per stream, tiles per segment
   // workspace byte offsets: stream positions, S at the end of the call, pool
-  // weights, far-field state at every tile start
-  long long ws_pos, ws_sfin, ws_w, ws_sst;
+  // weights, far-field state at every tile start, x (output modes other
+  // than SFA_OUT_F32)
+  long long ws_pos, ws_sfin, ws_w, ws_sst, ws_x;
   float gamma_far, alpha_far, ema_gamma, inv_temp, clip_eps, score_scale;
   unsigned spin_limit;      // polls of a bounded wait before it gives up
   long long withhold_tile;  // test hook: this tile's pool CTA waits on a barrier nothing completes
@@ -150,6 +156,7 @@ struct PrefillWorkspace {
   long long sfin;   // [streams][n_kv][d] fp32 far state at the end of the call
   long long w;      // [streams * tiles][hi, lo] 64 x 64 bf16 pool-weight blocks
   long long sst;    // [streams][tiles][n_kv][d] fp32 far state at every tile start
+  long long x;      // [streams][n][H] fp32 x when the result is not fp32 x + enhancement (else 0)
   long long total;
 };
 

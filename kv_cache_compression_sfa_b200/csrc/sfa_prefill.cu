@@ -75,6 +75,15 @@ __device__ __forceinline__ unsigned char* stream_block(const PrefillParams& p, i
   return p.state + kHeaderBytes + (static_cast<long long>(p.l0) * p.B + s) * p.so.stride;
 }
 
+// Tokens that call-relative stream s folds in: the call's n, or for a
+// ragged call its sequence's own count (a count outside 0 .. n counts as 0;
+// far_agg_kernel latches it).  Inputs and outputs keep a row pitch of n.
+__device__ __forceinline__ long long stream_len(const PrefillParams& p, int s) {
+  if (!p.lens) return p.n;
+  const int v = __ldg(p.lens + (s % p.B));
+  return (v < 0 || v > p.n) ? 0 : v;
+}
+
 // ======================================================================
 // 0. far-field state at every tile start [P1 §2.1 eq. S_t]
 // ======================================================================
@@ -110,10 +119,18 @@ __global__ void __launch_bounds__(NT) far_agg_kernel(const PrefillParams p) {
     return;
   }
   const long long pos0 = s_pos;
-  if (tid == 0 && tile == 0) reinterpret_cast<long long*>(p.ws + p.ws_pos)[s] = pos0;
+  const long long ns = stream_len(p, s);
+  if (tid == 0 && tile == 0) {
+    reinterpret_cast<long long*>(p.ws + p.ws_pos)[s] = pos0;
+    if (p.lens) {
+      const int v = __ldg(p.lens + (s % p.B));
+      if (v < 0 || v > p.n) latch_error(p.err, SFA_ERR_INVALID_ARG);
+    }
+  }
   const int K = p.K, nkv = p.nkv;
   const long long t0 = pos0 + static_cast<long long>(tile) * kTile;
-  const int Tt = static_cast<int>(min(static_cast<long long>(kTile), p.n - static_cast<long long>(tile) * kTile));
+  // tokens of this tile (<= 0 past a ragged stream's end: nothing evicts)
+  const int Tt = static_cast<int>(min(static_cast<long long>(kTile), ns - static_cast<long long>(tile) * kTile));
   if (tid < kTile)
     s_w[tid] = (tid < Tt && t0 + tid >= K) ? (1.0f - p.gamma_far) * powf(p.gamma_far, static_cast<float>(Tt - 1 - tid)) : 0.f;
   __syncthreads();
@@ -168,6 +185,7 @@ __global__ void __launch_bounds__(NT) far_carry_kernel(const PrefillParams p) {
   const int ne = p.nkv * (p.H / p.nq);
   if (!s_ok || e >= ne) return;
   const long long pos0 = reinterpret_cast<const long long*>(p.ws + p.ws_pos)[s];
+  const long long ns = stream_len(p, s);
   const float* far = reinterpret_cast<const float*>(stream_block(p, s) + p.so.far);
   float S = far[e];
   float* a = reinterpret_cast<float*>(p.ws + p.ws_sst) + static_cast<long long>(s) * p.tiles_per_stream * ne + e;
@@ -183,7 +201,7 @@ __global__ void __launch_bounds__(NT) far_carry_kernel(const PrefillParams p) {
       const int i = t8 + u;
       if (i < tiles) {
         const long long t0 = pos0 + static_cast<long long>(i) * kTile;
-        const long long Tt = min(static_cast<long long>(kTile), p.n - static_cast<long long>(i) * kTile);
+        const long long Tt = min(static_cast<long long>(kTile), ns - static_cast<long long>(i) * kTile);
         const long long ev = max(0LL, t0 + Tt - max(t0, static_cast<long long>(K)));
         const float gev = ev == kTile ? g64 : powf(gf, static_cast<float>(ev));
         a[static_cast<long long>(i) * ne] = S;
@@ -297,6 +315,7 @@ __global__ void __launch_bounds__(NT, 2) near_kernel(const PrefillParams p) {
   __syncthreads();
   if (!s_ok) return;  // latched by far_agg_kernel
   const long long pos0 = s_pos;
+  const long long ns = stream_len(p, s);  // tokens of this stream in the call
   const int K = p.K, nkv = p.nkv, g = h / p.G;
   const Tin* win_k = reinterpret_cast<const Tin*>(blk + p.so.win_k);
   const Tin* win_v = reinterpret_cast<const Tin*>(blk + p.so.win_v);
@@ -323,7 +342,7 @@ __global__ void __launch_bounds__(NT, 2) near_kernel(const PrefillParams p) {
   // never read and stay unloaded.
   auto issue = [&](int i, int st) {
     const long long t0 = pos0 + static_cast<long long>(i) * kTile;
-    const int Tt = static_cast<int>(min(static_cast<long long>(kTile), p.n - static_cast<long long>(i) * kTile));
+    const int Tt = static_cast<int>(min(static_cast<long long>(kTile), ns - static_cast<long long>(i) * kTile));
     unsigned char* qs = smb + np.q[st];
     for (int c = tid; c < Tt * C16; c += NT) {
       const int r = c / C16, u = c % C16;
@@ -346,8 +365,10 @@ __global__ void __launch_bounds__(NT, 2) near_kernel(const PrefillParams p) {
   };
 
   const float gf = p.gamma_far, af = p.alpha_far;
-  const int i0 = seg * p.tps, tiles = min(p.tiles_per_stream, i0 + p.tps);  // this CTA's tiles
-  issue(i0, 0);
+  // this CTA's tiles (a ragged stream may end before them)
+  const int tiles_s = static_cast<int>((ns + kTile - 1) / kTile);
+  const int i0 = seg * p.tps, tiles = min(min(p.tiles_per_stream, tiles_s), i0 + p.tps);
+  if (i0 < tiles) issue(i0, 0);
   for (int i = i0; i < tiles; ++i) {
     const int st = (np.stages == 2) ? ((i - i0) & 1) : 0;
     // S of KV head g, dim tid, at the tile start
@@ -360,7 +381,7 @@ __global__ void __launch_bounds__(NT, 2) near_kernel(const PrefillParams p) {
     }
     __syncthreads();
     const long long t0 = pos0 + static_cast<long long>(i) * kTile;
-    const int Tt = static_cast<int>(min(static_cast<long long>(kTile), p.n - static_cast<long long>(i) * kTile));
+    const int Tt = static_cast<int>(min(static_cast<long long>(kTile), ns - static_cast<long long>(i) * kTile));
     const unsigned char* qs = smb + np.q[st];
     const unsigned char* ks = smb + np.k[st];
     const unsigned char* vs = smb + np.v[st];
@@ -482,6 +503,7 @@ near_tc_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ 
   if (!s_ok) return;  // latched by far_agg_kernel
   if (warp == 0) tmem_alloc(&s_tmem, kTmemNear);
   const long long pos0 = s_pos;
+  const long long ns = stream_len(p, s);  // tokens of this stream in the call
   const int K = p.K, nkv = p.nkv, g = h / p.G;
   const Tin* win_k = reinterpret_cast<const Tin*>(blk + p.so.win_k);
   const Tin* win_v = reinterpret_cast<const Tin*>(blk + p.so.win_v);
@@ -571,10 +593,12 @@ near_tc_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ 
   const uint32_t tmem = s_tmem;
   const uint32_t idesc_qk = umma_idesc_bf16(kTile, kNS, false);
   const uint32_t idesc_pv = umma_idesc_bf16(kTile, D, true);
-  const int i0 = seg * p.tps, tiles = min(p.tiles_per_stream, i0 + p.tps);  // this CTA's tiles
+  // this CTA's tiles (a ragged stream may end before them)
+  const int tiles_s = static_cast<int>((ns + kTile - 1) / kTile);
+  const int i0 = seg * p.tps, tiles = min(min(p.tiles_per_stream, tiles_s), i0 + p.tps);
   unsigned par = 0;
   bool ok = true;
-  issue(i0, 0);
+  if (i0 < tiles) issue(i0, 0);
   for (int i = i0; i < tiles; ++i) {
     const int st = (np.stages == 2) ? ((i - i0) & 1) : 0;
     const unsigned ld_par = static_cast<unsigned>(((np.stages == 2) ? ((i - i0) >> 1) : (i - i0)) & 1);
@@ -587,7 +611,7 @@ near_tc_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ 
     if (!mbar_wait_bounded(&s_ld[st], ld_par, kMbarPollLimit, p.err)) ok = false;
     if (i == 0) fix_history(st);  // the call's first tile (the copies above have landed)
     const long long t0 = pos0 + static_cast<long long>(i) * kTile;
-    const int Tt = static_cast<int>(min(static_cast<long long>(kTile), p.n - static_cast<long long>(i) * kTile));
+    const int Tt = static_cast<int>(min(static_cast<long long>(kTile), ns - static_cast<long long>(i) * kTile));
     const int r_ev = static_cast<int>(max(0LL, min(static_cast<long long>(Tt), K - t0)));
     if (r_ev != g_built) {  // uniform: the first tile of a stream start, then once more
       build_g(r_ev);
@@ -739,11 +763,11 @@ __global__ void __launch_bounds__(NT, 2) pool_kernel(const PrefillParams p) {
     mbar_fence_init();
   }
   __syncthreads();
-  if (!s_ok) return;
+  if (!s_ok || stream_len(p, s) <= static_cast<long long>(tile) * kTile) return;  // past a ragged stream's end
   if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
   const int l = p.l0 + s / p.B;
   const long long n0 = static_cast<long long>(tile) * kTile;
-  const int Tt = static_cast<int>(min(static_cast<long long>(kTile), p.n - n0));
+  const int Tt = static_cast<int>(min(static_cast<long long>(kTile), stream_len(p, s) - n0));
   const int nch = p.H / kBlk;
   const float* xrow0 = p.out + (static_cast<long long>(s) * p.n + n0) * p.H;
   const unsigned char* img_l = p.slot_img + static_cast<size_t>(l) * nch * 2 * kBlkBytes;
@@ -955,7 +979,8 @@ __global__ void __launch_bounds__(NT, 2) out_kernel(const PrefillParams p) {
     mbar_fence_init();
   }
   __syncthreads();
-  if (!s_ok) return;
+  const long long ns = stream_len(p, s);  // tokens of this stream in the call
+  if (!s_ok || ns == 0) return;          // an empty ragged stream keeps its state
   if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
   const long long pos0 = s_pos;
   const int l = p.l0 + s / p.B;
@@ -964,13 +989,14 @@ __global__ void __launch_bounds__(NT, 2) out_kernel(const PrefillParams p) {
   float* field = reinterpret_cast<float*>(blk + p.so.field);
   float* ring_sum = reinterpret_cast<float*>(blk + p.so.ring_sum);
   float* ring = reinterpret_cast<float*>(blk + p.so.ring);
-  const int tiles = p.tiles_per_stream;
-  const unsigned char* wall = p.ws + p.ws_w + static_cast<long long>(s) * tiles * 2 * kBlkBytes;
+  const int tiles = static_cast<int>((ns + kTile - 1) / kTile);
+  // the stream's pool weights (workspace pitch: the call's tiles per stream)
+  const unsigned char* wall = p.ws + p.ws_w + static_cast<long long>(s) * p.tiles_per_stream * 2 * kBlkBytes;
   const float ge = p.ema_gamma;
   const float a_l = p.alpha_layer[l];
 
   auto tile_rows = [&](int i) -> int {
-    return static_cast<int>(min(static_cast<long long>(kTile), p.n - static_cast<long long>(i) * kTile));
+    return static_cast<int>(min(static_cast<long long>(kTile), ns - static_cast<long long>(i) * kTile));
   };
   constexpr int XR = kHalo + kTile;  // rows of an x stage
   auto xstage = [&](int st) -> float* { return reinterpret_cast<float*>(smb + OutPlan::xt) + st * XR * kBlk; };
@@ -1088,7 +1114,7 @@ __global__ void __launch_bounds__(NT, 2) out_kernel(const PrefillParams p) {
     float rs = 0.f;
 #pragma unroll
     for (int u = 0; u < kRing; ++u) rs += xv[u];
-    float* orow = p.out + (in_row0 + (t0 - pos0) + r_lo) * p.H + col0 + cc;
+    const long long orow = (in_row0 + (t0 - pos0) + r_lo) * p.H + col0 + cc;  // result element of token r_lo
 #pragma unroll
     for (int u = 0; u < kSegLen; ++u) {
       if (u > 0) rs += xv[kHalo + u] - xv[u - 1];
@@ -1098,7 +1124,7 @@ __global__ void __launch_bounds__(NT, 2) out_kernel(const PrefillParams p) {
       f = live ? fn : f;
       float uu = rs * (1.0f / kRing) + 0.5f * f + 0.5f * sv[u];
       uu = fminf(fmaxf(uu, -p.clip_eps), p.clip_eps);
-      if (live && ok) orow[static_cast<long long>(u) * p.H] = fmaf(a_l, uu, x);
+      if (live && ok) store_result(p.out_mode, p.res, orow + static_cast<long long>(u) * p.H, a_l, uu, x);
     }
     const bool seg_last = r_lo < Tt && r_lo + kSegLen >= Tt;  // this segment holds the tile's last token
     if (i == tiles - 1 && ok) {
@@ -1135,7 +1161,7 @@ __global__ void __launch_bounds__(NT, 2) out_kernel(const PrefillParams p) {
     const int D = p.H / p.nq;
     const float* sfin = reinterpret_cast<const float*>(p.ws + p.ws_sfin) + static_cast<long long>(s) * p.nkv * D;
     for (int idx = tid; idx < p.nkv * D; idx += NT) far[idx] = sfin[idx];
-    const long long t_end = pos0 + p.n - 1;
+    const long long t_end = pos0 + ns - 1;
     const long long w0 = max(pos0, t_end - p.K + 1);
     const Tin* kin = static_cast<const Tin*>(p.k) + in_row0 * p.nkv * D;
     const Tin* vin = static_cast<const Tin*>(p.v) + in_row0 * p.nkv * D;
@@ -1146,7 +1172,7 @@ __global__ void __launch_bounds__(NT, 2) out_kernel(const PrefillParams p) {
       win_k[(j % p.K) * row + e] = kin[(j - pos0) * row + e];
       win_v[(j % p.K) * row + e] = vin[(j - pos0) * row + e];
     }
-    if (tid == 0) *reinterpret_cast<long long*>(b2 + p.so.pos) = pos0 + p.n;
+    if (tid == 0) *reinterpret_cast<long long*>(b2 + p.so.pos) = pos0 + ns;
   }
   tc_fence_before();
   __syncthreads();

@@ -54,7 +54,7 @@ int static_ws_address(void** out) {
 extern "C" {
 
 int sfa_prefill_static_ws(const sfa_handle* h, const void* q, const void* k, const void* v,
-                          long long n, int batch, void* state, float* out, void* stream) {
+                          long long n, int batch, void* state, void* out, void* stream) {
   if (n < 0 || batch <= 0) return SFA_ERR_INVALID_ARG;
   if (n == 0) return SFA_OK;
   const size_t need = sfa_prefill_workspace_bytes(h, batch, n);

@@ -68,6 +68,8 @@ int main(void) {
   CHECK(sfa_check_device_status(NULL, NULL) == SFA_ERR_INVALID_ARG);
   CHECK(sfa_debug_set_wait_limit(NULL, 0, -1) == SFA_ERR_INVALID_ARG);
   CHECK(sfa_debug_set_paths(NULL, -1, 1) == SFA_ERR_INVALID_ARG);
+  CHECK(sfa_set_output_mode(NULL, SFA_OUT_BF16) == SFA_ERR_INVALID_ARG);
+  CHECK(sfa_prefill_ragged(NULL, NULL, NULL, NULL, 1, NULL, 1, NULL, NULL, NULL, 0, NULL) == SFA_ERR_INVALID_ARG);
 
   printf("ok\n");
   return 0;
