@@ -315,7 +315,10 @@ SFA_API int sfa_prefill_ragged(const sfa_handle* h, const void* q, const void* k
  * SFA_STATIC_WORKSPACE_BYTES that every GPU loading the library holds until
  * the process exits; nothing is allocated or freed.  The first call on a
  * device looks up the array's device address (with that device current)
- * and caches it, so make that first call before any stream capture.  Every
+ * and caches it; the runtime reserves the array on the device at that
+ * point (device arrays of the library are loaded lazily), so the first call
+ * may allocate and synchronise once: make it before any stream capture and
+ * outside any region that must not allocate.  Every
  * call on a device shares the array, which keeps the last call's contents
  * (nothing in it has to start at zero), and calls that overlap on the GPU
  * (other streams, other host threads) race on it.  Returns SFA_ERR_WORKSPACE when

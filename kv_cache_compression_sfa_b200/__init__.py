@@ -464,10 +464,18 @@ class SfaOperator:
             self._ensure_workspace(max_prefill)
         self.reset()
 
-    def _ensure_workspace(self, n: int):
-        need = sfa_prefill_workspace_bytes(self.handle, self.batch, n)
+    def _grow_workspace(self, need: int, stream=None):
+        """A workspace of at least `need` bytes.  The buffer it replaces may
+        still be in use by work enqueued on `stream`: it is marked as used
+        there, so the caching allocator hands it out again only after that
+        work."""
         if self.workspace is None or self.workspace.numel() < need:
+            if self.workspace is not None and isinstance(stream, torch.cuda.Stream):
+                self.workspace.record_stream(stream)
             self.workspace = torch.empty(need, dtype=torch.uint8, device=self.device)
+
+    def _ensure_workspace(self, n: int, stream=None):
+        self._grow_workspace(sfa_prefill_workspace_bytes(self.handle, self.batch, n), stream)
 
     def reset(self, stream=None):
         sfa_state_reset(self.handle, self.state, self.batch, stream)
@@ -475,18 +483,23 @@ class SfaOperator:
     def set_output_mode(self, mode: int) -> None:
         sfa_set_output_mode(self.handle, mode)
 
-    def _new_out(self, shape):
+    def _new_out(self, shape, stream=None):
+        """A result buffer allocated on the current stream; if the call runs
+        on another stream it is marked as used there too."""
         if self.handle.out_mode in (SFA_OUT_ADD_F32, SFA_OUT_ADD_BF16):
             raise ValueError("the add output modes need out: it holds the attention output")
-        return torch.empty(shape, dtype=self.handle.out_dtype, device=self.device)
+        out = torch.empty(shape, dtype=self.handle.out_dtype, device=self.device)
+        if isinstance(stream, torch.cuda.Stream):
+            out.record_stream(stream)
+        return out
 
     def prefill(self, q, k, v, out: Optional[torch.Tensor] = None, stream=None):
         n = q.shape[2]
         c = self.cfg
         if out is None:
-            out = self._new_out((c.n_layers, self.batch, n, c.hidden))
+            out = self._new_out((c.n_layers, self.batch, n, c.hidden), stream)
         if n > 0:
-            self._ensure_workspace(n)
+            self._ensure_workspace(n, stream)
             sfa_prefill(self.handle, q, k, v, n, self.batch, self.state, out, self.workspace,
                         stream)
         return out
@@ -499,9 +512,11 @@ class SfaOperator:
         n = q.shape[2]
         c = self.cfg
         if out is None:
-            out = self._new_out((c.n_layers, self.batch, n, c.hidden)).fill_(float("nan"))
+            out = self._new_out((c.n_layers, self.batch, n, c.hidden), stream).fill_(float("nan"))
+            if isinstance(stream, torch.cuda.Stream):
+                stream.wait_stream(torch.cuda.current_stream())  # the fill comes first
         if n > 0:
-            self._ensure_workspace(n)
+            self._ensure_workspace(n, stream)
             sfa_prefill_ragged(self.handle, q, k, v, n, lens, self.batch, self.state, out,
                                self.workspace, stream)
         return out
@@ -511,7 +526,7 @@ class SfaOperator:
         sfa_decode_step, with the per-operator constants looked up once."""
         if out is None:
             c = self.cfg
-            out = self._new_out((c.n_layers, self.batch, c.hidden))
+            out = self._new_out((c.n_layers, self.batch, c.hidden), stream)
         nq, nkv, nout = self._dec_numel
         dt = self._in_dtype
         rc = self._decode_fn(self.handle.ptr, _dev(q, "q", dt, nq), _dev(k, "k", dt, nkv),
@@ -527,11 +542,10 @@ class SfaOperator:
         """Prefill of layers layer_begin .. layer_begin + q.shape[0] - 1."""
         lc, n = q.shape[0], q.shape[2]
         if out is None:
-            out = self._new_out((lc, self.batch, n, self.cfg.hidden))
+            out = self._new_out((lc, self.batch, n, self.cfg.hidden), stream)
         if n > 0:
-            need = sfa_prefill_layers_workspace_bytes(self.handle, lc, self.batch, n)
-            if self.workspace is None or self.workspace.numel() < need:
-                self.workspace = torch.empty(need, dtype=torch.uint8, device=self.device)
+            self._grow_workspace(sfa_prefill_layers_workspace_bytes(self.handle, lc, self.batch, n),
+                                 stream)
             sfa_prefill_layers(self.handle, layer_begin, lc, q, k, v, n, self.batch, self.state,
                                out, self.workspace, stream)
         return out
@@ -542,7 +556,7 @@ class SfaOperator:
         sequences in seq_ids (int32, on the device; None = all)."""
         lc, ns = q.shape[0], q.shape[1]
         if out is None:
-            out = self._new_out((lc, ns, self.cfg.hidden))
+            out = self._new_out((lc, ns, self.cfg.hidden), stream)
         sfa_decode_step_ex(self.handle, layer_begin, lc, seq_ids, q, k, v, self.batch,
                            self.state, out, stream)
         return out

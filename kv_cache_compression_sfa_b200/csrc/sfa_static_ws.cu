@@ -7,9 +7,12 @@
 // steady state because an allocation can synchronise the device.  For them,
 // the prefill's scratch (stream positions, the far state at the end of the
 // call and the pool weights of every tile) lives in one file-scope device
-// array of fixed size, reserved when the library is loaded and held by every
-// GPU that loads it until the process exits.  The caller still passes
-// inputs, outputs and the state.
+// array of fixed size, held by every GPU that loads it until the process
+// exits.  The caller still passes inputs, outputs and the state.  The CUDA
+// runtime loads a module's device arrays lazily: the array is reserved on a
+// device when its address is first looked up, which the first call on that
+// device does (it may allocate and synchronise there, once), so that first
+// call belongs before any stream capture.
 //
 // The work itself is exactly sfa_prefill's: this entry point only supplies
 // the array's device address as the workspace.
@@ -55,7 +58,8 @@ extern "C" {
 
 int sfa_prefill_static_ws(const sfa_handle* h, const void* q, const void* k, const void* v,
                           long long n, int batch, void* state, void* out, void* stream) {
-  if (n < 0 || batch <= 0) return SFA_ERR_INVALID_ARG;
+  // the same argument checks, in the same order, as sfa_prefill
+  if (n < 0 || batch <= 0 || sfa_prefill_workspace_bytes(h, 1, 1) == 0) return SFA_ERR_INVALID_ARG;
   if (n == 0) return SFA_OK;
   const size_t need = sfa_prefill_workspace_bytes(h, batch, n);
   // 0: a bad handle or a call beyond sfa_prefill's limits; sfa_prefill
