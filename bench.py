@@ -74,6 +74,10 @@ def parse():
                     help="instead of the bench line: state footprint and decode time against "
                          "the context, or the enhancement share and its angle to x")
     ap.add_argument("--max-context", type=int, default=65536)
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the workload's batch (smaller cases for profiling)")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="override the workload's layer count (smaller cases for profiling)")
     return ap.parse_args()
 
 
@@ -683,8 +687,12 @@ def main():
     if args.report:
         run_report(args)
         return
-    headline_default = args.workload == HEADLINE
+    headline_default = args.workload == HEADLINE and not args.batch and not args.layers
     w = get_workload(args.workload)
+    if args.batch:
+        w = w.replace(batch=args.batch)
+    if args.layers:
+        w = w.replace(n_layers=args.layers)
     n_pre = args.context or w.prefill_n[0]
     if args.impl == "reference":
         run_reference(args, w, n_pre)

@@ -116,19 +116,34 @@ std::vector<int> cluster_candidates(int nq, int d) {
 // Workspace of a prefill call: the streams' positions, S at the end of the
 // call, the pool weights of every tile (two 8 KB bf16 blocks) and S at
 // every tile start.
-PrefillWorkspace prefill_workspace(const sfa_config* c, int layers, int batch, long long n, int out_mode) {
+// Segments of the output kernel's tile walk: about four rounds of two CTAs
+// per SM over (stream, 64-column block, segment).
+int out_segments(int n_sm, int hidden, long long streams, long long tiles_per_stream) {
+  const long long units = streams * (hidden / 64);
+  const long long target = 4LL * 2 * std::max(n_sm, 1);
+  long long nseg = std::max(1LL, std::min(tiles_per_stream, (target + units - 1) / units));
+  const long long tps = (tiles_per_stream + nseg - 1) / nseg;
+  return static_cast<int>((tiles_per_stream + tps - 1) / tps);
+}
+
+PrefillWorkspace prefill_workspace(const sfa_config* c, int layers, int batch, long long n, int out_mode,
+                                   int n_sm) {
   PrefillWorkspace w;
   const long long streams = static_cast<long long>(layers) * batch;
-  const long long tiles = streams * ((n + kTile - 1) / kTile);
+  const long long tps = (n + kTile - 1) / kTile;
+  const long long tiles = streams * tps;
   const long long sdim = static_cast<long long>(c->n_kv_heads) * c->head_dim;
+  const long long H = hidden_of(c);
   w.pos = 0;
   w.sfin = align256(8 * streams);
   w.w = w.sfin + align256(4 * streams * sdim);
   w.sst = w.w + tiles * 2LL * kBlkBytesHost;
   w.x = w.sst + align256(4 * tiles * sdim);
   // x between the kernels, where the result buffer cannot hold it
-  const long long xb = out_mode == SFA_OUT_F32 ? 0 : align256(4LL * streams * n * hidden_of(c));
-  w.total = w.x + xb;
+  const long long xb = out_mode == SFA_OUT_F32 ? 0 : align256(4LL * streams * n * H);
+  w.fagg = w.x + xb;
+  w.halo = w.fagg + align256(4LL * tiles * H);
+  w.total = w.halo + align256(4LL * streams * out_segments(n_sm, static_cast<int>(H), streams, tps) * kHalo * H);
   return w;
 }
 
@@ -402,7 +417,7 @@ size_t sfa_prefill_layers_workspace_bytes(const sfa_handle* h, int layer_count, 
       layer_count > h->cfg.n_layers)
     return 0;
   if (prefill_shape_status(layer_count, batch, n) != SFA_OK) return 0;
-  return static_cast<size_t>(prefill_workspace(&h->cfg, layer_count, batch, n, h->out_mode).total);
+  return static_cast<size_t>(prefill_workspace(&h->cfg, layer_count, batch, n, h->out_mode, h->n_sm).total);
 }
 
 int sfa_state_reset(const sfa_handle* h, void* state, int batch, void* stream) {
@@ -464,7 +479,7 @@ int prefill_impl(const sfa_handle* h, int layer_begin, int layer_count, const vo
   const int shape = prefill_shape_status(layer_count, batch, n);
   if (shape != SFA_OK) return shape;
   const sfa_config* c = &h->cfg;
-  const PrefillWorkspace w = prefill_workspace(c, layer_count, batch, n, h->out_mode);
+  const PrefillWorkspace w = prefill_workspace(c, layer_count, batch, n, h->out_mode, h->n_sm);
   if (!workspace || workspace_bytes < static_cast<size_t>(w.total)) return SFA_ERR_WORKSPACE;
   const long long streams = static_cast<long long>(layer_count) * batch;
   const long long tiles_per_stream = (n + kTile - 1) / kTile;
@@ -493,6 +508,10 @@ int prefill_impl(const sfa_handle* h, int layer_begin, int layer_count, const vo
   p.ws_w = w.w;
   p.ws_sst = w.sst;
   p.ws_x = w.x;
+  p.ws_fagg = w.fagg;
+  p.ws_halo = w.halo;
+  p.nseg_out = out_segments(h->n_sm, hidden_of(c), streams, tiles_per_stream);
+  p.tps_out = static_cast<int>((tiles_per_stream + p.nseg_out - 1) / p.nseg_out);
   {
     // Near-field segments: about four rounds of two CTAs per SM, each CTA a
     // run of consecutive tiles of one (stream, head).

@@ -132,10 +132,12 @@ struct PrefillParams {
   int l0;                   // first layer of the state served (streams are l0*B + ...)
   int tiles_per_stream, n_streams;
   int n_seg, tps;           // near field: segments per stream, tiles per segment
+  int nseg_out, tps_out;    // output kernel: segments per stream, tiles per segment
   // workspace byte offsets: stream positions, S at the end of the call, pool
   // weights, far-field state at every tile start, x (output modes other
   // than SFA_OUT_F32)
   long long ws_pos, ws_sfin, ws_w, ws_sst, ws_x;
+  long long ws_fagg, ws_halo;  // EMA field over each tile from zero; x rows before each output segment
   float gamma_far, alpha_far, ema_gamma, inv_temp, clip_eps, score_scale;
   unsigned spin_limit;      // polls of a bounded wait before it gives up
   long long withhold_tile;  // test hook: this tile's pool CTA waits on a barrier nothing completes
@@ -157,6 +159,8 @@ struct PrefillWorkspace {
   long long w;      // [streams * tiles][hi, lo] 64 x 64 bf16 pool-weight blocks
   long long sst;    // [streams][tiles][n_kv][d] fp32 far state at every tile start
   long long x;      // [streams][n][H] fp32 x when the result is not fp32 x + enhancement (else 0)
+  long long fagg;   // [streams][tiles][H] fp32 EMA field over each tile, from zero
+  long long halo;   // [streams][output segments][15][H] fp32 x rows before each output segment
   long long total;
 };
 

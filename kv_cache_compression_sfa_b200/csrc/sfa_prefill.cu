@@ -772,6 +772,19 @@ __global__ void __launch_bounds__(NT, 2) pool_kernel(const PrefillParams p) {
   const float* xrow0 = p.out + (static_cast<long long>(s) * p.n + n0) * p.H;
   const unsigned char* img_l = p.slot_img + static_cast<size_t>(l) * nch * 2 * kBlkBytes;
   bool ok = true;
+  // The EMA field over the tile from zero [P3 §2.1 channel 2], per column:
+  // A = sum over tokens r of (1-g) g^(Tt-1-r) x_r, so that the field after
+  // the tile is g^Tt F + A; out_kernel's segments start from these.  The
+  // last tile of an output segment also keeps its last kHalo x rows, the
+  // ring window of the next segment's first tokens.
+  __shared__ float s_fw[kTile];
+  __shared__ __align__(16) float s_fpart[2][kBlk];  // read and written as float4
+  if (tid < kTile) s_fw[tid] = tid < Tt ? (1.0f - p.ema_gamma) * powf(p.ema_gamma, static_cast<float>(Tt - 1 - tid)) : 0.f;
+  float* fagg = reinterpret_cast<float*>(p.ws + p.ws_fagg) +
+                (static_cast<long long>(s) * p.tiles_per_stream + tile) * p.H;
+  const bool seg_end = (tile + 1) % p.tps_out == 0 && (tile + 1) * static_cast<long long>(kTile) < stream_len(p, s);
+  float* halo = reinterpret_cast<float*>(p.ws + p.ws_halo) +
+                (static_cast<long long>(s) * p.nseg_out + (tile + 1) / p.tps_out - 1) * kHalo * p.H;
 
   // Thread tid handles 4 columns c4 .. c4+3 of rows r_m (m = 0..3) of every
   // chunk.  The mapping makes a warp's split stores cover whole 128-byte
@@ -807,6 +820,7 @@ __global__ void __launch_bounds__(NT, 2) pool_kernel(const PrefillParams p) {
   const uint32_t idesc = umma_idesc_bf16(kBlk, kSlots, false);
 
   float sq[4] = {0.f, 0.f, 0.f, 0.f};  // |x|^2 of rows r_m over this thread's columns
+  float s_fpart_keep[4];                // this half's field aggregate of the current chunk
   for (int c = 0; c < nch; ++c) {
     float4 cur[4];
 #pragma unroll
@@ -831,9 +845,36 @@ __global__ void __launch_bounds__(NT, 2) pool_kernel(const PrefillParams p) {
       *reinterpret_cast<uint2*>(xhi + off) = *reinterpret_cast<const uint2*>(hh);
       *reinterpret_cast<uint2*>(xlo + off) = *reinterpret_cast<const uint2*>(ll);
     }
+    {  // field aggregate of the chunk's columns; halo rows of a segment end
+      float fa[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const float wgt = s_fw[row_of(m)];
+        fa[0] = fmaf(wgt, cur[m].x, fa[0]);
+        fa[1] = fmaf(wgt, cur[m].y, fa[1]);
+        fa[2] = fmaf(wgt, cur[m].z, fa[2]);
+        fa[3] = fmaf(wgt, cur[m].w, fa[3]);
+        if (seg_end && row_of(m) >= kTile - kHalo)
+          *reinterpret_cast<float4*>(halo + static_cast<long long>(row_of(m) - (kTile - kHalo)) * p.H + c * kBlk + c4) = cur[m];
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e)  // the 8 lanes of this warp that share the columns
+        for (int off = 1; off < 8; off <<= 1) fa[e] += __shfl_xor_sync(0xffffffffu, fa[e], off);
+      if ((tid & 7) == 0 && (tid >> 7) == 1)
+        *reinterpret_cast<float4*>(&s_fpart[c & 1][c4]) = make_float4(fa[0], fa[1], fa[2], fa[3]);
+      s_fpart_keep[0] = fa[0];
+      s_fpart_keep[1] = fa[1];
+      s_fpart_keep[2] = fa[2];
+      s_fpart_keep[3] = fa[3];
+    }
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();  // split blocks of chunk c written
+    if ((tid & 7) == 0 && (tid >> 7) == 0) {  // the other half of the rows is in s_fpart
+      const float4 o = *reinterpret_cast<const float4*>(&s_fpart[c & 1][c4]);
+      *reinterpret_cast<float4*>(fagg + c * kBlk + c4) =
+          make_float4(s_fpart_keep[0] + o.x, s_fpart_keep[1] + o.y, s_fpart_keep[2] + o.z, s_fpart_keep[3] + o.w);
+    }
     if (tid == 0) {
       const int si = c % 3;
       if (!mbar_wait_bounded(bar_img + si, static_cast<unsigned>((c / 3) & 1), kMbarPollLimit, p.err)) ok = false;
@@ -954,7 +995,10 @@ struct OutPlan {
 
 template <typename Tin>
 __global__ void __launch_bounds__(NT, 2) out_kernel(const PrefillParams p) {
-  const int cb = blockIdx.x, s = blockIdx.y;  // 64-column block, call-relative stream
+  const int ncb = p.H / kBlk;
+  const int cb = static_cast<int>(blockIdx.x) % ncb;   // 64-column block
+  const int seg = static_cast<int>(blockIdx.x) / ncb;  // segment of tiles
+  const int s = blockIdx.y;                            // call-relative stream
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   extern __shared__ __align__(16) unsigned char smb[];
   uint64_t* bar_img = reinterpret_cast<uint64_t*>(smb + OutPlan::bars);
@@ -980,7 +1024,10 @@ __global__ void __launch_bounds__(NT, 2) out_kernel(const PrefillParams p) {
   }
   __syncthreads();
   const long long ns = stream_len(p, s);  // tokens of this stream in the call
-  if (!s_ok || ns == 0) return;          // an empty ragged stream keeps its state
+  const int tiles = static_cast<int>((ns + kTile - 1) / kTile);
+  // this CTA's tiles: segment seg of the stream's tiles
+  const int i_begin = seg * p.tps_out, i_end = min(tiles, i_begin + p.tps_out);
+  if (!s_ok || i_begin >= i_end) return;  // an empty ragged stream keeps its state
   if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
   const long long pos0 = s_pos;
   const int l = p.l0 + s / p.B;
@@ -989,7 +1036,6 @@ __global__ void __launch_bounds__(NT, 2) out_kernel(const PrefillParams p) {
   float* field = reinterpret_cast<float*>(blk + p.so.field);
   float* ring_sum = reinterpret_cast<float*>(blk + p.so.ring_sum);
   float* ring = reinterpret_cast<float*>(blk + p.so.ring);
-  const int tiles = static_cast<int>((ns + kTile - 1) / kTile);
   // the stream's pool weights (workspace pitch: the call's tiles per stream)
   const unsigned char* wall = p.ws + p.ws_w + static_cast<long long>(s) * p.tiles_per_stream * 2 * kBlkBytes;
   const float ge = p.ema_gamma;
@@ -1020,17 +1066,45 @@ __global__ void __launch_bounds__(NT, 2) out_kernel(const PrefillParams p) {
     bulk_g2s(smb + OutPlan::img,
              p.slot_img + (static_cast<size_t>(l) * (p.H / kBlk) + cb) * 2 * kBlkBytes, 2u * kBlkBytes,
              bar_img);
-    issue_w(0, 0);
+    issue_w(i_begin, 0);
   }
-  issue_x(0, 0);
-  // x of the 15 positions before the call (state ring; zero before position
-  // 0) and the field carried in, for this block's columns.
-  for (int idx = tid; idx < kHalo * kBlk; idx += NT) {
-    const int q = idx / kBlk, c = idx % kBlk;
-    const long long t = pos0 - kHalo + q;
-    xstage(0)[idx] = t >= 0 ? ring[static_cast<size_t>(t % kRing) * p.H + col0 + c] : 0.f;
+  issue_x(i_begin, 0);
+  if (i_begin == 0) {
+    // x of the 15 positions before the call (state ring; zero before
+    // position 0) and the field carried in, for this block's columns.
+    for (int idx = tid; idx < kHalo * kBlk; idx += NT) {
+      const int q = idx / kBlk, c = idx % kBlk;
+      const long long t = pos0 - kHalo + q;
+      xstage(0)[idx] = t >= 0 ? ring[static_cast<size_t>(t % kRing) * p.H + col0 + c] : 0.f;
+    }
+    if (tid < kBlk) fcar[tid] = field[col0 + tid];
+  } else {
+    // a later segment: the last x rows of the previous segment, kept by
+    // pool_kernel, and the field folded over the tiles before it (all full:
+    // field after tile i = g^64 field + A_i)
+    const float* halo = reinterpret_cast<const float*>(p.ws + p.ws_halo) +
+                        (static_cast<long long>(s) * p.nseg_out + seg - 1) * kHalo * p.H + col0;
+    for (int idx = tid; idx < kHalo * kBlk; idx += NT) {
+      const int q = idx / kBlk, c = idx % kBlk;
+      xstage(0)[idx] = halo[static_cast<long long>(q) * p.H + c];
+    }
+    if (tid < kBlk) {
+      const float g64 = powf(ge, static_cast<float>(kTile));
+      const float* agg = reinterpret_cast<const float*>(p.ws + p.ws_fagg) +
+                         static_cast<long long>(s) * p.tiles_per_stream * p.H + col0 + tid;
+      float f = field[col0 + tid];
+      constexpr int kAhead = 8;  // aggregates in flight
+      for (int i8 = 0; i8 < i_begin; i8 += kAhead) {
+        float av[kAhead];
+#pragma unroll
+        for (int u = 0; u < kAhead; ++u) av[u] = i8 + u < i_begin ? agg[static_cast<long long>(i8 + u) * p.H] : 0.f;
+#pragma unroll
+        for (int u = 0; u < kAhead; ++u)
+          if (i8 + u < i_begin) f = fmaf(g64, f, av[u]);
+      }
+      fcar[tid] = f;
+    }
   }
-  if (tid < kBlk) fcar[tid] = field[col0 + tid];
   if (tid < kSeg) s_gseg[tid] = powf(ge, static_cast<float>(kSegLen));
   tc_fence_before();
   __syncthreads();
@@ -1041,11 +1115,11 @@ __global__ void __launch_bounds__(NT, 2) out_kernel(const PrefillParams p) {
   if (!mbar_wait_bounded(bar_img, 0, kMbarPollLimit, p.err)) ok = false;
 
   const int cc = tid % kBlk, sg = tid / kBlk;  // column, token segment
-  for (int i = 0; i < tiles; ++i) {
-    const int st = i & 1;
+  for (int i = i_begin; i < i_end; ++i) {
+    const int st = (i - i_begin) & 1;
     const int Tt = tile_rows(i);
     const long long t0 = pos0 + static_cast<long long>(i) * kTile;
-    if (i + 1 < tiles) {
+    if (i + 1 < i_end) {
       issue_x(i + 1, st ^ 1);  // stage st^1 was released at the end of tile i-1
       if (tid == 0) issue_w(i + 1, st ^ 1);
       cp_async_wait<1>();
@@ -1054,7 +1128,7 @@ __global__ void __launch_bounds__(NT, 2) out_kernel(const PrefillParams p) {
     }
     // sem[T x 64] = w[T x 64 slots] . slot block [64 slots x 64 columns]
     if (tid == 0) {
-      if (!mbar_wait_bounded(bar_w + st, static_cast<unsigned>((i >> 1) & 1), kMbarPollLimit, p.err)) ok = false;
+      if (!mbar_wait_bounded(bar_w + st, static_cast<unsigned>(((i - i_begin) >> 1) & 1), kMbarPollLimit, p.err)) ok = false;
       tc_fence_after();
       const unsigned char* whi = smb + OutPlan::wb + st * 2 * kBlkBytes;
       const unsigned char* wlo = whi + kBlkBytes;
@@ -1090,7 +1164,7 @@ __global__ void __launch_bounds__(NT, 2) out_kernel(const PrefillParams p) {
       }
       segc[sg * kBlk + cc] = a;
     }
-    if (!mbar_wait_bounded(bar_mma, static_cast<unsigned>(i & 1), kMbarPollLimit, p.err)) ok = false;
+    if (!mbar_wait_bounded(bar_mma, static_cast<unsigned>((i - i_begin) & 1), kMbarPollLimit, p.err)) ok = false;
     tc_fence_after();
     {  // accumulator row r (token) sits in lane (r%16) + 32*(r/16) for M = 64
       const int sp = warp & 3, colh = (warp >> 2) * 32;
@@ -1127,7 +1201,7 @@ __global__ void __launch_bounds__(NT, 2) out_kernel(const PrefillParams p) {
       if (live && ok) store_result(p.out_mode, p.res, orow + static_cast<long long>(u) * p.H, a_l, uu, x);
     }
     const bool seg_last = r_lo < Tt && r_lo + kSegLen >= Tt;  // this segment holds the tile's last token
-    if (i == tiles - 1 && ok) {
+    if (i == tiles - 1 && ok) {  // the stream's last tile (in the last segment)
       const int gi = col0 + cc;
       if (seg_last) field[gi] = f;
       if (sg == 0) {
@@ -1147,13 +1221,13 @@ __global__ void __launch_bounds__(NT, 2) out_kernel(const PrefillParams p) {
     }
     __syncthreads();  // segc and fcar are read above
     if (seg_last) fcar[cc] = f;
-    if (i + 1 < tiles)  // the tile's last 15 x rows lead the next stage (Tt = 64 here)
+    if (i + 1 < i_end)  // the tile's last 15 x rows lead the next stage (Tt = 64 here)
       for (int idx = tid; idx < kHalo * kBlk; idx += NT) xstage(st ^ 1)[idx] = xb[kTile * kBlk + idx];
     __syncthreads();  // the x stage, halo rows and carries are ready for the next tile
   }
 
-  // One CTA per stream: window, S and position [P1 §2.2].
-  if (cb == 0 && ok) {
+  // One CTA per stream (the last segment's): window, S and position [P1 §2.2].
+  if (cb == 0 && i_end == tiles && ok) {
     unsigned char* b2 = blk;
     Tin* win_k = reinterpret_cast<Tin*>(b2 + p.so.win_k);
     Tin* win_v = reinterpret_cast<Tin*>(b2 + p.so.win_v);
@@ -1252,7 +1326,7 @@ cudaError_t launch_t(const PrefillParams& p, cudaStream_t s) {
   const dim3 gc(static_cast<unsigned>((ne + NT - 1) / NT), ns, 1);
   const dim3 g1(static_cast<unsigned>(p.nq * p.n_seg), ns, 1);
   const dim3 g2(static_cast<unsigned>(p.tiles_per_stream), ns, 1);
-  const dim3 g3(static_cast<unsigned>(p.H / kBlk), ns, 1);
+  const dim3 g3(static_cast<unsigned>((p.H / kBlk) * p.nseg_out), ns, 1);
   cudaError_t e = launch_pdl(far_agg_kernel<Tin, D>, g0, 4 * ne * 4, s, p);
   if (e == cudaSuccess) e = launch_pdl(far_carry_kernel, gc, 0, s, p);
   if (e != cudaSuccess) return e;
