@@ -36,6 +36,7 @@
 //
 // Every wait is bounded; a wait that runs out latches SFA_ERR_DEVICE_TIMEOUT
 // and the kernel still finishes.
+#include <cooperative_groups.h>
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 
@@ -44,6 +45,8 @@
 
 #include "sfa_common.cuh"
 #include "sfa_umma.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace sfa {
 namespace {
@@ -667,102 +670,115 @@ decode_near_mma_kernel(const __grid_constant__ DecodeParams p, const __grid_cons
 constexpr int NTC = 256;                // pool kernel: compute threads (8 warps)
 constexpr int NWC = NTC / 32;
 constexpr int NTP = NTC + 32;           // plus the MMA warp
-constexpr int TR = 16;                  // sequences per pool CTA (rows of the MMAs' M = 64)
-constexpr int kSlotStages = 3;
-constexpr int kABufs = 2;               // split x blocks
-constexpr int kSemBufs = 2;             // sem accumulators in tensor memory and their staging
-constexpr int kScStride = kSlots + 1;
+constexpr int TR = 16;                  // sequences per CTA pair: the N = 16 of the MMAs
+constexpr int kPair = 2;                // CTAs of a cluster: halves of the hidden columns
+constexpr int kSlotStages = 4;
+constexpr int kABufs = 4;               // split x^T blocks
+constexpr int kSemBufs = 4;             // sem^T accumulators and their staging
+constexpr int kScStride = kSlots + 1;   // 64 scores + |x|^2 per row
 constexpr int kSemStride = kBlk + 4;
-constexpr int kTmemCols = 256;          // scores (64) + two 64-column sem buffers
+constexpr int kTmemCols = 128;          // scores^T (16) + four 16-column sem^T buffers
+constexpr int kTmemSem = 32;
 static_assert(TR * 16 == NTC, "pool kernel: 16 threads per row, 4 columns each");
 
 // Pool CTA shared memory (byte offsets).
 struct PoolTilePlan {
-  static constexpr int bars = 0;                                     // mbarriers, tmem address
-  static constexpr int a = 512;                                      // [2][hi, lo] x blocks
-  static constexpr int w = a + kABufs * 2 * kBlkBytes;               // [hi, lo] weight block
-  static constexpr int sl = w + 2 * kBlkBytes;                       // [3][hi, lo] slot blocks
-  static constexpr int sem = sl + kSlotStages * 2 * kBlkBytes;       // [2][16][68] sem chunks
-  static constexpr int sc = sem + kSemBufs * TR * kSemStride * 4;    // [16][65] scores
-  static constexpr int total = sc + TR * kScStride * 4;
+  static constexpr int bars = 0;                                  // mbarriers, tmem address
+  static constexpr int sl = 1024;                                 // [4][hi, lo] slot blocks
+  static constexpr int xt = sl + kSlotStages * 2 * kBlkBytes;     // [4][hi, lo] x^T blocks [16 x 64]
+  static constexpr int wt = xt + kABufs * 2 * kBlk16Bytes;        // [hi, lo] w^T block [16 x 64]
+  static constexpr int sem = wt + 2 * kBlk16Bytes;                // [4][16][68] sem chunks
+  static constexpr int sc = sem + kSemBufs * TR * kSemStride * 4; // [16][65] own partial scores, |x|^2
+  static constexpr int scp = sc + TR * kScStride * 4;             // [16][65] the peer CTA's partial
+  static constexpr int total = scp + TR * kScStride * 4;
 };
 // barrier slots (arrival counts in brackets)
-constexpr int kPbSlFull = 0;                           // [3] slot block landed (1 + bytes)
-constexpr int kPbSlEmpty = kPbSlFull + kSlotStages;    // [3] MMAs done with a slot block (commit)
-constexpr int kPbAFull = kPbSlEmpty + kSlotStages;     // [2] x block written (8 warps)
-constexpr int kPbAEmpty = kPbAFull + kABufs;           // [2] MMAs done with an x block (commit)
+constexpr int kPbSlFull = 0;                           // [4] slot block landed (1 + bytes)
+constexpr int kPbSlEmpty = kPbSlFull + kSlotStages;    // [4] MMAs done with a slot block (commit)
+constexpr int kPbAFull = kPbSlEmpty + kSlotStages;     // [4] x^T block written (8 warps)
+constexpr int kPbAEmpty = kPbAFull + kABufs;           // [4] MMAs done with an x^T block (commit)
 constexpr int kPbScores = kPbAEmpty + kABufs;          // all score MMAs done (commit)
-constexpr int kPbWFull = kPbScores + 1;                // weight block written (8 warps)
-constexpr int kPbSemFull = kPbWFull + 1;               // [2] sem accumulator ready (commit)
-constexpr int kPbSemEmpty = kPbSemFull + kSemBufs;     // [2] sem accumulator read (2 warps)
-constexpr int kPbStFull = kPbSemEmpty + kSemBufs;      // [2] sem chunk staged (2 warps)
-constexpr int kPbStEmpty = kPbStFull + kSemBufs;       // [2] staged chunk used (8 warps)
+constexpr int kPbWFull = kPbScores + 1;                // w^T block written (8 warps)
+constexpr int kPbSemFull = kPbWFull + 1;               // [4] sem accumulator ready (commit)
+constexpr int kPbSemEmpty = kPbSemFull + kSemBufs;     // [4] sem accumulator read (4 warps)
+constexpr int kPbStFull = kPbSemEmpty + kSemBufs;      // [4] sem chunk staged (4 warps)
+constexpr int kPbStEmpty = kPbStFull + kSemBufs;       // [4] staged sem chunk used (8 warps)
 constexpr int kPbCount = kPbStEmpty + kSemBufs;
-static_assert(kPbCount * 8 + 4 <= PoolTilePlan::a, "barriers fit");
+static_assert(kPbCount * 8 + 4 <= PoolTilePlan::sl, "barriers fit");
 
-// Pass 1 and pass 2 run as a pipeline without CTA-wide barriers: warp 8
-// (one lane) loads the slot blocks and issues every MMA; warps 0-7 split x
-// into the MMA blocks, then run the epilogue; warps 0 and 4, which can read
-// tensor-memory lanes 0-15 (rows 0-15 of an M = 64 accumulator), stage each
-// sem chunk in shared memory for the others.  mbarriers carry every
-// hand-off.
-__global__ void __launch_bounds__(NTP, 2) decode_pool_kernel(const __grid_constant__ DecodeParams p) {
+// A cluster of two CTAs serves 16 sequences of one layer; CTA `rank` owns
+// the hidden columns of chunks [c0, c0 + nloc).  The 16 sequences are the
+// N = 16 of transposed MMAs: scores^T[64 slots x 16] += slot_c . x_c^T and
+// sem^T[64 columns x 16] = slot_c^T . w^T, split bf16 operands (hi*hi +
+// hi*lo + lo*hi), fp32 accumulators in tensor memory.  The two CTAs add
+// their partial scores and |x|^2 through distributed shared memory and both
+// form the same softmax weights.  Warp 8 (one lane) loads the slot blocks
+// and issues every MMA; warps 0-7 split x (pass 1) and run the epilogue
+// with x and the state rows two chunks ahead in registers (pass 2); warps
+// 0-3, which hold the accumulator lanes, stage each sem chunk for the
+// others.  mbarriers carry every hand-off.
+__global__ void __cluster_dims__(kPair, 1, 1) __launch_bounds__(NTP, 2)
+decode_pool_kernel(const __grid_constant__ DecodeParams p) {
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = static_cast<int>(cluster.block_rank());
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int tiles_per_layer = (p.n_seq + TR - 1) / TR;
-  const int li = static_cast<int>(blockIdx.x) / tiles_per_layer;
-  const int tb = static_cast<int>(blockIdx.x) % tiles_per_layer;
+  const int pair = static_cast<int>(blockIdx.x) / kPair;
+  const int li = pair / tiles_per_layer;
+  const int tb = pair % tiles_per_layer;
   const int l = p.l0 + li;
   const int nch = p.H / kBlk;
-  extern __shared__ __align__(128) unsigned char smb_raw[];
-  unsigned char* sm = aligned128(smb_raw);
+  const int half = (nch + 1) / 2;
+  const int c0 = rank == 0 ? 0 : half;
+  const int nloc = rank == 0 ? half : nch - half;  // chunks of this CTA
+  extern __shared__ __align__(128) unsigned char smb_pool[];
+  unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smb_pool) + 127) &
+                                                       ~static_cast<uintptr_t>(127));
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + PoolTilePlan::bars);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kPbCount);
-  unsigned char* ablk = sm + PoolTilePlan::a;
-  unsigned char* wblk = sm + PoolTilePlan::w;
   unsigned char* slb = sm + PoolTilePlan::sl;
-  float* sc = reinterpret_cast<float*>(sm + PoolTilePlan::sc);
+  unsigned char* xtb = sm + PoolTilePlan::xt;
+  unsigned char* wtb = sm + PoolTilePlan::wt;
   float* semst = reinterpret_cast<float*>(sm + PoolTilePlan::sem);
+  float* sc = reinterpret_cast<float*>(sm + PoolTilePlan::sc);
+  float* scp = reinterpret_cast<float*>(sm + PoolTilePlan::scp);
   __shared__ long long s_st[TR], s_pos[TR];
-  __shared__ float s_ssq[TR][2];
   __shared__ int s_ok;
 
   const unsigned char* img_l = p.slot_img + static_cast<size_t>(l) * nch * 2 * kBlkBytes;
-  // Slot block loads q = 0 .. 2*nch-1 (pass 1, then pass 2) through the
-  // three stages: load q is block q % nch in stage q % 3.
+  // Slot block loads q = 0 .. 2*nloc-1 (pass 1, then pass 2): load q is
+  // block c0 + q % nloc in stage q % 4.
   auto issue_slot = [&](int q) {  // the MMA lane
     const int st = q % kSlotStages;
     mbar_arrive_expect_tx(bars + kPbSlFull + st, 2u * kBlkBytes);
-    bulk_g2s(slb + st * 2 * kBlkBytes, img_l + static_cast<size_t>(q % nch) * 2 * kBlkBytes, 2u * kBlkBytes,
-             bars + kPbSlFull + st);
+    bulk_g2s(slb + st * 2 * kBlkBytes, img_l + static_cast<size_t>(c0 + q % nloc) * 2 * kBlkBytes,
+             2u * kBlkBytes, bars + kPbSlFull + st);
   };
   if (tid == 0) {
     for (int i = 0; i < kPbCount; ++i) {
-      const bool by_warps = i == kPbWFull || (i >= kPbAFull && i < kPbAFull + kABufs) ||
-                            (i >= kPbStEmpty && i < kPbStEmpty + kSemBufs);
-      const bool by_readers = (i >= kPbSemEmpty && i < kPbSemEmpty + kSemBufs) ||
-                              (i >= kPbStFull && i < kPbStFull + kSemBufs);
-      mbar_init(bars + i, by_warps ? NWC : by_readers ? 2 : 1);
+      int count = 1;
+      if ((i >= kPbAFull && i < kPbAFull + kABufs) || i == kPbWFull || (i >= kPbStEmpty && i < kPbStEmpty + kSemBufs))
+        count = NWC;
+      if ((i >= kPbSemEmpty && i < kPbSemEmpty + kSemBufs) || (i >= kPbStFull && i < kPbStFull + kSemBufs)) count = 4;
+      mbar_init(bars + i, count);
     }
     mbar_fence_init();
   }
   if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);  // at most two CTAs per SM: never waits
-  // rows 16..63 of the x and weight blocks stay zero
-  for (int i = tid; i < (kABufs * 2 + 2) * kBlkBytes / 16; i += NTP) {
-    const int bi = i / (kBlkBytes / 16), rem = i % (kBlkBytes / 16);
-    unsigned char* base = (bi < kABufs * 2 ? ablk + bi * kBlkBytes : wblk + (bi - kABufs * 2) * kBlkBytes);
-    reinterpret_cast<uint4*>(base)[rem] = make_uint4(0u, 0u, 0u, 0u);
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  if (tid == NTC) {
+  // The peer writes into this CTA's shared memory only after every CTA of
+  // the cluster has started: arrive now, wait before the exchange.
+  cluster_arrive();
+  if (warp == NWC && lane == 0) {
     // the slot blocks are constant since sfa_init: the first loads go out
     // before the wait for the previous kernel
-    for (int q = 0; q < kSlotStages && q < 2 * nch; ++q) issue_slot(q);
+    for (int q = 0; q < kSlotStages && q < 2 * nloc; ++q) issue_slot(q);
   }
   pdl_trigger();
-  pdl_wait();  // x from decode_near_kernel; the state
+  pdl_wait();  // x from the near-field kernel; the state
 
   if (tid == 0) {
     const uint4 h0v = __ldcg(reinterpret_cast<const uint4*>(p.state));
@@ -786,37 +802,37 @@ __global__ void __launch_bounds__(NTP, 2) decode_pool_kernel(const __grid_consta
     s_pos[tid] = ps;
   }
   __syncthreads();
-  bool ok = s_ok != 0;  // a mismatch was latched by decode_near_kernel
-  const uint32_t idesc_s = umma_idesc_bf16(kBlk, kSlots, false);
-  const uint32_t idesc_c = umma_idesc_bf16(kBlk, kBlk, true);
+  bool ok = s_ok != 0;  // a mismatch was latched by the near-field kernel
+  const uint32_t idesc_s = umma_idesc_bf16_ab(kBlk, TR, false, false);  // slot (K-major) . x^T (K-major)
+  const uint32_t idesc_c = umma_idesc_bf16_ab(kBlk, TR, true, false);   // slot^T (MN-major) . w^T
 
   if (warp == NWC) {
     // ---- MMA warp: slot loads and every MMA -------------------------------
     if (lane == 0) {
       // After the MMAs of load q: the stage of load q-1 (its MMAs committed
-      // one chunk earlier) takes load q+2.
+      // one chunk earlier) takes load q + 3.
       auto refill_slot = [&](int q) {
-        if (q < 1 || q + kSlotStages - 1 >= 2 * nch) return;
+        if (q < 1 || q + kSlotStages - 1 >= 2 * nloc) return;
         const int st = (q - 1) % kSlotStages;
         if (!mbar_wait_bounded(bars + kPbSlEmpty + st, static_cast<unsigned>(((q - 1) / kSlotStages) & 1),
                                kMbarPollLimit, p.err))
           ok = false;
         issue_slot(q + kSlotStages - 1);
       };
-      // pass 1: scores[16 x 64] += x_c . slot_c^T
-      for (int c = 0; c < nch; ++c) {
+      // pass 1: scores^T[64 slots x 16] += slot_c . x_c^T over this CTA's chunks
+      for (int c = 0; c < nloc; ++c) {
         const int stg = c % kSlotStages, b = c % kABufs;
         if (!mbar_wait_bounded(bars + kPbSlFull + stg, static_cast<unsigned>((c / kSlotStages) & 1), kMbarPollLimit, p.err))
           ok = false;
         if (!mbar_wait_bounded(bars + kPbAFull + b, static_cast<unsigned>((c / kABufs) & 1), kMbarPollLimit, p.err))
           ok = false;
         tc_fence_after();
-        const unsigned char* xhi = ablk + b * 2 * kBlkBytes;
         const unsigned char* shi = slb + stg * 2 * kBlkBytes;
+        const unsigned char* xhi = xtb + b * 2 * kBlk16Bytes;
 #pragma unroll
         for (int k = 0; k < kBlk / 16; ++k) {
-          const uint64_t ah = umma_desc(xhi + k * 2048, 1024, 128), al = umma_desc(xhi + kBlkBytes + k * 2048, 1024, 128);
-          const uint64_t bh = umma_desc(shi + k * 2048, 1024, 128), bl = umma_desc(shi + kBlkBytes + k * 2048, 1024, 128);
+          const uint64_t ah = umma_desc(shi + k * 2048, 1024, 128), al = umma_desc(shi + kBlkBytes + k * 2048, 1024, 128);
+          const uint64_t bh = umma_desc(xhi + k * 512, 256, 128), bl = umma_desc(xhi + kBlk16Bytes + k * 512, 256, 128);
           umma_bf16(tmem, ah, bh, idesc_s, c > 0 || k > 0);
           umma_bf16(tmem, ah, bl, idesc_s, true);
           umma_bf16(tmem, al, bh, idesc_s, true);
@@ -826,22 +842,36 @@ __global__ void __launch_bounds__(NTP, 2) decode_pool_kernel(const __grid_consta
         refill_slot(c);
       }
       umma_commit(bars + kPbScores);
-      // pass 2: sem chunk c = w . slot_c into accumulator c % 2
+    }
+    __syncwarp();
+    cluster_wait();    // phase 1: both CTAs started
+    cluster_arrive();  // phase 2: the partials are exchanged
+    cluster_wait();
+    if (lane == 0) {
+      auto refill_slot = [&](int q) {
+        if (q < 1 || q + kSlotStages - 1 >= 2 * nloc) return;
+        const int st = (q - 1) % kSlotStages;
+        if (!mbar_wait_bounded(bars + kPbSlEmpty + st, static_cast<unsigned>(((q - 1) / kSlotStages) & 1),
+                               kMbarPollLimit, p.err))
+          ok = false;
+        issue_slot(q + kSlotStages - 1);
+      };
+      // pass 2: sem^T chunk c [64 columns x 16] = slot_c^T . w^T
       if (!mbar_wait_bounded(bars + kPbWFull, 0, kMbarPollLimit, p.err)) ok = false;
-      for (int c = 0; c < nch; ++c) {
-        const int q = nch + c, stg = q % kSlotStages, b = c % kSemBufs;
+      for (int c = 0; c < nloc; ++c) {
+        const int q = nloc + c, stg = q % kSlotStages, b = c % kSemBufs;
         if (!mbar_wait_bounded(bars + kPbSlFull + stg, static_cast<unsigned>((q / kSlotStages) & 1), kMbarPollLimit, p.err))
           ok = false;
-        if (c >= kSemBufs &&
-            !mbar_wait_bounded(bars + kPbSemEmpty + b, static_cast<unsigned>(((c / kSemBufs) - 1) & 1), kMbarPollLimit, p.err))
+        if (c >= kSemBufs && !mbar_wait_bounded(bars + kPbSemEmpty + b, static_cast<unsigned>(((c / kSemBufs) - 1) & 1),
+                                                kMbarPollLimit, p.err))
           ok = false;
         tc_fence_after();
-        const uint32_t dst = tmem + kSlots + b * kBlk;
+        const uint32_t dst = tmem + kTmemSem + b * TR;
         const unsigned char* shi = slb + stg * 2 * kBlkBytes;
 #pragma unroll
         for (int k = 0; k < kSlots / 16; ++k) {
-          const uint64_t ah = umma_desc(wblk + k * 2048, 1024, 128), al = umma_desc(wblk + kBlkBytes + k * 2048, 1024, 128);
-          const uint64_t bh = umma_desc(shi + k * 256, 128, 1024), bl = umma_desc(shi + kBlkBytes + k * 256, 128, 1024);
+          const uint64_t ah = umma_desc(shi + k * 256, 128, 1024), al = umma_desc(shi + kBlkBytes + k * 256, 128, 1024);
+          const uint64_t bh = umma_desc(wtb + k * 512, 256, 128), bl = umma_desc(wtb + kBlk16Bytes + k * 512, 256, 128);
           umma_bf16(dst, ah, bh, idesc_c, k > 0);
           umma_bf16(dst, ah, bl, idesc_c, true);
           umma_bf16(dst, al, bh, idesc_c, true);
@@ -850,26 +880,23 @@ __global__ void __launch_bounds__(NTP, 2) decode_pool_kernel(const __grid_consta
         umma_commit(bars + kPbSlEmpty + stg);
         refill_slot(q);
       }
-      // the last slot loads have landed and been read: nothing in flight
-      if (!ok) latch_error(p.err, SFA_ERR_DEVICE_TIMEOUT);
     }
     __syncwarp();
   } else {
-    // ---- compute warps --------------------------------------------------
-    // Thread tid: row r = tid / 16, columns c4 .. c4+3 of every chunk.
+    // ---- compute warps: thread tid owns row r = tid / 16, columns c4 .. c4+3
     const int r = tid >> 4, c4 = (tid & 15) * 4;
     const long long st = s_st[r];
     const long long io = static_cast<long long>(li) * p.n_seq + static_cast<long long>(tb) * TR + r;
     const bool live = st >= 0 && ok;
-    const float* xrow = p.out + (live ? io : 0) * p.H + c4;
+    const float* xrow = p.out + (live ? io : 0) * p.H + c0 * kBlk + c4;
     auto load_x = [&](int c) -> float4 {
-      return (live && c < nch) ? __ldcg(reinterpret_cast<const float4*>(xrow + c * kBlk))
-                               : make_float4(0.f, 0.f, 0.f, 0.f);
+      return (live && c < nloc) ? __ldcg(reinterpret_cast<const float4*>(xrow + c * kBlk))
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
     };
-    // pass 1: split x chunk c into x block c % 2; |x|^2
+    // pass 1: x chunk c into x^T block c % 4 (split bf16), |x|^2
     float4 xn0 = load_x(0), xn1 = load_x(1);  // chunks c and c+1 in flight
     float sq = 0.f;
-    for (int c = 0; c < nch; ++c) {
+    for (int c = 0; c < nloc; ++c) {
       const int b = c % kABufs;
       const float4 v = xn0;
       xn0 = xn1;
@@ -878,55 +905,71 @@ __global__ void __launch_bounds__(NTP, 2) decode_pool_kernel(const __grid_consta
       if (c >= kABufs &&
           !mbar_wait_bounded(bars + kPbAEmpty + b, static_cast<unsigned>(((c / kABufs) - 1) & 1), kMbarPollLimit, p.err))
         ok = false;
-      unsigned char* xhi = ablk + b * 2 * kBlkBytes;
+      unsigned char* xhi = xtb + b * 2 * kBlk16Bytes;
       __nv_bfloat16 hh[4], ll[4];
       split_bf16(v.x, hh[0], ll[0]);
       split_bf16(v.y, hh[1], ll[1]);
       split_bf16(v.z, hh[2], ll[2]);
       split_bf16(v.w, hh[3], ll[3]);
-      const int off = blk_off(r, c4);
+      const int off = blk16_off(r, c4);
       *reinterpret_cast<uint2*>(xhi + off) = *reinterpret_cast<const uint2*>(hh);
-      *reinterpret_cast<uint2*>(xhi + kBlkBytes + off) = *reinterpret_cast<const uint2*>(ll);
+      *reinterpret_cast<uint2*>(xhi + kBlk16Bytes + off) = *reinterpret_cast<const uint2*>(ll);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(bars + kPbAFull + b);
     }
-    // |x|^2 per row: the 16 threads of a row (one half-warp) add their partials
 #pragma unroll
     for (int off = 8; off > 0; off >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, off);
-    if ((tid & 15) == 0) s_ssq[r][0] = sq;
-    if ((warp & 3) == 0) {  // rows 0..15 sit in lanes 0..15 of the first lane quarter (M = 64)
+    // partial scores and |x|^2 of this CTA's columns, into its own and the
+    // peer's shared memory
+    float* peer_scp = cluster.map_shared_rank(scp, rank ^ 1);
+    cluster_wait();  // phase 1: the peer has started
+    if ((tid & 15) == 0) {
+      sc[r * kScStride + kSlots] = sq;
+      peer_scp[r * kScStride + kSlots] = sq;
+    }
+    if (warp < 4) {  // slot 16w + i sits in lane i of lane quarter w (M = 64)
       if (!mbar_wait_bounded(bars + kPbScores, 0, kMbarPollLimit, p.err)) ok = false;
       tc_fence_after();
-      const int colh = (warp >> 2) * 32;
-      float v[32];
-      tmem_ld32(tmem + colh, v);
-      if (lane < TR) {
+      float v[16];
+      if (nloc > 0) {
+        tmem_ld16(tmem + (static_cast<uint32_t>(32 * warp) << 16), v);
+      } else {
 #pragma unroll
-        for (int jj = 0; jj < 32; ++jj) sc[lane * kScStride + colh + jj] = v[jj];
+        for (int rr = 0; rr < TR; ++rr) v[rr] = 0.f;
+      }
+      if (lane < 16) {
+#pragma unroll
+        for (int rr = 0; rr < TR; ++rr) {
+          sc[rr * kScStride + 16 * warp + lane] = v[rr];
+          peer_scp[rr * kScStride + 16 * warp + lane] = v[rr];
+        }
       }
     }
-    // scores and |x|^2 of every row in shared memory (compute warps only)
-    asm volatile("bar.sync 1, %0;" ::"n"(NTC) : "memory");
-    // softmax(cos/T) per row [P3 §2.1 channel 3]; weights as split bf16
+    __syncwarp();
+    cluster_arrive();  // phase 2: both partials in place
+    cluster_wait();
+    // softmax(cos/T) per row [P3 §2.1 channel 3]; weights as split bf16 w^T
     {
       const float* nrm = p.slot_norm + static_cast<size_t>(l) * kSlots;
       const float n0 = nrm[lane], n1 = nrm[lane + 32];
       for (int rr = warp; rr < TR; rr += NWC) {
-        const float nx = fmaxf(sqrtf(s_ssq[rr][0]), kNormFloor);
-        const float c0 = sc[rr * kScStride + lane] / (nx * n0) * p.inv_temp;
-        const float c1 = sc[rr * kScStride + lane + 32] / (nx * n1) * p.inv_temp;
-        const float mx = warp_max_redux(fmaxf(c0, c1));
-        const float e0 = expf(c0 - mx), e1 = expf(c1 - mx);
+        const float* a = sc + rr * kScStride;
+        const float* b = scp + rr * kScStride;
+        const float nx = fmaxf(sqrtf(a[kSlots] + b[kSlots]), kNormFloor);
+        const float c0v = (a[lane] + b[lane]) / (nx * n0) * p.inv_temp;
+        const float c1v = (a[lane + 32] + b[lane + 32]) / (nx * n1) * p.inv_temp;
+        const float mx = warp_max_redux(fmaxf(c0v, c1v));
+        const float e0 = expf(c0v - mx), e1 = expf(c1v - mx);
         const float inv = 1.f / warp_sum(e0 + e1);
         __nv_bfloat16 h0, l0, h1, l1;
         split_bf16(e0 * inv, h0, l0);
         split_bf16(e1 * inv, h1, l1);
-        const int o0 = blk_off(rr, lane), o1 = blk_off(rr, lane + 32);
-        *reinterpret_cast<__nv_bfloat16*>(wblk + o0) = h0;
-        *reinterpret_cast<__nv_bfloat16*>(wblk + kBlkBytes + o0) = l0;
-        *reinterpret_cast<__nv_bfloat16*>(wblk + o1) = h1;
-        *reinterpret_cast<__nv_bfloat16*>(wblk + kBlkBytes + o1) = l1;
+        const int o0 = blk16_off(rr, lane), o1 = blk16_off(rr, lane + 32);
+        *reinterpret_cast<__nv_bfloat16*>(wtb + o0) = h0;
+        *reinterpret_cast<__nv_bfloat16*>(wtb + kBlk16Bytes + o0) = l0;
+        *reinterpret_cast<__nv_bfloat16*>(wtb + o1) = h1;
+        *reinterpret_cast<__nv_bfloat16*>(wtb + kBlk16Bytes + o1) = l1;
       }
     }
     fence_proxy_async_smem();
@@ -936,16 +979,16 @@ __global__ void __launch_bounds__(NTP, 2) decode_pool_kernel(const __grid_consta
     // pass 2: ring, field, fusion, clip, output [P3 §2.1 channels 1-2, §2.2]
     const int slot_r = static_cast<int>(s_pos[r] & (kRing - 1));
     unsigned char* blk = p.state + kHeaderBytes + (live ? st : 0) * p.so.stride;
-    float* ring_r = reinterpret_cast<float*>(blk + p.so.ring) + static_cast<size_t>(slot_r) * p.H + c4;
-    float* rsum_r = reinterpret_cast<float*>(blk + p.so.ring_sum) + c4;
-    float* fld_r = reinterpret_cast<float*>(blk + p.so.field) + c4;
-    float* out_r = p.out + (live ? io : 0) * p.H + c4;
+    float* ring_r = reinterpret_cast<float*>(blk + p.so.ring) + static_cast<size_t>(slot_r) * p.H + c0 * kBlk + c4;
+    float* rsum_r = reinterpret_cast<float*>(blk + p.so.ring_sum) + c0 * kBlk + c4;
+    float* fld_r = reinterpret_cast<float*>(blk + p.so.field) + c0 * kBlk + c4;
+    float* out_r = p.out + (live ? io : 0) * p.H + c0 * kBlk + c4;
     struct Row4 {
       float4 x, old, rs, fl;
     };
     auto load_row = [&](int c) -> Row4 {
       Row4 v;
-      if (live && c < nch) {
+      if (live && c < nloc) {
         v.x = __ldcg(reinterpret_cast<const float4*>(out_r + c * kBlk));
         v.old = __ldcg(reinterpret_cast<const float4*>(ring_r + c * kBlk));
         v.rs = __ldcg(reinterpret_cast<const float4*>(rsum_r + c * kBlk));
@@ -957,28 +1000,26 @@ __global__ void __launch_bounds__(NTP, 2) decode_pool_kernel(const __grid_consta
     };
     Row4 rn0 = load_row(0), rn1 = load_row(1);  // chunks c and c+1 in flight
     const float a_l = p.alpha_layer[l];
-    const bool reader = (warp & 3) == 0;
-    for (int c = 0; c < nch; ++c) {
+    for (int c = 0; c < nloc; ++c) {
       const int b = c % kSemBufs;
       const unsigned ph = static_cast<unsigned>((c / kSemBufs) & 1);
-      float* stg = semst + b * TR * kSemStride;
-      if (reader) {
-        // accumulator b -> staging b (once the compute warps are done with it)
+      float* sstg = semst + b * TR * kSemStride;
+      if (warp < 4) {
+        // accumulator b (column 16w + i in lane i, rows along columns) ->
+        // sem staging b, once the compute warps are done with it
         if (!mbar_wait_bounded(bars + kPbSemFull + b, ph, kMbarPollLimit, p.err)) ok = false;
         tc_fence_after();
-        const int colh = (warp >> 2) * 32;
-        float v[32];
-        tmem_ld32(tmem + kSlots + b * kBlk + colh, v);
+        float v[16];
+        tmem_ld16(tmem + (static_cast<uint32_t>(32 * warp) << 16) + kTmemSem + b * TR, v);
         tc_fence_before();
+        __syncwarp();
         if (lane == 0) mbar_arrive(bars + kPbSemEmpty + b);
-        if (c >= kSemBufs &&
-            !mbar_wait_bounded(bars + kPbStEmpty + b, static_cast<unsigned>(((c / kSemBufs) - 1) & 1), kMbarPollLimit, p.err))
+        if (c >= kSemBufs && !mbar_wait_bounded(bars + kPbStEmpty + b, static_cast<unsigned>(((c / kSemBufs) - 1) & 1),
+                                                kMbarPollLimit, p.err))
           ok = false;
-        if (lane < TR) {
-          float* dst = stg + lane * kSemStride + colh;
+        if (lane < 16) {
 #pragma unroll
-          for (int jj = 0; jj < 32; jj += 4)
-            *reinterpret_cast<float4*>(dst + jj) = make_float4(v[jj], v[jj + 1], v[jj + 2], v[jj + 3]);
+          for (int rr = 0; rr < TR; ++rr) sstg[rr * kSemStride + 16 * warp + lane] = v[rr];
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(bars + kPbStFull + b);
@@ -987,7 +1028,7 @@ __global__ void __launch_bounds__(NTP, 2) decode_pool_kernel(const __grid_consta
       rn0 = rn1;
       rn1 = load_row(c + 2);
       if (!mbar_wait_bounded(bars + kPbStFull + b, ph, kMbarPollLimit, p.err)) ok = false;
-      const float4 sv = *reinterpret_cast<const float4*>(stg + r * kSemStride + c4);
+      const float4 sv = *reinterpret_cast<const float4*>(sstg + r * kSemStride + c4);
       __syncwarp();
       if (lane == 0) mbar_arrive(bars + kPbStEmpty + b);
       if (live && ok) {
@@ -1011,7 +1052,7 @@ __global__ void __launch_bounds__(NTP, 2) decode_pool_kernel(const __grid_consta
         *reinterpret_cast<float4*>(out_r + c * kBlk) = make_float4(ov[0], ov[1], ov[2], ov[3]);
       }
     }
-    if (live && ok && (tid & 15) == 0)
+    if (rank == 0 && live && ok && (tid & 15) == 0)
       *reinterpret_cast<long long*>(p.state + kHeaderBytes + st * p.so.stride + p.so.pos) = s_pos[r] + 1;
   }
 
@@ -1108,8 +1149,8 @@ cudaError_t launch_t(const DecodeParams& p, cudaStream_t s) {
     e = cudaLaunchKernelEx(&cfg, decode_near_kernel<Tin, D>, p, maps);
   }
   if (e != cudaSuccess) return e;
-  cfg.gridDim = dim3(static_cast<unsigned>(p.Lc * ((p.n_seq + TR - 1) / TR)), 1, 1);
-  cfg.blockDim = dim3(NTP, 1, 1);  // compute warps + the MMA warp
+  cfg.gridDim = dim3(static_cast<unsigned>(p.Lc * ((p.n_seq + TR - 1) / TR) * kPair), 1, 1);
+  cfg.blockDim = dim3(NTP, 1, 1);  // compute warps + the MMA warp; clusters of kPair
   cfg.dynamicSmemBytes = static_cast<size_t>(p.tp.pool_smem);
   return cudaLaunchKernelEx(&cfg, decode_pool_kernel, p);
 }

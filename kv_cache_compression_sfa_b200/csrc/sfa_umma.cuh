@@ -56,6 +56,20 @@ __host__ __device__ __forceinline__ uint32_t umma_idesc_bf16(int M, int N, bool 
   return d;
 }
 
+// The same with either operand MN-major (A: bit 15, B: bit 16).
+__host__ __device__ __forceinline__ uint32_t umma_idesc_bf16_ab(int M, int N, bool a_mn_major, bool b_mn_major) {
+  return umma_idesc_bf16(M, N, b_mn_major) | ((a_mn_major ? 1u : 0u) << 15);
+}
+
+// Byte offset of element (row, col) inside a [16 x 64] bf16 block in the
+// core-matrix layout (core matrix of rows 8*rg.., columns 8*cg.. at byte
+// (cg*2 + rg)*128): as a K-major operand the next row group is 128 bytes
+// on and the next K group 256 bytes on.
+__host__ __device__ __forceinline__ int blk16_off(int row, int col) {
+  return ((col >> 3) * 2 + (row >> 3)) * kCoreBytes + (row & 7) * 16 + (col & 7) * 2;
+}
+constexpr int kBlk16Bytes = 16 * kBlk * 2;  // one [16 x 64] bf16 block (2 KB)
+
 // D[tmem] (+)= A[smem] * B[smem]; issued by one thread.
 __device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc,
                                           bool accumulate) {
@@ -112,6 +126,21 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// 16 consecutive 32-bit columns of this thread's lane.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 // Splits x into bf16 hi = round(x) and lo = round(x - hi): hi + lo carries
