@@ -58,7 +58,7 @@
 extern "C" {
 #endif
 
-#define SFA_ABI_VERSION 2
+#define SFA_ABI_VERSION 3
 
 typedef enum sfa_status {
   SFA_OK = 0,
@@ -342,12 +342,14 @@ SFA_API int sfa_debug_set_wait_limit(sfa_handle* h, unsigned int spin_limit, lon
  * the operator's tolerance whichever runs).  decode_tile: -1 chooses the
  * decode kernel by the number of sequences per call (the default), 0 always
  * the per-sequence kernel, 1 always the batch-tiled kernel.
- * prefill_near_tc: 1 runs the prefill near field on the tensor cores where
- * they apply (bf16 inputs, k <= 16; the default), 0 on the CUDA cores.
- * SFA_ERR_INVALID_ARG for other values, SFA_ERR_UNSUPPORTED if the requested
- * kernel does not fit this configuration (nothing changes then).  Affects
- * later calls on this handle only. */
-SFA_API int sfa_debug_set_paths(sfa_handle* h, int decode_tile, int prefill_near_tc);
+ * prefill_near: where the tensor cores apply to the prefill near field
+ * (bf16 inputs, k <= 16), 2 runs it fused with the pool scores in one
+ * kernel (the default), 1 on the tensor cores followed by a separate pool
+ * kernel, 0 on the CUDA cores.  SFA_ERR_INVALID_ARG for other values,
+ * SFA_ERR_UNSUPPORTED if the requested kernel does not fit this
+ * configuration (nothing changes then).  Affects later calls on this handle
+ * only. */
+SFA_API int sfa_debug_set_paths(sfa_handle* h, int decode_tile, int prefill_near);
 
 #ifdef __cplusplus
 }

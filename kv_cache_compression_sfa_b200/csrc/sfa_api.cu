@@ -42,7 +42,8 @@ struct sfa_handle {
   bool tile_ok;          // the batch-tiled decode fits this configuration
   TilePlan tile_plan;    // its shared-memory plan
   int tile_mode;         // -1: by batch size; 0: never; 1: always (sfa_debug_set_paths)
-  bool near_tc;          // prefill near field on the tensor cores where it applies
+  int near_mode;         // prefill near field where the tensor cores apply: 2 fused with the
+                         // pool scores, 1 tensor cores and a separate pool kernel, 0 CUDA cores
   bool inputs_early;     // decode inputs declared complete before each call
   int out_mode;          // sfa_out_mode of the compute calls
 };
@@ -176,12 +177,14 @@ bool handle_ok(const sfa_handle* h) { return h != nullptr && h->magic == kHandle
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? SFA_OK : SFA_ERR_CUDA; }
 
 // Near-field plan of the prefill: on the tensor cores where they apply (bf16
-// inputs, k <= 16) unless h->near_tc is off, else on the CUDA cores.
+// inputs, k <= 16) unless h->near_mode is 0, there fused with the pool
+// scores unless it is 1; else on the CUDA cores.
 bool plan_near_field(sfa_handle* h, size_t limit) {
   const sfa_config* c = &h->cfg;
   const int esz = static_cast<int>(in_bytes(c->in_dtype));
-  return (h->near_tc && plan_near(c->head_dim, esz, c->window_k, limit, true, &h->near)) ||
-         plan_near(c->head_dim, esz, c->window_k, limit, false, &h->near);
+  return (h->near_mode > 0 &&
+          plan_near(c->head_dim, esz, c->window_k, limit, true, h->near_mode == 2, &h->near)) ||
+         plan_near(c->head_dim, esz, c->window_k, limit, false, false, &h->near);
 }
 
 template <typename P>
@@ -294,7 +297,7 @@ int sfa_init(const sfa_config* cfg, sfa_handle** out) {
   h->withhold_tile = -1;
   h->inputs_early = false;
   h->tile_mode = -1;
-  h->near_tc = true;
+  h->near_mode = 2;
   h->out_mode = SFA_OUT_F32;
   const int L = cfg->n_layers, H = hidden_of(cfg);
   bool no_fit = false;  // a kernel's shared-memory plan does not fit this device
@@ -512,7 +515,15 @@ int prefill_impl(const sfa_handle* h, int layer_begin, int layer_count, const vo
   p.ws_halo = w.halo;
   p.nseg_out = out_segments(h->n_sm, hidden_of(c), streams, tiles_per_stream);
   p.tps_out = static_cast<int>((tiles_per_stream + p.nseg_out - 1) / p.nseg_out);
-  {
+  if (h->near.fused) {
+    // Fused kernel: one CTA per SM, each a run of consecutive tiles of one
+    // stream, all heads; about one round over the SMs.
+    const long long total = streams * tiles_per_stream;
+    const long long tps = std::min(tiles_per_stream, std::max(1LL, (total + h->n_sm - 1) / std::max(h->n_sm, 1)));
+    const long long nseg = (tiles_per_stream + tps - 1) / tps;
+    p.n_seg = static_cast<int>(nseg);
+    p.tps = static_cast<int>(tps);
+  } else {
     // Near-field segments: about four rounds of two CTAs per SM, each CTA a
     // run of consecutive tiles of one (stream, head).
     const long long units = static_cast<long long>(c->n_q_heads) * streams;
@@ -635,16 +646,15 @@ int sfa_debug_set_wait_limit(sfa_handle* h, unsigned int spin_limit, long long w
   return SFA_OK;
 }
 
-int sfa_debug_set_paths(sfa_handle* h, int decode_tile, int prefill_near_tc) {
-  if (!handle_ok(h) || decode_tile < -1 || decode_tile > 1 || prefill_near_tc < 0 ||
-      prefill_near_tc > 1)
+int sfa_debug_set_paths(sfa_handle* h, int decode_tile, int prefill_near) {
+  if (!handle_ok(h) || decode_tile < -1 || decode_tile > 1 || prefill_near < 0 || prefill_near > 2)
     return SFA_ERR_INVALID_ARG;
   if (decode_tile == 1 && !h->tile_ok) return SFA_ERR_UNSUPPORTED;
-  const bool old_tc = h->near_tc;
+  const int old_mode = h->near_mode;
   const NearPlan old_plan = h->near;
-  h->near_tc = prefill_near_tc == 1;
+  h->near_mode = prefill_near;
   if (!plan_near_field(h, prefill_smem_limit(h->device))) {
-    h->near_tc = old_tc;
+    h->near_mode = old_mode;
     h->near = old_plan;
     return SFA_ERR_UNSUPPORTED;
   }

@@ -101,6 +101,7 @@ constexpr int kDecodeSmemBudget = 112 * 1024;  // keeps two decode CTAs per SM
 // span (positions t0-k .. t0+T-1), rows padded by 16 bytes.
 struct NearPlan {
   int tc;                 // near field on the tensor cores (bf16 inputs, k <= 16)
+  int fused;              // tensor cores: near field and pool scores in one kernel (fused_kernel)
   int stages;             // 2 or 1 staged buffers; 0: keys and values read from global memory
   int row;                // CUDA cores: padded bytes of one staged row
   int q[2], k[2], v[2];   // stage offsets (tensor cores: MMA operand blocks)
@@ -131,7 +132,7 @@ struct PrefillParams {
   int L, B, nq, nkv, K, H, G;
   int l0;                   // first layer of the state served (streams are l0*B + ...)
   int tiles_per_stream, n_streams;
-  int n_seg, tps;           // near field: segments per stream, tiles per segment
+  int n_seg, tps;           // near field (or fused kernel): segments per stream, tiles per segment
   int nseg_out, tps_out;    // output kernel: segments per stream, tiles per segment
   // workspace byte offsets: stream positions, S at the end of the call, pool
   // weights, far-field state at every tile start, x (output modes other
@@ -176,9 +177,9 @@ cudaError_t decode_tile_prepare(int device);
 bool plan_decode_tile(int H, int head_dim, int esz, int G, int K, size_t limit, TilePlan* out);
 cudaError_t launch_prefill(const PrefillParams& p, int in_dtype, int head_dim, cudaStream_t s);
 // Near-field plan for head_dim D, input element size esz and window K within
-// `limit` bytes of shared memory, on the tensor cores if tc (bf16, K <= 16);
-// false if none fits.
-bool plan_near(int D, int esz, int K, size_t limit, bool tc, NearPlan* out);
+// `limit` bytes of shared memory, on the tensor cores if tc (bf16, K <= 16),
+// there fused with the pool scores if fused; false if none fits.
+bool plan_near(int D, int esz, int K, size_t limit, bool tc, bool fused, NearPlan* out);
 int prefill_pool_smem();
 int prefill_out_smem();
 cudaError_t prefill_prepare(int device);

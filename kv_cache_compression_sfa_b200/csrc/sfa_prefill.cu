@@ -728,6 +728,559 @@ near_tc_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ 
 }
 
 // ======================================================================
+// 1+2. fused: near field, far field, x, pool scores and field aggregates
+// ======================================================================
+// One CTA per (stream, segment of consecutive tiles) walks its tiles and,
+// per tile, every query head h (step j = tile * n_q + h).  Per step, on the
+// tcgen05 tensor cores with fp32 accumulators in tensor memory:
+//   QK(j):   scores[64 x 80] = Q_h . K_span^T, the band softmax on warps 2-5
+//            [P1 §2.1 eq. O_near];
+//   PV(j):   X_h[64 x D] = P . V_span + G . K_span (hi and lo of P and of
+//            the far-field weights G, as in near_tc_kernel); warps 6-9 add
+//            alpha_far gamma^m S_start [P1 §2.1 eq. O], store x (fp32) for
+//            the output kernel and split it into bf16 hi/lo blocks;
+//   POOL(j): pool[64 x 64 slots] += X_h . slot_h^T (hi*hi + hi*lo + lo*hi)
+//            over the heads of the tile [P3 §2.1 channel 3], and the EMA
+//            field over the tile from zero for the head's columns,
+//            A[c] = sum_r (1-g) g^(Tt-1-r) x[r][c] [P3 §2.1 channel 2], as
+//            the transposed product X_h^T . F with the weights in column 0
+//            of F (column 1: the stream's last tile when it is short).
+// After a tile's last head its scores, |x|^2 per token and the slot norms
+// give softmax(cos/T); the weights go to the workspace as split bf16 blocks,
+// as pool_kernel writes them, and x, the field aggregates and the output
+// segments' halo rows as near_tc_kernel and pool_kernel write them: the
+// output kernel is the same.
+//
+// Warp roles (one elected lane issues): warp 0 loads (tensor copies of q per
+// head and of the key/value span per KV head, bulk copies of the head's
+// slot blocks); warp 1 issues the MMAs, for step j QK(j), PV(j-1) and
+// POOL(j-2); warps 2-5 run the band softmax and the tile's pool softmax;
+// warps 6-13 the x epilogue, two per lane quarter of the accumulator, each
+// on half of the head's columns.  Scores
+// and X accumulators are double-buffered in tensor memory, queries and slot
+// blocks double-buffered in shared memory; every hand-off is an mbarrier
+// with a bounded wait.
+constexpr int NTF = 448;              // threads of the fused kernel: 14 warps
+constexpr int kEpiWarps = 8;          // x epilogue warps (warps 6 .. 13)
+constexpr int kTmemFused = 512;       // all of an SM's tensor memory: one CTA per SM
+constexpr int kFColS = 0;             // [2] band scores, kNS columns each
+constexpr int kFColPool = 2 * kNS;    // pool scores, 64 columns
+constexpr int kFColFagg = kFColPool + kSlots;  // field aggregates, 16 columns
+constexpr int kFColX = 256;           // [2] X accumulators, D columns each
+static_assert(kFColFagg + 16 <= kFColX, "tensor-memory columns of the fused kernel");
+
+template <int D>
+struct FusedPlan {
+  static constexpr int kvb = (D / 8) * kDStr;             // key (or value) span block
+  static constexpr int qb = kTile * D * 2;                // one head's queries
+  static constexpr int slb = (D / kBlk) * 2 * kBlkBytes;  // one head's slot blocks (hi, lo per chunk)
+  static constexpr int pb = kTile * kNS * 2;              // a P or G block (hi or lo)
+  static constexpr int xb = kTile * D * 2;                // an X block (hi or lo)
+  static constexpr int kk = 1024;                         // mbarriers before it
+  static constexpr int vv = kk + kvb;
+  static constexpr int q0 = vv + kvb;                     // [2]
+  static constexpr int sl0 = q0 + 2 * qb;                 // [2]
+  static constexpr int pa = sl0 + 2 * slb;                // hi, lo
+  static constexpr int ga = pa + 2 * pb;                  // hi, lo
+  static constexpr int xa = ga + 2 * pb;                  // hi, lo
+  static constexpr int fa = xa + 2 * xb;                  // hi, lo [16 x 64] blocks of F
+  static constexpr int total = fa + 2 * kBlk16Bytes + 128;  // 128: base alignment slack
+};
+static_assert(FusedPlan<128>::total <= 227 * 1024 - 2048, "fused kernel shared memory");
+
+// barrier slots
+enum : int {
+  kFbKvFull = 0, kFbKvFix, kFbKvEmpty,
+  kFbQFull, kFbQEmpty = kFbQFull + 2,
+  kFbSlFull = kFbQEmpty + 2, kFbSlEmpty = kFbSlFull + 2,
+  kFbSFull = kFbSlEmpty + 2, kFbSEmpty = kFbSFull + 2,
+  kFbPFull = kFbSEmpty + 2, kFbPEmpty,
+  kFbOFull, kFbOEmpty = kFbOFull + 2,
+  kFbXFull = kFbOEmpty + 2, kFbXEmpty,
+  kFbScFull, kFbScEmpty, kFbSqFull, kFbSqEmpty, kFbProbe,
+  kFbCount
+};
+static_assert(kFbCount * 8 <= 1024, "fused kernel barriers");
+
+template <int D>
+__global__ void __launch_bounds__(NTF, 1)
+fused_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ NearMaps maps) {
+  using Tin = __nv_bfloat16;
+  using FP = FusedPlan<D>;
+  constexpr int C16 = D / 8;  // 16-byte chunks of one head row
+  const int seg = blockIdx.x, s = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  extern __shared__ __align__(128) unsigned char smf_raw[];
+  unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smf_raw) + 127) &
+                                                       ~static_cast<uintptr_t>(127));
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm);
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_ok;
+  __shared__ long long s_pos;
+  __shared__ float s_gpow[kTile + 1];  // gamma_far^m
+  __shared__ float s_norm[kSlots];     // slot norms of the layer
+  __shared__ float s_sq[2][kTile];     // |x|^2 per token of the tile being finished, per column half
+
+  pdl_trigger();
+  pdl_wait();  // far state at the tile starts from far_carry_kernel
+  const int l = p.l0 + s / p.B;
+  if (tid <= kTile) s_gpow[tid] = powf(p.gamma_far, static_cast<float>(tid));
+  if (tid < kSlots) s_norm[tid] = p.slot_norm[static_cast<size_t>(l) * kSlots + tid];
+  if (tid == 0) {
+    s_ok = header_matches(p);
+    s_pos = reinterpret_cast<const long long*>(p.ws + p.ws_pos)[s];
+    for (int b = 0; b < kFbCount; ++b) {
+      int count = 1;
+      if (b == kFbSEmpty || b == kFbSEmpty + 1 || b == kFbPFull || b == kFbScEmpty || b == kFbSqEmpty)
+        count = 4;  // one arrival per softmax warp
+      if (b == kFbOEmpty || b == kFbOEmpty + 1 || b == kFbXFull || b == kFbSqFull)
+        count = kEpiWarps;  // one arrival per epilogue warp
+      mbar_init(bar + b, count);
+    }
+    mbar_fence_init();
+  }
+  __syncthreads();
+  if (!s_ok) return;  // latched by far_agg_kernel
+  const long long pos0 = s_pos;
+  const long long ns = stream_len(p, s);  // tokens of this stream in the call
+  const int tiles_s = static_cast<int>((ns + kTile - 1) / kTile);
+  const int i0 = seg * p.tps, i1 = min(min(p.tiles_per_stream, tiles_s), i0 + p.tps);
+  if (i0 >= i1) return;  // past a ragged stream's end
+  const int nq = p.nq, G = p.G, nkv = p.nkv, K = p.K;
+  const int nsteps = (i1 - i0) * nq;
+  if (warp == 1) tmem_alloc(&s_tmem, kTmemFused);  // one CTA per SM (shared memory): never waits long
+
+  unsigned char* kk = sm + FP::kk;
+  unsigned char* vv = sm + FP::vv;
+  unsigned char* pa_hi = sm + FP::pa;
+  unsigned char* pa_lo = pa_hi + FP::pb;
+  unsigned char* ga_hi = sm + FP::ga;
+  unsigned char* ga_lo = ga_hi + FP::pb;
+  unsigned char* xa_hi = sm + FP::xa;
+  unsigned char* xa_lo = xa_hi + FP::xb;
+  unsigned char* fa_hi = sm + FP::fa;
+  unsigned char* fa_lo = fa_hi + kBlk16Bytes;
+  const float gf = p.gamma_far, af = p.alpha_far, ge = p.ema_gamma;
+  // P columns outside the bands stay zero; G for every tile (the rows a
+  // tile's first tokens would evict before position k multiply span rows
+  // before position 0, which are zero); F: column 0 the field weights of a
+  // full tile, column 1 those of the stream's last tile if it is short.
+  for (int i = tid; i < 2 * FP::pb / 16; i += NTF) reinterpret_cast<uint4*>(pa_hi)[i] = make_uint4(0u, 0u, 0u, 0u);
+  for (int i = tid; i < kTile * kNS; i += NTF) {
+    const int r = i / kNS, c = i % kNS;
+    const int j = c - 16 + K;  // token whose evicted key is span row c
+    const float gv = (j >= 0 && j <= r) ? af * (1.0f - gf) * powf(gf, static_cast<float>(r - j)) : 0.f;
+    __nv_bfloat16 hb, lb;
+    split_bf16(gv, hb, lb);
+    const int off = blk_off(r, c);
+    *reinterpret_cast<__nv_bfloat16*>(ga_hi + off) = hb;
+    *reinterpret_cast<__nv_bfloat16*>(ga_lo + off) = lb;
+  }
+  const int t_last = static_cast<int>(ns - static_cast<long long>(tiles_s - 1) * kTile);  // tokens of the last tile
+  for (int i = tid; i < 16 * kTile; i += NTF) {
+    const int n = i / kTile, r = i % kTile;
+    float fv = 0.f;
+    if (n == 0) fv = (1.0f - ge) * powf(ge, static_cast<float>(kTile - 1 - r));
+    if (n == 1 && r < t_last) fv = (1.0f - ge) * powf(ge, static_cast<float>(t_last - 1 - r));
+    __nv_bfloat16 hb, lb;
+    split_bf16(fv, hb, lb);
+    const int off = blk16_off(n, r);
+    *reinterpret_cast<__nv_bfloat16*>(fa_hi + off) = hb;
+    *reinterpret_cast<__nv_bfloat16*>(fa_lo + off) = lb;
+  }
+  fence_proxy_async_smem();  // zero fills, G and F seen by the MMAs
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+  const int row0 = static_cast<int>(static_cast<long long>(s) * p.n);  // first token row of the stream
+  const long long in_row0 = static_cast<long long>(s) * p.n;
+  bool ok = true;
+  auto wait = [&](int b, unsigned parity) {
+    if (!mbar_wait_bounded(bar + b, parity, kMbarPollLimit, p.err)) ok = false;
+  };
+  auto tile_rows = [&](int i) -> int {
+    return static_cast<int>(min(static_cast<long long>(kTile), ns - static_cast<long long>(i) * kTile));
+  };
+
+  if (warp == 0) {
+    // ---- loads ------------------------------------------------------------
+    unsigned char* blk = stream_block(p, s);
+    const Tin* win_k = reinterpret_cast<const Tin*>(blk + p.so.win_k);
+    const Tin* win_v = reinterpret_cast<const Tin*>(blk + p.so.win_v);
+    const unsigned char* img_l = p.slot_img + static_cast<size_t>(l) * (p.H / kBlk) * 2 * kBlkBytes;
+    constexpr unsigned kKvBytes = static_cast<unsigned>(2 * C16 * kNS * 16);
+    int kvc = 0;  // span copies issued
+    for (int j = 0; j < nsteps; ++j) {
+      const int h = j % nq, i = i0 + j / nq, g = h / G, b = j & 1;
+      if (h % G == 0) {
+        if (lane == 0) {
+          if (kvc > 0) wait(kFbKvEmpty, static_cast<unsigned>((kvc - 1) & 1));
+          mbar_arrive_expect_tx(bar + kFbKvFull, kKvBytes);
+          const int rkv = row0 + i * kTile - 16;
+#pragma unroll
+          for (int u = 0; u < C16; ++u) {
+            tma_load_3d(kk + u * kDStr, &maps.k, 8 * u, g, rkv, bar + kFbKvFull);
+            tma_load_3d(vv + u * kDStr, &maps.v, 8 * u, g, rkv, bar + kFbKvFull);
+          }
+        }
+        if (i == 0) {
+          // span rows 0..15 of the call's first tile: positions before the
+          // call from the state window, before position 0 zero
+          if (lane == 0) wait(kFbKvFull, static_cast<unsigned>(kvc & 1));
+          __syncwarp();
+          for (int c = lane; c < 16 * C16; c += 32) {
+            const int r = c / C16, u = c % C16;
+            const long long jp = pos0 - 16 + r;
+            uint4 kv4 = make_uint4(0u, 0u, 0u, 0u), vv4 = kv4;
+            if (jp >= 0) {
+              kv4 = *reinterpret_cast<const uint4*>(win_k + ((jp % K) * nkv + g) * D + 8 * u);
+              vv4 = *reinterpret_cast<const uint4*>(win_v + ((jp % K) * nkv + g) * D + 8 * u);
+            }
+            *reinterpret_cast<uint4*>(kk + kv_off(r, 8 * u)) = kv4;
+            *reinterpret_cast<uint4*>(vv + kv_off(r, 8 * u)) = vv4;
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar + kFbKvFix);
+        }
+        ++kvc;
+      }
+      if (lane == 0) {
+        if (j >= 2) wait(kFbQEmpty + b, static_cast<unsigned>(((j >> 1) - 1) & 1));
+        unsigned char* qa = sm + FP::q0 + b * FP::qb;
+        mbar_arrive_expect_tx(bar + kFbQFull + b, static_cast<unsigned>(FP::qb));
+#pragma unroll
+        for (int u = 0; u < C16; ++u) tma_load_3d(qa + u * 1024, &maps.q, 8 * u, h, row0 + i * kTile, bar + kFbQFull + b);
+        if (j >= 2) wait(kFbSlEmpty + b, static_cast<unsigned>(((j >> 1) - 1) & 1));
+        mbar_arrive_expect_tx(bar + kFbSlFull + b, static_cast<unsigned>(FP::slb));
+        bulk_g2s(sm + FP::sl0 + b * FP::slb, img_l + static_cast<size_t>(h) * FP::slb, static_cast<unsigned>(FP::slb),
+                 bar + kFbSlFull + b);
+      }
+    }
+  } else if (warp == 1) {
+    // ---- MMAs ---------------------------------------------------------------
+    if (lane == 0) {
+      const uint32_t idesc_qk = umma_idesc_bf16(kTile, kNS, false);
+      const uint32_t idesc_pv = umma_idesc_bf16(kTile, D, true);
+      const uint32_t idesc_sc = umma_idesc_bf16(kTile, kSlots, false);
+      const uint32_t idesc_fa = umma_idesc_bf16_ab(D, 16, true, false);  // X^T (MN-major) . F
+      int kvw = 0;  // span copies waited for
+      auto do_qk = [&](int j) {
+        const int h = j % nq, i = i0 + j / nq, b = j & 1;
+        if (h % G == 0) {
+          wait(kFbKvFull, static_cast<unsigned>(kvw & 1));
+          if (i == 0) wait(kFbKvFix, static_cast<unsigned>(kvw & 1));  // kvw = KV head here
+          ++kvw;
+        }
+        wait(kFbQFull + b, static_cast<unsigned>((j >> 1) & 1));
+        if (j >= 2) wait(kFbSEmpty + b, static_cast<unsigned>(((j >> 1) - 1) & 1));
+        tc_fence_after();
+        const unsigned char* qa = sm + FP::q0 + b * FP::qb;
+#pragma unroll
+        for (int k2 = 0; k2 < D / 16; ++k2)
+          umma_bf16(tmem + kFColS + b * kNS, umma_desc(qa + k2 * 2048, 1024, 128),
+                    umma_desc(kk + 2 * k2 * kDStr, kDStr, 128), idesc_qk, k2 > 0);
+        umma_commit(bar + kFbSFull + b);
+        umma_commit(bar + kFbQEmpty + b);
+      };
+      auto do_pv = [&](int j) {
+        const int h = j % nq, b = j & 1;
+        wait(kFbPFull, static_cast<unsigned>(j & 1));
+        if (j >= 2) wait(kFbOEmpty + b, static_cast<unsigned>(((j >> 1) - 1) & 1));
+        tc_fence_after();
+        const uint32_t dst = tmem + kFColX + b * D;
+#pragma unroll
+        for (int k2 = 0; k2 < kNS / 16; ++k2) {
+          const uint64_t bv = umma_desc(vv + k2 * 256, 128, kDStr);
+          const uint64_t bk = umma_desc(kk + k2 * 256, 128, kDStr);
+          umma_bf16(dst, umma_desc(pa_hi + k2 * 2048, 1024, 128), bv, idesc_pv, k2 > 0);
+          umma_bf16(dst, umma_desc(pa_lo + k2 * 2048, 1024, 128), bv, idesc_pv, true);
+          umma_bf16(dst, umma_desc(ga_hi + k2 * 2048, 1024, 128), bk, idesc_pv, true);
+          umma_bf16(dst, umma_desc(ga_lo + k2 * 2048, 1024, 128), bk, idesc_pv, true);
+        }
+        umma_commit(bar + kFbOFull + b);
+        umma_commit(bar + kFbPEmpty);
+        if (h % G == G - 1 || j == nsteps - 1) umma_commit(bar + kFbKvEmpty);  // span no longer read
+      };
+      auto do_pool = [&](int j) {
+        const int h = j % nq, ti = j / nq, b = j & 1;
+        wait(kFbXFull, static_cast<unsigned>(j & 1));
+        wait(kFbSlFull + b, static_cast<unsigned>((j >> 1) & 1));
+        if (h == 0 && ti >= 1) wait(kFbScEmpty, static_cast<unsigned>((ti - 1) & 1));
+        tc_fence_after();
+        const unsigned char* sl = sm + FP::sl0 + b * FP::slb;
+#pragma unroll
+        for (int c = 0; c < D / kBlk; ++c) {
+          const unsigned char* shi = sl + c * 2 * kBlkBytes;
+          const unsigned char* slo = shi + kBlkBytes;
+#pragma unroll
+          for (int k = 0; k < kBlk / 16; ++k) {
+            const uint64_t ah = umma_desc(xa_hi + c * kBlkBytes + k * 2048, 1024, 128);
+            const uint64_t al = umma_desc(xa_lo + c * kBlkBytes + k * 2048, 1024, 128);
+            const uint64_t bh = umma_desc(shi + k * 2048, 1024, 128), bl = umma_desc(slo + k * 2048, 1024, 128);
+            umma_bf16(tmem + kFColPool, ah, bh, idesc_sc, h > 0 || c > 0 || k > 0);
+            umma_bf16(tmem + kFColPool, ah, bl, idesc_sc, true);
+            umma_bf16(tmem + kFColPool, al, bh, idesc_sc, true);
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < kTile / 16; ++k) {
+          const uint64_t ah = umma_desc(xa_hi + k * 256, 128, 1024), al = umma_desc(xa_lo + k * 256, 128, 1024);
+          const uint64_t bh = umma_desc(fa_hi + k * 512, 256, 128), bl = umma_desc(fa_lo + k * 512, 256, 128);
+          umma_bf16(tmem + kFColFagg, ah, bh, idesc_fa, k > 0);
+          umma_bf16(tmem + kFColFagg, ah, bl, idesc_fa, true);
+          umma_bf16(tmem + kFColFagg, al, bh, idesc_fa, true);
+        }
+        umma_commit(bar + kFbXEmpty);
+        umma_commit(bar + kFbSlEmpty + b);
+        if (h == nq - 1) umma_commit(bar + kFbScFull);
+      };
+      // Step j: QK(j), PV(j-1), POOL(j-2); PV first where step j opens a
+      // KV head's span, whose copy waits for the last PV on the previous one.
+      for (int j = 0; j <= nsteps + 1; ++j) {
+        if (j < nsteps && (j % nq) % G == 0) {
+          if (j >= 1) do_pv(j - 1);
+          do_qk(j);
+        } else {
+          if (j < nsteps) do_qk(j);
+          if (j >= 1 && j <= nsteps) do_pv(j - 1);
+        }
+        if (j >= 2) do_pool(j - 2);
+      }
+    }
+    __syncwarp();
+  } else if (warp < 6) {
+    // ---- band softmax; the tile's pool softmax -------------------------------
+    const int qd = warp & 3;  // lane quarter: rows 16 qd .. 16 qd + 15 in lanes 0..15
+    const int r = 16 * qd + lane;
+    const uint32_t lane_base = static_cast<uint32_t>(32 * qd) << 16;
+    auto finish = [&](int ti) {
+      const int i = i0 + ti;
+      const int Tt = tile_rows(i);
+      wait(kFbScFull, static_cast<unsigned>(ti & 1));
+      wait(kFbSqFull, static_cast<unsigned>(ti & 1));
+      tc_fence_after();
+      float sv[kSlots];
+      tmem_ld32(tmem + lane_base + kFColPool, *reinterpret_cast<float(*)[32]>(sv));
+      tmem_ld32(tmem + lane_base + kFColPool + 32, *reinterpret_cast<float(*)[32]>(sv + 32));
+      const float sq = lane < 16 ? s_sq[0][r] + s_sq[1][r] : 0.f;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(bar + kFbScEmpty);
+        mbar_arrive(bar + kFbSqEmpty);
+      }
+      // Test hook: a bounded wait on a barrier that nothing completes.
+      if (tid == 64 && static_cast<long long>(i) * p.n_streams + s == p.withhold_tile) {
+        mbar_arrive_expect_tx(bar + kFbProbe, 16u);
+        mbar_wait_bounded(bar + kFbProbe, 0, p.spin_limit, p.err);
+      }
+      if (lane < 16) {
+        // softmax(cos/T) per token [P3 §2.1 channel 3]; rows past the tile
+        // get zero weights
+        const float nx = fmaxf(sqrtf(sq), kNormFloor);
+        float mx = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < kSlots; ++e) {
+          sv[e] = sv[e] / (nx * s_norm[e]) * p.inv_temp;
+          mx = fmaxf(mx, sv[e]);
+        }
+        float sum = 0.f;
+#pragma unroll
+        for (int e = 0; e < kSlots; ++e) {
+          sv[e] = expf(sv[e] - mx);
+          sum += sv[e];
+        }
+        const float inv = r < Tt ? 1.f / sum : 0.f;
+        unsigned char* wblk = p.ws + p.ws_w + (static_cast<long long>(s) * p.tiles_per_stream + i) * 2 * kBlkBytes;
+#pragma unroll
+        for (int g8 = 0; g8 < kSlots / 8; ++g8) {
+          uint32_t hw[4], lw[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            __nv_bfloat16 h0b, l0b, h1b, l1b;
+            split_bf16(sv[8 * g8 + 2 * e] * inv, h0b, l0b);
+            split_bf16(sv[8 * g8 + 2 * e + 1] * inv, h1b, l1b);
+            hw[e] = static_cast<uint32_t>(__bfloat16_as_ushort(h0b)) |
+                    (static_cast<uint32_t>(__bfloat16_as_ushort(h1b)) << 16);
+            lw[e] = static_cast<uint32_t>(__bfloat16_as_ushort(l0b)) |
+                    (static_cast<uint32_t>(__bfloat16_as_ushort(l1b)) << 16);
+          }
+          if (ok) {
+            const int off = blk_off(r, 8 * g8);
+            *reinterpret_cast<uint4*>(wblk + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+            *reinterpret_cast<uint4*>(wblk + kBlkBytes + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+          }
+        }
+      }
+    };
+    for (int j = 0; j < nsteps; ++j) {
+      const int ti = j / nq, b = j & 1;
+      const long long t0 = pos0 + static_cast<long long>(i0 + ti) * kTile;
+      wait(kFbSFull + b, static_cast<unsigned>((j >> 1) & 1));
+      tc_fence_after();
+      float v[32];
+      tmem_ld32(tmem + lane_base + kFColS + b * kNS + 16 * qd, v);  // the band of rows 16 qd .. lies in span columns 16 qd .. 16 qd + 31
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar + kFbSEmpty + b);
+      uint32_t hw[4][4], lw[4][4];
+      {
+        const int cmin = t0 < 16 ? static_cast<int>(16 - t0) : 0;  // first span row at position >= 0
+        float mx = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int c = 16 * qd + e;
+          const bool in = c >= r + 17 - K && c <= r + 16 && c >= cmin;
+          v[e] = in ? v[e] * p.score_scale : -INFINITY;
+          mx = fmaxf(mx, v[e]);
+        }
+        float sum = 0.f;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          v[e] = __expf(v[e] - mx);  // 0 outside the band
+          sum += v[e];
+        }
+        const float inv = 1.f / sum;
+#pragma unroll
+        for (int g8 = 0; g8 < 4; ++g8)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            __nv_bfloat16 h0b, l0b, h1b, l1b;
+            split_bf16(v[8 * g8 + 2 * e] * inv, h0b, l0b);
+            split_bf16(v[8 * g8 + 2 * e + 1] * inv, h1b, l1b);
+            hw[g8][e] = static_cast<uint32_t>(__bfloat16_as_ushort(h0b)) |
+                        (static_cast<uint32_t>(__bfloat16_as_ushort(h1b)) << 16);
+            lw[g8][e] = static_cast<uint32_t>(__bfloat16_as_ushort(l0b)) |
+                        (static_cast<uint32_t>(__bfloat16_as_ushort(l1b)) << 16);
+          }
+      }
+      if (j >= 1) wait(kFbPEmpty, static_cast<unsigned>((j - 1) & 1));  // PV(j-1) has read P
+      if (lane < 16) {
+#pragma unroll
+        for (int g8 = 0; g8 < 4; ++g8) {
+          const int off = blk_off(r, 16 * qd + 8 * g8);
+          *reinterpret_cast<uint4*>(pa_hi + off) = make_uint4(hw[g8][0], hw[g8][1], hw[g8][2], hw[g8][3]);
+          *reinterpret_cast<uint4*>(pa_lo + off) = make_uint4(lw[g8][0], lw[g8][1], lw[g8][2], lw[g8][3]);
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar + kFbPFull);
+      if (j % nq == 0 && ti >= 1) finish(ti - 1);
+    }
+    finish((nsteps - 1) / nq);
+  } else {
+    // ---- x epilogue ------------------------------------------------------------
+    const int qd = warp & 3;  // lane quarter: rows 16 qd .. 16 qd + 15 in lanes 0..15
+    const int hf = (warp - 6) >> 2;  // column half of the head
+    const int r = 16 * qd + lane;
+    const uint32_t lane_base = static_cast<uint32_t>(32 * qd) << 16;
+    const float* sst = reinterpret_cast<const float*>(p.ws + p.ws_sst) +
+                       static_cast<long long>(s) * p.tiles_per_stream * nkv * D;
+    float* fagg = reinterpret_cast<float*>(p.ws + p.ws_fagg) + static_cast<long long>(s) * p.tiles_per_stream * p.H;
+    // field aggregate of step j's columns: column 0 of the accumulator for a
+    // full tile, column 1 for a short last tile.  M = 128 (D = 128): column
+    // c in lane c; M = 64: column c in lane (c % 16) + 32 (c / 16).
+    auto store_fagg = [&](int j) {
+      const int h = j % nq, i = i0 + j / nq;
+      tc_fence_after();
+      float fv[2];
+      tmem_ld2(tmem + lane_base + kFColFagg, fv);
+      const int c = D == 128 ? 32 * qd + lane : 16 * qd + lane;
+      if (hf == 0 && (D == 128 || lane < 16) && ok)
+        fagg[static_cast<long long>(i) * p.H + h * D + c] = tile_rows(i) == kTile ? fv[0] : fv[1];
+    };
+    float sq4[4] = {0.f, 0.f, 0.f, 0.f};  // |x|^2 of row r over the tile's heads so far (four partial sums)
+    for (int j = 0; j < nsteps; ++j) {
+      const int h = j % nq, ti = j / nq, i = i0 + ti, g = h / G, b = j & 1;
+      const long long t0 = pos0 + static_cast<long long>(i) * kTile;
+      const int Tt = tile_rows(i);
+      const int r_ev = static_cast<int>(max(0LL, min(static_cast<long long>(Tt), K - t0)));
+      const float c0s = af * s_gpow[min(kTile, max(0, r - r_ev + 1))];
+      const float* s0 = sst + (static_cast<long long>(i) * nkv + g) * D;
+      const bool live = lane < 16 && r < Tt && ok;
+      float* orow = p.out + (in_row0 + static_cast<long long>(i) * kTile + r) * p.H + h * D;
+      // the last kHalo rows of a tile that ends an output segment lead the next one
+      const bool halo_row = r >= kTile - kHalo && (i + 1) % p.tps_out == 0 &&
+                            (i + 1) * static_cast<long long>(kTile) < ns;
+      float* hrow = reinterpret_cast<float*>(p.ws + p.ws_halo) +
+                    ((static_cast<long long>(s) * p.nseg_out + (i + 1) / p.tps_out - 1) * kHalo +
+                     (r - (kTile - kHalo))) * p.H + h * D;
+      wait(kFbOFull + b, static_cast<unsigned>((j >> 1) & 1));
+      tc_fence_after();
+#pragma unroll 1
+      for (int cc = hf * (D / 64); cc < (hf + 1) * (D / 64); ++cc) {
+        float v[32];
+        tmem_ld32(tmem + lane_base + kFColX + b * D + 32 * cc, v);
+#pragma unroll
+        for (int e = 0; e < 32; e += 4) {
+          const float4 sv4 = __ldg(reinterpret_cast<const float4*>(s0 + 32 * cc + e));
+          v[e] = r < Tt ? fmaf(c0s, sv4.x, v[e]) : 0.f;
+          v[e + 1] = r < Tt ? fmaf(c0s, sv4.y, v[e + 1]) : 0.f;
+          v[e + 2] = r < Tt ? fmaf(c0s, sv4.z, v[e + 2]) : 0.f;
+          v[e + 3] = r < Tt ? fmaf(c0s, sv4.w, v[e + 3]) : 0.f;
+          sq4[(e >> 2) & 3] = fmaf(v[e], v[e], fmaf(v[e + 1], v[e + 1], fmaf(v[e + 2], v[e + 2], fmaf(v[e + 3], v[e + 3], sq4[(e >> 2) & 3]))));
+          if (live) {
+            *reinterpret_cast<float4*>(orow + 32 * cc + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+            if (halo_row) *reinterpret_cast<float4*>(hrow + 32 * cc + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+          }
+        }
+        if (cc == hf * (D / 64) && j >= 1) {  // POOL(j-1) has read X: its field aggregate is ready
+          wait(kFbXEmpty, static_cast<unsigned>((j - 1) & 1));
+          store_fagg(j - 1);
+        }
+        if (lane < 16) {
+#pragma unroll
+          for (int g8 = 0; g8 < 4; ++g8) {
+            uint32_t hw[4], lw[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              __nv_bfloat16 h0b, l0b, h1b, l1b;
+              split_bf16(v[8 * g8 + 2 * e], h0b, l0b);
+              split_bf16(v[8 * g8 + 2 * e + 1], h1b, l1b);
+              hw[e] = static_cast<uint32_t>(__bfloat16_as_ushort(h0b)) |
+                      (static_cast<uint32_t>(__bfloat16_as_ushort(h1b)) << 16);
+              lw[e] = static_cast<uint32_t>(__bfloat16_as_ushort(l0b)) |
+                      (static_cast<uint32_t>(__bfloat16_as_ushort(l1b)) << 16);
+            }
+            const int col = 32 * cc + 8 * g8;  // X blocks: [64 x D], 8-column groups 1 KB apart
+            const int off = (col >> 3) * 1024 + (r >> 3) * 128 + (r & 7) * 16;
+            *reinterpret_cast<uint4*>(xa_hi + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+            *reinterpret_cast<uint4*>(xa_lo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+          }
+        }
+      }
+      tc_fence_before();
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(bar + kFbOEmpty + b);
+        mbar_arrive(bar + kFbXFull);
+      }
+      if (h == nq - 1) {  // |x|^2 of the tile's tokens for its pool softmax
+        if (ti >= 1) wait(kFbSqEmpty, static_cast<unsigned>((ti - 1) & 1));
+        if (lane < 16) s_sq[hf][r] = (sq4[0] + sq4[1]) + (sq4[2] + sq4[3]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sq4[e] = 0.f;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar + kFbSqFull);
+      }
+    }
+    wait(kFbXEmpty, static_cast<unsigned>((nsteps - 1) & 1));
+    store_fagg(nsteps - 1);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemFused);
+  }
+}
+
+// ======================================================================
 // 2. pool scores and weights
 // ======================================================================
 
@@ -1336,8 +1889,8 @@ cudaError_t launch_t(const PrefillParams& p, cudaStream_t s) {
       e = encode_near_maps(p, D, &maps);
       if (e == cudaSuccess) {
         cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = g1;
-        cfg.blockDim = dim3(NT, 1, 1);
+        cfg.gridDim = p.near.fused ? dim3(static_cast<unsigned>(p.n_seg), ns, 1) : g1;
+        cfg.blockDim = dim3(p.near.fused ? NTF : NT, 1, 1);
         cfg.dynamicSmemBytes = static_cast<size_t>(p.near.total);
         cfg.stream = s;
         cudaLaunchAttribute attr[1];
@@ -1345,7 +1898,8 @@ cudaError_t launch_t(const PrefillParams& p, cudaStream_t s) {
         attr[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        e = cudaLaunchKernelEx(&cfg, near_tc_kernel<D>, p, maps);
+        e = p.near.fused ? cudaLaunchKernelEx(&cfg, fused_kernel<D>, p, maps)
+                         : cudaLaunchKernelEx(&cfg, near_tc_kernel<D>, p, maps);
       }
     } else {
       e = launch_pdl(near_kernel<Tin, D>, g1, p.near.total, s, p);
@@ -1353,19 +1907,26 @@ cudaError_t launch_t(const PrefillParams& p, cudaStream_t s) {
   } else {
     e = launch_pdl(near_kernel<Tin, D>, g1, p.near.total, s, p);
   }
-  if (e == cudaSuccess) e = launch_pdl(pool_kernel, g2, p.pool_smem, s, p);
+  if (e == cudaSuccess && !p.near.fused) e = launch_pdl(pool_kernel, g2, p.pool_smem, s, p);
   if (e == cudaSuccess) e = launch_pdl(out_kernel<Tin>, g3, p.out_smem, s, p);
   return e;
 }
 
 }  // namespace
 
-bool plan_near(int D, int esz, int K, size_t limit, bool tc, NearPlan* out) {
+bool plan_near(int D, int esz, int K, size_t limit, bool tc, bool fused, NearPlan* out) {
   auto a16 = [](long long x) { return static_cast<int>((x + 15) & ~15LL); };
   NearPlan p;
   std::memset(&p, 0, sizeof(p));
   tc = tc && esz == 2 && K <= 16;
   p.tc = tc ? 1 : 0;
+  if (tc && fused) {
+    p.fused = 1;
+    p.total = D == 64 ? FusedPlan<64>::total : FusedPlan<128>::total;
+    if (static_cast<size_t>(p.total) > limit) return false;
+    *out = p;
+    return true;
+  }
   p.row = D * esz + 16;
   const int xs = a16(4LL * kTile * (D + kXsPad));
   const int qb = tc ? kTile * D * 2 : a16(static_cast<long long>(kTile) * p.row);
@@ -1426,6 +1987,8 @@ cudaError_t prefill_prepare(int device) {
   if (e == cudaSuccess) e = set_smem(near_kernel<__nv_bfloat16, 128>, optin);
   if (e == cudaSuccess) e = set_smem(near_tc_kernel<64>, optin);
   if (e == cudaSuccess) e = set_smem(near_tc_kernel<128>, optin);
+  if (e == cudaSuccess) e = set_smem(fused_kernel<64>, optin);
+  if (e == cudaSuccess) e = set_smem(fused_kernel<128>, optin);
   if (e == cudaSuccess) e = set_smem(far_agg_kernel<float, 64>, optin);
   if (e == cudaSuccess) e = set_smem(far_agg_kernel<float, 128>, optin);
   if (e == cudaSuccess) e = set_smem(far_agg_kernel<__nv_bfloat16, 64>, optin);

@@ -60,7 +60,7 @@ def test_plain_c_client_compiles_links_and_runs(lib, tmp_path):
 
 
 def test_abi_version(lib):
-    assert sfa.sfa_abi_version() == 2
+    assert sfa.sfa_abi_version() == 3
 
 
 def _golden(name):

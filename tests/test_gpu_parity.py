@@ -27,7 +27,7 @@ def _tiny_variant(**kw) -> Workload:
 
 def _run_schedule(w: Workload, schedule, layers=None, seqs=None, check_state=True, paths=None):
     """schedule: list of ("p", n) prefill calls and ("d", steps) decode runs;
-    paths: (decode_tile, prefill_near_tc) for sfa_debug_set_paths."""
+    paths: (decode_tile, prefill_near) for sfa_debug_set_paths."""
     pair = Pair(w, layers=layers, seqs=seqs)
     if paths is not None:
         sfa.sfa_debug_set_paths(pair.op.handle, *paths)
@@ -131,6 +131,15 @@ def test_cuda_core_near_field_on_bf16_inputs():
     w = _tiny_variant(name="cuda_core_near_bf16", n_layers=2, batch=2, n_q_heads=14,
                       n_kv_heads=2, head_dim=64, window_k=16, in_dtype="bf16")
     _run_schedule(w, [("p", 130), ("d", 5), ("p", 70)], paths=(-1, False))
+
+
+@pytest.mark.parametrize("name,over,schedule", [e for e in EDGE if e[1].get("in_dtype") == "bf16"],
+                         ids=[e[0] for e in EDGE if e[1].get("in_dtype") == "bf16"])
+def test_unfused_tensor_core_prefill(name, over, schedule):
+    """The tensor-core near field followed by the separate pool kernel (the
+    handle's test hook; by default the fused kernel serves these calls)."""
+    w = _tiny_variant(name=name + "_unfused", **over)
+    _run_schedule(w, schedule, paths=(-1, 1))
 
 
 def test_gqa7_bf16_chunked_prefill_and_decode():
