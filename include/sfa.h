@@ -343,9 +343,10 @@ SFA_API int sfa_debug_set_wait_limit(sfa_handle* h, unsigned int spin_limit, lon
  * decode kernel by the number of sequences per call (the default), 0 always
  * the per-sequence kernel, 1 always the batch-tiled kernel.
  * prefill_near: where the tensor cores apply to the prefill near field
- * (bf16 inputs, k <= 16), 2 runs it fused with the pool scores in one
- * kernel (the default), 1 on the tensor cores followed by a separate pool
- * kernel, 0 on the CUDA cores.  SFA_ERR_INVALID_ARG for other values,
+ * (bf16 inputs, k <= 16), 3 chooses by call size (the default: 2 for calls
+ * of at least four 64-token tiles per SM, else 1), 2 runs it fused with the
+ * pool scores in one kernel, 1 on the tensor cores followed by a separate
+ * pool kernel, 0 on the CUDA cores.  SFA_ERR_INVALID_ARG for other values,
  * SFA_ERR_UNSUPPORTED if the requested kernel does not fit this
  * configuration (nothing changes then).  Affects later calls on this handle
  * only. */

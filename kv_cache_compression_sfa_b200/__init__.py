@@ -427,13 +427,13 @@ def sfa_debug_set_wait_limit(h: Handle, spin_limit: int = 0, withhold_tile: int 
         raise SfaError(rc, "sfa_debug_set_wait_limit")
 
 
-def sfa_debug_set_paths(h: Handle, decode_tile: int = -1, prefill_near=2) -> None:
+def sfa_debug_set_paths(h: Handle, decode_tile: int = -1, prefill_near=3) -> None:
     """Test hook that pins the kernel variants: decode_tile -1 (by batch
     size), 0 (per-sequence kernel) or 1 (batch-tiled kernel); prefill near
-    field, where the tensor cores apply, 2 fused with the pool scores (the
-    default; also True), 1 tensor cores with a separate pool kernel, 0 CUDA
-    cores (also False)."""
-    mode = {True: 2, False: 0}[prefill_near] if isinstance(prefill_near, bool) else int(prefill_near)
+    field, where the tensor cores apply, 3 by call size (the default; also
+    True), 2 fused with the pool scores, 1 tensor cores with a separate pool
+    kernel, 0 CUDA cores (also False)."""
+    mode = {True: 3, False: 0}[prefill_near] if isinstance(prefill_near, bool) else int(prefill_near)
     rc = load_library().sfa_debug_set_paths(h.ptr, int(decode_tile), mode)
     if rc != SFA_OK:
         raise SfaError(rc, "sfa_debug_set_paths")

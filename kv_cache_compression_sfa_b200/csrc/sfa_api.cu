@@ -36,14 +36,16 @@ struct sfa_handle {
   int cs;               // CTAs per cluster of the decode kernels
   int n_sm;              // streaming multiprocessors of the device
   NearPlan near;         // shared-memory plan of the prefill near-field kernel
+  NearPlan near_small;   // near_mode 3: the plan for calls below kFusedMinTilesPerSm tiles per SM
   int decode_budget;
   unsigned spin_limit;
   long long withhold_tile;
   bool tile_ok;          // the batch-tiled decode fits this configuration
   TilePlan tile_plan;    // its shared-memory plan
   int tile_mode;         // -1: by batch size; 0: never; 1: always (sfa_debug_set_paths)
-  int near_mode;         // prefill near field where the tensor cores apply: 2 fused with the
-                         // pool scores, 1 tensor cores and a separate pool kernel, 0 CUDA cores
+  int near_mode;         // prefill near field where the tensor cores apply: 3 by call size (2
+                         // for large calls, else 1), 2 fused with the pool scores, 1 tensor
+                         // cores and a separate pool kernel, 0 CUDA cores
   bool inputs_early;     // decode inputs declared complete before each call
   int out_mode;          // sfa_out_mode of the compute calls
 };
@@ -182,9 +184,15 @@ int cuda_status(cudaError_t e) { return e == cudaSuccess ? SFA_OK : SFA_ERR_CUDA
 bool plan_near_field(sfa_handle* h, size_t limit) {
   const sfa_config* c = &h->cfg;
   const int esz = static_cast<int>(in_bytes(c->in_dtype));
-  return (h->near_mode > 0 &&
-          plan_near(c->head_dim, esz, c->window_k, limit, true, h->near_mode == 2, &h->near)) ||
-         plan_near(c->head_dim, esz, c->window_k, limit, false, false, &h->near);
+  const bool fused = h->near_mode >= 2;
+  if (!((h->near_mode > 0 && plan_near(c->head_dim, esz, c->window_k, limit, true, fused, &h->near)) ||
+        plan_near(c->head_dim, esz, c->window_k, limit, false, false, &h->near)))
+    return false;
+  h->near_small = h->near;
+  if (h->near_mode == 3 && h->near.fused &&
+      !plan_near(c->head_dim, esz, c->window_k, limit, true, false, &h->near_small))
+    h->near_small = h->near;
+  return true;
 }
 
 template <typename P>
@@ -297,7 +305,7 @@ int sfa_init(const sfa_config* cfg, sfa_handle** out) {
   h->withhold_tile = -1;
   h->inputs_early = false;
   h->tile_mode = -1;
-  h->near_mode = 2;
+  h->near_mode = 3;
   h->out_mode = SFA_OUT_F32;
   const int L = cfg->n_layers, H = hidden_of(cfg);
   bool no_fit = false;  // a kernel's shared-memory plan does not fit this device
@@ -515,7 +523,11 @@ int prefill_impl(const sfa_handle* h, int layer_begin, int layer_count, const vo
   p.ws_halo = w.halo;
   p.nseg_out = out_segments(h->n_sm, hidden_of(c), streams, tiles_per_stream);
   p.tps_out = static_cast<int>((tiles_per_stream + p.nseg_out - 1) / p.nseg_out);
-  if (h->near.fused) {
+  // Calls of few tiles per SM leave the fused kernel (one CTA per SM walking
+  // every head) with too little to overlap: they take the two-kernel path.
+  const NearPlan& np = (h->near_mode == 3 && streams * tiles_per_stream < kFusedMinTilesPerSm * h->n_sm)
+                           ? h->near_small : h->near;
+  if (np.fused) {
     // Fused kernel: one CTA per SM, each a run of consecutive tiles of one
     // stream, all heads; about one round over the SMs.
     const long long total = streams * tiles_per_stream;
@@ -537,7 +549,7 @@ int prefill_impl(const sfa_handle* h, int layer_begin, int layer_count, const vo
   }
   p.spin_limit = h->spin_limit;
   p.withhold_tile = h->withhold_tile;
-  p.near = h->near;
+  p.near = np;
   p.pool_smem = prefill_pool_smem();
   p.out_smem = prefill_out_smem();
   return cuda_status(launch_prefill(p, c->in_dtype, c->head_dim, s));
@@ -647,15 +659,16 @@ int sfa_debug_set_wait_limit(sfa_handle* h, unsigned int spin_limit, long long w
 }
 
 int sfa_debug_set_paths(sfa_handle* h, int decode_tile, int prefill_near) {
-  if (!handle_ok(h) || decode_tile < -1 || decode_tile > 1 || prefill_near < 0 || prefill_near > 2)
+  if (!handle_ok(h) || decode_tile < -1 || decode_tile > 1 || prefill_near < 0 || prefill_near > 3)
     return SFA_ERR_INVALID_ARG;
   if (decode_tile == 1 && !h->tile_ok) return SFA_ERR_UNSUPPORTED;
   const int old_mode = h->near_mode;
-  const NearPlan old_plan = h->near;
+  const NearPlan old_plan = h->near, old_small = h->near_small;
   h->near_mode = prefill_near;
   if (!plan_near_field(h, prefill_smem_limit(h->device))) {
     h->near_mode = old_mode;
     h->near = old_plan;
+    h->near_small = old_small;
     return SFA_ERR_UNSUPPORTED;
   }
   h->tile_mode = decode_tile;

@@ -178,6 +178,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, unsigned parity) {
   return ok != 0;
 }
 
+// Barrier `id` (1..15) among `count` threads (whole warps) of the CTA.
+__device__ __forceinline__ void named_bar_sync(unsigned id, unsigned count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 // Non-blocking test of phase `parity` (true once that phase has completed).
 __device__ __forceinline__ bool mbar_test(uint64_t* bar, unsigned parity) {
   unsigned ok;

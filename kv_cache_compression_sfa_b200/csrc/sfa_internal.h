@@ -31,6 +31,7 @@ constexpr int kTile = 64;                 // tokens per prefill tile
 constexpr int kHalo = kRing - 1;          // x rows a token needs from before its tile
 constexpr int kPrefillThreads = 256;
 constexpr int kDecodeThreads = 256;
+constexpr long long kFusedMinTilesPerSm = 4;  // prefill calls from this many tiles per SM take the fused kernel
 constexpr int kDecodeTileMinSeqs = 64;      // batch-tiled decode from this many sequences per call
 constexpr int kDecodeTileHeads = 8;         // most query heads per KV head it serves
 constexpr int kDecodeTileChunk = 16;        // window slots per staged chunk

@@ -752,16 +752,17 @@ near_tc_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ 
 // output kernel is the same.
 //
 // Warp roles (one elected lane issues): warp 0 loads (tensor copies of q per
-// head and of the key/value span per KV head, bulk copies of the head's
-// slot blocks); warp 1 issues the MMAs, for step j QK(j), PV(j-1) and
+// head and of the key/value span per KV head), warp 14 the bulk copies of
+// each head's slot blocks; warp 1 issues the MMAs, for step j QK(j), PV(j-1) and
 // POOL(j-2); warps 2-5 run the band softmax and the tile's pool softmax;
 // warps 6-13 the x epilogue, two per lane quarter of the accumulator, each
 // on half of the head's columns.  Scores
 // and X accumulators are double-buffered in tensor memory, queries and slot
 // blocks double-buffered in shared memory; every hand-off is an mbarrier
 // with a bounded wait.
-constexpr int NTF = 448;              // threads of the fused kernel: 14 warps
+constexpr int NTF = 480;              // threads of the fused kernel: 15 warps
 constexpr int kEpiWarps = 8;          // x epilogue warps (warps 6 .. 13)
+constexpr int kFusedWarps = NTF / 32;  // the last one loads slot blocks
 constexpr int kTmemFused = 512;       // all of an SM's tensor memory: one CTA per SM
 constexpr int kFColS = 0;             // [2] band scores, kNS columns each
 constexpr int kFColPool = 2 * kNS;    // pool scores, 64 columns
@@ -820,6 +821,7 @@ fused_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ Ne
   __shared__ float s_gpow[kTile + 1];  // gamma_far^m
   __shared__ float s_norm[kSlots];     // slot norms of the layer
   __shared__ float s_sq[2][kTile];     // |x|^2 per token of the tile being finished, per column half
+  __shared__ __align__(16) float s_s0[128];  // S at the tile start of the epilogue's KV head
 
   pdl_trigger();
   pdl_wait();  // far state at the tile starts from far_carry_kernel
@@ -908,7 +910,6 @@ fused_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ Ne
     unsigned char* blk = stream_block(p, s);
     const Tin* win_k = reinterpret_cast<const Tin*>(blk + p.so.win_k);
     const Tin* win_v = reinterpret_cast<const Tin*>(blk + p.so.win_v);
-    const unsigned char* img_l = p.slot_img + static_cast<size_t>(l) * (p.H / kBlk) * 2 * kBlkBytes;
     constexpr unsigned kKvBytes = static_cast<unsigned>(2 * C16 * kNS * 16);
     int kvc = 0;  // span copies issued
     for (int j = 0; j < nsteps; ++j) {
@@ -952,12 +953,22 @@ fused_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ Ne
         mbar_arrive_expect_tx(bar + kFbQFull + b, static_cast<unsigned>(FP::qb));
 #pragma unroll
         for (int u = 0; u < C16; ++u) tma_load_3d(qa + u * 1024, &maps.q, 8 * u, h, row0 + i * kTile, bar + kFbQFull + b);
+      }
+    }
+  } else if (warp == kFusedWarps - 1) {
+    // ---- slot blocks of each head (a warp of their own: their stage frees
+    // only when the head's pool MMAs complete) ------------------------------------
+    if (lane == 0) {
+      const unsigned char* img_l = p.slot_img + static_cast<size_t>(l) * (p.H / kBlk) * 2 * kBlkBytes;
+      for (int j = 0; j < nsteps; ++j) {
+        const int h = j % nq, b = j & 1;
         if (j >= 2) wait(kFbSlEmpty + b, static_cast<unsigned>(((j >> 1) - 1) & 1));
         mbar_arrive_expect_tx(bar + kFbSlFull + b, static_cast<unsigned>(FP::slb));
         bulk_g2s(sm + FP::sl0 + b * FP::slb, img_l + static_cast<size_t>(h) * FP::slb, static_cast<unsigned>(FP::slb),
                  bar + kFbSlFull + b);
       }
     }
+    __syncwarp();
   } else if (warp == 1) {
     // ---- MMAs ---------------------------------------------------------------
     if (lane == 0) {
@@ -1193,13 +1204,18 @@ fused_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ Ne
         fagg[static_cast<long long>(i) * p.H + h * D + c] = tile_rows(i) == kTile ? fv[0] : fv[1];
     };
     float sq4[4] = {0.f, 0.f, 0.f, 0.f};  // |x|^2 of row r over the tile's heads so far (four partial sums)
+    constexpr int NC = D / 64;             // 32-column chunks of this warp's half of a head
     for (int j = 0; j < nsteps; ++j) {
       const int h = j % nq, ti = j / nq, i = i0 + ti, g = h / G, b = j & 1;
       const long long t0 = pos0 + static_cast<long long>(i) * kTile;
       const int Tt = tile_rows(i);
       const int r_ev = static_cast<int>(max(0LL, min(static_cast<long long>(Tt), K - t0)));
       const float c0s = af * s_gpow[min(kTile, max(0, r - r_ev + 1))];
-      const float* s0 = sst + (static_cast<long long>(i) * nkv + g) * D;
+      if (h % G == 0) {  // the KV head's S at the tile start, staged once for the eight warps
+        named_bar_sync(1, kEpiWarps * 32);  // every epilogue warp is done with the previous one
+        for (int e = tid - 6 * 32; e < D; e += kEpiWarps * 32) s_s0[e] = sst[(static_cast<long long>(i) * nkv + g) * D + e];
+        named_bar_sync(1, kEpiWarps * 32);
+      }
       const bool live = lane < 16 && r < Tt && ok;
       float* orow = p.out + (in_row0 + static_cast<long long>(i) * kTile + r) * p.H + h * D;
       // the last kHalo rows of a tile that ends an output segment lead the next one
@@ -1210,55 +1226,62 @@ fused_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ Ne
                      (r - (kTile - kHalo))) * p.H + h * D;
       wait(kFbOFull + b, static_cast<unsigned>((j >> 1) & 1));
       tc_fence_after();
-#pragma unroll 1
-      for (int cc = hf * (D / 64); cc < (hf + 1) * (D / 64); ++cc) {
-        float v[32];
-        tmem_ld32(tmem + lane_base + kFColX + b * D + 32 * cc, v);
+      float v[NC][32];
+#pragma unroll
+      for (int u = 0; u < NC; ++u) tmem_ld32(tmem + lane_base + kFColX + b * D + 32 * (hf * NC + u), v[u]);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar + kFbOEmpty + b);  // the accumulator is in registers
+      // x = X + alpha_far gamma^m S_start [P1 §2.1 eq. O], stored for the output kernel
+#pragma unroll
+      for (int u = 0; u < NC; ++u) {
+        const int c0 = 32 * (hf * NC + u);
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
-          const float4 sv4 = __ldg(reinterpret_cast<const float4*>(s0 + 32 * cc + e));
-          v[e] = r < Tt ? fmaf(c0s, sv4.x, v[e]) : 0.f;
-          v[e + 1] = r < Tt ? fmaf(c0s, sv4.y, v[e + 1]) : 0.f;
-          v[e + 2] = r < Tt ? fmaf(c0s, sv4.z, v[e + 2]) : 0.f;
-          v[e + 3] = r < Tt ? fmaf(c0s, sv4.w, v[e + 3]) : 0.f;
-          sq4[(e >> 2) & 3] = fmaf(v[e], v[e], fmaf(v[e + 1], v[e + 1], fmaf(v[e + 2], v[e + 2], fmaf(v[e + 3], v[e + 3], sq4[(e >> 2) & 3]))));
+          const float4 sv4 = *reinterpret_cast<const float4*>(s_s0 + c0 + e);
+          v[u][e] = r < Tt ? fmaf(c0s, sv4.x, v[u][e]) : 0.f;
+          v[u][e + 1] = r < Tt ? fmaf(c0s, sv4.y, v[u][e + 1]) : 0.f;
+          v[u][e + 2] = r < Tt ? fmaf(c0s, sv4.z, v[u][e + 2]) : 0.f;
+          v[u][e + 3] = r < Tt ? fmaf(c0s, sv4.w, v[u][e + 3]) : 0.f;
+          sq4[(e >> 2) & 3] = fmaf(v[u][e], v[u][e], fmaf(v[u][e + 1], v[u][e + 1],
+                                   fmaf(v[u][e + 2], v[u][e + 2], fmaf(v[u][e + 3], v[u][e + 3], sq4[(e >> 2) & 3]))));
           if (live) {
-            *reinterpret_cast<float4*>(orow + 32 * cc + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
-            if (halo_row) *reinterpret_cast<float4*>(hrow + 32 * cc + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+            const float4 o4 = make_float4(v[u][e], v[u][e + 1], v[u][e + 2], v[u][e + 3]);
+            *reinterpret_cast<float4*>(orow + c0 + e) = o4;
+            if (halo_row) *reinterpret_cast<float4*>(hrow + c0 + e) = o4;
           }
         }
-        if (cc == hf * (D / 64) && j >= 1) {  // POOL(j-1) has read X: its field aggregate is ready
-          wait(kFbXEmpty, static_cast<unsigned>((j - 1) & 1));
-          store_fagg(j - 1);
-        }
-        if (lane < 16) {
+      }
+      if (j >= 1) {  // POOL(j-1) has read X: its field aggregate is ready
+        wait(kFbXEmpty, static_cast<unsigned>((j - 1) & 1));
+        store_fagg(j - 1);
+      }
+      if (lane < 16) {
+#pragma unroll
+        for (int u = 0; u < NC; ++u)
 #pragma unroll
           for (int g8 = 0; g8 < 4; ++g8) {
             uint32_t hw[4], lw[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               __nv_bfloat16 h0b, l0b, h1b, l1b;
-              split_bf16(v[8 * g8 + 2 * e], h0b, l0b);
-              split_bf16(v[8 * g8 + 2 * e + 1], h1b, l1b);
+              split_bf16(v[u][8 * g8 + 2 * e], h0b, l0b);
+              split_bf16(v[u][8 * g8 + 2 * e + 1], h1b, l1b);
               hw[e] = static_cast<uint32_t>(__bfloat16_as_ushort(h0b)) |
                       (static_cast<uint32_t>(__bfloat16_as_ushort(h1b)) << 16);
               lw[e] = static_cast<uint32_t>(__bfloat16_as_ushort(l0b)) |
                       (static_cast<uint32_t>(__bfloat16_as_ushort(l1b)) << 16);
             }
-            const int col = 32 * cc + 8 * g8;  // X blocks: [64 x D], 8-column groups 1 KB apart
+            const int col = 32 * (hf * NC + u) + 8 * g8;  // X blocks: [64 x D], 8-column groups 1 KB apart
             const int off = (col >> 3) * 1024 + (r >> 3) * 128 + (r & 7) * 16;
             *reinterpret_cast<uint4*>(xa_hi + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
             *reinterpret_cast<uint4*>(xa_lo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
           }
-        }
       }
       tc_fence_before();
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(bar + kFbOEmpty + b);
-        mbar_arrive(bar + kFbXFull);
-      }
+      if (lane == 0) mbar_arrive(bar + kFbXFull);
       if (h == nq - 1) {  // |x|^2 of the tile's tokens for its pool softmax
         if (ti >= 1) wait(kFbSqEmpty, static_cast<unsigned>((ti - 1) & 1));
         if (lane < 16) s_sq[hf][r] = (sq4[0] + sq4[1]) + (sq4[2] + sq4[3]);

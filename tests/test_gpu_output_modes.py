@@ -40,12 +40,13 @@ def _check(got, ref, tol, bf16_out, what):
 
 
 class Modes:
-    def __init__(self, w, mode, seed=7):
+    def __init__(self, w, mode, seed=7, prefill_near=3):
         self.w, self.mode = w, mode
         self.dev = torch.device("cuda")
         slots = make_slots(w, "cpu")
         self.slots_np = np32(slots)
         self.op = sfa.SfaOperator(sfa_config(w), slots.to(self.dev), w.batch, device=self.dev)
+        sfa.sfa_debug_set_paths(self.op.handle, -1, prefill_near)
         self.op.set_output_mode(mode)
         self.p = oracle_params(w)
         S = w.n_layers * w.batch
@@ -126,6 +127,17 @@ CONFIGS = [
 def test_output_mode_matches_the_oracle(name, over, mode):
     m = Modes(WORKLOADS["tiny"].replace(**over), mode)
     for n in (70, 0, 0, 0, 20):
+        m.step(n)
+    assert m.op.check() == 0
+    m.compare_state()
+
+
+@pytest.mark.parametrize("mode", MODES, ids=["bf16", "add_f32", "add_bf16"])
+def test_output_mode_with_the_fused_prefill(mode):
+    """The fused prefill kernel (pinned; these calls are small) keeps x in the
+    workspace for the output kernel in every mode."""
+    m = Modes(WORKLOADS["tiny"].replace(**CONFIGS[0][1]), mode, prefill_near=2)
+    for n in (70, 0, 20):
         m.step(n)
     assert m.op.check() == 0
     m.compare_state()

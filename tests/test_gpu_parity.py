@@ -133,20 +133,23 @@ def test_cuda_core_near_field_on_bf16_inputs():
     _run_schedule(w, [("p", 130), ("d", 5), ("p", 70)], paths=(-1, False))
 
 
+@pytest.mark.parametrize("mode", [1, 2], ids=["unfused", "fused"])
 @pytest.mark.parametrize("name,over,schedule", [e for e in EDGE if e[1].get("in_dtype") == "bf16"],
                          ids=[e[0] for e in EDGE if e[1].get("in_dtype") == "bf16"])
-def test_unfused_tensor_core_prefill(name, over, schedule):
-    """The tensor-core near field followed by the separate pool kernel (the
-    handle's test hook; by default the fused kernel serves these calls)."""
-    w = _tiny_variant(name=name + "_unfused", **over)
-    _run_schedule(w, schedule, paths=(-1, 1))
+def test_tensor_core_prefill_paths(name, over, schedule, mode):
+    """Each tensor-core prefill path pinned by the handle's test hook (by
+    default calls this small take the unfused one): the near field followed
+    by the separate pool kernel (1), and the fused kernel (2)."""
+    w = _tiny_variant(name=name + f"_tc{mode}", **over)
+    _run_schedule(w, schedule, paths=(-1, mode))
 
 
-def test_gqa7_bf16_chunked_prefill_and_decode():
+@pytest.mark.parametrize("mode", [1, 2], ids=["unfused", "fused"])
+def test_gqa7_bf16_chunked_prefill_and_decode(mode):
     """Seven query heads per KV head, bf16, prefill calls across a decode."""
-    w = _tiny_variant(name="gqa7_bf16_chunks", n_layers=2, batch=2, n_q_heads=14,
+    w = _tiny_variant(name=f"gqa7_bf16_chunks_tc{mode}", n_layers=2, batch=2, n_q_heads=14,
                       n_kv_heads=2, head_dim=64, window_k=16, in_dtype="bf16")
-    _run_schedule(w, [("p", 130), ("d", 5), ("p", 70)])
+    _run_schedule(w, [("p", 130), ("d", 5), ("p", 70)], paths=(-1, mode))
 
 
 @pytest.mark.parametrize("name,over,schedule", EDGE, ids=[e[0] for e in EDGE])

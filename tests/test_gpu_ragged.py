@@ -26,12 +26,13 @@ def _w(**kw):
 class Ragged:
     """One operator on the GPU and one oracle state per (layer, sequence)."""
 
-    def __init__(self, w, seed=0):
+    def __init__(self, w, seed=0, prefill_near=3):
         self.w = w
         self.dev = torch.device("cuda")
         slots = make_slots(w, "cpu")
         self.slots_np = np32(slots)
         self.op = sfa.SfaOperator(sfa_config(w), slots.to(self.dev), w.batch, device=self.dev)
+        sfa.sfa_debug_set_paths(self.op.handle, -1, prefill_near)
         self.p = oracle_params(w)
         self.ost = [[oracle.OracleState(self.p, 1) for _ in range(w.batch)]
                     for _ in range(w.n_layers)]
@@ -110,9 +111,13 @@ CASES = [
 ]
 
 
+@pytest.mark.parametrize("mode", [3, 2], ids=["default", "fused"])
 @pytest.mark.parametrize("name,over,calls", CASES, ids=[c[0] for c in CASES])
-def test_ragged_prefill_matches_the_oracle(name, over, calls):
-    r = Ragged(_w(**over))
+def test_ragged_prefill_matches_the_oracle(name, over, calls, mode):
+    """mode: the prefill near-field path (sfa_debug_set_paths); 2 pins the
+    fused kernel, which these small calls would not take by default (fp32
+    inputs keep the CUDA cores either way)."""
+    r = Ragged(_w(**over), prefill_near=mode)
     r.prefill(calls[0])
     r.decode()  # every sequence one token on, from different positions
     r.prefill(calls[1])
