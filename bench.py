@@ -569,21 +569,23 @@ def roofline_sections(run, pre_tot, dec_tot, steps, world, peak):
 
 
 def dominant_kernel(run):
-    """(part, kernel name, source file) of the kernel that dominates a step."""
+    """(part, kernel label, source file, traffic-file key) of the launch unit
+    that dominates a step: one decode call or one prefill call."""
     if run.has_b and (not run.has_a or run.kind == "decode"):
-        if run.w.batch >= 64 and run.w.window_k <= 64:  # the library's batch-tiled rule
-            return "decode", "decode_tile_kernel", "sfa_decode_tile.cu"
-        return "decode", "decode_kernel", "sfa_decode.cu"
-    return "prefill", "prefill", "sfa_prefill.cu"
+        if run.w.batch >= 64 and run.w.window_k <= 256:  # the library's batch-tiled rule
+            return ("decode", "decode_near_mma_kernel + decode_pool_kernel", "sfa_decode_tile.cu",
+                    "decode_tile")
+        return "decode", "decode_kernel", "sfa_decode.cu", "decode"
+    return "prefill", "prefill", "sfa_prefill.cu", "prefill"
 
 
 def roofline_for(run, section, peak, peak_src):
-    part, kernel, src = dominant_kernel(run)
+    part, kernel, src, key = dominant_kernel(run)
     if part not in section:  # a prefill-and-decode step whose prefill dominates
         part = "prefill" if "prefill" in section else "decode"
     dom = section[part]
     traffic, traffic_wl = kernel_traffic(
-        os.path.join(ROOT, "kv_cache_compression_sfa_b200", "csrc", src), kernel, run.w.name)
+        os.path.join(ROOT, "kv_cache_compression_sfa_b200", "csrc", src), key, run.w.name)
     return {"bound": "hbm", "kernel": kernel, "part": part, "achieved": dom["achieved_gbs"],
             "peak": peak, "unit": "GB/s", "frac": dom["achieved_gbs"] / peak,
             "peak_source": peak_src, "traffic": traffic,
