@@ -667,6 +667,16 @@ decode_near_mma_kernel(const __grid_constant__ DecodeParams p, const __grid_cons
 
 // ---------------------------------------------------------------- pool kernel
 
+// The split x^T and w^T blocks ([16 x 64] bf16, core-matrix layout) keep
+// their 8-column groups kGrp16 = 256 + 16 bytes apart: the 16 lanes that
+// write one row then spread over all 32 banks (256 apart they share four).
+// As a K-major MMA operand the next K group is kGrp16 bytes on.
+constexpr int kGrp16 = 272;
+constexpr int kBlk16Pad = 8 * kGrp16;
+__device__ __forceinline__ int pad16_off(int row, int col) {
+  return (col >> 3) * kGrp16 + (row >> 3) * kCoreBytes + (row & 7) * 16 + (col & 7) * 2;
+}
+
 constexpr int NTC = 256;                // pool kernel: compute threads (8 warps)
 constexpr int NWC = NTC / 32;
 constexpr int NTP = NTC + 32;           // plus the MMA warp
@@ -686,8 +696,8 @@ struct PoolTilePlan {
   static constexpr int bars = 0;                                  // mbarriers, tmem address
   static constexpr int sl = 1024;                                 // [4][hi, lo] slot blocks
   static constexpr int xt = sl + kSlotStages * 2 * kBlkBytes;     // [4][hi, lo] x^T blocks [16 x 64]
-  static constexpr int wt = xt + kABufs * 2 * kBlk16Bytes;        // [hi, lo] w^T block [16 x 64]
-  static constexpr int sem = wt + 2 * kBlk16Bytes;                // [4][16][68] sem chunks
+  static constexpr int wt = xt + kABufs * 2 * kBlk16Pad;        // [hi, lo] w^T block [16 x 64]
+  static constexpr int sem = wt + 2 * kBlk16Pad;                // [4][16][68] sem chunks
   static constexpr int sc = sem + kSemBufs * TR * kSemStride * 4; // [16][65] own partial scores, |x|^2
   static constexpr int scp = sc + TR * kScStride * 4;             // [16][65] the peer CTA's partial
   static constexpr int total = scp + TR * kScStride * 4;
@@ -828,11 +838,11 @@ decode_pool_kernel(const __grid_constant__ DecodeParams p) {
           ok = false;
         tc_fence_after();
         const unsigned char* shi = slb + stg * 2 * kBlkBytes;
-        const unsigned char* xhi = xtb + b * 2 * kBlk16Bytes;
+        const unsigned char* xhi = xtb + b * 2 * kBlk16Pad;
 #pragma unroll
         for (int k = 0; k < kBlk / 16; ++k) {
           const uint64_t ah = umma_desc(shi + k * 2048, 1024, 128), al = umma_desc(shi + kBlkBytes + k * 2048, 1024, 128);
-          const uint64_t bh = umma_desc(xhi + k * 512, 256, 128), bl = umma_desc(xhi + kBlk16Bytes + k * 512, 256, 128);
+          const uint64_t bh = umma_desc(xhi + k * 2 * kGrp16, kGrp16, 128), bl = umma_desc(xhi + kBlk16Pad + k * 2 * kGrp16, kGrp16, 128);
           umma_bf16(tmem, ah, bh, idesc_s, c > 0 || k > 0);
           umma_bf16(tmem, ah, bl, idesc_s, true);
           umma_bf16(tmem, al, bh, idesc_s, true);
@@ -871,7 +881,7 @@ decode_pool_kernel(const __grid_constant__ DecodeParams p) {
 #pragma unroll
         for (int k = 0; k < kSlots / 16; ++k) {
           const uint64_t ah = umma_desc(shi + k * 256, 128, 1024), al = umma_desc(shi + kBlkBytes + k * 256, 128, 1024);
-          const uint64_t bh = umma_desc(wtb + k * 512, 256, 128), bl = umma_desc(wtb + kBlk16Bytes + k * 512, 256, 128);
+          const uint64_t bh = umma_desc(wtb + k * 2 * kGrp16, kGrp16, 128), bl = umma_desc(wtb + kBlk16Pad + k * 2 * kGrp16, kGrp16, 128);
           umma_bf16(dst, ah, bh, idesc_c, k > 0);
           umma_bf16(dst, ah, bl, idesc_c, true);
           umma_bf16(dst, al, bh, idesc_c, true);
@@ -905,15 +915,15 @@ decode_pool_kernel(const __grid_constant__ DecodeParams p) {
       if (c >= kABufs &&
           !mbar_wait_bounded(bars + kPbAEmpty + b, static_cast<unsigned>(((c / kABufs) - 1) & 1), kMbarPollLimit, p.err))
         ok = false;
-      unsigned char* xhi = xtb + b * 2 * kBlk16Bytes;
+      unsigned char* xhi = xtb + b * 2 * kBlk16Pad;
       __nv_bfloat16 hh[4], ll[4];
       split_bf16(v.x, hh[0], ll[0]);
       split_bf16(v.y, hh[1], ll[1]);
       split_bf16(v.z, hh[2], ll[2]);
       split_bf16(v.w, hh[3], ll[3]);
-      const int off = blk16_off(r, c4);
+      const int off = pad16_off(r, c4);
       *reinterpret_cast<uint2*>(xhi + off) = *reinterpret_cast<const uint2*>(hh);
-      *reinterpret_cast<uint2*>(xhi + kBlk16Bytes + off) = *reinterpret_cast<const uint2*>(ll);
+      *reinterpret_cast<uint2*>(xhi + kBlk16Pad + off) = *reinterpret_cast<const uint2*>(ll);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(bars + kPbAFull + b);
@@ -965,11 +975,11 @@ decode_pool_kernel(const __grid_constant__ DecodeParams p) {
         __nv_bfloat16 h0, l0, h1, l1;
         split_bf16(e0 * inv, h0, l0);
         split_bf16(e1 * inv, h1, l1);
-        const int o0 = blk16_off(rr, lane), o1 = blk16_off(rr, lane + 32);
+        const int o0 = pad16_off(rr, lane), o1 = pad16_off(rr, lane + 32);
         *reinterpret_cast<__nv_bfloat16*>(wtb + o0) = h0;
-        *reinterpret_cast<__nv_bfloat16*>(wtb + kBlk16Bytes + o0) = l0;
+        *reinterpret_cast<__nv_bfloat16*>(wtb + kBlk16Pad + o0) = l0;
         *reinterpret_cast<__nv_bfloat16*>(wtb + o1) = h1;
-        *reinterpret_cast<__nv_bfloat16*>(wtb + kBlk16Bytes + o1) = l1;
+        *reinterpret_cast<__nv_bfloat16*>(wtb + kBlk16Pad + o1) = l1;
       }
     }
     fence_proxy_async_smem();
