@@ -1,6 +1,6 @@
-// sfa_prefill.cu — SFA prefill: n tokens per (layer, sequence) stream in
-// five kernels, each parallel over independent work units with no waits
-// between CTAs.
+// sfa_prefill.cu — SFA prefill: n tokens per (layer, sequence) stream,
+// each kernel parallel over independent work units with no waits between
+// CTAs, chained by programmatic dependent launch.
 //
 // Sources (web pages):
 //   [P1] "Signal Field Attention (SFA)：8KB代码实现4.16倍推理加速与248倍内存压缩"
@@ -12,33 +12,36 @@
 //    S_t] at every tile start of kTile tokens, as a two-level scan: one
 //    aggregate of the evicted keys per tile (independent terms), then one
 //    fold in tile order per (stream, KV head, dim).
-// 1. near_tc_kernel (bf16, k <= 16) or near_kernel (CUDA cores), one CTA per
-//    (stream, query head, segment of consecutive tiles).  Per tile: queries
-//    and the key/value span staged in shared memory by cp.async, the next
-//    tile's copy in flight during this one's arithmetic; the near field as a
-//    softmax over each token's window [P1 §2.1 eq. O_near] and
-//    x = O_near + alpha_far * S [P1 §2.1 eq. O] written into `out`, which
-//    holds x until step 3.
-// 2. pool_kernel, one CTA per (stream, tile): the cosine scores of the
-//    tile's tokens against the 64 slots, x[T x H] . slot^T on the tcgen05
-//    tensor cores (three bf16 MMAs per 64-column chunk, hi*hi + hi*lo +
-//    lo*hi of split operands, about 16 significant bits, fp32 accumulators
-//    in tensor memory) with the next chunk's copy in flight; |x|, softmax of
-//    cos/T [P3 §2.1 channel 3]; the weights stored in the workspace as split
-//    bf16 blocks in the MMA operand layout.
-// 3. out_kernel, one CTA per (stream, 64 hidden columns), walks the tiles in
-//    order: sem[T x 64] = w . slot_chunk on the tensor cores; per column the
-//    ring sum over the last 16 x (a sliding sum, the 15 rows before the tile
-//    kept from the previous one) and the EMA field (carried across tiles),
-//    four token segments per column joined by their carries; the fusion,
-//    clip and scale [P3 §2.1, §2.2] overwrite x in `out`.  At the stream's
-//    end: ring slots, ring sum, field; one CTA per stream also writes the
-//    window, S and the position.
+// 1. The near field [P1 §2.1 eq. O_near] and x = O_near + alpha_far * S
+//    [P1 §2.1 eq. O], then the pool scores, softmax(cos/T) weights and the
+//    EMA field over each tile [P3 §2.1 channels 2-3], by one of:
+//    * fused_kernel (bf16, k <= 16, large calls): one CTA per (stream,
+//      segment of tiles) walks every head of each tile; queries and the
+//      key/value span arrive by tensor copies, the band scores, P.V + G.K,
+//      the pool scores and the field aggregates are tcgen05 MMAs with
+//      accumulators in tensor memory, and warp-specialized roles hand off
+//      through mbarriers.  x is written once, for step 2.
+//    * near_tc_kernel (bf16, k <= 16) or near_kernel (CUDA cores), one CTA
+//      per (stream, query head, segment of tiles), writing x; then
+//      pool_kernel, one CTA per (stream, tile), reads x back for the
+//      scores (tcgen05, split bf16 operands), weights and field aggregates.
+//    The weights go to the workspace as split bf16 blocks in the MMA operand
+//    layout; x lives in `out` (fp32 results) or in the workspace.
+// 2. out_kernel, one CTA per (stream, 64 hidden columns, segment of tiles),
+//    walks its tiles in order: sem[T x 64] = w . slot_chunk on the tensor
+//    cores; per column the ring sum over the last 16 x (a sliding sum, the
+//    15 rows before the tile kept from the previous one or, at a segment
+//    start, from the halo rows step 1 kept) and the EMA field (from the fold
+//    of the earlier tiles' aggregates), four token segments per column
+//    joined by their carries; the fusion, clip and scale [P3 §2.1, §2.2]
+//    give the result in the output mode's form.  At the stream's end: ring
+//    slots, ring sum, field; one CTA per stream also writes the window, S
+//    and the position.
 //
-// Kernels are chained by programmatic dependent launch; each waits for its
-// predecessor before touching what that one writes.  Every wait of a kernel
-// is on its own copies or MMAs and is bounded; a wait that runs out latches
-// SFA_ERR_DEVICE_TIMEOUT and the kernel still finishes.
+// Each kernel waits for its predecessor before touching what that one
+// writes.  Every wait on a copy, MMA or role hand-off is bounded; a wait
+// that runs out latches SFA_ERR_DEVICE_TIMEOUT and the kernel still
+// finishes.
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 
