@@ -682,10 +682,10 @@ __device__ __forceinline__ int pad16_off(int row, int col) {
 constexpr int NTC = 256;                // pool kernel: compute threads (8 warps)
 constexpr int NWC = NTC / 32;
 constexpr int NTP = NTC + 32;           // plus the MMA warp
-constexpr int TR = 16;                  // sequences per cluster: the N = 16 of the MMAs
-constexpr int kMaxSplit = 3;            // most CTAs of a cluster (parts of the hidden columns)
+constexpr int TR = 16;                  // sequences per CTA pair: the N = 16 of the MMAs
+constexpr int kPair = 2;                // CTAs of a cluster: halves of the hidden columns
 constexpr int kSlotStages = 4;
-constexpr int kABufs = 3;               // split x^T blocks
+constexpr int kABufs = 4;               // split x^T blocks
 constexpr int kSemBufs = 4;             // sem^T accumulators and their staging
 constexpr int kScStride = kSlots + 1;   // 64 scores + |x|^2 per row
 constexpr int kSemStride = kBlk + 4;
@@ -697,17 +697,18 @@ static_assert(TR * 16 == NTC, "pool kernel: 16 threads per row, 4 columns each")
 struct PoolTilePlan {
   static constexpr int bars = 0;                                  // mbarriers, tmem address
   static constexpr int sl = 1024;                                 // [4][hi, lo] slot blocks
-  static constexpr int xt = sl + kSlotStages * 2 * kBlkBytes;     // [3][hi, lo] x^T blocks [16 x 64]
+  static constexpr int xt = sl + kSlotStages * 2 * kBlkBytes;     // [4][hi, lo] x^T blocks [16 x 64]
   static constexpr int wt = xt + kABufs * 2 * kBlk16Pad;        // [hi, lo] w^T block [16 x 64]
   static constexpr int sem = wt + 2 * kBlk16Pad;                // [4][16][68] sem chunks
-  static constexpr int sc = sem + kSemBufs * TR * kSemStride * 4; // [3][16][65] partial scores, |x|^2 per rank
-  static constexpr int total = sc + kMaxSplit * TR * kScStride * 4;
+  static constexpr int sc = sem + kSemBufs * TR * kSemStride * 4; // [16][65] own partial scores, |x|^2
+  static constexpr int scp = sc + TR * kScStride * 4;             // [16][65] the peer CTA's partial
+  static constexpr int total = scp + TR * kScStride * 4;
 };
 // barrier slots (arrival counts in brackets)
 constexpr int kPbSlFull = 0;                           // [4] slot block landed (1 + bytes)
 constexpr int kPbSlEmpty = kPbSlFull + kSlotStages;    // [4] MMAs done with a slot block (commit)
-constexpr int kPbAFull = kPbSlEmpty + kSlotStages;     // [3] x^T block written (8 warps)
-constexpr int kPbAEmpty = kPbAFull + kABufs;           // [3] MMAs done with an x^T block (commit)
+constexpr int kPbAFull = kPbSlEmpty + kSlotStages;     // [4] x^T block written (8 warps)
+constexpr int kPbAEmpty = kPbAFull + kABufs;           // [4] MMAs done with an x^T block (commit)
 constexpr int kPbScores = kPbAEmpty + kABufs;          // all score MMAs done (commit)
 constexpr int kPbWFull = kPbScores + 1;                // w^T block written (8 warps)
 constexpr int kPbSemFull = kPbWFull + 1;               // [4] sem accumulator ready (commit)
@@ -717,33 +718,31 @@ constexpr int kPbStEmpty = kPbStFull + kSemBufs;       // [4] staged sem chunk u
 constexpr int kPbCount = kPbStEmpty + kSemBufs;
 static_assert(kPbCount * 8 + 4 <= PoolTilePlan::sl, "barriers fit");
 
-// A cluster of 2 or 3 CTAs (chosen per launch, so that the grid ends close
-// to a whole round of resident clusters) serves 16 sequences of one layer;
-// CTA `rank` owns the hidden columns of chunks [c0, c0 + nloc).  The 16
-// sequences are the N = 16 of transposed MMAs: scores^T[64 slots x 16] +=
-// slot_c . x_c^T and sem^T[64 columns x 16] = slot_c^T . w^T, split bf16
-// operands (hi*hi + hi*lo + lo*hi), fp32 accumulators in tensor memory.
-// Each CTA writes its partial scores and |x|^2 into slot `rank` of every
-// CTA's shared memory; all add the slots in rank order and form the same
-// softmax weights.  Warp 8 (one lane) loads the slot blocks
+// A cluster of two CTAs serves 16 sequences of one layer; CTA `rank` owns
+// the hidden columns of chunks [c0, c0 + nloc).  The 16 sequences are the
+// N = 16 of transposed MMAs: scores^T[64 slots x 16] += slot_c . x_c^T and
+// sem^T[64 columns x 16] = slot_c^T . w^T, split bf16 operands (hi*hi +
+// hi*lo + lo*hi), fp32 accumulators in tensor memory.  The two CTAs add
+// their partial scores and |x|^2 through distributed shared memory and both
+// form the same softmax weights.  Warp 8 (one lane) loads the slot blocks
 // and issues every MMA; warps 0-7 split x (pass 1) and run the epilogue
 // with x and the state rows two chunks ahead in registers (pass 2); warps
 // 0-3, which hold the accumulator lanes, stage each sem chunk for the
 // others.  mbarriers carry every hand-off.
-__global__ void __launch_bounds__(NTP, 2)
+__global__ void __cluster_dims__(kPair, 1, 1) __launch_bounds__(NTP, 2)
 decode_pool_kernel(const __grid_constant__ DecodeParams p) {
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = static_cast<int>(cluster.block_rank());
-  const int cs = static_cast<int>(cluster.num_blocks());  // 2 or 3 (the launch checks)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int tiles_per_layer = (p.n_seq + TR - 1) / TR;
-  const int pair = static_cast<int>(blockIdx.x) / cs;
+  const int pair = static_cast<int>(blockIdx.x) / kPair;
   const int li = pair / tiles_per_layer;
   const int tb = pair % tiles_per_layer;
   const int l = p.l0 + li;
   const int nch = p.H / kBlk;
-  const int c0 = rank * nch / cs;
-  const int nloc = (rank + 1) * nch / cs - c0;  // chunks of this CTA
+  const int half = (nch + 1) / 2;
+  const int c0 = rank == 0 ? 0 : half;
+  const int nloc = rank == 0 ? half : nch - half;  // chunks of this CTA
   extern __shared__ __align__(128) unsigned char smb_pool[];
   unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smb_pool) + 127) &
                                                        ~static_cast<uintptr_t>(127));
@@ -753,7 +752,8 @@ decode_pool_kernel(const __grid_constant__ DecodeParams p) {
   unsigned char* xtb = sm + PoolTilePlan::xt;
   unsigned char* wtb = sm + PoolTilePlan::wt;
   float* semst = reinterpret_cast<float*>(sm + PoolTilePlan::sem);
-  float* sc = reinterpret_cast<float*>(sm + PoolTilePlan::sc);  // [rank][16][65]
+  float* sc = reinterpret_cast<float*>(sm + PoolTilePlan::sc);
+  float* scp = reinterpret_cast<float*>(sm + PoolTilePlan::scp);
   __shared__ long long s_st[TR], s_pos[TR];
   __shared__ int s_ok;
 
@@ -932,17 +932,13 @@ decode_pool_kernel(const __grid_constant__ DecodeParams p) {
     }
 #pragma unroll
     for (int off = 8; off > 0; off >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, off);
-    // partial scores and |x|^2 of this CTA's columns, into slot `rank` of
-    // every CTA of the cluster (this one included)
-    float* dst[kMaxSplit];
-#pragma unroll
-    for (int q = 0; q < kMaxSplit; ++q)
-      dst[q] = cluster.map_shared_rank(sc + rank * TR * kScStride, q < cs ? q : rank);
-    cluster_wait();  // phase 1: every CTA of the cluster has started
+    // partial scores and |x|^2 of this CTA's columns, into its own and the
+    // peer's shared memory
+    float* peer_scp = cluster.map_shared_rank(scp, rank ^ 1);
+    cluster_wait();  // phase 1: the peer has started
     if ((tid & 15) == 0) {
-#pragma unroll
-      for (int q = 0; q < kMaxSplit; ++q)
-        if (q < cs) dst[q][r * kScStride + kSlots] = sq;
+      sc[r * kScStride + kSlots] = sq;
+      peer_scp[r * kScStride + kSlots] = sq;
     }
     if (warp < 4) {  // slot 16w + i sits in lane i of lane quarter w (M = 64)
       if (!mbar_wait_bounded(bars + kPbScores, 0, kMbarPollLimit, p.err)) ok = false;
@@ -956,31 +952,25 @@ decode_pool_kernel(const __grid_constant__ DecodeParams p) {
       }
       if (lane < 16) {
 #pragma unroll
-        for (int q = 0; q < kMaxSplit; ++q)
-          if (q < cs) {
-#pragma unroll
-            for (int rr = 0; rr < TR; ++rr) dst[q][rr * kScStride + 16 * warp + lane] = v[rr];
-          }
+        for (int rr = 0; rr < TR; ++rr) {
+          sc[rr * kScStride + 16 * warp + lane] = v[rr];
+          peer_scp[rr * kScStride + 16 * warp + lane] = v[rr];
+        }
       }
     }
     __syncwarp();
-    cluster_arrive();  // phase 2: every partial in place
+    cluster_arrive();  // phase 2: both partials in place
     cluster_wait();
     // softmax(cos/T) per row [P3 §2.1 channel 3]; weights as split bf16 w^T
     {
       const float* nrm = p.slot_norm + static_cast<size_t>(l) * kSlots;
       const float n0 = nrm[lane], n1 = nrm[lane + 32];
       for (int rr = warp; rr < TR; rr += NWC) {
-        float s0 = 0.f, s1 = 0.f, sqx = 0.f;  // the ranks' partials, added in rank order
-        for (int q = 0; q < cs; ++q) {
-          const float* a = sc + (q * TR + rr) * kScStride;
-          s0 += a[lane];
-          s1 += a[lane + 32];
-          sqx += a[kSlots];
-        }
-        const float nx = fmaxf(sqrtf(sqx), kNormFloor);
-        const float c0v = s0 / (nx * n0) * p.inv_temp;
-        const float c1v = s1 / (nx * n1) * p.inv_temp;
+        const float* a = sc + rr * kScStride;
+        const float* b = scp + rr * kScStride;
+        const float nx = fmaxf(sqrtf(a[kSlots] + b[kSlots]), kNormFloor);
+        const float c0v = (a[lane] + b[lane]) / (nx * n0) * p.inv_temp;
+        const float c1v = (a[lane + 32] + b[lane + 32]) / (nx * n1) * p.inv_temp;
         const float mx = warp_max_redux(fmaxf(c0v, c1v));
         const float e0 = expf(c0v - mx), e1 = expf(c1v - mx);
         const float inv = 1.f / warp_sum(e0 + e1);
@@ -1204,35 +1194,9 @@ cudaError_t launch_t(const DecodeParams& p_in, cudaStream_t s) {
     e = cudaLaunchKernelEx(&cfg, decode_near_kernel<Tin, D>, p, maps);
   }
   if (e != cudaSuccess) return e;
-  // Clusters of 2 or 3 CTAs: the size whose rounds of resident clusters
-  // times the columns each CTA owns is smaller.
-  const long long tiles = static_cast<long long>(p.Lc) * ((p.n_seq + TR - 1) / TR);
-  cudaLaunchAttribute pattr[2];
-  pattr[0] = attr[0];
-  pattr[1].id = cudaLaunchAttributeClusterDimension;
-  cfg.blockDim = dim3(NTP, 1, 1);  // compute warps + the MMA warp
+  cfg.gridDim = dim3(static_cast<unsigned>(p.Lc * ((p.n_seq + TR - 1) / TR) * kPair), 1, 1);
+  cfg.blockDim = dim3(NTP, 1, 1);  // compute warps + the MMA warp; clusters of kPair
   cfg.dynamicSmemBytes = static_cast<size_t>(p.tp.pool_smem);
-  cfg.attrs = pattr;
-  cfg.numAttrs = 2;
-  int best_cs = 2;
-  double best_cost = -1.0;
-  for (int cs = 2; cs <= kMaxSplit; ++cs) {
-    pattr[1].val.clusterDim.x = static_cast<unsigned>(cs);
-    pattr[1].val.clusterDim.y = 1;
-    pattr[1].val.clusterDim.z = 1;
-    cfg.gridDim = dim3(static_cast<unsigned>(tiles * cs), 1, 1);
-    int active = 0;
-    if (cudaOccupancyMaxActiveClusters(&active, decode_pool_kernel, &cfg) != cudaSuccess || active < 1) continue;
-    const double cost = static_cast<double>((tiles + active - 1) / active) / cs;
-    if (best_cost < 0 || cost < best_cost - 1e-9) {
-      best_cost = cost;
-      best_cs = cs;
-    }
-  }
-  pattr[1].val.clusterDim.x = static_cast<unsigned>(best_cs);
-  pattr[1].val.clusterDim.y = 1;
-  pattr[1].val.clusterDim.z = 1;
-  cfg.gridDim = dim3(static_cast<unsigned>(tiles * best_cs), 1, 1);
   return cudaLaunchKernelEx(&cfg, decode_pool_kernel, p);
 }
 
