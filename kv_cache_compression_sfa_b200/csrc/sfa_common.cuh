@@ -183,19 +183,6 @@ __device__ __forceinline__ void named_bar_sync(unsigned id, unsigned count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
-// Non-blocking test of phase `parity` (true once that phase has completed).
-__device__ __forceinline__ bool mbar_test(uint64_t* bar, unsigned parity) {
-  unsigned ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
 // Waits for phase `parity` of a barrier, at most `limit` polls.  Returns
 // false (and latches SFA_ERR_DEVICE_TIMEOUT) if the wait ran out.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, unsigned parity, unsigned limit,
