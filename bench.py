@@ -142,6 +142,20 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def kernels_per_call(w, n_pre, n_sm):
+    """(prefill, decode) kernels the library launches per call for workload
+    w, following its routing: decode calls of 64 or more sequences (at most
+    8 query heads per KV head, hidden a multiple of 64) launch the near-field
+    and pool kernels, smaller ones the batch-1 kernel; a prefill launches the
+    two far-field kernels and the output kernel, plus the fused kernel (bf16,
+    k <= 16, at least 4 tiles per SM) or a near-field and a pool kernel."""
+    G = w.n_q_heads // w.n_kv_heads
+    tiled = w.batch >= 64 and w.window_k <= 256 and G <= 8 and w.hidden % 64 == 0
+    tiles = w.n_layers * w.batch * ((max(n_pre, 1) + 63) // 64)
+    fused = w.in_dtype == "bf16" and w.window_k <= 16 and tiles >= 4 * n_sm
+    return (4 if fused else 5), (2 if tiled else 1)
+
+
 def workload_bytes(w, n_pre=None):
     """Algorithmic bytes (what the method must move; no re-reads).
 
@@ -482,9 +496,10 @@ class Run:
         torch.cuda.current_stream().wait_stream(side)
         torch.cuda.synchronize()
         self.flush_each = kind != "decode"
-        # our kernels per step: state header write + five prefill kernels;
-        # one per decode call
-        self.launches_per_step = (1 + 5 if self.has_a else 0) + (self.n_dec if self.has_b else 0)
+        pre_k, dec_k = kernels_per_call(w, n_pre, torch.cuda.get_device_properties(dev).multi_processor_count)
+        # our kernels per step: the state header write and the prefill's
+        # kernels; the decode kernels of every call
+        self.launches_per_step = (1 + pre_k if self.has_a else 0) + (dec_k * self.n_dec if self.has_b else 0)
 
     def one_step(self, ev=None):
         if self.flush_each:
