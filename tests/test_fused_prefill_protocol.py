@@ -160,11 +160,19 @@ def _run(nq, G, ntiles, first_tile, seed, sq_handshake=True):
     pending = [None] * len(roles)
     alive = set(range(len(roles)))
     rng = random.Random(seed)
+    # each role gets its own speed: the chance of yielding the processor after
+    # a step, so that some roles fall far behind others
+    pause = [rng.choice((0.05, 0.3, 0.9)) for _ in roles]
+    # and a chance of sitting out a whole sweep (a starved warp)
+    skip = [rng.choice((0.0, 0.0, 0.5, 0.9)) for _ in roles]
+    all_in = False  # a sweep that skips nobody (after one without progress)
     while alive:
         progress = 0  # waits passed, roles started or finished in this sweep
         order = sorted(alive)
         rng.shuffle(order)
         for r in order:
+            if not all_in and rng.random() < skip[r]:
+                continue
             while True:
                 if pending[r] is not None:
                     _, name, phase = pending[r]
@@ -183,9 +191,13 @@ def _run(nq, G, ntiles, first_tile, seed, sq_handshake=True):
                     alive.discard(r)
                     progress += 1
                     break
-                if rng.random() < 0.3:
+                if rng.random() < pause[r]:
                     break
+        if progress == 0 and not all_in:
+            all_in = True
+            continue
         assert progress > 0, f"deadlock: {[pending[r] for r in sorted(alive)]}"
+        all_in = False
     return log
 
 
