@@ -200,9 +200,10 @@ SFA_API int sfa_prefill(const sfa_handle* h, const void* q, const void* k, const
  * per-step form of [P2]'s compute_enhancement(layer, attn_output), over all
  * layers at once.
  * Folds one token per sequence into the state and writes its output.
- * One kernel launch covers all layers and sequences; no workspace.
- * The kernel may start while the previous kernel on the stream is still
- * running (programmatic dependent launch): it fetches the handle's
+ * One launch covers all layers and sequences (for 64 or more sequences a
+ * near-field kernel, then a pool kernel); no workspace.
+ * The first kernel may start while the previous kernel on the stream is
+ * still running (programmatic dependent launch): it fetches the handle's
  * constants at once, and the state, q, k and v only once that kernel has
  * finished, so inputs produced by the kernel just before are safe.  See
  * sfa_set_decode_input_prefetch for fetching q, k and v earlier.
